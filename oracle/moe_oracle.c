@@ -1,0 +1,741 @@
+/*
+ * moe_oracle.c -- CPU oracle of the MoE layer.
+ *
+ * TEST INFRASTRUCTURE ONLY. Only tests/, __graft_entry__.smoke() and the
+ * cpu_baseline / reference legs of bench.py may load this library. It shares
+ * no code with the CUDA path and never calls it.
+ *
+ * What it computes, and where that is stated:
+ *
+ *  - The per-token MoE step of "Megatron-Core MoE -- 大规模稀疏专家并行实践"
+ *    (study notes, estelledc.github.io), section 实践案例 / 案例 1: score every
+ *    expert, keep the top-k, and sum gate(e) * Expert_e(x) over the kept ones.
+ *  - The memory-efficient permutation of "《使用 Megatron Core 大规模训练混合专家
+ *    模型（MoE）》技术总结" (gist.science), section 2.2: the routing weight is
+ *    absorbed into the activation, i.e. W_d (g a) is computed instead of
+ *    g (W_d a). oc_moe_fwd_tokens() can evaluate both orders.
+ *  - The load-balancing auxiliary loss named in section 2.4 of the same summary
+ *    ("fuse routing, permutation and aux-loss computation") and in 案例 3 of the
+ *    study notes. The pages give no formula; the reading used is
+ *    aux = E * sum_e f_e P_e with f_e = count_e / (T k) and P_e the mean full
+ *    softmax probability of expert e.
+ *  - MXFP8 (section 3 of the summary names the MXFP8 recipe for Blackwell):
+ *    OCP Microscaling Formats v1.0, section 6.3: per block of 32 elements the
+ *    shared scale is 2^(floor(log2(amax)) - 8) (8 = E4M3 emax), stored as an
+ *    UE8M0 byte, and each element is v/scale rounded to E4M3 (nearest-even,
+ *    clamped to +-448).
+ *
+ * Everything is plain loops in double precision. Expert operands are reached
+ * through oc_mat, which decodes one row at a time from bf16, MXFP8 or fp64
+ * storage; decoding is exact in every case.
+ */
+#include <math.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+
+#ifdef _OPENMP
+#include <omp.h>
+#endif
+
+/* ------------------------------------------------------------------ scalars */
+
+static double bf16_to_double(uint16_t v) {
+    uint32_t u = (uint32_t)v << 16;
+    float f;
+    memcpy(&f, &u, 4);
+    return (double)f;
+}
+
+/* E4M3 (OCP "fn" variant): 1 sign, 4 exponent (bias 7), 3 mantissa bits;
+ * exponent field 0 is subnormal (m * 2^-9); S.1111.111 is NaN; max 448. */
+double oc_e4m3_decode(uint8_t c) {
+    int s = c >> 7, ef = (c >> 3) & 15, m = c & 7;
+    double v;
+    if (ef == 15 && m == 7) return NAN;
+    if (ef == 0) v = ldexp((double)m, -9);
+    else v = ldexp(1.0 + m / 8.0, ef - 7);
+    return s ? -v : v;
+}
+
+/* Round |v| to the E4M3 grid, nearest-even, clamp to 448. v is finite. */
+uint8_t oc_e4m3_encode(double v) {
+    uint8_t sign = (signbit(v) ? 0x80 : 0x00);
+    double a = fabs(v);
+    if (a == 0.0) return sign;
+    int e = (int)floor(log2(a));
+    /* guard against log2 rounding at exact powers of two */
+    if (ldexp(1.0, e) > a) e -= 1;
+    if (ldexp(1.0, e + 1) <= a) e += 1;
+    if (e < -6) e = -6;                     /* subnormal range shares the 2^-9 quantum */
+    double q = ldexp(1.0, e - 3);           /* spacing of the grid in this binade */
+    double r = a / q;                       /* exact: power-of-two division */
+    double fl = floor(r);
+    double frac = r - fl;
+    double n;
+    if (frac > 0.5) n = fl + 1.0;
+    else if (frac < 0.5) n = fl;
+    else n = (fmod(fl, 2.0) == 0.0) ? fl : fl + 1.0;
+    double val = n * q;
+    if (val > 448.0) val = 448.0;
+    if (val == 0.0) return sign;
+    /* encode val */
+    int ve = (int)floor(log2(val));
+    if (ldexp(1.0, ve) > val) ve -= 1;
+    if (ldexp(1.0, ve + 1) <= val) ve += 1;
+    uint8_t code;
+    if (ve < -6) {
+        code = (uint8_t)(val / ldexp(1.0, -9));          /* subnormal: m = val / 2^-9 */
+    } else {
+        int mant = (int)(val / ldexp(1.0, ve - 3)) - 8;  /* 0..7 */
+        code = (uint8_t)(((ve + 7) << 3) | mant);
+    }
+    return sign | code;
+}
+
+/* UE8M0 scale byte of one block, OCP MX v1.0 section 6.3 with E4M3 emax = 8. */
+uint8_t oc_mx_scale_byte(double amax) {
+    if (!(amax > 0.0)) return 0;
+    int e = (int)floor(log2(amax));
+    if (ldexp(1.0, e) > amax) e -= 1;
+    if (ldexp(1.0, e + 1) <= amax) e += 1;
+    int b = e - 8 + 127;
+    if (b < 0) b = 0;
+    if (b > 254) b = 254;
+    return (uint8_t)b;
+}
+
+/* Quantise rows x K (K % 32 == 0) of fp32 values to E4M3 codes + UE8M0 bytes,
+ * 1x32 blocks along K. */
+void oc_mxfp8_quantize(long rows, int K, const float* src, uint8_t* codes, uint8_t* scales) {
+    long r;
+#pragma omp parallel for schedule(static)
+    for (r = 0; r < rows; ++r) {
+        for (int b = 0; b < K / 32; ++b) {
+            const float* v = src + r * (long)K + b * 32;
+            double amax = 0.0;
+            for (int i = 0; i < 32; ++i) {
+                double a = fabs((double)v[i]);
+                if (a > amax) amax = a;
+            }
+            uint8_t sb = oc_mx_scale_byte(amax);
+            scales[r * (long)(K / 32) + b] = sb;
+            double X = ldexp(1.0, (int)sb - 127);
+            for (int i = 0; i < 32; ++i)
+                codes[r * (long)K + b * 32 + i] = oc_e4m3_encode((double)v[i] / X);
+        }
+    }
+}
+
+/* Same, from bf16 storage. */
+void oc_mxfp8_quantize_bf16(long rows, int K, const uint16_t* src, uint8_t* codes, uint8_t* scales) {
+    long r;
+#pragma omp parallel for schedule(static)
+    for (r = 0; r < rows; ++r) {
+        float tmp[32];
+        for (int b = 0; b < K / 32; ++b) {
+            double amax = 0.0;
+            for (int i = 0; i < 32; ++i) {
+                tmp[i] = (float)bf16_to_double(src[r * (long)K + b * 32 + i]);
+                double a = fabs((double)tmp[i]);
+                if (a > amax) amax = a;
+            }
+            uint8_t sb = oc_mx_scale_byte(amax);
+            scales[r * (long)(K / 32) + b] = sb;
+            double X = ldexp(1.0, (int)sb - 127);
+            for (int i = 0; i < 32; ++i)
+                codes[r * (long)K + b * 32 + i] = oc_e4m3_encode((double)tmp[i] / X);
+        }
+    }
+}
+
+/* ------------------------------------------------------------ matrices */
+
+enum { OC_BF16 = 0, OC_MXFP8 = 1, OC_F64 = 2 };
+
+/* Row-major matrix [rows, cols]; for OC_MXFP8, sf holds rows x cols/32 bytes. */
+typedef struct {
+    int32_t kind;
+    int32_t cols;
+    int64_t rows;
+    const void* data;
+    const uint8_t* sf;
+} oc_mat;
+
+static void oc_row(const oc_mat* m, int64_t r, double* out) {
+    int C = m->cols;
+    if (m->kind == OC_BF16) {
+        const uint16_t* p = (const uint16_t*)m->data + r * C;
+        for (int c = 0; c < C; ++c) out[c] = bf16_to_double(p[c]);
+    } else if (m->kind == OC_MXFP8) {
+        const uint8_t* p = (const uint8_t*)m->data + r * C;
+        const uint8_t* s = m->sf + r * (C / 32);
+        for (int c = 0; c < C; ++c) out[c] = oc_e4m3_decode(p[c]) * ldexp(1.0, (int)s[c / 32] - 127);
+    } else {
+        const double* p = (const double*)m->data + r * C;
+        for (int c = 0; c < C; ++c) out[c] = p[c];
+    }
+}
+
+/* Sub-matrix view: rows [r0, r0+nrows) of m (an expert's slice of [E*R, C]). */
+static oc_mat oc_slice(const oc_mat* m, int64_t r0, int64_t nrows) {
+    oc_mat s = *m;
+    s.rows = nrows;
+    if (m->kind == OC_BF16) s.data = (const uint16_t*)m->data + r0 * m->cols;
+    else if (m->kind == OC_MXFP8) {
+        s.data = (const uint8_t*)m->data + r0 * m->cols;
+        s.sf = m->sf + r0 * (m->cols / 32);
+    } else s.data = (const double*)m->data + r0 * m->cols;
+    return s;
+}
+
+static double dot(const double* a, const double* b, int n) {
+    double s = 0.0;
+    for (int i = 0; i < n; ++i) s += a[i] * b[i];
+    return s;
+}
+
+/* y = M v  (M [R, C], v [C]) */
+static void matvec(const oc_mat* M, const double* v, double* y, double* rowbuf) {
+    for (int64_t r = 0; r < M->rows; ++r) {
+        oc_row(M, r, rowbuf);
+        y[r] = dot(rowbuf, v, M->cols);
+    }
+}
+
+/* y += M^T v  (M [R, C], v [R], y [C]) */
+static void matvec_t_acc(const oc_mat* M, const double* v, double* y, double* rowbuf) {
+    for (int64_t r = 0; r < M->rows; ++r) {
+        oc_row(M, r, rowbuf);
+        for (int c = 0; c < M->cols; ++c) y[c] += rowbuf[c] * v[r];
+    }
+}
+
+static double sigmoid(double z) { return 1.0 / (1.0 + exp(-z)); }
+static double silu(double z) { return z * sigmoid(z); }
+static double silu_grad(double z) { double s = sigmoid(z); return s * (1.0 + z * (1.0 - s)); }
+
+/* Round a double to the MXFP8 grid of its 32-block, in place, blocks along n.
+ * The values are first rounded to fp32 (the precision in which the quantiser
+ * takes its decisions), then quantised and decoded back. */
+static void mx_roundtrip(double* v, int n) {
+    for (int b = 0; b < n / 32; ++b) {
+        float t[32];
+        double amax = 0.0;
+        for (int i = 0; i < 32; ++i) {
+            t[i] = (float)v[b * 32 + i];
+            if (fabs((double)t[i]) > amax) amax = fabs((double)t[i]);
+        }
+        uint8_t sb = oc_mx_scale_byte(amax);
+        double X = ldexp(1.0, (int)sb - 127);
+        for (int i = 0; i < 32; ++i) v[b * 32 + i] = oc_e4m3_decode(oc_e4m3_encode((double)t[i] / X)) * X;
+    }
+}
+
+/* ------------------------------------------------------------ routing */
+
+/* logits[t,e] = sum_h x[t,h] W_r[e,h] (+ bias[e]); fp64 sum, one final rounding
+ * to fp32 when round_f32 (router logits are kept in high precision: the study
+ * notes' 踩过的坑 section warns that low-precision logits collapse routing). */
+void oc_router_logits(int T, int H, int E, const oc_mat* x, const oc_mat* Wr, const float* bias,
+                      int round_f32, double* logits) {
+    int t;
+#pragma omp parallel for schedule(static)
+    for (t = 0; t < T; ++t) {
+        double* xr = (double*)malloc(sizeof(double) * H);
+        double* wr = (double*)malloc(sizeof(double) * H);
+        oc_row(x, t, xr);
+        for (int e = 0; e < E; ++e) {
+            oc_row(Wr, e, wr);
+            double s = dot(xr, wr, H);
+            if (bias) s += (double)bias[e];
+            logits[(long)t * E + e] = round_f32 ? (double)(float)s : s;
+        }
+        free(xr);
+        free(wr);
+    }
+}
+
+/* s[t,:] = softmax(l[t,:]) (score 0) or sigmoid(l[t,e]) (score 1). */
+void oc_scores(int T, int E, int score, const double* logits, double* s) {
+    for (int t = 0; t < T; ++t) {
+        const double* l = logits + (long)t * E;
+        double* o = s + (long)t * E;
+        if (score == 0) {
+            double mx = l[0];
+            for (int e = 1; e < E; ++e) if (l[e] > mx) mx = l[e];
+            double z = 0.0;
+            for (int e = 0; e < E; ++e) { o[e] = exp(l[e] - mx); z += o[e]; }
+            for (int e = 0; e < E; ++e) o[e] /= z;
+        } else {
+            for (int e = 0; e < E; ++e) o[e] = sigmoid(l[e]);
+        }
+    }
+}
+
+/* Top-k by logit value, descending; equal values go to the lower expert index
+ * first. Slot j holds the j-th largest. (Selecting on logits is the same as
+ * selecting on softmax or sigmoid scores: both maps are increasing.) */
+void oc_topk(int T, int E, int k, const double* logits, int32_t* idx) {
+    for (int t = 0; t < T; ++t) {
+        const double* l = logits + (long)t * E;
+        for (int j = 0; j < k; ++j) {
+            int best = -1;
+            for (int e = 0; e < E; ++e) {
+                int taken = 0;
+                for (int i = 0; i < j; ++i) if (idx[(long)t * k + i] == e) taken = 1;
+                if (taken) continue;
+                if (best < 0 || l[e] > l[best]) best = e;   /* strict: ties keep the lower index */
+            }
+            idx[(long)t * k + j] = best;
+        }
+    }
+}
+
+/* gates[t,j] = s[t, idx[t,j]] (/ sum over the selected when norm) * route_scale */
+void oc_gates(int T, int E, int k, int norm, double route_scale, const double* s, const int32_t* idx,
+              double* gates) {
+    for (int t = 0; t < T; ++t) {
+        double z = 0.0;
+        for (int j = 0; j < k; ++j) z += s[(long)t * E + idx[(long)t * k + j]];
+        for (int j = 0; j < k; ++j) {
+            double g = s[(long)t * E + idx[(long)t * k + j]];
+            if (norm) g /= z;
+            gates[(long)t * k + j] = g * route_scale;
+        }
+    }
+}
+
+/* Expert-contiguous order: counts, exclusive-scan offsets, and a stable
+ * counting sort of the flattened pairs (t*k + j) by expert. */
+void oc_maps(int T, int E, int k, const int32_t* idx, int32_t* counts, int32_t* offsets, int32_t* row_of,
+             int32_t* src_of) {
+    for (int e = 0; e < E; ++e) counts[e] = 0;
+    for (long p = 0; p < (long)T * k; ++p) counts[idx[p]] += 1;
+    offsets[0] = 0;
+    for (int e = 0; e < E; ++e) offsets[e + 1] = offsets[e] + counts[e];
+    int32_t* fill = (int32_t*)malloc(sizeof(int32_t) * E);
+    for (int e = 0; e < E; ++e) fill[e] = offsets[e];
+    for (long p = 0; p < (long)T * k; ++p) {
+        int e = idx[p];
+        int r = fill[e]++;
+        row_of[p] = r;
+        src_of[r] = (int32_t)(p / k);
+    }
+    free(fill);
+}
+
+/* aux = E * sum_e f_e P_e, f_e = counts[e]/(T k), P_e = mean_t s[t,e] (full softmax). */
+double oc_aux(int T, int E, int k, const double* s, const int32_t* counts) {
+    double acc = 0.0;
+    for (int e = 0; e < E; ++e) {
+        double P = 0.0;
+        for (int t = 0; t < T; ++t) P += s[(long)t * E + e];
+        P /= (double)T;
+        double f = (double)counts[e] / ((double)T * k);
+        acc += f * P;
+    }
+    return (double)E * acc;
+}
+
+/* ------------------------------------------------------------ experts */
+
+/* One expert on one token vector xv [H]:
+ *   z_g = W_g xv, z_u = W_u xv, a = silu(z_g) * z_u   (W_g, W_u: [F, H])
+ * With mx != 0 the activation fed to the down projection is rounded to MXFP8
+ * after the gate is folded in (see oc_moe_fwd_tokens). */
+static void expert_act(const oc_mat* Wg, const oc_mat* Wu, const double* xv, double* zg, double* zu, double* a,
+                       double* rowbuf) {
+    int F = (int)Wg->rows;
+    matvec(Wg, xv, zg, rowbuf);
+    matvec(Wu, xv, zu, rowbuf);
+    for (int f = 0; f < F; ++f) a[f] = silu(zg[f]) * zu[f];
+}
+
+/*
+ * Forward output rows for a list of tokens, given the routing.
+ *
+ *   y[t] = sum_j g[t,j] * W_d[e_j] (silu(W_g[e_j] x_t) * (W_u[e_j] x_t))
+ *          (+ shared expert on every token, weight 1)
+ *
+ * fold = 1 evaluates W_d (g a) (the memory-efficient permutation order),
+ * fold = 0 evaluates g (W_d a); the two agree up to rounding.
+ * mx = 1 is the MXFP8 recipe: x is rounded to MXFP8 (1x32 blocks along H)
+ * before the expert GEMMs, and the folded activation g*a (and the shared
+ * expert's a) is rounded to MXFP8 along F before the down projection. The
+ * weight matrices are then given as OC_MXFP8 (already quantised).
+ * Weight layouts: Wg, Wu [E*F, H]; Wd [E*H, F]; shared Wgs, Wus [F, H], Wds [H, F].
+ */
+int oc_moe_fwd_tokens(int T, int H, int E, int k, int F, int S, int mx, int fold, const oc_mat* x,
+                      const oc_mat* Wg, const oc_mat* Wu, const oc_mat* Wd, const oc_mat* Wgs, const oc_mat* Wus,
+                      const oc_mat* Wds, const int32_t* idx, const double* gates, int n_tok, const int32_t* toks,
+                      double* y_out, double* shared_out) {
+    int i;
+    (void)T;
+    (void)E;
+#pragma omp parallel for schedule(dynamic, 1)
+    for (i = 0; i < n_tok; ++i) {
+        int t = toks[i];
+        int maxd = H > F ? H : F;
+        double* xv = (double*)malloc(sizeof(double) * H);
+        double* zg = (double*)malloc(sizeof(double) * F);
+        double* zu = (double*)malloc(sizeof(double) * F);
+        double* a = (double*)malloc(sizeof(double) * F);
+        double* o = (double*)malloc(sizeof(double) * H);
+        double* rowbuf = (double*)malloc(sizeof(double) * maxd);
+        double* y = y_out + (long)i * H;
+        oc_row(x, t, xv);
+        if (mx) mx_roundtrip(xv, H);
+        for (int h = 0; h < H; ++h) y[h] = 0.0;
+        for (int j = 0; j < k; ++j) {
+            int e = idx[(long)t * k + j];
+            double g = gates[(long)t * k + j];
+            oc_mat we_g = oc_slice(Wg, (int64_t)e * F, F);
+            oc_mat we_u = oc_slice(Wu, (int64_t)e * F, F);
+            oc_mat we_d = oc_slice(Wd, (int64_t)e * H, H);
+            expert_act(&we_g, &we_u, xv, zg, zu, a, rowbuf);
+            if (fold) {
+                for (int f = 0; f < F; ++f) a[f] *= g;
+                if (mx) mx_roundtrip(a, F);
+                matvec(&we_d, a, o, rowbuf);
+                for (int h = 0; h < H; ++h) y[h] += o[h];
+            } else {
+                if (mx) mx_roundtrip(a, F);
+                matvec(&we_d, a, o, rowbuf);
+                for (int h = 0; h < H; ++h) y[h] += g * o[h];
+            }
+        }
+        if (S) {
+            expert_act(Wgs, Wus, xv, zg, zu, a, rowbuf);
+            if (mx) mx_roundtrip(a, F);
+            matvec(Wds, a, o, rowbuf);
+            for (int h = 0; h < H; ++h) y[h] += o[h];
+            if (shared_out)
+                for (int h = 0; h < H; ++h) shared_out[(long)i * H + h] = o[h];
+        }
+        free(xv); free(zg); free(zu); free(a); free(o); free(rowbuf);
+    }
+    return 0;
+}
+
+/*
+ * Dense all-experts brute force (a pin for the per-token loop): every expert is
+ * evaluated on every token and the results are combined with a dense [T,E]
+ * gate matrix that is zero off the selected experts. No routing lists at all.
+ */
+int oc_moe_fwd_dense(int T, int H, int E, int F, const oc_mat* x, const oc_mat* Wg, const oc_mat* Wu,
+                     const oc_mat* Wd, const double* gate_dense, double* y_out) {
+    int t;
+#pragma omp parallel for schedule(dynamic, 1)
+    for (t = 0; t < T; ++t) {
+        int maxd = H > F ? H : F;
+        double* xv = (double*)malloc(sizeof(double) * H);
+        double* zg = (double*)malloc(sizeof(double) * F);
+        double* zu = (double*)malloc(sizeof(double) * F);
+        double* a = (double*)malloc(sizeof(double) * F);
+        double* o = (double*)malloc(sizeof(double) * H);
+        double* rowbuf = (double*)malloc(sizeof(double) * maxd);
+        oc_row(x, t, xv);
+        for (int h = 0; h < H; ++h) y_out[(long)t * H + h] = 0.0;
+        for (int e = 0; e < E; ++e) {
+            oc_mat we_g = oc_slice(Wg, (int64_t)e * F, F);
+            oc_mat we_u = oc_slice(Wu, (int64_t)e * F, F);
+            oc_mat we_d = oc_slice(Wd, (int64_t)e * H, H);
+            expert_act(&we_g, &we_u, xv, zg, zu, a, rowbuf);
+            matvec(&we_d, a, o, rowbuf);
+            for (int h = 0; h < H; ++h) y_out[(long)t * H + h] += gate_dense[(long)t * E + e] * o[h];
+        }
+        free(xv); free(zg); free(zu); free(a); free(o); free(rowbuf);
+    }
+    return 0;
+}
+
+/* Expert part of the layer for explicit (row -> expert, gate) lists, the way
+ * the grouped GEMM stage sees it: a row r holds activation xp[r] routed to
+ * expert e_of[r] with gate g_of[r]. Outputs ap [n, F] (g folded, optionally
+ * MXFP8-rounded) and o [n, H] = W_d ap. Rows are independent. */
+int oc_expert_rows(int H, int F, int mx, const oc_mat* xp, const int32_t* e_of, const double* g_of,
+                   const oc_mat* Wg, const oc_mat* Wu, const oc_mat* Wd, int n, const int32_t* rows,
+                   double* zg_out, double* zu_out, double* ap_out, double* o_out) {
+    int i;
+#pragma omp parallel for schedule(dynamic, 1)
+    for (i = 0; i < n; ++i) {
+        int r = rows[i];
+        int e = e_of[r];
+        int maxd = H > F ? H : F;
+        double* xv = (double*)malloc(sizeof(double) * H);
+        double* zg = (double*)malloc(sizeof(double) * F);
+        double* zu = (double*)malloc(sizeof(double) * F);
+        double* a = (double*)malloc(sizeof(double) * F);
+        double* rowbuf = (double*)malloc(sizeof(double) * maxd);
+        oc_row(xp, r, xv);
+        if (mx) mx_roundtrip(xv, H);
+        oc_mat we_g = oc_slice(Wg, (int64_t)e * F, F);
+        oc_mat we_u = oc_slice(Wu, (int64_t)e * F, F);
+        oc_mat we_d = oc_slice(Wd, (int64_t)e * H, H);
+        expert_act(&we_g, &we_u, xv, zg, zu, a, rowbuf);
+        for (int f = 0; f < F; ++f) a[f] *= g_of[r];
+        if (mx) mx_roundtrip(a, F);
+        if (zg_out) for (int f = 0; f < F; ++f) zg_out[(long)i * F + f] = zg[f];
+        if (zu_out) for (int f = 0; f < F; ++f) zu_out[(long)i * F + f] = zu[f];
+        if (ap_out) for (int f = 0; f < F; ++f) ap_out[(long)i * F + f] = a[f];
+        if (o_out) matvec(&we_d, a, o_out + (long)i * H, rowbuf);
+        free(xv); free(zg); free(zu); free(a); free(rowbuf);
+    }
+    return 0;
+}
+
+/* ------------------------------------------------------------ backward */
+
+/*
+ * Exact derivative of the forward (bf16 / fp64 operands, softmax or sigmoid
+ * scores with selected-normalised gates), for upstream dY [T,H] and d_aux.
+ * Per token t of the list:
+ *   for each selected j (e = idx[t,j]):
+ *     z_g, z_u, a = silu(z_g) z_u, v = W_d[e]^T dY_t,  dg_j = <v, a>
+ *     da = g_j v, dz_g = da z_u silu'(z_g), dz_u = da silu(z_g)
+ *     dx_t += W_g[e]^T dz_g + W_u[e]^T dz_u
+ *   gate path (c = route_scale, p = softmax over the selected logits):
+ *     softmax, normalised: g_j = c p_j, so
+ *       dl[sel_j] = g_j dg_j - g_j (sum_i g_i dg_i) / c
+ *     sigmoid, normalised: g_j = c s_j / Z, s = sigmoid(l), Z = sum_sel s_i, so
+ *       dl[sel_j] = s_j (1 - s_j) (c/Z) (dg_j - (sum_i g_i dg_i) / c)
+ *     softmax, unnormalised: g_j = c s_j, dl = s (ds - <s, ds>), ds_{e_j} = c dg_j
+ *   aux path (softmax only, counts are constants):
+ *     c_e = E count_e / (T k) / T,  dl[t,e] += d_aux s_e (c_e - sum_i s_i c_i)
+ *   router: dx_t += sum_e dl[t,e] W_r[e]
+ * logits, s (scores), gates, idx and counts are the forward's.
+ */
+int oc_moe_bwd_tokens(int T, int H, int E, int k, int F, int score, int norm, double route_scale, int aux_on,
+                      double d_aux, const oc_mat* x, const oc_mat* Wr, const oc_mat* Wg, const oc_mat* Wu,
+                      const oc_mat* Wd, const oc_mat* dY, const int32_t* idx, const double* s_all,
+                      const double* s_softmax, const int32_t* counts, int n_tok, const int32_t* toks,
+                      double* dx_out, double* dl_out, double* dg_out) {
+    int i;
+#pragma omp parallel for schedule(dynamic, 1)
+    for (i = 0; i < n_tok; ++i) {
+        int t = toks[i];
+        int maxd = H > F ? H : F;
+        double* xv = (double*)malloc(sizeof(double) * H);
+        double* dy = (double*)malloc(sizeof(double) * H);
+        double* zg = (double*)malloc(sizeof(double) * F);
+        double* zu = (double*)malloc(sizeof(double) * F);
+        double* a = (double*)malloc(sizeof(double) * F);
+        double* v = (double*)malloc(sizeof(double) * F);
+        double* dzg = (double*)malloc(sizeof(double) * F);
+        double* dzu = (double*)malloc(sizeof(double) * F);
+        double* rowbuf = (double*)malloc(sizeof(double) * maxd);
+        double* dg = (double*)malloc(sizeof(double) * k);
+        double* g = (double*)malloc(sizeof(double) * k);
+        double* dx = dx_out + (long)i * H;
+        double* dl = dl_out + (long)i * E;
+        const double* s = s_all + (long)t * E;
+        oc_row(x, t, xv);
+        oc_row(dY, t, dy);
+        for (int h = 0; h < H; ++h) dx[h] = 0.0;
+        for (int e = 0; e < E; ++e) dl[e] = 0.0;
+        /* gates again from the scores (as the forward defined them) */
+        double Z = 0.0;
+        for (int j = 0; j < k; ++j) Z += s[idx[(long)t * k + j]];
+        for (int j = 0; j < k; ++j) {
+            double gj = s[idx[(long)t * k + j]];
+            if (norm) gj /= Z;
+            g[j] = gj * route_scale;
+        }
+        for (int j = 0; j < k; ++j) {
+            int e = idx[(long)t * k + j];
+            oc_mat we_g = oc_slice(Wg, (int64_t)e * F, F);
+            oc_mat we_u = oc_slice(Wu, (int64_t)e * F, F);
+            oc_mat we_d = oc_slice(Wd, (int64_t)e * H, H);
+            expert_act(&we_g, &we_u, xv, zg, zu, a, rowbuf);
+            for (int f = 0; f < F; ++f) v[f] = 0.0;
+            matvec_t_acc(&we_d, dy, v, rowbuf);           /* v = W_d^T dY_t */
+            dg[j] = dot(v, a, F);
+            for (int f = 0; f < F; ++f) {
+                double da = g[j] * v[f];
+                dzg[f] = da * zu[f] * silu_grad(zg[f]);
+                dzu[f] = da * silu(zg[f]);
+            }
+            matvec_t_acc(&we_g, dzg, dx, rowbuf);
+            matvec_t_acc(&we_u, dzu, dx, rowbuf);
+        }
+        if (dg_out) for (int j = 0; j < k; ++j) dg_out[(long)i * k + j] = dg[j];
+        /* gate path */
+        double sgd = 0.0;
+        for (int j = 0; j < k; ++j) sgd += g[j] * dg[j];
+        for (int j = 0; j < k; ++j) {
+            int e = idx[(long)t * k + j];
+            if (score == 0) {
+                if (norm) {
+                    /* g_j = c exp(l_j) / sum_sel exp(l_i):  c p_j (dg_j - sum_i p_i dg_i) */
+                    dl[e] += g[j] * dg[j] - g[j] * sgd / route_scale;
+                }
+                /* unnormalised softmax gates are handled below (all E logits move) */
+            } else {
+                double sj = s[e];
+                if (norm) {
+                    /* g_j = c s_j / Z, dg/ds_j: c/Z (dg_j - sum_i g_i dg_i / c) */
+                    double dsj = (route_scale / Z) * (dg[j] - sgd / route_scale);
+                    dl[e] += dsj * sj * (1.0 - sj);
+                } else {
+                    dl[e] += route_scale * dg[j] * sj * (1.0 - sj);
+                }
+            }
+        }
+        if (score == 0 && !norm) {
+            /* g_j = c s_{e_j}, s = softmax over all E: ds_e = c dg_j at e = e_j */
+            double* ds = (double*)calloc(E, sizeof(double));
+            for (int j = 0; j < k; ++j) ds[idx[(long)t * k + j]] += route_scale * dg[j];
+            double sds = 0.0;
+            for (int e = 0; e < E; ++e) sds += s[e] * ds[e];
+            for (int e = 0; e < E; ++e) dl[e] += s[e] * (ds[e] - sds);
+            free(ds);
+        }
+        /* aux path */
+        if (aux_on) {
+            const double* ss = s_softmax + (long)t * E;
+            double sc = 0.0;
+            for (int e = 0; e < E; ++e) {
+                double ce = (double)E * (double)counts[e] / ((double)T * k) / (double)T;
+                sc += ss[e] * ce;
+            }
+            for (int e = 0; e < E; ++e) {
+                double ce = (double)E * (double)counts[e] / ((double)T * k) / (double)T;
+                dl[e] += d_aux * ss[e] * (ce - sc);
+            }
+        }
+        /* router path */
+        for (int e = 0; e < E; ++e) {
+            if (dl[e] == 0.0) continue;
+            oc_row(Wr, e, rowbuf);
+            for (int h = 0; h < H; ++h) dx[h] += dl[e] * rowbuf[h];
+        }
+        free(xv); free(dy); free(zg); free(zu); free(a); free(v); free(dzg); free(dzu); free(rowbuf);
+        free(dg); free(g);
+    }
+    return 0;
+}
+
+/*
+ * Expert weight gradients for a list of experts, summing over every token
+ * routed to each one (rows of the stable order, i.e. ascending token index):
+ *   dW_d[e] += g dY_t (x) a,  dW_g[e] += dz_g (x) x_t,  dW_u[e] += dz_u (x) x_t
+ * Outputs: dWg, dWu [n_exp, F, H]; dWd [n_exp, H, F]. Experts with no token
+ * get exact zeros. gates are the forward's [T,k].
+ */
+int oc_moe_bwd_expert_dw(int T, int H, int E, int k, int F, const oc_mat* x, const oc_mat* Wg,
+                         const oc_mat* Wu, const oc_mat* Wd, const oc_mat* dY, const int32_t* idx,
+                         const double* gates, int n_exp, const int32_t* exps, double* dWg, double* dWu,
+                         double* dWd) {
+    (void)E;
+    for (int q = 0; q < n_exp; ++q) {
+        int e = exps[q];
+        double* gG = dWg + (long)q * F * H;
+        double* gU = dWu + (long)q * F * H;
+        double* gD = dWd + (long)q * H * F;
+        memset(gG, 0, sizeof(double) * (size_t)F * H);
+        memset(gU, 0, sizeof(double) * (size_t)F * H);
+        memset(gD, 0, sizeof(double) * (size_t)F * H);
+        /* tokens routed to e, with their gate */
+        int n = 0;
+        int32_t* tl = (int32_t*)malloc(sizeof(int32_t) * (T > 0 ? T : 1));
+        double* gl = (double*)malloc(sizeof(double) * (T > 0 ? T : 1));
+        for (int t = 0; t < T; ++t)
+            for (int j = 0; j < k; ++j)
+                if (idx[(long)t * k + j] == e) { tl[n] = t; gl[n] = gates[(long)t * k + j]; ++n; }
+        oc_mat we_g = oc_slice(Wg, (int64_t)e * F, F);
+        oc_mat we_u = oc_slice(Wu, (int64_t)e * F, F);
+        oc_mat we_d = oc_slice(Wd, (int64_t)e * H, H);
+        /* per-token intermediates, then the outer products; parallel over the
+         * output rows so each thread owns its rows and the token order of each
+         * sum stays ascending. */
+        double* A = (double*)malloc(sizeof(double) * (size_t)(n > 0 ? n : 1) * F);
+        double* DZG = (double*)malloc(sizeof(double) * (size_t)(n > 0 ? n : 1) * F);
+        double* DZU = (double*)malloc(sizeof(double) * (size_t)(n > 0 ? n : 1) * F);
+        double* XV = (double*)malloc(sizeof(double) * (size_t)(n > 0 ? n : 1) * H);
+        double* DY = (double*)malloc(sizeof(double) * (size_t)(n > 0 ? n : 1) * H);
+        int i;
+#pragma omp parallel for schedule(dynamic, 1)
+        for (i = 0; i < n; ++i) {
+            int maxd = H > F ? H : F;
+            double* zg = (double*)malloc(sizeof(double) * F);
+            double* zu = (double*)malloc(sizeof(double) * F);
+            double* v = (double*)malloc(sizeof(double) * F);
+            double* rowbuf = (double*)malloc(sizeof(double) * maxd);
+            double* xv = XV + (long)i * H;
+            double* dy = DY + (long)i * H;
+            double* a = A + (long)i * F;
+            oc_row(x, tl[i], xv);
+            oc_row(dY, tl[i], dy);
+            expert_act(&we_g, &we_u, xv, zg, zu, a, rowbuf);
+            for (int f = 0; f < F; ++f) v[f] = 0.0;
+            matvec_t_acc(&we_d, dy, v, rowbuf);
+            for (int f = 0; f < F; ++f) {
+                double da = gl[i] * v[f];
+                DZG[(long)i * F + f] = da * zu[f] * silu_grad(zg[f]);
+                DZU[(long)i * F + f] = da * silu(zg[f]);
+            }
+            free(zg); free(zu); free(v); free(rowbuf);
+        }
+        int f;
+#pragma omp parallel for schedule(static)
+        for (f = 0; f < F; ++f) {
+            for (int ii = 0; ii < n; ++ii) {
+                double cg = DZG[(long)ii * F + f], cu = DZU[(long)ii * F + f];
+                const double* xv = XV + (long)ii * H;
+                for (int h = 0; h < H; ++h) {
+                    gG[(long)f * H + h] += cg * xv[h];
+                    gU[(long)f * H + h] += cu * xv[h];
+                }
+            }
+        }
+        int h;
+#pragma omp parallel for schedule(static)
+        for (h = 0; h < H; ++h) {
+            for (int ii = 0; ii < n; ++ii) {
+                double c = gl[ii] * DY[(long)ii * H + h];
+                const double* a = A + (long)ii * F;
+                for (int f2 = 0; f2 < F; ++f2) gD[(long)h * F + f2] += c * a[f2];
+            }
+        }
+        free(tl); free(gl); free(A); free(DZG); free(DZU); free(XV); free(DY);
+    }
+    return 0;
+}
+
+/* dW_r[e,h] = sum_t dl[t,e] x[t,h] over all T tokens (ascending t). */
+void oc_router_dwr(int T, int H, int E, const double* dl, const oc_mat* x, double* dWr) {
+    int e;
+#pragma omp parallel for schedule(static)
+    for (e = 0; e < E; ++e) {
+        double* xr = (double*)malloc(sizeof(double) * H);
+        double* out = dWr + (long)e * H;
+        for (int h = 0; h < H; ++h) out[h] = 0.0;
+        for (int t = 0; t < T; ++t) {
+            double c = dl[(long)t * E + e];
+            if (c == 0.0) continue;
+            oc_row(x, t, xr);
+            for (int h = 0; h < H; ++h) out[h] += c * xr[h];
+        }
+        free(xr);
+    }
+}
+
+/* Unpermute-sum with unit weights: y[t] = sum_j o[row_of[t,j]] (+ shared[t]). */
+void oc_unpermute(int T, int H, int k, const double* o, const int32_t* row_of, const double* shared, double* y) {
+    for (int t = 0; t < T; ++t)
+        for (int h = 0; h < H; ++h) {
+            double s = 0.0;
+            for (int j = 0; j < k; ++j) s += o[(long)row_of[(long)t * k + j] * H + h];
+            if (shared) s += shared[(long)t * H + h];
+            y[(long)t * H + h] = s;
+        }
+}
+
+int oc_num_threads(void) {
+#ifdef _OPENMP
+    return omp_get_max_threads();
+#else
+    return 1;
+#endif
+}

@@ -1,0 +1,398 @@
+"""Pins of the CPU oracle against things other than itself (no GPU).
+
+Each test ties one oracle function to an independent fact: a dense brute
+force, a library routine (torch fp64 matmul / sort / float8 cast), a closed
+form, an invariant, central finite differences, or hand-computed OCP MX
+values (tests/golden/mxfp8_ocp_cases.txt). A plausible mistake anywhere in the
+oracle (a dropped term, a wrong sign or index, a transposed operand) fails at
+least one of them.
+"""
+import math
+import os
+
+import pytest
+import torch
+
+from mixture_experts_layer_aux_b200.synthetic import Workload, make_inputs, random_logits
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden", "mxfp8_ocp_cases.txt")
+
+
+def small(T=24, H=64, E=6, k=2, F=96, **kw):
+    return Workload("small", T=T, H=H, E=E, k=k, F=F, **kw)
+
+
+def ref_swiglu(x, Wg, Wu, Wd):
+    """torch fp64: W_d (silu(W_g x) * (W_u x)) for rows of x."""
+    zg = x @ Wg.T
+    zu = x @ Wu.T
+    return (torch.nn.functional.silu(zg) * zu) @ Wd.T
+
+
+# --------------------------------------------------------------- routing
+
+
+def test_router_logits_match_torch_fp64_matmul(oracle):
+    wl = small(T=33, H=96, E=7)
+    inp = make_inputs(wl, seed=1)
+    bias = torch.linspace(-1, 1, wl.E)
+    l = oracle.router_logits(inp["x"], inp["W_r"], bias)
+    ref = (inp["x"].double() @ inp["W_r"].double().T + bias.double()).float().double()
+    # fp64 sums in a different order may round to an adjacent fp32
+    assert torch.allclose(l, ref, rtol=2e-7, atol=1e-9)
+    l64 = oracle.router_logits(inp["x"], inp["W_r"], None, round_f32=False)
+    assert torch.allclose(l64, inp["x"].double() @ inp["W_r"].double().T, rtol=1e-13, atol=1e-13)
+
+
+def test_scores_match_torch(oracle):
+    l = random_logits(17, 9, seed=3).double()
+    assert torch.allclose(oracle.scores(l, "softmax"), torch.softmax(l, dim=1), rtol=1e-14, atol=1e-16)
+    assert torch.allclose(oracle.scores(l, "sigmoid"), torch.sigmoid(l), rtol=1e-14, atol=1e-16)
+
+
+@pytest.mark.parametrize("ties", [False, True])
+@pytest.mark.parametrize("E,k", [(8, 2), (128, 8), (5, 5), (1, 1)])
+def test_topk_matches_stable_sort(oracle, E, k, ties):
+    l = random_logits(64, E, seed=E + k, ties=ties).double()
+    idx = oracle.topk(l, k)
+    ref = torch.sort(-l, dim=1, stable=True).indices[:, :k].to(torch.int32)
+    assert torch.equal(idx, ref)
+
+
+def test_topk_all_equal_logits_picks_lowest_indices(oracle):
+    l = torch.zeros(5, 16, dtype=torch.float64)
+    idx = oracle.topk(l, 4)
+    assert torch.equal(idx, torch.arange(4, dtype=torch.int32).repeat(5, 1))
+    r = oracle.route(l, 4)
+    assert torch.allclose(r["gates"], torch.full((5, 4), 0.25, dtype=torch.float64), rtol=0, atol=1e-16)
+    # uniform probabilities: aux = E * sum_e f_e / E = 1 for any f
+    assert r["aux"] == pytest.approx(1.0, abs=1e-14)
+
+
+def test_gates_sum_to_route_scale(oracle):
+    l = random_logits(40, 32, seed=5).double()
+    r = oracle.route(l, 8, "softmax", True, 1.0)
+    assert torch.allclose(r["gates"].sum(1), torch.ones(40, dtype=torch.float64), atol=1e-14)
+    r = oracle.route(l, 8, "sigmoid", True, 2.5)
+    assert torch.allclose(r["gates"].sum(1), torch.full((40,), 2.5, dtype=torch.float64), atol=1e-14)
+    # softmax renormalised over the selected = softmax of the selected logits
+    r = oracle.route(l, 8, "softmax", True, 1.0)
+    sel = torch.gather(l, 1, r["idx"].long())
+    assert torch.allclose(r["gates"], torch.softmax(sel, dim=1), atol=1e-15)
+    # sigmoid: g = 2.5 * sigma(l_sel) / sum sigma(l_sel)
+    r = oracle.route(l, 8, "sigmoid", True, 2.5)
+    sg = torch.sigmoid(torch.gather(l, 1, r["idx"].long()))
+    assert torch.allclose(r["gates"], 2.5 * sg / sg.sum(1, keepdim=True), atol=1e-15)
+
+
+def test_aux_matches_vectorised_closed_form(oracle):
+    T, E, k = 50, 12, 3
+    l = random_logits(T, E, seed=7).double()
+    r = oracle.route(l, k)
+    counts = torch.bincount(r["idx"].flatten().long(), minlength=E).double()
+    ref = E * ((counts / (T * k)) * torch.softmax(l, 1).mean(0)).sum().item()
+    assert r["aux"] == pytest.approx(ref, rel=1e-13)
+    # perfectly balanced counts and uniform P: aux = 1
+    s = torch.full((T, E), 1.0 / E, dtype=torch.float64)
+    c = torch.full((E,), T * k // E, dtype=torch.int32)
+    assert oracle.aux(s, c, k) == pytest.approx(T * k // E * E / (T * k), abs=1e-14)
+
+
+@pytest.mark.parametrize("T,E,k,zero", [(64, 8, 2, 0), (300, 128, 8, 4), (1, 4, 4, 0), (77, 16, 1, 3)])
+def test_maps_match_stable_sort_and_invariants(oracle, T, E, k, zero):
+    from mixture_experts_layer_aux_b200.synthetic import random_routing
+    idx = random_routing(T, E, k, seed=T, zero_experts=zero)
+    counts, offsets, row_of, src_of = oracle.maps(idx, E)
+    flat = idx.flatten().long()
+    srt = torch.sort(flat, stable=True)
+    assert torch.equal(counts.long(), torch.bincount(flat, minlength=E))
+    assert torch.equal(offsets[1:].long(), torch.cumsum(counts.long(), 0)) and offsets[0] == 0
+    assert int(counts.sum()) == T * k == int(offsets[-1])
+    assert torch.equal(src_of.long(), srt.indices // k)
+    ref_row = torch.empty(T * k, dtype=torch.long)
+    ref_row[srt.indices] = torch.arange(T * k)
+    assert torch.equal(row_of.flatten().long(), ref_row)
+    # bijection and src_of[row_of[t,j]] == t
+    assert torch.equal(torch.sort(row_of.flatten()).values.long(), torch.arange(T * k))
+    assert torch.equal(src_of[row_of.flatten().long()].long(), torch.arange(T).repeat_interleave(k))
+    if zero:
+        assert (counts[E - zero:] == 0).all()
+
+
+def test_permute_then_unpermute_is_k_times_identity(oracle):
+    from mixture_experts_layer_aux_b200.synthetic import random_routing
+    T, E, k, H = 40, 8, 3, 16
+    idx = random_routing(T, E, k, seed=2)
+    _, _, row_of, src_of = oracle.maps(idx, E)
+    x = torch.randn(T, H, dtype=torch.float64)
+    xp = x[src_of.long()]                     # permute = gather by src_of
+    y = oracle.unpermute(xp, row_of)
+    assert torch.equal(y, k * x) or torch.allclose(y, k * x, rtol=1e-15, atol=0)
+    # one-hot selection: only slot 0 rows non-zero -> recovers x exactly
+    o = torch.zeros_like(xp)
+    o[row_of[:, 0].long()] = x
+    assert torch.equal(oracle.unpermute(o, row_of), x)
+
+
+# --------------------------------------------------------------- experts
+
+
+def test_single_expert_is_plain_swiglu_mlp(oracle):
+    wl = small(T=9, H=64, E=1, k=1, F=96)
+    inp = make_inputs(wl, seed=4)
+    r = oracle.layer_fwd(wl, inp)
+    assert torch.equal(r["idx"], torch.zeros(9, 1, dtype=torch.int32))
+    assert torch.allclose(r["gates"], torch.ones(9, 1, dtype=torch.float64))
+    ref = ref_swiglu(inp["x"].double(), inp["W_g"][0].double(), inp["W_u"][0].double(), inp["W_d"][0].double())
+    assert torch.allclose(r["y"], ref, rtol=1e-12, atol=1e-14)
+
+
+def test_k_equals_E_is_dense_softmax_mixture(oracle):
+    wl = small(T=11, H=32, E=4, k=4, F=64)
+    inp = make_inputs(wl, seed=5)
+    r = oracle.layer_fwd(wl, inp)
+    l = r["logits"]
+    p = torch.softmax(l, 1)
+    ref = torch.zeros(11, 32, dtype=torch.float64)
+    for e in range(4):
+        ref += p[:, e:e + 1] * ref_swiglu(inp["x"].double(), inp["W_g"][e].double(), inp["W_u"][e].double(),
+                                          inp["W_d"][e].double())
+    assert torch.allclose(r["y"], ref, rtol=1e-12, atol=1e-14)
+
+
+def test_per_token_loop_equals_dense_masked_brute_force(oracle):
+    wl = small(T=30, H=64, E=6, k=2, F=96)
+    inp = make_inputs(wl, seed=6)
+    r = oracle.layer_fwd(wl, inp)
+    gd = torch.zeros(wl.T, wl.E, dtype=torch.float64)
+    gd.scatter_(1, r["idx"].long(), r["gates"])
+    yd = oracle.moe_fwd_dense(inp["x"], inp["W_g"], inp["W_u"], inp["W_d"], gd)
+    assert torch.allclose(r["y"], yd, rtol=1e-12, atol=1e-13)
+
+
+def test_fold_before_down_projection_equals_after(oracle):
+    wl = small(T=20, H=64, E=5, k=3, F=96)
+    inp = make_inputs(wl, seed=7)
+    r = oracle.layer_fwd(wl, inp)
+    y_fold = oracle.moe_fwd_tokens(inp["x"], inp["W_g"], inp["W_u"], inp["W_d"], r["idx"], r["gates"], fold=True)
+    y_post = oracle.moe_fwd_tokens(inp["x"], inp["W_g"], inp["W_u"], inp["W_d"], r["idx"], r["gates"], fold=False)
+    assert torch.allclose(y_fold, y_post, rtol=1e-12, atol=1e-13)
+    # ...and the fold really changes the intermediate (g applied): ap = g * a
+    assert not torch.equal(y_fold, torch.zeros_like(y_fold))
+
+
+def test_row_stage_composes_to_per_token_loop(oracle):
+    """permute (gather by src_of) -> per-row expert stage -> unpermute-sum equals the per-token loop."""
+    wl = small(T=25, H=64, E=5, k=2, F=64)
+    inp = make_inputs(wl, seed=8)
+    r = oracle.layer_fwd(wl, inp)
+    off = r["offsets"].long()
+    e_of = torch.bucketize(torch.arange(wl.T * wl.k), off[1:], right=True).to(torch.int32)
+    g_of = torch.empty(wl.T * wl.k, dtype=torch.float64)
+    g_of[r["row_of"].flatten().long()] = r["gates"].flatten()
+    xp = inp["x"][r["src_of"].long()].contiguous()
+    st = oracle.expert_rows(xp, e_of, g_of, inp["W_g"], inp["W_u"], inp["W_d"])
+    y = oracle.unpermute(st["o"], r["row_of"])
+    assert torch.allclose(y, r["y"], rtol=1e-13, atol=1e-14)
+
+
+def test_shared_expert_adds_plain_mlp(oracle):
+    wl = small(T=10, H=64, E=4, k=2, F=64, S=1, score="sigmoid", route_scale=2.5, aux=False)
+    inp = make_inputs(wl, seed=9)
+    r = oracle.layer_fwd(wl, inp)
+    y0 = oracle.moe_fwd_tokens(inp["x"], inp["W_g"], inp["W_u"], inp["W_d"], r["idx"], r["gates"])
+    sh = ref_swiglu(inp["x"].double(), inp["W_gs"].double(), inp["W_us"].double(), inp["W_ds"].double())
+    assert torch.allclose(r["y"], y0 + sh, rtol=1e-12, atol=1e-13)
+
+
+# --------------------------------------------------------------- MXFP8
+
+
+def _golden():
+    elems, scales, blocks = [], [], []
+    for line in open(GOLDEN):
+        line = line.strip()
+        if not line or line.startswith("#"):
+            continue
+        tag, rest = line.split(" ", 1)
+        if tag == "elem":
+            v, c = rest.split()
+            elems.append((float(v), int(c, 16)))
+        elif tag == "scale":
+            a, b = rest.split()
+            scales.append((float(a), int(b)))
+        elif tag == "block":
+            head, tail = rest.split(" : ")
+            name, byte = head.split()
+            vals, codes = tail.split(" => ")
+            blocks.append((name, int(byte), [float(v) for v in vals.split()], [int(c, 16) for c in codes.split()]))
+    return elems, scales, blocks
+
+
+def test_mxfp8_golden_elements_and_scales(oracle):
+    elems, scales, _ = _golden()
+    assert len(elems) > 20 and len(scales) > 5
+    for v, c in elems:
+        assert oracle.e4m3_encode(v) == c, (v, hex(oracle.e4m3_encode(v)), hex(c))
+    for a, b in scales:
+        assert oracle.mx_scale_byte(a) == b, (a, oracle.mx_scale_byte(a), b)
+
+
+def test_mxfp8_golden_blocks(oracle):
+    _, _, blocks = _golden()
+    for name, byte, vals, codes in blocks:
+        v = torch.zeros(1, 32, dtype=torch.float32)
+        v[0, :len(vals)] = torch.tensor(vals, dtype=torch.float32)
+        q, s = oracle.mxfp8_quantize(v)
+        assert int(s[0, 0]) == byte, name
+        exp = codes + [0] * (32 - len(codes))
+        assert q[0].tolist() == exp, (name, [hex(c) for c in q[0].tolist()])
+
+
+def test_e4m3_decode_matches_torch_float8(oracle):
+    codes = torch.arange(256, dtype=torch.int32).to(torch.uint8)
+    ref = codes.view(torch.float8_e4m3fn).to(torch.float64)
+    mine = torch.tensor([oracle.e4m3_decode(c) for c in range(256)], dtype=torch.float64)
+    nan = torch.isnan(ref)
+    assert torch.equal(torch.isnan(mine), nan)
+    assert torch.equal(mine[~nan], ref[~nan])
+
+
+def test_e4m3_encode_matches_torch_cast_in_range(oracle):
+    g = torch.Generator().manual_seed(0)
+    v = (torch.rand(4000, generator=g, dtype=torch.float64) * 2 - 1) * 448.0
+    v = torch.cat([v, v * 1e-3, torch.tensor([0.0009765625, 0.0029296875, 1.0625, 1.1875, 15.5, -0.3])])
+    v32 = v.float()
+    ref = v32.to(torch.float8_e4m3fn).view(torch.uint8)
+    mine = torch.tensor([oracle.e4m3_encode(float(x)) for x in v32], dtype=torch.uint8)
+    assert torch.equal(mine, ref)
+
+
+def test_mxfp8_roundtrip_error_bound(oracle):
+    g = torch.Generator().manual_seed(1)
+    v = torch.randn(64, 256, generator=g) * torch.logspace(-6, 6, 64).unsqueeze(1)
+    q, s = oracle.mxfp8_quantize(v)
+    dq = oracle.mxfp8_decode(q, s)
+    X = torch.pow(2.0, s.double() - 127.0).repeat_interleave(32, 1)
+    a = (v.double() / X).abs()
+    assert (a < 512).all()                                   # scale puts amax in [256, 512)
+    blk_amax = a.view(64, 8, 32).amax(-1)
+    assert ((blk_amax >= 256) & (blk_amax < 512)).all()
+    e = torch.floor(torch.log2(a.clamp_min(2.0 ** -9))).clamp_min(-6)
+    half_ulp = torch.pow(2.0, e - 4) * X
+    err = (dq - v.double()).abs()
+    inrange = a <= 448
+    assert (err[inrange] <= half_ulp[inrange] * (1 + 1e-12)).all()
+    assert torch.equal(dq[~inrange].abs(), 448.0 * X[~inrange])
+
+
+def test_mxfp8_bf16_and_fp32_entry_points_agree(oracle):
+    g = torch.Generator().manual_seed(2)
+    v = (torch.randn(16, 128, generator=g) * 0.02).bfloat16()
+    a = oracle.mxfp8_quantize(v)
+    b = oracle.mxfp8_quantize(v.float())
+    assert torch.equal(a[0], b[0]) and torch.equal(a[1], b[1])
+
+
+# --------------------------------------------------------------- backward
+
+
+def _fd_setup(score, norm, scale, aux_on, seed=0, T=8, H=16, E=4, k=2, F=32):
+    g = torch.Generator().manual_seed(seed)
+    t = dict(
+        x=torch.randn(T, H, generator=g, dtype=torch.float64),
+        W_r=torch.randn(E, H, generator=g, dtype=torch.float64) * 0.4,
+        W_g=torch.randn(E, F, H, generator=g, dtype=torch.float64) * 0.3,
+        W_u=torch.randn(E, F, H, generator=g, dtype=torch.float64) * 0.3,
+        W_d=torch.randn(E, H, F, generator=g, dtype=torch.float64) * 0.3,
+        dY=torch.randn(T, H, generator=g, dtype=torch.float64),
+    )
+    cfg = dict(k=k, score=score, norm=norm, scale=scale, aux_on=aux_on, d_aux=0.7 if aux_on else 0.0)
+    return t, cfg
+
+
+def _loss(o, t, cfg, logits=None):
+    if logits is None:
+        logits = o.router_logits(t["x"], t["W_r"], None, round_f32=False)
+    r = o.route(logits, cfg["k"], cfg["score"], cfg["norm"], cfg["scale"], with_aux=cfg["aux_on"])
+    y = o.moe_fwd_tokens(t["x"], t["W_g"], t["W_u"], t["W_d"], r["idx"], r["gates"])
+    L = (t["dY"] * y).sum().item()
+    if cfg["aux_on"]:
+        L += cfg["d_aux"] * r["aux"]
+    return L, r
+
+
+@pytest.mark.parametrize("score,norm,scale,aux_on", [("softmax", True, 1.0, True), ("sigmoid", True, 2.5, False),
+                                                     ("softmax", False, 1.0, True)])
+def test_backward_matches_central_finite_differences(oracle, score, norm, scale, aux_on):
+    o = oracle
+    t, cfg = _fd_setup(score, norm, scale, aux_on)
+    L0, r = _loss(o, t, cfg)
+    E = t["W_r"].shape[0]
+    dx, dl, dg = o.moe_bwd_tokens(t["x"], t["W_r"], t["W_g"], t["W_u"], t["W_d"], t["dY"], r, score=score,
+                                  norm=norm, route_scale=scale, aux_on=aux_on, d_aux=cfg["d_aux"])
+    dWg, dWu, dWd = o.moe_bwd_expert_dw(t["x"], t["W_g"], t["W_u"], t["W_d"], t["dY"], r["idx"], r["gates"],
+                                        list(range(E)))
+    dWr = o.router_dwr(dl, t["x"])
+    grads = dict(x=dx, W_r=dWr, W_g=dWg, W_u=dWu, W_d=dWd)
+    h = 1e-6
+    g = torch.Generator().manual_seed(11)
+    checked = 0
+    for name, G in grads.items():
+        P = t[name]
+        flat = P.view(-1)
+        for i in torch.randperm(flat.numel(), generator=g)[:12].tolist():
+            old = flat[i].item()
+            flat[i] = old + h
+            Lp, rp = _loss(o, t, cfg)
+            flat[i] = old - h
+            Lm, rm = _loss(o, t, cfg)
+            flat[i] = old
+            if not (torch.equal(rp["idx"], r["idx"]) and torch.equal(rm["idx"], r["idx"])):
+                continue                              # selection changed: not differentiable here
+            fd = (Lp - Lm) / (2 * h)
+            an = G.reshape(-1)[i].item()
+            assert abs(fd - an) <= 1e-6 * max(1.0, abs(an)), (name, i, fd, an)
+            checked += 1
+    assert checked >= 40
+    # dlogits against finite differences in the logits themselves
+    l0 = o.router_logits(t["x"], t["W_r"], None, round_f32=False)
+    for tt in range(l0.shape[0]):
+        for e in range(E):
+            lp = l0.clone(); lp[tt, e] += h
+            lm = l0.clone(); lm[tt, e] -= h
+            Lp, rp = _loss(o, t, cfg, lp)
+            Lm, rm = _loss(o, t, cfg, lm)
+            if not (torch.equal(rp["idx"], r["idx"]) and torch.equal(rm["idx"], r["idx"])):
+                continue
+            fd = (Lp - Lm) / (2 * h)
+            assert abs(fd - dl[tt, e].item()) <= 1e-6 * max(1.0, abs(fd)), (tt, e, fd, dl[tt, e].item())
+
+
+def test_zero_token_expert_gets_exact_zero_weight_grads(oracle):
+    from mixture_experts_layer_aux_b200.synthetic import random_routing
+    wl = small(T=12, H=32, E=5, k=2, F=32)
+    inp = make_inputs(wl, seed=12, with_dy=True)
+    idx = random_routing(12, 5, 2, seed=1, zero_experts=2)
+    gts = torch.full((12, 2), 0.5, dtype=torch.float64)
+    dWg, dWu, dWd = oracle.moe_bwd_expert_dw(inp["x"], inp["W_g"], inp["W_u"], inp["W_d"], inp["dY"], idx, gts,
+                                             [3, 4, 0])
+    assert (dWg[:2] == 0).all() and (dWu[:2] == 0).all() and (dWd[:2] == 0).all()
+    assert dWd[2].abs().sum() > 0
+
+
+def test_weight_grad_of_down_is_gated_outer_product_sum(oracle):
+    """dW_d[e] = sum over e's tokens of g * dY_t (x) a_t, checked with torch fp64."""
+    wl = small(T=14, H=32, E=3, k=2, F=32)
+    inp = make_inputs(wl, seed=13, with_dy=True)
+    r = oracle.layer_fwd(wl, inp)
+    _, _, dWd = oracle.moe_bwd_expert_dw(inp["x"], inp["W_g"], inp["W_u"], inp["W_d"], inp["dY"], r["idx"],
+                                         r["gates"], [1])
+    x, dY = inp["x"].double(), inp["dY"].double()
+    ref = torch.zeros(32, 32, dtype=torch.float64)
+    for t in range(14):
+        for j in range(2):
+            if int(r["idx"][t, j]) == 1:
+                a = torch.nn.functional.silu(x[t] @ inp["W_g"][1].double().T) * (x[t] @ inp["W_u"][1].double().T)
+                ref += r["gates"][t, j] * torch.outer(dY[t], a)
+    assert torch.allclose(dWd[0], ref, rtol=1e-12, atol=1e-13)
