@@ -1,0 +1,244 @@
+/*
+ * moe.h -- C ABI of the B200 (sm_100a) single-GPU Mixture-of-Experts layer.
+ *
+ * The layer follows the per-token MoE step of the study notes
+ * "Megatron-Core MoE -- 大规模稀疏专家并行实践" (实践案例 / 案例 1): score every
+ * expert, keep the top-k, and sum gate(e) * Expert_e(x) over the kept experts.
+ * Its system design follows the technical summary
+ * "《使用 Megatron Core 大规模训练混合专家模型（MoE）》技术总结":
+ *   - 2.2 memory-efficient permutation: the routing weight is folded into the
+ *     activation before the down projection (W_d (g a) instead of g (W_d a)),
+ *     so the unpermute step is an unweighted sum and the backward needs no
+ *     saved down-projection output;
+ *   - 2.4 grouped GEMM and fused routing / permutation / aux-loss kernels, and
+ *     sync-free kernels: expert sizes stay on the device, no entry point ever
+ *     synchronises the host, so every call can be captured in a CUDA graph;
+ *   - 3 (contributions) the MXFP8 training recipe on Blackwell: E4M3 elements
+ *     with one UE8M0 scale per 1x32 block (OCP MX v1.0).
+ *
+ * Conventions for every entry point:
+ *   - All tensor pointers are DEVICE pointers to row-major, contiguous memory
+ *     that the caller owns. The library never allocates, frees or
+ *     synchronises; scratch memory is the caller's `ws` buffer, sized by the
+ *     matching *_workspace_size() query. Pointers must be 16-byte aligned.
+ *   - bf16 = IEEE bfloat16 stored as uint16; e4m3 = OCP FP8 E4M3 ("fn") byte;
+ *     ue8m0 = power-of-two scale byte 2^(b-127).
+ *   - `stream` is a cudaStream_t (NULL = legacy default stream). Work is only
+ *     enqueued; results are ready when the stream reaches them.
+ *   - Return value: MOE_OK, or an error code returned BEFORE anything is
+ *     enqueued (bad arguments, unsupported shapes, misalignment, too small a
+ *     workspace), or MOE_ERR_CUDA when a launch failed.
+ *   - Kernels that wait on the hardware (mbarriers) do so with bounded waits;
+ *     on time-out they record a code in a device status word, release their
+ *     tensor memory and return. moe_get_device_status() reads that word.
+ *
+ * Notation: T tokens, H hidden, E routed experts, k top-k, F expert FFN
+ * width, S shared experts (0 or 1). "rows" = T*k, the permuted (expert-
+ * contiguous) order; expert e owns rows [offsets[e], offsets[e+1]).
+ * Within an expert rows are in ascending token order (a stable counting sort
+ * of the flattened (t*k + j) pairs by expert).
+ */
+#ifndef MOE_B200_H
+#define MOE_B200_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    MOE_OK = 0,
+    MOE_ERR_INVALID_ARG = 1,  /* null pointer, non-positive or inconsistent size */
+    MOE_ERR_UNSUPPORTED = 2,  /* shape or dtype outside what the kernels handle */
+    MOE_ERR_ALIGNMENT = 3,    /* a pointer is not 16-byte aligned */
+    MOE_ERR_WORKSPACE = 4,    /* ws is NULL or smaller than the size query */
+    MOE_ERR_CUDA = 5,         /* a CUDA call or launch failed */
+    MOE_ERR_DEVICE = 6        /* a kernel recorded a device-side failure */
+} moe_status;
+
+typedef enum { MOE_SCORE_SOFTMAX = 0, MOE_SCORE_SIGMOID = 1 } moe_score_fn;
+typedef enum { MOE_DT_BF16 = 0, MOE_DT_MXFP8 = 1 } moe_dtype;
+typedef enum { MOE_GEMM_GATEUP_SWIGLU = 0, MOE_GEMM_DOWN = 1 } moe_gemm_kind;
+
+/* Layer shape and routing recipe. Limits: 1 <= k <= min(E, 16); E <= 512;
+ * H % 128 == 0; F % 128 == 0 (MXFP8: H, F % 128 too); T >= 1. */
+typedef struct moe_config {
+    int32_t T, H, E, k, F;
+    int32_t n_shared;     /* 0, or 1 always-on shared expert of width F */
+    int32_t score;        /* moe_score_fn: softmax over E, or per-expert sigmoid */
+    int32_t norm_topk;    /* 1: gates renormalised to sum 1 over the selected */
+    float route_scale;    /* multiplies every gate (1.0; 2.5 in the DeepSeek-V3 recipe) */
+    int32_t expert_dtype; /* moe_dtype of the expert GEMM operands */
+    int32_t compute_aux;  /* 1: load-balancing aux statistic (softmax scores only) */
+    int32_t save_for_bwd; /* 1: moe_layer_fwd fills `saved` for moe_layer_bwd */
+} moe_config;
+
+/* Human-readable name of a status code (static string). */
+const char* moe_status_string(int status);
+
+/* Device status word written by bounded waits that timed out (0 = none).
+ * Synchronises the current device; do not call during stream capture.
+ * `clear` != 0 resets the word to 0 afterwards. */
+int moe_get_device_status(int32_t* word_out, int clear);
+
+/* ------------------------------------------------------------------------
+ * Router: logits, scores, top-k, gates, counts, aux.
+ *   logits[t,e] = sum_h x[t,h] W_r[e,h] (+ logit_bias[e]), fp32 accumulate
+ *     (router precision stays high: the study notes' 踩过的坑 section warns
+ *     that low-precision logits collapse routing onto a few experts);
+ *   scores: softmax over the E logits, or sigmoid per logit (fp32);
+ *   idx[t,0..k-1]: the k largest logits, descending; equal logits go to the
+ *     lower expert index first (selection on logits = selection on scores);
+ *   gates[t,j] = score / (sum of the selected scores if norm_topk) * route_scale;
+ *   counts[e] = number of (t,j) with idx[t,j] == e;
+ *   aux = E * sum_e (counts[e] / (T k)) * mean_t probs[t,e]  (softmax only;
+ *     the load-balancing loss named in 2.4 of the summary and 案例 3 of the
+ *     study notes; unscaled -- the caller applies its coefficient).
+ * Arguments:
+ *   x [T,H] bf16, W_r [E,H] bf16, logit_bias [E] fp32 or NULL.
+ *   If x == NULL and W_r == NULL, `logits` is an INPUT [T,E] fp32 and only the
+ *   routing steps run (logit_bias is then ignored).
+ *   logits [T,E] fp32 out (required), probs [T,E] fp32 out or NULL,
+ *   idx [T,k] int32 out, gates [T,k] fp32 out, counts [E] int32 out or NULL,
+ *   aux [1] fp32 out or NULL (must be NULL unless compute_aux and softmax).
+ * ------------------------------------------------------------------------ */
+size_t moe_router_workspace_size(const moe_config* cfg);
+int moe_router_topk(const moe_config* cfg, const void* x, const void* W_r, const float* logit_bias,
+                    float* logits, float* probs, int32_t* idx, float* gates, int32_t* counts, float* aux,
+                    void* ws, size_t ws_bytes, void* stream);
+
+/* ------------------------------------------------------------------------
+ * Permutation into expert-contiguous order (memory-efficient permutation,
+ * 2.2 of the summary; sync-free, 2.4): per-expert counts, exclusive-scan
+ * offsets, the stable row maps, the per-row gate, and the gathered rows --
+ * all on the device.
+ *   counts[e], offsets[0..E] (offsets[E] = T*k),
+ *   row_of[t,j] = offsets[e] + #{t' < t : e in idx[t',:]} for e = idx[t,j],
+ *   src_of[row_of[t,j]] = t, row_gate[row_of[t,j]] = gates[t,j],
+ *   xp[row_of[t,j], :] = x[t, :].
+ * For expert_dtype == MXFP8 each row is quantised on the way (1x32 blocks
+ * along H; block-local, so it commutes with the permutation): xp is e4m3
+ * [T*k, H] and xp_sf ue8m0 [T*k, H/32].
+ * Arguments: x [T,H] bf16; idx [T,k] int32 (k distinct experts per token,
+ * each in [0,E) -- checked on the device, violations set the status word);
+ * gates [T,k] fp32 or NULL (then row_gate must be NULL); outputs as above,
+ * counts/row_gate/xp may be NULL to skip them.
+ * ------------------------------------------------------------------------ */
+size_t moe_permute_workspace_size(const moe_config* cfg);
+int moe_permute(const moe_config* cfg, const void* x, const int32_t* idx, const float* gates, int32_t* counts,
+                int32_t* offsets, int32_t* row_of, int32_t* src_of, float* row_gate, void* xp, uint8_t* xp_sf,
+                void* ws, size_t ws_bytes, void* stream);
+
+/* ------------------------------------------------------------------------
+ * Grouped expert GEMMs, forward (tcgen05 tensor cores, TMEM accumulators,
+ * TMA operand staging; expert row ranges read from device `offsets`).
+ * which == MOE_GEMM_GATEUP_SWIGLU:
+ *   for each expert e and row r in e:
+ *     gate = W_g[e] A[r], up = W_u[e] A[r]   (fp32 accumulate)
+ *     C[r] = row_gate[r] * silu(gate) * up   (the gate folded in before the
+ *            down projection: memory-efficient permutation)
+ *   A = xp [rows,H]; B0 = W_g [E,F,H]; B1 = W_u [E,F,H]; C = ap [rows,F].
+ *   save_gateup [rows, 2F] bf16 (optional): gate in columns [0,F), up in [F,2F),
+ *   the pre-activations the backward recomputes the SwiGLU from.
+ * which == MOE_GEMM_DOWN:
+ *   C[r] = W_d[e] A[r];  A = ap [rows,F]; B0 = W_d [E,H,F]; B1 unused; C = o [rows,H].
+ * dtype BF16: A, B bf16, *_sf NULL, C bf16.
+ * dtype MXFP8: A, B e4m3 with ue8m0 scales per 1x32 block along K (A_sf
+ *   [rows, K/32], B_sf [E, N, K/32]); GATEUP writes C as e4m3 + C_sf
+ *   [rows, F/32] (quantised from the fp32 epilogue values); DOWN writes bf16.
+ * rows = T*k (the routed rows). offsets [E+1] device int32.
+ * ------------------------------------------------------------------------ */
+size_t moe_grouped_gemm_workspace_size(const moe_config* cfg, int which);
+int moe_grouped_gemm_fwd(const moe_config* cfg, int which, const void* A, const uint8_t* A_sf, const void* B0,
+                         const uint8_t* B0_sf, const void* B1, const uint8_t* B1_sf, const int32_t* offsets,
+                         const float* row_gate, void* C, uint8_t* C_sf, void* save_gateup, void* ws,
+                         size_t ws_bytes, void* stream);
+
+/* ------------------------------------------------------------------------
+ * Grouped expert GEMMs, backward (bf16 operands, fp32 accumulate). The data
+ * gradient (dgrad) and weight gradient (wgrad) outputs may each be NULL, so
+ * the two can be run apart (the W/D split of 2.3 of the summary).
+ * which == MOE_GEMM_DOWN:
+ *   dgrad: v = W_d[e]^T dO[r]  (fp32), a = silu(gate) * up from save_gateup,
+ *          dg[r] = <v, a>,  d_in[r] = [ g_r v silu'(gate) up | g_r v silu(gate) ]
+ *          (dgate in columns [0,F), dup in [F,2F)), bf16 [rows, 2F];
+ *          dg fp32 [rows].
+ *   wgrad: dW0[e] = sum_{r in e} dO[r]^T (x) act[r]  -> dW_d [E,H,F] bf16
+ *          (act = ap, the gate-folded activation).
+ *   dO = dYp [rows,H] (dY gathered by src_of), act = ap [rows,F],
+ *   saved_gateup [rows,2F], row_gate [rows], W0 = W_d.
+ * which == MOE_GEMM_GATEUP_SWIGLU:
+ *   dgrad: d_in[r] = dO[r,:F] W_g[e] + dO[r,F:] W_u[e]  -> dXp [rows,H] bf16
+ *   wgrad: dW0[e] = sum dO[r,:F]^T (x) act[r], dW1[e] = sum dO[r,F:]^T (x) act[r]
+ *          -> dW_g, dW_u [E,F,H] bf16;  dO = dgu [rows,2F], act = xp [rows,H],
+ *          W0 = W_g, W1 = W_u; saved_gateup, row_gate, dg unused (NULL).
+ * Experts that own no rows get exact-zero weight gradients.
+ * ------------------------------------------------------------------------ */
+size_t moe_grouped_gemm_bwd_workspace_size(const moe_config* cfg, int which);
+int moe_grouped_gemm_bwd(const moe_config* cfg, int which, const void* dO, const void* act,
+                         const void* saved_gateup, const float* row_gate, const void* W0, const void* W1,
+                         const int32_t* offsets, void* d_in, float* dg, void* dW0, void* dW1, void* ws,
+                         size_t ws_bytes, void* stream);
+
+/* ------------------------------------------------------------------------
+ * Unpermute-sum: y[t] = sum_{j=0..k-1} o[row_of[t,j]] (+ extra[t]), summed in
+ * fp32 in the fixed order j = 0..k-1 and rounded once to bf16. No weights:
+ * they were folded in before the down projection (2.2 of the summary).
+ * o [rows,H] bf16, row_of [T,k] int32, extra [T,H] bf16 or NULL (the shared
+ * expert's output, or the router path of dX), y [T,H] bf16.
+ * ------------------------------------------------------------------------ */
+int moe_unpermute(const moe_config* cfg, const void* o, const int32_t* row_of, const void* extra, void* y,
+                  void* stream);
+
+/* ------------------------------------------------------------------------
+ * MXFP8 quantisation (OCP MX v1.0, 6.3): src [rows,K] bf16 -> dst e4m3
+ * [rows,K], sf ue8m0 [rows,K/32]; per 1x32 block along K the scale byte is
+ * clamp(floor(log2 amax) - 8 + 127, 0, 254) (0 for an all-zero block) and each
+ * element is src / 2^(b-127) rounded to nearest-even, saturated to +-448.
+ * K % 32 == 0. Used once per weight tensor (W_g, W_u: K = H; W_d: K = F).
+ * ------------------------------------------------------------------------ */
+int moe_quantize_mxfp8(const void* src, int64_t rows, int32_t K, uint8_t* dst, uint8_t* sf, void* stream);
+
+/* ------------------------------------------------------------------------
+ * Whole layer, forward: router -> permute -> GEMM gate/up (SwiGLU, gate
+ * folded) -> GEMM down -> [shared expert] -> unpermute-sum.
+ *   x [T,H] bf16; W_r [E,H] bf16; logit_bias [E] fp32 or NULL;
+ *   BF16: W_g, W_u [E,F,H], W_d [E,H,F] bf16, *_sf NULL;
+ *   MXFP8: the same tensors as e4m3 with ue8m0 scales (W_g_sf, W_u_sf
+ *     [E,F,H/32], W_d_sf [E,H,F/32]), as moe_quantize_mxfp8 produces them;
+ *   shared expert (n_shared = 1): Ws_g, Ws_u [F,H], Ws_d [H,F] (+ scales);
+ *   y [T,H] bf16 out; aux [1] fp32 out or NULL; idx [T,k], gates [T,k],
+ *   counts [E], offsets [E+1] optional outputs (NULL to skip);
+ *   saved: moe_layer_saved_size() bytes, filled when save_for_bwd (else NULL).
+ * ------------------------------------------------------------------------ */
+size_t moe_layer_workspace_size(const moe_config* cfg);
+size_t moe_layer_saved_size(const moe_config* cfg);
+int moe_layer_fwd(const moe_config* cfg, const void* x, const void* W_r, const float* logit_bias, const void* W_g,
+                  const void* W_u, const void* W_d, const uint8_t* W_g_sf, const uint8_t* W_u_sf,
+                  const uint8_t* W_d_sf, const void* Ws_g, const void* Ws_u, const void* Ws_d,
+                  const uint8_t* Ws_g_sf, const uint8_t* Ws_u_sf, const uint8_t* Ws_d_sf, void* y, float* aux,
+                  int32_t* idx, float* gates, int32_t* counts, int32_t* offsets, void* saved, void* ws,
+                  size_t ws_bytes, void* stream);
+
+/* ------------------------------------------------------------------------
+ * Whole layer, backward (BF16 experts, no shared expert), the exact
+ * derivative of moe_layer_fwd for upstream dY [T,H] bf16 and d_aux (the
+ * coefficient of the aux statistic in the loss):
+ *   dX [T,H] bf16 (expert path + router path), dW_r [E,H] bf16,
+ *   dW_g, dW_u [E,F,H] bf16, dW_d [E,H,F] bf16 (fp32 accumulate; experts with
+ *   no token get zeros), dlogits [T,E] fp32 (or NULL).
+ * Gate path (norm_topk, softmax): dl[sel_j] = g_j dg_j - g_j sum_i g_i dg_i / c;
+ * aux path: dl[t,e] += d_aux s_e (c_e - sum_i s_i c_i), c_e = E counts_e/(T k)/T
+ * (counts are constants). `saved` is what moe_layer_fwd(save_for_bwd=1) wrote.
+ * ------------------------------------------------------------------------ */
+size_t moe_layer_bwd_workspace_size(const moe_config* cfg);
+int moe_layer_bwd(const moe_config* cfg, const void* dY, float d_aux, const void* x, const void* W_r,
+                  const void* W_g, const void* W_u, const void* W_d, const void* saved, void* dX, void* dW_r,
+                  void* dW_g, void* dW_u, void* dW_d, float* dlogits, void* ws, size_t ws_bytes, void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* MOE_B200_H */

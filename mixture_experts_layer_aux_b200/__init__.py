@@ -7,18 +7,21 @@ include/moe.h. This package is a thin ctypes binding with the same names
 (argument marshalling only). Attributes are resolved lazily so that the
 seeded-input module `synthetic` can be imported without loading the library.
 """
+import importlib
 
 __all__ = ["load"]
 
+_SUBMODULES = ("binding", "build", "synthetic")
+
 
 def __getattr__(name):
-    if name.startswith("__"):
+    if name.startswith("__") or name in _SUBMODULES:
+        if name in _SUBMODULES:
+            return importlib.import_module(f"{__name__}.{name}")
         raise AttributeError(name)
-    from . import binding
-    return getattr(binding, name)
+    return getattr(importlib.import_module(f"{__name__}.binding"), name)
 
 
 def load():
     """Load the CUDA library (raises if it is missing or fails to load)."""
-    from . import binding
-    return binding.load()
+    return importlib.import_module(f"{__name__}.binding").load()

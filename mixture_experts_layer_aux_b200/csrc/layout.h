@@ -1,0 +1,38 @@
+// layout.h -- carving caller-provided workspace / saved buffers into tensors.
+#pragma once
+
+#include <stddef.h>
+#include <stdint.h>
+#include <cuda_runtime.h>
+
+#include "../../include/moe.h"
+
+static inline size_t ws_round(size_t b) { return (b + 255) & ~size_t(255); }
+
+// Sequential bump allocator over a caller buffer (base may be NULL to size).
+struct Carve {
+  uint8_t* base;
+  size_t used = 0;
+  explicit Carve(void* b) : base(static_cast<uint8_t*>(b)) {}
+  template <class T>
+  T* take(size_t count) {
+    T* p = base ? reinterpret_cast<T*>(base + used) : nullptr;
+    used += ws_round(count * sizeof(T));
+    return p;
+  }
+};
+
+namespace moe_impl {
+int check_cfg(const moe_config* c);
+size_t router_ws(const moe_config* c);
+size_t permute_ws(const moe_config* c);
+int router_topk(const moe_config* c, const void* x, const void* W_r, const float* bias, float* logits, float* probs,
+                int32_t* idx, float* gates, int32_t* counts, float* aux, void* ws, size_t ws_bytes, cudaStream_t st);
+int permute(const moe_config* c, const void* x, const int32_t* idx, const float* gates, int32_t* counts,
+            int32_t* offsets, int32_t* row_of, int32_t* src_of, float* row_gate, void* xp, uint8_t* xp_sf, void* ws,
+            size_t ws_bytes, cudaStream_t st);
+int scatter_rows(const moe_config* c, const void* x, const int32_t* row_of, void* xp, cudaStream_t st);
+int unpermute(const moe_config* c, const void* o, const int32_t* row_of, const void* extra, void* y, cudaStream_t st);
+int quantize_mxfp8(const void* src, int64_t rows, int32_t K, uint8_t* dst, uint8_t* sf, cudaStream_t st);
+int fill_offsets2(int32_t* off, int n, cudaStream_t st);
+}  // namespace moe_impl

@@ -1,0 +1,403 @@
+// permute.cu -- sync-free token permutation into expert-contiguous order,
+// unpermute-sum, and MXFP8 quantisation.
+//
+// Memory-efficient permutation (section 2.2 of the Megatron Core MoE technical
+// summary): the routing weight is not applied to the gathered rows; it travels
+// as row_gate[r] and is folded into the activation in the gate/up GEMM
+// epilogue, so unpermute is a plain sum. The maps are built on the device
+// (sync-free kernels, section 2.4): no count ever reaches the host.
+//
+// Kernels:
+//   rank     one warp per 128 tokens: stable in-block rank of every (t, j)
+//            among the block's earlier tokens with the same expert (bitmask
+//            per expert in shared memory, popc of the lanes below), and the
+//            block's expert histogram.
+//   scan     one block: counts, exclusive-scan offsets, per-block bases.
+//   scatter  one warp per token: row = base[block, e] + rank; writes row_of,
+//            src_of, row_gate; copies the token's row once from HBM and writes
+//            it to its k destination rows with 16-byte vector stores
+//            (quantising each 1x32 block to MXFP8 on the way when asked).
+//   unpermute one warp per token: fp32 sum of its k rows in slot order, 16-byte
+//            loads, one bf16 rounding.
+#include <cuda_fp8.h>
+
+#include "common.cuh"
+#include "layout.h"
+
+namespace perm {
+
+constexpr int RANK_TOK = 128;  // tokens per rank block (one warp)
+constexpr int SC_WARPS = 8;    // warps per scatter / unpermute block
+
+__global__ void __launch_bounds__(32) rank_kernel(const int32_t* __restrict__ idx, int T, int E, int k,
+                                                  int32_t* __restrict__ lrank, int* __restrict__ hist, int* status) {
+  extern __shared__ uint32_t s_rank[];
+  uint32_t* mask = s_rank;                                // [E]
+  int* cnt = reinterpret_cast<int*>(s_rank + E);          // [E]
+  const int lane = threadIdx.x;
+  for (int e = lane; e < E; e += 32) {
+    mask[e] = 0;
+    cnt[e] = 0;
+  }
+  __syncwarp();
+  for (int c = 0; c < RANK_TOK / 32; ++c) {
+    const int t = blockIdx.x * RANK_TOK + c * 32 + lane;
+    const bool tv = t < T;
+    int es[16];
+    int bad = 0;
+#pragma unroll
+    for (int j = 0; j < 16; ++j) {
+      es[j] = -1;
+      if (j < k && tv) {
+        int e = idx[(long long)t * k + j];
+        if (e < 0 || e >= E) {
+          bad = 1;
+          e = -1;
+        }
+        for (int i = 0; i < j; ++i)
+          if (es[i] == e && e >= 0) {
+            bad = 1;
+            e = -1;
+          }
+        es[j] = e;
+      }
+    }
+    if (bad) record_status(status, DEV_BAD_INDEX);
+#pragma unroll
+    for (int j = 0; j < 16; ++j)
+      if (j < k && es[j] >= 0) atomicOr(&mask[es[j]], 1u << lane);
+    __syncwarp();
+#pragma unroll
+    for (int j = 0; j < 16; ++j)
+      if (j < k && tv) {
+        const int e = es[j];
+        lrank[(long long)t * k + j] = e >= 0 ? cnt[e] + __popc(mask[e] & ((1u << lane) - 1u)) : -1;
+      }
+    __syncwarp();
+#pragma unroll
+    for (int j = 0; j < 16; ++j)
+      if (j < k && es[j] >= 0) {
+        const int e = es[j];
+        const uint32_t m = mask[e];
+        if (m != 0 && (__ffs(m) - 1) == lane) cnt[e] += __popc(m);
+      }
+    __syncwarp();
+#pragma unroll
+    for (int j = 0; j < 16; ++j)
+      if (j < k && es[j] >= 0) mask[es[j]] = 0;
+    __syncwarp();
+  }
+  for (int e = lane; e < E; e += 32) hist[(long long)blockIdx.x * E + e] = cnt[e];
+}
+
+// counts, offsets [E+1], base[b,e] = offsets[e] + sum_{b'<b} hist[b',e].
+__global__ void __launch_bounds__(512) scan_kernel(const int* __restrict__ hist, int nblk, int E,
+                                                   int* __restrict__ base, int32_t* __restrict__ counts,
+                                                   int32_t* __restrict__ offsets) {
+  __shared__ int s[512];
+  const int e = threadIdx.x;
+  int run = 0;
+  if (e < E) {
+    for (int b = 0; b < nblk; ++b) {
+      base[(long long)b * E + e] = run;
+      run += hist[(long long)b * E + e];
+    }
+    if (counts) counts[e] = run;
+  }
+  s[e] = (e < E) ? run : 0;
+  __syncthreads();
+  for (int o = 1; o < 512; o <<= 1) {  // inclusive Hillis-Steele scan
+    const int v = (e >= o) ? s[e - o] : 0;
+    __syncthreads();
+    s[e] += v;
+    __syncthreads();
+  }
+  const int excl = s[e] - ((e < E) ? run : 0);
+  if (e < E) {
+    offsets[e] = excl;
+    for (int b = 0; b < nblk; ++b) base[(long long)b * E + e] += excl;
+  }
+  if (e == E - 1) offsets[E] = s[e];
+}
+
+__device__ __forceinline__ uint8_t mx_scale_byte(float amax) {
+  const uint32_t b = __float_as_uint(amax);
+  const int eb = (int)((b >> 23) & 0xFFu);
+  if (!(amax > 0.f) || eb == 0) return 0;
+  int s = eb - 8;  // floor(log2 amax) - 8 + 127
+  s = s < 0 ? 0 : (s > 254 ? 254 : s);
+  return (uint8_t)s;
+}
+// 2^(127 - byte): exact power of two (byte <= 246 for finite fp32 input)
+__device__ __forceinline__ float mx_inv_scale(uint8_t byte) { return __uint_as_float((uint32_t)(254 - byte) << 23); }
+
+__device__ __forceinline__ uint2 quant8(const float (&f)[8], float inv) {
+  uint32_t w[2];
+#pragma unroll
+  for (int h = 0; h < 2; ++h) {
+    uint32_t acc = 0;
+#pragma unroll
+    for (int i = 0; i < 4; i += 2) {
+      const __nv_fp8x2_storage_t pr =
+          __nv_cvt_float2_to_fp8x2(make_float2(f[4 * h + i] * inv, f[4 * h + i + 1] * inv), __NV_SATFINITE, __NV_E4M3);
+      acc |= (uint32_t)pr << (8 * i);
+    }
+    w[h] = acc;
+  }
+  return make_uint2(w[0], w[1]);
+}
+
+// MODE 0: rows computed here from (idx, lrank, base) -- the permute itself.
+// MODE 1: rows read from row_of -- a plain scatter of another [T,H] tensor.
+template <int MODE, bool MX>
+__global__ void __launch_bounds__(SC_WARPS * 32) scatter_kernel(
+    const __nv_bfloat16* __restrict__ x, int T, int H, int E, int k, const int32_t* __restrict__ idx,
+    const int32_t* __restrict__ lrank, const int* __restrict__ base, const float* __restrict__ gates,
+    int32_t* __restrict__ row_of, int32_t* __restrict__ src_of, float* __restrict__ row_gate, void* __restrict__ xp,
+    uint8_t* __restrict__ xp_sf) {
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int t = blockIdx.x * SC_WARPS + warp;
+  if (t >= T) return;
+  const int rows_total = T * k;
+  int r = -1;
+  if (lane < k) {
+    if (MODE == 0) {
+      const int e = idx[(long long)t * k + lane];
+      const int lr = lrank[(long long)t * k + lane];
+      if (e >= 0 && e < E && lr >= 0) {
+        r = base[(long long)(t / RANK_TOK) * E + e] + lr;
+        if (r >= rows_total) r = -1;
+      }
+      row_of[(long long)t * k + lane] = r;
+      if (r >= 0) {
+        src_of[r] = t;
+        if (row_gate) row_gate[r] = gates[(long long)t * k + lane];
+      }
+    } else {
+      r = row_of[(long long)t * k + lane];
+      if (r < 0 || r >= rows_total) r = -1;
+    }
+  }
+  if (xp == nullptr) return;
+  int rows[16];
+#pragma unroll
+  for (int j = 0; j < 16; ++j) rows[j] = __shfl_sync(0xffffffffu, r, j < k ? j : 0);
+  const uint4* src = reinterpret_cast<const uint4*>(x + (long long)t * H);
+  const int nchunk = H / 8;
+  for (int i0 = 0; i0 < nchunk; i0 += 32) {
+    const int i = i0 + lane;
+    const bool v = i < nchunk;
+    const uint4 d = v ? src[i] : make_uint4(0, 0, 0, 0);
+    if constexpr (!MX) {
+      if (v) {
+#pragma unroll
+        for (int j = 0; j < 16; ++j)
+          if (j < k && rows[j] >= 0)
+            reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(xp) + (long long)rows[j] * H)[i] = d;
+      }
+    } else {
+      float f[8];
+      unpack_bf16x8(d, f);
+      float am = 0.f;
+#pragma unroll
+      for (int q = 0; q < 8; ++q) am = fmaxf(am, fabsf(f[q]));
+      am = fmaxf(am, __shfl_xor_sync(0xffffffffu, am, 1));
+      am = fmaxf(am, __shfl_xor_sync(0xffffffffu, am, 2));
+      const uint8_t sb = mx_scale_byte(am);
+      const uint2 codes = quant8(f, mx_inv_scale(sb));
+      if (v) {
+#pragma unroll
+        for (int j = 0; j < 16; ++j)
+          if (j < k && rows[j] >= 0) {
+            reinterpret_cast<uint2*>(static_cast<uint8_t*>(xp) + (long long)rows[j] * H)[i] = codes;
+            if ((i & 3) == 0) xp_sf[(long long)rows[j] * (H / 32) + (i >> 2)] = sb;
+          }
+      }
+    }
+  }
+}
+
+__global__ void __launch_bounds__(SC_WARPS * 32) unpermute_kernel(const __nv_bfloat16* __restrict__ o,
+                                                                  const int32_t* __restrict__ row_of,
+                                                                  const __nv_bfloat16* __restrict__ extra, int T,
+                                                                  int H, int k, __nv_bfloat16* __restrict__ y) {
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int t = blockIdx.x * SC_WARPS + warp;
+  if (t >= T) return;
+  const int rows_total = T * k;
+  int r = -1;
+  if (lane < k) {
+    r = row_of[(long long)t * k + lane];
+    if (r < 0 || r >= rows_total) r = -1;
+  }
+  int rows[16];
+#pragma unroll
+  for (int j = 0; j < 16; ++j) rows[j] = __shfl_sync(0xffffffffu, r, j < k ? j : 0);
+  const int nchunk = H / 8;
+  for (int i = lane; i < nchunk; i += 32) {
+    uint4 d[16];
+#pragma unroll
+    for (int j = 0; j < 16; ++j)
+      if (j < k) d[j] = rows[j] >= 0 ? reinterpret_cast<const uint4*>(o + (long long)rows[j] * H)[i] : make_uint4(0, 0, 0, 0);
+    float acc[8];
+#pragma unroll
+    for (int q = 0; q < 8; ++q) acc[q] = 0.f;
+#pragma unroll
+    for (int j = 0; j < 16; ++j)
+      if (j < k) {
+        float f[8];
+        unpack_bf16x8(d[j], f);
+#pragma unroll
+        for (int q = 0; q < 8; ++q) acc[q] += f[q];
+      }
+    if (extra) {
+      float f[8];
+      unpack_bf16x8(reinterpret_cast<const uint4*>(extra + (long long)t * H)[i], f);
+#pragma unroll
+      for (int q = 0; q < 8; ++q) acc[q] += f[q];
+    }
+    uint4 out;
+    out.x = pack_bf16x2(acc[0], acc[1]);
+    out.y = pack_bf16x2(acc[2], acc[3]);
+    out.z = pack_bf16x2(acc[4], acc[5]);
+    out.w = pack_bf16x2(acc[6], acc[7]);
+    reinterpret_cast<uint4*>(y + (long long)t * H)[i] = out;
+  }
+}
+
+// One thread per 1x32 block.
+__global__ void quantize_kernel(const __nv_bfloat16* __restrict__ src, long long nblocks, uint8_t* __restrict__ dst,
+                                uint8_t* __restrict__ sf) {
+  for (long long b = blockIdx.x * (long long)blockDim.x + threadIdx.x; b < nblocks;
+       b += (long long)gridDim.x * blockDim.x) {
+    const uint4* s4 = reinterpret_cast<const uint4*>(src + b * 32);
+    float f[4][8];
+    float am = 0.f;
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      unpack_bf16x8(s4[q], f[q]);
+#pragma unroll
+      for (int i = 0; i < 8; ++i) am = fmaxf(am, fabsf(f[q][i]));
+    }
+    const uint8_t sb = mx_scale_byte(am);
+    const float inv = mx_inv_scale(sb);
+    uint2* d2 = reinterpret_cast<uint2*>(dst + b * 32);
+#pragma unroll
+    for (int q = 0; q < 4; ++q) d2[q] = quant8(f[q], inv);
+    sf[b] = sb;
+  }
+}
+
+__global__ void fill_offsets2_kernel(int32_t* off, int n) {
+  off[0] = 0;
+  off[1] = n;
+}
+
+}  // namespace perm
+
+static bool al16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+namespace moe_impl {
+
+size_t permute_ws(const moe_config* c) {
+  const size_t nblk = (c->T + perm::RANK_TOK - 1) / perm::RANK_TOK;
+  return ws_round((size_t)c->T * c->k * sizeof(int32_t)) + 2 * ws_round(nblk * c->E * sizeof(int));
+}
+
+int permute(const moe_config* c, const void* x, const int32_t* idx, const float* gates, int32_t* counts,
+            int32_t* offsets, int32_t* row_of, int32_t* src_of, float* row_gate, void* xp, uint8_t* xp_sf, void* ws,
+            size_t ws_bytes, cudaStream_t st) {
+  int rc = check_cfg(c);
+  if (rc) return rc;
+  if (!idx || !offsets || !row_of || !src_of) return MOE_ERR_INVALID_ARG;
+  if (row_gate && !gates) return MOE_ERR_INVALID_ARG;
+  if (xp && !x) return MOE_ERR_INVALID_ARG;
+  const bool mx = c->expert_dtype == MOE_DT_MXFP8;
+  if (xp && mx && !xp_sf) return MOE_ERR_INVALID_ARG;
+  if ((x && !al16(x)) || (xp && !al16(xp))) return MOE_ERR_ALIGNMENT;
+  if (!ws || ws_bytes < permute_ws(c)) return MOE_ERR_WORKSPACE;
+  const int nblk = (c->T + perm::RANK_TOK - 1) / perm::RANK_TOK;
+  Carve cv(ws);
+  int32_t* lrank = cv.take<int32_t>((size_t)c->T * c->k);
+  int* hist = cv.take<int>((size_t)nblk * c->E);
+  int* base = cv.take<int>((size_t)nblk * c->E);
+  int* status = moe_host::device_status_ptr();
+  perm::rank_kernel<<<nblk, 32, 2 * c->E * sizeof(uint32_t), st>>>(idx, c->T, c->E, c->k, lrank, hist, status);
+  MOE_CHECK_LAUNCH();
+  perm::scan_kernel<<<1, 512, 0, st>>>(hist, nblk, c->E, base, counts, offsets);
+  MOE_CHECK_LAUNCH();
+  const int sgrid = (c->T + perm::SC_WARPS - 1) / perm::SC_WARPS;
+  if (mx)
+    perm::scatter_kernel<0, true><<<sgrid, perm::SC_WARPS * 32, 0, st>>>(
+        static_cast<const __nv_bfloat16*>(x), c->T, c->H, c->E, c->k, idx, lrank, base, gates, row_of, src_of,
+        row_gate, xp, xp_sf);
+  else
+    perm::scatter_kernel<0, false><<<sgrid, perm::SC_WARPS * 32, 0, st>>>(
+        static_cast<const __nv_bfloat16*>(x), c->T, c->H, c->E, c->k, idx, lrank, base, gates, row_of, src_of,
+        row_gate, xp, nullptr);
+  MOE_CHECK_LAUNCH();
+  return MOE_OK;
+}
+
+int scatter_rows(const moe_config* c, const void* x, const int32_t* row_of, void* xp, cudaStream_t st) {
+  const int sgrid = (c->T + perm::SC_WARPS - 1) / perm::SC_WARPS;
+  perm::scatter_kernel<1, false><<<sgrid, perm::SC_WARPS * 32, 0, st>>>(
+      static_cast<const __nv_bfloat16*>(x), c->T, c->H, c->E, c->k, nullptr, nullptr, nullptr, nullptr,
+      const_cast<int32_t*>(row_of), nullptr, nullptr, xp, nullptr);
+  MOE_CHECK_LAUNCH();
+  return MOE_OK;
+}
+
+int unpermute(const moe_config* c, const void* o, const int32_t* row_of, const void* extra, void* y, cudaStream_t st) {
+  int rc = check_cfg(c);
+  if (rc) return rc;
+  if (!o || !row_of || !y) return MOE_ERR_INVALID_ARG;
+  if (!al16(o) || !al16(y) || (extra && !al16(extra))) return MOE_ERR_ALIGNMENT;
+  const int grid = (c->T + perm::SC_WARPS - 1) / perm::SC_WARPS;
+  perm::unpermute_kernel<<<grid, perm::SC_WARPS * 32, 0, st>>>(static_cast<const __nv_bfloat16*>(o), row_of,
+                                                               static_cast<const __nv_bfloat16*>(extra), c->T, c->H,
+                                                               c->k, static_cast<__nv_bfloat16*>(y));
+  MOE_CHECK_LAUNCH();
+  return MOE_OK;
+}
+
+int quantize_mxfp8(const void* src, int64_t rows, int32_t K, uint8_t* dst, uint8_t* sf, cudaStream_t st) {
+  if (!src || !dst || !sf || rows < 1 || K < 32) return MOE_ERR_INVALID_ARG;
+  if (K % 32 != 0) return MOE_ERR_UNSUPPORTED;
+  if (!al16(src) || !al16(dst)) return MOE_ERR_ALIGNMENT;
+  const long long nb = (long long)rows * (K / 32);
+  long long grid = (nb + 255) / 256;
+  if (grid > 148LL * 16) grid = 148LL * 16;
+  perm::quantize_kernel<<<(int)grid, 256, 0, st>>>(static_cast<const __nv_bfloat16*>(src), nb, dst, sf);
+  MOE_CHECK_LAUNCH();
+  return MOE_OK;
+}
+
+int fill_offsets2(int32_t* off, int n, cudaStream_t st) {
+  perm::fill_offsets2_kernel<<<1, 1, 0, st>>>(off, n);
+  MOE_CHECK_LAUNCH();
+  return MOE_OK;
+}
+
+}  // namespace moe_impl
+
+extern "C" size_t moe_permute_workspace_size(const moe_config* cfg) {
+  if (moe_impl::check_cfg(cfg)) return 0;
+  return moe_impl::permute_ws(cfg);
+}
+
+extern "C" int moe_permute(const moe_config* cfg, const void* x, const int32_t* idx, const float* gates,
+                           int32_t* counts, int32_t* offsets, int32_t* row_of, int32_t* src_of, float* row_gate,
+                           void* xp, uint8_t* xp_sf, void* ws, size_t ws_bytes, void* stream) {
+  return moe_impl::permute(cfg, x, idx, gates, counts, offsets, row_of, src_of, row_gate, xp, xp_sf, ws, ws_bytes,
+                           static_cast<cudaStream_t>(stream));
+}
+
+extern "C" int moe_unpermute(const moe_config* cfg, const void* o, const int32_t* row_of, const void* extra, void* y,
+                             void* stream) {
+  return moe_impl::unpermute(cfg, o, row_of, extra, y, static_cast<cudaStream_t>(stream));
+}
+
+extern "C" int moe_quantize_mxfp8(const void* src, int64_t rows, int32_t K, uint8_t* dst, uint8_t* sf, void* stream) {
+  return moe_impl::quantize_mxfp8(src, rows, K, dst, sf, static_cast<cudaStream_t>(stream));
+}

@@ -1,0 +1,296 @@
+// router.cu -- router logits, scores, top-k, gates, counts and the aux statistic.
+//
+// Per token (the study notes' 案例 1: score every expert, keep the top-k):
+//   logits = x W_r^T (+ bias), fp32 accumulate on the tensor cores (the router
+//   stays in high precision: 踩过的坑 in the notes);
+//   scores = softmax over E, or sigmoid per expert (fp32);
+//   top-k over the logits, descending, ties to the lower expert index, by k
+//   rounds of a warp-shuffle argmax;
+//   gates = score / sum of selected scores (norm_topk) * route_scale.
+// Fused with routing, the per-block expert histogram and the per-block sums of
+// the softmax probabilities feed the aux statistic (section 2.4 of the
+// technical summary fuses routing and aux-loss computation):
+//   aux = E * sum_e (count_e / (T k)) * mean_t p[t,e].
+// All reductions run in a fixed order, so results are bitwise reproducible.
+#include <cmath>
+
+#include "common.cuh"
+#include "gemm.cuh"
+#include "layout.h"
+
+namespace router {
+
+constexpr int TOK_PER_WARP = 8;
+constexpr int WARPS = 8;
+constexpr int TOK_PER_BLOCK = TOK_PER_WARP * WARPS;  // 64
+
+struct TopkArgs {
+  const float* logits;
+  float* probs;     // opt
+  int32_t* idx;
+  float* gates;
+  int* hist;        // [nblk, E]
+  float* pblk;      // [nblk, E] (aux only)
+  int T, E, k;
+  int score, norm;
+  float scale;
+  int want_aux;
+};
+
+__device__ __forceinline__ bool better(float v1, int i1, float v2, int i2) {
+  return (v1 > v2) || (v1 == v2 && i1 < i2);
+}
+
+template <int EPL>
+__global__ void __launch_bounds__(WARPS * 32) topk_kernel(TopkArgs a) {
+  extern __shared__ __align__(16) uint8_t sm[];
+  int* s_hist = reinterpret_cast<int*>(sm);                 // [E]
+  float* s_p = reinterpret_cast<float*>(s_hist + a.E);      // [WARPS, E]
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  for (int e = threadIdx.x; e < a.E; e += blockDim.x) s_hist[e] = 0;
+  __syncthreads();
+
+  float pacc[EPL];
+#pragma unroll
+  for (int i = 0; i < EPL; ++i) pacc[i] = 0.f;
+
+  for (int tt = 0; tt < TOK_PER_WARP; ++tt) {
+    const int t = blockIdx.x * TOK_PER_BLOCK + warp * TOK_PER_WARP + tt;
+    if (t >= a.T) break;  // warp-uniform
+    float l[EPL], s[EPL];
+    const float* lr = a.logits + (long long)t * a.E;
+#pragma unroll
+    for (int i = 0; i < EPL; ++i) {
+      const int e = lane + 32 * i;
+      l[i] = (e < a.E) ? lr[e] : -INFINITY;
+    }
+    if (a.score == MOE_SCORE_SOFTMAX) {
+      float m = -INFINITY;
+#pragma unroll
+      for (int i = 0; i < EPL; ++i) m = fmaxf(m, l[i]);
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+      float z = 0.f;
+#pragma unroll
+      for (int i = 0; i < EPL; ++i) {
+        const int e = lane + 32 * i;
+        s[i] = (e < a.E) ? expf(l[i] - m) : 0.f;
+        z += s[i];
+      }
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) z += __shfl_xor_sync(0xffffffffu, z, o);
+#pragma unroll
+      for (int i = 0; i < EPL; ++i) s[i] = s[i] / z;
+    } else {
+#pragma unroll
+      for (int i = 0; i < EPL; ++i) s[i] = 1.f / (1.f + expf(-l[i]));
+    }
+    if (a.probs) {
+#pragma unroll
+      for (int i = 0; i < EPL; ++i) {
+        const int e = lane + 32 * i;
+        if (e < a.E) a.probs[(long long)t * a.E + e] = s[i];
+      }
+    }
+    if (a.want_aux) {
+#pragma unroll
+      for (int i = 0; i < EPL; ++i) pacc[i] += s[i];
+    }
+    // top-k by k rounds of a warp argmax (value desc, index asc)
+    uint32_t taken = 0;
+    int my_e = -1;
+    float my_s = 0.f, ssum = 0.f;
+    for (int j = 0; j < a.k; ++j) {
+      float bv = -INFINITY;
+      int bi = 0x7fffffff;
+#pragma unroll
+      for (int i = 0; i < EPL; ++i) {
+        const int e = lane + 32 * i;
+        if (e < a.E && !((taken >> i) & 1u) && better(l[i], e, bv, bi)) {
+          bv = l[i];
+          bi = e;
+        }
+      }
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) {
+        const float ov = __shfl_xor_sync(0xffffffffu, bv, o);
+        const int oi = __shfl_xor_sync(0xffffffffu, bi, o);
+        if (better(ov, oi, bv, bi)) {
+          bv = ov;
+          bi = oi;
+        }
+      }
+      // owner lane marks it taken and shares its score
+      float sc = 0.f;
+#pragma unroll
+      for (int i = 0; i < EPL; ++i)
+        if (lane + 32 * i == bi) {
+          taken |= 1u << i;
+          sc = s[i];
+        }
+      sc = __shfl_sync(0xffffffffu, sc, bi & 31);
+      ssum += sc;  // same order (j) in every lane
+      if (lane == j) {
+        my_e = bi;
+        my_s = sc;
+      }
+    }
+    if (lane < a.k) {
+      float g = a.norm ? my_s / ssum : my_s;
+      g *= a.scale;
+      a.idx[(long long)t * a.k + lane] = my_e;
+      a.gates[(long long)t * a.k + lane] = g;
+      if (a.hist) atomicAdd(&s_hist[my_e], 1);
+    }
+  }
+  if (a.want_aux) {
+#pragma unroll
+    for (int i = 0; i < EPL; ++i) {
+      const int e = lane + 32 * i;
+      if (e < a.E) s_p[warp * a.E + e] = pacc[i];
+    }
+  }
+  __syncthreads();
+  for (int e = threadIdx.x; e < a.E; e += blockDim.x) {
+    if (a.hist) a.hist[(long long)blockIdx.x * a.E + e] = s_hist[e];
+    if (a.want_aux) {
+      float acc = 0.f;
+      for (int w = 0; w < WARPS; ++w) acc += s_p[w * a.E + e];
+      a.pblk[(long long)blockIdx.x * a.E + e] = acc;
+    }
+  }
+}
+
+// counts[e] = sum_b hist[b,e]; aux = E sum_e (counts_e / (T k)) (sum_b pblk[b,e] / T).
+__global__ void __launch_bounds__(512) finalize_kernel(const int* hist, const float* pblk, int nblk, int T, int E,
+                                                       int k, int32_t* counts, float* aux) {
+  __shared__ float red[512];
+  const int e = threadIdx.x;
+  float term = 0.f;
+  if (e < E) {
+    int c = 0;
+    float P = 0.f;
+    for (int b = 0; b < nblk; ++b) {
+      c += hist[(long long)b * E + e];
+      if (pblk) P += pblk[(long long)b * E + e];
+    }
+    if (counts) counts[e] = c;
+    term = ((float)c / ((float)T * (float)k)) * (P / (float)T);
+  }
+  red[threadIdx.x] = term;
+  __syncthreads();
+  for (int s = 256; s > 0; s >>= 1) {
+    if (threadIdx.x < s) red[threadIdx.x] += red[threadIdx.x + s];
+    __syncthreads();
+  }
+  if (threadIdx.x == 0 && aux) *aux = (float)E * red[0];
+}
+
+}  // namespace router
+
+static bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+namespace moe_impl {
+
+int check_cfg(const moe_config* c) {
+  if (!c) return MOE_ERR_INVALID_ARG;
+  if (c->T < 1 || c->H < 1 || c->E < 1 || c->k < 1 || c->F < 1) return MOE_ERR_INVALID_ARG;
+  if (c->k > c->E || c->k > 16 || c->E > 512) return MOE_ERR_UNSUPPORTED;
+  if (c->H % 128 != 0 || c->F % 128 != 0) return MOE_ERR_UNSUPPORTED;
+  if (c->score != MOE_SCORE_SOFTMAX && c->score != MOE_SCORE_SIGMOID) return MOE_ERR_INVALID_ARG;
+  if (c->expert_dtype != MOE_DT_BF16 && c->expert_dtype != MOE_DT_MXFP8) return MOE_ERR_INVALID_ARG;
+  if (c->n_shared != 0 && c->n_shared != 1) return MOE_ERR_UNSUPPORTED;
+  if (c->compute_aux && c->score != MOE_SCORE_SOFTMAX) return MOE_ERR_UNSUPPORTED;
+  if ((long long)c->T * c->k >= (1LL << 31) / 2) return MOE_ERR_UNSUPPORTED;
+  return MOE_OK;
+}
+
+size_t router_ws(const moe_config* c) {
+  const size_t nblk = (c->T + router::TOK_PER_BLOCK - 1) / router::TOK_PER_BLOCK;
+  return ws_round(nblk * c->E * sizeof(int)) + ws_round(nblk * c->E * sizeof(float));
+}
+
+// Router logits on the tensor cores: [T,H] x [E,H]^T -> fp32 [T,E] (+ bias).
+int router_logits(const moe_config* c, const void* x, const void* W_r, const float* bias, float* logits,
+                  cudaStream_t st) {
+  gg::Params p{};
+  const uint32_t bn = c->E <= 128 ? 128 : 256;
+  if (!moe_host::encode_tmap_2d(&p.tmA, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, x, c->H, c->T, (uint64_t)c->H * 2, 64, 128))
+    return MOE_ERR_CUDA;
+  if (!moe_host::encode_tmap_2d(&p.tmB0, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, W_r, c->H, c->E, (uint64_t)c->H * 2, 64,
+                                128))
+    return MOE_ERR_CUDA;
+  p.tmB1 = p.tmB0;
+  p.M = c->T;
+  p.N = c->E;
+  p.K = c->H;
+  p.G = 1;
+  p.offsets = nullptr;
+  p.b_group_rows = 0;
+  p.C = logits;
+  p.ldc = c->E;
+  p.bias = bias;
+  p.status = moe_host::device_status_ptr();
+  const int tiles = ((c->T + 127) / 128) * ((c->E + bn - 1) / bn);
+  if (bn == 128) return gg::launch<gg::Cfg<128, false, false, gg::EPI_F32, gg::GROUP_NONE, gg::B_SINGLE>>(p, tiles, st);
+  return gg::launch<gg::Cfg<256, false, false, gg::EPI_F32, gg::GROUP_NONE, gg::B_SINGLE>>(p, tiles, st);
+}
+
+int router_topk(const moe_config* c, const void* x, const void* W_r, const float* bias, float* logits, float* probs,
+                int32_t* idx, float* gates, int32_t* counts, float* aux, void* ws, size_t ws_bytes, cudaStream_t st) {
+  int rc = check_cfg(c);
+  if (rc) return rc;
+  const bool logits_in = (x == nullptr && W_r == nullptr);
+  if (!logits || !idx || !gates) return MOE_ERR_INVALID_ARG;
+  if (!logits_in && (!x || !W_r)) return MOE_ERR_INVALID_ARG;
+  if (aux && !c->compute_aux) return MOE_ERR_INVALID_ARG;
+  if (!logits_in && (!aligned16(x) || !aligned16(W_r))) return MOE_ERR_ALIGNMENT;
+  if (!aligned16(logits)) return MOE_ERR_ALIGNMENT;
+  const size_t need = router_ws(c);
+  if (!ws || ws_bytes < need) return MOE_ERR_WORKSPACE;
+  if (!logits_in) {
+    rc = router_logits(c, x, W_r, bias, logits, st);
+    if (rc) return rc;
+  }
+  const int nblk = (c->T + router::TOK_PER_BLOCK - 1) / router::TOK_PER_BLOCK;
+  router::TopkArgs a;
+  a.logits = logits;
+  a.probs = probs;
+  a.idx = idx;
+  a.gates = gates;
+  a.hist = reinterpret_cast<int*>(ws);
+  a.pblk = reinterpret_cast<float*>(static_cast<uint8_t*>(ws) + ws_round((size_t)nblk * c->E * sizeof(int)));
+  a.T = c->T;
+  a.E = c->E;
+  a.k = c->k;
+  a.score = c->score;
+  a.norm = c->norm_topk;
+  a.scale = c->route_scale;
+  a.want_aux = (aux != nullptr);
+  const size_t smem = (size_t)c->E * sizeof(int) + (size_t)router::WARPS * c->E * sizeof(float);
+  const dim3 grid(nblk), block(router::WARPS * 32);
+  if (c->E <= 32) router::topk_kernel<1><<<grid, block, smem, st>>>(a);
+  else if (c->E <= 128) router::topk_kernel<4><<<grid, block, smem, st>>>(a);
+  else if (c->E <= 256) router::topk_kernel<8><<<grid, block, smem, st>>>(a);
+  else router::topk_kernel<16><<<grid, block, smem, st>>>(a);
+  MOE_CHECK_LAUNCH();
+  if (counts || aux) {
+    router::finalize_kernel<<<1, 512, 0, st>>>(a.hist, aux ? a.pblk : nullptr, nblk, c->T, c->E, c->k, counts, aux);
+    MOE_CHECK_LAUNCH();
+  }
+  return MOE_OK;
+}
+
+}  // namespace moe_impl
+
+extern "C" size_t moe_router_workspace_size(const moe_config* cfg) {
+  if (moe_impl::check_cfg(cfg)) return 0;
+  return moe_impl::router_ws(cfg);
+}
+
+extern "C" int moe_router_topk(const moe_config* cfg, const void* x, const void* W_r, const float* logit_bias,
+                               float* logits, float* probs, int32_t* idx, float* gates, int32_t* counts, float* aux,
+                               void* ws, size_t ws_bytes, void* stream) {
+  return moe_impl::router_topk(cfg, x, W_r, logit_bias, logits, probs, idx, gates, counts, aux, ws, ws_bytes,
+                               static_cast<cudaStream_t>(stream));
+}

@@ -162,3 +162,16 @@ def random_gates(T: int, k: int, device="cpu", seed: int = 0) -> torch.Tensor:
     gen.manual_seed(seed)
     g = torch.rand((T, k), generator=gen) * 0.9 + 0.05
     return g.to(device)
+
+
+def randn_bf16(shape, std: float = 1.0, seed: int = 0, device="cpu", scale_rows: bool = False) -> torch.Tensor:
+    """Seeded N(0, std^2) tensor cast to bf16 (RNE). With scale_rows, each row
+    is further multiplied by 2^u, u uniform in [-12, 12] (a wide dynamic range
+    for quantiser tests)."""
+    gen = torch.Generator(device=device)
+    gen.manual_seed(seed)
+    t = torch.randn(shape, generator=gen, dtype=torch.float32, device=device) * std
+    if scale_rows:
+        u = torch.randint(-12, 13, (shape[0],) + (1,) * (len(shape) - 1), generator=gen, device=device)
+        t = t * torch.pow(2.0, u.to(torch.float32))
+    return t.to(torch.bfloat16)

@@ -1,0 +1,151 @@
+"""The C-ABI library: loads, exports what include/moe.h declares, and rejects
+bad arguments on the host before anything is launched (no GPU needed).
+
+Every call below fails validation before any CUDA call, so the (fake,
+never-dereferenced) pointer values are safe on any machine.
+"""
+import ctypes
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "moe.h")
+
+OK, INVALID, UNSUPPORTED, ALIGN, WS = 0, 1, 2, 3, 4
+
+
+@pytest.fixture(scope="module")
+def lib():
+    from mixture_experts_layer_aux_b200 import binding
+    return binding.load()
+
+
+@pytest.fixture(scope="module")
+def B():
+    from mixture_experts_layer_aux_b200 import binding
+    binding.load()
+    return binding
+
+
+def declared_functions():
+    src = open(HEADER).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(moe_[a-z0-9_]+)\s*\(", src)))
+
+
+def test_header_declares_the_layer_entry_points():
+    names = declared_functions()
+    for n in ["moe_router_topk", "moe_permute", "moe_grouped_gemm_fwd", "moe_grouped_gemm_bwd", "moe_unpermute",
+              "moe_layer_fwd", "moe_layer_bwd", "moe_quantize_mxfp8"]:
+        assert n in names
+
+
+def test_library_exports_every_declared_symbol(lib, B):
+    names = declared_functions()
+    assert len(names) >= 15
+    for n in names:
+        assert hasattr(lib, n), n
+        assert n in B.exported_symbols(), n   # and the binding wraps it
+
+
+def test_library_is_built_for_sm100a():
+    from mixture_experts_layer_aux_b200 import build
+    assert "arch=compute_100a,code=sm_100a" in " ".join(build.ARCH)
+    assert os.path.exists(build.LIB)
+
+
+def test_status_strings(lib):
+    for s in range(7):
+        assert lib.moe_status_string(s)
+    assert b"WORKSPACE" in lib.moe_status_string(WS)
+
+
+def cfg(B, **kw):
+    base = dict(T=512, H=256, E=8, k=2, F=512)
+    base.update(kw)
+    return B.make_config(**base)
+
+
+FAKE = 0x10000  # aligned, never dereferenced (every call fails validation first)
+
+
+def test_config_validation(lib, B):
+    c = cfg(B)
+    assert lib.moe_router_workspace_size(ctypes.byref(c)) > 0
+    for bad, code in [(dict(k=9), UNSUPPORTED), (dict(k=0), INVALID), (dict(E=600, k=2), UNSUPPORTED),
+                      (dict(H=200), UNSUPPORTED), (dict(F=100), UNSUPPORTED), (dict(T=0), INVALID),
+                      (dict(score=5), INVALID), (dict(n_shared=2), UNSUPPORTED),
+                      (dict(compute_aux=1, score=1), UNSUPPORTED)]:
+        c = cfg(B, **bad)
+        assert lib.moe_router_workspace_size(ctypes.byref(c)) == 0
+        rc = lib.moe_router_topk(ctypes.byref(c), FAKE, FAKE, None, FAKE, None, FAKE, FAKE, None, None, FAKE, 1 << 30,
+                                 None)
+        assert rc == code, (bad, rc)
+
+
+def test_router_argument_errors(lib, B):
+    c = cfg(B)
+    ws = lib.moe_router_workspace_size(ctypes.byref(c))
+    f = lib.moe_router_topk
+    assert f(ctypes.byref(c), FAKE, FAKE, None, None, None, FAKE, FAKE, None, None, FAKE, ws, None) == INVALID
+    assert f(ctypes.byref(c), FAKE, None, None, FAKE, None, FAKE, FAKE, None, None, FAKE, ws, None) == INVALID
+    assert f(ctypes.byref(c), FAKE + 2, FAKE, None, FAKE, None, FAKE, FAKE, None, None, FAKE, ws, None) == ALIGN
+    assert f(ctypes.byref(c), FAKE, FAKE, None, FAKE, None, FAKE, FAKE, None, None, FAKE, ws - 1, None) == WS
+    assert f(ctypes.byref(c), FAKE, FAKE, None, FAKE, None, FAKE, FAKE, None, None, None, ws, None) == WS
+    # aux requested without compute_aux
+    assert f(ctypes.byref(c), FAKE, FAKE, None, FAKE, None, FAKE, FAKE, None, FAKE, FAKE, ws, None) == INVALID
+
+
+def test_permute_argument_errors(lib, B):
+    c = cfg(B)
+    ws = lib.moe_permute_workspace_size(ctypes.byref(c))
+    f = lib.moe_permute
+    assert f(ctypes.byref(c), FAKE, None, None, None, FAKE, FAKE, FAKE, None, FAKE, None, FAKE, ws, None) == INVALID
+    assert f(ctypes.byref(c), FAKE, FAKE, None, None, FAKE, FAKE, FAKE, FAKE, FAKE, None, FAKE, ws, None) == INVALID
+    assert f(ctypes.byref(c), FAKE + 4, FAKE, None, None, FAKE, FAKE, FAKE, None, FAKE, None, FAKE, ws, None) == ALIGN
+    assert f(ctypes.byref(c), FAKE, FAKE, None, None, FAKE, FAKE, FAKE, None, FAKE, None, FAKE, ws - 1, None) == WS
+    cm = cfg(B, expert_dtype=1)
+    assert f(ctypes.byref(cm), FAKE, FAKE, None, None, FAKE, FAKE, FAKE, None, FAKE, None, FAKE, ws, None) == INVALID
+
+
+def test_gemm_and_layer_argument_errors(lib, B):
+    c = cfg(B)
+    g = lib.moe_grouped_gemm_fwd
+    ws = lib.moe_grouped_gemm_workspace_size(ctypes.byref(c), 0)
+    assert g(ctypes.byref(c), 7, FAKE, None, FAKE, None, FAKE, None, FAKE, FAKE, FAKE, None, None, FAKE, ws,
+             None) == INVALID
+    assert g(ctypes.byref(c), 0, FAKE, None, FAKE, None, None, None, FAKE, FAKE, FAKE, None, None, FAKE, ws,
+             None) == INVALID
+    assert g(ctypes.byref(c), 0, FAKE, None, FAKE + 8, None, FAKE, None, FAKE, FAKE, FAKE, None, None, FAKE, ws,
+             None) == ALIGN
+    assert g(ctypes.byref(c), 0, FAKE, None, FAKE, None, FAKE, None, FAKE, FAKE, FAKE, None, None, None, ws,
+             None) == WS
+    lw = lib.moe_layer_workspace_size(ctypes.byref(c))
+    assert lw > lib.moe_layer_saved_size(ctypes.byref(c)) // 8
+    L = lib.moe_layer_fwd
+    args = [FAKE, FAKE, None, FAKE, FAKE, FAKE, None, None, None, None, None, None, None, None, None, FAKE, None, None,
+            None, None, None, None]
+    assert L(ctypes.byref(c), *args, FAKE, lw - 1, None) == WS
+    args2 = list(args)
+    args2[0] = None
+    assert L(ctypes.byref(c), *args2, FAKE, lw, None) == INVALID
+    cs = cfg(B, save_for_bwd=1)
+    assert L(ctypes.byref(cs), *args, FAKE, lw, None) == INVALID     # saved buffer missing
+    csh = cfg(B, n_shared=1)
+    assert L(ctypes.byref(csh), *args, FAKE, lw, None) == INVALID    # shared weights missing
+    u = lib.moe_unpermute
+    assert u(ctypes.byref(c), FAKE, None, None, FAKE, None) == INVALID
+    assert u(ctypes.byref(c), FAKE + 1, FAKE, None, FAKE, None) == ALIGN
+    q = lib.moe_quantize_mxfp8
+    assert q(FAKE, 4, 48, FAKE, FAKE, None) == UNSUPPORTED
+    assert q(None, 4, 64, FAKE, FAKE, None) == INVALID
+    bw = lib.moe_layer_bwd
+    cb = cfg(B, save_for_bwd=1)
+    bws = lib.moe_layer_bwd_workspace_size(ctypes.byref(cb))
+    assert bw(ctypes.byref(cb), FAKE, ctypes.c_float(0.0), FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE,
+              FAKE, None, FAKE, bws - 1, None) == WS
+    cbm = cfg(B, expert_dtype=1)
+    assert bw(ctypes.byref(cbm), FAKE, ctypes.c_float(0.0), FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE,
+              FAKE, None, FAKE, bws, None) == UNSUPPORTED
