@@ -32,6 +32,8 @@ _lock = threading.Lock()
 _lib = None
 
 OC_BF16, OC_MXFP8, OC_F64 = 0, 1, 2
+# rounding points of the precision recipes (see moe_oracle.c)
+RECIPES = {"exact": 0, "mxfp8": 1, "bf16": 2}
 
 
 def build(force: bool = False) -> str:
@@ -61,6 +63,8 @@ def lib():
             _lib.oc_mx_scale_byte.restype = ctypes.c_uint8
             _lib.oc_mx_scale_byte.argtypes = [ctypes.c_double]
             _lib.oc_aux.restype = ctypes.c_double
+            _lib.oc_bf16_round.restype = ctypes.c_double
+            _lib.oc_bf16_round.argtypes = [ctypes.c_double]
             _lib.oc_num_threads.restype = ctypes.c_int
         return _lib
 
@@ -113,6 +117,15 @@ def mat_mx(codes: torch.Tensor, sf: torch.Tensor) -> Mat:
 
 def nthreads() -> int:
     return lib().oc_num_threads()
+
+
+def bf16_round(v: float) -> float:
+    """fp32-then-bf16 round-to-nearest-even of one value."""
+    return float(lib().oc_bf16_round(float(v)))
+
+
+def _recipe(r):
+    return RECIPES[r] if isinstance(r, str) else int(r)
 
 
 # ----------------------------------------------------------------- MXFP8
@@ -233,13 +246,16 @@ def _wmat(W, sf=None):
     return mat(W.reshape(-1, W.shape[-1]))
 
 
-def moe_fwd_tokens(x, W_g, W_u, W_d, idx, g, toks=None, *, mx=False, fold=True,
+def moe_fwd_tokens(x, W_g, W_u, W_d, idx, g, toks=None, *, recipe="exact", fold=True,
                    sf_g=None, sf_u=None, sf_d=None, shared=None, return_shared=False):
-    """Layer output rows y[toks] (fp64) for given routing (idx [T,k], gates g [T,k] fp64).
+    """Layer output rows y[toks] (fp64, unrounded) for given routing (idx [T,k], gates g [T,k] fp64).
 
+    recipe: "exact" (no rounding), "bf16" (the BF16 recipe's rounding points) or
+    "mxfp8" (the weight tensors are MXFP8 codes and sf_* their scales).
     shared = (W_gs, W_us, W_ds[, sf_gs, sf_us, sf_ds]) adds the always-on shared expert.
-    With mx, the weight tensors are MXFP8 codes and sf_* their scales.
     """
+    rc = _recipe(recipe)
+    mx = rc == RECIPES["mxfp8"]
     T, H = x.shape
     E, F = W_g.shape[0], W_g.shape[1]
     k = idx.shape[1]
@@ -262,7 +278,7 @@ def moe_fwd_tokens(x, W_g, W_u, W_d, idx, g, toks=None, *, mx=False, fold=True,
             sm = [_wmat(gs), _wmat(us), _wmat(ds)]
         sref = [m.ref for m in sm]
     null = ctypes.c_void_p(0)
-    lib().oc_moe_fwd_tokens(T, H, E, k, F, S, int(mx), int(fold), mxm.ref, mg.ref, mu.ref, md.ref,
+    lib().oc_moe_fwd_tokens(T, H, E, k, F, S, rc, int(fold), mxm.ref, mg.ref, mu.ref, md.ref,
                             sref[0] or null, sref[1] or null, sref[2] or null,
                             _p(_chk(idx.contiguous(), torch.int32)), _p(_chk(g.contiguous(), torch.float64)),
                             n, _p(toks), _p(y), _p(sh_out))
@@ -279,13 +295,15 @@ def moe_fwd_dense(x, W_g, W_u, W_d, gate_dense):
     return y
 
 
-def expert_rows(xp, e_of, g_of, W_g, W_u, W_d, rows=None, *, mx=False, sf_g=None, sf_u=None, sf_d=None,
+def expert_rows(xp, e_of, g_of, W_g, W_u, W_d, rows=None, *, recipe="exact", sf_g=None, sf_u=None, sf_d=None,
                 want=("ap", "o")):
     """Per-row expert stage: row r of xp goes to expert e_of[r] with gate g_of[r].
 
-    Returns a dict with any of zg, zu [n,F], ap [n,F] (= g * silu(zg) * zu, MXFP8-rounded
-    when mx) and o [n,H] = W_d[e] ap, all fp64, for the rows listed (default: all).
+    Returns a dict with any of zg, zu [n,F] (unrounded), ap [n,F] (= g * silu(zg) * zu,
+    rounded per recipe) and o [n,H] = W_d[e] ap (bf16-rounded under the bf16 and
+    mxfp8 recipes), all fp64, for the rows listed (default: all).
     """
+    rc = _recipe(recipe)
     R, H = xp.shape
     F = W_g.shape[1]
     if rows is None:
@@ -294,7 +312,7 @@ def expert_rows(xp, e_of, g_of, W_g, W_u, W_d, rows=None, *, mx=False, sf_g=None
     n = rows.numel()
     out = {w: torch.empty((n, H if w == "o" else F), dtype=torch.float64) for w in want}
     mxp, mg, mu, md = mat(xp), _wmat(W_g, sf_g), _wmat(W_u, sf_u), _wmat(W_d, sf_d)
-    lib().oc_expert_rows(H, F, int(mx), mxp.ref, _p(_chk(e_of.to(torch.int32).contiguous(), torch.int32)),
+    lib().oc_expert_rows(H, F, rc, mxp.ref, _p(_chk(e_of.to(torch.int32).contiguous(), torch.int32)),
                          _p(_chk(g_of.to(torch.float64).contiguous(), torch.float64)), mg.ref, mu.ref, md.ref,
                          n, _p(rows), _p(out.get("zg")), _p(out.get("zu")), _p(out.get("ap")), _p(out.get("o")))
     return out
@@ -312,7 +330,7 @@ def unpermute(o, row_of, shared=None):
 # ----------------------------------------------------------------- backward
 
 def moe_bwd_tokens(x, W_r, W_g, W_u, W_d, dY, r: dict, toks=None, *, score="softmax", norm=True,
-                   route_scale=1.0, aux_on=True, d_aux=0.0):
+                   route_scale=1.0, aux_on=True, d_aux=0.0, recipe="exact"):
     """dX[toks] (fp64, expert + router paths), dlogits[toks] [n,E] and dg [n,k] for routing r
     (the dict returned by route())."""
     T, H = x.shape
@@ -328,13 +346,13 @@ def moe_bwd_tokens(x, W_r, W_g, W_u, W_d, dY, r: dict, toks=None, *, score="soft
     s_soft = r["probs"] if score == "softmax" else scores(r["logits"], "softmax")
     ms = [mat(x), mat(W_r), _wmat(W_g), _wmat(W_u), _wmat(W_d), mat(dY)]
     lib().oc_moe_bwd_tokens(T, H, E, k, F, 0 if score == "softmax" else 1, int(norm), ctypes.c_double(route_scale),
-                            int(aux_on), ctypes.c_double(d_aux), *[m.ref for m in ms],
+                            int(aux_on), ctypes.c_double(d_aux), _recipe(recipe), *[m.ref for m in ms],
                             _p(r["idx"]), _p(_chk(r["probs"], torch.float64)), _p(s_soft), _p(r["counts"]),
                             n, _p(toks), _p(dx), _p(dl), _p(dg))
     return dx, dl, dg
 
 
-def moe_bwd_expert_dw(x, W_g, W_u, W_d, dY, idx, g, experts):
+def moe_bwd_expert_dw(x, W_g, W_u, W_d, dY, idx, g, experts, recipe="exact"):
     """dW_g, dW_u [n,F,H] and dW_d [n,H,F] (fp64) for the listed experts."""
     T, H = x.shape
     E, F = W_g.shape[0], W_g.shape[1]
@@ -345,23 +363,23 @@ def moe_bwd_expert_dw(x, W_g, W_u, W_d, dY, idx, g, experts):
     dWu = torch.empty((n, F, H), dtype=torch.float64)
     dWd = torch.empty((n, H, F), dtype=torch.float64)
     ms = [mat(x), _wmat(W_g), _wmat(W_u), _wmat(W_d), mat(dY)]
-    lib().oc_moe_bwd_expert_dw(T, H, E, k, F, *[m.ref for m in ms], _p(_chk(idx.contiguous(), torch.int32)),
+    lib().oc_moe_bwd_expert_dw(T, H, E, k, F, _recipe(recipe), *[m.ref for m in ms], _p(_chk(idx.contiguous(), torch.int32)),
                                _p(_chk(g.contiguous(), torch.float64)), n, _p(experts), _p(dWg), _p(dWu), _p(dWd))
     return dWg, dWu, dWd
 
 
-def router_dwr(dl: torch.Tensor, x: torch.Tensor) -> torch.Tensor:
+def router_dwr(dl: torch.Tensor, x: torch.Tensor, round_dl: bool = False) -> torch.Tensor:
     T, E = dl.shape
     H = x.shape[1]
     out = torch.empty((E, H), dtype=torch.float64)
     mx_ = mat(x)
-    lib().oc_router_dwr(T, H, E, _p(_chk(dl.contiguous(), torch.float64)), mx_.ref, _p(out))
+    lib().oc_router_dwr(T, H, E, _p(_chk(dl.contiguous(), torch.float64)), int(round_dl), mx_.ref, _p(out))
     return out
 
 
 # ----------------------------------------------------------------- whole layer
 
-def layer_fwd(wl, inp: dict, toks=None, logits=None, mx_weights=None) -> dict:
+def layer_fwd(wl, inp: dict, toks=None, logits=None, mx_weights=None, recipe=None) -> dict:
     """Full forward of workload `wl` on host inputs `inp` (synthetic.make_inputs layout).
 
     Routing is computed for every token; outputs y are computed for `toks`
@@ -374,6 +392,8 @@ def layer_fwd(wl, inp: dict, toks=None, logits=None, mx_weights=None) -> dict:
     r = route(logits.to(torch.float64), wl.k, wl.score, wl.norm_topk, wl.route_scale,
               with_aux=wl.aux and wl.score == "softmax")
     mx = wl.dtype == "mxfp8"
+    if recipe is None:
+        recipe = "mxfp8" if mx else "exact"
     kw = {}
     if mx:
         W = mx_weights
@@ -385,6 +405,6 @@ def layer_fwd(wl, inp: dict, toks=None, logits=None, mx_weights=None) -> dict:
     else:
         wg, wu, wd = inp["W_g"], inp["W_u"], inp["W_d"]
         shared = (inp["W_gs"], inp["W_us"], inp["W_ds"]) if wl.S else None
-    y = moe_fwd_tokens(inp["x"], wg, wu, wd, r["idx"], r["gates"], toks, mx=mx, shared=shared, **kw)
+    y = moe_fwd_tokens(inp["x"], wg, wu, wd, r["idx"], r["gates"], toks, recipe=recipe, shared=shared, **kw)
     r["y"] = y
     return r

@@ -47,6 +47,36 @@ static double bf16_to_double(uint16_t v) {
     return (double)f;
 }
 
+/* Round to bf16 the way a kernel that works in fp32 does: first to fp32, then
+ * to the nearest bf16 with ties to even (IEEE round-to-nearest-even on the
+ * upper 16 bits of the fp32 pattern). Inf/NaN pass through. */
+double oc_bf16_round(double v) {
+    float f = (float)v;
+    uint32_t u;
+    memcpy(&u, &f, 4);
+    if ((u & 0x7f800000u) == 0x7f800000u) return (double)f;
+    u += 0x7fffu + ((u >> 16) & 1u);
+    u &= 0xffff0000u;
+    memcpy(&f, &u, 4);
+    return (double)f;
+}
+
+/* Rounding points of the layer's precision recipes:
+ *   OC_EXACT  no rounding at all (fp64 throughout; used by the pins);
+ *   OC_MX     MXFP8 recipe: the expert GEMM operands are MXFP8 (x and the
+ *             gate-folded activation, 1x32 blocks along K), the expert GEMM
+ *             outputs are bf16;
+ *   OC_BF16R  BF16 recipe: the expert GEMM operands and outputs are bf16 (the
+ *             gate-folded activation, each expert's output; in the backward
+ *             the saved pre-activations, dgate/dup, the per-row dXp and the
+ *             router-gradient operand). */
+enum { OC_EXACT = 0, OC_MX = 1, OC_BF16R = 2 };
+
+static void round_vec(double* v, int n, int recipe) {
+    if (recipe == OC_BF16R || recipe == OC_MX)
+        for (int i = 0; i < n; ++i) v[i] = oc_bf16_round(v[i]);
+}
+
 /* E4M3 (OCP "fn" variant): 1 sign, 4 exponent (bias 7), 3 mantissa bits;
  * exponent field 0 is subnormal (m * 2^-9); S.1111.111 is NaN; max 448. */
 double oc_e4m3_decode(uint8_t c) {
@@ -352,6 +382,13 @@ static void expert_act(const oc_mat* Wg, const oc_mat* Wu, const double* xv, dou
     for (int f = 0; f < F; ++f) a[f] = silu(zg[f]) * zu[f];
 }
 
+/* The gate-folded activation as the down projection's operand: MXFP8 blocks
+ * along F (MXFP8 recipe) or bf16 (BF16 recipe). */
+static void round_act(double* a, int F, int recipe) {
+    if (recipe == OC_MX) mx_roundtrip(a, F);
+    else if (recipe == OC_BF16R) round_vec(a, F, recipe);
+}
+
 /*
  * Forward output rows for a list of tokens, given the routing.
  *
@@ -360,13 +397,17 @@ static void expert_act(const oc_mat* Wg, const oc_mat* Wu, const double* xv, dou
  *
  * fold = 1 evaluates W_d (g a) (the memory-efficient permutation order),
  * fold = 0 evaluates g (W_d a); the two agree up to rounding.
- * mx = 1 is the MXFP8 recipe: x is rounded to MXFP8 (1x32 blocks along H)
- * before the expert GEMMs, and the folded activation g*a (and the shared
- * expert's a) is rounded to MXFP8 along F before the down projection. The
- * weight matrices are then given as OC_MXFP8 (already quantised).
+ * recipe (OC_EXACT / OC_MX / OC_BF16R) selects the rounding points:
+ *   OC_MX: x is rounded to MXFP8 (1x32 blocks along H) before the expert
+ *     GEMMs, the gate-folded activation g*a (and the shared expert's a) to
+ *     MXFP8 along F before the down projection; the weights are given as
+ *     OC_MXFP8 matrices (already quantised);
+ *   OC_BF16R: g*a (and the shared a) is rounded to bf16;
+ *   both: each expert's down-projection output is rounded to bf16 before
+ *     the sum. y itself is returned unrounded.
  * Weight layouts: Wg, Wu [E*F, H]; Wd [E*H, F]; shared Wgs, Wus [F, H], Wds [H, F].
  */
-int oc_moe_fwd_tokens(int T, int H, int E, int k, int F, int S, int mx, int fold, const oc_mat* x,
+int oc_moe_fwd_tokens(int T, int H, int E, int k, int F, int S, int recipe, int fold, const oc_mat* x,
                       const oc_mat* Wg, const oc_mat* Wu, const oc_mat* Wd, const oc_mat* Wgs, const oc_mat* Wus,
                       const oc_mat* Wds, const int32_t* idx, const double* gates, int n_tok, const int32_t* toks,
                       double* y_out, double* shared_out) {
@@ -385,7 +426,7 @@ int oc_moe_fwd_tokens(int T, int H, int E, int k, int F, int S, int mx, int fold
         double* rowbuf = (double*)malloc(sizeof(double) * maxd);
         double* y = y_out + (long)i * H;
         oc_row(x, t, xv);
-        if (mx) mx_roundtrip(xv, H);
+        if (recipe == OC_MX) mx_roundtrip(xv, H);
         for (int h = 0; h < H; ++h) y[h] = 0.0;
         for (int j = 0; j < k; ++j) {
             int e = idx[(long)t * k + j];
@@ -396,19 +437,22 @@ int oc_moe_fwd_tokens(int T, int H, int E, int k, int F, int S, int mx, int fold
             expert_act(&we_g, &we_u, xv, zg, zu, a, rowbuf);
             if (fold) {
                 for (int f = 0; f < F; ++f) a[f] *= g;
-                if (mx) mx_roundtrip(a, F);
+                round_act(a, F, recipe);
                 matvec(&we_d, a, o, rowbuf);
+                round_vec(o, H, recipe);
                 for (int h = 0; h < H; ++h) y[h] += o[h];
             } else {
-                if (mx) mx_roundtrip(a, F);
+                round_act(a, F, recipe);
                 matvec(&we_d, a, o, rowbuf);
+                round_vec(o, H, recipe);
                 for (int h = 0; h < H; ++h) y[h] += g * o[h];
             }
         }
         if (S) {
             expert_act(Wgs, Wus, xv, zg, zu, a, rowbuf);
-            if (mx) mx_roundtrip(a, F);
+            round_act(a, F, recipe);
             matvec(Wds, a, o, rowbuf);
+            round_vec(o, H, recipe);
             for (int h = 0; h < H; ++h) y[h] += o[h];
             if (shared_out)
                 for (int h = 0; h < H; ++h) shared_out[(long)i * H + h] = o[h];
@@ -452,9 +496,11 @@ int oc_moe_fwd_dense(int T, int H, int E, int F, const oc_mat* x, const oc_mat* 
 
 /* Expert part of the layer for explicit (row -> expert, gate) lists, the way
  * the grouped GEMM stage sees it: a row r holds activation xp[r] routed to
- * expert e_of[r] with gate g_of[r]. Outputs ap [n, F] (g folded, optionally
- * MXFP8-rounded) and o [n, H] = W_d ap. Rows are independent. */
-int oc_expert_rows(int H, int F, int mx, const oc_mat* xp, const int32_t* e_of, const double* g_of,
+ * expert e_of[r] with gate g_of[r]. Outputs z_g, z_u [n, F] (unrounded),
+ * ap [n, F] = g * silu(z_g) * z_u rounded per `recipe` (it is the down
+ * projection's operand), and o [n, H] = W_d ap (rounded to bf16 under the MX
+ * and BF16 recipes). Rows are independent. */
+int oc_expert_rows(int H, int F, int recipe, const oc_mat* xp, const int32_t* e_of, const double* g_of,
                    const oc_mat* Wg, const oc_mat* Wu, const oc_mat* Wd, int n, const int32_t* rows,
                    double* zg_out, double* zu_out, double* ap_out, double* o_out) {
     int i;
@@ -469,17 +515,20 @@ int oc_expert_rows(int H, int F, int mx, const oc_mat* xp, const int32_t* e_of, 
         double* a = (double*)malloc(sizeof(double) * F);
         double* rowbuf = (double*)malloc(sizeof(double) * maxd);
         oc_row(xp, r, xv);
-        if (mx) mx_roundtrip(xv, H);
+        if (recipe == OC_MX) mx_roundtrip(xv, H);
         oc_mat we_g = oc_slice(Wg, (int64_t)e * F, F);
         oc_mat we_u = oc_slice(Wu, (int64_t)e * F, F);
         oc_mat we_d = oc_slice(Wd, (int64_t)e * H, H);
         expert_act(&we_g, &we_u, xv, zg, zu, a, rowbuf);
         for (int f = 0; f < F; ++f) a[f] *= g_of[r];
-        if (mx) mx_roundtrip(a, F);
+        round_act(a, F, recipe);
         if (zg_out) for (int f = 0; f < F; ++f) zg_out[(long)i * F + f] = zg[f];
         if (zu_out) for (int f = 0; f < F; ++f) zu_out[(long)i * F + f] = zu[f];
         if (ap_out) for (int f = 0; f < F; ++f) ap_out[(long)i * F + f] = a[f];
-        if (o_out) matvec(&we_d, a, o_out + (long)i * H, rowbuf);
+        if (o_out) {
+            matvec(&we_d, a, o_out + (long)i * H, rowbuf);
+            round_vec(o_out + (long)i * H, H, recipe);
+        }
         free(xv); free(zg); free(zu); free(a); free(rowbuf);
     }
     return 0;
@@ -488,8 +537,8 @@ int oc_expert_rows(int H, int F, int mx, const oc_mat* xp, const int32_t* e_of, 
 /* ------------------------------------------------------------ backward */
 
 /*
- * Exact derivative of the forward (bf16 / fp64 operands, softmax or sigmoid
- * scores with selected-normalised gates), for upstream dY [T,H] and d_aux.
+ * Derivative of the forward (bf16 / fp64 operands, softmax or sigmoid scores
+ * with selected-normalised gates), for upstream dY [T,H] and d_aux.
  * Per token t of the list:
  *   for each selected j (e = idx[t,j]):
  *     z_g, z_u, a = silu(z_g) z_u, v = W_d[e]^T dY_t,  dg_j = <v, a>
@@ -504,11 +553,16 @@ int oc_expert_rows(int H, int F, int mx, const oc_mat* xp, const int32_t* e_of, 
  *   aux path (softmax only, counts are constants):
  *     c_e = E count_e / (T k) / T,  dl[t,e] += d_aux s_e (c_e - sum_i s_i c_i)
  *   router: dx_t += sum_e dl[t,e] W_r[e]
+ * recipe OC_BF16R applies the BF16 recipe's rounding points: z_g and z_u are
+ * the saved bf16 pre-activations (a, silu, silu' are computed from them),
+ * dz_g and dz_u are rounded to bf16, each selected expert's contribution
+ * W_g^T dz_g + W_u^T dz_u is rounded to bf16, and the router path uses dl
+ * rounded to bf16 and rounds its result to bf16. dl itself stays unrounded.
  * logits, s (scores), gates, idx and counts are the forward's.
  */
 int oc_moe_bwd_tokens(int T, int H, int E, int k, int F, int score, int norm, double route_scale, int aux_on,
-                      double d_aux, const oc_mat* x, const oc_mat* Wr, const oc_mat* Wg, const oc_mat* Wu,
-                      const oc_mat* Wd, const oc_mat* dY, const int32_t* idx, const double* s_all,
+                      double d_aux, int recipe, const oc_mat* x, const oc_mat* Wr, const oc_mat* Wg,
+                      const oc_mat* Wu, const oc_mat* Wd, const oc_mat* dY, const int32_t* idx, const double* s_all,
                       const double* s_softmax, const int32_t* counts, int n_tok, const int32_t* toks,
                       double* dx_out, double* dl_out, double* dg_out) {
     int i;
@@ -524,6 +578,7 @@ int oc_moe_bwd_tokens(int T, int H, int E, int k, int F, int score, int norm, do
         double* v = (double*)malloc(sizeof(double) * F);
         double* dzg = (double*)malloc(sizeof(double) * F);
         double* dzu = (double*)malloc(sizeof(double) * F);
+        double* dxp = (double*)malloc(sizeof(double) * H);
         double* rowbuf = (double*)malloc(sizeof(double) * maxd);
         double* dg = (double*)malloc(sizeof(double) * k);
         double* g = (double*)malloc(sizeof(double) * k);
@@ -548,6 +603,11 @@ int oc_moe_bwd_tokens(int T, int H, int E, int k, int F, int score, int norm, do
             oc_mat we_u = oc_slice(Wu, (int64_t)e * F, F);
             oc_mat we_d = oc_slice(Wd, (int64_t)e * H, H);
             expert_act(&we_g, &we_u, xv, zg, zu, a, rowbuf);
+            if (recipe == OC_BF16R) {
+                round_vec(zg, F, recipe);
+                round_vec(zu, F, recipe);
+                for (int f = 0; f < F; ++f) a[f] = silu(zg[f]) * zu[f];
+            }
             for (int f = 0; f < F; ++f) v[f] = 0.0;
             matvec_t_acc(&we_d, dy, v, rowbuf);           /* v = W_d^T dY_t */
             dg[j] = dot(v, a, F);
@@ -556,8 +616,15 @@ int oc_moe_bwd_tokens(int T, int H, int E, int k, int F, int score, int norm, do
                 dzg[f] = da * zu[f] * silu_grad(zg[f]);
                 dzu[f] = da * silu(zg[f]);
             }
-            matvec_t_acc(&we_g, dzg, dx, rowbuf);
-            matvec_t_acc(&we_u, dzu, dx, rowbuf);
+            if (recipe == OC_BF16R) {
+                round_vec(dzg, F, recipe);
+                round_vec(dzu, F, recipe);
+            }
+            for (int h = 0; h < H; ++h) dxp[h] = 0.0;
+            matvec_t_acc(&we_g, dzg, dxp, rowbuf);
+            matvec_t_acc(&we_u, dzu, dxp, rowbuf);
+            if (recipe == OC_BF16R) round_vec(dxp, H, recipe);
+            for (int h = 0; h < H; ++h) dx[h] += dxp[h];
         }
         if (dg_out) for (int j = 0; j < k; ++j) dg_out[(long)i * k + j] = dg[j];
         /* gate path */
@@ -605,12 +672,16 @@ int oc_moe_bwd_tokens(int T, int H, int E, int k, int F, int score, int norm, do
             }
         }
         /* router path */
+        for (int h = 0; h < H; ++h) dxp[h] = 0.0;
         for (int e = 0; e < E; ++e) {
-            if (dl[e] == 0.0) continue;
+            double c = (recipe == OC_BF16R) ? oc_bf16_round(dl[e]) : dl[e];
+            if (c == 0.0) continue;
             oc_row(Wr, e, rowbuf);
-            for (int h = 0; h < H; ++h) dx[h] += dl[e] * rowbuf[h];
+            for (int h = 0; h < H; ++h) dxp[h] += c * rowbuf[h];
         }
-        free(xv); free(dy); free(zg); free(zu); free(a); free(v); free(dzg); free(dzu); free(rowbuf);
+        if (recipe == OC_BF16R) round_vec(dxp, H, recipe);
+        for (int h = 0; h < H; ++h) dx[h] += dxp[h];
+        free(xv); free(dy); free(zg); free(zu); free(a); free(v); free(dzg); free(dzu); free(dxp); free(rowbuf);
         free(dg); free(g);
     }
     return 0;
@@ -619,11 +690,13 @@ int oc_moe_bwd_tokens(int T, int H, int E, int k, int F, int score, int norm, do
 /*
  * Expert weight gradients for a list of experts, summing over every token
  * routed to each one (rows of the stable order, i.e. ascending token index):
- *   dW_d[e] += g dY_t (x) a,  dW_g[e] += dz_g (x) x_t,  dW_u[e] += dz_u (x) x_t
+ *   dW_d[e] += dY_t (x) (g a),  dW_g[e] += dz_g (x) x_t,  dW_u[e] += dz_u (x) x_t
  * Outputs: dWg, dWu [n_exp, F, H]; dWd [n_exp, H, F]. Experts with no token
- * get exact zeros. gates are the forward's [T,k].
+ * get exact zeros. gates are the forward's [T,k]. Under OC_BF16R, g a is the
+ * forward's bf16 activation (from the unrounded z), and dz_g, dz_u are the
+ * bf16 values of the backward (from the saved bf16 z, rounded).
  */
-int oc_moe_bwd_expert_dw(int T, int H, int E, int k, int F, const oc_mat* x, const oc_mat* Wg,
+int oc_moe_bwd_expert_dw(int T, int H, int E, int k, int F, int recipe, const oc_mat* x, const oc_mat* Wg,
                          const oc_mat* Wu, const oc_mat* Wd, const oc_mat* dY, const int32_t* idx,
                          const double* gates, int n_exp, const int32_t* exps, double* dWg, double* dWu,
                          double* dWd) {
@@ -668,12 +741,23 @@ int oc_moe_bwd_expert_dw(int T, int H, int E, int k, int F, const oc_mat* x, con
             oc_row(x, tl[i], xv);
             oc_row(dY, tl[i], dy);
             expert_act(&we_g, &we_u, xv, zg, zu, a, rowbuf);
+            /* A holds the down projection's operand g a */
+            for (int f = 0; f < F; ++f) a[f] *= gl[i];
+            if (recipe == OC_BF16R) {
+                round_vec(a, F, recipe);
+                round_vec(zg, F, recipe);
+                round_vec(zu, F, recipe);
+            }
             for (int f = 0; f < F; ++f) v[f] = 0.0;
             matvec_t_acc(&we_d, dy, v, rowbuf);
             for (int f = 0; f < F; ++f) {
                 double da = gl[i] * v[f];
                 DZG[(long)i * F + f] = da * zu[f] * silu_grad(zg[f]);
                 DZU[(long)i * F + f] = da * silu(zg[f]);
+            }
+            if (recipe == OC_BF16R) {
+                round_vec(DZG + (long)i * F, F, recipe);
+                round_vec(DZU + (long)i * F, F, recipe);
             }
             free(zg); free(zu); free(v); free(rowbuf);
         }
@@ -693,7 +777,7 @@ int oc_moe_bwd_expert_dw(int T, int H, int E, int k, int F, const oc_mat* x, con
 #pragma omp parallel for schedule(static)
         for (h = 0; h < H; ++h) {
             for (int ii = 0; ii < n; ++ii) {
-                double c = gl[ii] * DY[(long)ii * H + h];
+                double c = DY[(long)ii * H + h];
                 const double* a = A + (long)ii * F;
                 for (int f2 = 0; f2 < F; ++f2) gD[(long)h * F + f2] += c * a[f2];
             }
@@ -703,8 +787,9 @@ int oc_moe_bwd_expert_dw(int T, int H, int E, int k, int F, const oc_mat* x, con
     return 0;
 }
 
-/* dW_r[e,h] = sum_t dl[t,e] x[t,h] over all T tokens (ascending t). */
-void oc_router_dwr(int T, int H, int E, const double* dl, const oc_mat* x, double* dWr) {
+/* dW_r[e,h] = sum_t dl[t,e] x[t,h] over all T tokens (ascending t); with
+ * round_dl the bf16 value of dl is used (the BF16 recipe's operand). */
+void oc_router_dwr(int T, int H, int E, const double* dl, int round_dl, const oc_mat* x, double* dWr) {
     int e;
 #pragma omp parallel for schedule(static)
     for (e = 0; e < E; ++e) {
@@ -713,6 +798,7 @@ void oc_router_dwr(int T, int H, int E, const double* dl, const oc_mat* x, doubl
         for (int h = 0; h < H; ++h) out[h] = 0.0;
         for (int t = 0; t < T; ++t) {
             double c = dl[(long)t * E + e];
+            if (round_dl) c = oc_bf16_round(c);
             if (c == 0.0) continue;
             oc_row(x, t, xr);
             for (int h = 0; h < H; ++h) out[h] += c * xr[h];

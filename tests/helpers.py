@@ -30,3 +30,35 @@ def e_of_rows(offsets: torch.Tensor) -> torch.Tensor:
 
 def empty(shape, dtype, device="cuda"):
     return torch.empty(shape, dtype=dtype, device=device)
+
+
+def bf16_of(t: torch.Tensor) -> torch.Tensor:
+    """fp64 -> fp32 -> bf16 (round to nearest even) -> fp64, via torch's casts."""
+    return t.double().float().bfloat16().double()
+
+
+def check_bf16(got: torch.Tensor, ref: torch.Tensor, tol: float = TOL_BF16, max_flip_frac: float = 1e-3):
+    """Compare a bf16 kernel output with the oracle's value of the same tensor.
+
+    `ref` is the oracle's value before the output's own bf16 rounding, computed
+    with the kernels' bf16 rounding applied at every earlier point (identical
+    quantisation). Every element must lie within tol * rms(ref) of bf16(ref),
+    except elements where the two sides' pre-rounding values fall on either
+    side of a bf16 rounding boundary: those may differ by exactly one bf16 ulp
+    of the element, and at most max_flip_frac of the elements may do so.
+    Returns (max |got - bf16(ref)| / rms, max |got - ref| / rms, flips).
+    """
+    g = got.detach().double().cpu()
+    r = ref.detach().double().cpu()
+    assert g.shape == r.shape, (g.shape, r.shape)
+    r16 = bf16_of(r)
+    den = max(float(r.pow(2).mean().sqrt()), 1e-30)
+    d = (g - r16).abs()
+    bad = d > tol * den
+    flips = int(bad.sum())
+    if flips:
+        ulp = torch.pow(2.0, torch.floor(torch.log2(torch.maximum(r16.abs(), g.abs()).clamp_min(1e-38))) - 7)
+        assert bool((d[bad] <= ulp[bad] * (1 + 1e-9)).all()), \
+            f"elements beyond {tol}*rms that are not a single bf16 ulp apart: max {float(d.max()) / den:.3g} rms"
+        assert flips <= max(1, max_flip_frac * g.numel()), f"{flips} one-ulp differences beyond {tol}*rms"
+    return float(d.max()) / den, float((g - r).abs().max()) / den, flips

@@ -11,7 +11,7 @@ whose routing agrees (all of them, in practice).
 import pytest
 import torch
 
-from helpers import TOL_BF16, empty, err_rms
+from helpers import TOL_BF16, check_bf16, empty, err_rms
 from mixture_experts_layer_aux_b200.synthetic import WORKLOADS, Workload, make_inputs
 
 pytestmark = pytest.mark.gpu
@@ -67,9 +67,9 @@ def check_fwd(moe, oracle, wl, n_sample=None, seed=0):
         toks = torch.randperm(wl.T, generator=gen)[:n_sample].sort().values.to(torch.int32)
     toks = toks[same[toks.long()]]
     shared = (h["W_gs"], h["W_us"], h["W_ds"]) if wl.S else None
-    y_ref = oracle.moe_fwd_tokens(h["x"], h["W_g"], h["W_u"], h["W_d"], r["idx"], r["gates"], toks, shared=shared)
-    e = err_rms(out["y"].cpu()[toks.long()], y_ref)
-    assert e <= TOL_BF16, e
+    y_ref = oracle.moe_fwd_tokens(h["x"], h["W_g"], h["W_u"], h["W_d"], r["idx"], r["gates"], toks, shared=shared,
+                                  recipe="bf16")
+    e = check_bf16(out["y"].cpu()[toks.long()], y_ref)[0]
     ge = (out["gates"].cpu().double()[toks.long()] - r["gates"][toks.long()]).abs().max().item()
     assert ge <= 1e-5, ge
     if out["aux"] is not None:
@@ -139,27 +139,28 @@ def check_bwd(moe, oracle, wl, seed=0, d_aux=0.01, n_tok=None, experts=None):
     aux_on = wl.aux and wl.score == "softmax"
     dx, dl, _ = oracle.moe_bwd_tokens(h["x"], h["W_r"], h["W_g"], h["W_u"], h["W_d"], h["dY"], r, toks,
                                       score=wl.score, norm=wl.norm_topk, route_scale=wl.route_scale, aux_on=aux_on,
-                                      d_aux=d_aux)
+                                      d_aux=d_aux, recipe="bf16")
     res = {}
-    res["dX"] = err_rms(g["dX"].cpu()[toks.long()], dx)
+    res["dX"] = check_bf16(g["dX"].cpu()[toks.long()], dx)[0]
     res["dlogits"] = err_rms(g["dlogits"].cpu()[toks.long()], dl)
     if experts is None:
         experts = list(range(wl.E))
     dWg, dWu, dWd = oracle.moe_bwd_expert_dw(h["x"], h["W_g"], h["W_u"], h["W_d"], h["dY"], r["idx"], r["gates"],
-                                             experts)
+                                             experts, recipe="bf16")
     for name, ref in (("dW_g", dWg), ("dW_u", dWu), ("dW_d", dWd)):
         worst = 0.0
         for q, e in enumerate(experts):
             if int(r["counts"][e]) == 0:
                 assert (g[name][e] == 0).all(), (name, e)   # exact zeros for an expert with no token
             else:
-                worst = max(worst, err_rms(g[name][e].cpu(), ref[q]))
+                worst = max(worst, check_bf16(g[name][e].cpu(), ref[q])[0])
         res[name] = worst
     if n_tok is None:
-        res["dW_r"] = err_rms(g["dW_r"], oracle.router_dwr(dl, h["x"]))
+        res["dW_r"] = check_bf16(g["dW_r"].cpu(), oracle.router_dwr(dl, h["x"], round_dl=True))[0]
     else:
-        # property at any size: dW_r = dlogits^T x (with the GPU's own dlogits)
-        res["dW_r"] = err_rms(g["dW_r"], g["dlogits"].double().cpu().T @ h["x"].double())
+        # property at any size: dW_r = bf16(dlogits)^T x (with the GPU's own dlogits)
+        dl16 = g["dlogits"].double().cpu().float().bfloat16().double()
+        res["dW_r"] = check_bf16(g["dW_r"].cpu(), dl16.T @ h["x"].double())[0]
     bad = {k: v for k, v in res.items() if not v <= TOL_BF16}
     assert not bad, res
     assert moe.moe_get_device_status() == 0

@@ -396,3 +396,73 @@ def test_weight_grad_of_down_is_gated_outer_product_sum(oracle):
                 a = torch.nn.functional.silu(x[t] @ inp["W_g"][1].double().T) * (x[t] @ inp["W_u"][1].double().T)
                 ref += r["gates"][t, j] * torch.outer(dY[t], a)
     assert torch.allclose(dWd[0], ref, rtol=1e-12, atol=1e-13)
+
+
+# --------------------------------------------------------------- precision recipes
+
+
+def test_bf16_round_matches_torch_cast(oracle):
+    g = torch.Generator().manual_seed(3)
+    v = torch.randn(5000, generator=g, dtype=torch.float64) * torch.logspace(-30, 30, 5000, dtype=torch.float64)
+    # exact ties of the fp32 -> bf16 step: low 16 bits of the fp32 pattern = 0x8000
+    ties = (torch.randint(0, 2 ** 15, (200,), generator=g, dtype=torch.int32) * 65536 + 32768).view(torch.float32)
+    v = torch.cat([v, ties.double(), torch.tensor([0.0, -0.0, 1.0, -3.5, 65504.0])])
+    ref = v.float().bfloat16().double()
+    mine = torch.tensor([oracle.bf16_round(float(x)) for x in v], dtype=torch.float64)
+    assert torch.equal(mine, ref)
+
+
+def test_bf16_recipe_rounds_operand_and_output(oracle):
+    """ap is the bf16 value of the exact g*silu(zg)*zu; o is the bf16 value of W_d ap
+    (torch fp64 matmul as the library routine)."""
+    from mixture_experts_layer_aux_b200.synthetic import random_gates, randn_bf16
+    R, H, F, E = 40, 64, 96, 3
+    xp = randn_bf16((R, H), 1.0, seed=1)
+    e_of = torch.arange(R, dtype=torch.int32) % E
+    g = random_gates(R, 1, seed=2).flatten().double()
+    Wg, Wu, Wd = (randn_bf16((E, F, H), 0.02, seed=3), randn_bf16((E, F, H), 0.02, seed=4),
+                  randn_bf16((E, H, F), 0.02, seed=5))
+    ex = oracle.expert_rows(xp, e_of, g, Wg, Wu, Wd, want=("ap", "o"))
+    b = oracle.expert_rows(xp, e_of, g, Wg, Wu, Wd, recipe="bf16", want=("zg", "ap", "o"))
+    assert torch.equal(b["ap"], ex["ap"].float().bfloat16().double())
+    o_ref = torch.stack([Wd[int(e_of[r])].double() @ b["ap"][r] for r in range(R)])
+    assert torch.allclose(b["o"], o_ref.float().bfloat16().double(), rtol=0, atol=0) or \
+        (b["o"] - o_ref.float().bfloat16().double()).abs().max() <= 2.0 ** -8 * o_ref.abs().max()
+    assert not torch.equal(b["o"], ex["o"])
+
+
+def test_bf16_recipe_forward_composes_and_stays_near_exact(oracle):
+    wl = small(T=25, H=64, E=5, k=2, F=64)
+    inp = make_inputs(wl, seed=8)
+    r = oracle.layer_fwd(wl, inp)
+    yb = oracle.moe_fwd_tokens(inp["x"], inp["W_g"], inp["W_u"], inp["W_d"], r["idx"], r["gates"], recipe="bf16")
+    off = r["offsets"].long()
+    e_of = torch.bucketize(torch.arange(wl.T * wl.k), off[1:], right=True).to(torch.int32)
+    g_of = torch.empty(wl.T * wl.k, dtype=torch.float64)
+    g_of[r["row_of"].flatten().long()] = r["gates"].flatten()
+    xp = inp["x"][r["src_of"].long()].contiguous()
+    st = oracle.expert_rows(xp, e_of, g_of, inp["W_g"], inp["W_u"], inp["W_d"], recipe="bf16")
+    assert torch.allclose(oracle.unpermute(st["o"], r["row_of"]), yb, rtol=1e-14, atol=1e-15)
+    rms = r["y"].pow(2).mean().sqrt()
+    assert (yb - r["y"]).abs().max() <= 0.02 * rms
+
+
+def test_bf16_recipe_backward_stays_near_exact(oracle):
+    wl = small(T=30, H=64, E=4, k=2, F=64)
+    inp = make_inputs(wl, seed=9, with_dy=True)
+    r = oracle.layer_fwd(wl, inp)
+    args = (inp["x"], inp["W_r"], inp["W_g"], inp["W_u"], inp["W_d"], inp["dY"], r)
+    dx0, dl0, _ = oracle.moe_bwd_tokens(*args, d_aux=0.3)
+    dx1, dl1, _ = oracle.moe_bwd_tokens(*args, d_aux=0.3, recipe="bf16")
+    for a, b in ((dx0, dx1), (dl0, dl1)):
+        rms = a.pow(2).mean().sqrt()
+        assert 0 < (a - b).abs().max() <= 0.03 * rms
+    w0 = oracle.moe_bwd_expert_dw(inp["x"], inp["W_g"], inp["W_u"], inp["W_d"], inp["dY"], r["idx"], r["gates"], [0, 1])
+    w1 = oracle.moe_bwd_expert_dw(inp["x"], inp["W_g"], inp["W_u"], inp["W_d"], inp["dY"], r["idx"], r["gates"], [0, 1],
+                                  recipe="bf16")
+    for a, b in zip(w0, w1):
+        rms = a.pow(2).mean().sqrt()
+        assert 0 < (a - b).abs().max() <= 0.03 * rms
+    # the router-gradient operand: dl rounded to bf16
+    d_r = oracle.router_dwr(dl0, inp["x"], round_dl=True)
+    assert torch.allclose(d_r, dl0.float().bfloat16().double().T @ inp["x"].double(), rtol=1e-12, atol=1e-12)
