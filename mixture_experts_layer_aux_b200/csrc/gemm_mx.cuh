@@ -1,0 +1,454 @@
+// gemm_mx.cuh -- grouped MXFP8 GEMM on the sm_100a tensor cores
+// (tcgen05.mma kind::mxf8f6f4 with UE8M0 block scales, one scale per 1x32
+// block along K, E4M3 operands, fp32 accumulation in TMEM).
+//
+// The MXFP8 recipe is the Blackwell training recipe that section 3 of the
+// Megatron Core MoE technical summary lists (MXFP8 native support on Blackwell);
+// the block format is OCP MX v1.0.
+//
+// Layout of one stage (128 of K = 128 bytes of E4M3 per row):
+//   A tile 128 x 128 B and B tile 256 x 128 B, TMA, 128-byte swizzle;
+//   scale words: per row one uint32 holding the 4 UE8M0 bytes of its four
+//   32-wide K blocks (byte j = block j), gathered by a loader warp straight
+//   from the natural [rows, K/32] scale layout into the order that
+//   tcgen05.cp 32x128b.warpx4 expects: the 16 bytes of lane l hold rows l,
+//   l+32, l+64, l+96 (a 512-byte chunk per 128 rows).
+// MMA: per stage, tcgen05.cp copies the scale chunks into TMEM (SFA 4
+// columns, SFB 8 columns, two slots alternating by stage), then four
+// M128 N256 K32 MMAs select scale byte j through the instruction descriptor.
+// TMEM: one 256-column fp32 accumulator (the scale slots take the rest of the
+// 512 columns); eight epilogue warps (two per lane quadrant, 128 columns
+// each) first copy their accumulator columns into registers and release TMEM,
+// so the next tile's MMAs run while they finish the element-wise work.
+// Roles: warp 0 TMA producer, warp 1 MMA issuer (+ TMEM owner), warp 2 scale
+// loader, warps 3..10 epilogue. All waits are bounded like gemm.cuh.
+#pragma once
+
+#include <cuda_fp8.h>
+
+#include "common.cuh"
+
+namespace ggmx {
+
+constexpr int BM = 128;
+constexpr int BN = 256;
+constexpr int BK = 128;                 // bytes = E4M3 elements per stage
+constexpr int kStages = 4;
+constexpr int NUM_THREADS = 11 * 32;
+constexpr int MAX_G = 512;
+constexpr int A_BYTES = BM * BK;        // 16 KB
+constexpr int B_BYTES = BN * BK;        // 32 KB
+constexpr int SFA_BYTES = 512;
+constexpr int SFB_BYTES = 1024;
+constexpr int STAGE_BYTES = 51200;      // A + B + SFA + SFB, padded to 1024
+constexpr int TX_BYTES = A_BYTES + B_BYTES;
+constexpr int TMEM_COLS = 512;
+constexpr int SFA_COL = 256;            // + 4 * slot
+constexpr int SFB_COL = 264;            // + 8 * slot
+constexpr int BAR_BYTES = 1024;
+constexpr int SMEM_BYTES = 1024 + kStages * STAGE_BYTES + BAR_BYTES + 2 * (MAX_G + 1) * 4;
+static_assert(A_BYTES + B_BYTES + SFA_BYTES + SFB_BYTES <= STAGE_BYTES, "stage");
+static_assert(SMEM_BYTES <= 232448, "smem");
+
+enum Epi : int {
+  EPI_MX_SWIGLU = 0,  // acc = [gate | up] -> g * silu(gate) * up, quantised to MXFP8 (e4m3 + ue8m0 per 32)
+  EPI_MX_BF16 = 1,    // acc -> bf16
+};
+
+struct __align__(64) Params {
+  CUtensorMap tmA;
+  CUtensorMap tmB0;
+  CUtensorMap tmB1;
+  int M;              // rows of A (all groups)
+  int N;              // output columns per group
+  int K;              // reduction length (multiple of 128)
+  int G;
+  const int* offsets;
+  int b_group_rows;   // rows of one group in B's [G*rows, K] view
+  const uint8_t* sfa;   // [M, K/32]
+  const uint8_t* sfb0;  // [G*b_group_rows, K/32]
+  const uint8_t* sfb1;
+  void* C;              // SWIGLU: e4m3 [M, N]; BF16: bf16 [M, N]
+  uint8_t* C_sf;        // SWIGLU: ue8m0 [M, N/32]
+  long long ldc;
+  const float* row_gate;
+  int* status;
+};
+
+struct Tile {
+  int g, m0, n0, row0, m_valid;
+};
+
+__device__ __forceinline__ Tile get_tile(const Params& p, int t, const int* s_off, const int* s_tstart, int n_step) {
+  int lo = 0, hi = p.G - 1;
+  while (lo < hi) {
+    const int mid = (lo + hi + 1) >> 1;
+    if (s_tstart[mid] <= t) lo = mid;
+    else hi = mid - 1;
+  }
+  const int g = lo;
+  const int mg = s_off[g + 1] - s_off[g];
+  const int MB = (mg + BM - 1) / BM;
+  const int local = t - s_tstart[g];
+  Tile ti;
+  ti.g = g;
+  ti.m0 = (local % MB) * BM;
+  ti.n0 = (local / MB) * n_step;
+  ti.row0 = s_off[g] + ti.m0;
+  ti.m_valid = min(BM, mg - ti.m0);
+  return ti;
+}
+
+MOE_DEV void mma_mxf8(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc, uint32_t sfa_tmem,
+                      uint32_t sfb_tmem, uint32_t accumulate) {
+  asm volatile(
+      "{ .reg .pred p; setp.ne.b32 p, %4, 0; "
+      "tcgen05.mma.cta_group::1.kind::mxf8f6f4.block_scale [%0], %1, %2, %3, [%5], [%6], p; }" ::"r"(d_tmem),
+      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate), "r"(sfa_tmem), "r"(sfb_tmem)
+      : "memory");
+}
+
+// smem (32 rows x 16 bytes, no swizzle) -> TMEM lanes 0..31 of every quadrant, 4 columns.
+MOE_DEV void tmem_cp_32x128b_x4(uint32_t taddr, uint64_t sdesc) {
+  asm volatile("tcgen05.cp.cta_group::1.32x128b.warpx4 [%0], %1;" ::"r"(taddr), "l"(sdesc) : "memory");
+}
+
+// No-swizzle K-major descriptor of a 32-row x 16-byte chunk: 8-row core
+// matrices of 128 bytes, 128 bytes apart.
+MOE_DEV uint64_t sf_desc(uint32_t saddr) {
+  uint64_t d = 0;
+  d |= (uint64_t)((saddr >> 4) & 0x3FFF);
+  d |= (uint64_t)((128 >> 4) & 0x3FFF) << 32;  // stride byte offset
+  d |= (uint64_t)1 << 46;                      // version
+  return d;                                    // layout type 0: no swizzle
+}
+
+// Block-scaled instruction descriptor: E4M3 x E4M3, UE8M0 scales, K-major.
+__host__ __device__ constexpr uint32_t idesc_mx(int M, int N, int sf_id) {
+  return ((uint32_t)sf_id << 4) | (0u << 7) | (0u << 10) | ((uint32_t)(N >> 3) << 17) | (1u << 23) |
+         ((uint32_t)(M >> 4) << 24) | ((uint32_t)sf_id << 29);
+}
+
+// UE8M0 byte of a 1x32 block: clamp(floor(log2 amax) - 8 + 127, 0, 254), 0 for amax == 0.
+MOE_DEV uint8_t mx_scale_byte(float amax) {
+  const uint32_t b = __float_as_uint(amax);
+  const int eb = (int)((b >> 23) & 0xFFu);
+  if (!(amax > 0.f) || eb == 0) return 0;
+  int s = eb - 8;
+  s = s < 0 ? 0 : (s > 254 ? 254 : s);
+  return (uint8_t)s;
+}
+MOE_DEV float mx_inv_scale(uint8_t byte) { return __uint_as_float((uint32_t)(254 - byte) << 23); }
+
+// 32 fp32 values -> 32 e4m3 bytes (x inv, nearest-even, saturated) as 8 words.
+MOE_DEV void quant32(const float* v, float inv, uint32_t (&w)[8]) {
+#pragma unroll
+  for (int q = 0; q < 8; ++q) {
+    const __nv_fp8x2_storage_t lo =
+        __nv_cvt_float2_to_fp8x2(make_float2(v[4 * q] * inv, v[4 * q + 1] * inv), __NV_SATFINITE, __NV_E4M3);
+    const __nv_fp8x2_storage_t hi =
+        __nv_cvt_float2_to_fp8x2(make_float2(v[4 * q + 2] * inv, v[4 * q + 3] * inv), __NV_SATFINITE, __NV_E4M3);
+    w[q] = (uint32_t)lo | ((uint32_t)hi << 16);
+  }
+}
+
+template <int EPI, bool SPLIT_N>
+__global__ void __launch_bounds__(NUM_THREADS, 1) gemm_mx_kernel(const __grid_constant__ Params p) {
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* bar_area = smem + kStages * STAGE_BYTES;
+  uint64_t* full = reinterpret_cast<uint64_t*>(bar_area);
+  uint64_t* empty = full + kStages;
+  uint64_t* tfull = empty + kStages;
+  uint64_t* tempty = tfull + 1;
+  uint64_t* drain = tempty + 1;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  int* s_off = reinterpret_cast<int*>(bar_area + BAR_BYTES);
+  int* s_tstart = s_off + (MAX_G + 1);
+  constexpr int N_STEP = SPLIT_N ? BN / 2 : BN;
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  for (int i = threadIdx.x; i <= p.G; i += NUM_THREADS) s_off[i] = p.offsets[i];
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < kStages; ++i) {
+      mbar_init(&full[i], 2);  // TMA (expect_tx) + scale loader
+      mbar_init(&empty[i], 1);
+    }
+    mbar_init(tfull, 1);
+    mbar_init(tempty, 8);
+    mbar_init(drain, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, TMEM_COLS);
+    tmem_relinquish();
+  }
+  __syncthreads();
+  if (warp == 0) {
+    int bad = 0;
+    for (int i = lane; i < p.G; i += 32)
+      if (s_off[i + 1] < s_off[i] || s_off[i] < 0 || s_off[i + 1] > p.M) bad = 1;
+    bad = __any_sync(0xffffffffu, bad);
+    if (lane == 0) {
+      const int NT = (p.N + N_STEP - 1) / N_STEP;
+      int acc = 0;
+      for (int g = 0; g < p.G; ++g) {
+        s_tstart[g] = acc;
+        if (!bad) acc += ((s_off[g + 1] - s_off[g] + BM - 1) / BM) * NT;
+      }
+      s_tstart[p.G] = acc;
+      if (bad) record_status(p.status, DEV_BAD_OFFSETS);
+    }
+  }
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+  const int total = s_tstart[p.G];
+  const int KB = p.K / BK;
+  bool aborted = false;
+
+  if (warp == 0) {
+    // ======================= TMA producer (A and B tiles)
+    if (lane == 0) {
+      tma_prefetch_desc(&p.tmA);
+      tma_prefetch_desc(&p.tmB0);
+      if (SPLIT_N) tma_prefetch_desc(&p.tmB1);
+      int stage = 0;
+      uint32_t phase = 0, issued_mask = 0, issued_par = 0;
+      for (int t = blockIdx.x; t < total && !aborted; t += gridDim.x) {
+        const Tile ti = get_tile(p, t, s_off, s_tstart, N_STEP);
+        const int brow = ti.g * p.b_group_rows + ti.n0;
+        for (int kb = 0; kb < KB; ++kb) {
+          if (!mbar_wait(&empty[stage], phase ^ 1, abort_flag, p.status, DEV_WAIT_TIMEOUT_PRODUCER)) {
+            aborted = true;
+            break;
+          }
+          mbar_arrive_expect_tx(&full[stage], TX_BYTES);
+          issued_mask |= 1u << stage;
+          issued_par = (issued_par & ~(1u << stage)) | (phase << stage);
+          uint8_t* sA = smem + stage * STAGE_BYTES;
+          uint8_t* sB = sA + A_BYTES;
+          const int kc = kb * BK;
+          tma_load_2d(sA, &p.tmA, kc, ti.row0, &full[stage]);
+          if (SPLIT_N) {
+            tma_load_2d(sB, &p.tmB0, kc, brow, &full[stage]);
+            tma_load_2d(sB + 128 * BK, &p.tmB1, kc, brow, &full[stage]);
+          } else {
+            tma_load_2d(sB, &p.tmB0, kc, brow, &full[stage]);
+            tma_load_2d(sB + 128 * BK, &p.tmB0, kc, brow + 128, &full[stage]);
+          }
+          if (++stage == kStages) {
+            stage = 0;
+            phase ^= 1;
+          }
+        }
+      }
+      if (*abort_flag) {
+        for (int s = 0; s < kStages; ++s)
+          if (issued_mask & (1u << s)) {
+            const uint32_t par = (issued_par >> s) & 1u;
+            const uint64_t t0 = globaltimer_ns();
+            while (!mbar_try_wait(&full[s], par) && globaltimer_ns() - t0 < MOE_WAIT_NS) {
+            }
+          }
+      }
+    }
+  } else if (warp == 2) {
+    // ======================= scale loader: natural [rows, K/32] bytes -> UTCCP chunk order
+    const int kw = p.K / 32;  // scale bytes per row
+    int stage = 0;
+    uint32_t phase = 0;
+    for (int t = blockIdx.x; t < total && !aborted; t += gridDim.x) {
+      const Tile ti = get_tile(p, t, s_off, s_tstart, N_STEP);
+      const long long brow = (long long)ti.g * p.b_group_rows + ti.n0;
+      for (int kb = 0; kb < KB; ++kb) {
+        if (!__all_sync(0xffffffffu,
+                        mbar_wait(&empty[stage], phase ^ 1, abort_flag, p.status, DEV_WAIT_TIMEOUT_PRODUCER))) {
+          aborted = true;
+          break;
+        }
+        uint8_t* sSF = smem + stage * STAGE_BYTES + A_BYTES + B_BYTES;
+        uint32_t va[4], vb[8];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          const int r = ti.row0 + lane + 32 * i;
+          va[i] = (r < p.M) ? __ldg(reinterpret_cast<const uint32_t*>(p.sfa + (long long)r * kw) + kb) : 0u;
+        }
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          const uint8_t* base;
+          long long r;
+          if (SPLIT_N) {
+            base = i < 4 ? p.sfb0 : p.sfb1;
+            r = brow + lane + 32 * (i & 3);
+          } else {
+            base = p.sfb0;
+            r = brow + lane + 32 * i;
+          }
+          vb[i] = __ldg(reinterpret_cast<const uint32_t*>(base + r * kw) + kb);
+        }
+        *reinterpret_cast<uint4*>(sSF + 16 * lane) = make_uint4(va[0], va[1], va[2], va[3]);
+        *reinterpret_cast<uint4*>(sSF + SFA_BYTES + 16 * lane) = make_uint4(vb[0], vb[1], vb[2], vb[3]);
+        *reinterpret_cast<uint4*>(sSF + SFA_BYTES + 512 + 16 * lane) = make_uint4(vb[4], vb[5], vb[6], vb[7]);
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&full[stage]);
+        if (++stage == kStages) {
+          stage = 0;
+          phase ^= 1;
+        }
+      }
+    }
+  } else if (warp == 1) {
+    // ======================= MMA issuer
+    int stage = 0;
+    uint32_t phase = 0, acc_phase = 0;
+    int kcount = 0;  // stages consumed so far (selects the scale slot)
+    for (int t = blockIdx.x; t < total && !aborted; t += gridDim.x) {
+      if (!__all_sync(0xffffffffu, mbar_wait(tempty, acc_phase ^ 1, abort_flag, p.status, DEV_WAIT_TIMEOUT_MMA))) {
+        aborted = true;
+        break;
+      }
+      tc_fence_after();
+      for (int kb = 0; kb < KB; ++kb) {
+        if (!__all_sync(0xffffffffu, mbar_wait(&full[stage], phase, abort_flag, p.status, DEV_WAIT_TIMEOUT_MMA))) {
+          aborted = true;
+          break;
+        }
+        tc_fence_after();
+        if (lane == 0) {
+          uint8_t* sA = smem + stage * STAGE_BYTES;
+          uint8_t* sB = sA + A_BYTES;
+          uint8_t* sSF = sB + B_BYTES;
+          const int slot = kcount & 1;
+          const uint32_t sfa_t = tmem_base + SFA_COL + 4 * slot;
+          const uint32_t sfb_t = tmem_base + SFB_COL + 8 * slot;
+          tmem_cp_32x128b_x4(sfa_t, sf_desc(smem_u32(sSF)));
+          tmem_cp_32x128b_x4(sfb_t, sf_desc(smem_u32(sSF + SFA_BYTES)));
+          tmem_cp_32x128b_x4(sfb_t + 4, sf_desc(smem_u32(sSF + SFA_BYTES + 512)));
+          const uint32_t a0 = smem_u32(sA), b0 = smem_u32(sB);
+#pragma unroll
+          for (int j = 0; j < BK / 32; ++j) {
+            // scale byte j of each 32-bit TMEM word: in the descriptor's sf ids and in
+            // the top two bits of the scale addresses
+            mma_mxf8(tmem_base, smem_desc_sw128(a0 + j * 32, 16, 1024), smem_desc_sw128(b0 + j * 32, 16, 1024),
+                     idesc_mx(BM, BN, j), sfa_t | ((uint32_t)j << 30), sfb_t | ((uint32_t)j << 30),
+                     (kb | j) != 0 ? 1u : 0u);
+          }
+          mma_commit(&empty[stage]);
+        }
+        __syncwarp();
+        ++kcount;
+        if (++stage == kStages) {
+          stage = 0;
+          phase ^= 1;
+        }
+      }
+      if (aborted) break;
+      if (lane == 0) mma_commit(tfull);
+      __syncwarp();
+      acc_phase ^= 1;
+    }
+    if (*abort_flag && lane == 0) {
+      mma_commit(drain);
+      const uint64_t t0 = globaltimer_ns();
+      while (!mbar_try_wait(drain, 0) && globaltimer_ns() - t0 < MOE_WAIT_NS) {
+      }
+    }
+    __syncwarp();
+  } else {
+    // ======================= epilogue (warps 3..10): quadrant q, column half h
+    const int q = warp & 3;
+    const int h = (warp - 3) >> 2;
+    const int row = q * 32 + lane;
+    uint32_t acc_phase = 0;
+    for (int t = blockIdx.x; t < total && !aborted; t += gridDim.x) {
+      const Tile ti = get_tile(p, t, s_off, s_tstart, N_STEP);
+      if (!__all_sync(0xffffffffu, mbar_wait(tfull, acc_phase, abort_flag, p.status, DEV_WAIT_TIMEOUT_EPILOGUE))) {
+        aborted = true;
+        break;
+      }
+      tc_fence_after();
+      const uint32_t tb = tmem_base + ((uint32_t)(q * 32) << 16);
+      float v[128];
+      if (EPI == EPI_MX_SWIGLU) {
+        // gate columns [64h, 64h+64), up columns [128 + 64h, ...)
+        tmem_ld32(tb + 64 * h, *reinterpret_cast<float(*)[32]>(&v[0]));
+        tmem_ld32(tb + 64 * h + 32, *reinterpret_cast<float(*)[32]>(&v[32]));
+        tmem_ld32(tb + 128 + 64 * h, *reinterpret_cast<float(*)[32]>(&v[64]));
+        tmem_ld32(tb + 128 + 64 * h + 32, *reinterpret_cast<float(*)[32]>(&v[96]));
+      } else {
+#pragma unroll
+        for (int c = 0; c < 4; ++c) tmem_ld32(tb + 128 * h + 32 * c, *reinterpret_cast<float(*)[32]>(&v[32 * c]));
+      }
+      tmem_ld_wait();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(tempty);  // accumulator free: the next tile's MMAs may start
+      acc_phase ^= 1;
+      const bool valid = row < ti.m_valid;
+      const long long orow = (long long)ti.row0 + row;
+      if (valid) {
+        if (EPI == EPI_MX_SWIGLU) {
+          const float g = p.row_gate ? p.row_gate[orow] : 1.f;
+          float a[64];
+#pragma unroll
+          for (int i = 0; i < 64; ++i) a[i] = g * silu_f(v[i]) * v[64 + i];
+          const int col0 = ti.n0 + 64 * h;  // F column of a[0]
+          uint8_t* out = reinterpret_cast<uint8_t*>(p.C) + orow * p.ldc + col0;
+          uint8_t sb[2];
+#pragma unroll
+          for (int b = 0; b < 2; ++b) {
+            float am = 0.f;
+#pragma unroll
+            for (int i = 0; i < 32; ++i) am = fmaxf(am, fabsf(a[32 * b + i]));
+            sb[b] = mx_scale_byte(am);
+            uint32_t w[8];
+            quant32(a + 32 * b, mx_inv_scale(sb[b]), w);
+            uint4* o4 = reinterpret_cast<uint4*>(out + 32 * b);
+            o4[0] = make_uint4(w[0], w[1], w[2], w[3]);
+            o4[1] = make_uint4(w[4], w[5], w[6], w[7]);
+          }
+          *reinterpret_cast<uint16_t*>(p.C_sf + orow * (p.ldc / 32) + col0 / 32) =
+              (uint16_t)sb[0] | ((uint16_t)sb[1] << 8);
+        } else {
+          __nv_bfloat16* out = reinterpret_cast<__nv_bfloat16*>(p.C) + orow * p.ldc + ti.n0 + 128 * h;
+#pragma unroll
+          for (int c = 0; c < 16; ++c) {
+            uint4 u;
+            u.x = pack_bf16x2(v[8 * c], v[8 * c + 1]);
+            u.y = pack_bf16x2(v[8 * c + 2], v[8 * c + 3]);
+            u.z = pack_bf16x2(v[8 * c + 4], v[8 * c + 5]);
+            u.w = pack_bf16x2(v[8 * c + 6], v[8 * c + 7]);
+            reinterpret_cast<uint4*>(out)[c] = u;
+          }
+        }
+      }
+    }
+  }
+
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem_base, TMEM_COLS);
+  }
+}
+
+template <int EPI, bool SPLIT_N>
+int launch(const Params& p, int max_tiles, cudaStream_t stream) {
+  if (max_tiles <= 0) return MOE_OK;
+  auto kern = gemm_mx_kernel<EPI, SPLIT_N>;
+  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES) != cudaSuccess) {
+    (void)cudaGetLastError();
+    return MOE_ERR_CUDA;
+  }
+  int grid = moe_host::num_sms();
+  if (grid > max_tiles) grid = max_tiles;
+  kern<<<grid, NUM_THREADS, SMEM_BYTES, stream>>>(p);
+  MOE_CHECK_LAUNCH();
+  return MOE_OK;
+}
+
+}  // namespace ggmx

@@ -43,9 +43,11 @@ def check_bf16(got: torch.Tensor, ref: torch.Tensor, tol: float = TOL_BF16, max_
     `ref` is the oracle's value before the output's own bf16 rounding, computed
     with the kernels' bf16 rounding applied at every earlier point (identical
     quantisation). Every element must lie within tol * rms(ref) of bf16(ref),
-    except elements where the two sides' pre-rounding values fall on either
-    side of a bf16 rounding boundary: those may differ by exactly one bf16 ulp
-    of the element, and at most max_flip_frac of the elements may do so.
+    except elements downstream of a rounding decision that the two sides took
+    differently (their fp32 pre-rounding values straddled a bf16 rounding
+    boundary): such an element may differ by at most two bf16 ulps of itself
+    (one for its own rounding, one for a flipped term it sums), and at most
+    max_flip_frac of the elements may do so.
     Returns (max |got - bf16(ref)| / rms, max |got - ref| / rms, flips).
     """
     g = got.detach().double().cpu()
@@ -58,7 +60,33 @@ def check_bf16(got: torch.Tensor, ref: torch.Tensor, tol: float = TOL_BF16, max_
     flips = int(bad.sum())
     if flips:
         ulp = torch.pow(2.0, torch.floor(torch.log2(torch.maximum(r16.abs(), g.abs()).clamp_min(1e-38))) - 7)
-        assert bool((d[bad] <= ulp[bad] * (1 + 1e-9)).all()), \
-            f"elements beyond {tol}*rms that are not a single bf16 ulp apart: max {float(d.max()) / den:.3g} rms"
+        assert bool((d[bad] <= 2 * ulp[bad] * (1 + 1e-9)).all()), \
+            f"elements beyond {tol}*rms that are more than two bf16 ulps apart: max {float(d.max()) / den:.3g} rms"
         assert flips <= max(1, max_flip_frac * g.numel()), f"{flips} one-ulp differences beyond {tol}*rms"
     return float(d.max()) / den, float((g - r).abs().max()) / den, flips
+
+
+def e4m3_ulp(v: torch.Tensor) -> torch.Tensor:
+    """Spacing of the E4M3 grid at |v| (v already divided by its block scale)."""
+    a = v.abs().clamp_min(2.0 ** -6)
+    return torch.pow(2.0, torch.floor(torch.log2(a)) - 3)
+
+
+def check_mx(got_dq: torch.Tensor, ref_dq: torch.Tensor, scale: torch.Tensor, tol: float = 6e-2,
+             max_flip_frac: float = 1e-2):
+    """Compare dequantised MXFP8 kernel values with the oracle's MXFP8 values
+    (identical quantisation). Elements beyond tol*rms(ref) must be one E4M3 step
+    apart at their block scale (a rounding decision taken differently from
+    slightly different fp32 inputs), and be at most max_flip_frac of all."""
+    g = got_dq.double().cpu()
+    r = ref_dq.double().cpu()
+    s = scale.double().cpu()
+    den = max(float(r.pow(2).mean().sqrt()), 1e-30)
+    d = (g - r).abs()
+    bad = d > tol * den
+    flips = int(bad.sum())
+    if flips:
+        step = e4m3_ulp(torch.maximum(g.abs(), r.abs()) / s) * s
+        assert bool((d[bad] <= step[bad] * (1 + 1e-9)).all()), f"MXFP8 values more than one step apart"
+        assert flips <= max(1, max_flip_frac * g.numel()), f"{flips} MXFP8 step differences beyond {tol}*rms"
+    return float(d.max()) / den, flips

@@ -231,3 +231,54 @@ def test_grouped_gemm_fwd_matches_oracle(moe, oracle, T, H, E, k, F, zero, hot):
     check_bf16(save[:, F:].contiguous(), ref["zu"])
     check_bf16(o, ref["o"])
     _status_clean(moe)
+
+
+# ------------------------------------------------------------------ MXFP8 grouped GEMMs
+
+
+MX_CASES = [
+    # T, H, E, k, F, zero_experts, hot
+    (300, 256, 8, 2, 256, 2, 0.0),
+    (200, 512, 4, 1, 384, 0, 0.9),
+    (513, 1024, 16, 4, 512, 3, 0.3),
+]
+
+
+def _gpu_quant(moe, w):
+    codes = torch.empty(w.shape, dtype=torch.uint8, device="cuda")
+    sf = torch.empty(w.shape[:-1] + (w.shape[-1] // 32,), dtype=torch.uint8, device="cuda")
+    moe.moe_quantize_mxfp8(w.cuda().contiguous(), codes, sf)
+    return codes, sf
+
+
+@pytest.mark.parametrize("T,H,E,k,F,zero,hot", MX_CASES)
+def test_grouped_gemm_mxfp8_matches_oracle(moe, oracle, T, H, E, k, F, zero, hot):
+    from helpers import check_mx
+    idx = random_routing(T, E, k, seed=T + F + 1, zero_experts=zero, hot=hot)
+    counts, offsets, _, _ = oracle.maps(idx, E)
+    rows = T * k
+    xp = randn_bf16((rows, H), 1.0, seed=rows + 1)
+    g = random_gates(rows, 1, seed=rows + 2).flatten() * 2.5
+    Wg = randn_bf16((E, F, H), 0.02, seed=11)
+    Wu = randn_bf16((E, F, H), 0.02, seed=12)
+    Wd = randn_bf16((E, H, F), 0.02, seed=13)
+    cfg = moe.make_config(T=T, H=H, E=E, k=k, F=F, expert_dtype=1)
+    xq, xs = _gpu_quant(moe, xp)
+    (gq, gs), (uq, us), (dq, ds) = _gpu_quant(moe, Wg), _gpu_quant(moe, Wu), _gpu_quant(moe, Wd)
+    ap = empty((rows, F), torch.uint8)
+    ap_sf = empty((rows, F // 32), torch.uint8)
+    o = empty((rows, H), torch.bfloat16)
+    ws = moe.workspace(256)
+    off = offsets.cuda()
+    moe.moe_grouped_gemm_fwd(cfg, 0, xq, xs, gq, gs, uq, us, off, g.cuda(), ap, ap_sf, None, ws)
+    moe.moe_grouped_gemm_fwd(cfg, 1, ap, ap_sf, dq, ds, None, None, off, None, o, None, None, ws)
+    torch.cuda.synchronize()
+    # the oracle quantises the same bf16 weights itself (bit-identical codes, tested above)
+    Q = {n: oracle.mxfp8_quantize(w) for n, w in (("g", Wg), ("u", Wu), ("d", Wd))}
+    ref = oracle.expert_rows(xp, e_of_rows(offsets), g.double(), Q["g"][0], Q["u"][0], Q["d"][0], recipe="mxfp8",
+                             sf_g=Q["g"][1], sf_u=Q["u"][1], sf_d=Q["d"][1], want=("ap", "o"))
+    ap_dq = oracle.mxfp8_decode(ap.cpu(), ap_sf.cpu())
+    scale = torch.pow(2.0, ap_sf.cpu().double() - 127).repeat_interleave(32, 1)
+    check_mx(ap_dq, ref["ap"], scale)
+    check_bf16(o, ref["o"], tol=6e-2)
+    _status_clean(moe)
