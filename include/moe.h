@@ -132,6 +132,30 @@ int moe_permute(const moe_config* cfg, const void* x, const int32_t* idx, const 
                 void* ws, size_t ws_bytes, void* stream);
 
 /* ------------------------------------------------------------------------
+ * moe_permute without a workspace argument. The pages have no counterpart: this
+ * entry point exists for callers that cannot give the library device memory --
+ * for example code running where cudaMalloc is not allowed or would stall the
+ * device (inside a framework that owns all of HBM through its own pool, or in a
+ * host callback), and that cannot carve a workspace out of memory it owns.
+ *   Same arguments, results and errors as moe_permute, minus ws/ws_bytes.
+ *   Its scratch is one array of moe_permute_noalloc_scratch_capacity() bytes
+ *   (8 MiB) compiled into the library: every GPU that loads the library holds
+ *   it until the process exits. A configuration whose moe_permute workspace
+ *   would exceed it is rejected with MOE_ERR_UNSUPPORTED before any launch.
+ *   The first call on each device looks up the array's device address (no
+ *   allocation); make that first call before any stream capture.
+ *   All calls share the one array: two calls whose kernels overlap on the GPU
+ *   (different streams, or different host threads, on the same device) race.
+ *   Every scratch word is written before it is read within a call, so nothing
+ *   from an earlier call leaks into a later one.
+ *   It allocates and frees nothing, on the host or on the device.
+ * ------------------------------------------------------------------------ */
+size_t moe_permute_noalloc_scratch_capacity(void);
+int moe_permute_noalloc(const moe_config* cfg, const void* x, const int32_t* idx, const float* gates,
+                        int32_t* counts, int32_t* offsets, int32_t* row_of, int32_t* src_of, float* row_gate,
+                        void* xp, uint8_t* xp_sf, void* stream);
+
+/* ------------------------------------------------------------------------
  * Grouped expert GEMMs, forward (tcgen05 tensor cores, TMEM accumulators,
  * TMA operand staging; expert row ranges read from device `offsets`).
  * which == MOE_GEMM_GATEUP_SWIGLU:

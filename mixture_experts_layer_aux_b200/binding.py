@@ -49,6 +49,8 @@ _SIGS = {
     "moe_router_topk": (_I, [_CFG, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _SZ, _VP]),
     "moe_permute_workspace_size": (_SZ, [_CFG]),
     "moe_permute": (_I, [_CFG, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _SZ, _VP]),
+    "moe_permute_noalloc_scratch_capacity": (_SZ, []),
+    "moe_permute_noalloc": (_I, [_CFG, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP]),
     "moe_grouped_gemm_workspace_size": (_SZ, [_CFG, _I]),
     "moe_grouped_gemm_fwd": (_I, [_CFG, _I, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _SZ, _VP]),
     "moe_grouped_gemm_bwd_workspace_size": (_SZ, [_CFG, _I]),
@@ -165,6 +167,17 @@ def moe_permute(cfg, x, idx, gates, counts, offsets, row_of, src_of, row_gate, x
     return _check("moe_permute", load().moe_permute(
         ctypes.byref(cfg), _p(x), _p(idx), _p(gates), _p(counts), _p(offsets), _p(row_of), _p(src_of), _p(row_gate),
         _p(xp), _p(xp_sf), _p(ws), ws.numel() if ws is not None else 0, _st(stream)))
+
+
+def moe_permute_noalloc_scratch_capacity() -> int:
+    return load().moe_permute_noalloc_scratch_capacity()
+
+
+def moe_permute_noalloc(cfg, x, idx, gates, counts, offsets, row_of, src_of, row_gate, xp, xp_sf, stream=None):
+    """moe_permute with its scratch in the library's own fixed device array (no workspace argument)."""
+    return _check("moe_permute_noalloc", load().moe_permute_noalloc(
+        ctypes.byref(cfg), _p(x), _p(idx), _p(gates), _p(counts), _p(offsets), _p(row_of), _p(src_of),
+        _p(row_gate), _p(xp), _p(xp_sf), _st(stream)))
 
 
 def moe_grouped_gemm_workspace_size(cfg, which) -> int:

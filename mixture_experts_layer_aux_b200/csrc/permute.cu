@@ -21,6 +21,8 @@
 //            loads, one bf16 rounding.
 #include <cuda_fp8.h>
 
+#include <mutex>
+
 #include "common.cuh"
 #include "layout.h"
 
@@ -400,4 +402,59 @@ extern "C" int moe_unpermute(const moe_config* cfg, const void* o, const int32_t
 
 extern "C" int moe_quantize_mxfp8(const void* src, int64_t rows, int32_t K, uint8_t* dst, uint8_t* sf, void* stream) {
   return moe_impl::quantize_mxfp8(src, rows, K, dst, sf, static_cast<cudaStream_t>(stream));
+}
+
+// ---------------------------------------------------------------------------
+// moe_permute_noalloc: moe_permute for callers that cannot hand over device
+// memory. Its scratch (in-block ranks, per-block histograms and bases) lives in
+// one fixed array compiled into this library, so the caller passes only the
+// layer's inputs and outputs. The array is shared by every call on a device.
+// ---------------------------------------------------------------------------
+
+#define MOE_PERMUTE_NOALLOC_SCRATCH_BYTES (8u << 20)
+
+static __device__ __align__(256) uint8_t g_permute_noalloc_scratch[MOE_PERMUTE_NOALLOC_SCRATCH_BYTES];
+
+namespace {
+
+// Device address of the scratch array for the current device. The runtime only
+// knows it per device, so it is looked up once per device (with that device
+// current) and cached; the lookup allocates nothing.
+void* noalloc_scratch_ptr() {
+  static void* ptrs[64] = {};
+  static std::mutex mu;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) {
+    (void)cudaGetLastError();
+    return nullptr;
+  }
+  std::lock_guard<std::mutex> lk(mu);
+  if (!ptrs[dev]) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_permute_noalloc_scratch) != cudaSuccess) {
+      (void)cudaGetLastError();
+      return nullptr;
+    }
+    ptrs[dev] = p;
+  }
+  return ptrs[dev];
+}
+
+}  // namespace
+
+extern "C" size_t moe_permute_noalloc_scratch_capacity(void) { return MOE_PERMUTE_NOALLOC_SCRATCH_BYTES; }
+
+extern "C" int moe_permute_noalloc(const moe_config* cfg, const void* x, const int32_t* idx, const float* gates,
+                                   int32_t* counts, int32_t* offsets, int32_t* row_of, int32_t* src_of,
+                                   float* row_gate, void* xp, uint8_t* xp_sf, void* stream) {
+  int rc = moe_impl::check_cfg(cfg);
+  if (rc) return rc;
+  const size_t need = moe_impl::permute_ws(cfg);
+  if (need > MOE_PERMUTE_NOALLOC_SCRATCH_BYTES) return MOE_ERR_UNSUPPORTED;
+  void* scratch = noalloc_scratch_ptr();
+  if (!scratch) return MOE_ERR_CUDA;
+  // every scratch word the kernels read is written earlier in the same call
+  // (ranks, histograms, bases), so nothing needs clearing between calls
+  return moe_impl::permute(cfg, x, idx, gates, counts, offsets, row_of, src_of, row_gate, xp, xp_sf, scratch,
+                           MOE_PERMUTE_NOALLOC_SCRATCH_BYTES, static_cast<cudaStream_t>(stream));
 }
