@@ -73,6 +73,8 @@ struct __align__(64) Params {
   const __nv_bfloat16* gateup;  // SWIGLU_BWD: saved [rows, 2F]
   float* dg_part;               // SWIGLU_BWD: [rows, N/BN] partial <v, a>
   int F;                        // SwiGLU width: column offset of the 'up' half
+  int ksplit;                   // GROUP_NONE: K split into this many slices (0/1: none); EPI_F32 only
+  long long c_split_stride;     // elements between the slices' partial outputs
   int* status;
 };
 
@@ -91,7 +93,10 @@ struct Cfg {
   static constexpr int TMEM_COLS = 2 * BN;
   static constexpr int N_STEP = (BMODE == B_SPLIT_N) ? BN / 2 : BN;  // output columns per tile
   static constexpr int BAR_BYTES = 1024;
-  static constexpr int SMEM_BYTES = 1024 + kStages * STAGE_BYTES + BAR_BYTES + 2 * (MAX_G + 1) * 4;
+  // bf16 epilogue staging: per epilogue warp 32 rows x (128 + 16) bytes (64 columns at a time)
+  static constexpr int STG_ROW = 144;
+  static constexpr int STG_BYTES = (EPI == EPI_BF16) ? 4 * 32 * STG_ROW : 0;
+  static constexpr int SMEM_BYTES = 1024 + kStages * STAGE_BYTES + BAR_BYTES + 2 * (MAX_G + 1) * 4 + 128 + STG_BYTES;
   static_assert(BN == 128 || BN == 256, "BN");
   static_assert(!(BMODE == B_SPLIT_N && B_MN), "split-N is for K-major weights");
 };
@@ -104,6 +109,7 @@ struct Tile {
   int k0;       // first K coordinate (GROUP_K: offsets[g])
   int kblocks;  // k-blocks of BK
   int klast;    // valid K rows in the last k-block (GROUP_K tails)
+  int ks;       // K slice (GROUP_NONE with ksplit > 1)
 };
 
 template <class C>
@@ -138,9 +144,12 @@ __device__ __forceinline__ Tile get_tile(const Params& p, int t, const int* s_of
   } else {
     const int MT = (p.M + BM - 1) / BM;
     const int per_g = MT * NT;
+    // GROUP_K: t / per_g is the group; GROUP_NONE: it is the K slice
     const int g = (C::GROUP == GROUP_K) ? t / per_g : 0;
-    const int local = t - g * per_g;
+    const int ks = (C::GROUP == GROUP_NONE && p.ksplit > 1) ? t / per_g : 0;
+    const int local = t - (g + ks) * per_g;
     const int mb = local % MT, nb = local / MT;
+    ti.ks = ks;
     ti.g = g;
     ti.m0 = mb * BM;
     ti.n0 = nb * C::N_STEP;
@@ -152,8 +161,11 @@ __device__ __forceinline__ Tile get_tile(const Params& p, int t, const int* s_of
       ti.kblocks = (kg + BK - 1) / BK;
       ti.klast = kg - (ti.kblocks - 1) * BK;
     } else {
-      ti.k0 = 0;
-      ti.kblocks = (p.K + BK - 1) / BK;
+      const int kb_total = (p.K + BK - 1) / BK;
+      const int ns = p.ksplit > 1 ? p.ksplit : 1;
+      const int kb_per = (kb_total + ns - 1) / ns;
+      ti.k0 = ks * kb_per * BK;
+      ti.kblocks = max(0, min(kb_per, kb_total - ks * kb_per));
       ti.klast = BK;  // a ragged dense K is zero-filled by TMA (out of the tensor)
     }
   }
@@ -175,6 +187,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) gemm_kernel(const __grid_const
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   int* s_off = reinterpret_cast<int*>(bar_area + C::BAR_BYTES);
   int* s_tstart = s_off + (MAX_G + 1);
+  uint8_t* stg_area = reinterpret_cast<uint8_t*>(
+      (reinterpret_cast<uintptr_t>(s_tstart + (MAX_G + 1)) + 127) & ~uintptr_t(127));
+  (void)stg_area;
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -233,7 +248,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) gemm_kernel(const __grid_const
     const int MT = (p.M + BM - 1) / BM;
     if constexpr (C::GROUP == GROUP_M) total = s_tstart[p.G];
     else if constexpr (C::GROUP == GROUP_K) total = s_tstart[0] ? p.G * MT * NT : 0;
-    else total = MT * NT;
+    else total = MT * NT * (p.ksplit > 1 ? p.ksplit : 1);
   }
 
   bool aborted = false;
@@ -435,23 +450,64 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) gemm_kernel(const __grid_const
           }
         }
       } else if constexpr (C::EPI == EPI_BF16) {
-        __nv_bfloat16* out;
+        // Row q*32+i of the tile goes to out_base + (row0 + q*32 + i) * ld. Each warp converts
+        // 64 columns of its 32 rows to bf16, stages them in shared memory, and stores them
+        // back row-contiguously: one warp store = 4 rows x 128 bytes.
+        __nv_bfloat16* out_base;
+        long long ld, rbase;
         if constexpr (C::GROUP == GROUP_K) {
-          long long r = orow;
+          rbase = ti.row0;
           __nv_bfloat16* base = reinterpret_cast<__nv_bfloat16*>(p.C);
-          long long ld = p.ldc;
-          if (p.c2_row_split > 0 && r >= p.c2_row_split) {
-            r -= p.c2_row_split;
+          ld = p.ldc;
+          if (p.c2_row_split > 0 && rbase >= p.c2_row_split) {  // whole tile on one side (split % 128 == 0)
+            rbase -= p.c2_row_split;
             base = reinterpret_cast<__nv_bfloat16*>(p.C2);
             ld = p.ldc2;
           }
-          out = base + (long long)ti.g * p.c_group_stride + r * ld + ti.n0;
+          out_base = base + (long long)ti.g * p.c_group_stride;
         } else {
-          out = reinterpret_cast<__nv_bfloat16*>(p.C) + orow * p.ldc + ti.n0;
+          rbase = ti.row0;
+          ld = p.ldc;
+          out_base = reinterpret_cast<__nv_bfloat16*>(p.C);
         }
+        uint8_t* stg = stg_area + (warp - 2) * 32 * C::STG_ROW;
+        const int nvalid = min(C::BN, p.N - ti.n0);
+#pragma unroll 1
+        for (int cg = 0; cg < C::BN / 64; ++cg) {
+          if (cg * 64 >= nvalid) break;  // warp-uniform
+          float v[64];
+          if (!empty_k) {
+            tmem_ld32(tb + cg * 64, *reinterpret_cast<float(*)[32]>(&v[0]));
+            tmem_ld32(tb + cg * 64 + 32, *reinterpret_cast<float(*)[32]>(&v[32]));
+            tmem_ld_wait();
+          } else {
+#pragma unroll
+            for (int i = 0; i < 64; ++i) v[i] = 0.f;
+          }
+#pragma unroll
+          for (int j = 0; j < 8; ++j)
+            *reinterpret_cast<uint4*>(stg + lane * C::STG_ROW + 16 * j) =
+                make_uint4(pack_bf16x2(v[8 * j], v[8 * j + 1]), pack_bf16x2(v[8 * j + 2], v[8 * j + 3]),
+                           pack_bf16x2(v[8 * j + 4], v[8 * j + 5]), pack_bf16x2(v[8 * j + 6], v[8 * j + 7]));
+          __syncwarp();
+          const int ch = lane & 7;  // 16-byte chunk of the 128-byte row segment
+#pragma unroll
+          for (int i = 0; i < 8; ++i) {
+            const int r = 4 * i + (lane >> 3);  // row within this warp's 32
+            const int col = cg * 64 + ch * 8;
+            if (q * 32 + r < ti.m_valid && col < nvalid) {
+              const uint4 val = *reinterpret_cast<const uint4*>(stg + r * C::STG_ROW + 16 * ch);
+              *reinterpret_cast<uint4*>(out_base + (rbase + q * 32 + r) * ld + ti.n0 + col) = val;
+            }
+          }
+          __syncwarp();
+        }
+      } else if constexpr (C::EPI == EPI_F32) {
+        float* out = reinterpret_cast<float*>(p.C) + ti.ks * p.c_split_stride + orow * p.ldc + ti.n0;
         const int nvalid = min(C::BN, p.N - ti.n0);
 #pragma unroll 1
         for (int c = 0; c < C::BN / 32; ++c) {
+          if (c * 32 >= nvalid) break;  // warp-uniform
           float v[32];
           if (!empty_k) {
             tmem_ld32(tb + c * 32, v);
@@ -460,24 +516,6 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) gemm_kernel(const __grid_const
 #pragma unroll
             for (int i = 0; i < 32; ++i) v[i] = 0.f;
           }
-          if (valid && c * 32 < nvalid) {
-            uint32_t pk[16];
-#pragma unroll
-            for (int i = 0; i < 16; ++i) pk[i] = pack_bf16x2(v[2 * i], v[2 * i + 1]);
-            uint4* o4 = reinterpret_cast<uint4*>(out + c * 32);
-#pragma unroll
-            for (int i = 0; i < 4; ++i) o4[i] = make_uint4(pk[4 * i], pk[4 * i + 1], pk[4 * i + 2], pk[4 * i + 3]);
-          }
-        }
-      } else if constexpr (C::EPI == EPI_F32) {
-        float* out = reinterpret_cast<float*>(p.C) + orow * p.ldc + ti.n0;
-        const int nvalid = min(C::BN, p.N - ti.n0);
-#pragma unroll 1
-        for (int c = 0; c < C::BN / 32; ++c) {
-          if (c * 32 >= nvalid) break;  // warp-uniform
-          float v[32];
-          tmem_ld32(tb + c * 32, v);
-          tmem_ld_wait();
           if (valid) {
 #pragma unroll
             for (int i = 0; i < 32; ++i) {

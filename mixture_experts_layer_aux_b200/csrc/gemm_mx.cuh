@@ -9,10 +9,11 @@
 // Layout of one stage (128 of K = 128 bytes of E4M3 per row):
 //   A tile 128 x 128 B and B tile 256 x 128 B, TMA, 128-byte swizzle;
 //   scale words: per row one uint32 holding the 4 UE8M0 bytes of its four
-//   32-wide K blocks (byte j = block j), gathered by a loader warp straight
-//   from the natural [rows, K/32] scale layout into the order that
-//   tcgen05.cp 32x128b.warpx4 expects: the 16 bytes of lane l hold rows l,
-//   l+32, l+64, l+96 (a 512-byte chunk per 128 rows).
+//   32-wide K blocks (byte j = block j), gathered by a loader warp with
+//   asynchronous 4-byte copies straight from the natural [rows, K/32] scale
+//   layout into the order that tcgen05.cp 32x128b.warpx4 expects: the 16
+//   bytes of lane l hold rows l, l+32, l+64, l+96 (a 512-byte chunk per 128
+//   rows); the copies' completion is an arrival on the stage's barrier.
 // MMA: per stage, tcgen05.cp copies the scale chunks into TMEM (SFA 4
 // columns, SFB 8 columns, two slots alternating by stage), then four
 // M128 N256 K32 MMAs select scale byte j through the instruction descriptor.
@@ -108,6 +109,17 @@ MOE_DEV void mma_mxf8(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t 
       : "memory");
 }
 
+// 4-byte asynchronous global -> shared copy; src_bytes 0 writes zeros.
+MOE_DEV void cp_async_4(void* smem_dst, const void* gsrc, uint32_t src_bytes) {
+  asm volatile("cp.async.ca.shared.global [%0], [%1], 4, %2;" ::"r"(smem_u32(smem_dst)), "l"(gsrc), "r"(src_bytes)
+               : "memory");
+}
+// Arrive on `bar` once all cp.async copies of this thread so far have landed
+// (counts as one of the barrier's expected arrivals).
+MOE_DEV void cp_async_arrive_noinc(uint64_t* bar) {
+  asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(smem_u32(bar)) : "memory");
+}
+
 // smem (32 rows x 16 bytes, no swizzle) -> TMEM lanes 0..31 of every quadrant, 4 columns.
 MOE_DEV void tmem_cp_32x128b_x4(uint32_t taddr, uint64_t sdesc) {
   asm volatile("tcgen05.cp.cta_group::1.32x128b.warpx4 [%0], %1;" ::"r"(taddr), "l"(sdesc) : "memory");
@@ -172,7 +184,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) gemm_mx_kernel(const __grid_co
   for (int i = threadIdx.x; i <= p.G; i += NUM_THREADS) s_off[i] = p.offsets[i];
   if (threadIdx.x == 0) {
     for (int i = 0; i < kStages; ++i) {
-      mbar_init(&full[i], 2);  // TMA (expect_tx) + scale loader
+      mbar_init(&full[i], 33);  // TMA (expect_tx) + the scale loader's 32 lanes (cp.async)
       mbar_init(&empty[i], 1);
     }
     mbar_init(tfull, 1);
@@ -270,11 +282,12 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) gemm_mx_kernel(const __grid_co
           break;
         }
         uint8_t* sSF = smem + stage * STAGE_BYTES + A_BYTES + B_BYTES;
-        uint32_t va[4], vb[8];
+        // lane l: words of rows l, l+32, l+64, l+96 (A), the same for both 128-row halves of B
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
           const int r = ti.row0 + lane + 32 * i;
-          va[i] = (r < p.M) ? __ldg(reinterpret_cast<const uint32_t*>(p.sfa + (long long)r * kw) + kb) : 0u;
+          const bool ok = r < p.M;
+          cp_async_4(sSF + 16 * lane + 4 * i, p.sfa + (long long)(ok ? r : 0) * kw + 4 * kb, ok ? 4u : 0u);
         }
 #pragma unroll
         for (int i = 0; i < 8; ++i) {
@@ -287,20 +300,17 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) gemm_mx_kernel(const __grid_co
             base = p.sfb0;
             r = brow + lane + 32 * i;
           }
-          vb[i] = __ldg(reinterpret_cast<const uint32_t*>(base + r * kw) + kb);
+          cp_async_4(sSF + SFA_BYTES + (i >> 2) * 512 + 16 * lane + 4 * (i & 3), base + r * kw + 4 * kb, 4u);
         }
-        *reinterpret_cast<uint4*>(sSF + 16 * lane) = make_uint4(va[0], va[1], va[2], va[3]);
-        *reinterpret_cast<uint4*>(sSF + SFA_BYTES + 16 * lane) = make_uint4(vb[0], vb[1], vb[2], vb[3]);
-        *reinterpret_cast<uint4*>(sSF + SFA_BYTES + 512 + 16 * lane) = make_uint4(vb[4], vb[5], vb[6], vb[7]);
-        fence_proxy_async_smem();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&full[stage]);
+        cp_async_arrive_noinc(&full[stage]);
         if (++stage == kStages) {
           stage = 0;
           phase ^= 1;
         }
       }
     }
+    // every copy this warp issued lands before the CTA can exit (also on abort)
+    asm volatile("cp.async.wait_all;" ::: "memory");
   } else if (warp == 1) {
     // ======================= MMA issuer
     int stage = 0;
@@ -319,6 +329,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) gemm_mx_kernel(const __grid_co
         }
         tc_fence_after();
         if (lane == 0) {
+          // the scale words arrived through the generic proxy (cp.async); tcgen05.cp reads
+          // shared memory through the async proxy
+          fence_proxy_async_smem();
           uint8_t* sA = smem + stage * STAGE_BYTES;
           uint8_t* sB = sA + A_BYTES;
           uint8_t* sSF = sB + B_BYTES;

@@ -8,10 +8,10 @@
 // (sync-free kernels, section 2.4): no count ever reaches the host.
 //
 // Kernels:
-//   rank     one warp per 128 tokens: stable in-block rank of every (t, j)
-//            among the block's earlier tokens with the same expert (bitmask
-//            per expert in shared memory, popc of the lanes below), and the
-//            block's expert histogram.
+//   rank     eight warps per 256 tokens: each warp ranks its 32 tokens per
+//            expert (a lane bitmask per expert in shared memory, popc of the
+//            lanes below), a per-expert scan over the warps turns that into the
+//            stable in-block rank of every (t, j), and the block's histogram.
 //   scan     one block: counts, exclusive-scan offsets, per-block bases.
 //   scatter  one warp per token: row = base[block, e] + rank; writes row_of,
 //            src_of, row_gate; copies the token's row once from HBM and writes
@@ -28,68 +28,78 @@
 
 namespace perm {
 
-constexpr int RANK_TOK = 128;  // tokens per rank block (one warp)
+constexpr int RANK_WARPS = 8;                 // warps per rank block
+constexpr int RANK_TOK = RANK_WARPS * 32;     // tokens per rank block
 constexpr int SC_WARPS = 8;    // warps per scatter / unpermute block
 
-__global__ void __launch_bounds__(32) rank_kernel(const int32_t* __restrict__ idx, int T, int E, int k,
-                                                  int32_t* __restrict__ lrank, int* __restrict__ hist, int* status) {
+__global__ void __launch_bounds__(RANK_WARPS * 32) rank_kernel(const int32_t* __restrict__ idx, int T, int E,
+                                                                int k, int32_t* __restrict__ lrank,
+                                                                int* __restrict__ hist, int* status) {
   extern __shared__ uint32_t s_rank[];
-  uint32_t* mask = s_rank;                                // [E]
-  int* cnt = reinterpret_cast<int*>(s_rank + E);          // [E]
-  const int lane = threadIdx.x;
-  for (int e = lane; e < E; e += 32) {
-    mask[e] = 0;
-    cnt[e] = 0;
+  uint32_t* mask = s_rank;                                         // [RANK_WARPS][E]: lanes holding expert e
+  int* cnt = reinterpret_cast<int*>(s_rank + RANK_WARPS * E);      // [RANK_WARPS][E]: count, then warp base
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  for (int i = threadIdx.x; i < RANK_WARPS * E; i += blockDim.x) {
+    mask[i] = 0;
+    cnt[i] = 0;
   }
-  __syncwarp();
-  for (int c = 0; c < RANK_TOK / 32; ++c) {
-    const int t = blockIdx.x * RANK_TOK + c * 32 + lane;
-    const bool tv = t < T;
-    int es[16];
-    int bad = 0;
+  __syncthreads();
+  // 1. each warp ranks its 32 tokens among themselves (ascending lane = ascending token)
+  const int t = blockIdx.x * RANK_TOK + warp * 32 + lane;
+  const bool tv = t < T;
+  uint32_t* wm = mask + warp * E;
+  int* wc = cnt + warp * E;
+  int es[16], lr[16];
+  int bad = 0;
 #pragma unroll
-    for (int j = 0; j < 16; ++j) {
-      es[j] = -1;
-      if (j < k && tv) {
-        int e = idx[(long long)t * k + j];
-        if (e < 0 || e >= E) {
+  for (int j = 0; j < 16; ++j) {
+    es[j] = -1;
+    if (j < k && tv) {
+      int e = idx[(long long)t * k + j];
+      if (e < 0 || e >= E) {
+        bad = 1;
+        e = -1;
+      }
+      for (int i = 0; i < j; ++i)
+        if (es[i] == e && e >= 0) {
           bad = 1;
           e = -1;
         }
-        for (int i = 0; i < j; ++i)
-          if (es[i] == e && e >= 0) {
-            bad = 1;
-            e = -1;
-          }
-        es[j] = e;
-      }
+      es[j] = e;
     }
-    if (bad) record_status(status, DEV_BAD_INDEX);
-#pragma unroll
-    for (int j = 0; j < 16; ++j)
-      if (j < k && es[j] >= 0) atomicOr(&mask[es[j]], 1u << lane);
-    __syncwarp();
-#pragma unroll
-    for (int j = 0; j < 16; ++j)
-      if (j < k && tv) {
-        const int e = es[j];
-        lrank[(long long)t * k + j] = e >= 0 ? cnt[e] + __popc(mask[e] & ((1u << lane) - 1u)) : -1;
-      }
-    __syncwarp();
-#pragma unroll
-    for (int j = 0; j < 16; ++j)
-      if (j < k && es[j] >= 0) {
-        const int e = es[j];
-        const uint32_t m = mask[e];
-        if (m != 0 && (__ffs(m) - 1) == lane) cnt[e] += __popc(m);
-      }
-    __syncwarp();
-#pragma unroll
-    for (int j = 0; j < 16; ++j)
-      if (j < k && es[j] >= 0) mask[es[j]] = 0;
-    __syncwarp();
   }
-  for (int e = lane; e < E; e += 32) hist[(long long)blockIdx.x * E + e] = cnt[e];
+  if (bad) record_status(status, DEV_BAD_INDEX);
+#pragma unroll
+  for (int j = 0; j < 16; ++j)
+    if (j < k && es[j] >= 0) atomicOr(&wm[es[j]], 1u << lane);
+  __syncwarp();
+#pragma unroll
+  for (int j = 0; j < 16; ++j) {
+    lr[j] = -1;
+    if (j < k && es[j] >= 0) {
+      const uint32_t m = wm[es[j]];
+      lr[j] = __popc(m & ((1u << lane) - 1u));
+      if ((__ffs(m) - 1) == lane) wc[es[j]] = __popc(m);  // one writer per expert
+    }
+  }
+  __syncthreads();
+  // 2. per expert: exclusive scan over the warps (warp order = token order) and the block total
+  for (int e = threadIdx.x; e < E; e += blockDim.x) {
+    int run = 0;
+    for (int w = 0; w < RANK_WARPS; ++w) {
+      const int c = cnt[w * E + e];
+      cnt[w * E + e] = run;
+      run += c;
+    }
+    hist[(long long)blockIdx.x * E + e] = run;
+  }
+  __syncthreads();
+  // 3. block-local rank = warp base + rank within the warp
+  if (tv) {
+#pragma unroll
+    for (int j = 0; j < 16; ++j)
+      if (j < k) lrank[(long long)t * k + j] = es[j] >= 0 ? wc[es[j]] + lr[j] : -1;
+  }
 }
 
 // counts, offsets [E+1], base[b,e] = offsets[e] + sum_{b'<b} hist[b',e].
@@ -219,6 +229,7 @@ __global__ void __launch_bounds__(SC_WARPS * 32) scatter_kernel(
   }
 }
 
+template <int KM>  // compile-time bound on k: the per-slot arrays hold KM entries
 __global__ void __launch_bounds__(SC_WARPS * 32) unpermute_kernel(const __nv_bfloat16* __restrict__ o,
                                                                   const int32_t* __restrict__ row_of,
                                                                   const __nv_bfloat16* __restrict__ extra, int T,
@@ -232,38 +243,55 @@ __global__ void __launch_bounds__(SC_WARPS * 32) unpermute_kernel(const __nv_bfl
     r = row_of[(long long)t * k + lane];
     if (r < 0 || r >= rows_total) r = -1;
   }
-  int rows[16];
+  int rows[KM];
 #pragma unroll
-  for (int j = 0; j < 16; ++j) rows[j] = __shfl_sync(0xffffffffu, r, j < k ? j : 0);
+  for (int j = 0; j < KM; ++j) rows[j] = __shfl_sync(0xffffffffu, r, j < k ? j : 0);
   const int nchunk = H / 8;
-  for (int i = lane; i < nchunk; i += 32) {
-    uint4 d[16];
+  // loads of up to UNP_ILP chunks x k rows are issued before any sum (memory-level parallelism);
+  // each chunk is still summed in slot order j = 0..k-1
+  constexpr int UNP_ILP = KM <= 2 ? 4 : (KM <= 4 ? 2 : 1);
+  for (int i0 = lane; i0 < nchunk; i0 += 32 * UNP_ILP) {
+    uint4 d[UNP_ILP][KM];
+    uint4 ex[UNP_ILP];
 #pragma unroll
-    for (int j = 0; j < 16; ++j)
-      if (j < k) d[j] = rows[j] >= 0 ? reinterpret_cast<const uint4*>(o + (long long)rows[j] * H)[i] : make_uint4(0, 0, 0, 0);
-    float acc[8];
+    for (int u = 0; u < UNP_ILP; ++u) {
+      const int i = i0 + 32 * u;
 #pragma unroll
-    for (int q = 0; q < 8; ++q) acc[q] = 0.f;
+      for (int j = 0; j < KM; ++j)
+        if (j < k)
+          d[u][j] = (i < nchunk && rows[j] >= 0) ? reinterpret_cast<const uint4*>(o + (long long)rows[j] * H)[i]
+                                                 : make_uint4(0, 0, 0, 0);
+      ex[u] = (extra && i < nchunk) ? reinterpret_cast<const uint4*>(extra + (long long)t * H)[i]
+                                    : make_uint4(0, 0, 0, 0);
+    }
 #pragma unroll
-    for (int j = 0; j < 16; ++j)
-      if (j < k) {
+    for (int u = 0; u < UNP_ILP; ++u) {
+      const int i = i0 + 32 * u;
+      if (i >= nchunk) break;
+      float acc[8];
+#pragma unroll
+      for (int q = 0; q < 8; ++q) acc[q] = 0.f;
+#pragma unroll
+      for (int j = 0; j < KM; ++j)
+        if (j < k) {
+          float f[8];
+          unpack_bf16x8(d[u][j], f);
+#pragma unroll
+          for (int q = 0; q < 8; ++q) acc[q] += f[q];
+        }
+      if (extra) {
         float f[8];
-        unpack_bf16x8(d[j], f);
+        unpack_bf16x8(ex[u], f);
 #pragma unroll
         for (int q = 0; q < 8; ++q) acc[q] += f[q];
       }
-    if (extra) {
-      float f[8];
-      unpack_bf16x8(reinterpret_cast<const uint4*>(extra + (long long)t * H)[i], f);
-#pragma unroll
-      for (int q = 0; q < 8; ++q) acc[q] += f[q];
+      uint4 out;
+      out.x = pack_bf16x2(acc[0], acc[1]);
+      out.y = pack_bf16x2(acc[2], acc[3]);
+      out.z = pack_bf16x2(acc[4], acc[5]);
+      out.w = pack_bf16x2(acc[6], acc[7]);
+      reinterpret_cast<uint4*>(y + (long long)t * H)[i] = out;
     }
-    uint4 out;
-    out.x = pack_bf16x2(acc[0], acc[1]);
-    out.y = pack_bf16x2(acc[2], acc[3]);
-    out.z = pack_bf16x2(acc[4], acc[5]);
-    out.w = pack_bf16x2(acc[6], acc[7]);
-    reinterpret_cast<uint4*>(y + (long long)t * H)[i] = out;
   }
 }
 
@@ -324,7 +352,8 @@ int permute(const moe_config* c, const void* x, const int32_t* idx, const float*
   int* hist = cv.take<int>((size_t)nblk * c->E);
   int* base = cv.take<int>((size_t)nblk * c->E);
   int* status = moe_host::device_status_ptr();
-  perm::rank_kernel<<<nblk, 32, 2 * c->E * sizeof(uint32_t), st>>>(idx, c->T, c->E, c->k, lrank, hist, status);
+  perm::rank_kernel<<<nblk, perm::RANK_WARPS * 32, 2 * perm::RANK_WARPS * c->E * sizeof(uint32_t), st>>>(
+      idx, c->T, c->E, c->k, lrank, hist, status);
   MOE_CHECK_LAUNCH();
   perm::scan_kernel<<<1, 512, 0, st>>>(hist, nblk, c->E, base, counts, offsets);
   MOE_CHECK_LAUNCH();
@@ -356,9 +385,13 @@ int unpermute(const moe_config* c, const void* o, const int32_t* row_of, const v
   if (!o || !row_of || !y) return MOE_ERR_INVALID_ARG;
   if (!al16(o) || !al16(y) || (extra && !al16(extra))) return MOE_ERR_ALIGNMENT;
   const int grid = (c->T + perm::SC_WARPS - 1) / perm::SC_WARPS;
-  perm::unpermute_kernel<<<grid, perm::SC_WARPS * 32, 0, st>>>(static_cast<const __nv_bfloat16*>(o), row_of,
-                                                               static_cast<const __nv_bfloat16*>(extra), c->T, c->H,
-                                                               c->k, static_cast<__nv_bfloat16*>(y));
+  const auto* o16 = static_cast<const __nv_bfloat16*>(o);
+  const auto* e16 = static_cast<const __nv_bfloat16*>(extra);
+  auto* y16 = static_cast<__nv_bfloat16*>(y);
+  if (c->k <= 2) perm::unpermute_kernel<2><<<grid, perm::SC_WARPS * 32, 0, st>>>(o16, row_of, e16, c->T, c->H, c->k, y16);
+  else if (c->k <= 4) perm::unpermute_kernel<4><<<grid, perm::SC_WARPS * 32, 0, st>>>(o16, row_of, e16, c->T, c->H, c->k, y16);
+  else if (c->k <= 8) perm::unpermute_kernel<8><<<grid, perm::SC_WARPS * 32, 0, st>>>(o16, row_of, e16, c->T, c->H, c->k, y16);
+  else perm::unpermute_kernel<16><<<grid, perm::SC_WARPS * 32, 0, st>>>(o16, row_of, e16, c->T, c->H, c->k, y16);
   MOE_CHECK_LAUNCH();
   return MOE_OK;
 }

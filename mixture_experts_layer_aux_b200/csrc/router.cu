@@ -20,11 +20,16 @@
 
 namespace router {
 
-constexpr int TOK_PER_WARP = 8;
+constexpr int TOK_PER_WARP = 2;
 constexpr int WARPS = 8;
-constexpr int TOK_PER_BLOCK = TOK_PER_WARP * WARPS;  // 64
+constexpr int TOK_PER_BLOCK = TOK_PER_WARP * WARPS;  // 16
 
 struct TopkArgs {
+  const float* partials;  // [nsplit, T, E] fp32 partial logits (nsplit = 1: the logits themselves)
+  int nsplit;
+  long long split_stride;
+  const float* bias;      // [E] or NULL, added after the partial sums
+  float* logits_out;      // [T,E] written when partials are not the logits themselves
   const float* logits;
   float* probs;     // opt
   int32_t* idx;
@@ -58,11 +63,18 @@ __global__ void __launch_bounds__(WARPS * 32) topk_kernel(TopkArgs a) {
     const int t = blockIdx.x * TOK_PER_BLOCK + warp * TOK_PER_WARP + tt;
     if (t >= a.T) break;  // warp-uniform
     float l[EPL], s[EPL];
-    const float* lr = a.logits + (long long)t * a.E;
 #pragma unroll
     for (int i = 0; i < EPL; ++i) {
       const int e = lane + 32 * i;
-      l[i] = (e < a.E) ? lr[e] : -INFINITY;
+      if (e < a.E) {
+        float v = 0.f;
+        for (int q = 0; q < a.nsplit; ++q) v += a.partials[q * a.split_stride + (long long)t * a.E + e];
+        if (a.bias) v += a.bias[e];
+        if (a.logits_out) a.logits_out[(long long)t * a.E + e] = v;
+        l[i] = v;
+      } else {
+        l[i] = -INFINITY;
+      }
     }
     if (a.score == MOE_SCORE_SOFTMAX) {
       float m = -INFINITY;
@@ -170,6 +182,7 @@ __global__ void __launch_bounds__(512) finalize_kernel(const int* hist, const fl
   if (e < E) {
     int c = 0;
     float P = 0.f;
+#pragma unroll 8
     for (int b = 0; b < nblk; ++b) {
       c += hist[(long long)b * E + e];
       if (pblk) P += pblk[(long long)b * E + e];
@@ -205,13 +218,27 @@ int check_cfg(const moe_config* c) {
   return MOE_OK;
 }
 
-size_t router_ws(const moe_config* c) {
-  const size_t nblk = (c->T + router::TOK_PER_BLOCK - 1) / router::TOK_PER_BLOCK;
-  return ws_round(nblk * c->E * sizeof(int)) + ws_round(nblk * c->E * sizeof(float));
+// K slices of the logits GEMM: enough CTAs to fill the GPU (tiles x slices >= SMs),
+// each slice at least 4 k-blocks of 64, the slices dividing the k-blocks evenly.
+static int router_ksplit(const moe_config* c, int nsm) {
+  const int bn = c->E <= 128 ? 128 : 256;
+  const int tiles = ((c->T + 127) / 128) * ((c->E + bn - 1) / bn);
+  const int kb = (c->H + 63) / 64;
+  int s = 1;
+  while (tiles * s < nsm && kb % (2 * s) == 0 && kb / (2 * s) >= 4) s *= 2;
+  return s;
 }
 
-// Router logits on the tensor cores: [T,H] x [E,H]^T -> fp32 [T,E] (+ bias).
-int router_logits(const moe_config* c, const void* x, const void* W_r, const float* bias, float* logits,
+size_t router_ws(const moe_config* c) {
+  const size_t nblk = (c->T + router::TOK_PER_BLOCK - 1) / router::TOK_PER_BLOCK;
+  const size_t ns = router_ksplit(c, 148 * 2);  // upper bound for any SM count <= 296
+  return ws_round(nblk * c->E * sizeof(int)) + ws_round(nblk * c->E * sizeof(float)) +
+         ws_round(ns * (size_t)c->T * c->E * sizeof(float));
+}
+
+// Router logits on the tensor cores: [T,H] x [E,H]^T -> fp32 partial sums over `ns`
+// slices of H, [ns, T, E] (summed, plus the bias, by the top-k kernel).
+int router_logits(const moe_config* c, const void* x, const void* W_r, float* partials, int ns,
                   cudaStream_t st) {
   gg::Params p{};
   const uint32_t bn = c->E <= 128 ? 128 : 256;
@@ -227,11 +254,13 @@ int router_logits(const moe_config* c, const void* x, const void* W_r, const flo
   p.G = 1;
   p.offsets = nullptr;
   p.b_group_rows = 0;
-  p.C = logits;
+  p.C = partials;
   p.ldc = c->E;
-  p.bias = bias;
+  p.bias = nullptr;
+  p.ksplit = ns;
+  p.c_split_stride = (long long)c->T * c->E;
   p.status = moe_host::device_status_ptr();
-  const int tiles = ((c->T + 127) / 128) * ((c->E + bn - 1) / bn);
+  const int tiles = ((c->T + 127) / 128) * ((c->E + bn - 1) / bn) * ns;
   if (bn == 128) return gg::launch<gg::Cfg<128, false, false, gg::EPI_F32, gg::GROUP_NONE, gg::B_SINGLE>>(p, tiles, st);
   return gg::launch<gg::Cfg<256, false, false, gg::EPI_F32, gg::GROUP_NONE, gg::B_SINGLE>>(p, tiles, st);
 }
@@ -248,12 +277,25 @@ int router_topk(const moe_config* c, const void* x, const void* W_r, const float
   if (!aligned16(logits)) return MOE_ERR_ALIGNMENT;
   const size_t need = router_ws(c);
   if (!ws || ws_bytes < need) return MOE_ERR_WORKSPACE;
-  if (!logits_in) {
-    rc = router_logits(c, x, W_r, bias, logits, st);
-    if (rc) return rc;
-  }
   const int nblk = (c->T + router::TOK_PER_BLOCK - 1) / router::TOK_PER_BLOCK;
+  uint8_t* part = static_cast<uint8_t*>(ws) + ws_round((size_t)nblk * c->E * sizeof(int)) +
+                  ws_round((size_t)nblk * c->E * sizeof(float));
   router::TopkArgs a;
+  if (!logits_in) {
+    const int ns = router_ksplit(c, moe_host::num_sms());
+    rc = router_logits(c, x, W_r, reinterpret_cast<float*>(part), ns, st);
+    if (rc) return rc;
+    a.partials = reinterpret_cast<float*>(part);
+    a.nsplit = ns;
+    a.bias = bias;
+    a.logits_out = logits;
+  } else {
+    a.partials = logits;
+    a.nsplit = 1;
+    a.bias = nullptr;
+    a.logits_out = nullptr;
+  }
+  a.split_stride = (long long)c->T * c->E;
   a.logits = logits;
   a.probs = probs;
   a.idx = idx;
