@@ -52,6 +52,24 @@ def peaks():
     return d
 
 
+METRIC = "MoE-layer tokens/s (grouped-GEMM TFLOP/s as fraction of B200 peak in roofline), 1 GPU per replica"
+DATA = "synthetic (seeded; x~N(0,1), weights~N(0,0.02^2), bf16)"
+
+
+def workload_config(wl, ws):
+    return {"workload": f"{wl.name}: {'fwd+bwd' if wl.bwd else 'fwd'} T={wl.T} H={wl.H} E={wl.E} k={wl.k} "
+                        f"F={wl.F}{' +1 shared' if wl.S else ''} {wl.score} {wl.dtype}",
+            "T": wl.T, "H": wl.H, "E": wl.E, "k": wl.k, "F": wl.F, "shared": wl.S,
+            "parallelism": f"replicas x{ws} (no data-path collective)",
+            "l2": (f"inputs larger than L2 (expert weights {wl.expert_weight_bytes() / 1e9:.1f} GB vs 126 MB), "
+                   "no flush" if wl.expert_weight_bytes() > 126e6 else "weights fit in L2 (parity-size case)")}
+
+
+def aggregate_tokens_per_s(tokens_per_rank, ws, ms_max):
+    """Whole-job throughput: every rank's tokens over the slowest rank's step time."""
+    return round(tokens_per_rank * ws / (ms_max * 1e-3), 1)
+
+
 # ------------------------------------------------------------------ distributed plumbing
 
 def dist_setup(n_gpus):
@@ -423,8 +441,8 @@ def run_ours(args, rank, ws):
     assert moe.moe_get_device_status() == 0
 
     line = {
-        "metric": "MoE-layer tokens/s (grouped-GEMM TFLOP/s as fraction of B200 peak in roofline), 1 GPU per replica",
-        "value": round(wl.T * ws / (ms * 1e-3), 1),
+        "metric": METRIC,
+        "value": aggregate_tokens_per_s(wl.T, ws, ms),
         "unit": "tokens/s",
         "n_gpus": ws,
         "steps": args.steps,
@@ -434,15 +452,11 @@ def run_ours(args, rank, ws):
         "scaling": "weak",
         "vs_baseline": None,
         "dtype": "mxfp8" if wl.dtype == "mxfp8" else "bf16",
-        "data": "synthetic (seeded; x~N(0,1), weights~N(0,0.02^2), bf16)",
-        "config": {"workload": f"{wl.name}: {'fwd+bwd' if wl.bwd else 'fwd'} T={wl.T} H={wl.H} E={wl.E} k={wl.k} "
-                               f"F={wl.F}{' +1 shared' if wl.S else ''} {wl.score} {wl.dtype}",
-                   "T": wl.T, "H": wl.H, "E": wl.E, "k": wl.k, "F": wl.F, "shared": wl.S,
-                   "parallelism": f"replicas x{ws} (no data-path collective)",
-                   "l2": "inputs larger than L2 (weights >= 2.8 GB vs 126 MB), no flush"},
+        "data": DATA,
+        "config": workload_config(wl, ws),
         "roofline": roof,
         "kernels": kernels,
-        "e2e": {"value": round(wl.T * ws / (e2e_ms * 1e-3), 1), "unit": "tokens/s", "ms_per_step": round(e2e_ms, 4),
+        "e2e": {"value": aggregate_tokens_per_s(wl.T, ws, e2e_ms), "unit": "tokens/s", "ms_per_step": round(e2e_ms, 4),
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "api": "moe_layer_fwd" +
                 ("+moe_layer_bwd" if wl.bwd else "")},
         "gpu_launches": L.launches_per_step() * args.steps,
@@ -451,34 +465,72 @@ def run_ours(args, rank, ws):
     return line, L
 
 
-def cpu_baseline(wl, budget_s=12.0, max_tok=256, seed=0):
-    """Time the oracle (as it stands) on a bounded sample of the workload's tokens."""
-    import oracle
-    oracle.build()
-    # the sample's inputs on the host: x rows, the router, and every expert (tokens may pick any)
-    d = make_inputs(wl, device="cuda" if torch.cuda.is_available() else "cpu", seed=seed)
-    h = {k: (v.cpu() if torch.is_tensor(v) else v) for k, v in d.items()}
-    del d
-    mxw = None
-    if wl.dtype == "mxfp8":
-        mxw = {n: oracle.mxfp8_quantize(h[n]) for n in ["W_g", "W_u", "W_d"] + (["W_gs", "W_us", "W_ds"] if wl.S
-                                                                              else [])}
+class OracleTimer:
+    """Times the oracle (as it stands) on a bounded sample of a workload's tokens on the host."""
 
-    def run(n):
+    def __init__(self, wl, seed=0):
+        import oracle
+        oracle.build()
+        self.oracle = oracle
+        self.wl = wl
+        # the sample's inputs on the host: x rows, the router, and every expert (tokens may pick any)
+        d = make_inputs(wl, device="cuda" if torch.cuda.is_available() else "cpu", seed=seed)
+        self.h = {k: (v.cpu() if torch.is_tensor(v) else v) for k, v in d.items()}
+        del d
+        self.mxw = None
+        if wl.dtype == "mxfp8":
+            names = ["W_g", "W_u", "W_d"] + (["W_gs", "W_us", "W_ds"] if wl.S else [])
+            self.mxw = {n: oracle.mxfp8_quantize(self.h[n]) for n in names}
+
+    def run(self, n):
+        """Seconds the oracle's layer forward takes on the first n tokens."""
         toks = torch.arange(n, dtype=torch.int32)
+        sub = dict(self.h)
+        sub["x"] = self.h["x"][:n].contiguous()
         t0 = time.perf_counter()
-        sub = dict(h)
-        sub["x"] = h["x"][:n].contiguous()
-        wls = wl.with_(T=n)
-        oracle.layer_fwd(wls, sub, toks=toks, mx_weights=mxw)
+        self.oracle.layer_fwd(self.wl.with_(T=n), sub, toks=toks, mx_weights=self.mxw)
         return time.perf_counter() - t0
 
-    t1 = run(2)
-    n = int(max(2, min(max_tok, budget_s / max(t1 / 2, 1e-6))))
-    t = run(n)
-    return {"value": round(n / t, 3), "unit": "tokens/s", "cores": oracle.nthreads(), "kind": "oracle",
-            "sample": f"{n} of {wl.T} tokens of the {wl.name} layer forward (router + top-k + experts), "
-                      f"{t:.1f} s on the host"}, n, t
+    def sample_size(self, budget_s, max_tok):
+        t1 = self.run(2)
+        return int(max(2, min(max_tok, self.wl.T, budget_s / max(t1 / 2, 1e-6))))
+
+    def describe(self, n, t, value):
+        return {"value": value, "unit": "tokens/s", "cores": self.oracle.nthreads(), "kind": "oracle",
+                "sample": f"{n} of {self.wl.T} tokens of the {self.wl.name} layer forward (router + top-k + "
+                          f"experts), {t:.2f} s on the host per sample"}
+
+
+def cpu_baseline(wl, budget_s=12.0, max_tok=256, seed=0):
+    ot = OracleTimer(wl, seed)
+    n = ot.sample_size(budget_s, max_tok)
+    t = ot.run(n)
+    return ot.describe(n, t, round(n / t, 3)), n, t
+
+
+def run_reference(args, rank, ws):
+    """The oracle on the host cores: each step times a bounded sample of the workload's tokens,
+    sized so that warm-up plus timed steps stay within a few minutes."""
+    if rank != 0:
+        return None
+    wl = WORKLOADS[args.workload]
+    ot = OracleTimer(wl, seed=0)
+    budget = max(0.05, min(4.0, 150.0 / (args.warmup + args.steps)))
+    n = ot.sample_size(budget, 256)
+    vals, tsum = [], 0.0
+    for i in range(args.warmup + args.steps):
+        t = ot.run(n)
+        if i >= args.warmup:
+            vals.append(t / n)
+            tsum += t
+    sec_per_tok = statistics.mean(vals)
+    v = round(1.0 / sec_per_tok, 3)
+    return {"impl": "reference", "metric": METRIC, "value": v, "unit": "tokens/s", "n_gpus": ws,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(sec_per_tok * wl.T * 1e3, 1),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": DATA, "config": workload_config(wl, ws),
+            "cpu_baseline": ot.describe(n, tsum / args.steps, v),
+            "e2e": {"value": v, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
 
 
 def main():
@@ -494,25 +546,8 @@ def main():
     rank, ws = dist_setup(args.gpus)
     wl = WORKLOADS[args.workload]
     if args.impl == "reference":
+        line = run_reference(args, rank, ws)
         if rank == 0:
-            vals = []
-            info = None
-            for i in range(args.warmup + args.steps):
-                info, n, t = cpu_baseline(wl, budget_s=4.0, max_tok=64, seed=0)
-                if i >= args.warmup:
-                    vals.append(t / n)
-            sec_per_tok = statistics.mean(vals)
-            v = round(1.0 / sec_per_tok, 3)
-            info["value"] = v
-            line = {"impl": "reference", "metric": "MoE-layer tokens/s (grouped-GEMM TFLOP/s as fraction of B200 "
-                                                   "peak in roofline), 1 GPU per replica",
-                    "value": v, "unit": "tokens/s", "n_gpus": 1, "steps": args.steps, "warmup": args.warmup,
-                    "ms_per_step": round(sec_per_tok * wl.T * 1e3, 1), "higher_is_better": True,
-                    "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-                    "config": {"workload": f"{wl.name} (oracle, sampled tokens)", "T": wl.T, "H": wl.H, "E": wl.E,
-                               "k": wl.k, "F": wl.F},
-                    "cpu_baseline": info,
-                    "e2e": {"value": v, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
             print(json.dumps(line), flush=True)
         dist_done(ws)
         return

@@ -58,6 +58,11 @@ class Workload:
         """Algorithmic expert FLOPs of one forward pass (routed + shared)."""
         return 6.0 * self.H * self.F * (self.T * self.k + self.T * self.S)
 
+    def expert_weight_bytes(self) -> float:
+        """Bytes of the routed and shared expert weights (bf16, or fp8 + 1/32 scale bytes)."""
+        per = 1.0 + 1.0 / 32 if self.dtype == "mxfp8" else 2.0
+        return 3.0 * self.H * self.F * (self.E + self.S) * per
+
     def router_flops(self) -> float:
         return 2.0 * self.T * self.H * self.E
 

@@ -1,0 +1,78 @@
+"""Replica plumbing of bench.py on CPU: world size 2 over gloo.
+
+The layer shards as independent replicas (each rank its own tokens, no
+collective in the data path); what crosses ranks is only the timing: a
+barrier and the max of the step time over ranks. These tests run that
+plumbing with two gloo processes, and the reference arm under torchrun,
+where rank 0 alone times the oracle and prints the single JSON line.
+"""
+import json
+import os
+import socket
+import subprocess
+import sys
+
+import torch.multiprocessing as mp
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _free_port():
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
+
+
+def _worker(rank, ws, port, q):
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port), RANK=str(rank), WORLD_SIZE=str(ws),
+                      LOCAL_RANK=str(rank))
+    sys.path.insert(0, ROOT)
+    import bench
+    r, w = bench.dist_setup(ws)
+    bench.barrier(w)
+    ms = [3.0, 5.0][r]  # rank 1 is the slower replica
+    m = bench.max_over_ranks(ms, w)
+    v = bench.aggregate_tokens_per_s(1000, w, m)
+    bench.barrier(w)
+    bench.dist_done(w)
+    q.put((r, w, m, v))
+
+
+def test_max_over_ranks_and_aggregate_gloo():
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_worker, args=(r, 2, port, q)) for r in range(2)]
+    for p in procs:
+        p.start()
+    for p in procs:
+        p.join(120)
+        assert p.exitcode == 0
+    res = sorted(q.get(timeout=10) for _ in range(2))
+    for r, w, m, v in res:
+        assert w == 2
+        assert m == 5.0  # every rank sees the slowest rank's time
+        assert v == 2 * 1000 / 5e-3  # both replicas' tokens over the slowest step
+
+
+def test_aggregate_single_rank():
+    sys.path.insert(0, ROOT)
+    import bench
+    assert bench.aggregate_tokens_per_s(4096, 1, 2.0) == 4096 / 2e-3
+    assert bench.max_over_ranks(1.25, 1) == 1.25
+
+
+def test_reference_arm_under_torchrun_two_ranks():
+    port = _free_port()
+    cmd = [sys.executable, "-m", "torch.distributed.run", "--nnodes=1", "--nproc-per-node", "2", "--master-addr",
+           "127.0.0.1", "--master-port", str(port), "bench.py", "--impl", "reference", "--workload", "tiny",
+           "--gpus", "2", "--steps", "2", "--warmup", "3"]
+    env = dict(os.environ, CUDA_VISIBLE_DEVICES="")
+    r = subprocess.run(cmd, cwd=ROOT, env=env, capture_output=True, text=True, timeout=600)
+    assert r.returncode == 0, r.stderr[-2000:]
+    lines = [x for x in r.stdout.splitlines() if x.startswith("{")]
+    assert len(lines) == 1  # rank 0 alone prints
+    d = json.loads(lines[0])
+    assert d["impl"] == "reference" and d["n_gpus"] == 2 and d["value"] > 0
+    assert d["cpu_baseline"]["kind"] == "oracle"
+    assert d["e2e"]["h2d_bytes_per_step"] == 0
