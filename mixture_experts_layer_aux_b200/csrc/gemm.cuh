@@ -34,7 +34,6 @@ namespace gg {
 
 constexpr int BM = 128;
 constexpr int BK = 64;  // bf16 elements of K per stage (one 128-byte swizzle row)
-constexpr int NUM_THREADS = 192;
 constexpr int MAX_G = 512;
 
 enum Epi : int {
@@ -93,9 +92,14 @@ struct Cfg {
   static constexpr int TMEM_COLS = 2 * BN;
   static constexpr int N_STEP = (BMODE == B_SPLIT_N) ? BN / 2 : BN;  // output columns per tile
   static constexpr int BAR_BYTES = 1024;
-  // bf16 epilogue staging: per epilogue warp 32 rows x (128 + 16) bytes (64 columns at a time)
-  static constexpr int STG_ROW = 144;
-  static constexpr int STG_BYTES = (EPI == EPI_BF16) ? 4 * 32 * STG_ROW : 0;
+  // Epilogue warps: two per TMEM lane quadrant (each takes half of the columns), except the
+  // SwiGLU backward, whose staged loads and stores need the shared memory of four.
+  static constexpr int EPI_WARPS = (EPI == EPI_SWIGLU_BWD) ? 4 : 8;
+  static constexpr int NH = EPI_WARPS / 4;  // column slices per lane quadrant
+  static constexpr int NUM_THREADS = 64 + 32 * EPI_WARPS;
+  // staging: per epilogue warp 32 rows x (64 + 16) bytes (x2 for the SwiGLU backward's gate and up)
+  static constexpr int STG_ROW = 80;
+  static constexpr int STG_BYTES = EPI_WARPS * 32 * STG_ROW * (EPI == EPI_SWIGLU_BWD ? 2 : 1);
   static constexpr int SMEM_BYTES = 1024 + kStages * STAGE_BYTES + BAR_BYTES + 2 * (MAX_G + 1) * 4 + 128 + STG_BYTES;
   static_assert(BN == 128 || BN == 256, "BN");
   static_assert(!(BMODE == B_SPLIT_N && B_MN), "split-N is for K-major weights");
@@ -173,7 +177,7 @@ __device__ __forceinline__ Tile get_tile(const Params& p, int t, const int* s_of
 }
 
 template <class C>
-__global__ void __launch_bounds__(NUM_THREADS, 1) gemm_kernel(const __grid_constant__ Params p) {
+__global__ void __launch_bounds__(C::NUM_THREADS, 1) gemm_kernel(const __grid_constant__ Params p) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* stages = smem;
@@ -196,7 +200,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) gemm_kernel(const __grid_const
 
   // ---- group table: offsets and (GROUP_M) tile prefix sums, validated
   if (C::GROUP != GROUP_NONE) {
-    for (int i = threadIdx.x; i <= p.G; i += NUM_THREADS) s_off[i] = p.offsets[i];
+    for (int i = threadIdx.x; i <= p.G; i += C::NUM_THREADS) s_off[i] = p.offsets[i];
   }
   if (threadIdx.x == 0) {
     for (int i = 0; i < C::kStages; ++i) {
@@ -205,7 +209,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) gemm_kernel(const __grid_const
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(&tfull[i], 1);
-      mbar_init(&tempty[i], 4);
+      mbar_init(&tempty[i], C::EPI_WARPS);
     }
     mbar_init(drain, 1);
     *abort_flag = 0;
@@ -399,9 +403,13 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) gemm_kernel(const __grid_const
     }
     __syncwarp();
   } else {
-    // ======================= epilogue (warps 2..5)
+    // ======================= epilogue (warps 2 .. 2+EPI_WARPS-1)
+    // warp w reads TMEM lanes 32*(w%4) .. +31 (its quadrant q) and the columns of slice h
+    const int ew = warp - 2;
     const int q = warp & 3;
+    const int h = ew >> 2;
     const int row = q * 32 + lane;
+    uint8_t* stg = stg_area + ew * 32 * C::STG_ROW * (C::EPI == EPI_SWIGLU_BWD ? 2 : 1);
     int acc = 0;
     uint32_t acc_phase = 0;
     for (int t = blockIdx.x; t < total && !aborted; t += gridDim.x) {
@@ -415,44 +423,46 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) gemm_kernel(const __grid_const
       const bool valid = row < ti.m_valid;
       const bool empty_k = ti.kblocks == 0;  // GROUP_K group with no rows: result is exactly 0
       const long long orow = (long long)ti.row0 + row;
+      // staged store pattern: 4 warp stores, each 8 rows x 64 bytes
+      const int st_piece = lane & 3;
+      const int st_r0 = lane >> 2;
 
       if constexpr (C::EPI == EPI_SWIGLU_FWD) {
         constexpr int HALF = C::BN / 2;
+        constexpr int W = HALF / C::NH;  // output columns of this warp
         const float g = valid ? (p.row_gate ? p.row_gate[orow] : 1.f) : 0.f;
         __nv_bfloat16* out = reinterpret_cast<__nv_bfloat16*>(p.C) + orow * p.ldc + ti.n0;
         __nv_bfloat16* sv = p.C2 ? reinterpret_cast<__nv_bfloat16*>(p.C2) + orow * p.ldc2 + ti.n0 : nullptr;
 #pragma unroll 1
-        for (int c = 0; c < HALF / 32; ++c) {
+        for (int c = h * W; c < (h + 1) * W; c += 32) {
           float gv[32], uv[32];
-          tmem_ld32(tb + c * 32, gv);
-          tmem_ld32(tb + HALF + c * 32, uv);
+          tmem_ld32(tb + c, gv);
+          tmem_ld32(tb + HALF + c, uv);
           tmem_ld_wait();
           if (valid) {
             uint32_t pk[16];
 #pragma unroll
             for (int i = 0; i < 16; ++i)
               pk[i] = pack_bf16x2(g * silu_f(gv[2 * i]) * uv[2 * i], g * silu_f(gv[2 * i + 1]) * uv[2 * i + 1]);
-            uint4* o4 = reinterpret_cast<uint4*>(out + c * 32);
+            uint4* o4 = reinterpret_cast<uint4*>(out + c);
 #pragma unroll
             for (int i = 0; i < 4; ++i) o4[i] = make_uint4(pk[4 * i], pk[4 * i + 1], pk[4 * i + 2], pk[4 * i + 3]);
             if (sv) {
 #pragma unroll
               for (int i = 0; i < 16; ++i) pk[i] = pack_bf16x2(gv[2 * i], gv[2 * i + 1]);
-              uint4* s4 = reinterpret_cast<uint4*>(sv + c * 32);
+              uint4* s4 = reinterpret_cast<uint4*>(sv + c);
 #pragma unroll
               for (int i = 0; i < 4; ++i) s4[i] = make_uint4(pk[4 * i], pk[4 * i + 1], pk[4 * i + 2], pk[4 * i + 3]);
 #pragma unroll
               for (int i = 0; i < 16; ++i) pk[i] = pack_bf16x2(uv[2 * i], uv[2 * i + 1]);
-              uint4* u4 = reinterpret_cast<uint4*>(sv + p.F + c * 32);
+              uint4* u4 = reinterpret_cast<uint4*>(sv + p.F + c);
 #pragma unroll
               for (int i = 0; i < 4; ++i) u4[i] = make_uint4(pk[4 * i], pk[4 * i + 1], pk[4 * i + 2], pk[4 * i + 3]);
             }
           }
         }
       } else if constexpr (C::EPI == EPI_BF16) {
-        // Row q*32+i of the tile goes to out_base + (row0 + q*32 + i) * ld. Each warp converts
-        // 64 columns of its 32 rows to bf16, stages them in shared memory, and stores them
-        // back row-contiguously: one warp store = 4 rows x 128 bytes.
+        // 32 columns at a time: convert, stage in shared memory, store row-contiguously
         __nv_bfloat16* out_base;
         long long ld, rbase;
         if constexpr (C::GROUP == GROUP_K) {
@@ -470,98 +480,149 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) gemm_kernel(const __grid_const
           ld = p.ldc;
           out_base = reinterpret_cast<__nv_bfloat16*>(p.C);
         }
-        uint8_t* stg = stg_area + (warp - 2) * 32 * C::STG_ROW;
+        constexpr int W = C::BN / C::NH;
         const int nvalid = min(C::BN, p.N - ti.n0);
 #pragma unroll 1
-        for (int cg = 0; cg < C::BN / 64; ++cg) {
-          if (cg * 64 >= nvalid) break;  // warp-uniform
-          float v[64];
+        for (int c = h * W; c < (h + 1) * W; c += 32) {
+          if (c >= nvalid) break;  // warp-uniform
+          float v[32];
           if (!empty_k) {
-            tmem_ld32(tb + cg * 64, *reinterpret_cast<float(*)[32]>(&v[0]));
-            tmem_ld32(tb + cg * 64 + 32, *reinterpret_cast<float(*)[32]>(&v[32]));
+            tmem_ld32(tb + c, v);
             tmem_ld_wait();
           } else {
 #pragma unroll
-            for (int i = 0; i < 64; ++i) v[i] = 0.f;
+            for (int i = 0; i < 32; ++i) v[i] = 0.f;
           }
 #pragma unroll
-          for (int j = 0; j < 8; ++j)
+          for (int j = 0; j < 4; ++j)
             *reinterpret_cast<uint4*>(stg + lane * C::STG_ROW + 16 * j) =
                 make_uint4(pack_bf16x2(v[8 * j], v[8 * j + 1]), pack_bf16x2(v[8 * j + 2], v[8 * j + 3]),
                            pack_bf16x2(v[8 * j + 4], v[8 * j + 5]), pack_bf16x2(v[8 * j + 6], v[8 * j + 7]));
           __syncwarp();
-          const int ch = lane & 7;  // 16-byte chunk of the 128-byte row segment
 #pragma unroll
-          for (int i = 0; i < 8; ++i) {
-            const int r = 4 * i + (lane >> 3);  // row within this warp's 32
-            const int col = cg * 64 + ch * 8;
+          for (int i = 0; i < 4; ++i) {
+            const int r = 8 * i + st_r0;
+            const int col = c + st_piece * 8;
             if (q * 32 + r < ti.m_valid && col < nvalid) {
-              const uint4 val = *reinterpret_cast<const uint4*>(stg + r * C::STG_ROW + 16 * ch);
+              const uint4 val = *reinterpret_cast<const uint4*>(stg + r * C::STG_ROW + 16 * st_piece);
               *reinterpret_cast<uint4*>(out_base + (rbase + q * 32 + r) * ld + ti.n0 + col) = val;
             }
           }
           __syncwarp();
         }
       } else if constexpr (C::EPI == EPI_F32) {
-        float* out = reinterpret_cast<float*>(p.C) + ti.ks * p.c_split_stride + orow * p.ldc + ti.n0;
+        // 16 fp32 columns at a time through the staging buffer (64 bytes per row)
+        float* out = reinterpret_cast<float*>(p.C) + ti.ks * p.c_split_stride + (long long)ti.row0 * p.ldc + ti.n0;
+        constexpr int W = C::BN / C::NH;
         const int nvalid = min(C::BN, p.N - ti.n0);
 #pragma unroll 1
-        for (int c = 0; c < C::BN / 32; ++c) {
-          if (c * 32 >= nvalid) break;  // warp-uniform
+        for (int c = h * W; c < (h + 1) * W; c += 32) {
+          if (c >= nvalid) break;  // warp-uniform
           float v[32];
           if (!empty_k) {
-            tmem_ld32(tb + c * 32, v);
+            tmem_ld32(tb + c, v);
             tmem_ld_wait();
           } else {
 #pragma unroll
             for (int i = 0; i < 32; ++i) v[i] = 0.f;
           }
-          if (valid) {
+          if (p.bias) {
 #pragma unroll
-            for (int i = 0; i < 32; ++i) {
-              const int col = c * 32 + i;
-              if (col < nvalid) out[col] = v[i] + (p.bias ? p.bias[ti.n0 + col] : 0.f);
+            for (int i = 0; i < 32; ++i) v[i] += (c + i < nvalid) ? p.bias[ti.n0 + c + i] : 0.f;
+          }
+#pragma unroll
+          for (int half = 0; half < 2; ++half) {
+#pragma unroll
+            for (int j = 0; j < 4; ++j)
+              *reinterpret_cast<float4*>(stg + lane * C::STG_ROW + 16 * j) =
+                  make_float4(v[16 * half + 4 * j], v[16 * half + 4 * j + 1], v[16 * half + 4 * j + 2],
+                              v[16 * half + 4 * j + 3]);
+            __syncwarp();
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+              const int r = 8 * i + st_r0;
+              const int col = c + 16 * half + st_piece * 4;
+              if (q * 32 + r < ti.m_valid) {
+                const float4 val = *reinterpret_cast<const float4*>(stg + r * C::STG_ROW + 16 * st_piece);
+                float* dst = out + (long long)(q * 32 + r) * p.ldc + col;
+                if (col + 3 < nvalid && (p.ldc & 3) == 0) {
+                  *reinterpret_cast<float4*>(dst) = val;
+                } else {
+                  if (col < nvalid) dst[0] = val.x;
+                  if (col + 1 < nvalid) dst[1] = val.y;
+                  if (col + 2 < nvalid) dst[2] = val.z;
+                  if (col + 3 < nvalid) dst[3] = val.w;
+                }
+              }
             }
+            __syncwarp();
           }
         }
       } else if constexpr (C::EPI == EPI_SWIGLU_BWD) {
-        // acc = v = W_d^T dO for columns [n0, n0 + BN) of F
+        // acc = v = W_d^T dO for columns [n0, n0 + BN) of F. Per 32 columns: the saved gate/up
+        // of the warp's 32 rows are loaded row-contiguously into shared memory, each lane
+        // computes its row, and dgate/dup leave the same way.
         const float g = valid ? p.row_gate[orow] : 0.f;
-        const __nv_bfloat16* gu = p.gateup + orow * (2LL * p.F) + ti.n0;
-        __nv_bfloat16* dgu = reinterpret_cast<__nv_bfloat16*>(p.C) + orow * (2LL * p.F) + ti.n0;
+        const long long ld2 = 2LL * p.F;
+        uint8_t* sG = stg;
+        uint8_t* sU = stg + 32 * C::STG_ROW;
+        __nv_bfloat16* dgu = reinterpret_cast<__nv_bfloat16*>(p.C);
         float part = 0.f;
 #pragma unroll 1
-        for (int c = 0; c < C::BN / 32; ++c) {
+        for (int c = 0; c < C::BN; c += 32) {
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            const int r = 8 * i + st_r0;
+            uint4 zg4 = make_uint4(0, 0, 0, 0), zu4 = make_uint4(0, 0, 0, 0);
+            if (q * 32 + r < ti.m_valid) {
+              const __nv_bfloat16* src = p.gateup + ((long long)ti.row0 + q * 32 + r) * ld2 + ti.n0 + c + 8 * st_piece;
+              zg4 = *reinterpret_cast<const uint4*>(src);
+              zu4 = *reinterpret_cast<const uint4*>(src + p.F);
+            }
+            *reinterpret_cast<uint4*>(sG + r * C::STG_ROW + 16 * st_piece) = zg4;
+            *reinterpret_cast<uint4*>(sU + r * C::STG_ROW + 16 * st_piece) = zu4;
+          }
           float v[32];
-          tmem_ld32(tb + c * 32, v);
+          tmem_ld32(tb + c, v);
           tmem_ld_wait();
-          if (valid) {
+          __syncwarp();
 #pragma unroll
-            for (int i8 = 0; i8 < 4; ++i8) {
-              float zg[8], zu[8];
-              unpack_bf16x8(*reinterpret_cast<const uint4*>(gu + c * 32 + i8 * 8), zg);
-              unpack_bf16x8(*reinterpret_cast<const uint4*>(gu + p.F + c * 32 + i8 * 8), zu);
-              uint32_t pg[4], pu[4];
+          for (int j = 0; j < 4; ++j) {
+            float zg[8], zu[8];
+            unpack_bf16x8(*reinterpret_cast<const uint4*>(sG + lane * C::STG_ROW + 16 * j), zg);
+            unpack_bf16x8(*reinterpret_cast<const uint4*>(sU + lane * C::STG_ROW + 16 * j), zu);
+            uint32_t pg[4], pu[4];
 #pragma unroll
-              for (int i = 0; i < 8; i += 2) {
-                float dgv[2], duv[2];
+            for (int i = 0; i < 8; i += 2) {
+              float dgv[2], duv[2];
 #pragma unroll
-                for (int h = 0; h < 2; ++h) {
-                  const float z = zg[i + h], u = zu[i + h], vv = v[i8 * 8 + i + h];
-                  const float s = sigmoid_f(z);
-                  const float sl = z * s;
-                  part += vv * sl * u;
-                  const float da = g * vv;
-                  dgv[h] = da * u * s * (1.f + z * (1.f - s));
-                  duv[h] = da * sl;
-                }
-                pg[i / 2] = pack_bf16x2(dgv[0], dgv[1]);
-                pu[i / 2] = pack_bf16x2(duv[0], duv[1]);
+              for (int hh = 0; hh < 2; ++hh) {
+                const float z = zg[i + hh], u = zu[i + hh], vv = v[8 * j + i + hh];
+                const float sg = sigmoid_f(z);
+                const float sl = z * sg;
+                part += vv * sl * u;
+                const float da = g * vv;
+                dgv[hh] = da * u * sg * (1.f + z * (1.f - sg));
+                duv[hh] = da * sl;
               }
-              *reinterpret_cast<uint4*>(dgu + c * 32 + i8 * 8) = make_uint4(pg[0], pg[1], pg[2], pg[3]);
-              *reinterpret_cast<uint4*>(dgu + p.F + c * 32 + i8 * 8) = make_uint4(pu[0], pu[1], pu[2], pu[3]);
+              pg[i / 2] = pack_bf16x2(dgv[0], dgv[1]);
+              pu[i / 2] = pack_bf16x2(duv[0], duv[1]);
+            }
+            *reinterpret_cast<uint4*>(sG + lane * C::STG_ROW + 16 * j) = make_uint4(pg[0], pg[1], pg[2], pg[3]);
+            *reinterpret_cast<uint4*>(sU + lane * C::STG_ROW + 16 * j) = make_uint4(pu[0], pu[1], pu[2], pu[3]);
+          }
+          __syncwarp();
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            const int r = 8 * i + st_r0;
+            if (q * 32 + r < ti.m_valid) {
+              __nv_bfloat16* dst = dgu + ((long long)ti.row0 + q * 32 + r) * ld2 + ti.n0 + c + 8 * st_piece;
+              *reinterpret_cast<uint4*>(dst) = *reinterpret_cast<const uint4*>(sG + r * C::STG_ROW + 16 * st_piece);
+              *reinterpret_cast<uint4*>(dst + p.F) =
+                  *reinterpret_cast<const uint4*>(sU + r * C::STG_ROW + 16 * st_piece);
             }
           }
+          __syncwarp();
         }
         if (valid) p.dg_part[orow * (long long)(p.N / C::BN) + ti.n0 / C::BN] = part;
       }
@@ -594,7 +655,7 @@ int launch(const Params& p, int max_tiles, cudaStream_t stream) {
   }
   int grid = moe_host::num_sms();
   if (grid > max_tiles) grid = max_tiles;
-  kern<<<grid, NUM_THREADS, C::SMEM_BYTES, stream>>>(p);
+  kern<<<grid, C::NUM_THREADS, C::SMEM_BYTES, stream>>>(p);
   MOE_CHECK_LAUNCH();
   return MOE_OK;
 }

@@ -14,11 +14,24 @@
 //                    (MN-major, K rows [0,F) from W_g, [F,2F) from W_u).
 #include "common.cuh"
 #include "gemm.cuh"
+#include "gemm2.cuh"
 #include "layout.h"
+
+#include <cstdlib>
 
 namespace moe_impl {
 
 using gg::Cfg;
+
+// The SM-pair kernel (256-row tiles) pays off when experts are large: it
+// halves each SM's operand traffic per FLOP but pads each expert to a
+// multiple of 256 rows. Used when the average rows per group reach this
+// threshold (MOE_B200_PAIR_MIN_ROWS overrides it; a huge value disables it).
+static bool use_pair_kernel(int rows, int groups) {
+  long long thr = 768;
+  if (const char* e = std::getenv("MOE_B200_PAIR_MIN_ROWS")) thr = std::atoll(e);
+  return (long long)rows >= thr * (long long)groups;
+}
 
 static bool a16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
@@ -47,6 +60,10 @@ int gemm_gateup_bf16(int rows, int groups, int H, int F, const void* A, const vo
   p.row_gate = row_gate;
   p.F = F;
   p.status = moe_host::device_status_ptr();
+  if (use_pair_kernel(rows, groups)) {
+    const int pair_tiles = ((rows + 255) / 256 + groups) * (F / 128);
+    return gg2::launch<gg::EPI_SWIGLU_FWD, true>(p, pair_tiles, st);
+  }
   const int tiles = ((rows + 127) / 128 + groups) * (F / 128);
   return gg::launch<Cfg<256, false, false, gg::EPI_SWIGLU_FWD, gg::GROUP_M, gg::B_SPLIT_N>>(p, tiles, st);
 }
@@ -66,6 +83,10 @@ int gemm_down_bf16(int rows, int groups, int H, int F, const void* A, const void
   p.C = C;
   p.ldc = H;
   p.status = moe_host::device_status_ptr();
+  if (use_pair_kernel(rows, groups)) {
+    const int pair_tiles = ((rows + 255) / 256 + groups) * (H / 256);
+    return gg2::launch<gg::EPI_BF16, false>(p, pair_tiles, st);
+  }
   const int tiles = ((rows + 127) / 128 + groups) * (H / 256);
   return gg::launch<Cfg<256, false, false, gg::EPI_BF16, gg::GROUP_M, gg::B_SINGLE>>(p, tiles, st);
 }

@@ -173,30 +173,49 @@ __global__ void __launch_bounds__(WARPS * 32) topk_kernel(TopkArgs a) {
   }
 }
 
-// counts[e] = sum_b hist[b,e]; aux = E sum_e (counts_e / (T k)) (sum_b pblk[b,e] / T).
-__global__ void __launch_bounds__(512) finalize_kernel(const int* hist, const float* pblk, int nblk, int T, int E,
-                                                       int k, int32_t* counts, float* aux) {
-  __shared__ float red[512];
-  const int e = threadIdx.x;
-  float term = 0.f;
+// counts[e] = sum_b hist[b,e] and Psum[e] = sum_b pblk[b,e]: 32 experts per block, 32 threads
+// per expert each summing a fixed stride of blocks, then the 32 partials in order.
+__global__ void __launch_bounds__(1024) finalize_kernel(const int* hist, const float* pblk, int nblk, int E,
+                                                        int32_t* counts, float* psum) {
+  __shared__ int sc[32][33];
+  __shared__ float sp[32][33];
+  const int tx = threadIdx.x & 31, ty = threadIdx.x >> 5;
+  const int e = blockIdx.x * 32 + tx;
+  int c = 0;
+  float P = 0.f;
   if (e < E) {
-    int c = 0;
-    float P = 0.f;
-#pragma unroll 8
-    for (int b = 0; b < nblk; ++b) {
+    for (int b = ty; b < nblk; b += 32) {
       c += hist[(long long)b * E + e];
       if (pblk) P += pblk[(long long)b * E + e];
     }
-    if (counts) counts[e] = c;
-    term = ((float)c / ((float)T * (float)k)) * (P / (float)T);
   }
-  red[threadIdx.x] = term;
+  sc[ty][tx] = c;
+  sp[ty][tx] = P;
+  __syncthreads();
+  if (ty == 0 && e < E) {
+    int cs = 0;
+    float ps = 0.f;
+    for (int i = 0; i < 32; ++i) {
+      cs += sc[i][tx];
+      ps += sp[i][tx];
+    }
+    if (counts) counts[e] = cs;
+    if (psum) psum[e] = ps;
+  }
+}
+
+// aux = E * sum_e (counts_e / (T k)) * (Psum_e / T), summed by a fixed tree.
+__global__ void __launch_bounds__(512) aux_kernel(const int32_t* counts, const float* psum, int T, int E, int k,
+                                                  float* aux) {
+  __shared__ float red[512];
+  const int e = threadIdx.x;
+  red[e] = (e < E) ? ((float)counts[e] / ((float)T * (float)k)) * (psum[e] / (float)T) : 0.f;
   __syncthreads();
   for (int s = 256; s > 0; s >>= 1) {
-    if (threadIdx.x < s) red[threadIdx.x] += red[threadIdx.x + s];
+    if (e < s) red[e] += red[e + s];
     __syncthreads();
   }
-  if (threadIdx.x == 0 && aux) *aux = (float)E * red[0];
+  if (e == 0) *aux = (float)E * red[0];
 }
 
 }  // namespace router
@@ -233,7 +252,8 @@ size_t router_ws(const moe_config* c) {
   const size_t nblk = (c->T + router::TOK_PER_BLOCK - 1) / router::TOK_PER_BLOCK;
   const size_t ns = router_ksplit(c, 148 * 2);  // upper bound for any SM count <= 296
   return ws_round(nblk * c->E * sizeof(int)) + ws_round(nblk * c->E * sizeof(float)) +
-         ws_round(ns * (size_t)c->T * c->E * sizeof(float));
+         ws_round(ns * (size_t)c->T * c->E * sizeof(float)) + ws_round(c->E * sizeof(float)) +
+         ws_round(c->E * sizeof(int32_t));
 }
 
 // Router logits on the tensor cores: [T,H] x [E,H]^T -> fp32 partial sums over `ns`
@@ -280,6 +300,7 @@ int router_topk(const moe_config* c, const void* x, const void* W_r, const float
   const int nblk = (c->T + router::TOK_PER_BLOCK - 1) / router::TOK_PER_BLOCK;
   uint8_t* part = static_cast<uint8_t*>(ws) + ws_round((size_t)nblk * c->E * sizeof(int)) +
                   ws_round((size_t)nblk * c->E * sizeof(float));
+  uint8_t* psum_ws = part + ws_round((size_t)router_ksplit(c, 148 * 2) * c->T * c->E * sizeof(float));
   router::TopkArgs a;
   if (!logits_in) {
     const int ns = router_ksplit(c, moe_host::num_sms());
@@ -317,8 +338,15 @@ int router_topk(const moe_config* c, const void* x, const void* W_r, const float
   else router::topk_kernel<16><<<grid, block, smem, st>>>(a);
   MOE_CHECK_LAUNCH();
   if (counts || aux) {
-    router::finalize_kernel<<<1, 512, 0, st>>>(a.hist, aux ? a.pblk : nullptr, nblk, c->T, c->E, c->k, counts, aux);
+    // the aux path needs the counts; use the tail of the workspace when the caller does not want them
+    int32_t* cnt = counts ? counts : reinterpret_cast<int32_t*>(psum_ws + ws_round((size_t)c->E * sizeof(float)));
+    router::finalize_kernel<<<(c->E + 31) / 32, 1024, 0, st>>>(a.hist, aux ? a.pblk : nullptr, nblk, c->E, cnt,
+                                                               aux ? reinterpret_cast<float*>(psum_ws) : nullptr);
     MOE_CHECK_LAUNCH();
+    if (aux) {
+      router::aux_kernel<<<1, 512, 0, st>>>(cnt, reinterpret_cast<float*>(psum_ws), c->T, c->E, c->k, aux);
+      MOE_CHECK_LAUNCH();
+    }
   }
   return MOE_OK;
 }

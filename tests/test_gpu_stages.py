@@ -202,11 +202,23 @@ GEMM_CASES = [
     (200, 512, 4, 1, 256, 0, 0.95),   # one expert holds almost every row
     (100, 256, 16, 4, 384, 3, 0.0),   # F a multiple of 128 only
     (1000, 1024, 32, 8, 1536, 0, 0.3),
+    (2100, 512, 4, 2, 512, 1, 0.0),   # large experts (1400 rows): the SM-pair kernel's own regime
 ]
 
 
+@pytest.fixture(params=["auto", "pair", "single"])
+def fwd_kernel(request, monkeypatch):
+    """Run the forward GEMMs with the library's own kernel choice, or forced onto the
+    SM-pair (256-row tile) or the single-SM (128-row tile) kernel."""
+    if request.param == "pair":
+        monkeypatch.setenv("MOE_B200_PAIR_MIN_ROWS", "0")
+    elif request.param == "single":
+        monkeypatch.setenv("MOE_B200_PAIR_MIN_ROWS", str(1 << 40))
+    return request.param
+
+
 @pytest.mark.parametrize("T,H,E,k,F,zero,hot", GEMM_CASES)
-def test_grouped_gemm_fwd_matches_oracle(moe, oracle, T, H, E, k, F, zero, hot):
+def test_grouped_gemm_fwd_matches_oracle(moe, oracle, fwd_kernel, T, H, E, k, F, zero, hot):
     idx = random_routing(T, E, k, seed=T + F, zero_experts=zero, hot=hot)
     counts, offsets, _, _ = oracle.maps(idx, E)
     rows = T * k
