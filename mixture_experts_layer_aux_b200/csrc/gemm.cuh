@@ -350,21 +350,27 @@ __global__ void __launch_bounds__(C::NUM_THREADS, 1) gemm_kernel(const __grid_co
         tc_fence_after();
         uint8_t* sA = stages + stage * C::STAGE_BYTES;
         uint8_t* sB = sA + C::A_BYTES;
+        int kk_end = BK / 16;
         if constexpr (C::GROUP == GROUP_K) {
           if (kb == ti.kblocks - 1 && ti.klast < BK) {
-            // rows of K past the group's end belong to the next group: zero them.
-            // In the MN-major layout each K index is one 128-byte line of a
-            // 64-row box, so whole lines are cleared (swizzle-invariant).
-            const int nz = BK - ti.klast;
-            const int boxes = 2 + C::BN / 64;
-            for (int i = lane; i < boxes * nz * 8; i += 32) {
-              const int box = i / (nz * 8);
-              const int rem = i % (nz * 8);
-              const int r = ti.klast + rem / 8;
-              uint8_t* base = (box < 2) ? (sA + box * 64 * BK * 2) : (sB + (box - 2) * 64 * BK * 2);
-              *reinterpret_cast<uint4*>(base + r * 128 + (rem % 8) * 16) = make_uint4(0, 0, 0, 0);
+            // Rows of K past the group's end belong to the next group. K16 steps wholly
+            // past the end are not issued; the lines of the last partial K16 step past
+            // the end are zeroed. In the MN-major layout each K index is one 128-byte
+            // line of a 64-row box, so the lines [klast, kv) of a box are one
+            // contiguous, swizzle-invariant range.
+            const int kv = (ti.klast + 15) & ~15;
+            kk_end = kv / 16;
+            const int nbytes = (kv - ti.klast) * 128;
+            if (nbytes > 0) {
+#pragma unroll
+              for (int box = 0; box < 2 + C::BN / 64; ++box) {
+                uint8_t* base = ((box < 2) ? (sA + box * 64 * BK * 2) : (sB + (box - 2) * 64 * BK * 2)) +
+                                ti.klast * 128;
+                for (int i = 16 * lane; i < nbytes; i += 16 * 32)
+                  *reinterpret_cast<uint4*>(base + i) = make_uint4(0, 0, 0, 0);
+              }
+              fence_proxy_async_smem();
             }
-            fence_proxy_async_smem();
             __syncwarp();
           }
         }
@@ -372,6 +378,7 @@ __global__ void __launch_bounds__(C::NUM_THREADS, 1) gemm_kernel(const __grid_co
           const uint32_t a0 = smem_u32(sA), b0 = smem_u32(sB);
 #pragma unroll
           for (int kk = 0; kk < BK / 16; ++kk) {
+            if (kk >= kk_end) break;
             const uint64_t ad = C::A_MN ? smem_desc_sw128(a0 + kk * 2048, 64 * BK * 2, 1024)
                                         : smem_desc_sw128(a0 + kk * 32, 16, 1024);
             const uint64_t bd = C::B_MN ? smem_desc_sw128(b0 + kk * 2048, 64 * BK * 2, 1024)
