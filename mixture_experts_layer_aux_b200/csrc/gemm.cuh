@@ -85,16 +85,16 @@ struct Cfg {
   static constexpr int EPI = EPI_;
   static constexpr int GROUP = GROUP_;
   static constexpr int BMODE = BMODE_;
-  static constexpr int kStages = (BN == 256) ? 4 : 6;
+  // the SwiGLU backward's staging buffers take the room of a fourth stage
+  static constexpr int kStages = (BN == 256) ? (EPI == EPI_SWIGLU_BWD ? 3 : 4) : 6;
   static constexpr int A_BYTES = BM * BK * 2;
   static constexpr int B_BYTES = BN * BK * 2;
   static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
   static constexpr int TMEM_COLS = 2 * BN;
   static constexpr int N_STEP = (BMODE == B_SPLIT_N) ? BN / 2 : BN;  // output columns per tile
   static constexpr int BAR_BYTES = 1024;
-  // Epilogue warps: two per TMEM lane quadrant (each takes half of the columns), except the
-  // SwiGLU backward, whose staged loads and stores need the shared memory of four.
-  static constexpr int EPI_WARPS = (EPI == EPI_SWIGLU_BWD) ? 4 : 8;
+  // Epilogue warps: two per TMEM lane quadrant, each taking half of the columns.
+  static constexpr int EPI_WARPS = 8;
   static constexpr int NH = EPI_WARPS / 4;  // column slices per lane quadrant
   static constexpr int NUM_THREADS = 64 + 32 * EPI_WARPS;
   // staging: per epilogue warp 32 rows x (64 + 16) bytes (x2 for the SwiGLU backward's gate and up)
@@ -566,9 +566,11 @@ __global__ void __launch_bounds__(C::NUM_THREADS, 1) gemm_kernel(const __grid_co
           }
         }
       } else if constexpr (C::EPI == EPI_SWIGLU_BWD) {
-        // acc = v = W_d^T dO for columns [n0, n0 + BN) of F. Per 32 columns: the saved gate/up
-        // of the warp's 32 rows are loaded row-contiguously into shared memory, each lane
-        // computes its row, and dgate/dup leave the same way.
+        // acc = v = W_d^T dO for columns [n0, n0 + BN) of F; this warp takes the slice
+        // [n0 + h W, n0 + (h + 1) W). Per 32 columns: the saved gate/up of the warp's 32 rows
+        // are loaded row-contiguously into shared memory, each lane computes its row, and
+        // dgate/dup leave the same way. dg partial sums: one per row and W-wide slice.
+        constexpr int W = C::BN / C::NH;
         const float g = valid ? p.row_gate[orow] : 0.f;
         const long long ld2 = 2LL * p.F;
         uint8_t* sG = stg;
@@ -576,7 +578,7 @@ __global__ void __launch_bounds__(C::NUM_THREADS, 1) gemm_kernel(const __grid_co
         __nv_bfloat16* dgu = reinterpret_cast<__nv_bfloat16*>(p.C);
         float part = 0.f;
 #pragma unroll 1
-        for (int c = 0; c < C::BN; c += 32) {
+        for (int c = h * W; c < (h + 1) * W; c += 32) {
 #pragma unroll
           for (int i = 0; i < 4; ++i) {
             const int r = 8 * i + st_r0;
@@ -631,7 +633,7 @@ __global__ void __launch_bounds__(C::NUM_THREADS, 1) gemm_kernel(const __grid_co
           }
           __syncwarp();
         }
-        if (valid) p.dg_part[orow * (long long)(p.N / C::BN) + ti.n0 / C::BN] = part;
+        if (valid) p.dg_part[orow * (long long)(p.N / W) + (ti.n0 + h * W) / W] = part;
       }
       tc_fence_before();
       __syncwarp();

@@ -7,20 +7,23 @@
 // the block format is OCP MX v1.0.
 //
 // Layout of one stage (128 of K = 128 bytes of E4M3 per row):
-//   A tile 128 x 128 B and B tile 256 x 128 B, TMA, 128-byte swizzle;
-//   scale words: per row one uint32 holding the 4 UE8M0 bytes of its four
-//   32-wide K blocks (byte j = block j), gathered by a loader warp with
-//   asynchronous 4-byte copies straight from the natural [rows, K/32] scale
-//   layout into the order that tcgen05.cp 32x128b.warpx4 expects: the 16
-//   bytes of lane l hold rows l, l+32, l+64, l+96 (a 512-byte chunk per 128
-//   rows); the copies' completion is an arrival on the stage's barrier.
-// MMA: per stage, tcgen05.cp copies the scale chunks into TMEM (SFA 4
-// columns, SFB 8 columns, two slots alternating by stage), then four
-// M128 N256 K32 MMAs select scale byte j through the instruction descriptor.
-// TMEM: one 256-column fp32 accumulator (the scale slots take the rest of the
-// 512 columns); eight epilogue warps (two per lane quadrant, 128 columns
-// each) first copy their accumulator columns into registers and release TMEM,
-// so the next tile's MMAs run while they finish the element-wise work.
+//   A tile 128 x 128 B and B tile 256 x 128 B, TMA, 128-byte swizzle.
+// Scales travel in batches of SB = 4 k-blocks on a ring of their own: per row
+//   the loader warp reads the SB scale words of the batch (one 16-byte load
+//   from the natural [rows, K/32] layout; word = the 4 UE8M0 bytes of one
+//   k-block, byte j = 32-wide block j) and stores them into the order that
+//   tcgen05.cp 32x128b.warpx4 expects, one 512-byte chunk per 128 rows and
+//   k-block: the 16 bytes of lane l hold rows l, l+32, l+64, l+96. The loader
+//   fences the generic-proxy stores for the async proxy before it arrives on
+//   the batch's barrier, so the MMA thread does no fence of its own.
+// MMA: per batch, tcgen05.cp copies the batch's chunks into one of two TMEM
+// scale slots (SFA 4 columns and SFB 8 columns per k-block) and a commit frees
+// the batch's shared memory; per k-block, four M128 N256 K32 MMAs select scale
+// byte j through the instruction descriptor.
+// TMEM: one 256-column fp32 accumulator and the two scale slots; eight
+// epilogue warps (two per lane quadrant, 128 columns each) first copy their
+// accumulator columns into registers and release TMEM, so the next tile's MMAs
+// run while they finish the element-wise work.
 // Roles: warp 0 TMA producer, warp 1 MMA issuer (+ TMEM owner), warp 2 scale
 // loader, warps 3..10 epilogue. All waits are bounded like gemm.cuh.
 #pragma once
@@ -39,16 +42,21 @@ constexpr int NUM_THREADS = 11 * 32;
 constexpr int MAX_G = 512;
 constexpr int A_BYTES = BM * BK;        // 16 KB
 constexpr int B_BYTES = BN * BK;        // 32 KB
-constexpr int SFA_BYTES = 512;
+constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
+constexpr int TX_BYTES = STAGE_BYTES;
+constexpr int SFA_BYTES = 512;          // scale chunk of one k-block: 128 rows x 4 bytes
 constexpr int SFB_BYTES = 1024;
-constexpr int STAGE_BYTES = 51200;      // A + B + SFA + SFB, padded to 1024
-constexpr int TX_BYTES = A_BYTES + B_BYTES;
+constexpr int SF_KB_BYTES = SFA_BYTES + SFB_BYTES;
+constexpr int SB = 4;                   // k-blocks per scale batch
+constexpr int kSfBufs = 3;              // scale batches in shared memory
+constexpr int SF_BATCH_BYTES = SB * SF_KB_BYTES;
 constexpr int TMEM_COLS = 512;
-constexpr int SFA_COL = 256;            // + 4 * slot
-constexpr int SFB_COL = 264;            // + 8 * slot
+constexpr int SF_COL = 256;             // TMEM scale slots after the accumulator
+constexpr int SF_SLOT_COLS = SB * 12;   // per k-block: SFA 4 columns, SFB 8 columns
 constexpr int BAR_BYTES = 1024;
-constexpr int SMEM_BYTES = 1024 + kStages * STAGE_BYTES + BAR_BYTES + 2 * (MAX_G + 1) * 4;
-static_assert(A_BYTES + B_BYTES + SFA_BYTES + SFB_BYTES <= STAGE_BYTES, "stage");
+constexpr int SMEM_BYTES =
+    1024 + kStages * STAGE_BYTES + kSfBufs * SF_BATCH_BYTES + BAR_BYTES + 2 * (MAX_G + 1) * 4;
+static_assert(SF_COL + 2 * SF_SLOT_COLS <= TMEM_COLS, "tmem");
 static_assert(SMEM_BYTES <= 232448, "smem");
 
 enum Epi : int {
@@ -109,17 +117,6 @@ MOE_DEV void mma_mxf8(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t 
       : "memory");
 }
 
-// 4-byte asynchronous global -> shared copy; src_bytes 0 writes zeros.
-MOE_DEV void cp_async_4(void* smem_dst, const void* gsrc, uint32_t src_bytes) {
-  asm volatile("cp.async.ca.shared.global [%0], [%1], 4, %2;" ::"r"(smem_u32(smem_dst)), "l"(gsrc), "r"(src_bytes)
-               : "memory");
-}
-// Arrive on `bar` once all cp.async copies of this thread so far have landed
-// (counts as one of the barrier's expected arrivals).
-MOE_DEV void cp_async_arrive_noinc(uint64_t* bar) {
-  asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(smem_u32(bar)) : "memory");
-}
-
 // smem (32 rows x 16 bytes, no swizzle) -> TMEM lanes 0..31 of every quadrant, 4 columns.
 MOE_DEV void tmem_cp_32x128b_x4(uint32_t taddr, uint64_t sdesc) {
   asm volatile("tcgen05.cp.cta_group::1.32x128b.warpx4 [%0], %1;" ::"r"(taddr), "l"(sdesc) : "memory");
@@ -168,10 +165,13 @@ template <int EPI, bool SPLIT_N>
 __global__ void __launch_bounds__(NUM_THREADS, 1) gemm_mx_kernel(const __grid_constant__ Params p) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint8_t* bar_area = smem + kStages * STAGE_BYTES;
+  uint8_t* sf_area = smem + kStages * STAGE_BYTES;
+  uint8_t* bar_area = sf_area + kSfBufs * SF_BATCH_BYTES;
   uint64_t* full = reinterpret_cast<uint64_t*>(bar_area);
   uint64_t* empty = full + kStages;
-  uint64_t* tfull = empty + kStages;
+  uint64_t* sfull = empty + kStages;
+  uint64_t* sempty = sfull + kSfBufs;
+  uint64_t* tfull = sempty + kSfBufs;
   uint64_t* tempty = tfull + 1;
   uint64_t* drain = tempty + 1;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
@@ -184,8 +184,12 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) gemm_mx_kernel(const __grid_co
   for (int i = threadIdx.x; i <= p.G; i += NUM_THREADS) s_off[i] = p.offsets[i];
   if (threadIdx.x == 0) {
     for (int i = 0; i < kStages; ++i) {
-      mbar_init(&full[i], 33);  // TMA (expect_tx) + the scale loader's 32 lanes (cp.async)
+      mbar_init(&full[i], 1);
       mbar_init(&empty[i], 1);
+    }
+    for (int i = 0; i < kSfBufs; ++i) {
+      mbar_init(&sfull[i], 1);
+      mbar_init(&sempty[i], 1);
     }
     mbar_init(tfull, 1);
     mbar_init(tempty, 8);
@@ -268,54 +272,93 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) gemm_mx_kernel(const __grid_co
       }
     }
   } else if (warp == 2) {
-    // ======================= scale loader: natural [rows, K/32] bytes -> UTCCP chunk order
-    const int kw = p.K / 32;  // scale bytes per row
-    int stage = 0;
-    uint32_t phase = 0;
+    // ======================= scale loader: natural [rows, K/32] bytes -> UTCCP chunk order, SB k-blocks at a time
+    const int kw = p.K / 32;  // scale bytes per row (a multiple of 4)
+    const uint8_t* sfb1 = SPLIT_N ? p.sfb1 : p.sfb0;
+    // one 16-byte load per row and batch where every row start is 16-byte aligned
+    const bool v16 = (kw % 16) == 0 &&
+                     ((reinterpret_cast<uintptr_t>(p.sfa) | reinterpret_cast<uintptr_t>(p.sfb0) |
+                       reinterpret_cast<uintptr_t>(sfb1)) & 15u) == 0;
+    int sb = 0;
+    uint32_t sphase = 0;
     for (int t = blockIdx.x; t < total && !aborted; t += gridDim.x) {
       const Tile ti = get_tile(p, t, s_off, s_tstart, N_STEP);
       const long long brow = (long long)ti.g * p.b_group_rows + ti.n0;
-      for (int kb = 0; kb < KB; ++kb) {
+      for (int kb0 = 0; kb0 < KB; kb0 += SB) {
+        const int nb = min(SB, KB - kb0);
         if (!__all_sync(0xffffffffu,
-                        mbar_wait(&empty[stage], phase ^ 1, abort_flag, p.status, DEV_WAIT_TIMEOUT_PRODUCER))) {
+                        mbar_wait(&sempty[sb], sphase ^ 1, abort_flag, p.status, DEV_WAIT_TIMEOUT_PRODUCER))) {
           aborted = true;
           break;
         }
-        uint8_t* sSF = smem + stage * STAGE_BYTES + A_BYTES + B_BYTES;
-        // lane l: words of rows l, l+32, l+64, l+96 (A), the same for both 128-row halves of B
+        uint8_t* sf = sf_area + sb * SF_BATCH_BYTES;
+        // lane l: rows l, l+32, l+64, l+96 of A (i < 4), and of each 128-row half of B (i >= 4).
+        // All twelve rows' loads are issued before any is used, so their latencies overlap;
+        // rows past A's end read row 0 and are zeroed.
+        const uint8_t* src[12];
+        bool ok[12];
 #pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          const int r = ti.row0 + lane + 32 * i;
-          const bool ok = r < p.M;
-          cp_async_4(sSF + 16 * lane + 4 * i, p.sfa + (long long)(ok ? r : 0) * kw + 4 * kb, ok ? 4u : 0u);
-        }
-#pragma unroll
-        for (int i = 0; i < 8; ++i) {
+        for (int i = 0; i < 12; ++i) {
           const uint8_t* base;
           long long r;
-          if (SPLIT_N) {
-            base = i < 4 ? p.sfb0 : p.sfb1;
-            r = brow + lane + 32 * (i & 3);
+          ok[i] = true;
+          if (i < 4) {
+            base = p.sfa;
+            r = ti.row0 + lane + 32 * i;
+            ok[i] = r < p.M;
+            if (!ok[i]) r = 0;
           } else {
-            base = p.sfb0;
-            r = brow + lane + 32 * i;
+            const int ib = i - 4;
+            if (SPLIT_N) {
+              base = ib < 4 ? p.sfb0 : sfb1;
+              r = brow + lane + 32 * (ib & 3);
+            } else {
+              base = p.sfb0;
+              r = brow + lane + 32 * ib;
+            }
           }
-          cp_async_4(sSF + SFA_BYTES + (i >> 2) * 512 + 16 * lane + 4 * (i & 3), base + r * kw + 4 * kb, 4u);
+          src[i] = base + r * kw + 4 * kb0;
         }
-        cp_async_arrive_noinc(&full[stage]);
-        if (++stage == kStages) {
-          stage = 0;
-          phase ^= 1;
+        uint32_t w[12][SB];
+        if (v16 && nb == SB) {
+#pragma unroll
+          for (int i = 0; i < 12; ++i) {
+            const uint4 u = __ldg(reinterpret_cast<const uint4*>(src[i]));
+            w[i][0] = u.x;
+            w[i][1] = u.y;
+            w[i][2] = u.z;
+            w[i][3] = u.w;
+          }
+        } else {
+#pragma unroll
+          for (int i = 0; i < 12; ++i)
+#pragma unroll
+            for (int j = 0; j < SB; ++j) w[i][j] = __ldg(reinterpret_cast<const uint32_t*>(src[i]) + min(j, nb - 1));
+        }
+#pragma unroll
+        for (int i = 0; i < 12; ++i) {
+          const int ib = i - 4;
+          const int dst = i < 4 ? 16 * lane + 4 * i : SFA_BYTES + (ib >> 2) * 512 + 16 * lane + 4 * (ib & 3);
+#pragma unroll
+          for (int j = 0; j < SB; ++j)
+            if (j < nb) *reinterpret_cast<uint32_t*>(sf + j * SF_KB_BYTES + dst) = ok[i] ? w[i][j] : 0u;
+        }
+        // the chunks are read by tcgen05.cp through the async proxy
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&sfull[sb]);
+        if (++sb == kSfBufs) {
+          sb = 0;
+          sphase ^= 1;
         }
       }
     }
-    // every copy this warp issued lands before the CTA can exit (also on abort)
-    asm volatile("cp.async.wait_all;" ::: "memory");
   } else if (warp == 1) {
     // ======================= MMA issuer
     int stage = 0;
     uint32_t phase = 0, acc_phase = 0;
-    int kcount = 0;  // stages consumed so far (selects the scale slot)
+    int sb = 0, slot = 0;  // scale batch in shared memory, TMEM scale slot
+    uint32_t sphase = 0;
     for (int t = blockIdx.x; t < total && !aborted; t += gridDim.x) {
       if (!__all_sync(0xffffffffu, mbar_wait(tempty, acc_phase ^ 1, abort_flag, p.status, DEV_WAIT_TIMEOUT_MMA))) {
         aborted = true;
@@ -323,37 +366,57 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) gemm_mx_kernel(const __grid_co
       }
       tc_fence_after();
       for (int kb = 0; kb < KB; ++kb) {
+        const int j = kb % SB;
+        if (j == 0) {
+          // a new scale batch: copy its chunks into the TMEM slot (in issue order after the
+          // MMAs that read the slot's previous batch), then free its shared memory
+          if (!__all_sync(0xffffffffu,
+                          mbar_wait(&sfull[sb], sphase, abort_flag, p.status, DEV_WAIT_TIMEOUT_MMA))) {
+            aborted = true;
+            break;
+          }
+          tc_fence_after();
+          if (lane == 0) {
+            const int nb = min(SB, KB - kb);
+            const uint8_t* sf = sf_area + sb * SF_BATCH_BYTES;
+            const uint32_t col = tmem_base + SF_COL + SF_SLOT_COLS * slot;
+            for (int jj = 0; jj < nb; ++jj) {
+              const uint32_t sa = smem_u32(sf + jj * SF_KB_BYTES);
+              tmem_cp_32x128b_x4(col + 4 * jj, sf_desc(sa));
+              tmem_cp_32x128b_x4(col + 4 * SB + 8 * jj, sf_desc(sa + SFA_BYTES));
+              tmem_cp_32x128b_x4(col + 4 * SB + 8 * jj + 4, sf_desc(sa + SFA_BYTES + 512));
+            }
+            mma_commit(&sempty[sb]);
+          }
+          __syncwarp();
+          if (++sb == kSfBufs) {
+            sb = 0;
+            sphase ^= 1;
+          }
+        }
         if (!__all_sync(0xffffffffu, mbar_wait(&full[stage], phase, abort_flag, p.status, DEV_WAIT_TIMEOUT_MMA))) {
           aborted = true;
           break;
         }
         tc_fence_after();
         if (lane == 0) {
-          // the scale words arrived through the generic proxy (cp.async); tcgen05.cp reads
-          // shared memory through the async proxy
-          fence_proxy_async_smem();
           uint8_t* sA = smem + stage * STAGE_BYTES;
           uint8_t* sB = sA + A_BYTES;
-          uint8_t* sSF = sB + B_BYTES;
-          const int slot = kcount & 1;
-          const uint32_t sfa_t = tmem_base + SFA_COL + 4 * slot;
-          const uint32_t sfb_t = tmem_base + SFB_COL + 8 * slot;
-          tmem_cp_32x128b_x4(sfa_t, sf_desc(smem_u32(sSF)));
-          tmem_cp_32x128b_x4(sfb_t, sf_desc(smem_u32(sSF + SFA_BYTES)));
-          tmem_cp_32x128b_x4(sfb_t + 4, sf_desc(smem_u32(sSF + SFA_BYTES + 512)));
+          const uint32_t sfa_t = tmem_base + SF_COL + SF_SLOT_COLS * slot + 4 * j;
+          const uint32_t sfb_t = tmem_base + SF_COL + SF_SLOT_COLS * slot + 4 * SB + 8 * j;
           const uint32_t a0 = smem_u32(sA), b0 = smem_u32(sB);
 #pragma unroll
-          for (int j = 0; j < BK / 32; ++j) {
-            // scale byte j of each 32-bit TMEM word: in the descriptor's sf ids and in
+          for (int q = 0; q < BK / 32; ++q) {
+            // scale byte q of each 32-bit TMEM word: in the descriptor's sf ids and in
             // the top two bits of the scale addresses
-            mma_mxf8(tmem_base, smem_desc_sw128(a0 + j * 32, 16, 1024), smem_desc_sw128(b0 + j * 32, 16, 1024),
-                     idesc_mx(BM, BN, j), sfa_t | ((uint32_t)j << 30), sfb_t | ((uint32_t)j << 30),
-                     (kb | j) != 0 ? 1u : 0u);
+            mma_mxf8(tmem_base, smem_desc_sw128(a0 + q * 32, 16, 1024), smem_desc_sw128(b0 + q * 32, 16, 1024),
+                     idesc_mx(BM, BN, q), sfa_t | ((uint32_t)q << 30), sfb_t | ((uint32_t)q << 30),
+                     (kb | q) != 0 ? 1u : 0u);
           }
           mma_commit(&empty[stage]);
         }
         __syncwarp();
-        ++kcount;
+        if (j == SB - 1 || kb == KB - 1) slot ^= 1;
         if (++stage == kStages) {
           stage = 0;
           phase ^= 1;

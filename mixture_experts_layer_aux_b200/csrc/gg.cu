@@ -27,8 +27,11 @@ using gg::Cfg;
 // halves each SM's operand traffic per FLOP but pads each expert to a
 // multiple of 256 rows. Used when the average rows per group reach this
 // threshold (MOE_B200_PAIR_MIN_ROWS overrides it; a huge value disables it).
+// The SM-pair kernel is opt-in: MOE_B200_PAIR_MIN_ROWS=n selects it for GEMMs whose experts
+// average at least n rows. On B200 it matches the one-SM kernel on aligned experts and loses on
+// ragged ones (its 256-row tiles waste more rows at each expert's end).
 static bool use_pair_kernel(int rows, int groups) {
-  long long thr = 768;
+  long long thr = 1LL << 40;
   if (const char* e = std::getenv("MOE_B200_PAIR_MIN_ROWS")) thr = std::atoll(e);
   return (long long)rows >= thr * (long long)groups;
 }
@@ -93,7 +96,7 @@ int gemm_down_bf16(int rows, int groups, int H, int F, const void* A, const void
 
 // ---------------------------------------------------------------- backward
 
-// dgu = SwiGLU-backward(dYp W_d), dg partials [rows, F/256].
+// dgu = SwiGLU-backward(dYp W_d), dg partials [rows, F/128].
 int gemm_dgrad_down(int rows, int groups, int H, int F, const void* dYp, const void* Wd, const int32_t* offsets,
                     const void* gateup, const float* row_gate, void* dgu, float* dg_part, cudaStream_t st) {
   gg::Params p{};
@@ -172,7 +175,7 @@ __global__ void dg_reduce_kernel(const float* __restrict__ part, int rows, int n
 
 size_t gg_fwd_ws(const moe_config*, int) { return 256; }
 size_t gg_bwd_ws(const moe_config* c, int which) {
-  if (which == MOE_GEMM_DOWN) return ws_round((size_t)c->T * c->k * (c->F / 256) * sizeof(float));
+  if (which == MOE_GEMM_DOWN) return ws_round((size_t)c->T * c->k * (c->F / 128) * sizeof(float));
   return 256;
 }
 
@@ -238,7 +241,7 @@ extern "C" int moe_grouped_gemm_bwd(const moe_config* cfg, int which, const void
       float* part = static_cast<float*>(ws);
       rc = gemm_dgrad_down(rows, E, H, F, dO, W0, offsets, saved_gateup, row_gate, d_in, part, st);
       if (rc) return rc;
-      dg_reduce_kernel<<<(rows + 255) / 256, 256, 0, st>>>(part, rows, F / 256, dg);
+      dg_reduce_kernel<<<(rows + 255) / 256, 256, 0, st>>>(part, rows, F / 128, dg);
       MOE_CHECK_LAUNCH();
     }
     if (dW0) {

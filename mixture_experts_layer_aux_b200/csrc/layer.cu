@@ -280,7 +280,7 @@ static size_t carve_bwd(void* ws, const moe_config* c, BwdWs* w) {
   const size_t T = c->T, E = c->E, k = c->k, H = c->H, F = c->F, rows = T * k;
   w->dYp = cv.take<__nv_bfloat16>(rows * H);
   w->dgu = cv.take<__nv_bfloat16>(rows * 2 * F);
-  w->dg_part = cv.take<float>(rows * (F / 256));
+  w->dg_part = cv.take<float>(rows * (F / 128));
   w->dXp = cv.take<__nv_bfloat16>(rows * H);
   w->dl = cv.take<float>(T * E);
   w->dl16 = cv.take<__nv_bfloat16>(T * E);
@@ -303,7 +303,7 @@ int layer_bwd(const moe_config* c, const void* dY, float d_aux, const void* x, c
   RC(gemm_dgrad_gateup(rows, E, H, F, w.dgu, W_g, W_u, sv.offsets, w.dXp, st));
   RC(gemm_wgrad(rows, E, 2 * F, H, w.dgu, 2 * F, sv.xp, sv.offsets, dW_g, dW_u, F, st));
   float* dl = dlogits ? dlogits : w.dl;
-  router_bwd_kernel<<<(T + 7) / 8, 256, 0, st>>>(w.dg_part, F / 256, sv.row_of, sv.idx, sv.gates, sv.probs, sv.counts,
+  router_bwd_kernel<<<(T + 7) / 8, 256, 0, st>>>(w.dg_part, F / 128, sv.row_of, sv.idx, sv.gates, sv.probs, sv.counts,
                                                  T, E, k, c->score, c->norm_topk, c->route_scale,
                                                  c->compute_aux ? 1 : 0, d_aux, dl, w.dl16);
   MOE_CHECK_LAUNCH();

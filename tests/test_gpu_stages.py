@@ -206,14 +206,15 @@ GEMM_CASES = [
 ]
 
 
-@pytest.fixture(params=["auto", "pair", "single"])
+@pytest.fixture(params=["default", "pair"])
 def fwd_kernel(request, monkeypatch):
-    """Run the forward GEMMs with the library's own kernel choice, or forced onto the
-    SM-pair (256-row tile) or the single-SM (128-row tile) kernel."""
+    """Run the forward GEMMs with the library's own kernel choice (the one-SM, 128-row
+    tile kernel unless MOE_B200_PAIR_MIN_ROWS opts in), or forced onto the SM-pair
+    (256-row tile) kernel."""
     if request.param == "pair":
         monkeypatch.setenv("MOE_B200_PAIR_MIN_ROWS", "0")
-    elif request.param == "single":
-        monkeypatch.setenv("MOE_B200_PAIR_MIN_ROWS", str(1 << 40))
+    else:
+        monkeypatch.delenv("MOE_B200_PAIR_MIN_ROWS", raising=False)
     return request.param
 
 
