@@ -46,6 +46,7 @@ class Workload:
     aux: bool = True           # compute the load-balancing aux statistic
     skew: bool = False         # add the skew logit bias
     bwd: bool = False          # the workload includes the backward pass
+    capacity_factor: float = 0.0  # > 0: each expert keeps its first ceil(cf T k / E) pairs
 
     def with_(self, **kw) -> "Workload":
         return replace(self, **kw)

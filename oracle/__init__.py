@@ -205,16 +205,34 @@ def gates(s: torch.Tensor, idx: torch.Tensor, norm: bool, route_scale: float) ->
     return g
 
 
-def maps(idx: torch.Tensor, E: int):
-    """-> counts [E], offsets [E+1], row_of [T,k], src_of [T*k] (all int32)."""
+def maps(idx: torch.Tensor, E: int, keep: torch.Tensor | None = None):
+    """-> counts [E], offsets [E+1], row_of [T,k], src_of [T*k] (all int32).
+
+    With a capacity keep mask (uint8 [T,k]), only kept pairs get rows: counts are
+    the kept counts and row_of is -1 for dropped pairs (src_of beyond offsets[E]
+    is unused)."""
     idx = _chk(idx.contiguous(), torch.int32)
     T, k = idx.shape
     counts = torch.empty(E, dtype=torch.int32)
     offsets = torch.empty(E + 1, dtype=torch.int32)
     row_of = torch.empty((T, k), dtype=torch.int32)
-    src_of = torch.empty(T * k, dtype=torch.int32)
-    lib().oc_maps(T, E, k, _p(idx), _p(counts), _p(offsets), _p(row_of), _p(src_of))
+    src_of = torch.full((T * k,), -1, dtype=torch.int32)
+    if keep is None:
+        lib().oc_maps(T, E, k, _p(idx), _p(counts), _p(offsets), _p(row_of), _p(src_of))
+    else:
+        keep = _chk(keep.contiguous(), torch.uint8)
+        lib().oc_maps_kept(T, E, k, _p(idx), _p(keep), _p(counts), _p(offsets), _p(row_of), _p(src_of))
     return counts, offsets, row_of, src_of
+
+
+def capacity_keep(idx: torch.Tensor, E: int, capacity_factor: float):
+    """-> (keep uint8 [T,k], C): each expert keeps its first C = ceil(cf T k / E) pairs in
+    token order (cf <= 0: no limit, C = T k)."""
+    idx = _chk(idx.contiguous(), torch.int32)
+    T, k = idx.shape
+    keep = torch.empty((T, k), dtype=torch.uint8)
+    C = lib().oc_capacity_keep(T, E, k, ctypes.c_double(capacity_factor), _p(idx), _p(keep))
+    return keep, int(C)
 
 
 def aux(s_softmax: torch.Tensor, counts: torch.Tensor, k: int) -> float:
@@ -223,15 +241,25 @@ def aux(s_softmax: torch.Tensor, counts: torch.Tensor, k: int) -> float:
 
 
 def route(logits: torch.Tensor, k: int, score: str = "softmax", norm: bool = True,
-          route_scale: float = 1.0, with_aux: bool = True) -> dict:
-    """All routing steps from given logits: scores, top-k, gates, maps, aux."""
+          route_scale: float = 1.0, with_aux: bool = True, capacity_factor: float = 0.0) -> dict:
+    """All routing steps from given logits: scores, top-k, gates, maps, aux.
+
+    counts are the router's (every selected pair; they feed aux). With a capacity
+    factor > 0, pairs past an expert's capacity are dropped: keep marks the kept
+    pairs, idx_kept is idx with -1 at dropped pairs, kept_counts / offsets /
+    row_of / src_of describe the kept rows only."""
     E = logits.shape[1]
     s = scores(logits, score)
     idx = topk(logits, k)
     g = gates(s, idx, norm, route_scale)
     counts, offsets, row_of, src_of = maps(idx, E)
     out = dict(logits=logits, probs=s, idx=idx, gates=g, counts=counts, offsets=offsets,
-               row_of=row_of, src_of=src_of)
+               row_of=row_of, src_of=src_of, idx_kept=idx, kept_counts=counts, keep=None, capacity=idx.numel())
+    if capacity_factor > 0:
+        keep, C = capacity_keep(idx, E, capacity_factor)
+        kc, offsets, row_of, src_of = maps(idx, E, keep)
+        out.update(keep=keep, capacity=C, idx_kept=torch.where(keep.bool(), idx, torch.full_like(idx, -1)),
+                   kept_counts=kc, offsets=offsets, row_of=row_of, src_of=src_of)
     if with_aux and score == "softmax":
         out["aux"] = aux(s, counts, k)
     return out
@@ -348,6 +376,7 @@ def moe_bwd_tokens(x, W_r, W_g, W_u, W_d, dY, r: dict, toks=None, *, score="soft
     lib().oc_moe_bwd_tokens(T, H, E, k, F, 0 if score == "softmax" else 1, int(norm), ctypes.c_double(route_scale),
                             int(aux_on), ctypes.c_double(d_aux), _recipe(recipe), *[m.ref for m in ms],
                             _p(r["idx"]), _p(_chk(r["probs"], torch.float64)), _p(s_soft), _p(r["counts"]),
+                            _p(_chk(r["keep"].contiguous(), torch.uint8)) if r.get("keep") is not None else None,
                             n, _p(toks), _p(dx), _p(dl), _p(dg))
     return dx, dl, dg
 
@@ -390,7 +419,7 @@ def layer_fwd(wl, inp: dict, toks=None, logits=None, mx_weights=None, recipe=Non
     if logits is None:
         logits = router_logits(inp["x"], inp["W_r"], inp.get("logit_bias"))
     r = route(logits.to(torch.float64), wl.k, wl.score, wl.norm_topk, wl.route_scale,
-              with_aux=wl.aux and wl.score == "softmax")
+              with_aux=wl.aux and wl.score == "softmax", capacity_factor=getattr(wl, "capacity_factor", 0.0))
     mx = wl.dtype == "mxfp8"
     if recipe is None:
         recipe = "mxfp8" if mx else "exact"
@@ -405,6 +434,6 @@ def layer_fwd(wl, inp: dict, toks=None, logits=None, mx_weights=None, recipe=Non
     else:
         wg, wu, wd = inp["W_g"], inp["W_u"], inp["W_d"]
         shared = (inp["W_gs"], inp["W_us"], inp["W_ds"]) if wl.S else None
-    y = moe_fwd_tokens(inp["x"], wg, wu, wd, r["idx"], r["gates"], toks, recipe=recipe, shared=shared, **kw)
+    y = moe_fwd_tokens(inp["x"], wg, wu, wd, r["idx_kept"], r["gates"], toks, recipe=recipe, shared=shared, **kw)
     r["y"] = y
     return r

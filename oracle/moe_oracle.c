@@ -355,6 +355,54 @@ void oc_maps(int T, int E, int k, const int32_t* idx, int32_t* counts, int32_t* 
     free(fill);
 }
 
+/*
+ * Capacity factor (the expert-slot limit the practice cases name as the first
+ * knob for imbalance: an expert whose slots are full drops the excess tokens).
+ * Reading: C = ceil(cf * T * k / E) slots per expert; an expert keeps the
+ * first C of its (token, slot) pairs in ascending token order and drops the
+ * rest; cf <= 0 means no limit. keep[t*k + j] = 1 for kept pairs, 0 for
+ * dropped ones. Returns C (or T*k without a limit).
+ */
+int oc_capacity_keep(int T, int E, int k, double cf, const int32_t* idx, uint8_t* keep) {
+    long cap = (long)T * k;
+    if (cf > 0.0) {
+        double c = ceil(cf * (double)T * (double)k / (double)E);
+        cap = c < (double)cap ? (long)c : cap;
+    }
+    long* seen = (long*)calloc(E, sizeof(long));
+    for (long p = 0; p < (long)T * k; ++p) {
+        int e = idx[p];
+        keep[p] = (uint8_t)(seen[e] < cap);
+        seen[e] += 1;
+    }
+    free(seen);
+    return (int)cap;
+}
+
+/* Maps of the kept pairs only (keep == NULL: every pair): counts of kept pairs,
+ * offsets, the stable order, and row_of = -1 for dropped pairs. */
+void oc_maps_kept(int T, int E, int k, const int32_t* idx, const uint8_t* keep, int32_t* counts, int32_t* offsets,
+                  int32_t* row_of, int32_t* src_of) {
+    for (int e = 0; e < E; ++e) counts[e] = 0;
+    for (long p = 0; p < (long)T * k; ++p)
+        if (!keep || keep[p]) counts[idx[p]] += 1;
+    offsets[0] = 0;
+    for (int e = 0; e < E; ++e) offsets[e + 1] = offsets[e] + counts[e];
+    int32_t* fill = (int32_t*)malloc(sizeof(int32_t) * E);
+    for (int e = 0; e < E; ++e) fill[e] = offsets[e];
+    for (long p = 0; p < (long)T * k; ++p) {
+        if (keep && !keep[p]) {
+            row_of[p] = -1;
+            continue;
+        }
+        int e = idx[p];
+        int r = fill[e]++;
+        row_of[p] = r;
+        src_of[r] = (int32_t)(p / k);
+    }
+    free(fill);
+}
+
 /* aux = E * sum_e f_e P_e, f_e = counts[e]/(T k), P_e = mean_t s[t,e] (full softmax). */
 double oc_aux(int T, int E, int k, const double* s, const int32_t* counts) {
     double acc = 0.0;
@@ -395,6 +443,7 @@ static void round_act(double* a, int F, int recipe) {
  *   y[t] = sum_j g[t,j] * W_d[e_j] (silu(W_g[e_j] x_t) * (W_u[e_j] x_t))
  *          (+ shared expert on every token, weight 1)
  *
+ * A slot with idx < 0 (a pair dropped at an expert's capacity) is skipped.
  * fold = 1 evaluates W_d (g a) (the memory-efficient permutation order),
  * fold = 0 evaluates g (W_d a); the two agree up to rounding.
  * recipe (OC_EXACT / OC_MX / OC_BF16R) selects the rounding points:
@@ -431,6 +480,7 @@ int oc_moe_fwd_tokens(int T, int H, int E, int k, int F, int S, int recipe, int 
         for (int j = 0; j < k; ++j) {
             int e = idx[(long)t * k + j];
             double g = gates[(long)t * k + j];
+            if (e < 0) continue; /* a pair dropped at an expert's capacity contributes nothing */
             oc_mat we_g = oc_slice(Wg, (int64_t)e * F, F);
             oc_mat we_u = oc_slice(Wu, (int64_t)e * F, F);
             oc_mat we_d = oc_slice(Wd, (int64_t)e * H, H);
@@ -558,13 +608,17 @@ int oc_expert_rows(int H, int F, int recipe, const oc_mat* xp, const int32_t* e_
  * dz_g and dz_u are rounded to bf16, each selected expert's contribution
  * W_g^T dz_g + W_u^T dz_u is rounded to bf16, and the router path uses dl
  * rounded to bf16 and rounds its result to bf16. dl itself stays unrounded.
- * logits, s (scores), gates, idx and counts are the forward's.
+ * logits, s (scores), gates, idx and counts are the forward's (counts: every
+ * selected pair, as the router counted them for aux). keep: NULL, or the
+ * capacity mask of oc_capacity_keep: a dropped pair contributes nothing to y,
+ * so it gets dg = 0 and no expert gradient, while its score still enters the
+ * normalisation of the other gates.
  */
 int oc_moe_bwd_tokens(int T, int H, int E, int k, int F, int score, int norm, double route_scale, int aux_on,
                       double d_aux, int recipe, const oc_mat* x, const oc_mat* Wr, const oc_mat* Wg,
                       const oc_mat* Wu, const oc_mat* Wd, const oc_mat* dY, const int32_t* idx, const double* s_all,
-                      const double* s_softmax, const int32_t* counts, int n_tok, const int32_t* toks,
-                      double* dx_out, double* dl_out, double* dg_out) {
+                      const double* s_softmax, const int32_t* counts, const uint8_t* keep, int n_tok,
+                      const int32_t* toks, double* dx_out, double* dl_out, double* dg_out) {
     int i;
 #pragma omp parallel for schedule(dynamic, 1)
     for (i = 0; i < n_tok; ++i) {
@@ -599,6 +653,10 @@ int oc_moe_bwd_tokens(int T, int H, int E, int k, int F, int score, int norm, do
         }
         for (int j = 0; j < k; ++j) {
             int e = idx[(long)t * k + j];
+            if (keep && !keep[(long)t * k + j]) {
+                dg[j] = 0.0; /* dropped at capacity: the output does not depend on its gate */
+                continue;
+            }
             oc_mat we_g = oc_slice(Wg, (int64_t)e * F, F);
             oc_mat we_u = oc_slice(Wu, (int64_t)e * F, F);
             oc_mat we_d = oc_slice(Wd, (int64_t)e * H, H);

@@ -294,6 +294,58 @@ def test_mxfp8_bf16_and_fp32_entry_points_agree(oracle):
     assert torch.equal(a[0], b[0]) and torch.equal(a[1], b[1])
 
 
+# --------------------------------------------------------------- capacity factor
+
+
+def _stable_rank_within_expert(idx, E):
+    """Position of each (t, j) among its expert's pairs in token order, by a library stable sort."""
+    flat = idx.flatten().long()
+    order = torch.sort(flat, stable=True).indices
+    counts = torch.bincount(flat, minlength=E)
+    starts = torch.cumsum(counts, 0) - counts
+    rank = torch.empty_like(flat)
+    rank[order] = torch.arange(flat.numel()) - starts[flat[order]]
+    return rank.view(idx.shape), counts
+
+
+@pytest.mark.parametrize("cf", [0.5, 1.0, 1.25, 100.0])
+def test_capacity_keep_matches_stable_sort_rank_and_maps_invariants(oracle, cf):
+    from mixture_experts_layer_aux_b200.synthetic import random_routing
+    T, E, k = 60, 6, 2
+    idx = random_routing(T, E, k, seed=3, hot=0.6)
+    keep, C = oracle.capacity_keep(idx, E, cf)
+    assert C == min(T * k, math.ceil(cf * T * k / E))
+    rank, counts = _stable_rank_within_expert(idx, E)
+    assert torch.equal(keep.bool(), rank < C)
+    kc, off, row_of, src_of = oracle.maps(idx, E, keep)
+    assert torch.equal(kc.long(), torch.clamp(counts, max=C))
+    assert int(off[-1]) == int(kc.sum())
+    kept = keep.bool()
+    assert bool((row_of[~kept] == -1).all())
+    rows = row_of[kept].long()
+    assert torch.equal(torch.sort(rows).values, torch.arange(int(off[-1])))      # a bijection onto the kept rows
+    tok = torch.arange(T).unsqueeze(1).expand(T, k)
+    assert torch.equal(src_of[rows].long(), tok[kept])
+    # a kept row sits in its expert's segment at its rank
+    e = idx[kept].long()
+    assert torch.equal(rows, off[e].long() + rank[kept])
+    if cf >= 100.0:                                                              # no drops: the dropless maps
+        c0, o0, r0, s0 = oracle.maps(idx, E)
+        assert torch.equal(row_of, r0) and torch.equal(off, o0)
+
+
+def test_capacity_forward_equals_dense_brute_force_without_dropped_pairs(oracle):
+    """y with capacity = the dense all-experts mixture whose gate matrix is zero at dropped pairs."""
+    wl = small(T=40, H=64, E=4, k=2, F=96, capacity_factor=0.75)
+    inp = make_inputs(wl, seed=21)
+    r = oracle.layer_fwd(wl, inp)
+    assert r["keep"] is not None and int((r["keep"] == 0).sum()) > 0            # some pairs are dropped
+    gd = torch.zeros(wl.T, wl.E, dtype=torch.float64)
+    gd.scatter_(1, r["idx"].long(), r["gates"] * r["keep"].double())
+    yd = oracle.moe_fwd_dense(inp["x"], inp["W_g"], inp["W_u"], inp["W_d"], gd)
+    assert torch.allclose(r["y"], yd, rtol=1e-12, atol=1e-13)
+
+
 # --------------------------------------------------------------- backward
 
 
@@ -314,24 +366,30 @@ def _fd_setup(score, norm, scale, aux_on, seed=0, T=8, H=16, E=4, k=2, F=32):
 def _loss(o, t, cfg, logits=None):
     if logits is None:
         logits = o.router_logits(t["x"], t["W_r"], None, round_f32=False)
-    r = o.route(logits, cfg["k"], cfg["score"], cfg["norm"], cfg["scale"], with_aux=cfg["aux_on"])
-    y = o.moe_fwd_tokens(t["x"], t["W_g"], t["W_u"], t["W_d"], r["idx"], r["gates"])
+    r = o.route(logits, cfg["k"], cfg["score"], cfg["norm"], cfg["scale"], with_aux=cfg["aux_on"],
+                capacity_factor=cfg.get("cf", 0.0))
+    y = o.moe_fwd_tokens(t["x"], t["W_g"], t["W_u"], t["W_d"], r["idx_kept"], r["gates"])
     L = (t["dY"] * y).sum().item()
     if cfg["aux_on"]:
         L += cfg["d_aux"] * r["aux"]
     return L, r
 
 
-@pytest.mark.parametrize("score,norm,scale,aux_on", [("softmax", True, 1.0, True), ("sigmoid", True, 2.5, False),
-                                                     ("softmax", False, 1.0, True)])
-def test_backward_matches_central_finite_differences(oracle, score, norm, scale, aux_on):
+@pytest.mark.parametrize("score,norm,scale,aux_on,cf", [("softmax", True, 1.0, True, 0.0),
+                                                        ("sigmoid", True, 2.5, False, 0.0),
+                                                        ("softmax", False, 1.0, True, 0.0),
+                                                        ("softmax", True, 1.0, True, 0.75)])
+def test_backward_matches_central_finite_differences(oracle, score, norm, scale, aux_on, cf):
     o = oracle
     t, cfg = _fd_setup(score, norm, scale, aux_on)
+    cfg["cf"] = cf
     L0, r = _loss(o, t, cfg)
+    if cf > 0:
+        assert int((r["keep"] == 0).sum()) > 0                                  # the case drops pairs
     E = t["W_r"].shape[0]
     dx, dl, dg = o.moe_bwd_tokens(t["x"], t["W_r"], t["W_g"], t["W_u"], t["W_d"], t["dY"], r, score=score,
                                   norm=norm, route_scale=scale, aux_on=aux_on, d_aux=cfg["d_aux"])
-    dWg, dWu, dWd = o.moe_bwd_expert_dw(t["x"], t["W_g"], t["W_u"], t["W_d"], t["dY"], r["idx"], r["gates"],
+    dWg, dWu, dWd = o.moe_bwd_expert_dw(t["x"], t["W_g"], t["W_u"], t["W_d"], t["dY"], r["idx_kept"], r["gates"],
                                         list(range(E)))
     dWr = o.router_dwr(dl, t["x"])
     grads = dict(x=dx, W_r=dWr, W_g=dWg, W_u=dWu, W_d=dWd)
