@@ -309,6 +309,39 @@ class Layer:
                         self.dW_r, self.dW_g, self.dW_u, self.dW_d, None, self.ws_bwd)
 
 
+def graph_replay(L, wl, args, st, ws):
+    """Capture one whole step in a CUDA graph and time K replays (after W) with CUDA events."""
+    def one():
+        if wl.bwd:
+            L.layer_call(L.d["x"], L.y, L.aux)
+            L.bwd_call()
+        else:
+            L.step()
+    side = torch.cuda.Stream()
+    side.wait_stream(st)
+    with torch.cuda.stream(side):
+        one()  # warm the capture stream (tensor maps, function attributes)
+    st.wait_stream(side)
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        one()
+    for _ in range(args.warmup):
+        g.replay()
+    torch.cuda.synchronize()
+    barrier(ws)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(st)
+    for _ in range(args.steps):
+        g.replay()
+    e1.record(st)
+    torch.cuda.synchronize()
+    ms = max_over_ranks(e0.elapsed_time(e1) / args.steps, ws)
+    del g
+    return {"ms_per_step": round(ms, 4), "value": aggregate_tokens_per_s(wl.T, ws, ms), "unit": "tokens/s",
+            "how": "one step captured in a CUDA graph, replayed K times"}
+
+
 def run_ours(args, rank, ws):
     import mixture_experts_layer_aux_b200 as moe
     moe.load()
@@ -410,6 +443,9 @@ def run_ours(args, rank, ws):
                 "peak": peak_t, "unit": "TFLOP/s", "frac": round(ach / peak_t, 4), "traffic": None,
                 "peak_source": f"{P['source']}: {peak_note}"}
 
+    # the same step under CUDA-graph replay (one captured step, replayed K times)
+    graph = graph_replay(L, wl, args, st, ws)
+
     # end to end: public whole-layer call, tokens H2D from pinned memory, y (+aux) D2H, every step
     x_host = L.d["x"].cpu().pin_memory()
     y_host = torch.empty(wl.T, wl.H, dtype=torch.bfloat16).pin_memory()
@@ -459,6 +495,7 @@ def run_ours(args, rank, ws):
         "e2e": {"value": aggregate_tokens_per_s(wl.T, ws, e2e_ms), "unit": "tokens/s", "ms_per_step": round(e2e_ms, 4),
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "api": "moe_layer_fwd" +
                 ("+moe_layer_bwd" if wl.bwd else "")},
+        "graph": graph,
         "gpu_launches": L.launches_per_step() * args.steps,
         "clocks": clocks,
     }

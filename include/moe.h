@@ -73,6 +73,12 @@ typedef struct moe_config {
     int32_t expert_dtype; /* moe_dtype of the expert GEMM operands */
     int32_t compute_aux;  /* 1: load-balancing aux statistic (softmax scores only) */
     int32_t save_for_bwd; /* 1: moe_layer_fwd fills `saved` for moe_layer_bwd */
+    float capacity_factor; /* 0: dropless. > 0: every expert has C = ceil(cf T k / E) slots
+                              and keeps the first C of its (token, slot) pairs in token
+                              order; the others are dropped (no row, no contribution to y,
+                              no expert gradient). The router's counts and aux still count
+                              every selected pair; the permutation's counts and offsets
+                              count the kept rows. NaN or negative: MOE_ERR_INVALID_ARG. */
 } moe_config;
 
 /* Human-readable name of a status code (static string). */
@@ -114,7 +120,9 @@ int moe_router_topk(const moe_config* cfg, const void* x, const void* W_r, const
  * 2.2 of the summary; sync-free, 2.4): per-expert counts, exclusive-scan
  * offsets, the stable row maps, the per-row gate, and the gathered rows --
  * all on the device.
- *   counts[e], offsets[0..E] (offsets[E] = T*k),
+ *   counts[e], offsets[0..E] (offsets[E] = T*k; with a capacity factor, the
+ *   kept rows: counts[e] = min(#pairs of e, C), and row_of = -1 for a dropped
+ *   pair, which gets no row),
  *   row_of[t,j] = offsets[e] + #{t' < t : e in idx[t',:]} for e = idx[t,j],
  *   src_of[row_of[t,j]] = t, row_gate[row_of[t,j]] = gates[t,j],
  *   xp[row_of[t,j], :] = x[t, :].
@@ -234,7 +242,9 @@ int moe_quantize_mxfp8(const void* src, int64_t rows, int32_t K, uint8_t* dst, u
  *     [E,F,H/32], W_d_sf [E,H,F/32]), as moe_quantize_mxfp8 produces them;
  *   shared expert (n_shared = 1): Ws_g, Ws_u [F,H], Ws_d [H,F] (+ scales);
  *   y [T,H] bf16 out; aux [1] fp32 out or NULL; idx [T,k], gates [T,k],
- *   counts [E], offsets [E+1] optional outputs (NULL to skip);
+ *   counts [E], offsets [E+1] optional outputs (NULL to skip): counts are the
+ *   router's (every selected pair, as aux counts them), offsets those of the
+ *   kept rows (they differ only under a capacity factor);
  *   saved: moe_layer_saved_size() bytes, filled when save_for_bwd (else NULL).
  * ------------------------------------------------------------------------ */
 size_t moe_layer_workspace_size(const moe_config* cfg);

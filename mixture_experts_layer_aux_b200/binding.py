@@ -34,7 +34,8 @@ class moe_config(ctypes.Structure):
     _fields_ = [("T", ctypes.c_int32), ("H", ctypes.c_int32), ("E", ctypes.c_int32), ("k", ctypes.c_int32),
                 ("F", ctypes.c_int32), ("n_shared", ctypes.c_int32), ("score", ctypes.c_int32),
                 ("norm_topk", ctypes.c_int32), ("route_scale", ctypes.c_float), ("expert_dtype", ctypes.c_int32),
-                ("compute_aux", ctypes.c_int32), ("save_for_bwd", ctypes.c_int32)]
+                ("compute_aux", ctypes.c_int32), ("save_for_bwd", ctypes.c_int32),
+                ("capacity_factor", ctypes.c_float)]
 
 
 _VP = ctypes.c_void_p
@@ -120,13 +121,14 @@ def _check(fn, rc):
 def make_config(wl=None, **kw) -> moe_config:
     """moe_config from a synthetic.Workload (or keyword fields)."""
     d = dict(T=0, H=0, E=0, k=0, F=0, n_shared=0, score=MOE_SCORE_SOFTMAX, norm_topk=1, route_scale=1.0,
-             expert_dtype=MOE_DT_BF16, compute_aux=0, save_for_bwd=0)
+             expert_dtype=MOE_DT_BF16, compute_aux=0, save_for_bwd=0, capacity_factor=0.0)
     if wl is not None:
         d.update(T=wl.T, H=wl.H, E=wl.E, k=wl.k, F=wl.F, n_shared=wl.S,
                  score=MOE_SCORE_SOFTMAX if wl.score == "softmax" else MOE_SCORE_SIGMOID,
                  norm_topk=int(wl.norm_topk), route_scale=wl.route_scale,
                  expert_dtype=MOE_DT_BF16 if wl.dtype == "bf16" else MOE_DT_MXFP8,
-                 compute_aux=int(wl.aux and wl.score == "softmax"), save_for_bwd=int(wl.bwd))
+                 compute_aux=int(wl.aux and wl.score == "softmax"), save_for_bwd=int(wl.bwd),
+                 capacity_factor=wl.capacity_factor)
     d.update(kw)
     return moe_config(**d)
 

@@ -16,10 +16,11 @@
 //   k-block: the 16 bytes of lane l hold rows l, l+32, l+64, l+96. The loader
 //   fences the generic-proxy stores for the async proxy before it arrives on
 //   the batch's barrier, so the MMA thread does no fence of its own.
-// MMA: per batch, tcgen05.cp copies the batch's chunks into one of two TMEM
-// scale slots (SFA 4 columns and SFB 8 columns per k-block) and a commit frees
-// the batch's shared memory; per k-block, four M128 N256 K32 MMAs select scale
-// byte j through the instruction descriptor.
+// MMA: per k-block, tcgen05.cp copies its chunks from the batch into one of
+// two TMEM scale slots (SFA 4 columns, SFB 8 columns; alternating by k-block)
+// right before four M128 N256 K32 MMAs that select scale byte j through the
+// instruction descriptor; after a batch's last k-block a commit frees its
+// shared memory.
 // TMEM: one 256-column fp32 accumulator and the two scale slots; eight
 // epilogue warps (two per lane quadrant, 128 columns each) first copy their
 // accumulator columns into registers and release TMEM, so the next tile's MMAs
@@ -52,7 +53,7 @@ constexpr int kSfBufs = 3;              // scale batches in shared memory
 constexpr int SF_BATCH_BYTES = SB * SF_KB_BYTES;
 constexpr int TMEM_COLS = 512;
 constexpr int SF_COL = 256;             // TMEM scale slots after the accumulator
-constexpr int SF_SLOT_COLS = SB * 12;   // per k-block: SFA 4 columns, SFB 8 columns
+constexpr int SF_SLOT_COLS = 12;        // one k-block: SFA 4 columns, SFB 8 columns
 constexpr int BAR_BYTES = 1024;
 constexpr int SMEM_BYTES =
     1024 + kStages * STAGE_BYTES + kSfBufs * SF_BATCH_BYTES + BAR_BYTES + 2 * (MAX_G + 1) * 4;
@@ -357,7 +358,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) gemm_mx_kernel(const __grid_co
     // ======================= MMA issuer
     int stage = 0;
     uint32_t phase = 0, acc_phase = 0;
-    int sb = 0, slot = 0;  // scale batch in shared memory, TMEM scale slot
+    int sb = 0;  // scale batch in shared memory
     uint32_t sphase = 0;
     for (int t = blockIdx.x; t < total && !aborted; t += gridDim.x) {
       if (!__all_sync(0xffffffffu, mbar_wait(tempty, acc_phase ^ 1, abort_flag, p.status, DEV_WAIT_TIMEOUT_MMA))) {
@@ -367,31 +368,13 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) gemm_mx_kernel(const __grid_co
       tc_fence_after();
       for (int kb = 0; kb < KB; ++kb) {
         const int j = kb % SB;
+        const bool batch_end = (j == SB - 1) || (kb == KB - 1);
         if (j == 0) {
-          // a new scale batch: copy its chunks into the TMEM slot (in issue order after the
-          // MMAs that read the slot's previous batch), then free its shared memory
+          // a new scale batch in shared memory
           if (!__all_sync(0xffffffffu,
                           mbar_wait(&sfull[sb], sphase, abort_flag, p.status, DEV_WAIT_TIMEOUT_MMA))) {
             aborted = true;
             break;
-          }
-          tc_fence_after();
-          if (lane == 0) {
-            const int nb = min(SB, KB - kb);
-            const uint8_t* sf = sf_area + sb * SF_BATCH_BYTES;
-            const uint32_t col = tmem_base + SF_COL + SF_SLOT_COLS * slot;
-            for (int jj = 0; jj < nb; ++jj) {
-              const uint32_t sa = smem_u32(sf + jj * SF_KB_BYTES);
-              tmem_cp_32x128b_x4(col + 4 * jj, sf_desc(sa));
-              tmem_cp_32x128b_x4(col + 4 * SB + 8 * jj, sf_desc(sa + SFA_BYTES));
-              tmem_cp_32x128b_x4(col + 4 * SB + 8 * jj + 4, sf_desc(sa + SFA_BYTES + 512));
-            }
-            mma_commit(&sempty[sb]);
-          }
-          __syncwarp();
-          if (++sb == kSfBufs) {
-            sb = 0;
-            sphase ^= 1;
           }
         }
         if (!__all_sync(0xffffffffu, mbar_wait(&full[stage], phase, abort_flag, p.status, DEV_WAIT_TIMEOUT_MMA))) {
@@ -400,10 +383,20 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) gemm_mx_kernel(const __grid_co
         }
         tc_fence_after();
         if (lane == 0) {
+          // this k-block's scale chunks into its TMEM slot (alternating by k-block; in issue order
+          // after the MMAs that read the slot two k-blocks ago), copied right before its MMAs:
+          // on B200 three copies per k-block cost the tensor pipe far less than a batch of twelve
+          const uint8_t* sf = sf_area + sb * SF_BATCH_BYTES + j * SF_KB_BYTES;
+          const uint32_t col = tmem_base + SF_COL + SF_SLOT_COLS * (kb & 1);
+          const uint32_t sa = smem_u32(sf);
+          tmem_cp_32x128b_x4(col, sf_desc(sa));
+          tmem_cp_32x128b_x4(col + 4, sf_desc(sa + SFA_BYTES));
+          tmem_cp_32x128b_x4(col + 8, sf_desc(sa + SFA_BYTES + 512));
+          if (batch_end) mma_commit(&sempty[sb]);  // the batch's shared memory is free once its copies are done
           uint8_t* sA = smem + stage * STAGE_BYTES;
           uint8_t* sB = sA + A_BYTES;
-          const uint32_t sfa_t = tmem_base + SF_COL + SF_SLOT_COLS * slot + 4 * j;
-          const uint32_t sfb_t = tmem_base + SF_COL + SF_SLOT_COLS * slot + 4 * SB + 8 * j;
+          const uint32_t sfa_t = col;
+          const uint32_t sfb_t = col + 4;
           const uint32_t a0 = smem_u32(sA), b0 = smem_u32(sB);
 #pragma unroll
           for (int q = 0; q < BK / 32; ++q) {
@@ -416,7 +409,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) gemm_mx_kernel(const __grid_co
           mma_commit(&empty[stage]);
         }
         __syncwarp();
-        if (j == SB - 1 || kb == KB - 1) slot ^= 1;
+        if (batch_end && ++sb == kSfBufs) {
+          sb = 0;
+          sphase ^= 1;
+        }
         if (++stage == kStages) {
           stage = 0;
           phase ^= 1;

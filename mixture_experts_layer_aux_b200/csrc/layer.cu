@@ -171,8 +171,9 @@ __global__ void __launch_bounds__(256) router_bwd_kernel(const float* __restrict
   float dgj = 0.f, gj = 0.f, sj = 0.f;
   int ej = -1;
   if (lane < k) {
-    const int r = row_of[(long long)t * k + lane];
-    for (int i = 0; i < nparts; ++i) dgj += dg_part[(long long)r * nparts + i];
+    const int r = row_of[(long long)t * k + lane];  // -1: dropped at capacity, dg = 0
+    if (r >= 0)
+      for (int i = 0; i < nparts; ++i) dgj += dg_part[(long long)r * nparts + i];
     gj = gates[(long long)t * k + lane];
     ej = idx[(long long)t * k + lane];
     sj = probs[(long long)t * E + ej];

@@ -21,6 +21,7 @@
 //            loads, one bf16 rounding.
 #include <cuda_fp8.h>
 
+#include <cmath>
 #include <mutex>
 
 #include "common.cuh"
@@ -102,8 +103,10 @@ __global__ void __launch_bounds__(RANK_WARPS * 32) rank_kernel(const int32_t* __
   }
 }
 
-// counts, offsets [E+1], base[b,e] = offsets[e] + sum_{b'<b} hist[b',e].
-__global__ void __launch_bounds__(512) scan_kernel(const int* __restrict__ hist, int nblk, int E,
+// counts, offsets [E+1], base[b,e] = offsets[e] + sum_{b'<b} hist[b',e]. With an expert
+// capacity `cap`, counts and offsets count min(count, cap) kept rows per expert; a pair
+// whose row base + rank reaches offsets[e+1] is then a dropped one.
+__global__ void __launch_bounds__(512) scan_kernel(const int* __restrict__ hist, int nblk, int E, int cap,
                                                    int* __restrict__ base, int32_t* __restrict__ counts,
                                                    int32_t* __restrict__ offsets) {
   __shared__ int s[512];
@@ -114,6 +117,7 @@ __global__ void __launch_bounds__(512) scan_kernel(const int* __restrict__ hist,
       base[(long long)b * E + e] = run;
       run += hist[(long long)b * E + e];
     }
+    run = min(run, cap);
     if (counts) counts[e] = run;
   }
   s[e] = (e < E) ? run : 0;
@@ -164,7 +168,8 @@ __device__ __forceinline__ uint2 quant8(const float (&f)[8], float inv) {
 template <int MODE, bool MX>
 __global__ void __launch_bounds__(SC_WARPS * 32) scatter_kernel(
     const __nv_bfloat16* __restrict__ x, int T, int H, int E, int k, const int32_t* __restrict__ idx,
-    const int32_t* __restrict__ lrank, const int* __restrict__ base, const float* __restrict__ gates,
+    const int32_t* __restrict__ lrank, const int* __restrict__ base, const int32_t* __restrict__ offsets,
+    const float* __restrict__ gates,
     int32_t* __restrict__ row_of, int32_t* __restrict__ src_of, float* __restrict__ row_gate, void* __restrict__ xp,
     uint8_t* __restrict__ xp_sf) {
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -178,7 +183,7 @@ __global__ void __launch_bounds__(SC_WARPS * 32) scatter_kernel(
       const int lr = lrank[(long long)t * k + lane];
       if (e >= 0 && e < E && lr >= 0) {
         r = base[(long long)(t / RANK_TOK) * E + e] + lr;
-        if (r >= rows_total) r = -1;
+        if (r >= offsets[e + 1]) r = -1;  // past the expert's capacity: dropped
       }
       row_of[(long long)t * k + lane] = r;
       if (r >= 0) {
@@ -355,17 +360,23 @@ int permute(const moe_config* c, const void* x, const int32_t* idx, const float*
   perm::rank_kernel<<<nblk, perm::RANK_WARPS * 32, 2 * perm::RANK_WARPS * c->E * sizeof(uint32_t), st>>>(
       idx, c->T, c->E, c->k, lrank, hist, status);
   MOE_CHECK_LAUNCH();
-  perm::scan_kernel<<<1, 512, 0, st>>>(hist, nblk, c->E, base, counts, offsets);
+  // expert capacity in rows (every pair when the config sets no capacity factor)
+  int cap = c->T * c->k;
+  if (c->capacity_factor > 0.f) {
+    const double cd = std::ceil((double)c->capacity_factor * c->T * c->k / c->E);
+    if (cd < (double)cap) cap = (int)cd;
+  }
+  perm::scan_kernel<<<1, 512, 0, st>>>(hist, nblk, c->E, cap, base, counts, offsets);
   MOE_CHECK_LAUNCH();
   const int sgrid = (c->T + perm::SC_WARPS - 1) / perm::SC_WARPS;
   if (mx)
     perm::scatter_kernel<0, true><<<sgrid, perm::SC_WARPS * 32, 0, st>>>(
-        static_cast<const __nv_bfloat16*>(x), c->T, c->H, c->E, c->k, idx, lrank, base, gates, row_of, src_of,
-        row_gate, xp, xp_sf);
+        static_cast<const __nv_bfloat16*>(x), c->T, c->H, c->E, c->k, idx, lrank, base, offsets, gates, row_of,
+        src_of, row_gate, xp, xp_sf);
   else
     perm::scatter_kernel<0, false><<<sgrid, perm::SC_WARPS * 32, 0, st>>>(
-        static_cast<const __nv_bfloat16*>(x), c->T, c->H, c->E, c->k, idx, lrank, base, gates, row_of, src_of,
-        row_gate, xp, nullptr);
+        static_cast<const __nv_bfloat16*>(x), c->T, c->H, c->E, c->k, idx, lrank, base, offsets, gates, row_of,
+        src_of, row_gate, xp, nullptr);
   MOE_CHECK_LAUNCH();
   return MOE_OK;
 }
@@ -373,7 +384,7 @@ int permute(const moe_config* c, const void* x, const int32_t* idx, const float*
 int scatter_rows(const moe_config* c, const void* x, const int32_t* row_of, void* xp, cudaStream_t st) {
   const int sgrid = (c->T + perm::SC_WARPS - 1) / perm::SC_WARPS;
   perm::scatter_kernel<1, false><<<sgrid, perm::SC_WARPS * 32, 0, st>>>(
-      static_cast<const __nv_bfloat16*>(x), c->T, c->H, c->E, c->k, nullptr, nullptr, nullptr, nullptr,
+      static_cast<const __nv_bfloat16*>(x), c->T, c->H, c->E, c->k, nullptr, nullptr, nullptr, nullptr, nullptr,
       const_cast<int32_t*>(row_of), nullptr, nullptr, xp, nullptr);
   MOE_CHECK_LAUNCH();
   return MOE_OK;

@@ -234,6 +234,7 @@ int check_cfg(const moe_config* c) {
   if (c->n_shared != 0 && c->n_shared != 1) return MOE_ERR_UNSUPPORTED;
   if (c->compute_aux && c->score != MOE_SCORE_SOFTMAX) return MOE_ERR_UNSUPPORTED;
   if ((long long)c->T * c->k >= (1LL << 31) / 2) return MOE_ERR_UNSUPPORTED;
+  if (!(c->capacity_factor >= 0.f) || c->capacity_factor > 1e30f) return MOE_ERR_INVALID_ARG;  // NaN, < 0, inf
   return MOE_OK;
 }
 

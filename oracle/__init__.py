@@ -227,11 +227,14 @@ def maps(idx: torch.Tensor, E: int, keep: torch.Tensor | None = None):
 
 def capacity_keep(idx: torch.Tensor, E: int, capacity_factor: float):
     """-> (keep uint8 [T,k], C): each expert keeps its first C = ceil(cf T k / E) pairs in
-    token order (cf <= 0: no limit, C = T k)."""
+    token order (cf <= 0: no limit, C = T k). cf is the layer configuration's value, an
+    IEEE float32 (so 0.6 means 0.60000002384...), and C is computed from it in double
+    precision as ((cf T) k) / E."""
     idx = _chk(idx.contiguous(), torch.int32)
     T, k = idx.shape
+    cf32 = float(torch.tensor(float(capacity_factor), dtype=torch.float32))
     keep = torch.empty((T, k), dtype=torch.uint8)
-    C = lib().oc_capacity_keep(T, E, k, ctypes.c_double(capacity_factor), _p(idx), _p(keep))
+    C = lib().oc_capacity_keep(T, E, k, ctypes.c_double(cf32), _p(idx), _p(keep))
     return keep, int(C)
 
 

@@ -77,7 +77,8 @@ def test_config_validation(lib, B):
     for bad, code in [(dict(k=9), UNSUPPORTED), (dict(k=0), INVALID), (dict(E=600, k=2), UNSUPPORTED),
                       (dict(H=200), UNSUPPORTED), (dict(F=100), UNSUPPORTED), (dict(T=0), INVALID),
                       (dict(score=5), INVALID), (dict(n_shared=2), UNSUPPORTED),
-                      (dict(compute_aux=1, score=1), UNSUPPORTED)]:
+                      (dict(compute_aux=1, score=1), UNSUPPORTED), (dict(capacity_factor=-1.0), INVALID),
+                      (dict(capacity_factor=float("nan")), INVALID), (dict(capacity_factor=float("inf")), INVALID)]:
         c = cfg(B, **bad)
         assert lib.moe_router_workspace_size(ctypes.byref(c)) == 0
         rc = lib.moe_router_topk(ctypes.byref(c), FAKE, FAKE, None, FAKE, None, FAKE, FAKE, None, None, FAKE, 1 << 30,

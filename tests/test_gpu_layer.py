@@ -37,7 +37,8 @@ def run_fwd(moe, wl, d, save=False):
 def routing_agreement(oracle, wl, h, gpu_idx):
     """Oracle logits + routing; returns (route dict, tokens whose indices agree)."""
     logits = oracle.router_logits(h["x"], h["W_r"], h.get("logit_bias"))
-    r = oracle.route(logits, wl.k, wl.score, wl.norm_topk, wl.route_scale, with_aux=wl.aux and wl.score == "softmax")
+    r = oracle.route(logits, wl.k, wl.score, wl.norm_topk, wl.route_scale, with_aux=wl.aux and wl.score == "softmax",
+                     capacity_factor=wl.capacity_factor)
     same = (gpu_idx.cpu() == r["idx"]).all(1)
     bound = 1e-4 * float(logits.pow(2).mean().sqrt())
     for t in (~same).nonzero().flatten().tolist():
@@ -69,8 +70,8 @@ def check_fwd(moe, oracle, wl, n_sample=None, seed=0):
         toks = torch.randperm(wl.T, generator=gen)[:n_sample].sort().values.to(torch.int32)
     toks = toks[same[toks.long()]]
     shared = (h["W_gs"], h["W_us"], h["W_ds"]) if wl.S else None
-    y_ref = oracle.moe_fwd_tokens(h["x"], h["W_g"], h["W_u"], h["W_d"], r["idx"], r["gates"], toks, shared=shared,
-                                  recipe="bf16")
+    y_ref = oracle.moe_fwd_tokens(h["x"], h["W_g"], h["W_u"], h["W_d"], r["idx_kept"], r["gates"], toks,
+                                  shared=shared, recipe="bf16")
     e = check_bf16(out["y"].cpu()[toks.long()], y_ref)[0]
     ge = (out["gates"].cpu().double()[toks.long()] - r["gates"][toks.long()]).abs().max().item()
     assert ge <= 1e-5, ge
@@ -95,6 +96,38 @@ def test_layer_fwd_small_cases_full_oracle(moe, oracle, wl):
 @pytest.mark.parametrize("name,n", [("mixtral", 48), ("qwen3", 96)])
 def test_layer_fwd_workload_sampled(moe, oracle, name, n):
     check_fwd(moe, oracle, WORKLOADS[name], n_sample=n)
+
+
+@pytest.mark.parametrize("cf", [0.6, 1.0])
+def test_layer_fwd_capacity_factor_full_oracle(moe, oracle, cf):
+    """Each expert keeps its first ceil(cf T k / E) pairs in token order; dropped pairs add nothing."""
+    wl = Workload("capacity", T=600, H=512, E=8, k=2, F=512, skew=True, capacity_factor=cf)
+    check_fwd(moe, oracle, wl)
+
+
+def test_permute_capacity_maps_bit_exact(moe, oracle):
+    """Capacity through moe_permute alone: kept counts, offsets and maps equal the oracle's, bit for bit."""
+    from mixture_experts_layer_aux_b200.synthetic import random_routing
+    T, E, k, H = 1000, 16, 4, 256
+    wl = Workload("cap-perm", T=T, H=H, E=E, k=k, F=128, capacity_factor=0.7)
+    cfg = moe.make_config(wl)
+    idx = random_routing(T, E, k, seed=4, hot=0.5)
+    x = torch.randn(T, H, generator=torch.Generator().manual_seed(2)).bfloat16()
+    xd, idd = x.cuda(), idx.cuda()
+    counts, offsets = empty((E,), torch.int32), empty((E + 1,), torch.int32)
+    row_of, src_of = empty((T, k), torch.int32), empty((T * k,), torch.int32)
+    xp = torch.zeros(T * k, H, dtype=torch.bfloat16, device="cuda")
+    moe.moe_permute(cfg, xd, idd, None, counts, offsets, row_of, src_of, None, xp, None,
+                    moe.workspace(moe.moe_permute_workspace_size(cfg)))
+    torch.cuda.synchronize()
+    keep, C = oracle.capacity_keep(idx, E, 0.7)
+    assert int((keep == 0).sum()) > 0
+    kc, off, ro, so = oracle.maps(idx, E, keep)
+    assert torch.equal(counts.cpu(), kc) and torch.equal(offsets.cpu(), off) and torch.equal(row_of.cpu(), ro)
+    n = int(off[-1])
+    assert torch.equal(src_of.cpu()[:n], so[:n])
+    assert torch.equal(xp.cpu()[:n].view(torch.int16), x[so[:n].long()].view(torch.int16))
+    assert moe.moe_get_device_status() == 0
 
 
 def test_layer_fwd_is_deterministic(moe):
@@ -146,14 +179,14 @@ def check_bwd(moe, oracle, wl, seed=0, d_aux=0.01, n_tok=None, experts=None):
     res["dlogits"] = err_rms(g["dlogits"].cpu()[toks.long()], dl)
     if experts is None:
         experts = list(range(wl.E))
-    dWg, dWu, dWd = oracle.moe_bwd_expert_dw(h["x"], h["W_g"], h["W_u"], h["W_d"], h["dY"], r["idx"], r["gates"],
-                                             experts, recipe="bf16")
+    dWg, dWu, dWd = oracle.moe_bwd_expert_dw(h["x"], h["W_g"], h["W_u"], h["W_d"], h["dY"], r["idx_kept"],
+                                             r["gates"], experts, recipe="bf16")
     ex = torch.tensor(experts).long()
     for name, ref in (("dW_g", dWg), ("dW_u", dWu), ("dW_d", dWd)):
         # the bar applies over the compared tensor (every compared expert's slice)
         res[name] = check_bf16(g[name].cpu()[ex], ref)[0]
         for q, e in enumerate(experts):
-            if int(r["counts"][e]) == 0:
+            if int(r["kept_counts"][e]) == 0:
                 assert (g[name][e] == 0).all(), (name, e)   # exact zeros for an expert with no token
             else:
                 # and no expert, however small, may be grossly off relative to its own size
@@ -179,6 +212,11 @@ def test_layer_bwd_small_full_oracle(moe, oracle):
 def test_layer_bwd_ragged_full_oracle(moe, oracle):
     wl = Workload("bwd-ragged", T=700, H=512, E=16, k=4, F=256, skew=True, bwd=True)
     check_bwd(moe, oracle, wl, seed=3, d_aux=0.5)
+
+
+def test_layer_bwd_capacity_factor_full_oracle(moe, oracle):
+    wl = Workload("bwd-capacity", T=512, H=256, E=8, k=2, F=512, skew=True, bwd=True, capacity_factor=0.8)
+    check_bwd(moe, oracle, wl, seed=2, d_aux=0.3)
 
 
 def test_layer_bwd_skewed_workload_sampled(moe, oracle):

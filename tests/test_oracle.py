@@ -314,7 +314,8 @@ def test_capacity_keep_matches_stable_sort_rank_and_maps_invariants(oracle, cf):
     T, E, k = 60, 6, 2
     idx = random_routing(T, E, k, seed=3, hot=0.6)
     keep, C = oracle.capacity_keep(idx, E, cf)
-    assert C == min(T * k, math.ceil(cf * T * k / E))
+    cf32 = float(torch.tensor(cf, dtype=torch.float32))  # the configuration carries cf as float32
+    assert C == min(T * k, math.ceil(cf32 * T * k / E))
     rank, counts = _stable_rank_within_expert(idx, E)
     assert torch.equal(keep.bool(), rank < C)
     kc, off, row_of, src_of = oracle.maps(idx, E, keep)
