@@ -281,10 +281,13 @@ class Layer:
         mark(6)
 
     def launches_per_step(self):
-        """Kernels of ours launched per step: router GEMM, top-k, finalize, rank, scan,
-        scatter, gate/up GEMM, down GEMM, unpermute (+ shared expert GEMMs, its
-        quantiser), and for fwd+bwd the nine kernels of moe_layer_bwd."""
-        n = 9
+        """Kernels of ours launched per step (as the ncu launch list shows them): router GEMM,
+        top-k, finalize (+ aux when computed), rank, scan, scatter, gate/up GEMM, down GEMM,
+        unpermute; + the shared expert's two GEMMs (and, for MXFP8, its input quantiser); and
+        for fwd+bwd the nine kernels of moe_layer_bwd (dY gather, down dgrad with the SwiGLU
+        backward, two weight-gradient GEMMs, gate/up dgrad, router backward, two router
+        GEMMs, dXp unpermute)."""
+        n = 9 + (1 if self.cfg.compute_aux else 0)
         if self.wl.S:
             n += 2 + (1 if self.mx else 0)
         if self.wl.bwd:
