@@ -40,6 +40,27 @@ from mixture_experts_layer_aux_b200.synthetic import WORKLOADS, make_inputs  # n
 PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
 
+def measured_traffic(workload: str):
+    """DRAM bytes per launch of the gate/up GEMM from the committed ncu capture, or None when the
+    capture is of another workload or the kernel's sources have changed since it was taken."""
+    import hashlib
+    import re
+    p = os.path.join(ROOT, "profiles", "gemm_gateup_mixtral.md")
+    if not os.path.exists(p):
+        return None
+    m = re.search(r"```json traffic\n(.*?)\n```", open(p).read(), re.S)
+    if not m:
+        return None
+    meta = json.loads(m.group(1))
+    if meta.get("workload") != workload:
+        return None
+    h = hashlib.sha256()
+    for f in meta["sources"]:
+        with open(os.path.join(ROOT, f), "rb") as fh:
+            h.update(fh.read())
+    return meta["dram_bytes_per_launch"] if h.hexdigest() == meta["sources_sha256"] else None
+
+
 def peaks():
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(p):
@@ -416,7 +437,8 @@ def run_ours(args, rank, ws):
         d_ms = stage_ms["gemm_down"]
         ach = flops_gateup / (g_ms * 1e-3) / 1e12
         roof = {"kernel": "grouped GEMM gate/up + SwiGLU epilogue", "bound": "tensor", "achieved": round(ach, 1),
-                "peak": peak_t, "unit": "TFLOP/s", "frac": round(ach / peak_t, 4), "traffic": None,
+                "peak": peak_t, "unit": "TFLOP/s", "frac": round(ach / peak_t, 4),
+                "traffic": measured_traffic(wl.name) if wl.dtype == "bf16" else None,
                 "peak_source": f"{P['source']}: {peak_note}"}
         hbm = P["hbm_gbs"]
         perm_bytes = T * H * 2 + rows * H * (1 + 1 / 32 if wl.dtype == "mxfp8" else 2) + 16 * rows
