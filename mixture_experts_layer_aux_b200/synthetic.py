@@ -47,6 +47,9 @@ class Workload:
     skew: bool = False         # add the skew logit bias
     bwd: bool = False          # the workload includes the backward pass
     capacity_factor: float = 0.0  # > 0: each expert keeps its first ceil(cf T k / E) pairs
+    n_group: int = 0           # > 1: group-limited routing over n_group groups of experts
+    topk_group: int = 0        # groups kept per token when n_group > 1
+    sel_bias: bool = False     # draw a per-expert selection bias (moves selection, not gates)
 
     def with_(self, **kw) -> "Workload":
         return replace(self, **kw)
@@ -124,6 +127,9 @@ def make_inputs(wl: Workload, device="cpu", seed: int = 0, with_dy: bool | None 
     if with_dy:
         d["dY"] = _randn_bf16((T, H), 1.0, gen, device)
     d["logit_bias"] = skew_bias(E).to(device) if wl.skew else None
+    # per-expert selection bias (drawn last so the other inputs do not change): uniform in
+    # [-0.1, 0.1), the order of the balancing corrections a DeepSeek-V3-style router carries
+    d["expert_bias"] = ((torch.rand((E,), generator=gen, device=device) - 0.5) * 0.2) if wl.sel_bias else None
     return d
 
 

@@ -196,6 +196,15 @@ def topk(logits: torch.Tensor, k: int) -> torch.Tensor:
     return idx
 
 
+def topk_grouped(sel: torch.Tensor, k: int, n_group: int = 0, topk_group: int = 0) -> torch.Tensor:
+    """Group-limited top-k on selection scores sel [T,E] (see oc_topk_grouped)."""
+    v = _chk(sel.to(torch.float64).contiguous(), torch.float64)
+    T, E = v.shape
+    idx = torch.empty((T, k), dtype=torch.int32)
+    lib().oc_topk_grouped(T, E, k, n_group, topk_group, _p(v), _p(idx))
+    return idx
+
+
 def gates(s: torch.Tensor, idx: torch.Tensor, norm: bool, route_scale: float) -> torch.Tensor:
     T, E = s.shape
     k = idx.shape[1]
@@ -244,7 +253,8 @@ def aux(s_softmax: torch.Tensor, counts: torch.Tensor, k: int) -> float:
 
 
 def route(logits: torch.Tensor, k: int, score: str = "softmax", norm: bool = True,
-          route_scale: float = 1.0, with_aux: bool = True, capacity_factor: float = 0.0) -> dict:
+          route_scale: float = 1.0, with_aux: bool = True, capacity_factor: float = 0.0,
+          expert_bias: torch.Tensor | None = None, n_group: int = 0, topk_group: int = 0) -> dict:
     """All routing steps from given logits: scores, top-k, gates, maps, aux.
 
     counts are the router's (every selected pair; they feed aux). With a capacity
@@ -253,11 +263,18 @@ def route(logits: torch.Tensor, k: int, score: str = "softmax", norm: bool = Tru
     row_of / src_of describe the kept rows only."""
     E = logits.shape[1]
     s = scores(logits, score)
-    idx = topk(logits, k)
+    if expert_bias is None and n_group <= 1:
+        idx = topk(logits, k)
+        sel = None
+    else:
+        # DeepSeek-V3 variant: selection on score + per-expert bias, group-limited
+        sel = s + (expert_bias.to(torch.float64) if expert_bias is not None else 0.0)
+        idx = topk_grouped(sel, k, n_group, topk_group)
     g = gates(s, idx, norm, route_scale)
     counts, offsets, row_of, src_of = maps(idx, E)
     out = dict(logits=logits, probs=s, idx=idx, gates=g, counts=counts, offsets=offsets,
-               row_of=row_of, src_of=src_of, idx_kept=idx, kept_counts=counts, keep=None, capacity=idx.numel())
+               row_of=row_of, src_of=src_of, idx_kept=idx, kept_counts=counts, keep=None, capacity=idx.numel(),
+               sel=sel)
     if capacity_factor > 0:
         keep, C = capacity_keep(idx, E, capacity_factor)
         kc, offsets, row_of, src_of = maps(idx, E, keep)
@@ -422,7 +439,9 @@ def layer_fwd(wl, inp: dict, toks=None, logits=None, mx_weights=None, recipe=Non
     if logits is None:
         logits = router_logits(inp["x"], inp["W_r"], inp.get("logit_bias"))
     r = route(logits.to(torch.float64), wl.k, wl.score, wl.norm_topk, wl.route_scale,
-              with_aux=wl.aux and wl.score == "softmax", capacity_factor=getattr(wl, "capacity_factor", 0.0))
+              with_aux=wl.aux and wl.score == "softmax", capacity_factor=getattr(wl, "capacity_factor", 0.0),
+              expert_bias=inp.get("expert_bias"), n_group=getattr(wl, "n_group", 0),
+              topk_group=getattr(wl, "topk_group", 0))
     mx = wl.dtype == "mxfp8"
     if recipe is None:
         recipe = "mxfp8" if mx else "exact"

@@ -322,6 +322,58 @@ void oc_topk(int T, int E, int k, const double* logits, int32_t* idx) {
     }
 }
 
+/*
+ * Group-limited top-k on selection scores (the DeepSeek-V3 router variant; the
+ * pages name DeepSeek-V3's routing but give no rule, so this is the reading):
+ * the E experts form n_group equal groups of consecutive indices; a group's
+ * score is the sum of its two largest selection scores (its one score when a
+ * group holds a single expert); the topk_group best groups are kept
+ * (descending, lower group index first on ties); then the k best experts of
+ * the kept groups by selection score (descending, lower index first). The
+ * selection score is sel[t,e] = s[t,e] + b[e], a per-expert bias that moves
+ * selection only, never the gate values. n_group <= 1 is plain top-k on sel.
+ */
+void oc_topk_grouped(int T, int E, int k, int n_group, int topk_group, const double* sel, int32_t* idx) {
+    int G = n_group > 1 ? E / n_group : E;
+    int ng = n_group > 1 ? n_group : 1;
+    int tg = n_group > 1 ? topk_group : 1;
+    double* gscore = (double*)malloc(sizeof(double) * ng);
+    int* gkeep = (int*)malloc(sizeof(int) * ng);
+    for (int t = 0; t < T; ++t) {
+        const double* v = sel + (long)t * E;
+        for (int g = 0; g < ng; ++g) {
+            double a1 = -INFINITY, a2 = -INFINITY;
+            for (int e = g * G; e < (g + 1) * G; ++e) {
+                if (v[e] > a1) { a2 = a1; a1 = v[e]; }
+                else if (v[e] > a2) { a2 = v[e]; }
+            }
+            gscore[g] = (G >= 2) ? a1 + a2 : a1;
+            gkeep[g] = 0;
+        }
+        for (int r = 0; r < tg; ++r) {
+            int best = -1;
+            for (int g = 0; g < ng; ++g) {
+                if (gkeep[g]) continue;
+                if (best < 0 || gscore[g] > gscore[best]) best = g;   /* strict: ties keep the lower group */
+            }
+            gkeep[best] = 1;
+        }
+        for (int j = 0; j < k; ++j) {
+            int best = -1;
+            for (int e = 0; e < E; ++e) {
+                if (!gkeep[e / G]) continue;
+                int taken = 0;
+                for (int i = 0; i < j; ++i) if (idx[(long)t * k + i] == e) taken = 1;
+                if (taken) continue;
+                if (best < 0 || v[e] > v[best]) best = e;
+            }
+            idx[(long)t * k + j] = best;
+        }
+    }
+    free(gscore);
+    free(gkeep);
+}
+
 /* gates[t,j] = s[t, idx[t,j]] (/ sum over the selected when norm) * route_scale */
 void oc_gates(int T, int E, int k, int norm, double route_scale, const double* s, const int32_t* idx,
               double* gates) {

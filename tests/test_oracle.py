@@ -294,6 +294,52 @@ def test_mxfp8_bf16_and_fp32_entry_points_agree(oracle):
     assert torch.equal(a[0], b[0]) and torch.equal(a[1], b[1])
 
 
+# --------------------------------------------------------------- group-limited routing (DeepSeek-V3 variant)
+
+
+def _torch_grouped_topk(sel, k, n_group, topk_group):
+    """The same rule with library sorts: group score = sum of the two largest in the group;
+    the topk_group best groups (stable descending sort: lower index first on ties); then the
+    k best experts of those groups."""
+    T, E = sel.shape
+    G = E // n_group
+    grp = sel.view(T, n_group, G)
+    gscore = torch.topk(grp, min(2, G), dim=-1).values.sum(-1)
+    gorder = torch.sort(-gscore, dim=1, stable=True).indices[:, :topk_group]
+    mask = torch.zeros(T, n_group, dtype=torch.bool)
+    mask.scatter_(1, gorder, True)
+    v = torch.where(mask.repeat_interleave(G, dim=1), sel, torch.full_like(sel, -float("inf")))
+    return torch.sort(-v, dim=1, stable=True).indices[:, :k].to(torch.int32)
+
+
+@pytest.mark.parametrize("E,n_group,topk_group,k", [(16, 4, 2, 3), (32, 8, 4, 8), (12, 3, 1, 2), (8, 8, 3, 3)])
+def test_grouped_topk_matches_library_sorts(oracle, E, n_group, topk_group, k):
+    g = torch.Generator().manual_seed(E + k)
+    sel = torch.rand(64, E, generator=g, dtype=torch.float64)
+    sel[::7, :] = torch.round(sel[::7, :] * 4) / 4            # some rows with many exact ties
+    idx = oracle.topk_grouped(sel, k, n_group, topk_group)
+    assert torch.equal(idx, _torch_grouped_topk(sel, k, n_group, topk_group))
+
+
+def test_grouped_topk_without_groups_or_bias_is_plain_topk(oracle):
+    l = random_logits(50, 16, seed=8).double()
+    s = oracle.scores(l, "sigmoid")
+    assert torch.equal(oracle.topk_grouped(s, 4, 0, 0), oracle.topk(l, 4))    # sigmoid is increasing
+    assert torch.equal(oracle.topk_grouped(s, 4, 4, 4), oracle.topk(l, 4))    # every group kept
+
+
+def test_selection_bias_moves_selection_not_gates(oracle):
+    l = random_logits(40, 16, seed=9).double()
+    b = torch.zeros(16, dtype=torch.float64)
+    b[5] = 10.0                                               # expert 5 wins every token's selection
+    r = oracle.route(l, 3, "sigmoid", True, 2.5, with_aux=False, expert_bias=b)
+    assert bool((r["idx"][:, 0] == 5).all())
+    s = torch.sigmoid(l)                                      # gates from the unbiased scores
+    ref = s.gather(1, r["idx"].long())
+    ref = ref / ref.sum(1, keepdim=True) * 2.5
+    assert torch.allclose(r["gates"], ref, rtol=1e-13, atol=0)
+
+
 # --------------------------------------------------------------- capacity factor
 
 
