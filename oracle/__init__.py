@@ -377,12 +377,20 @@ def unpermute(o, row_of, shared=None):
 
 # ----------------------------------------------------------------- backward
 
+def _mx_mats(mx, names):
+    return [_wmat(mx[n][0], mx[n][1]) for n in names]
+
+
 def moe_bwd_tokens(x, W_r, W_g, W_u, W_d, dY, r: dict, toks=None, *, score="softmax", norm=True,
-                   route_scale=1.0, aux_on=True, d_aux=0.0, recipe="exact"):
+                   route_scale=1.0, aux_on=True, d_aux=0.0, recipe="exact", mx=None):
     """dX[toks] (fp64, expert + router paths), dlogits[toks] [n,E] and dg [n,k] for routing r
-    (the dict returned by route())."""
+    (the dict returned by route()).
+
+    recipe "mxfp8" (the MXFP8 backward) takes mx = dict of (codes, scales) pairs: W_g, W_u, W_d
+    (the forward's, MXFP8 along their K) and W_dT [E,F,H], W_gT, W_uT [E,H,F] (transposed, MXFP8
+    along H resp. F); W_g, W_u, W_d are then ignored."""
     T, H = x.shape
-    E, F = W_g.shape[0], W_g.shape[1]
+    E, F = (mx["W_g"][0] if recipe == "mxfp8" else W_g).shape[:2]
     k = r["idx"].shape[1]
     if toks is None:
         toks = torch.arange(T, dtype=torch.int32)
@@ -392,27 +400,44 @@ def moe_bwd_tokens(x, W_r, W_g, W_u, W_d, dY, r: dict, toks=None, *, score="soft
     dl = torch.empty((n, E), dtype=torch.float64)
     dg = torch.empty((n, k), dtype=torch.float64)
     s_soft = r["probs"] if score == "softmax" else scores(r["logits"], "softmax")
-    ms = [mat(x), mat(W_r), _wmat(W_g), _wmat(W_u), _wmat(W_d), mat(dY)]
+    if recipe == "mxfp8":
+        wg, wu, wd, wdt, wgt, wut = _mx_mats(mx, ["W_g", "W_u", "W_d", "W_dT", "W_gT", "W_uT"])
+    else:
+        wg, wu, wd = _wmat(W_g), _wmat(W_u), _wmat(W_d)
+        wdt = wgt = wut = None
+    mdy = mat(dY)
+    ms = [mat(x), mat(W_r), wg, wu, wd]
+    tr = [m.ref if m is not None else None for m in (wdt, wgt, wut)]
     lib().oc_moe_bwd_tokens(T, H, E, k, F, 0 if score == "softmax" else 1, int(norm), ctypes.c_double(route_scale),
-                            int(aux_on), ctypes.c_double(d_aux), _recipe(recipe), *[m.ref for m in ms],
+                            int(aux_on), ctypes.c_double(d_aux), _recipe(recipe), *[m.ref for m in ms], *tr,
+                            mdy.ref,
                             _p(r["idx"]), _p(_chk(r["probs"], torch.float64)), _p(s_soft), _p(r["counts"]),
                             _p(_chk(r["keep"].contiguous(), torch.uint8)) if r.get("keep") is not None else None,
                             n, _p(toks), _p(dx), _p(dl), _p(dg))
     return dx, dl, dg
 
 
-def moe_bwd_expert_dw(x, W_g, W_u, W_d, dY, idx, g, experts, recipe="exact"):
-    """dW_g, dW_u [n,F,H] and dW_d [n,H,F] (fp64) for the listed experts."""
+def moe_bwd_expert_dw(x, W_g, W_u, W_d, dY, idx, g, experts, recipe="exact", mx=None):
+    """dW_g, dW_u [n,F,H] and dW_d [n,H,F] (fp64) for the listed experts.
+
+    recipe "mxfp8" takes mx as moe_bwd_tokens does (W_g, W_u, W_d, W_dT are used)."""
     T, H = x.shape
-    E, F = W_g.shape[0], W_g.shape[1]
+    E, F = (mx["W_g"][0] if recipe == "mxfp8" else W_g).shape[:2]
     k = idx.shape[1]
     experts = _chk(torch.as_tensor(experts, dtype=torch.int32).contiguous(), torch.int32)
     n = experts.numel()
     dWg = torch.empty((n, F, H), dtype=torch.float64)
     dWu = torch.empty((n, F, H), dtype=torch.float64)
     dWd = torch.empty((n, H, F), dtype=torch.float64)
-    ms = [mat(x), _wmat(W_g), _wmat(W_u), _wmat(W_d), mat(dY)]
-    lib().oc_moe_bwd_expert_dw(T, H, E, k, F, _recipe(recipe), *[m.ref for m in ms], _p(_chk(idx.contiguous(), torch.int32)),
+    if recipe == "mxfp8":
+        wg, wu, wd, wdt = _mx_mats(mx, ["W_g", "W_u", "W_d", "W_dT"])
+    else:
+        wg, wu, wd, wdt = _wmat(W_g), _wmat(W_u), _wmat(W_d), None
+    mdy = mat(dY)
+    ms = [mat(x), wg, wu, wd]
+    lib().oc_moe_bwd_expert_dw(T, H, E, k, F, _recipe(recipe), *[m.ref for m in ms],
+                               wdt.ref if wdt is not None else None, mdy.ref,
+                               _p(_chk(idx.contiguous(), torch.int32)),
                                _p(_chk(g.contiguous(), torch.float64)), n, _p(experts), _p(dWg), _p(dWu), _p(dWd))
     return dWg, dWu, dWd
 

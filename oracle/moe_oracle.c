@@ -262,6 +262,23 @@ static void mx_roundtrip(double* v, int n) {
     }
 }
 
+/* The same along a strided column: v[i * stride] for i in [0, n), in blocks of
+ * 32 consecutive i (the last block zero-padded; padding never changes amax). */
+static void mx_roundtrip_strided(double* v, long n, long stride) {
+    for (long b0 = 0; b0 < n; b0 += 32) {
+        long nb = n - b0 < 32 ? n - b0 : 32;
+        float t[32];
+        double amax = 0.0;
+        for (long i = 0; i < nb; ++i) {
+            t[i] = (float)v[(b0 + i) * stride];
+            if (fabs((double)t[i]) > amax) amax = fabs((double)t[i]);
+        }
+        uint8_t sb = oc_mx_scale_byte(amax);
+        double X = ldexp(1.0, (int)sb - 127);
+        for (long i = 0; i < nb; ++i) v[(b0 + i) * stride] = oc_e4m3_decode(oc_e4m3_encode((double)t[i] / X)) * X;
+    }
+}
+
 /* ------------------------------------------------------------ routing */
 
 /* logits[t,e] = sum_h x[t,h] W_r[e,h] (+ bias[e]); fp64 sum, one final rounding
@@ -660,6 +677,13 @@ int oc_expert_rows(int H, int F, int recipe, const oc_mat* xp, const int32_t* e_
  * dz_g and dz_u are rounded to bf16, each selected expert's contribution
  * W_g^T dz_g + W_u^T dz_u is rounded to bf16, and the router path uses dl
  * rounded to bf16 and rounds its result to bf16. dl itself stays unrounded.
+ * Under OC_MX (the MXFP8 backward): z is recomputed from MXFP8 x and the
+ * forward's MXFP8 weights and rounded to bf16 (the saved pre-activations);
+ * v = W_d^T dY takes WdT (W_d^T [E*F, H], MXFP8 along H) and dY in MXFP8 along
+ * H; dz_g, dz_u are rounded to bf16 and then to MXFP8 along F, and the gate/up
+ * dgrad takes WgT, WuT (W_g^T, W_u^T [E*H, F], MXFP8 along F); its result and
+ * the router path are rounded as under OC_BF16R. (WdT, WgT, WuT are unused
+ * otherwise and may be NULL.)
  * logits, s (scores), gates, idx and counts are the forward's (counts: every
  * selected pair, as the router counted them for aux). keep: NULL, or the
  * capacity mask of oc_capacity_keep: a dropped pair contributes nothing to y,
@@ -668,7 +692,8 @@ int oc_expert_rows(int H, int F, int recipe, const oc_mat* xp, const int32_t* e_
  */
 int oc_moe_bwd_tokens(int T, int H, int E, int k, int F, int score, int norm, double route_scale, int aux_on,
                       double d_aux, int recipe, const oc_mat* x, const oc_mat* Wr, const oc_mat* Wg,
-                      const oc_mat* Wu, const oc_mat* Wd, const oc_mat* dY, const int32_t* idx, const double* s_all,
+                      const oc_mat* Wu, const oc_mat* Wd, const oc_mat* WdT, const oc_mat* WgT, const oc_mat* WuT,
+                      const oc_mat* dY, const int32_t* idx, const double* s_all,
                       const double* s_softmax, const int32_t* counts, const uint8_t* keep, int n_tok,
                       const int32_t* toks, double* dx_out, double* dl_out, double* dg_out) {
     int i;
@@ -693,6 +718,20 @@ int oc_moe_bwd_tokens(int T, int H, int E, int k, int F, int score, int norm, do
         const double* s = s_all + (long)t * E;
         oc_row(x, t, xv);
         oc_row(dY, t, dy);
+        double* xe = xv;           /* the expert GEMMs' copy of x (MXFP8 along H under OC_MX) */
+        double* dye = dy;          /* dY as the down dgrad's operand */
+        double* xq = NULL;
+        double* dyq = NULL;
+        if (recipe == OC_MX) {
+            xq = (double*)malloc(sizeof(double) * H);
+            dyq = (double*)malloc(sizeof(double) * H);
+            memcpy(xq, xv, sizeof(double) * H);
+            memcpy(dyq, dy, sizeof(double) * H);
+            mx_roundtrip(xq, H);
+            mx_roundtrip(dyq, H);
+            xe = xq;
+            dye = dyq;
+        }
         for (int h = 0; h < H; ++h) dx[h] = 0.0;
         for (int e = 0; e < E; ++e) dl[e] = 0.0;
         /* gates again from the scores (as the forward defined them) */
@@ -712,28 +751,46 @@ int oc_moe_bwd_tokens(int T, int H, int E, int k, int F, int score, int norm, do
             oc_mat we_g = oc_slice(Wg, (int64_t)e * F, F);
             oc_mat we_u = oc_slice(Wu, (int64_t)e * F, F);
             oc_mat we_d = oc_slice(Wd, (int64_t)e * H, H);
-            expert_act(&we_g, &we_u, xv, zg, zu, a, rowbuf);
-            if (recipe == OC_BF16R) {
-                round_vec(zg, F, recipe);
-                round_vec(zu, F, recipe);
+            expert_act(&we_g, &we_u, xe, zg, zu, a, rowbuf);
+            if (recipe == OC_BF16R || recipe == OC_MX) {
+                /* the backward reads the forward's gate/up pre-activations saved in bf16 */
+                for (int f = 0; f < F; ++f) { zg[f] = oc_bf16_round(zg[f]); zu[f] = oc_bf16_round(zu[f]); }
                 for (int f = 0; f < F; ++f) a[f] = silu(zg[f]) * zu[f];
             }
-            for (int f = 0; f < F; ++f) v[f] = 0.0;
-            matvec_t_acc(&we_d, dy, v, rowbuf);           /* v = W_d^T dY_t */
+            if (recipe == OC_MX) {
+                oc_mat wt_d = oc_slice(WdT, (int64_t)e * F, F);   /* W_d^T [F, H], MXFP8 along H */
+                matvec(&wt_d, dye, v, rowbuf);                      /* v = W_d^T dY_t */
+            } else {
+                for (int f = 0; f < F; ++f) v[f] = 0.0;
+                matvec_t_acc(&we_d, dy, v, rowbuf);           /* v = W_d^T dY_t */
+            }
             dg[j] = dot(v, a, F);
             for (int f = 0; f < F; ++f) {
                 double da = g[j] * v[f];
                 dzg[f] = da * zu[f] * silu_grad(zg[f]);
                 dzu[f] = da * silu(zg[f]);
             }
-            if (recipe == OC_BF16R) {
-                round_vec(dzg, F, recipe);
-                round_vec(dzu, F, recipe);
+            if (recipe == OC_BF16R || recipe == OC_MX) {
+                for (int f = 0; f < F; ++f) { dzg[f] = oc_bf16_round(dzg[f]); dzu[f] = oc_bf16_round(dzu[f]); }
             }
             for (int h = 0; h < H; ++h) dxp[h] = 0.0;
-            matvec_t_acc(&we_g, dzg, dxp, rowbuf);
-            matvec_t_acc(&we_u, dzu, dxp, rowbuf);
-            if (recipe == OC_BF16R) round_vec(dxp, H, recipe);
+            if (recipe == OC_MX) {
+                /* dgate/dup as the gate/up dgrad's operand: MXFP8 along F; W_g^T, W_u^T [H, F] MXFP8 along F */
+                mx_roundtrip(dzg, F);
+                mx_roundtrip(dzu, F);
+                oc_mat wt_g = oc_slice(WgT, (int64_t)e * H, H);
+                oc_mat wt_u = oc_slice(WuT, (int64_t)e * H, H);
+                double* tmp = (double*)malloc(sizeof(double) * H);
+                matvec(&wt_g, dzg, tmp, rowbuf);
+                for (int h = 0; h < H; ++h) dxp[h] += tmp[h];
+                matvec(&wt_u, dzu, tmp, rowbuf);
+                for (int h = 0; h < H; ++h) dxp[h] += tmp[h];
+                free(tmp);
+            } else {
+                matvec_t_acc(&we_g, dzg, dxp, rowbuf);
+                matvec_t_acc(&we_u, dzu, dxp, rowbuf);
+            }
+            if (recipe == OC_BF16R || recipe == OC_MX) round_vec(dxp, H, OC_BF16R);
             for (int h = 0; h < H; ++h) dx[h] += dxp[h];
         }
         if (dg_out) for (int j = 0; j < k; ++j) dg_out[(long)i * k + j] = dg[j];
@@ -784,13 +841,14 @@ int oc_moe_bwd_tokens(int T, int H, int E, int k, int F, int score, int norm, do
         /* router path */
         for (int h = 0; h < H; ++h) dxp[h] = 0.0;
         for (int e = 0; e < E; ++e) {
-            double c = (recipe == OC_BF16R) ? oc_bf16_round(dl[e]) : dl[e];
+            double c = (recipe == OC_BF16R || recipe == OC_MX) ? oc_bf16_round(dl[e]) : dl[e];
             if (c == 0.0) continue;
             oc_row(Wr, e, rowbuf);
             for (int h = 0; h < H; ++h) dxp[h] += c * rowbuf[h];
         }
-        if (recipe == OC_BF16R) round_vec(dxp, H, recipe);
+        if (recipe == OC_BF16R || recipe == OC_MX) round_vec(dxp, H, OC_BF16R);
         for (int h = 0; h < H; ++h) dx[h] += dxp[h];
+        free(xq); free(dyq);
         free(xv); free(dy); free(zg); free(zu); free(a); free(v); free(dzg); free(dzu); free(dxp); free(rowbuf);
         free(dg); free(g);
     }
@@ -805,9 +863,15 @@ int oc_moe_bwd_tokens(int T, int H, int E, int k, int F, int score, int norm, do
  * get exact zeros. gates are the forward's [T,k]. Under OC_BF16R, g a is the
  * forward's bf16 activation (from the unrounded z), and dz_g, dz_u are the
  * bf16 values of the backward (from the saved bf16 z, rounded).
+ * Under OC_MX (the MXFP8 backward): z is recomputed from MXFP8 x and weights
+ * and rounded to bf16 (the saved pre-activations), g a is recomputed from it;
+ * v = W_d^T dY uses WdT (W_d^T [E*F, H], MXFP8 along H) and dY in MXFP8 along
+ * H; dz_g, dz_u are rounded to bf16; then every weight-gradient operand (g a,
+ * dz_g, dz_u, x, dY) is quantised to MXFP8 along the expert's tokens, in blocks
+ * of 32 consecutive tokens of its stable order.
  */
 int oc_moe_bwd_expert_dw(int T, int H, int E, int k, int F, int recipe, const oc_mat* x, const oc_mat* Wg,
-                         const oc_mat* Wu, const oc_mat* Wd, const oc_mat* dY, const int32_t* idx,
+                         const oc_mat* Wu, const oc_mat* Wd, const oc_mat* WdT, const oc_mat* dY, const int32_t* idx,
                          const double* gates, int n_exp, const int32_t* exps, double* dWg, double* dWu,
                          double* dWd) {
     (void)E;
@@ -850,26 +914,60 @@ int oc_moe_bwd_expert_dw(int T, int H, int E, int k, int F, int recipe, const oc
             double* a = A + (long)i * F;
             oc_row(x, tl[i], xv);
             oc_row(dY, tl[i], dy);
-            expert_act(&we_g, &we_u, xv, zg, zu, a, rowbuf);
-            /* A holds the down projection's operand g a */
-            for (int f = 0; f < F; ++f) a[f] *= gl[i];
-            if (recipe == OC_BF16R) {
-                round_vec(a, F, recipe);
-                round_vec(zg, F, recipe);
-                round_vec(zu, F, recipe);
+            if (recipe == OC_MX) {
+                /* the forward's gate/up GEMM saw x in MXFP8 along H; its bf16 pre-activations were
+                 * saved, and the backward recomputes g a from them */
+                double* xq = (double*)malloc(sizeof(double) * H);
+                double* dyq = (double*)malloc(sizeof(double) * H);
+                memcpy(xq, xv, sizeof(double) * H);
+                memcpy(dyq, dy, sizeof(double) * H);
+                mx_roundtrip(xq, H);
+                mx_roundtrip(dyq, H);
+                expert_act(&we_g, &we_u, xq, zg, zu, a, rowbuf);
+                for (int f = 0; f < F; ++f) { zg[f] = oc_bf16_round(zg[f]); zu[f] = oc_bf16_round(zu[f]); }
+                for (int f = 0; f < F; ++f) a[f] = gl[i] * silu(zg[f]) * zu[f];
+                oc_mat wt_d = oc_slice(WdT, (int64_t)e * F, F);
+                matvec(&wt_d, dyq, v, rowbuf);                      /* v = W_d^T dY_t, MXFP8 along H */
+                free(xq);
+                free(dyq);
+            } else {
+                expert_act(&we_g, &we_u, xv, zg, zu, a, rowbuf);
+                /* A holds the down projection's operand g a */
+                for (int f = 0; f < F; ++f) a[f] *= gl[i];
+                if (recipe == OC_BF16R) {
+                    round_vec(a, F, recipe);
+                    round_vec(zg, F, recipe);
+                    round_vec(zu, F, recipe);
+                }
+                for (int f = 0; f < F; ++f) v[f] = 0.0;
+                matvec_t_acc(&we_d, dy, v, rowbuf);
             }
-            for (int f = 0; f < F; ++f) v[f] = 0.0;
-            matvec_t_acc(&we_d, dy, v, rowbuf);
             for (int f = 0; f < F; ++f) {
                 double da = gl[i] * v[f];
                 DZG[(long)i * F + f] = da * zu[f] * silu_grad(zg[f]);
                 DZU[(long)i * F + f] = da * silu(zg[f]);
             }
-            if (recipe == OC_BF16R) {
-                round_vec(DZG + (long)i * F, F, recipe);
-                round_vec(DZU + (long)i * F, F, recipe);
+            if (recipe == OC_BF16R || recipe == OC_MX) {
+                round_vec(DZG + (long)i * F, F, OC_BF16R);
+                round_vec(DZU + (long)i * F, F, OC_BF16R);
             }
             free(zg); free(zu); free(v); free(rowbuf);
+        }
+        if (recipe == OC_MX) {
+            /* weight-gradient GEMM operands: MXFP8 along the expert's tokens (K = its rows), in blocks of
+             * 32 consecutive tokens of its stable order; x and dY from their bf16 values */
+            int c;
+#pragma omp parallel for schedule(static)
+            for (c = 0; c < F; ++c) {
+                mx_roundtrip_strided(A + c, n, F);
+                mx_roundtrip_strided(DZG + c, n, F);
+                mx_roundtrip_strided(DZU + c, n, F);
+            }
+#pragma omp parallel for schedule(static)
+            for (c = 0; c < H; ++c) {
+                mx_roundtrip_strided(XV + c, n, H);
+                mx_roundtrip_strided(DY + c, n, H);
+            }
         }
         int f;
 #pragma omp parallel for schedule(static)

@@ -571,3 +571,94 @@ def test_bf16_recipe_backward_stays_near_exact(oracle):
     # the router-gradient operand: dl rounded to bf16
     d_r = oracle.router_dwr(dl0, inp["x"], round_dl=True)
     assert torch.allclose(d_r, dl0.float().bfloat16().double().T @ inp["x"].double(), rtol=1e-12, atol=1e-12)
+
+
+# --------------------------------------------------------------- MXFP8 backward
+
+
+def _mxq(t):
+    """MXFP8 round trip along the last dim (fp32 in), with the pinned quantiser."""
+    c, s = oracle_mod().mxfp8_quantize(t.float().contiguous())
+    return oracle_mod().mxfp8_decode(c, s)
+
+
+def _mxq_rows(t):
+    """MXFP8 round trip along dim 0 in blocks of 32 rows (zero-padded at the end)."""
+    n = t.shape[0]
+    pad = (-n) % 32
+    tp = torch.cat([t, torch.zeros(pad, t.shape[1], dtype=t.dtype)]) if pad else t
+    return _mxq(tp.T.contiguous()).T[:n]
+
+
+def oracle_mod():
+    import oracle
+    return oracle
+
+
+def _mx_bwd_case(seed=31):
+    wl = small(T=40, H=64, E=3, k=2, F=64, bwd=True)
+    inp = make_inputs(wl, seed=seed, with_dy=True)
+    o = oracle_mod()
+    mx = {n: o.mxfp8_quantize(inp[n]) for n in ("W_g", "W_u", "W_d")}
+    mx["W_dT"] = o.mxfp8_quantize(inp["W_d"].transpose(1, 2).contiguous())
+    mx["W_gT"] = o.mxfp8_quantize(inp["W_g"].transpose(1, 2).contiguous())
+    mx["W_uT"] = o.mxfp8_quantize(inp["W_u"].transpose(1, 2).contiguous())
+    return wl, inp, mx
+
+
+def test_mxfp8_backward_composes_from_quantised_operands(oracle):
+    """The MXFP8 backward equals fp64 products of the operands rounded at the recipe's points:
+    dY and x along H, W_d^T along H, dgate/dup to bf16 then along F, W_g^T / W_u^T along F, and
+    for the weight gradients every operand along the expert's tokens (torch fp64 + the pinned
+    quantiser; a transposed operand or a missing rounding point fails it)."""
+    wl, inp, mx = _mx_bwd_case()
+    r = oracle.route(oracle.router_logits(inp["x"], inp["W_r"]).double(), wl.k, with_aux=False)
+    dx, dl, dg = oracle.moe_bwd_tokens(inp["x"], inp["W_r"], None, None, None, inp["dY"], r, aux_on=False,
+                                       recipe="mxfp8", mx=mx)
+    dWg, dWu, dWd = oracle.moe_bwd_expert_dw(inp["x"], None, None, None, inp["dY"], r["idx"], r["gates"],
+                                             list(range(wl.E)), recipe="mxfp8", mx=mx)
+    dec = {n: oracle.mxfp8_decode(*mx[n]) for n in mx}
+    x, dY = inp["x"].double(), inp["dY"].double()
+    xq, dYq = _mxq(x), _mxq(dY)
+    bf = lambda t: t.float().bfloat16().double()
+    silu = torch.nn.functional.silu
+    ref_dx = torch.zeros_like(x)
+    rows = {e: [] for e in range(wl.E)}
+    for t in range(wl.T):
+        for j in range(wl.k):
+            e, g = int(r["idx"][t, j]), float(r["gates"][t, j])
+            zg, zu = bf(xq[t] @ dec["W_g"][e].T), bf(xq[t] @ dec["W_u"][e].T)
+            v = dec["W_dT"][e] @ dYq[t]
+            sg = torch.sigmoid(zg)
+            dzg = bf(g * v * zu * sg * (1 + zg * (1 - sg)))
+            dzu = bf(g * v * silu(zg))
+            assert abs(float(v @ (silu(zg) * zu)) - float(dg[t, j])) <= 1e-12 * max(1.0, abs(float(dg[t, j])))
+            ref_dx[t] += bf(dec["W_gT"][e] @ _mxq(dzg[None])[0] + dec["W_uT"][e] @ _mxq(dzu[None])[0])
+            rows[e].append((t, g * silu(zg) * zu, dzg, dzu))
+    router = bf(bf(dl) @ inp["W_r"].double())                 # the router path, rounded as under bf16
+    assert torch.allclose(dx, ref_dx + router, rtol=0, atol=1e-12)
+    for e in range(wl.E):
+        ts = torch.tensor([q[0] for q in rows[e]])
+        A = _mxq_rows(torch.stack([q[1] for q in rows[e]]))
+        DZG = _mxq_rows(torch.stack([q[2] for q in rows[e]]))
+        DZU = _mxq_rows(torch.stack([q[3] for q in rows[e]]))
+        X, DY = _mxq_rows(x[ts]), _mxq_rows(dY[ts])
+        assert torch.allclose(dWd[e], DY.T @ A, rtol=1e-12, atol=1e-13)
+        assert torch.allclose(dWg[e], DZG.T @ X, rtol=1e-12, atol=1e-13)
+        assert torch.allclose(dWu[e], DZU.T @ X, rtol=1e-12, atol=1e-13)
+
+
+def test_mxfp8_backward_stays_near_exact(oracle):
+    wl, inp, mx = _mx_bwd_case(seed=32)
+    r = oracle.route(oracle.router_logits(inp["x"], inp["W_r"]).double(), wl.k, with_aux=False)
+    args = (inp["x"], inp["W_r"], inp["W_g"], inp["W_u"], inp["W_d"], inp["dY"], r)
+    dx_e, _, _ = oracle.moe_bwd_tokens(*args, aux_on=False)
+    dx_m, _, _ = oracle.moe_bwd_tokens(*args, aux_on=False, recipe="mxfp8", mx=mx)
+    gw_e = oracle.moe_bwd_expert_dw(inp["x"], inp["W_g"], inp["W_u"], inp["W_d"], inp["dY"], r["idx"], r["gates"],
+                                    [0, 1, 2])
+    gw_m = oracle.moe_bwd_expert_dw(inp["x"], None, None, None, inp["dY"], r["idx"], r["gates"], [0, 1, 2],
+                                    recipe="mxfp8", mx=mx)
+    rms = lambda t: float(t.pow(2).mean().sqrt())
+    assert rms(dx_m - dx_e) <= 0.08 * rms(dx_e)
+    for a, b in zip(gw_m, gw_e):
+        assert rms(a - b) <= 0.12 * rms(b)
