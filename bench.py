@@ -78,8 +78,11 @@ DATA = "synthetic (seeded; x~N(0,1), weights~N(0,0.02^2), bf16)"
 
 
 def workload_config(wl, ws):
+    variant = (f" groups {wl.topk_group}/{wl.n_group}" if wl.n_group > 1 else "") + \
+        (" +selection bias" if wl.sel_bias else "") + \
+        (f" capacity {wl.capacity_factor}" if wl.capacity_factor > 0 else "")
     return {"workload": f"{wl.name}: {'fwd+bwd' if wl.bwd else 'fwd'} T={wl.T} H={wl.H} E={wl.E} k={wl.k} "
-                        f"F={wl.F}{' +1 shared' if wl.S else ''} {wl.score} {wl.dtype}",
+                        f"F={wl.F}{' +1 shared' if wl.S else ''} {wl.score} {wl.dtype}{variant}",
             "T": wl.T, "H": wl.H, "E": wl.E, "k": wl.k, "F": wl.F, "shared": wl.S,
             "parallelism": f"replicas x{ws} (no data-path collective)",
             "l2": (f"inputs larger than L2 (expert weights {wl.expert_weight_bytes() / 1e9:.1f} GB vs 126 MB), "
@@ -268,7 +271,7 @@ class Layer:
                 ev[i].record()
         mark(0)
         m.moe_router_topk(c, d["x"], d["W_r"], d["logit_bias"], self.logits, self.probs, self.idx, self.gates,
-                          self.counts, self.aux, self.ws_r)
+                          self.counts, self.aux, self.ws_r, expert_bias=d.get("expert_bias"))
         mark(1)
         m.moe_permute(c, d["x"], self.idx, self.gates, None, self.offsets, self.row_of, self.src_of, self.row_gate,
                       self.xp, self.xp_sf, self.ws_p)
@@ -325,7 +328,7 @@ class Layer:
             (a, sa), (b, sb), (e, se) = self.w("W_gs"), self.w("W_us"), self.w("W_ds")
             sh = [a, b, e, sa, sb, se]
         m.moe_layer_fwd(c, x, d["W_r"], d["logit_bias"], Wg, Wu, Wd, sg, su, sd, *sh, y, aux, None, None, None, None,
-                        self.saved, self.ws_layer)
+                        self.saved, self.ws_layer, expert_bias=d.get("expert_bias"))
 
     def bwd_call(self):
         m, c, d = self.moe, self.cfg, self.d

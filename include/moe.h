@@ -79,6 +79,11 @@ typedef struct moe_config {
                               no expert gradient). The router's counts and aux still count
                               every selected pair; the permutation's counts and offsets
                               count the kept rows. NaN or negative: MOE_ERR_INVALID_ARG. */
+    int32_t n_group;       /* 0 or 1: top-k over all experts. 2..32: group-limited routing (the
+                              DeepSeek-V3 router shape): experts form n_group groups of E/n_group
+                              consecutive indices, and the k experts are chosen within the
+                              topk_group best groups (see moe_router_topk). E % n_group == 0. */
+    int32_t topk_group;    /* groups kept per token when n_group > 1; k <= topk_group E/n_group */
 } moe_config;
 
 /* Human-readable name of a status code (static string). */
@@ -99,11 +104,19 @@ int moe_get_device_status(int32_t* word_out, int clear);
  *     lower expert index first (selection on logits = selection on scores);
  *   gates[t,j] = score / (sum of the selected scores if norm_topk) * route_scale;
  *   counts[e] = number of (t,j) with idx[t,j] == e;
+ *   DeepSeek-V3 variant (expert_bias != NULL or cfg->n_group > 1): selection
+ *     runs on sel[t,e] = score[t,e] + expert_bias[e] instead of the logits
+ *     (the bias balances load by moving selection only, never the gate
+ *     values); with n_group > 1 a group's score is the sum of its two largest
+ *     sel values, the topk_group best groups are kept (score descending, lower
+ *     group index first), and the k largest sel among their experts are chosen
+ *     (descending, lower index first);
  *   aux = E * sum_e (counts[e] / (T k)) * mean_t probs[t,e]  (softmax only;
  *     the load-balancing loss named in 2.4 of the summary and 案例 3 of the
  *     study notes; unscaled -- the caller applies its coefficient).
  * Arguments:
- *   x [T,H] bf16, W_r [E,H] bf16, logit_bias [E] fp32 or NULL.
+ *   x [T,H] bf16, W_r [E,H] bf16, logit_bias [E] fp32 or NULL (added to the
+ *   logits), expert_bias [E] fp32 or NULL (selection only, as above).
  *   If x == NULL and W_r == NULL, `logits` is an INPUT [T,E] fp32 and only the
  *   routing steps run (logit_bias is then ignored).
  *   logits [T,E] fp32 out (required), probs [T,E] fp32 out or NULL,
@@ -112,8 +125,8 @@ int moe_get_device_status(int32_t* word_out, int clear);
  * ------------------------------------------------------------------------ */
 size_t moe_router_workspace_size(const moe_config* cfg);
 int moe_router_topk(const moe_config* cfg, const void* x, const void* W_r, const float* logit_bias,
-                    float* logits, float* probs, int32_t* idx, float* gates, int32_t* counts, float* aux,
-                    void* ws, size_t ws_bytes, void* stream);
+                    const float* expert_bias, float* logits, float* probs, int32_t* idx, float* gates,
+                    int32_t* counts, float* aux, void* ws, size_t ws_bytes, void* stream);
 
 /* ------------------------------------------------------------------------
  * Permutation into expert-contiguous order (memory-efficient permutation,
@@ -234,9 +247,42 @@ int moe_unpermute(const moe_config* cfg, const void* o, const int32_t* row_of, c
 int moe_quantize_mxfp8(const void* src, int64_t rows, int32_t K, uint8_t* dst, uint8_t* sf, void* stream);
 
 /* ------------------------------------------------------------------------
+ * Transposed MXFP8 operands of the MXFP8 backward (the same 1x32 quantiser,
+ * blocks along the backward GEMM's K).
+ *
+ * moe_quantize_mxfp8_t: weights. src [batch, R, C] bf16 -> dst [batch, C, ldd]
+ *   e4m3 with dst[b, c, r] the code of src[b, r, c], quantised in blocks of
+ *   32 consecutive r; sf [batch, C, ldd/32]. R % 32 == 0, C % 8 == 0,
+ *   ldd >= R and ldd % 32 == 0 (ldd > R leaves room to place W_g^T and W_u^T
+ *   side by side in one [E, H, 2F] buffer: pass dst + F, sf + F/32).
+ *   Once per weight update: W_d [E,H,F] -> W_d^T [E,F,H] (blocks along H),
+ *   W_g, W_u [E,F,H] -> W_g^T | W_u^T [E,H,2F] (blocks along F).
+ *
+ * moe_quantize_mxfp8_t_grouped: activations of the weight-gradient GEMMs,
+ *   quantised along the tokens of each expert. The T*k permuted rows are
+ *   grouped by offsets [E+1]; poff [E+1] (out) receives the padded offsets
+ *   (each expert's segment rounded up to a multiple of 128 rows), and
+ *   dst [C, ldd] e4m3 / sf [C, ldd/32] ue8m0 receive, for expert e and its
+ *   i-th row, dst[c, poff[e] + i] = the code of that row's column c, in
+ *   blocks of 32 consecutive padded rows (pad rows are zero). The source row
+ *   of permuted row r is, by mode: 0 src[r] (src [T*k, C]); 1 src[src_of[r]]
+ *   (src [T, C], e.g. x or dY through the permutation); 2 the gate-folded
+ *   activation row_gate[r] * silu(gate) * up recomputed from the saved
+ *   pre-activations src [T*k, 2C] (gate columns, then up). C % 8 == 0;
+ *   ldd >= moe_mxfp8_t_padded_rows(cfg) and ldd % 512 == 0.
+ * ------------------------------------------------------------------------ */
+int moe_quantize_mxfp8_t(const void* src, int32_t batch, int32_t R, int32_t C, void* dst, int64_t ldd, uint8_t* sf,
+                         void* stream);
+int64_t moe_mxfp8_t_padded_rows(const moe_config* cfg);
+int moe_quantize_mxfp8_t_grouped(const moe_config* cfg, int32_t mode, const void* src, const int32_t* src_of,
+                                 const float* row_gate, const int32_t* offsets, int32_t* poff, int32_t C, void* dst,
+                                 int64_t ldd, uint8_t* sf, void* stream);
+
+/* ------------------------------------------------------------------------
  * Whole layer, forward: router -> permute -> GEMM gate/up (SwiGLU, gate
  * folded) -> GEMM down -> [shared expert] -> unpermute-sum.
- *   x [T,H] bf16; W_r [E,H] bf16; logit_bias [E] fp32 or NULL;
+ *   x [T,H] bf16; W_r [E,H] bf16; logit_bias [E] fp32 or NULL; expert_bias [E]
+ *   fp32 or NULL (the router's selection bias, see moe_router_topk);
  *   BF16: W_g, W_u [E,F,H], W_d [E,H,F] bf16, *_sf NULL;
  *   MXFP8: the same tensors as e4m3 with ue8m0 scales (W_g_sf, W_u_sf
  *     [E,F,H/32], W_d_sf [E,H,F/32]), as moe_quantize_mxfp8 produces them;
@@ -249,8 +295,8 @@ int moe_quantize_mxfp8(const void* src, int64_t rows, int32_t K, uint8_t* dst, u
  * ------------------------------------------------------------------------ */
 size_t moe_layer_workspace_size(const moe_config* cfg);
 size_t moe_layer_saved_size(const moe_config* cfg);
-int moe_layer_fwd(const moe_config* cfg, const void* x, const void* W_r, const float* logit_bias, const void* W_g,
-                  const void* W_u, const void* W_d, const uint8_t* W_g_sf, const uint8_t* W_u_sf,
+int moe_layer_fwd(const moe_config* cfg, const void* x, const void* W_r, const float* logit_bias,
+                  const float* expert_bias, const void* W_g, const void* W_u, const void* W_d, const uint8_t* W_g_sf, const uint8_t* W_u_sf,
                   const uint8_t* W_d_sf, const void* Ws_g, const void* Ws_u, const void* Ws_d,
                   const uint8_t* Ws_g_sf, const uint8_t* Ws_u_sf, const uint8_t* Ws_d_sf, void* y, float* aux,
                   int32_t* idx, float* gates, int32_t* counts, int32_t* offsets, void* saved, void* ws,

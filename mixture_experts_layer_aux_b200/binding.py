@@ -35,7 +35,7 @@ class moe_config(ctypes.Structure):
                 ("F", ctypes.c_int32), ("n_shared", ctypes.c_int32), ("score", ctypes.c_int32),
                 ("norm_topk", ctypes.c_int32), ("route_scale", ctypes.c_float), ("expert_dtype", ctypes.c_int32),
                 ("compute_aux", ctypes.c_int32), ("save_for_bwd", ctypes.c_int32),
-                ("capacity_factor", ctypes.c_float)]
+                ("capacity_factor", ctypes.c_float), ("n_group", ctypes.c_int32), ("topk_group", ctypes.c_int32)]
 
 
 _VP = ctypes.c_void_p
@@ -47,7 +47,7 @@ _SIGS = {
     "moe_status_string": (ctypes.c_char_p, [_I]),
     "moe_get_device_status": (_I, [ctypes.POINTER(ctypes.c_int32), _I]),
     "moe_router_workspace_size": (_SZ, [_CFG]),
-    "moe_router_topk": (_I, [_CFG, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _SZ, _VP]),
+    "moe_router_topk": (_I, [_CFG, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _SZ, _VP]),
     "moe_permute_workspace_size": (_SZ, [_CFG]),
     "moe_permute": (_I, [_CFG, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _SZ, _VP]),
     "moe_permute_noalloc_scratch_capacity": (_SZ, []),
@@ -60,11 +60,16 @@ _SIGS = {
     "moe_quantize_mxfp8": (_I, [_VP, ctypes.c_int64, ctypes.c_int32, _VP, _VP, _VP]),
     "moe_layer_workspace_size": (_SZ, [_CFG]),
     "moe_layer_saved_size": (_SZ, [_CFG]),
-    "moe_layer_fwd": (_I, [_CFG, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP,
+    "moe_layer_fwd": (_I, [_CFG, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP,
                            _VP, _VP, _VP, _VP, _VP, _VP, _VP, _SZ, _VP]),
     "moe_layer_bwd_workspace_size": (_SZ, [_CFG]),
     "moe_layer_bwd": (_I, [_CFG, _VP, ctypes.c_float, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP,
                            _VP, _SZ, _VP]),
+    "moe_quantize_mxfp8_t": (_I, [_VP, ctypes.c_int32, ctypes.c_int32, ctypes.c_int32, _VP, ctypes.c_int64, _VP,
+                                  _VP]),
+    "moe_mxfp8_t_padded_rows": (ctypes.c_int64, [_CFG]),
+    "moe_quantize_mxfp8_t_grouped": (_I, [_CFG, ctypes.c_int32, _VP, _VP, _VP, _VP, _VP, ctypes.c_int32, _VP,
+                                          ctypes.c_int64, _VP, _VP]),
 }
 
 
@@ -121,14 +126,14 @@ def _check(fn, rc):
 def make_config(wl=None, **kw) -> moe_config:
     """moe_config from a synthetic.Workload (or keyword fields)."""
     d = dict(T=0, H=0, E=0, k=0, F=0, n_shared=0, score=MOE_SCORE_SOFTMAX, norm_topk=1, route_scale=1.0,
-             expert_dtype=MOE_DT_BF16, compute_aux=0, save_for_bwd=0, capacity_factor=0.0)
+             expert_dtype=MOE_DT_BF16, compute_aux=0, save_for_bwd=0, capacity_factor=0.0, n_group=0, topk_group=0)
     if wl is not None:
         d.update(T=wl.T, H=wl.H, E=wl.E, k=wl.k, F=wl.F, n_shared=wl.S,
                  score=MOE_SCORE_SOFTMAX if wl.score == "softmax" else MOE_SCORE_SIGMOID,
                  norm_topk=int(wl.norm_topk), route_scale=wl.route_scale,
                  expert_dtype=MOE_DT_BF16 if wl.dtype == "bf16" else MOE_DT_MXFP8,
                  compute_aux=int(wl.aux and wl.score == "softmax"), save_for_bwd=int(wl.bwd),
-                 capacity_factor=wl.capacity_factor)
+                 capacity_factor=wl.capacity_factor, n_group=wl.n_group, topk_group=wl.topk_group)
     d.update(kw)
     return moe_config(**d)
 
@@ -155,9 +160,11 @@ def moe_router_workspace_size(cfg) -> int:
     return load().moe_router_workspace_size(ctypes.byref(cfg))
 
 
-def moe_router_topk(cfg, x, W_r, logit_bias, logits, probs, idx, gates, counts, aux, ws, stream=None):
+def moe_router_topk(cfg, x, W_r, logit_bias, logits, probs, idx, gates, counts, aux, ws, stream=None,
+                    expert_bias=None):
+    """expert_bias (the DeepSeek-V3 selection bias) is a keyword here; in the C ABI it follows logit_bias."""
     return _check("moe_router_topk", load().moe_router_topk(
-        ctypes.byref(cfg), _p(x), _p(W_r), _p(logit_bias), _p(logits), _p(probs), _p(idx), _p(gates), _p(counts),
+        ctypes.byref(cfg), _p(x), _p(W_r), _p(logit_bias), _p(expert_bias), _p(logits), _p(probs), _p(idx), _p(gates), _p(counts),
         _p(aux), _p(ws), ws.numel() if ws is not None else 0, _st(stream)))
 
 
@@ -224,9 +231,10 @@ def moe_layer_saved_size(cfg) -> int:
 
 
 def moe_layer_fwd(cfg, x, W_r, logit_bias, W_g, W_u, W_d, W_g_sf, W_u_sf, W_d_sf, Ws_g, Ws_u, Ws_d, Ws_g_sf,
-                  Ws_u_sf, Ws_d_sf, y, aux, idx, gates, counts, offsets, saved, ws, stream=None):
+                  Ws_u_sf, Ws_d_sf, y, aux, idx, gates, counts, offsets, saved, ws, stream=None, expert_bias=None):
+    """expert_bias (the DeepSeek-V3 selection bias) is a keyword here; in the C ABI it follows logit_bias."""
     return _check("moe_layer_fwd", load().moe_layer_fwd(
-        ctypes.byref(cfg), _p(x), _p(W_r), _p(logit_bias), _p(W_g), _p(W_u), _p(W_d), _p(W_g_sf), _p(W_u_sf),
+        ctypes.byref(cfg), _p(x), _p(W_r), _p(logit_bias), _p(expert_bias), _p(W_g), _p(W_u), _p(W_d), _p(W_g_sf), _p(W_u_sf),
         _p(W_d_sf), _p(Ws_g), _p(Ws_u), _p(Ws_d), _p(Ws_g_sf), _p(Ws_u_sf), _p(Ws_d_sf), _p(y), _p(aux), _p(idx),
         _p(gates), _p(counts), _p(offsets), _p(saved), _p(ws), ws.numel() if ws is not None else 0, _st(stream)))
 
@@ -240,4 +248,21 @@ def moe_layer_bwd(cfg, dY, d_aux, x, W_r, W_g, W_u, W_d, saved, dX, dW_r, dW_g, 
     return _check("moe_layer_bwd", load().moe_layer_bwd(
         ctypes.byref(cfg), _p(dY), float(d_aux), _p(x), _p(W_r), _p(W_g), _p(W_u), _p(W_d), _p(saved), _p(dX),
         _p(dW_r), _p(dW_g), _p(dW_u), _p(dW_d), _p(dlogits), _p(ws), ws.numel() if ws is not None else 0,
+        _st(stream)))
+
+
+def moe_quantize_mxfp8_t(src, dst, sf, ldd=None, stream=None):
+    """src [B, R, C] bf16 -> dst [B, C, ldd] e4m3 (blocks along R), sf [B, C, ldd/32]."""
+    B, R, C = src.shape
+    return _check("moe_quantize_mxfp8_t", load().moe_quantize_mxfp8_t(
+        _p(src), B, R, C, _p(dst), ldd if ldd is not None else R, _p(sf), _st(stream)))
+
+
+def moe_mxfp8_t_padded_rows(cfg) -> int:
+    return load().moe_mxfp8_t_padded_rows(ctypes.byref(cfg))
+
+
+def moe_quantize_mxfp8_t_grouped(cfg, mode, src, src_of, row_gate, offsets, poff, C, dst, ldd, sf, stream=None):
+    return _check("moe_quantize_mxfp8_t_grouped", load().moe_quantize_mxfp8_t_grouped(
+        ctypes.byref(cfg), mode, _p(src), _p(src_of), _p(row_gate), _p(offsets), _p(poff), C, _p(dst), ldd, _p(sf),
         _st(stream)))

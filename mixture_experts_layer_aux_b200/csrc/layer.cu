@@ -29,7 +29,8 @@ int gemm_dgrad_gateup(int rows, int groups, int H, int F, const void* dgu, const
                       const int32_t* offsets, void* dXp, cudaStream_t st);
 int gemm_wgrad(int rows, int groups, int M, int N, const void* dO, int ld_dO, const void* act, const int32_t* offsets,
                void* C, void* C2, int split, cudaStream_t st);
-int layer_fwd_mxfp8(const moe_config* c, const void* x, const void* W_r, const float* bias, const void* W_g,
+int layer_fwd_mxfp8(const moe_config* c, const void* x, const void* W_r, const float* bias, const float* sel_bias,
+                    const void* W_g,
                     const void* W_u, const void* W_d, const uint8_t* W_g_sf, const uint8_t* W_u_sf,
                     const uint8_t* W_d_sf, const void* Ws_g, const void* Ws_u, const void* Ws_d,
                     const uint8_t* Ws_g_sf, const uint8_t* Ws_u_sf, const uint8_t* Ws_d_sf, void* y, float* aux,
@@ -116,7 +117,8 @@ static int copy_out(void* dst, const void* src, size_t bytes, cudaStream_t st) {
     if (_rc) return _rc;  \
   } while (0)
 
-int layer_fwd(const moe_config* c, const void* x, const void* W_r, const float* bias, const void* W_g, const void* W_u,
+int layer_fwd(const moe_config* c, const void* x, const void* W_r, const float* bias, const float* sel_bias,
+              const void* W_g, const void* W_u,
               const void* W_d, const void* Ws_g, const void* Ws_u, const void* Ws_d, void* y, float* aux,
               int32_t* idx, float* gates, int32_t* counts, int32_t* offsets, void* saved, void* ws, size_t ws_bytes,
               cudaStream_t st) {
@@ -132,7 +134,7 @@ int layer_fwd(const moe_config* c, const void* x, const void* W_r, const float* 
     sv = w.sv;
   }
   const int T = c->T, H = c->H, F = c->F, E = c->E, k = c->k, rows = T * k;
-  RC(router_topk(c, x, W_r, bias, w.logits, sv.probs, sv.idx, sv.gates, sv.counts, c->compute_aux ? aux : nullptr,
+  RC(router_topk(c, x, W_r, bias, sel_bias, w.logits, sv.probs, sv.idx, sv.gates, sv.counts, c->compute_aux ? aux : nullptr,
                  w.router_ws, router_ws(c), st));
   RC(permute(c, x, sv.idx, sv.gates, nullptr, sv.offsets, sv.row_of, sv.src_of, sv.row_gate, sv.xp, nullptr,
              w.permute_ws, permute_ws(c), st));
@@ -333,7 +335,7 @@ extern "C" size_t moe_layer_saved_size(const moe_config* cfg) {
 }
 
 extern "C" int moe_layer_fwd(const moe_config* cfg, const void* x, const void* W_r, const float* logit_bias,
-                             const void* W_g, const void* W_u, const void* W_d, const uint8_t* W_g_sf,
+                             const float* expert_bias, const void* W_g, const void* W_u, const void* W_d, const uint8_t* W_g_sf,
                              const uint8_t* W_u_sf, const uint8_t* W_d_sf, const void* Ws_g, const void* Ws_u,
                              const void* Ws_d, const uint8_t* Ws_g_sf, const uint8_t* Ws_u_sf, const uint8_t* Ws_d_sf,
                              void* y, float* aux, int32_t* idx, float* gates, int32_t* counts, int32_t* offsets,
@@ -351,11 +353,11 @@ extern "C" int moe_layer_fwd(const moe_config* cfg, const void* x, const void* W
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   if (cfg->expert_dtype == MOE_DT_MXFP8) {
     if (cfg->save_for_bwd) return MOE_ERR_UNSUPPORTED;
-    return layer_fwd_mxfp8(cfg, x, W_r, logit_bias, W_g, W_u, W_d, W_g_sf, W_u_sf, W_d_sf, Ws_g, Ws_u, Ws_d, Ws_g_sf,
+    return layer_fwd_mxfp8(cfg, x, W_r, logit_bias, expert_bias, W_g, W_u, W_d, W_g_sf, W_u_sf, W_d_sf, Ws_g, Ws_u, Ws_d, Ws_g_sf,
                            Ws_u_sf, Ws_d_sf, y, aux, idx, gates, counts, offsets, ws, ws_bytes, st);
   }
   if (W_g_sf || W_u_sf || W_d_sf || Ws_g_sf || Ws_u_sf || Ws_d_sf) return MOE_ERR_INVALID_ARG;
-  return layer_fwd(cfg, x, W_r, logit_bias, W_g, W_u, W_d, Ws_g, Ws_u, Ws_d, y, aux, idx, gates, counts, offsets,
+  return layer_fwd(cfg, x, W_r, logit_bias, expert_bias, W_g, W_u, W_d, Ws_g, Ws_u, Ws_d, y, aux, idx, gates, counts, offsets,
                    saved, ws, ws_bytes, st);
 }
 

@@ -26,7 +26,8 @@ namespace moe_impl {
 int check_cfg(const moe_config* c);
 size_t router_ws(const moe_config* c);
 size_t permute_ws(const moe_config* c);
-int router_topk(const moe_config* c, const void* x, const void* W_r, const float* bias, float* logits, float* probs,
+int router_topk(const moe_config* c, const void* x, const void* W_r, const float* bias, const float* sel_bias,
+                float* logits, float* probs,
                 int32_t* idx, float* gates, int32_t* counts, float* aux, void* ws, size_t ws_bytes, cudaStream_t st);
 int permute(const moe_config* c, const void* x, const int32_t* idx, const float* gates, int32_t* counts,
             int32_t* offsets, int32_t* row_of, int32_t* src_of, float* row_gate, void* xp, uint8_t* xp_sf, void* ws,
@@ -35,4 +36,10 @@ int scatter_rows(const moe_config* c, const void* x, const int32_t* row_of, void
 int unpermute(const moe_config* c, const void* o, const int32_t* row_of, const void* extra, void* y, cudaStream_t st);
 int quantize_mxfp8(const void* src, int64_t rows, int32_t K, uint8_t* dst, uint8_t* sf, cudaStream_t st);
 int fill_offsets2(int32_t* off, int n, cudaStream_t st);
+int dg_reduce(const float* part, int rows, int nparts, float* dg, cudaStream_t st);
+int pad_offsets(const int32_t* off, int E, int32_t* poff, cudaStream_t st);
+long long padded_rows_max(long long rows, int E);
+int quant_t_rows(int mode, const void* src, const int32_t* src_of, const float* row_gate, const int32_t* off,
+                 const int32_t* poff, int E, long long rows, int C, uint8_t* dst, uint8_t* sf, long long ldd,
+                 cudaStream_t st);
 }  // namespace moe_impl

@@ -157,7 +157,8 @@ static int copy_out(void* dst, const void* src, size_t bytes, cudaStream_t st) {
   return MOE_OK;
 }
 
-int layer_fwd_mxfp8(const moe_config* c, const void* x, const void* W_r, const float* bias, const void* W_g,
+int layer_fwd_mxfp8(const moe_config* c, const void* x, const void* W_r, const float* bias, const float* sel_bias,
+                    const void* W_g,
                     const void* W_u, const void* W_d, const uint8_t* W_g_sf, const uint8_t* W_u_sf,
                     const uint8_t* W_d_sf, const void* Ws_g, const void* Ws_u, const void* Ws_d,
                     const uint8_t* Ws_g_sf, const uint8_t* Ws_u_sf, const uint8_t* Ws_d_sf, void* y, float* aux,
@@ -173,7 +174,7 @@ int layer_fwd_mxfp8(const moe_config* c, const void* x, const void* W_r, const f
   if (!ws || ws_bytes < carve_mx(nullptr, c, &w)) return MOE_ERR_WORKSPACE;
   carve_mx(ws, c, &w);
   const int T = c->T, H = c->H, F = c->F, E = c->E, k = c->k, rows = T * k;
-  RCM(router_topk(c, x, W_r, bias, w.logits, w.probs, w.idx, w.gates, w.counts, c->compute_aux ? aux : nullptr,
+  RCM(router_topk(c, x, W_r, bias, sel_bias, w.logits, w.probs, w.idx, w.gates, w.counts, c->compute_aux ? aux : nullptr,
                   w.router_ws, router_ws(c), st));
   RCM(permute(c, x, w.idx, w.gates, nullptr, w.offsets, w.row_of, w.src_of, w.row_gate, w.xp, w.xp_sf,
               w.permute_ws, permute_ws(c), st));

@@ -40,6 +40,10 @@ struct TopkArgs {
   int score, norm;
   float scale;
   int want_aux;
+  // DeepSeek-V3 variant: select on score + sel_bias[e] within the topk_group best of n_group
+  // expert groups (sel_mode = 0: select on the logits)
+  const float* sel_bias;
+  int n_group, topk_group, sel_mode;
 };
 
 __device__ __forceinline__ bool better(float v1, int i1, float v2, int i2) {
@@ -108,6 +112,68 @@ __global__ void __launch_bounds__(WARPS * 32) topk_kernel(TopkArgs a) {
 #pragma unroll
       for (int i = 0; i < EPL; ++i) pacc[i] += s[i];
     }
+    // selection values: the logits, or (DeepSeek-V3 variant) score + selection bias, with the
+    // experts of all but the topk_group best groups removed
+    float v[EPL];
+#pragma unroll
+    for (int i = 0; i < EPL; ++i) v[i] = l[i];
+    if (a.sel_mode) {
+#pragma unroll
+      for (int i = 0; i < EPL; ++i) {
+        const int e = lane + 32 * i;
+        v[i] = (e < a.E) ? s[i] + (a.sel_bias ? a.sel_bias[e] : 0.f) : -INFINITY;
+      }
+      if (a.n_group > 1) {
+        const int G = a.E / a.n_group;
+        // lane g ends up with group g's score: the sum of its two largest selection values
+        float my_gs = -INFINITY;
+        for (int g = 0; g < a.n_group; ++g) {
+          float b1 = -INFINITY, b2 = -INFINITY;
+#pragma unroll
+          for (int i = 0; i < EPL; ++i) {
+            const int e = lane + 32 * i;
+            if (e < a.E && e / G == g) {
+              if (v[i] > b1) {
+                b2 = b1;
+                b1 = v[i];
+              } else if (v[i] > b2) {
+                b2 = v[i];
+              }
+            }
+          }
+#pragma unroll
+          for (int o = 16; o > 0; o >>= 1) {
+            const float o1 = __shfl_xor_sync(0xffffffffu, b1, o);
+            const float o2 = __shfl_xor_sync(0xffffffffu, b2, o);
+            const float n2 = fmaxf(fminf(b1, o1), fmaxf(b2, o2));  // second of the union's two largest
+            b1 = fmaxf(b1, o1);
+            b2 = n2;
+          }
+          if (lane == g) my_gs = (G >= 2) ? b1 + b2 : b1;
+        }
+        // the topk_group best groups (score desc, group index asc)
+        uint32_t kept = 0;
+        for (int r = 0; r < a.topk_group; ++r) {
+          float bv = ((kept >> lane) & 1u) ? -INFINITY : my_gs;
+          int bi = (lane < a.n_group && !((kept >> lane) & 1u)) ? lane : 0x7fffffff;
+#pragma unroll
+          for (int o = 16; o > 0; o >>= 1) {
+            const float ov = __shfl_xor_sync(0xffffffffu, bv, o);
+            const int oi = __shfl_xor_sync(0xffffffffu, bi, o);
+            if (better(ov, oi, bv, bi)) {
+              bv = ov;
+              bi = oi;
+            }
+          }
+          kept |= 1u << (bi & 31);
+        }
+#pragma unroll
+        for (int i = 0; i < EPL; ++i) {
+          const int e = lane + 32 * i;
+          if (e < a.E && !((kept >> (e / G)) & 1u)) v[i] = -INFINITY;
+        }
+      }
+    }
     // top-k by k rounds of a warp argmax (value desc, index asc)
     uint32_t taken = 0;
     int my_e = -1;
@@ -118,8 +184,8 @@ __global__ void __launch_bounds__(WARPS * 32) topk_kernel(TopkArgs a) {
 #pragma unroll
       for (int i = 0; i < EPL; ++i) {
         const int e = lane + 32 * i;
-        if (e < a.E && !((taken >> i) & 1u) && better(l[i], e, bv, bi)) {
-          bv = l[i];
+        if (e < a.E && !((taken >> i) & 1u) && better(v[i], e, bv, bi)) {
+          bv = v[i];
           bi = e;
         }
       }
@@ -235,6 +301,11 @@ int check_cfg(const moe_config* c) {
   if (c->compute_aux && c->score != MOE_SCORE_SOFTMAX) return MOE_ERR_UNSUPPORTED;
   if ((long long)c->T * c->k >= (1LL << 31) / 2) return MOE_ERR_UNSUPPORTED;
   if (!(c->capacity_factor >= 0.f) || c->capacity_factor > 1e30f) return MOE_ERR_INVALID_ARG;  // NaN, < 0, inf
+  if (c->n_group < 0 || c->n_group > 32) return MOE_ERR_INVALID_ARG;
+  if (c->n_group > 1) {
+    if (c->E % c->n_group != 0 || c->topk_group < 1 || c->topk_group > c->n_group) return MOE_ERR_INVALID_ARG;
+    if (c->k > c->topk_group * (c->E / c->n_group)) return MOE_ERR_INVALID_ARG;
+  }
   return MOE_OK;
 }
 
@@ -286,8 +357,9 @@ int router_logits(const moe_config* c, const void* x, const void* W_r, float* pa
   return gg::launch<gg::Cfg<256, false, false, gg::EPI_F32, gg::GROUP_NONE, gg::B_SINGLE>>(p, tiles, st);
 }
 
-int router_topk(const moe_config* c, const void* x, const void* W_r, const float* bias, float* logits, float* probs,
-                int32_t* idx, float* gates, int32_t* counts, float* aux, void* ws, size_t ws_bytes, cudaStream_t st) {
+int router_topk(const moe_config* c, const void* x, const void* W_r, const float* bias, const float* sel_bias,
+                float* logits, float* probs, int32_t* idx, float* gates, int32_t* counts, float* aux, void* ws,
+                size_t ws_bytes, cudaStream_t st) {
   int rc = check_cfg(c);
   if (rc) return rc;
   const bool logits_in = (x == nullptr && W_r == nullptr);
@@ -331,6 +403,10 @@ int router_topk(const moe_config* c, const void* x, const void* W_r, const float
   a.norm = c->norm_topk;
   a.scale = c->route_scale;
   a.want_aux = (aux != nullptr);
+  a.sel_bias = sel_bias;
+  a.n_group = c->n_group > 1 ? c->n_group : 1;
+  a.topk_group = c->n_group > 1 ? c->topk_group : 1;
+  a.sel_mode = (sel_bias != nullptr || c->n_group > 1) ? 1 : 0;
   const size_t smem = (size_t)c->E * sizeof(int) + (size_t)router::WARPS * c->E * sizeof(float);
   const dim3 grid(nblk), block(router::WARPS * 32);
   if (c->E <= 32) router::topk_kernel<1><<<grid, block, smem, st>>>(a);
@@ -360,8 +436,8 @@ extern "C" size_t moe_router_workspace_size(const moe_config* cfg) {
 }
 
 extern "C" int moe_router_topk(const moe_config* cfg, const void* x, const void* W_r, const float* logit_bias,
-                               float* logits, float* probs, int32_t* idx, float* gates, int32_t* counts, float* aux,
-                               void* ws, size_t ws_bytes, void* stream) {
-  return moe_impl::router_topk(cfg, x, W_r, logit_bias, logits, probs, idx, gates, counts, aux, ws, ws_bytes,
-                               static_cast<cudaStream_t>(stream));
+                               const float* expert_bias, float* logits, float* probs, int32_t* idx, float* gates,
+                               int32_t* counts, float* aux, void* ws, size_t ws_bytes, void* stream) {
+  return moe_impl::router_topk(cfg, x, W_r, logit_bias, expert_bias, logits, probs, idx, gates, counts, aux, ws,
+                               ws_bytes, static_cast<cudaStream_t>(stream));
 }

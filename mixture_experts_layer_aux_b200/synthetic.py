@@ -79,6 +79,12 @@ WORKLOADS = {
                      score="sigmoid", route_scale=2.5, dtype="mxfp8", aux=False),
     "skewed": Workload("skewed", T=8192, H=4096, E=128, k=8, F=1536,
                        skew=True, bwd=True),
+    # the ranked variants on the same shapes: DeepSeek-V3 routing (selection bias, 8 groups, 4 kept)
+    # and the capacity factor (1.25) on the skewed fwd+bwd step
+    "dsv3-grouped": Workload("dsv3-grouped", T=8192, H=7168, E=256, k=8, F=2048, S=1, score="sigmoid",
+                             route_scale=2.5, dtype="mxfp8", aux=False, n_group=8, topk_group=4, sel_bias=True),
+    "skewed-capacity": Workload("skewed-capacity", T=8192, H=4096, E=128, k=8, F=1536, skew=True, bwd=True,
+                                capacity_factor=1.25),
 }
 
 

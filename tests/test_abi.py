@@ -78,10 +78,13 @@ def test_config_validation(lib, B):
                       (dict(H=200), UNSUPPORTED), (dict(F=100), UNSUPPORTED), (dict(T=0), INVALID),
                       (dict(score=5), INVALID), (dict(n_shared=2), UNSUPPORTED),
                       (dict(compute_aux=1, score=1), UNSUPPORTED), (dict(capacity_factor=-1.0), INVALID),
-                      (dict(capacity_factor=float("nan")), INVALID), (dict(capacity_factor=float("inf")), INVALID)]:
+                      (dict(capacity_factor=float("nan")), INVALID), (dict(capacity_factor=float("inf")), INVALID),
+                      (dict(n_group=3), INVALID), (dict(n_group=4, topk_group=0), INVALID),
+                      (dict(n_group=4, topk_group=5), INVALID), (dict(n_group=33), INVALID),
+                      (dict(n_group=4, topk_group=1, k=3), INVALID)]:
         c = cfg(B, **bad)
         assert lib.moe_router_workspace_size(ctypes.byref(c)) == 0
-        rc = lib.moe_router_topk(ctypes.byref(c), FAKE, FAKE, None, FAKE, None, FAKE, FAKE, None, None, FAKE, 1 << 30,
+        rc = lib.moe_router_topk(ctypes.byref(c), FAKE, FAKE, None, None, FAKE, None, FAKE, FAKE, None, None, FAKE, 1 << 30,
                                  None)
         assert rc == code, (bad, rc)
 
@@ -90,13 +93,13 @@ def test_router_argument_errors(lib, B):
     c = cfg(B)
     ws = lib.moe_router_workspace_size(ctypes.byref(c))
     f = lib.moe_router_topk
-    assert f(ctypes.byref(c), FAKE, FAKE, None, None, None, FAKE, FAKE, None, None, FAKE, ws, None) == INVALID
-    assert f(ctypes.byref(c), FAKE, None, None, FAKE, None, FAKE, FAKE, None, None, FAKE, ws, None) == INVALID
-    assert f(ctypes.byref(c), FAKE + 2, FAKE, None, FAKE, None, FAKE, FAKE, None, None, FAKE, ws, None) == ALIGN
-    assert f(ctypes.byref(c), FAKE, FAKE, None, FAKE, None, FAKE, FAKE, None, None, FAKE, ws - 1, None) == WS
-    assert f(ctypes.byref(c), FAKE, FAKE, None, FAKE, None, FAKE, FAKE, None, None, None, ws, None) == WS
+    assert f(ctypes.byref(c), FAKE, FAKE, None, None, None, None, FAKE, FAKE, None, None, FAKE, ws, None) == INVALID
+    assert f(ctypes.byref(c), FAKE, None, None, None, FAKE, None, FAKE, FAKE, None, None, FAKE, ws, None) == INVALID
+    assert f(ctypes.byref(c), FAKE + 2, FAKE, None, None, FAKE, None, FAKE, FAKE, None, None, FAKE, ws, None) == ALIGN
+    assert f(ctypes.byref(c), FAKE, FAKE, None, None, FAKE, None, FAKE, FAKE, None, None, FAKE, ws - 1, None) == WS
+    assert f(ctypes.byref(c), FAKE, FAKE, None, None, FAKE, None, FAKE, FAKE, None, None, None, ws, None) == WS
     # aux requested without compute_aux
-    assert f(ctypes.byref(c), FAKE, FAKE, None, FAKE, None, FAKE, FAKE, None, FAKE, FAKE, ws, None) == INVALID
+    assert f(ctypes.byref(c), FAKE, FAKE, None, None, FAKE, None, FAKE, FAKE, None, FAKE, FAKE, ws, None) == INVALID
 
 
 def test_permute_argument_errors(lib, B):
@@ -126,8 +129,8 @@ def test_gemm_and_layer_argument_errors(lib, B):
     lw = lib.moe_layer_workspace_size(ctypes.byref(c))
     assert lw > lib.moe_layer_saved_size(ctypes.byref(c)) // 8
     L = lib.moe_layer_fwd
-    args = [FAKE, FAKE, None, FAKE, FAKE, FAKE, None, None, None, None, None, None, None, None, None, FAKE, None, None,
-            None, None, None, None]
+    args = [FAKE, FAKE, None, None, FAKE, FAKE, FAKE, None, None, None, None, None, None, None, None, None, FAKE, None,
+            None, None, None, None, None]
     assert L(ctypes.byref(c), *args, FAKE, lw - 1, None) == WS
     args2 = list(args)
     args2[0] = None

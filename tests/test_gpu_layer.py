@@ -27,7 +27,7 @@ def run_fwd(moe, wl, d, save=False):
     saved = moe.workspace(moe.moe_layer_saved_size(cfg)) if save else None
     moe.moe_layer_fwd(cfg, d["x"], d["W_r"], d.get("logit_bias"), d["W_g"], d["W_u"], d["W_d"], None, None, None,
                       d.get("W_gs"), d.get("W_us"), d.get("W_ds"), None, None, None, out["y"], out["aux"],
-                      out["idx"], out["gates"], out["counts"], out["offsets"], saved, ws)
+                      out["idx"], out["gates"], out["counts"], out["offsets"], saved, ws, expert_bias=d.get("expert_bias"))
     torch.cuda.synchronize()
     out["saved"] = saved
     out["cfg"] = cfg
@@ -38,14 +38,22 @@ def routing_agreement(oracle, wl, h, gpu_idx):
     """Oracle logits + routing; returns (route dict, tokens whose indices agree)."""
     logits = oracle.router_logits(h["x"], h["W_r"], h.get("logit_bias"))
     r = oracle.route(logits, wl.k, wl.score, wl.norm_topk, wl.route_scale, with_aux=wl.aux and wl.score == "softmax",
-                     capacity_factor=wl.capacity_factor)
+                     capacity_factor=wl.capacity_factor, expert_bias=h.get("expert_bias"), n_group=wl.n_group,
+                     topk_group=wl.topk_group)
     same = (gpu_idx.cpu() == r["idx"]).all(1)
     bound = 1e-4 * float(logits.pow(2).mean().sqrt())
+    # selection values: the logits, or (DeepSeek-V3 variant) score + bias, whose slope is at most 1/4 of the logits'
+    sel = r["sel"] if r.get("sel") is not None else logits
     for t in (~same).nonzero().flatten().tolist():
         gi, ri = gpu_idx[t].cpu(), r["idx"][t]
         # experts in disagreeing slots (a swap of slot order leaves the sets equal)
         a = sorted(set(gi[gi != ri].tolist()) | set(ri[gi != ri].tolist()))
-        gap = (logits[t, a].max() - logits[t, a].min()).item()
+        gap = (sel[t, a].max() - sel[t, a].min()).item()
+        if wl.n_group > 1 and gap > 2 * bound:
+            # a near-tie between groups moves whole groups: check the group scores around the cut
+            G = wl.E // wl.n_group
+            gs = torch.topk(sel[t].view(wl.n_group, G), min(2, G), dim=-1).values.sum(-1).sort(descending=True).values
+            gap = (gs[wl.topk_group - 1] - gs[wl.topk_group]).item()
         assert gap <= 2 * bound, f"token {t}: routing differs by more than a near-tie (gap {gap})"
     assert int((~same).sum()) <= max(2, wl.T // 1000)
     return r, same
@@ -128,6 +136,16 @@ def test_permute_capacity_maps_bit_exact(moe, oracle):
     assert torch.equal(src_of.cpu()[:n], so[:n])
     assert torch.equal(xp.cpu()[:n].view(torch.int16), x[so[:n].long()].view(torch.int16))
     assert moe.moe_get_device_status() == 0
+
+
+@pytest.mark.parametrize("wl", [
+    Workload("dsv3-router", T=600, H=512, E=64, k=6, F=256, score="sigmoid", route_scale=2.5, aux=False,
+             n_group=8, topk_group=4, sel_bias=True),
+    Workload("bias-only", T=300, H=256, E=16, k=2, F=256, score="sigmoid", route_scale=2.5, aux=False,
+             sel_bias=True)])
+def test_layer_fwd_deepseek_router_variant_full_oracle(moe, oracle, wl):
+    """Selection on sigmoid score + per-expert bias within the best expert groups; gates from the scores."""
+    check_fwd(moe, oracle, wl)
 
 
 def test_layer_fwd_is_deterministic(moe):
@@ -255,7 +273,8 @@ def run_fwd_mx(moe, wl, d):
     if wl.S:
         sh = [q["W_gs"][0], q["W_us"][0], q["W_ds"][0], q["W_gs"][1], q["W_us"][1], q["W_ds"][1]]
     moe.moe_layer_fwd(cfg, d["x"], d["W_r"], d.get("logit_bias"), q["W_g"][0], q["W_u"][0], q["W_d"][0], q["W_g"][1],
-                      q["W_u"][1], q["W_d"][1], *sh, y, None, idx, gates, None, None, None, ws)
+                      q["W_u"][1], q["W_d"][1], *sh, y, None, idx, gates, None, None, None, ws,
+                      expert_bias=d.get("expert_bias"))
     torch.cuda.synchronize()
     return y, idx, gates
 
@@ -264,7 +283,9 @@ def check_fwd_mx(moe, oracle, wl, n_sample=None, seed=0):
     d = make_inputs(wl, device="cuda", seed=seed)
     y, idx, gates = run_fwd_mx(moe, wl, d)
     logits = oracle.router_logits(d["x"].cpu(), d["W_r"].cpu(), None)
-    r, same = routing_agreement(oracle, wl, {"x": d["x"].cpu(), "W_r": d["W_r"].cpu()}, idx)
+    r, same = routing_agreement(oracle, wl, {"x": d["x"].cpu(), "W_r": d["W_r"].cpu(),
+                                             "expert_bias": None if d.get("expert_bias") is None
+                                             else d["expert_bias"].cpu()}, idx)
     if n_sample is None:
         toks = torch.arange(wl.T, dtype=torch.int32)
     else:
@@ -298,6 +319,12 @@ def check_fwd_mx(moe, oracle, wl, n_sample=None, seed=0):
 def test_layer_fwd_mxfp8_small_full_oracle(moe, oracle):
     wl = Workload("mx-small", T=256, H=512, E=16, k=4, F=256, S=1, score="sigmoid", route_scale=2.5, dtype="mxfp8",
                   aux=False)
+    check_fwd_mx(moe, oracle, wl)
+
+
+def test_layer_fwd_mxfp8_deepseek_router_variant(moe, oracle):
+    wl = Workload("mx-dsv3-router", T=256, H=512, E=32, k=4, F=256, S=1, score="sigmoid", route_scale=2.5,
+                  aux=False, dtype="mxfp8", n_group=4, topk_group=2, sel_bias=True)
     check_fwd_mx(moe, oracle, wl)
 
 

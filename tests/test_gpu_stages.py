@@ -92,6 +92,39 @@ def test_routing_from_logits_bit_exact(moe, oracle, T, E, k, score, norm, scale,
     _status_clean(moe)
 
 
+@pytest.mark.parametrize("T,E,k,n_group,topk_group", [(4096, 256, 8, 8, 4), (1000, 64, 6, 8, 3), (333, 32, 4, 0, 0),
+                                                      (64, 16, 4, 16, 4)])
+def test_routing_deepseek_variant_from_logits(moe, oracle, T, E, k, n_group, topk_group):
+    """Selection on the fp32 score + bias (group-limited): the oracle selects on the same fp32
+    values (the GPU's scores plus the bias, added in fp32), so indices must agree except where two
+    group scores (summed in fp32 on the GPU, exactly by the oracle) are within an fp32 ulp."""
+    l = random_logits(T, E, seed=T + E + 5)
+    g = torch.Generator().manual_seed(E)
+    b = ((torch.rand(E, generator=g) - 0.5) * 0.2).float()
+    cfg = moe.make_config(T=T, H=256, E=E, k=k, F=128, score=1, norm_topk=1, route_scale=2.5, n_group=n_group,
+                          topk_group=topk_group)
+    probs, idx, gates = empty((T, E), torch.float32), empty((T, k), torch.int32), empty((T, k), torch.float32)
+    ws = moe.workspace(moe.moe_router_workspace_size(cfg))
+    moe.moe_router_topk(cfg, None, None, None, l.cuda(), probs, idx, gates, None, None, ws, expert_bias=b.cuda())
+    torch.cuda.synchronize()
+    r = oracle.route(l.double(), k, "sigmoid", True, 2.5, with_aux=False, expert_bias=b.double(), n_group=n_group,
+                     topk_group=topk_group)
+    assert (probs.cpu().double() - r["probs"]).abs().max().item() <= 2e-6
+    sel32 = (probs.cpu() + b).double()                       # the GPU's selection values, exactly
+    ref = oracle.topk_grouped(sel32, k, n_group, topk_group)
+    bad = (~(idx.cpu() == ref).all(1)).nonzero().flatten().tolist()
+    G = E // max(n_group, 1)
+    for t in bad:                                             # only group-score near-ties may differ
+        assert n_group > 1
+        gs = torch.topk(sel32[t].view(n_group, G), min(2, G), dim=-1).values.sum(-1).sort(descending=True).values
+        assert (gs[topk_group - 1] - gs[topk_group]).item() <= 1e-6, t
+    assert len(bad) <= max(1, T // 1000)
+    ok = (idx.cpu() == r["idx"]).all(1)
+    gref = r["gates"][ok]
+    assert (gates.cpu().double()[ok] - gref).abs().max().item() <= 5e-6
+    _status_clean(moe)
+
+
 # ------------------------------------------------------------------ permute
 
 
