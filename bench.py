@@ -557,8 +557,9 @@ class OracleTimer:
         return time.perf_counter() - t0
 
     def sample_size(self, budget_s, max_tok):
-        t1 = self.run(2)
-        return int(max(2, min(max_tok, self.wl.T, budget_s / max(t1 / 2, 1e-6))))
+        self.run(2)                       # warm: threads, page faults
+        per_tok = self.run(4) / 4
+        return int(max(2, min(max_tok, self.wl.T, budget_s / max(per_tok, 1e-6))))
 
     def describe(self, n, t, value):
         return {"value": value, "unit": "tokens/s", "cores": self.oracle.nthreads(), "kind": "oracle",
