@@ -205,6 +205,15 @@ class Layer:
         self.mx = wl.dtype == "mxfp8"
         if self.mx:
             q = {}
+            if wl.bwd:
+                # the backward's transposed MXFP8 weights: W_d^T [E,F,H] along H, W_g^T | W_u^T [E,H,2F] along F
+                self.wdt = torch.empty((E, F, H), dtype=torch.uint8, device="cuda")
+                self.wdt_sf = torch.empty((E, F, H // 32), dtype=torch.uint8, device="cuda")
+                moe.moe_quantize_mxfp8_t(d["W_d"], self.wdt, self.wdt_sf)
+                self.wgu = torch.empty((E, H, 2 * F), dtype=torch.uint8, device="cuda")
+                self.wgu_sf = torch.empty((E, H, 2 * F // 32), dtype=torch.uint8, device="cuda")
+                moe.moe_quantize_mxfp8_t(d["W_g"], self.wgu, self.wgu_sf, ldd=2 * F)
+                moe.moe_quantize_mxfp8_t(d["W_u"], self.wgu, self.wgu_sf, ldd=2 * F, col0=F)
             for name in ["W_g", "W_u", "W_d"] + (["W_gs", "W_us", "W_ds"] if wl.S else []):
                 w = d[name]
                 codes = torch.empty(w.shape, dtype=torch.uint8, device="cuda")
@@ -246,13 +255,15 @@ class Layer:
             self.dW_g = torch.empty(E, F, H, dtype=torch.bfloat16, device=dev)
             self.dW_u = torch.empty(E, F, H, dtype=torch.bfloat16, device=dev)
             self.dW_d = torch.empty(E, H, F, dtype=torch.bfloat16, device=dev)
-            self.ws_bwd = moe.workspace(moe.moe_layer_bwd_workspace_size(self.cfg))
+            self.ws_bwd = moe.workspace(moe.moe_layer_bwd_mxfp8_workspace_size(self.cfg) if self.mx
+                                        else moe.moe_layer_bwd_workspace_size(self.cfg))
         if wl.S:
             self.off2 = torch.tensor([0, T], dtype=torch.int32, device=dev)
             self.as_ = torch.empty(T, F, dtype=torch.uint8 if self.mx else torch.bfloat16, device=dev)
             self.as_sf = torch.empty(T, F // 32, dtype=torch.uint8, device=dev) if self.mx else None
             self.so = torch.empty(T, H, dtype=torch.bfloat16, device=dev)
-            self.cfg_sh = moe.make_config(wl, T=T, E=1, k=1, n_shared=0, compute_aux=0, save_for_bwd=0)
+            self.cfg_sh = moe.make_config(wl, T=T, E=1, k=1, n_shared=0, compute_aux=0, save_for_bwd=0, n_group=0,
+                                          topk_group=0, capacity_factor=0.0)
             if self.mx:
                 self.xq = torch.empty(T, H, dtype=torch.uint8, device=dev)
                 self.xq_sf = torch.empty(T, H // 32, dtype=torch.uint8, device=dev)
@@ -315,7 +326,9 @@ class Layer:
         if self.wl.S:
             n += 2 + (1 if self.mx else 0)
         if self.wl.bwd:
-            n += 9
+            # MXFP8: dY gather-quantise, two dgrad GEMMs, dgate|dup quantiser, padded offsets, four
+            # transposed quantisers, two weight-gradient GEMMs, router backward, two router GEMMs, unpermute
+            n += 15 if self.mx else 9
         return n
 
     def layer_call(self, x, y, aux):
@@ -332,6 +345,10 @@ class Layer:
 
     def bwd_call(self):
         m, c, d = self.moe, self.cfg, self.d
+        if self.mx:
+            m.moe_layer_bwd_mxfp8(c, self.dY, 0.01, d["x"], d["W_r"], self.wdt, self.wdt_sf, self.wgu, self.wgu_sf,
+                                  self.saved, self.dX, self.dW_r, self.dW_g, self.dW_u, self.dW_d, None, self.ws_bwd)
+            return
         m.moe_layer_bwd(c, self.dY, 0.01, d["x"], d["W_r"], d["W_g"], d["W_u"], d["W_d"], self.saved, self.dX,
                         self.dW_r, self.dW_g, self.dW_u, self.dW_d, None, self.ws_bwd)
 

@@ -279,6 +279,47 @@ int moe_quantize_mxfp8_t_grouped(const moe_config* cfg, int32_t mode, const void
                                  int64_t ldd, uint8_t* sf, void* stream);
 
 /* ------------------------------------------------------------------------
+ * MXFP8 backward GEMMs (the MXFP8 recipe on every backward GEMM; operands
+ * blocked along that GEMM's K; fp32 accumulation; bf16 results).
+ *
+ * moe_grouped_gemm_dgrad_mxfp8: data gradients, grouped by offsets.
+ *   which == MOE_GEMM_DOWN: A = dY in permuted order, MXFP8 [T*k, H] (blocks
+ *     along H; moe_quantize_mxfp8 of the gathered rows), B = W_d^T MXFP8
+ *     [E, F, H]; out = dgate|dup bf16 [T*k, 2F] (the SwiGLU backward of
+ *     v = W_d^T dY with the saved bf16 pre-activations saved_gateup [T*k, 2F]
+ *     and row_gate [T*k]), dg [T*k] fp32 = <v, silu(gate) up>. ws >= T*k*F/128*4
+ *     bytes.
+ *   which == MOE_GEMM_GATEUP_SWIGLU: A = dgate|dup MXFP8 [T*k, 2F] (blocks
+ *     along F), B = W_g^T|W_u^T MXFP8 [E, H, 2F]; out = dXp bf16 [T*k, H].
+ *   H % 256 == 0, F % 256 == 0.
+ *
+ * moe_grouped_gemm_wgrad_mxfp8: weight gradients, grouped along K: AT, BT
+ *   are moe_quantize_mxfp8_t_grouped outputs sharing poff and ldp.
+ *   which == MOE_GEMM_DOWN: AT = dY^T [H, ldp], BT = (g a)^T [F, ldp];
+ *     dW0 = dW_d bf16 [E, H, F].
+ *   which == MOE_GEMM_GATEUP_SWIGLU: AT = (dgate|dup)^T [2F, ldp], BT = x^T
+ *     [H, ldp]; dW0 = dW_g, dW1 = dW_u bf16 [E, F, H].
+ *   An expert without tokens gets exact zeros.
+ *
+ * moe_layer_bwd_mxfp8: the whole MXFP8 backward after moe_layer_fwd with
+ *   expert_dtype == MXFP8 and save_for_bwd (which saves the routing state and
+ *   the bf16 gate/up pre-activations): W_dT/W_dT_sf = W_d^T and W_guT/W_guT_sf
+ *   = W_g^T|W_u^T from moe_quantize_mxfp8_t; the other arguments and outputs
+ *   as moe_layer_bwd. Workspace: moe_layer_bwd_mxfp8_workspace_size.
+ * ------------------------------------------------------------------------ */
+int moe_grouped_gemm_dgrad_mxfp8(const moe_config* cfg, int which, const void* A, const uint8_t* A_sf, const void* B,
+                                 const uint8_t* B_sf, const int32_t* offsets, const void* saved_gateup,
+                                 const float* row_gate, void* out, float* dg, void* ws, size_t ws_bytes, void* stream);
+int moe_grouped_gemm_wgrad_mxfp8(const moe_config* cfg, int which, const void* AT, const uint8_t* AT_sf,
+                                 const void* BT, const uint8_t* BT_sf, const int32_t* poff, int64_t ldp, void* dW0,
+                                 void* dW1, void* stream);
+size_t moe_layer_bwd_mxfp8_workspace_size(const moe_config* cfg);
+int moe_layer_bwd_mxfp8(const moe_config* cfg, const void* dY, float d_aux, const void* x, const void* W_r,
+                        const void* W_dT, const uint8_t* W_dT_sf, const void* W_guT, const uint8_t* W_guT_sf,
+                        const void* saved, void* dX, void* dW_r, void* dW_g, void* dW_u, void* dW_d, float* dlogits,
+                        void* ws, size_t ws_bytes, void* stream);
+
+/* ------------------------------------------------------------------------
  * Whole layer, forward: router -> permute -> GEMM gate/up (SwiGLU, gate
  * folded) -> GEMM down -> [shared expert] -> unpermute-sum.
  *   x [T,H] bf16; W_r [E,H] bf16; logit_bias [E] fp32 or NULL; expert_bias [E]

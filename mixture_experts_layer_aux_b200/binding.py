@@ -70,6 +70,11 @@ _SIGS = {
     "moe_mxfp8_t_padded_rows": (ctypes.c_int64, [_CFG]),
     "moe_quantize_mxfp8_t_grouped": (_I, [_CFG, ctypes.c_int32, _VP, _VP, _VP, _VP, _VP, ctypes.c_int32, _VP,
                                           ctypes.c_int64, _VP, _VP]),
+    "moe_grouped_gemm_dgrad_mxfp8": (_I, [_CFG, _I, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _SZ, _VP]),
+    "moe_grouped_gemm_wgrad_mxfp8": (_I, [_CFG, _I, _VP, _VP, _VP, _VP, _VP, ctypes.c_int64, _VP, _VP, _VP]),
+    "moe_layer_bwd_mxfp8_workspace_size": (_SZ, [_CFG]),
+    "moe_layer_bwd_mxfp8": (_I, [_CFG, _VP, ctypes.c_float, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP,
+                                 _VP, _VP, _VP, _SZ, _VP]),
 }
 
 
@@ -251,11 +256,13 @@ def moe_layer_bwd(cfg, dY, d_aux, x, W_r, W_g, W_u, W_d, saved, dX, dW_r, dW_g, 
         _st(stream)))
 
 
-def moe_quantize_mxfp8_t(src, dst, sf, ldd=None, stream=None):
-    """src [B, R, C] bf16 -> dst [B, C, ldd] e4m3 (blocks along R), sf [B, C, ldd/32]."""
+def moe_quantize_mxfp8_t(src, dst, sf, ldd=None, col0=0, stream=None):
+    """src [B, R, C] bf16 -> dst [B, C, ldd] e4m3 (blocks along R), sf [B, C, ldd/32], written from column
+    col0 of each dst row (col0 % 32 == 0; e.g. W_u^T beside W_g^T in one [E, H, 2F] buffer)."""
     B, R, C = src.shape
+    assert col0 % 32 == 0
     return _check("moe_quantize_mxfp8_t", load().moe_quantize_mxfp8_t(
-        _p(src), B, R, C, _p(dst), ldd if ldd is not None else R, _p(sf), _st(stream)))
+        _p(src), B, R, C, _p(dst) + col0, ldd if ldd is not None else R, _p(sf) + col0 // 32, _st(stream)))
 
 
 def moe_mxfp8_t_padded_rows(cfg) -> int:
@@ -266,3 +273,28 @@ def moe_quantize_mxfp8_t_grouped(cfg, mode, src, src_of, row_gate, offsets, poff
     return _check("moe_quantize_mxfp8_t_grouped", load().moe_quantize_mxfp8_t_grouped(
         ctypes.byref(cfg), mode, _p(src), _p(src_of), _p(row_gate), _p(offsets), _p(poff), C, _p(dst), ldd, _p(sf),
         _st(stream)))
+
+
+def moe_grouped_gemm_dgrad_mxfp8(cfg, which, A, A_sf, B, B_sf, offsets, saved_gateup, row_gate, out, dg, ws,
+                                 stream=None):
+    return _check("moe_grouped_gemm_dgrad_mxfp8", load().moe_grouped_gemm_dgrad_mxfp8(
+        ctypes.byref(cfg), which, _p(A), _p(A_sf), _p(B), _p(B_sf), _p(offsets), _p(saved_gateup), _p(row_gate),
+        _p(out), _p(dg), _p(ws), ws.numel() if ws is not None else 0, _st(stream)))
+
+
+def moe_grouped_gemm_wgrad_mxfp8(cfg, which, AT, AT_sf, BT, BT_sf, poff, ldp, dW0, dW1, stream=None):
+    return _check("moe_grouped_gemm_wgrad_mxfp8", load().moe_grouped_gemm_wgrad_mxfp8(
+        ctypes.byref(cfg), which, _p(AT), _p(AT_sf), _p(BT), _p(BT_sf), _p(poff), ldp, _p(dW0), _p(dW1),
+        _st(stream)))
+
+
+def moe_layer_bwd_mxfp8_workspace_size(cfg) -> int:
+    return load().moe_layer_bwd_mxfp8_workspace_size(ctypes.byref(cfg))
+
+
+def moe_layer_bwd_mxfp8(cfg, dY, d_aux, x, W_r, W_dT, W_dT_sf, W_guT, W_guT_sf, saved, dX, dW_r, dW_g, dW_u, dW_d,
+                        dlogits, ws, stream=None):
+    return _check("moe_layer_bwd_mxfp8", load().moe_layer_bwd_mxfp8(
+        ctypes.byref(cfg), _p(dY), ctypes.c_float(d_aux), _p(x), _p(W_r), _p(W_dT), _p(W_dT_sf), _p(W_guT),
+        _p(W_guT_sf), _p(saved), _p(dX), _p(dW_r), _p(dW_g), _p(dW_u), _p(dW_d), _p(dlogits), _p(ws),
+        ws.numel() if ws is not None else 0, _st(stream)))

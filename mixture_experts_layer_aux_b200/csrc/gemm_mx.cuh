@@ -61,8 +61,10 @@ static_assert(SF_COL + 2 * SF_SLOT_COLS <= TMEM_COLS, "tmem");
 static_assert(SMEM_BYTES <= 232448, "smem");
 
 enum Epi : int {
-  EPI_MX_SWIGLU = 0,  // acc = [gate | up] -> g * silu(gate) * up, quantised to MXFP8 (e4m3 + ue8m0 per 32)
-  EPI_MX_BF16 = 1,    // acc -> bf16
+  EPI_MX_SWIGLU = 0,      // acc = [gate | up] -> g * silu(gate) * up, quantised to MXFP8 (e4m3 + ue8m0 per 32);
+                          // optionally the bf16 gate/up pre-activations for the backward
+  EPI_MX_BF16 = 1,        // acc -> bf16
+  EPI_MX_SWIGLU_BWD = 2,  // acc = v = W_d^T dY -> dgate, dup (bf16) and <v, a> partials from saved gate/up
 };
 
 struct __align__(64) Params {
@@ -83,12 +85,25 @@ struct __align__(64) Params {
   long long ldc;
   const float* row_gate;
   int* status;
+  // grouped along K (weight gradients): offsets are the groups' K offsets (multiples of BK), A [M, K] and
+  // B [N, K] are shared by all groups, group g writes C (+ g c_group_stride); output rows >= c2_row_split
+  // (when > 0) go to C2 instead, at row - c2_row_split
+  long long c_group_stride;
+  void* C2;
+  int c2_row_split;
+  // SWIGLU: save_gateup [M, 2N] bf16 or NULL. SWIGLU_BWD: gateup [M, 2N] bf16 (the saved pre-activations),
+  // row_gate, C = dgu [M, 2N] bf16, dg_part [M, N/128] fp32
+  __nv_bfloat16* save_gateup;
+  const __nv_bfloat16* gateup;
+  float* dg_part;
 };
 
 struct Tile {
   int g, m0, n0, row0, m_valid;
+  int kb0, nkb;  // first k-block (of BK) and k-block count
 };
 
+template <bool GK>
 __device__ __forceinline__ Tile get_tile(const Params& p, int t, const int* s_off, const int* s_tstart, int n_step) {
   int lo = 0, hi = p.G - 1;
   while (lo < hi) {
@@ -97,15 +112,28 @@ __device__ __forceinline__ Tile get_tile(const Params& p, int t, const int* s_of
     else hi = mid - 1;
   }
   const int g = lo;
-  const int mg = s_off[g + 1] - s_off[g];
-  const int MB = (mg + BM - 1) / BM;
   const int local = t - s_tstart[g];
   Tile ti;
   ti.g = g;
-  ti.m0 = (local % MB) * BM;
-  ti.n0 = (local / MB) * n_step;
-  ti.row0 = s_off[g] + ti.m0;
-  ti.m_valid = min(BM, mg - ti.m0);
+  if constexpr (GK) {
+    // every group: the whole [M, N] output; its K range is the group's segment
+    const int MB = (p.M + BM - 1) / BM;
+    ti.m0 = (local % MB) * BM;
+    ti.n0 = (local / MB) * n_step;
+    ti.row0 = ti.m0;
+    ti.m_valid = min(BM, p.M - ti.m0);
+    ti.kb0 = s_off[g] / BK;
+    ti.nkb = (s_off[g + 1] - s_off[g]) / BK;
+  } else {
+    const int mg = s_off[g + 1] - s_off[g];
+    const int MB = (mg + BM - 1) / BM;
+    ti.m0 = (local % MB) * BM;
+    ti.n0 = (local / MB) * n_step;
+    ti.row0 = s_off[g] + ti.m0;
+    ti.m_valid = min(BM, mg - ti.m0);
+    ti.kb0 = 0;
+    ti.nkb = p.K / BK;
+  }
   return ti;
 }
 
@@ -162,7 +190,7 @@ MOE_DEV void quant32(const float* v, float inv, uint32_t (&w)[8]) {
   }
 }
 
-template <int EPI, bool SPLIT_N>
+template <int EPI, bool SPLIT_N, bool GK>
 __global__ void __launch_bounds__(NUM_THREADS, 1) gemm_mx_kernel(const __grid_constant__ Params p) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -205,15 +233,17 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) gemm_mx_kernel(const __grid_co
   __syncthreads();
   if (warp == 0) {
     int bad = 0;
-    for (int i = lane; i < p.G; i += 32)
-      if (s_off[i + 1] < s_off[i] || s_off[i] < 0 || s_off[i + 1] > p.M) bad = 1;
+    for (int i = lane; i < p.G; i += 32) {
+      if (s_off[i + 1] < s_off[i] || s_off[i] < 0 || s_off[i + 1] > (GK ? p.K : p.M)) bad = 1;
+      if (GK && (s_off[i] % BK) != 0) bad = 1;
+    }
     bad = __any_sync(0xffffffffu, bad);
     if (lane == 0) {
       const int NT = (p.N + N_STEP - 1) / N_STEP;
       int acc = 0;
       for (int g = 0; g < p.G; ++g) {
         s_tstart[g] = acc;
-        if (!bad) acc += ((s_off[g + 1] - s_off[g] + BM - 1) / BM) * NT;
+        if (!bad) acc += (GK ? (p.M + BM - 1) / BM : (s_off[g + 1] - s_off[g] + BM - 1) / BM) * NT;
       }
       s_tstart[p.G] = acc;
       if (bad) record_status(p.status, DEV_BAD_OFFSETS);
@@ -223,7 +253,6 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) gemm_mx_kernel(const __grid_co
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
   const int total = s_tstart[p.G];
-  const int KB = p.K / BK;
   bool aborted = false;
 
   if (warp == 0) {
@@ -235,9 +264,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) gemm_mx_kernel(const __grid_co
       int stage = 0;
       uint32_t phase = 0, issued_mask = 0, issued_par = 0;
       for (int t = blockIdx.x; t < total && !aborted; t += gridDim.x) {
-        const Tile ti = get_tile(p, t, s_off, s_tstart, N_STEP);
-        const int brow = ti.g * p.b_group_rows + ti.n0;
-        for (int kb = 0; kb < KB; ++kb) {
+        const Tile ti = get_tile<GK>(p, t, s_off, s_tstart, N_STEP);
+        const int brow = (GK ? 0 : ti.g * p.b_group_rows) + ti.n0;
+        for (int kb = 0; kb < ti.nkb; ++kb) {
           if (!mbar_wait(&empty[stage], phase ^ 1, abort_flag, p.status, DEV_WAIT_TIMEOUT_PRODUCER)) {
             aborted = true;
             break;
@@ -247,7 +276,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) gemm_mx_kernel(const __grid_co
           issued_par = (issued_par & ~(1u << stage)) | (phase << stage);
           uint8_t* sA = smem + stage * STAGE_BYTES;
           uint8_t* sB = sA + A_BYTES;
-          const int kc = kb * BK;
+          const int kc = (ti.kb0 + kb) * BK;
           tma_load_2d(sA, &p.tmA, kc, ti.row0, &full[stage]);
           if (SPLIT_N) {
             tma_load_2d(sB, &p.tmB0, kc, brow, &full[stage]);
@@ -283,10 +312,11 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) gemm_mx_kernel(const __grid_co
     int sb = 0;
     uint32_t sphase = 0;
     for (int t = blockIdx.x; t < total && !aborted; t += gridDim.x) {
-      const Tile ti = get_tile(p, t, s_off, s_tstart, N_STEP);
-      const long long brow = (long long)ti.g * p.b_group_rows + ti.n0;
-      for (int kb0 = 0; kb0 < KB; kb0 += SB) {
-        const int nb = min(SB, KB - kb0);
+      const Tile ti = get_tile<GK>(p, t, s_off, s_tstart, N_STEP);
+      const long long brow = (GK ? 0LL : (long long)ti.g * p.b_group_rows) + ti.n0;
+      for (int kb0 = 0; kb0 < ti.nkb; kb0 += SB) {
+        const int nb = min(SB, ti.nkb - kb0);
+        const int kbg = ti.kb0 + kb0;  // the batch's first k-block in the operands' K
         if (!__all_sync(0xffffffffu,
                         mbar_wait(&sempty[sb], sphase ^ 1, abort_flag, p.status, DEV_WAIT_TIMEOUT_PRODUCER))) {
           aborted = true;
@@ -317,11 +347,15 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) gemm_mx_kernel(const __grid_co
               base = p.sfb0;
               r = brow + lane + 32 * ib;
             }
+            if (GK) {  // B [N, K] is shared by the groups: rows past N read row 0 and are zeroed
+              ok[i] = r < p.N;
+              if (!ok[i]) r = 0;
+            }
           }
-          src[i] = base + r * kw + 4 * kb0;
+          src[i] = base + r * kw + 4 * kbg;
         }
         uint32_t w[12][SB];
-        if (v16 && nb == SB) {
+        if (v16 && nb == SB && (kbg & 3) == 0) {
 #pragma unroll
           for (int i = 0; i < 12; ++i) {
             const uint4 u = __ldg(reinterpret_cast<const uint4*>(src[i]));
@@ -361,14 +395,15 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) gemm_mx_kernel(const __grid_co
     int sb = 0;  // scale batch in shared memory
     uint32_t sphase = 0;
     for (int t = blockIdx.x; t < total && !aborted; t += gridDim.x) {
+      const Tile ti = get_tile<GK>(p, t, s_off, s_tstart, N_STEP);
       if (!__all_sync(0xffffffffu, mbar_wait(tempty, acc_phase ^ 1, abort_flag, p.status, DEV_WAIT_TIMEOUT_MMA))) {
         aborted = true;
         break;
       }
       tc_fence_after();
-      for (int kb = 0; kb < KB; ++kb) {
+      for (int kb = 0; kb < ti.nkb; ++kb) {
         const int j = kb % SB;
-        const bool batch_end = (j == SB - 1) || (kb == KB - 1);
+        const bool batch_end = (j == SB - 1) || (kb == ti.nkb - 1);
         if (j == 0) {
           // a new scale batch in shared memory
           if (!__all_sync(0xffffffffu,
@@ -437,7 +472,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) gemm_mx_kernel(const __grid_co
     const int row = q * 32 + lane;
     uint32_t acc_phase = 0;
     for (int t = blockIdx.x; t < total && !aborted; t += gridDim.x) {
-      const Tile ti = get_tile(p, t, s_off, s_tstart, N_STEP);
+      const Tile ti = get_tile<GK>(p, t, s_off, s_tstart, N_STEP);
       if (!__all_sync(0xffffffffu, mbar_wait(tfull, acc_phase, abort_flag, p.status, DEV_WAIT_TIMEOUT_EPILOGUE))) {
         aborted = true;
         break;
@@ -445,7 +480,11 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) gemm_mx_kernel(const __grid_co
       tc_fence_after();
       const uint32_t tb = tmem_base + ((uint32_t)(q * 32) << 16);
       float v[128];
-      if (EPI == EPI_MX_SWIGLU) {
+      if (ti.nkb == 0) {
+        // a group with no rows (grouped along K): the result is exactly zero, TMEM holds nothing of it
+#pragma unroll
+        for (int i = 0; i < 128; ++i) v[i] = 0.f;
+      } else if (EPI == EPI_MX_SWIGLU) {
         // gate columns [64h, 64h+64), up columns [128 + 64h, ...)
         tmem_ld32(tb + 64 * h, *reinterpret_cast<float(*)[32]>(&v[0]));
         tmem_ld32(tb + 64 * h + 32, *reinterpret_cast<float(*)[32]>(&v[32]));
@@ -455,7 +494,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) gemm_mx_kernel(const __grid_co
 #pragma unroll
         for (int c = 0; c < 4; ++c) tmem_ld32(tb + 128 * h + 32 * c, *reinterpret_cast<float(*)[32]>(&v[32 * c]));
       }
-      tmem_ld_wait();
+      if (ti.nkb != 0) tmem_ld_wait();
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(tempty);  // accumulator free: the next tile's MMAs may start
@@ -465,30 +504,89 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) gemm_mx_kernel(const __grid_co
       if (valid) {
         if (EPI == EPI_MX_SWIGLU) {
           const float g = p.row_gate ? p.row_gate[orow] : 1.f;
-          float a[64];
+          const int col0 = ti.n0 + 64 * h;  // F column of v[0]
+          if (p.save_gateup) {
+            // the fp32 gate/up pre-activations, rounded to bf16, for the backward's recomputation
+            __nv_bfloat16* sv = p.save_gateup + orow * 2LL * p.N + col0;
 #pragma unroll
-          for (int i = 0; i < 64; ++i) a[i] = g * silu_f(v[i]) * v[64 + i];
-          const int col0 = ti.n0 + 64 * h;  // F column of a[0]
+            for (int c = 0; c < 8; ++c) {
+              reinterpret_cast<uint4*>(sv)[c] =
+                  make_uint4(pack_bf16x2(v[8 * c], v[8 * c + 1]), pack_bf16x2(v[8 * c + 2], v[8 * c + 3]),
+                             pack_bf16x2(v[8 * c + 4], v[8 * c + 5]), pack_bf16x2(v[8 * c + 6], v[8 * c + 7]));
+              reinterpret_cast<uint4*>(sv + p.N)[c] =
+                  make_uint4(pack_bf16x2(v[64 + 8 * c], v[64 + 8 * c + 1]),
+                             pack_bf16x2(v[64 + 8 * c + 2], v[64 + 8 * c + 3]),
+                             pack_bf16x2(v[64 + 8 * c + 4], v[64 + 8 * c + 5]),
+                             pack_bf16x2(v[64 + 8 * c + 6], v[64 + 8 * c + 7]));
+            }
+          }
+          // a = g silu(gate) up, in place over the gate values
+#pragma unroll
+          for (int i = 0; i < 64; ++i) v[i] = g * silu_f(v[i]) * v[64 + i];
           uint8_t* out = reinterpret_cast<uint8_t*>(p.C) + orow * p.ldc + col0;
           uint8_t sb[2];
 #pragma unroll
           for (int b = 0; b < 2; ++b) {
             float am = 0.f;
 #pragma unroll
-            for (int i = 0; i < 32; ++i) am = fmaxf(am, fabsf(a[32 * b + i]));
+            for (int i = 0; i < 32; ++i) am = fmaxf(am, fabsf(v[32 * b + i]));
             sb[b] = mx_scale_byte(am);
             uint32_t w[8];
-            quant32(a + 32 * b, mx_inv_scale(sb[b]), w);
+            quant32(v + 32 * b, mx_inv_scale(sb[b]), w);
             uint4* o4 = reinterpret_cast<uint4*>(out + 32 * b);
             o4[0] = make_uint4(w[0], w[1], w[2], w[3]);
             o4[1] = make_uint4(w[4], w[5], w[6], w[7]);
           }
           *reinterpret_cast<uint16_t*>(p.C_sf + orow * (p.ldc / 32) + col0 / 32) =
               (uint16_t)sb[0] | ((uint16_t)sb[1] << 8);
-        } else {
-          __nv_bfloat16* out = reinterpret_cast<__nv_bfloat16*>(p.C) + orow * p.ldc + ti.n0 + 128 * h;
+        } else if (EPI == EPI_MX_SWIGLU_BWD) {
+          // columns [col0, col0 + 128) of F: dgate, dup from the saved bf16 pre-activations z
+          const float g = p.row_gate[orow];
+          const int col0 = ti.n0 + 128 * h;
+          const __nv_bfloat16* zp = p.gateup + orow * 2LL * p.N + col0;
+          __nv_bfloat16* dp = reinterpret_cast<__nv_bfloat16*>(p.C) + orow * 2LL * p.N + col0;
+          float part = 0.f;
 #pragma unroll
           for (int c = 0; c < 16; ++c) {
+            float zg[8], zu[8];
+            unpack_bf16x8(reinterpret_cast<const uint4*>(zp)[c], zg);
+            unpack_bf16x8(reinterpret_cast<const uint4*>(zp + p.N)[c], zu);
+            float dgv[8], duv[8];
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+              const float vv = v[8 * c + i];
+              const float sg = 1.0f / (1.0f + __expf(-zg[i]));
+              const float sl = zg[i] * sg;
+              part += vv * sl * zu[i];
+              const float da = g * vv;
+              dgv[i] = da * zu[i] * sg * (1.f + zg[i] * (1.f - sg));
+              duv[i] = da * sl;
+            }
+            reinterpret_cast<uint4*>(dp)[c] =
+                make_uint4(pack_bf16x2(dgv[0], dgv[1]), pack_bf16x2(dgv[2], dgv[3]), pack_bf16x2(dgv[4], dgv[5]),
+                           pack_bf16x2(dgv[6], dgv[7]));
+            reinterpret_cast<uint4*>(dp + p.N)[c] =
+                make_uint4(pack_bf16x2(duv[0], duv[1]), pack_bf16x2(duv[2], duv[3]), pack_bf16x2(duv[4], duv[5]),
+                           pack_bf16x2(duv[6], duv[7]));
+          }
+          p.dg_part[orow * (long long)(p.N / 128) + col0 / 128] = part;
+        } else {
+          __nv_bfloat16* out;
+          if constexpr (GK) {
+            long long r = orow;
+            void* base = p.C;
+            if (p.c2_row_split > 0 && r >= p.c2_row_split) {
+              r -= p.c2_row_split;
+              base = p.C2;
+            }
+            out = reinterpret_cast<__nv_bfloat16*>(base) + ti.g * p.c_group_stride + r * p.ldc + ti.n0 + 128 * h;
+          } else {
+            out = reinterpret_cast<__nv_bfloat16*>(p.C) + orow * p.ldc + ti.n0 + 128 * h;
+          }
+          const int ncol = min(128, p.N - ti.n0 - 128 * h);  // columns of this half inside the output
+#pragma unroll
+          for (int c = 0; c < 16; ++c) {
+            if (8 * c >= ncol) break;
             uint4 u;
             u.x = pack_bf16x2(v[8 * c], v[8 * c + 1]);
             u.y = pack_bf16x2(v[8 * c + 2], v[8 * c + 3]);
@@ -508,10 +606,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) gemm_mx_kernel(const __grid_co
   }
 }
 
-template <int EPI, bool SPLIT_N>
+template <int EPI, bool SPLIT_N, bool GK = false>
 int launch(const Params& p, int max_tiles, cudaStream_t stream) {
   if (max_tiles <= 0) return MOE_OK;
-  auto kern = gemm_mx_kernel<EPI, SPLIT_N>;
+  auto kern = gemm_mx_kernel<EPI, SPLIT_N, GK>;
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES) != cudaSuccess) {
     (void)cudaGetLastError();
     return MOE_ERR_CUDA;

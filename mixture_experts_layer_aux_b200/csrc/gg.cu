@@ -173,6 +173,12 @@ __global__ void dg_reduce_kernel(const float* __restrict__ part, int rows, int n
   }
 }
 
+int dg_reduce(const float* part, int rows, int nparts, float* dg, cudaStream_t st) {
+  dg_reduce_kernel<<<(rows + 255) / 256, 256, 0, st>>>(part, rows, nparts, dg);
+  MOE_CHECK_LAUNCH();
+  return MOE_OK;
+}
+
 size_t gg_fwd_ws(const moe_config*, int) { return 256; }
 size_t gg_bwd_ws(const moe_config* c, int which) {
   if (which == MOE_GEMM_DOWN) return ws_round((size_t)c->T * c->k * (c->F / 128) * sizeof(float));

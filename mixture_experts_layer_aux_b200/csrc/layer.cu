@@ -34,8 +34,8 @@ int layer_fwd_mxfp8(const moe_config* c, const void* x, const void* W_r, const f
                     const void* W_u, const void* W_d, const uint8_t* W_g_sf, const uint8_t* W_u_sf,
                     const uint8_t* W_d_sf, const void* Ws_g, const void* Ws_u, const void* Ws_d,
                     const uint8_t* Ws_g_sf, const uint8_t* Ws_u_sf, const uint8_t* Ws_d_sf, void* y, float* aux,
-                    int32_t* idx, float* gates, int32_t* counts, int32_t* offsets, void* ws, size_t ws_bytes,
-                    cudaStream_t st);
+                    int32_t* idx, float* gates, int32_t* counts, int32_t* offsets, void* saved, void* ws,
+                    size_t ws_bytes, cudaStream_t st);
 size_t layer_ws_mxfp8(const moe_config* c);
 
 // Tensors that the backward reads, in the `saved` buffer (or in the workspace
@@ -316,9 +316,116 @@ int layer_bwd(const moe_config* c, const void* dY, float d_aux, const void* x, c
   return MOE_OK;
 }
 
+// ------------------------------------------------------------------ MXFP8 backward
+
+struct BwdWsMx {
+  uint8_t *dYq, *dYq_sf, *dYT, *dYT_sf;
+  int32_t* poff;
+  __nv_bfloat16* dgu;
+  float* dg_part;
+  uint8_t *dguq, *dguq_sf, *dguT, *dguT_sf, *apT, *apT_sf, *xT, *xT_sf;
+  __nv_bfloat16* dXp;
+  float* dl;
+  __nv_bfloat16* dl16;
+  __nv_bfloat16* dXr;
+  long long ldp;
+};
+
+static size_t carve_bwd_mx(void* ws, const moe_config* c, BwdWsMx* w) {
+  Carve cv(ws);
+  const size_t T = c->T, E = c->E, k = c->k, H = c->H, F = c->F, rows = T * k;
+  const size_t ldp = (size_t)padded_rows_max((long long)rows, c->E);
+  w->ldp = (long long)ldp;
+  w->dYq = cv.take<uint8_t>(rows * H);
+  w->dYq_sf = cv.take<uint8_t>(rows * H / 32);
+  w->dYT = cv.take<uint8_t>(H * ldp);
+  w->dYT_sf = cv.take<uint8_t>(H * ldp / 32);
+  w->poff = cv.take<int32_t>(E + 1);
+  w->dgu = cv.take<__nv_bfloat16>(rows * 2 * F);
+  w->dg_part = cv.take<float>(rows * (F / 128));
+  w->dguq = cv.take<uint8_t>(rows * 2 * F);
+  w->dguq_sf = cv.take<uint8_t>(rows * 2 * F / 32);
+  w->dguT = cv.take<uint8_t>(2 * F * ldp);
+  w->dguT_sf = cv.take<uint8_t>(2 * F * ldp / 32);
+  w->apT = cv.take<uint8_t>(F * ldp);
+  w->apT_sf = cv.take<uint8_t>(F * ldp / 32);
+  w->xT = cv.take<uint8_t>(H * ldp);
+  w->xT_sf = cv.take<uint8_t>(H * ldp / 32);
+  w->dXp = cv.take<__nv_bfloat16>(rows * H);
+  w->dl = cv.take<float>(T * E);
+  w->dl16 = cv.take<__nv_bfloat16>(T * E);
+  w->dXr = cv.take<__nv_bfloat16>(T * H);
+  return cv.used;
+}
+
+// The MXFP8 backward: every backward GEMM takes MXFP8 operands blocked along its own K (dY and x along
+// H, W_d^T along H, dgate/dup along F, W_g^T and W_u^T along F, and the weight gradients' operands along
+// each expert's tokens); the SwiGLU is recomputed from the saved bf16 pre-activations.
+int layer_bwd_mxfp8(const moe_config* c, const void* dY, float d_aux, const void* x, const void* W_r,
+                    const void* W_dT, const uint8_t* W_dT_sf, const void* W_guT, const uint8_t* W_guT_sf,
+                    const void* saved, void* dX, void* dW_r, void* dW_g, void* dW_u, void* dW_d, float* dlogits,
+                    void* ws, size_t ws_bytes, cudaStream_t st) {
+  BwdWsMx w;
+  if (!ws || ws_bytes < carve_bwd_mx(nullptr, c, &w)) return MOE_ERR_WORKSPACE;
+  carve_bwd_mx(ws, c, &w);
+  Carve cs(const_cast<void*>(saved));
+  const SavedMx sv = carve_saved_mx(cs, c);
+  const int T = c->T, H = c->H, F = c->F, E = c->E, k = c->k, rows = T * k;
+  const long long ldp = w.ldp;
+  // data gradients
+  RC(scatter_rows_mx(c, dY, sv.row_of, w.dYq, w.dYq_sf, st));
+  RC(gemm_dgrad_down_mx(rows, E, H, F, w.dYq, w.dYq_sf, W_dT, W_dT_sf, sv.offsets, sv.gateup, sv.row_gate, w.dgu,
+                        w.dg_part, st));
+  RC(quantize_mxfp8(w.dgu, rows, 2 * F, w.dguq, w.dguq_sf, st));
+  RC(gemm_dgrad_gateup_mx(rows, E, H, F, w.dguq, w.dguq_sf, W_guT, W_guT_sf, sv.offsets, w.dXp, st));
+  // weight gradients: operands along each expert's tokens
+  RC(pad_offsets(sv.offsets, E, w.poff, st));
+  RC(quant_t_rows(1, dY, sv.src_of, nullptr, sv.offsets, w.poff, E, rows, H, w.dYT, w.dYT_sf, ldp, st));
+  RC(quant_t_rows(2, sv.gateup, nullptr, sv.row_gate, sv.offsets, w.poff, E, rows, F, w.apT, w.apT_sf, ldp, st));
+  RC(gemm_wgrad_mx(E, H, F, ldp, w.dYT, w.dYT_sf, w.apT, w.apT_sf, w.poff, dW_d, nullptr, 0, st));
+  RC(quant_t_rows(0, w.dgu, nullptr, nullptr, sv.offsets, w.poff, E, rows, 2 * F, w.dguT, w.dguT_sf, ldp, st));
+  RC(quant_t_rows(1, x, sv.src_of, nullptr, sv.offsets, w.poff, E, rows, H, w.xT, w.xT_sf, ldp, st));
+  RC(gemm_wgrad_mx(E, 2 * F, H, ldp, w.dguT, w.dguT_sf, w.xT, w.xT_sf, w.poff, dW_g, dW_u, F, st));
+  // router
+  float* dl = dlogits ? dlogits : w.dl;
+  router_bwd_kernel<<<(T + 7) / 8, 256, 0, st>>>(w.dg_part, F / 128, sv.row_of, sv.idx, sv.gates, sv.probs, sv.counts,
+                                                 T, E, k, c->score, c->norm_topk, c->route_scale,
+                                                 c->compute_aux ? 1 : 0, d_aux, dl, w.dl16);
+  MOE_CHECK_LAUNCH();
+  RC(gemm_router_dwr(T, E, H, w.dl16, x, dW_r, st));
+  RC(gemm_router_dx(T, E, H, w.dl16, W_r, w.dXr, st));
+  RC(unpermute(c, w.dXp, sv.row_of, w.dXr, dX, st));
+  return MOE_OK;
+}
+
 }  // namespace moe_impl
 
 using namespace moe_impl;
+
+extern "C" size_t moe_layer_bwd_mxfp8_workspace_size(const moe_config* cfg) {
+  if (check_cfg(cfg)) return 0;
+  BwdWsMx w;
+  return carve_bwd_mx(nullptr, cfg, &w);
+}
+
+extern "C" int moe_layer_bwd_mxfp8(const moe_config* cfg, const void* dY, float d_aux, const void* x,
+                                   const void* W_r, const void* W_dT, const uint8_t* W_dT_sf, const void* W_guT,
+                                   const uint8_t* W_guT_sf, const void* saved, void* dX, void* dW_r, void* dW_g,
+                                   void* dW_u, void* dW_d, float* dlogits, void* ws, size_t ws_bytes, void* stream) {
+  int rc = check_cfg(cfg);
+  if (rc) return rc;
+  if (cfg->expert_dtype != MOE_DT_MXFP8) return MOE_ERR_INVALID_ARG;
+  if (cfg->H % 256 != 0 || cfg->F % 256 != 0 || cfg->E % 8 != 0 || cfg->n_shared != 0) return MOE_ERR_UNSUPPORTED;
+  if (!dY || !x || !W_r || !W_dT || !W_dT_sf || !W_guT || !W_guT_sf || !saved || !dX || !dW_r || !dW_g || !dW_u ||
+      !dW_d)
+    return MOE_ERR_INVALID_ARG;
+  const void* ptrs[] = {dY, x, W_r, W_dT, W_guT, saved, dX, dW_r, dW_g, dW_u, dW_d, ws};
+  for (const void* p : ptrs)
+    if (p && !al16(p)) return MOE_ERR_ALIGNMENT;
+  if ((reinterpret_cast<uintptr_t>(W_dT_sf) | reinterpret_cast<uintptr_t>(W_guT_sf)) & 3u) return MOE_ERR_ALIGNMENT;
+  return layer_bwd_mxfp8(cfg, dY, d_aux, x, W_r, W_dT, W_dT_sf, W_guT, W_guT_sf, saved, dX, dW_r, dW_g, dW_u, dW_d,
+                         dlogits, ws, ws_bytes, static_cast<cudaStream_t>(stream));
+}
 
 extern "C" size_t moe_layer_workspace_size(const moe_config* cfg) {
   if (check_cfg(cfg)) return 0;
@@ -330,7 +437,8 @@ extern "C" size_t moe_layer_workspace_size(const moe_config* cfg) {
 extern "C" size_t moe_layer_saved_size(const moe_config* cfg) {
   if (check_cfg(cfg)) return 0;
   Carve cv(nullptr);
-  carve_saved(cv, cfg);
+  if (cfg->expert_dtype == MOE_DT_MXFP8) carve_saved_mx(cv, cfg);
+  else carve_saved(cv, cfg);
   return cv.used;
 }
 
@@ -352,9 +460,8 @@ extern "C" int moe_layer_fwd(const moe_config* cfg, const void* x, const void* W
     if (p && !al16(p)) return MOE_ERR_ALIGNMENT;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   if (cfg->expert_dtype == MOE_DT_MXFP8) {
-    if (cfg->save_for_bwd) return MOE_ERR_UNSUPPORTED;
     return layer_fwd_mxfp8(cfg, x, W_r, logit_bias, expert_bias, W_g, W_u, W_d, W_g_sf, W_u_sf, W_d_sf, Ws_g, Ws_u, Ws_d, Ws_g_sf,
-                           Ws_u_sf, Ws_d_sf, y, aux, idx, gates, counts, offsets, ws, ws_bytes, st);
+                           Ws_u_sf, Ws_d_sf, y, aux, idx, gates, counts, offsets, saved, ws, ws_bytes, st);
   }
   if (W_g_sf || W_u_sf || W_d_sf || Ws_g_sf || Ws_u_sf || Ws_d_sf) return MOE_ERR_INVALID_ARG;
   return layer_fwd(cfg, x, W_r, logit_bias, expert_bias, W_g, W_u, W_d, Ws_g, Ws_u, Ws_d, y, aux, idx, gates, counts, offsets,

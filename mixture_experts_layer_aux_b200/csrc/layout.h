@@ -23,6 +23,32 @@ struct Carve {
 };
 
 namespace moe_impl {
+// What the MXFP8 backward reads from an MXFP8 forward that saved for it.
+struct SavedMx {
+  float* probs;
+  int32_t* idx;
+  float* gates;
+  int32_t* counts;
+  int32_t* offsets;
+  int32_t* row_of;
+  int32_t* src_of;
+  float* row_gate;
+  __nv_bfloat16* gateup;  // [T*k, 2F] gate/up pre-activations (bf16)
+};
+inline SavedMx carve_saved_mx(Carve& cv, const moe_config* c) {
+  const size_t T = c->T, E = c->E, k = c->k, rows = T * k, F = c->F;
+  SavedMx s;
+  s.probs = cv.take<float>(T * E);
+  s.idx = cv.take<int32_t>(T * k);
+  s.gates = cv.take<float>(T * k);
+  s.counts = cv.take<int32_t>(E);
+  s.offsets = cv.take<int32_t>(E + 1);
+  s.row_of = cv.take<int32_t>(T * k);
+  s.src_of = cv.take<int32_t>(rows);
+  s.row_gate = cv.take<float>(rows);
+  s.gateup = cv.take<__nv_bfloat16>(rows * 2 * F);
+  return s;
+}
 int check_cfg(const moe_config* c);
 size_t router_ws(const moe_config* c);
 size_t permute_ws(const moe_config* c);
@@ -33,12 +59,21 @@ int permute(const moe_config* c, const void* x, const int32_t* idx, const float*
             int32_t* offsets, int32_t* row_of, int32_t* src_of, float* row_gate, void* xp, uint8_t* xp_sf, void* ws,
             size_t ws_bytes, cudaStream_t st);
 int scatter_rows(const moe_config* c, const void* x, const int32_t* row_of, void* xp, cudaStream_t st);
+int scatter_rows_mx(const moe_config* c, const void* x, const int32_t* row_of, uint8_t* xq, uint8_t* xq_sf,
+                    cudaStream_t st);
 int unpermute(const moe_config* c, const void* o, const int32_t* row_of, const void* extra, void* y, cudaStream_t st);
 int quantize_mxfp8(const void* src, int64_t rows, int32_t K, uint8_t* dst, uint8_t* sf, cudaStream_t st);
 int fill_offsets2(int32_t* off, int n, cudaStream_t st);
 int dg_reduce(const float* part, int rows, int nparts, float* dg, cudaStream_t st);
 int pad_offsets(const int32_t* off, int E, int32_t* poff, cudaStream_t st);
 long long padded_rows_max(long long rows, int E);
+int gemm_dgrad_down_mx(int rows, int E, int H, int F, const void* dYq, const uint8_t* dYq_sf, const void* WdT,
+                       const uint8_t* WdT_sf, const int32_t* offsets, const void* gateup, const float* row_gate,
+                       void* dgu, float* dg_part, cudaStream_t st);
+int gemm_dgrad_gateup_mx(int rows, int E, int H, int F, const void* dguq, const uint8_t* dguq_sf, const void* WguT,
+                         const uint8_t* WguT_sf, const int32_t* offsets, void* dxp, cudaStream_t st);
+int gemm_wgrad_mx(int E, int M, int N, long long ldp, const void* AT, const uint8_t* AT_sf, const void* BT,
+                  const uint8_t* BT_sf, const int32_t* poff, void* C, void* C2, int split, cudaStream_t st);
 int quant_t_rows(int mode, const void* src, const int32_t* src_of, const float* row_gate, const int32_t* off,
                  const int32_t* poff, int E, long long rows, int C, uint8_t* dst, uint8_t* sf, long long ldd,
                  cudaStream_t st);

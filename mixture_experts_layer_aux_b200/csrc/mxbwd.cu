@@ -1,0 +1,362 @@
+// mxbwd.cu -- operands of the MXFP8 backward GEMMs that are quantised along a
+// dimension other than the one their bf16 source is contiguous in.
+//
+// The MXFP8 recipe (the Blackwell training recipe the Megatron Core MoE summary
+// names in section 3) blocks every GEMM operand along that GEMM's reduction
+// dimension K, and the tensor cores read K-major MXFP8 operands. In the
+// backward two kinds of operands are transposed with respect to the forward:
+//   weights: the data gradients reduce over F (gate/up) or H (down), so W_g^T,
+//     W_u^T [H, F] and W_d^T [F, H] are quantised along F resp. H
+//     (moe_quantize_mxfp8_t, once per weight update);
+//   activations: the weight gradients reduce over an expert's tokens, so dY,
+//     x, the gate-folded activation g a and dgate/dup are quantised along
+//     the tokens, transposed into [C, rows_pad] with each expert's rows
+//     starting on a 128-row boundary (pad rows zero), so that the grouped
+//     weight-gradient GEMM's K range of each expert is whole 128-row k-blocks
+//     and its 32-row scale blocks never straddle two experts.
+#include <cuda_fp8.h>
+
+#include "common.cuh"
+#include "gemm_mx.cuh"
+#include "layout.h"
+
+namespace mxb {
+
+constexpr int PAD = 128;  // expert segments of the transposed activations start on this row boundary
+
+// poff[e] = sum_{e' < e} roundup(count_e', 128), poff[E] = the padded total (one block, E <= 512)
+__global__ void __launch_bounds__(512) pad_offsets_kernel(const int32_t* __restrict__ off, int E,
+                                                          int32_t* __restrict__ poff) {
+  __shared__ int s[512];
+  const int e = threadIdx.x;
+  const int c = e < E ? ((off[e + 1] - off[e] + PAD - 1) / PAD) * PAD : 0;
+  s[e] = c;
+  __syncthreads();
+  for (int o = 1; o < 512; o <<= 1) {
+    const int v = e >= o ? s[e - o] : 0;
+    __syncthreads();
+    s[e] += v;
+    __syncthreads();
+  }
+  if (e < E) poff[e + 1] = s[e];
+  if (e == 0) poff[0] = 0;
+}
+
+__device__ __forceinline__ uint8_t mx_scale_byte(float amax) {
+  const uint32_t b = __float_as_uint(amax);
+  const int eb = (int)((b >> 23) & 0xFFu);
+  if (!(amax > 0.f) || eb == 0) return 0;
+  int s = eb - 8;  // floor(log2 amax) - 8 + 127
+  s = s < 0 ? 0 : (s > 254 ? 254 : s);
+  return (uint8_t)s;
+}
+__device__ __forceinline__ float mx_inv_scale(uint8_t byte) { return __uint_as_float((uint32_t)(254 - byte) << 23); }
+
+enum Mode : int {
+  MODE_ROWS = 0,    // source row r of [rows, C]
+  MODE_GATHER = 1,  // source row src_of[r] of [T, C]
+  MODE_AP = 2,      // row_gate[r] * silu(gate) * up from the saved pre-activations [rows, 2F] (C = F)
+  MODE_WEIGHT = 3,  // batch b = blockIdx.z of [B, R, C], no experts, no padding (R % 32 == 0)
+};
+
+struct QtArgs {
+  const __nv_bfloat16* src;  // ROWS: [rows, C]; GATHER: [T, C]; AP: gate/up [rows, 2C]; WEIGHT: [B, R, C]
+  const int32_t* src_of;
+  const float* row_gate;
+  const int32_t* off;        // [E+1] expert row offsets (not WEIGHT)
+  const int32_t* poff;       // [E+1] padded offsets (not WEIGHT)
+  int E;
+  int R;                     // WEIGHT: rows per batch
+  int C;                     // columns of the source = rows of the output
+  uint8_t* dst;              // [C, ldd] (WEIGHT: [B, C, ldd]) e4m3
+  long long ldd;
+  uint8_t* sf;               // [C, ldd / 32] (WEIGHT: [B, C, ldd / 32]) ue8m0
+};
+
+// One block: 32 consecutive output positions (padded rows) x 64 columns. The 32 x 64 tile is staged
+// in fp32 through shared memory; then each warp takes 8 columns: lane i holds position i, a warp max
+// gives the 32-row block's amax, and each column's 32 codes leave as one 32-byte store.
+template <int MODE>
+__global__ void __launch_bounds__(256) quant_t_kernel(const QtArgs a) {
+  __shared__ float tile[32][65];
+  __shared__ int s_meta[2];  // first source row of the tile (-1: none), valid rows in the tile
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int p0 = blockIdx.x * 32;  // first output position (padded row)
+  const int c0 = blockIdx.y * 64;
+  const int b = MODE == MODE_WEIGHT ? blockIdx.z : 0;
+  if (tid == 0) {
+    int r0 = -1, nv = 0;
+    if constexpr (MODE == MODE_WEIGHT) {
+      r0 = p0;
+      nv = min(32, a.R - p0);
+    } else if (p0 < a.poff[a.E]) {
+      int lo = 0, hi = a.E - 1;  // expert whose padded segment holds p0
+      while (lo < hi) {
+        const int mid = (lo + hi + 1) >> 1;
+        if (a.poff[mid] <= p0) lo = mid;
+        else hi = mid - 1;
+      }
+      const int i = p0 - a.poff[lo];
+      const int cnt = a.off[lo + 1] - a.off[lo];
+      r0 = a.off[lo] + i;
+      nv = max(0, min(32, cnt - i));
+    }
+    s_meta[0] = r0;
+    s_meta[1] = nv;
+  }
+  __syncthreads();
+  const int r0 = s_meta[0], nv = s_meta[1];
+  if (r0 < 0) return;  // past the padded total (block-uniform)
+  // load: thread t -> row t/8, columns 8*(t%8) .. +7 of the tile
+  {
+    const int rr = tid >> 3, cc = (tid & 7) * 8;
+    float f[8];
+#pragma unroll
+    for (int q = 0; q < 8; ++q) f[q] = 0.f;
+    if (rr < nv && c0 + cc < a.C) {
+      const long long r = r0 + rr;
+      if constexpr (MODE == MODE_AP) {
+        const __nv_bfloat16* gp = a.src + r * 2LL * a.C + c0 + cc;
+        float zg[8], zu[8];
+        unpack_bf16x8(*reinterpret_cast<const uint4*>(gp), zg);
+        unpack_bf16x8(*reinterpret_cast<const uint4*>(gp + a.C), zu);
+        const float g = a.row_gate[r];
+#pragma unroll
+        for (int q = 0; q < 8; ++q) f[q] = g * silu_f(zg[q]) * zu[q];
+      } else {
+        long long sr = r;
+        if constexpr (MODE == MODE_GATHER) sr = a.src_of[r];
+        const __nv_bfloat16* base = a.src;
+        if constexpr (MODE == MODE_WEIGHT) base += (long long)b * a.R * a.C;
+        unpack_bf16x8(*reinterpret_cast<const uint4*>(base + sr * a.C + c0 + cc), f);
+      }
+    }
+#pragma unroll
+    for (int q = 0; q < 8; ++q) tile[rr][cc + q] = f[q];
+  }
+  __syncthreads();
+  uint8_t* dst = a.dst;
+  uint8_t* sf = a.sf;
+  if constexpr (MODE == MODE_WEIGHT) {
+    dst += (long long)b * a.C * a.ldd;
+    sf += (long long)b * a.C * (a.ldd / 32);
+  }
+#pragma unroll
+  for (int j = 0; j < 8; ++j) {
+    const int c = warp * 8 + j;
+    if (c0 + c >= a.C) break;  // warp-uniform
+    const float v = tile[lane][c];
+    float am = fabsf(v);
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) am = fmaxf(am, __shfl_xor_sync(0xffffffffu, am, o));
+    const uint8_t sb = mx_scale_byte(am);
+    const float inv = mx_inv_scale(sb);
+    const __nv_fp8_storage_t code = __nv_cvt_float_to_fp8(v * inv, __NV_SATFINITE, __NV_E4M3);
+    dst[(long long)(c0 + c) * a.ldd + p0 + lane] = code;
+    if (lane == 0) sf[(long long)(c0 + c) * (a.ldd / 32) + p0 / 32] = sb;
+  }
+}
+
+}  // namespace mxb
+
+namespace moe_impl {
+
+int pad_offsets(const int32_t* off, int E, int32_t* poff, cudaStream_t st) {
+  mxb::pad_offsets_kernel<<<1, 512, 0, st>>>(off, E, poff);
+  MOE_CHECK_LAUNCH();
+  return MOE_OK;
+}
+
+// Largest padded total for `rows` rows over E experts, rounded up to 512 so that every row of the
+// transposed buffers (and of their scales) starts 16-byte aligned.
+long long padded_rows_max(long long rows, int E) { return ((rows + (long long)mxb::PAD * E + 511) / 512) * 512; }
+
+// mode: 0 rows, 1 gather through src_of, 2 the gate-folded activation from saved gate/up
+int quant_t_rows(int mode, const void* src, const int32_t* src_of, const float* row_gate, const int32_t* off,
+                 const int32_t* poff, int E, long long rows, int C, uint8_t* dst, uint8_t* sf, long long ldd,
+                 cudaStream_t st) {
+  mxb::QtArgs a{};
+  a.src = static_cast<const __nv_bfloat16*>(src);
+  a.src_of = src_of;
+  a.row_gate = row_gate;
+  a.off = off;
+  a.poff = poff;
+  a.E = E;
+  a.C = C;
+  a.dst = dst;
+  a.ldd = ldd;
+  a.sf = sf;
+  const long long pmax = rows + (long long)mxb::PAD * E;
+  const dim3 grid((unsigned)((pmax + 31) / 32), (unsigned)((C + 63) / 64));
+  if (mode == 0) mxb::quant_t_kernel<mxb::MODE_ROWS><<<grid, 256, 0, st>>>(a);
+  else if (mode == 1) mxb::quant_t_kernel<mxb::MODE_GATHER><<<grid, 256, 0, st>>>(a);
+  else mxb::quant_t_kernel<mxb::MODE_AP><<<grid, 256, 0, st>>>(a);
+  MOE_CHECK_LAUNCH();
+  return MOE_OK;
+}
+
+static bool tmap_u8b(CUtensorMap* m, const void* base, uint64_t inner, uint64_t outer) {
+  return moe_host::encode_tmap_2d(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, base, inner, outer, inner, 128, 128);
+}
+
+// dgu = SwiGLU-backward(W_d^T dY) with MXFP8 operands: dYq [rows, H] and W_d^T [E*F, H] along H;
+// dgu [rows, 2F] bf16 and the <v, a> partials [rows, F/128].
+int gemm_dgrad_down_mx(int rows, int E, int H, int F, const void* dYq, const uint8_t* dYq_sf, const void* WdT,
+                       const uint8_t* WdT_sf, const int32_t* offsets, const void* gateup, const float* row_gate,
+                       void* dgu, float* dg_part, cudaStream_t st) {
+  ggmx::Params p{};
+  if (!tmap_u8b(&p.tmA, dYq, H, rows) || !tmap_u8b(&p.tmB0, WdT, H, (uint64_t)E * F)) return MOE_ERR_CUDA;
+  p.tmB1 = p.tmB0;
+  p.M = rows;
+  p.N = F;
+  p.K = H;
+  p.G = E;
+  p.offsets = offsets;
+  p.b_group_rows = F;
+  p.sfa = dYq_sf;
+  p.sfb0 = WdT_sf;
+  p.sfb1 = WdT_sf;
+  p.C = dgu;
+  p.ldc = 2LL * F;
+  p.row_gate = row_gate;
+  p.gateup = static_cast<const __nv_bfloat16*>(gateup);
+  p.dg_part = dg_part;
+  p.status = moe_host::device_status_ptr();
+  const int tiles = ((rows + 127) / 128 + E) * (F / 256);
+  return ggmx::launch<ggmx::EPI_MX_SWIGLU_BWD, false>(p, tiles, st);
+}
+
+// dXp = dgu W_gu with MXFP8 operands: dguq [rows, 2F] and [W_g^T | W_u^T] [E*H, 2F] along F; bf16 [rows, H].
+int gemm_dgrad_gateup_mx(int rows, int E, int H, int F, const void* dguq, const uint8_t* dguq_sf, const void* WguT,
+                         const uint8_t* WguT_sf, const int32_t* offsets, void* dxp, cudaStream_t st) {
+  ggmx::Params p{};
+  if (!tmap_u8b(&p.tmA, dguq, 2ULL * F, rows) || !tmap_u8b(&p.tmB0, WguT, 2ULL * F, (uint64_t)E * H))
+    return MOE_ERR_CUDA;
+  p.tmB1 = p.tmB0;
+  p.M = rows;
+  p.N = H;
+  p.K = 2 * F;
+  p.G = E;
+  p.offsets = offsets;
+  p.b_group_rows = H;
+  p.sfa = dguq_sf;
+  p.sfb0 = WguT_sf;
+  p.sfb1 = WguT_sf;
+  p.C = dxp;
+  p.ldc = H;
+  p.status = moe_host::device_status_ptr();
+  const int tiles = ((rows + 127) / 128 + E) * (H / 256);
+  return ggmx::launch<ggmx::EPI_MX_BF16, false>(p, tiles, st);
+}
+
+// dW[e] = AT[:, seg e] BT[:, seg e]^T for every expert e, with MXFP8 operands quantised along the tokens:
+// AT [M, ldp], BT [N, ldp] (padded segments poff), bf16 out [E, M, N] (rows >= split -> C2 [E, M - split, N]).
+int gemm_wgrad_mx(int E, int M, int N, long long ldp, const void* AT, const uint8_t* AT_sf, const void* BT,
+                  const uint8_t* BT_sf, const int32_t* poff, void* C, void* C2, int split, cudaStream_t st) {
+  ggmx::Params p{};
+  if (!tmap_u8b(&p.tmA, AT, ldp, M) || !tmap_u8b(&p.tmB0, BT, ldp, N)) return MOE_ERR_CUDA;
+  p.tmB1 = p.tmB0;
+  p.M = M;
+  p.N = N;
+  p.K = (int)ldp;
+  p.G = E;
+  p.offsets = poff;
+  p.b_group_rows = 0;
+  p.sfa = AT_sf;
+  p.sfb0 = BT_sf;
+  p.sfb1 = BT_sf;
+  p.C = C;
+  p.C2 = C2;
+  p.c2_row_split = split;
+  p.ldc = N;
+  p.c_group_stride = (long long)(split > 0 ? split : M) * N;
+  p.status = moe_host::device_status_ptr();
+  const int tiles = E * ((M + 127) / 128) * ((N + 255) / 256);
+  return ggmx::launch<ggmx::EPI_MX_BF16, false, true>(p, tiles, st);
+}
+
+}  // namespace moe_impl
+
+extern "C" int moe_quantize_mxfp8_t(const void* src, int32_t batch, int32_t R, int32_t C, void* dst, int64_t ldd,
+                                    uint8_t* sf, void* stream) {
+  if (!src || !dst || !sf || batch < 1 || R < 1 || C < 1) return MOE_ERR_INVALID_ARG;
+  if (R % 32 != 0 || C % 8 != 0 || ldd < R || ldd % 32 != 0) return MOE_ERR_UNSUPPORTED;
+  if ((reinterpret_cast<uintptr_t>(src) & 15u) != 0) return MOE_ERR_ALIGNMENT;
+  mxb::QtArgs a{};
+  a.src = static_cast<const __nv_bfloat16*>(src);
+  a.R = R;
+  a.C = C;
+  a.dst = static_cast<uint8_t*>(dst);
+  a.ldd = ldd;
+  a.sf = sf;
+  const dim3 grid((unsigned)(R / 32), (unsigned)((C + 63) / 64), (unsigned)batch);
+  mxb::quant_t_kernel<mxb::MODE_WEIGHT><<<grid, 256, 0, static_cast<cudaStream_t>(stream)>>>(a);
+  MOE_CHECK_LAUNCH();
+  return MOE_OK;
+}
+
+extern "C" int64_t moe_mxfp8_t_padded_rows(const moe_config* cfg) {
+  if (moe_impl::check_cfg(cfg)) return 0;
+  return moe_impl::padded_rows_max((long long)cfg->T * cfg->k, cfg->E);
+}
+
+extern "C" int moe_quantize_mxfp8_t_grouped(const moe_config* cfg, int32_t mode, const void* src,
+                                            const int32_t* src_of, const float* row_gate, const int32_t* offsets,
+                                            int32_t* poff, int32_t C, void* dst, int64_t ldd, uint8_t* sf,
+                                            void* stream) {
+  int rc = moe_impl::check_cfg(cfg);
+  if (rc) return rc;
+  if (!src || !offsets || !poff || !dst || !sf || mode < 0 || mode > 2) return MOE_ERR_INVALID_ARG;
+  if ((mode == 1 && !src_of) || (mode == 2 && !row_gate)) return MOE_ERR_INVALID_ARG;
+  if (C < 1 || C % 8 != 0) return MOE_ERR_UNSUPPORTED;
+  const long long rows = (long long)cfg->T * cfg->k;
+  if (ldd < moe_impl::padded_rows_max(rows, cfg->E) || ldd % 512 != 0) return MOE_ERR_INVALID_ARG;
+  if ((reinterpret_cast<uintptr_t>(src) & 15u) != 0) return MOE_ERR_ALIGNMENT;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  rc = moe_impl::pad_offsets(offsets, cfg->E, poff, st);
+  if (rc) return rc;
+  return moe_impl::quant_t_rows(mode, src, src_of, row_gate, offsets, poff, cfg->E, rows, C,
+                                static_cast<uint8_t*>(dst), sf, ldd, st);
+}
+
+extern "C" int moe_grouped_gemm_dgrad_mxfp8(const moe_config* cfg, int which, const void* A, const uint8_t* A_sf,
+                                            const void* B, const uint8_t* B_sf, const int32_t* offsets,
+                                            const void* saved_gateup, const float* row_gate, void* out, float* dg,
+                                            void* ws, size_t ws_bytes, void* stream) {
+  using namespace moe_impl;
+  int rc = check_cfg(cfg);
+  if (rc) return rc;
+  if (cfg->H % 256 != 0 || cfg->F % 256 != 0) return MOE_ERR_UNSUPPORTED;
+  if (!A || !A_sf || !B || !B_sf || !offsets || !out) return MOE_ERR_INVALID_ARG;
+  const void* ptrs[] = {A, B, out, saved_gateup};
+  for (const void* q : ptrs)
+    if (q && (reinterpret_cast<uintptr_t>(q) & 15u) != 0) return MOE_ERR_ALIGNMENT;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const int rows = cfg->T * cfg->k, H = cfg->H, F = cfg->F, E = cfg->E;
+  if (which == MOE_GEMM_DOWN) {
+    if (!saved_gateup || !row_gate || !dg) return MOE_ERR_INVALID_ARG;
+    if (!ws || ws_bytes < (size_t)rows * (F / 128) * sizeof(float)) return MOE_ERR_WORKSPACE;
+    float* part = static_cast<float*>(ws);
+    rc = gemm_dgrad_down_mx(rows, E, H, F, A, A_sf, B, B_sf, offsets, saved_gateup, row_gate, out, part, st);
+    if (rc) return rc;
+    return dg_reduce(part, rows, F / 128, dg, st);
+  }
+  if (which != MOE_GEMM_GATEUP_SWIGLU) return MOE_ERR_INVALID_ARG;
+  return gemm_dgrad_gateup_mx(rows, E, H, F, A, A_sf, B, B_sf, offsets, out, st);
+}
+
+extern "C" int moe_grouped_gemm_wgrad_mxfp8(const moe_config* cfg, int which, const void* AT, const uint8_t* AT_sf,
+                                            const void* BT, const uint8_t* BT_sf, const int32_t* poff, int64_t ldp,
+                                            void* dW0, void* dW1, void* stream) {
+  using namespace moe_impl;
+  int rc = check_cfg(cfg);
+  if (rc) return rc;
+  if (!AT || !AT_sf || !BT || !BT_sf || !poff || !dW0) return MOE_ERR_INVALID_ARG;
+  if (ldp < padded_rows_max((long long)cfg->T * cfg->k, cfg->E) || ldp % 512 != 0) return MOE_ERR_INVALID_ARG;
+  if (cfg->H % 256 != 0 || cfg->F % 128 != 0) return MOE_ERR_UNSUPPORTED;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const int H = cfg->H, F = cfg->F, E = cfg->E;
+  if (which == MOE_GEMM_DOWN) return gemm_wgrad_mx(E, H, F, ldp, AT, AT_sf, BT, BT_sf, poff, dW0, nullptr, 0, st);
+  if (which != MOE_GEMM_GATEUP_SWIGLU || !dW1) return MOE_ERR_INVALID_ARG;
+  return gemm_wgrad_mx(E, 2 * F, H, ldp, AT, AT_sf, BT, BT_sf, poff, dW0, dW1, F, st);
+}

@@ -16,7 +16,7 @@ static bool tmap_u8(CUtensorMap* m, const void* base, uint64_t inner, uint64_t o
 
 int gemm_gateup_mx(int rows, int groups, int H, int F, const void* A, const uint8_t* A_sf, const void* Wg,
                    const uint8_t* Wg_sf, const void* Wu, const uint8_t* Wu_sf, const int32_t* offsets,
-                   const float* row_gate, void* C, uint8_t* C_sf, cudaStream_t st) {
+                   const float* row_gate, void* C, uint8_t* C_sf, void* save, cudaStream_t st) {
   ggmx::Params p{};
   if (!tmap_u8(&p.tmA, A, H, rows) || !tmap_u8(&p.tmB0, Wg, H, (uint64_t)groups * F) ||
       !tmap_u8(&p.tmB1, Wu, H, (uint64_t)groups * F))
@@ -34,6 +34,7 @@ int gemm_gateup_mx(int rows, int groups, int H, int F, const void* A, const uint
   p.C_sf = C_sf;
   p.ldc = F;
   p.row_gate = row_gate;
+  p.save_gateup = static_cast<__nv_bfloat16*>(save);
   p.status = moe_host::device_status_ptr();
   const int tiles = ((rows + 127) / 128 + groups) * (F / 128);
   return ggmx::launch<ggmx::EPI_MX_SWIGLU, true>(p, tiles, st);
@@ -68,13 +69,13 @@ int grouped_gemm_fwd(const moe_config* c, int which, const void* A, const uint8_
                      const uint8_t* B0_sf, const void* B1, const uint8_t* B1_sf, const int32_t* offsets,
                      const float* row_gate, void* C, uint8_t* C_sf, void* save, void*, size_t, cudaStream_t st) {
   if (c->H % 256 != 0 || c->F % 128 != 0) return MOE_ERR_UNSUPPORTED;
-  if (save) return MOE_ERR_UNSUPPORTED;  // the MXFP8 path keeps no bf16 pre-activations
   if (!A_sf || !B0_sf) return MOE_ERR_INVALID_ARG;
   if (!a4(A_sf) || !a4(B0_sf) || (B1_sf && !a4(B1_sf)) || (C_sf && !a4(C_sf))) return MOE_ERR_ALIGNMENT;
   const int rows = c->T * c->k;
   if (which == MOE_GEMM_GATEUP_SWIGLU) {
     if (!B1_sf || !C_sf) return MOE_ERR_INVALID_ARG;
-    return gemm_gateup_mx(rows, c->E, c->H, c->F, A, A_sf, B0, B0_sf, B1, B1_sf, offsets, row_gate, C, C_sf, st);
+    return gemm_gateup_mx(rows, c->E, c->H, c->F, A, A_sf, B0, B0_sf, B1, B1_sf, offsets, row_gate, C, C_sf, save,
+                          st);
   }
   return gemm_down_mx(rows, c->E, c->H, c->F, A, A_sf, B0, B0_sf, offsets, C, st);
 }
@@ -162,8 +163,8 @@ int layer_fwd_mxfp8(const moe_config* c, const void* x, const void* W_r, const f
                     const void* W_u, const void* W_d, const uint8_t* W_g_sf, const uint8_t* W_u_sf,
                     const uint8_t* W_d_sf, const void* Ws_g, const void* Ws_u, const void* Ws_d,
                     const uint8_t* Ws_g_sf, const uint8_t* Ws_u_sf, const uint8_t* Ws_d_sf, void* y, float* aux,
-                    int32_t* idx, float* gates, int32_t* counts, int32_t* offsets, void* ws, size_t ws_bytes,
-                    cudaStream_t st) {
+                    int32_t* idx, float* gates, int32_t* counts, int32_t* offsets, void* saved, void* ws,
+                    size_t ws_bytes, cudaStream_t st) {
   if (c->H % 256 != 0 || c->F % 128 != 0) return MOE_ERR_UNSUPPORTED;
   if (!W_g_sf || !W_u_sf || !W_d_sf) return MOE_ERR_INVALID_ARG;
   if (c->n_shared && (!Ws_g_sf || !Ws_u_sf || !Ws_d_sf)) return MOE_ERR_INVALID_ARG;
@@ -173,19 +174,34 @@ int layer_fwd_mxfp8(const moe_config* c, const void* x, const void* W_r, const f
   MxWs w;
   if (!ws || ws_bytes < carve_mx(nullptr, c, &w)) return MOE_ERR_WORKSPACE;
   carve_mx(ws, c, &w);
+  __nv_bfloat16* save_gu = nullptr;
+  if (c->save_for_bwd) {
+    // the routing state and the bf16 gate/up pre-activations go to `saved` for the MXFP8 backward
+    Carve cs(saved);
+    const SavedMx sv = carve_saved_mx(cs, c);
+    w.probs = sv.probs;
+    w.idx = sv.idx;
+    w.gates = sv.gates;
+    w.counts = sv.counts;
+    w.offsets = sv.offsets;
+    w.row_of = sv.row_of;
+    w.src_of = sv.src_of;
+    w.row_gate = sv.row_gate;
+    save_gu = sv.gateup;
+  }
   const int T = c->T, H = c->H, F = c->F, E = c->E, k = c->k, rows = T * k;
   RCM(router_topk(c, x, W_r, bias, sel_bias, w.logits, w.probs, w.idx, w.gates, w.counts, c->compute_aux ? aux : nullptr,
                   w.router_ws, router_ws(c), st));
   RCM(permute(c, x, w.idx, w.gates, nullptr, w.offsets, w.row_of, w.src_of, w.row_gate, w.xp, w.xp_sf,
               w.permute_ws, permute_ws(c), st));
   RCM(gemm_gateup_mx(rows, E, H, F, w.xp, w.xp_sf, W_g, W_g_sf, W_u, W_u_sf, w.offsets, w.row_gate, w.ap, w.ap_sf,
-                     st));
+                     save_gu, st));
   RCM(gemm_down_mx(rows, E, H, F, w.ap, w.ap_sf, W_d, W_d_sf, w.offsets, w.o, st));
   if (c->n_shared) {
     RCM(fill_offsets2(w.off2, T, st));
     RCM(quantize_mxfp8(x, T, H, w.xq, w.xq_sf, st));
     RCM(gemm_gateup_mx(T, 1, H, F, w.xq, w.xq_sf, Ws_g, Ws_g_sf, Ws_u, Ws_u_sf, w.off2, nullptr, w.as_, w.as_sf,
-                       st));
+                       nullptr, st));
     RCM(gemm_down_mx(T, 1, H, F, w.as_, w.as_sf, Ws_d, Ws_d_sf, w.off2, w.so, st));
   }
   RCM(unpermute(c, w.o, w.row_of, w.so, y, st));

@@ -390,6 +390,17 @@ int scatter_rows(const moe_config* c, const void* x, const int32_t* row_of, void
   return MOE_OK;
 }
 
+// rows of x [T, H] to their permuted positions, quantised to MXFP8 along H on the way
+int scatter_rows_mx(const moe_config* c, const void* x, const int32_t* row_of, uint8_t* xq, uint8_t* xq_sf,
+                    cudaStream_t st) {
+  const int sgrid = (c->T + perm::SC_WARPS - 1) / perm::SC_WARPS;
+  perm::scatter_kernel<1, true><<<sgrid, perm::SC_WARPS * 32, 0, st>>>(
+      static_cast<const __nv_bfloat16*>(x), c->T, c->H, c->E, c->k, nullptr, nullptr, nullptr, nullptr, nullptr,
+      const_cast<int32_t*>(row_of), nullptr, nullptr, xq, xq_sf);
+  MOE_CHECK_LAUNCH();
+  return MOE_OK;
+}
+
 int unpermute(const moe_config* c, const void* o, const int32_t* row_of, const void* extra, void* y, cudaStream_t st) {
   int rc = check_cfg(c);
   if (rc) return rc;

@@ -83,6 +83,9 @@ WORKLOADS = {
     # and the capacity factor (1.25) on the skewed fwd+bwd step
     "dsv3-grouped": Workload("dsv3-grouped", T=8192, H=7168, E=256, k=8, F=2048, S=1, score="sigmoid",
                              route_scale=2.5, dtype="mxfp8", aux=False, n_group=8, topk_group=4, sel_bias=True),
+    # the MXFP8 backward on the DeepSeek-V3 routed experts (the backward has no shared expert)
+    "dsv3-train": Workload("dsv3-train", T=8192, H=7168, E=256, k=8, F=2048, score="sigmoid", route_scale=2.5,
+                           dtype="mxfp8", aux=False, bwd=True),
     "skewed-capacity": Workload("skewed-capacity", T=8192, H=4096, E=128, k=8, F=1536, skew=True, bwd=True,
                                 capacity_factor=1.25),
 }
