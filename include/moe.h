@@ -264,11 +264,14 @@ int moe_quantize_mxfp8(const void* src, int64_t rows, int32_t K, uint8_t* dst, u
  *   (each expert's segment rounded up to a multiple of 128 rows), and
  *   dst [C, ldd] e4m3 / sf [C, ldd/32] ue8m0 receive, for expert e and its
  *   i-th row, dst[c, poff[e] + i] = the code of that row's column c, in
- *   blocks of 32 consecutive padded rows (pad rows are zero). The source row
+ *   blocks of 32 consecutive padded rows (pad rows are zero). sf is TILED for
+ *   the weight-gradient GEMM's scale copies: the scale of row c and 32-block
+ *   j = p/32 is byte ((c/128) * (ldd/128) + j/4) * 512 + 16 (c%32) +
+ *   4 ((c%128)/32) + j%4 of sf (C * ldd/32 bytes in all). The source row
  *   of permuted row r is, by mode: 0 src[r] (src [T*k, C]); 1 src[src_of[r]]
  *   (src [T, C], e.g. x or dY through the permutation); 2 the gate-folded
  *   activation row_gate[r] * silu(gate) * up recomputed from the saved
- *   pre-activations src [T*k, 2C] (gate columns, then up). C % 8 == 0;
+ *   pre-activations src [T*k, 2C] (gate columns, then up). C % 128 == 0;
  *   ldd >= moe_mxfp8_t_padded_rows(cfg) and ldd % 512 == 0.
  * ------------------------------------------------------------------------ */
 int moe_quantize_mxfp8_t(const void* src, int32_t batch, int32_t R, int32_t C, void* dst, int64_t ldd, uint8_t* sf,

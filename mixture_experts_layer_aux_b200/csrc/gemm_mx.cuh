@@ -55,8 +55,10 @@ constexpr int TMEM_COLS = 512;
 constexpr int SF_COL = 256;             // TMEM scale slots after the accumulator
 constexpr int SF_SLOT_COLS = 12;        // one k-block: SFA 4 columns, SFB 8 columns
 constexpr int BAR_BYTES = 1024;
+constexpr int STG_WARP_BYTES = 32 * 32;  // bf16 epilogue staging: 32 rows x 16 columns per epilogue warp
 constexpr int SMEM_BYTES =
-    1024 + kStages * STAGE_BYTES + kSfBufs * SF_BATCH_BYTES + BAR_BYTES + 2 * (MAX_G + 1) * 4;
+    1024 + kStages * STAGE_BYTES + kSfBufs * SF_BATCH_BYTES + BAR_BYTES + 2 * (MAX_G + 1) * 4 + 16 +
+    8 * STG_WARP_BYTES;
 static_assert(SF_COL + 2 * SF_SLOT_COLS <= TMEM_COLS, "tmem");
 static_assert(SMEM_BYTES <= 232448, "smem");
 
@@ -87,7 +89,10 @@ struct __align__(64) Params {
   int* status;
   // grouped along K (weight gradients): offsets are the groups' K offsets (multiples of BK), A [M, K] and
   // B [N, K] are shared by all groups, group g writes C (+ g c_group_stride); output rows >= c2_row_split
-  // (when > 0) go to C2 instead, at row - c2_row_split
+  // (when > 0) go to C2 instead, at row - c2_row_split. Their scales sfa, sfb0 are then TILED: the
+  // 512-byte chunk of 128-row block rb and k-block kb sits at (rb * K/BK + kb) * 512 in the order the
+  // MMA's scale copies read (byte 16 (r % 32) + 4 ((r % 128) / 32) + j for row r, 32-block j of kb),
+  // so the producer bulk-copies them and the scale loader warp idles
   long long c_group_stride;
   void* C2;
   int c2_row_split;
@@ -207,6 +212,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) gemm_mx_kernel(const __grid_co
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   int* s_off = reinterpret_cast<int*>(bar_area + BAR_BYTES);
   int* s_tstart = s_off + (MAX_G + 1);
+  uint8_t* stg_area =
+      reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(s_tstart + (MAX_G + 1)) + 15) & ~uintptr_t(15));
   constexpr int N_STEP = SPLIT_N ? BN / 2 : BN;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -263,10 +270,39 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) gemm_mx_kernel(const __grid_co
       if (SPLIT_N) tma_prefetch_desc(&p.tmB1);
       int stage = 0;
       uint32_t phase = 0, issued_mask = 0, issued_par = 0;
+      int sb = 0;  // GK: the scale batch this thread fills next
+      uint32_t sphase = 0, s_issued_mask = 0, s_issued_par = 0;
       for (int t = blockIdx.x; t < total && !aborted; t += gridDim.x) {
         const Tile ti = get_tile<GK>(p, t, s_off, s_tstart, N_STEP);
         const int brow = (GK ? 0 : ti.g * p.b_group_rows) + ti.n0;
         for (int kb = 0; kb < ti.nkb; ++kb) {
+          if (GK && kb % SB == 0) {
+            // the batch's tiled scale chunks: SFA of the m-block, SFB of the (one or two) n-blocks
+            if (!mbar_wait(&sempty[sb], sphase ^ 1, abort_flag, p.status, DEV_WAIT_TIMEOUT_PRODUCER)) {
+              aborted = true;
+              break;
+            }
+            const int nb = min(SB, ti.nkb - kb);
+            const int kbt = p.K / BK;
+            const bool two = ti.n0 + 128 < p.N;
+            mbar_arrive_expect_tx(&sfull[sb], (uint32_t)nb * (two ? 3u : 2u) * 512u);
+            s_issued_mask |= 1u << sb;
+            s_issued_par = (s_issued_par & ~(1u << sb)) | (sphase << sb);
+            uint8_t* sf = sf_area + sb * SF_BATCH_BYTES;
+            for (int j = 0; j < nb; ++j) {
+              const long long kbg = ti.kb0 + kb + j;
+              bulk_load(sf + j * SF_KB_BYTES, p.sfa + ((long long)(ti.m0 / 128) * kbt + kbg) * 512, 512, &sfull[sb]);
+              bulk_load(sf + j * SF_KB_BYTES + SFA_BYTES, p.sfb0 + ((long long)(ti.n0 / 128) * kbt + kbg) * 512, 512,
+                        &sfull[sb]);
+              if (two)
+                bulk_load(sf + j * SF_KB_BYTES + SFA_BYTES + 512,
+                          p.sfb0 + ((long long)(ti.n0 / 128 + 1) * kbt + kbg) * 512, 512, &sfull[sb]);
+            }
+            if (++sb == kSfBufs) {
+              sb = 0;
+              sphase ^= 1;
+            }
+          }
           if (!mbar_wait(&empty[stage], phase ^ 1, abort_flag, p.status, DEV_WAIT_TIMEOUT_PRODUCER)) {
             aborted = true;
             break;
@@ -292,6 +328,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) gemm_mx_kernel(const __grid_co
         }
       }
       if (*abort_flag) {
+        // every copy this thread issued lands before the CTA can exit
         for (int s = 0; s < kStages; ++s)
           if (issued_mask & (1u << s)) {
             const uint32_t par = (issued_par >> s) & 1u;
@@ -299,10 +336,19 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) gemm_mx_kernel(const __grid_co
             while (!mbar_try_wait(&full[s], par) && globaltimer_ns() - t0 < MOE_WAIT_NS) {
             }
           }
+        for (int s = 0; s < kSfBufs; ++s)
+          if (s_issued_mask & (1u << s)) {
+            const uint32_t par = (s_issued_par >> s) & 1u;
+            const uint64_t t0 = globaltimer_ns();
+            while (!mbar_try_wait(&sfull[s], par) && globaltimer_ns() - t0 < MOE_WAIT_NS) {
+            }
+          }
       }
     }
   } else if (warp == 2) {
     // ======================= scale loader: natural [rows, K/32] bytes -> UTCCP chunk order, SB k-blocks at a time
+    // (grouped along K the producer bulk-copies tiled scales instead, and this warp has nothing to do)
+    if constexpr (!GK) {
     const int kw = p.K / 32;  // scale bytes per row (a multiple of 4)
     const uint8_t* sfb1 = SPLIT_N ? p.sfb1 : p.sfb0;
     // one 16-byte load per row and batch where every row start is 16-byte aligned
@@ -387,6 +433,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) gemm_mx_kernel(const __grid_co
           sphase ^= 1;
         }
       }
+    }
     }
   } else if (warp == 1) {
     // ======================= MMA issuer
@@ -570,30 +617,45 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) gemm_mx_kernel(const __grid_co
                            pack_bf16x2(duv[6], duv[7]));
           }
           p.dg_part[orow * (long long)(p.N / 128) + col0 / 128] = part;
-        } else {
-          __nv_bfloat16* out;
-          if constexpr (GK) {
-            long long r = orow;
-            void* base = p.C;
-            if (p.c2_row_split > 0 && r >= p.c2_row_split) {
-              r -= p.c2_row_split;
-              base = p.C2;
-            }
-            out = reinterpret_cast<__nv_bfloat16*>(base) + ti.g * p.c_group_stride + r * p.ldc + ti.n0 + 128 * h;
-          } else {
-            out = reinterpret_cast<__nv_bfloat16*>(p.C) + orow * p.ldc + ti.n0 + 128 * h;
-          }
-          const int ncol = min(128, p.N - ti.n0 - 128 * h);  // columns of this half inside the output
+        }
+      }
+      if constexpr (EPI == EPI_MX_BF16) {
+        // 16 columns at a time through shared memory, so that each warp store writes whole 32-byte
+        // sectors: lanes 2i, 2i+1 write the two halves of one row's 32 bytes (16 rows per store)
+        uint8_t* stg = stg_area + (warp - 3) * STG_WARP_BYTES;
+        const int ncol = min(128, p.N - ti.n0 - 128 * h);  // columns of this half inside the output
 #pragma unroll
-          for (int c = 0; c < 16; ++c) {
-            if (8 * c >= ncol) break;
-            uint4 u;
-            u.x = pack_bf16x2(v[8 * c], v[8 * c + 1]);
-            u.y = pack_bf16x2(v[8 * c + 2], v[8 * c + 3]);
-            u.z = pack_bf16x2(v[8 * c + 4], v[8 * c + 5]);
-            u.w = pack_bf16x2(v[8 * c + 6], v[8 * c + 7]);
-            reinterpret_cast<uint4*>(out)[c] = u;
+        for (int pass = 0; pass < 8; ++pass) {
+          if (16 * pass >= ncol) break;  // warp-uniform
+          *reinterpret_cast<uint4*>(stg + lane * 32) =
+              make_uint4(pack_bf16x2(v[16 * pass], v[16 * pass + 1]), pack_bf16x2(v[16 * pass + 2], v[16 * pass + 3]),
+                         pack_bf16x2(v[16 * pass + 4], v[16 * pass + 5]),
+                         pack_bf16x2(v[16 * pass + 6], v[16 * pass + 7]));
+          *reinterpret_cast<uint4*>(stg + lane * 32 + 16) =
+              make_uint4(pack_bf16x2(v[16 * pass + 8], v[16 * pass + 9]),
+                         pack_bf16x2(v[16 * pass + 10], v[16 * pass + 11]),
+                         pack_bf16x2(v[16 * pass + 12], v[16 * pass + 13]),
+                         pack_bf16x2(v[16 * pass + 14], v[16 * pass + 15]));
+          __syncwarp();
+#pragma unroll
+          for (int i = 0; i < 2; ++i) {
+            const int rr = 16 * i + (lane >> 1);
+            const int trow = q * 32 + rr;  // row within the tile
+            if (trow < ti.m_valid) {
+              long long r = (long long)ti.row0 + trow;
+              __nv_bfloat16* base = reinterpret_cast<__nv_bfloat16*>(p.C);
+              if constexpr (GK) {
+                if (p.c2_row_split > 0 && r >= p.c2_row_split) {
+                  r -= p.c2_row_split;
+                  base = reinterpret_cast<__nv_bfloat16*>(p.C2);
+                }
+                base += ti.g * p.c_group_stride;
+              }
+              *reinterpret_cast<uint4*>(base + r * p.ldc + ti.n0 + 128 * h + 16 * pass + 8 * (lane & 1)) =
+                  *reinterpret_cast<const uint4*>(stg + rr * 32 + 16 * (lane & 1));
+            }
           }
+          __syncwarp();
         }
       }
     }

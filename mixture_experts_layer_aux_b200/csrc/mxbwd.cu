@@ -73,30 +73,37 @@ struct QtArgs {
   uint8_t* sf;               // [C, ldd / 32] (WEIGHT: [B, C, ldd / 32]) ue8m0
 };
 
-// One block: 32 consecutive output positions (padded rows) x 64 columns. The 32 x 64 tile is staged
-// in fp32 through shared memory; then each warp takes 8 columns: lane i holds position i, a warp max
-// gives the 32-row block's amax, and each column's 32 codes leave as one 32-byte store.
+// One block: 32 consecutive output positions (padded rows) x 128 columns. The 32 x 128 tile is staged
+// in fp32 through shared memory; then each warp takes 16 columns: lane i holds position i, a warp max
+// gives the 32-row block's amax, and each column's 32 codes leave as one 32-byte store. The padded
+// offsets are read into shared memory first, so finding the tile's expert is a shared-memory search.
+constexpr int QT_COLS = 128;
 template <int MODE>
 __global__ void __launch_bounds__(256) quant_t_kernel(const QtArgs a) {
-  __shared__ float tile[32][65];
+  __shared__ float tile[32][QT_COLS + 1];
+  __shared__ int s_poff[513];
   __shared__ int s_meta[2];  // first source row of the tile (-1: none), valid rows in the tile
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int p0 = blockIdx.x * 32;  // first output position (padded row)
-  const int c0 = blockIdx.y * 64;
+  const int c0 = blockIdx.y * QT_COLS;
   const int b = MODE == MODE_WEIGHT ? blockIdx.z : 0;
+  if constexpr (MODE != MODE_WEIGHT) {
+    for (int i = tid; i <= a.E; i += blockDim.x) s_poff[i] = a.poff[i];
+    __syncthreads();
+  }
   if (tid == 0) {
     int r0 = -1, nv = 0;
     if constexpr (MODE == MODE_WEIGHT) {
       r0 = p0;
       nv = min(32, a.R - p0);
-    } else if (p0 < a.poff[a.E]) {
+    } else if (p0 < s_poff[a.E]) {
       int lo = 0, hi = a.E - 1;  // expert whose padded segment holds p0
       while (lo < hi) {
         const int mid = (lo + hi + 1) >> 1;
-        if (a.poff[mid] <= p0) lo = mid;
+        if (s_poff[mid] <= p0) lo = mid;
         else hi = mid - 1;
       }
-      const int i = p0 - a.poff[lo];
+      const int i = p0 - s_poff[lo];
       const int cnt = a.off[lo + 1] - a.off[lo];
       r0 = a.off[lo] + i;
       nv = max(0, min(32, cnt - i));
@@ -107,9 +114,10 @@ __global__ void __launch_bounds__(256) quant_t_kernel(const QtArgs a) {
   __syncthreads();
   const int r0 = s_meta[0], nv = s_meta[1];
   if (r0 < 0) return;  // past the padded total (block-uniform)
-  // load: thread t -> row t/8, columns 8*(t%8) .. +7 of the tile
-  {
-    const int rr = tid >> 3, cc = (tid & 7) * 8;
+  // load: thread t -> rows t/16 and t/16 + 16, columns 8*(t%16) .. +7 of the tile
+#pragma unroll
+  for (int half = 0; half < 2; ++half) {
+    const int rr = (tid >> 4) + 16 * half, cc = (tid & 15) * 8;
     float f[8];
 #pragma unroll
     for (int q = 0; q < 8; ++q) f[q] = 0.f;
@@ -141,9 +149,9 @@ __global__ void __launch_bounds__(256) quant_t_kernel(const QtArgs a) {
     dst += (long long)b * a.C * a.ldd;
     sf += (long long)b * a.C * (a.ldd / 32);
   }
-#pragma unroll
-  for (int j = 0; j < 8; ++j) {
-    const int c = warp * 8 + j;
+#pragma unroll 4
+  for (int j = 0; j < QT_COLS / 8; ++j) {
+    const int c = warp * (QT_COLS / 8) + j;
     if (c0 + c >= a.C) break;  // warp-uniform
     const float v = tile[lane][c];
     float am = fabsf(v);
@@ -153,7 +161,16 @@ __global__ void __launch_bounds__(256) quant_t_kernel(const QtArgs a) {
     const float inv = mx_inv_scale(sb);
     const __nv_fp8_storage_t code = __nv_cvt_float_to_fp8(v * inv, __NV_SATFINITE, __NV_E4M3);
     dst[(long long)(c0 + c) * a.ldd + p0 + lane] = code;
-    if (lane == 0) sf[(long long)(c0 + c) * (a.ldd / 32) + p0 / 32] = sb;
+    if (lane == 0) {
+      if constexpr (MODE == MODE_WEIGHT) {
+        sf[(long long)(c0 + c) * (a.ldd / 32) + p0 / 32] = sb;  // natural [C, ldd/32]
+      } else {
+        // tiled for the weight-gradient GEMM: chunk (row block, k-block of 128), then the UTCCP order
+        const int r = c0 + c, kb32 = p0 / 32;
+        sf[((long long)(r / 128) * (a.ldd / 128) + kb32 / 4) * 512 + (r % 32) * 16 + ((r % 128) / 32) * 4 + kb32 % 4] =
+            sb;
+      }
+    }
   }
 }
 
@@ -187,7 +204,7 @@ int quant_t_rows(int mode, const void* src, const int32_t* src_of, const float* 
   a.ldd = ldd;
   a.sf = sf;
   const long long pmax = rows + (long long)mxb::PAD * E;
-  const dim3 grid((unsigned)((pmax + 31) / 32), (unsigned)((C + 63) / 64));
+  const dim3 grid((unsigned)((pmax + 31) / 32), (unsigned)((C + mxb::QT_COLS - 1) / mxb::QT_COLS));
   if (mode == 0) mxb::quant_t_kernel<mxb::MODE_ROWS><<<grid, 256, 0, st>>>(a);
   else if (mode == 1) mxb::quant_t_kernel<mxb::MODE_GATHER><<<grid, 256, 0, st>>>(a);
   else mxb::quant_t_kernel<mxb::MODE_AP><<<grid, 256, 0, st>>>(a);
@@ -289,7 +306,7 @@ extern "C" int moe_quantize_mxfp8_t(const void* src, int32_t batch, int32_t R, i
   a.dst = static_cast<uint8_t*>(dst);
   a.ldd = ldd;
   a.sf = sf;
-  const dim3 grid((unsigned)(R / 32), (unsigned)((C + 63) / 64), (unsigned)batch);
+  const dim3 grid((unsigned)(R / 32), (unsigned)((C + mxb::QT_COLS - 1) / mxb::QT_COLS), (unsigned)batch);
   mxb::quant_t_kernel<mxb::MODE_WEIGHT><<<grid, 256, 0, static_cast<cudaStream_t>(stream)>>>(a);
   MOE_CHECK_LAUNCH();
   return MOE_OK;
@@ -308,7 +325,7 @@ extern "C" int moe_quantize_mxfp8_t_grouped(const moe_config* cfg, int32_t mode,
   if (rc) return rc;
   if (!src || !offsets || !poff || !dst || !sf || mode < 0 || mode > 2) return MOE_ERR_INVALID_ARG;
   if ((mode == 1 && !src_of) || (mode == 2 && !row_gate)) return MOE_ERR_INVALID_ARG;
-  if (C < 1 || C % 8 != 0) return MOE_ERR_UNSUPPORTED;
+  if (C < 1 || C % 128 != 0) return MOE_ERR_UNSUPPORTED;
   const long long rows = (long long)cfg->T * cfg->k;
   if (ldd < moe_impl::padded_rows_max(rows, cfg->E) || ldd % 512 != 0) return MOE_ERR_INVALID_ARG;
   if ((reinterpret_cast<uintptr_t>(src) & 15u) != 0) return MOE_ERR_ALIGNMENT;

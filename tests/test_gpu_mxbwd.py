@@ -33,6 +33,14 @@ def test_weight_transpose_quantise_bit_exact(moe, oracle, B, R, C, extra):
     assert moe.moe_get_device_status() == 0
 
 
+def untile(sf_tiled, C, ldd):
+    """The tiled scale layout of the grouped transposed quantiser -> natural [C, ldd/32]."""
+    r = torch.arange(C)[:, None]
+    j = torch.arange(ldd // 32)[None, :]
+    pos = ((r // 128) * (ldd // 128) + j // 4) * 512 + (r % 32) * 16 + ((r % 128) // 32) * 4 + j % 4
+    return sf_tiled.reshape(-1)[pos.reshape(-1)].reshape(C, ldd // 32)
+
+
 def _grouped_case(moe, T, E, k, C, zero, hot, seed):
     idx = random_routing(T, E, k, seed=seed, zero_experts=zero, hot=hot)
     cnt = torch.bincount(idx.flatten().long(), minlength=E)
@@ -64,8 +72,8 @@ def _expected_segments(oracle, rows_src, off, poff, E, C, ldd):
     return codes, scales
 
 
-@pytest.mark.parametrize("T,E,k,C,zero,hot", [(300, 8, 2, 64, 0, 0.0), (1000, 16, 4, 96, 3, 0.5),
-                                              (64, 4, 1, 8, 3, 0.0)])
+@pytest.mark.parametrize("T,E,k,C,zero,hot", [(300, 8, 2, 128, 0, 0.0), (1000, 16, 4, 384, 3, 0.5),
+                                              (64, 4, 1, 128, 3, 0.0)])
 @pytest.mark.parametrize("mode", [0, 1])
 def test_grouped_transpose_quantise_bit_exact(moe, oracle, T, E, k, C, zero, hot, mode):
     cfg, off, poff_ref, ldd = _grouped_case(moe, T, E, k, C, zero, hot, seed=T + mode)
@@ -89,12 +97,12 @@ def test_grouped_transpose_quantise_bit_exact(moe, oracle, T, E, k, C, zero, hot
     codes, scales = _expected_segments(oracle, rows_src, off, poff_ref, E, C, ldd)
     tot = int(poff_ref[-1])
     assert torch.equal(dst.cpu()[:, :tot], codes[:, :tot])
-    assert torch.equal(sf.cpu()[:, :tot // 32], scales[:, :tot // 32])
+    assert torch.equal(untile(sf.cpu(), C, ldd)[:, :tot // 32], scales[:, :tot // 32])
     assert moe.moe_get_device_status() == 0
 
 
 def test_grouped_transpose_of_recomputed_activation(moe, oracle):
-    T, E, k, F = 500, 8, 2, 96
+    T, E, k, F = 500, 8, 2, 128
     cfg, off, poff_ref, ldd = _grouped_case(moe, T, E, k, F, 1, 0.3, seed=7)
     rows = T * k
     gu = randn_bf16((rows, 2 * F), 1.5, seed=9)
@@ -108,9 +116,10 @@ def test_grouped_transpose_of_recomputed_activation(moe, oracle):
     ap = rg.double()[:, None] * torch.nn.functional.silu(zg) * zu      # the gate-folded activation, fp64
     codes, scales = _expected_segments(oracle, ap.float(), off, poff_ref, E, F, ldd)
     tot = int(poff_ref[-1])
-    got = oracle.mxfp8_decode(dst.cpu()[:, :tot], sf.cpu()[:, :tot // 32])
+    sfn = untile(sf.cpu(), F, ldd)
+    got = oracle.mxfp8_decode(dst.cpu()[:, :tot], sfn[:, :tot // 32])
     ref = oracle.mxfp8_decode(codes[:, :tot], scales[:, :tot // 32])
-    scale = torch.pow(2.0, sf.cpu()[:, :tot // 32].double() - 127.0).repeat_interleave(32, dim=1)
+    scale = torch.pow(2.0, sfn[:, :tot // 32].double() - 127.0).repeat_interleave(32, dim=1)
     check_mx(got, ref, scale)
     assert moe.moe_get_device_status() == 0
 
@@ -154,7 +163,8 @@ def test_wgrad_mxfp8_grouped_along_tokens(moe, oracle, which):
         dW0, dW1 = empty((E, F, H), torch.bfloat16), empty((E, F, H), torch.bfloat16)
     moe.moe_grouped_gemm_wgrad_mxfp8(cfg, 1 if which == "down" else 0, *bufs["A"], *bufs["B"], poff, ldp, dW0, dW1)
     torch.cuda.synchronize()
-    A, B = _dq(oracle, *bufs["A"]), _dq(oracle, *bufs["B"])
+    A = oracle.mxfp8_decode(bufs["A"][0].cpu(), untile(bufs["A"][1].cpu(), M, ldp))
+    B = oracle.mxfp8_decode(bufs["B"][0].cpu(), untile(bufs["B"][1].cpu(), N, ldp))
     p = poff.cpu()
     ref = torch.stack([A[:, int(p[e]):int(p[e + 1])] @ B[:, int(p[e]):int(p[e + 1])].T for e in range(E)])
     got = dW0.cpu() if which == "down" else torch.cat([dW0.cpu(), dW1.cpu()], dim=1)
