@@ -404,6 +404,13 @@ def run_ours(args, rank, ws):
             L.step()
     torch.cuda.synchronize()
     assert moe.moe_get_device_status() == 0
+    # rows the experts compute: every (token, slot) pair, or the kept ones under a capacity factor
+    # (read once, outside the timed region, from a staged routing + permutation)
+    rows_kept = wl.T * wl.k
+    if wl.capacity_factor > 0:
+        L.step()
+        torch.cuda.synchronize()
+        rows_kept = int(L.offsets[-1].item())
 
     if wl.bwd:
         ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
@@ -441,7 +448,7 @@ def run_ours(args, rank, ws):
         stage_ms[n] = sum(ev[i][j].elapsed_time(ev[i][j + 1]) for i in range(args.steps)) / args.steps
 
     # dominant kernel: the grouped gate/up GEMM (2/3 of the expert FLOPs)
-    F, H, rows = wl.F, wl.H, wl.T * wl.k
+    F, H, rows = wl.F, wl.H, rows_kept
     flops_gateup = 4.0 * rows * H * F
     flops_down = 2.0 * rows * H * F
     if wl.dtype == "mxfp8":
@@ -480,7 +487,7 @@ def run_ours(args, rank, ws):
             "hbm_peak_GBps": hbm,
         }
     else:
-        tot = 3.0 * wl.expert_flops_fwd()
+        tot = 3.0 * 6.0 * H * F * (rows_kept + wl.T * wl.S)  # algorithmic fwd + bwd expert FLOPs
         kernels = {"fwd_ms": round(stage_ms["fwd"], 4), "bwd_ms": round(stage_ms["bwd"], 4),
                    "expert_TFLOPs_fwd_bwd": round(tot / (ms * 1e-3) / 1e12, 1)}
         ach = tot / (ms * 1e-3) / 1e12
@@ -491,36 +498,62 @@ def run_ours(args, rank, ws):
     # the same step under CUDA-graph replay (one captured step, replayed K times)
     graph = graph_replay(L, wl, args, st, ws)
 
-    # end to end: public whole-layer call, tokens H2D from pinned memory, y (+aux) D2H, every step
+    # end to end: public whole-layer call, tokens H2D from pinned memory, y (+aux) D2H, every step. The copies
+    # run on two copy streams (H2D, D2H) and overlap the neighbouring steps' compute, double-buffered as an
+    # input pipeline would: step i's tokens go up while step i-1 computes, its output comes down while step
+    # i+1 computes.
     x_host = L.d["x"].cpu().pin_memory()
-    y_host = torch.empty(wl.T, wl.H, dtype=torch.bfloat16).pin_memory()
-    aux_host = torch.empty(1, dtype=torch.float32).pin_memory()
-    x_dev = torch.empty_like(L.d["x"])
-    y_dev = torch.empty_like(L.y)
-    for _ in range(2):
-        x_dev.copy_(x_host, non_blocking=True)
-        L.layer_call(x_dev, y_dev, L.aux)
-        y_host.copy_(y_dev, non_blocking=True)
+    y_host = [torch.empty(wl.T, wl.H, dtype=torch.bfloat16).pin_memory() for _ in range(2)]
+    aux_host = [torch.empty(1, dtype=torch.float32).pin_memory() for _ in range(2)]
+    x_dev = [torch.empty_like(L.d["x"]) for _ in range(2)]
+    y_dev = [torch.empty_like(L.y) for _ in range(2)]
+    aux_dev = [torch.empty_like(L.aux) if L.aux is not None else None for _ in range(2)]
+    h2d_s, d2h_s = torch.cuda.Stream(), torch.cuda.Stream()
+    ev_h2d = [torch.cuda.Event() for _ in range(2)]
+    ev_comp = [torch.cuda.Event() for _ in range(2)]
+    ev_d2h = [torch.cuda.Event() for _ in range(2)]
+
+    def e2e_step(i):
+        b = i % 2
+        with torch.cuda.stream(h2d_s):
+            if i >= 2:
+                h2d_s.wait_event(ev_comp[b])      # step i-2 has finished reading x_dev[b]
+            x_dev[b].copy_(x_host, non_blocking=True)
+            ev_h2d[b].record(h2d_s)
+        st.wait_event(ev_h2d[b])
+        if i >= 2:
+            st.wait_event(ev_d2h[b])              # step i-2's output has left y_dev[b]
+        L.layer_call(x_dev[b], y_dev[b], aux_dev[b])
+        if wl.bwd:
+            L.bwd_call()
+        ev_comp[b].record(st)
+        with torch.cuda.stream(d2h_s):
+            d2h_s.wait_event(ev_comp[b])
+            y_host[b].copy_(y_dev[b], non_blocking=True)
+            if aux_dev[b] is not None:
+                aux_host[b].copy_(aux_dev[b], non_blocking=True)
+            ev_d2h[b].record(d2h_s)
+
+    for i in range(2):
+        e2e_step(i)
     torch.cuda.synchronize()
     barrier(ws)
     a0 = torch.cuda.Event(enable_timing=True)
     a1 = torch.cuda.Event(enable_timing=True)
     a0.record(st)
-    for _ in range(args.steps):
-        x_dev.copy_(x_host, non_blocking=True)
-        L.layer_call(x_dev, y_dev, L.aux)
-        if wl.bwd:
-            L.bwd_call()
-        y_host.copy_(y_dev, non_blocking=True)
-        if L.aux is not None:
-            aux_host.copy_(L.aux, non_blocking=True)
+    for i in range(args.steps):
+        e2e_step(i)
+    st.wait_event(ev_d2h[(args.steps - 1) % 2])
     a1.record(st)
     torch.cuda.synchronize()
     e2e_ms = max_over_ranks(a0.elapsed_time(a1) / args.steps, ws)
     h2d = x_host.numel() * 2
-    d2h = y_host.numel() * 2 + (4 if L.aux is not None else 0)
+    d2h = y_host[0].numel() * 2 + (4 if L.aux is not None else 0)
     assert moe.moe_get_device_status() == 0
 
+    cfg_line = workload_config(wl, ws)
+    if wl.capacity_factor > 0:
+        cfg_line["rows_computed"] = rows_kept  # of T*k: the pairs kept at the experts' capacity
     line = {
         "metric": METRIC,
         "value": aggregate_tokens_per_s(wl.T, ws, ms),
@@ -534,12 +567,13 @@ def run_ours(args, rank, ws):
         "vs_baseline": None,
         "dtype": "mxfp8" if wl.dtype == "mxfp8" else "bf16",
         "data": DATA,
-        "config": workload_config(wl, ws),
+        "config": cfg_line,
         "roofline": roof,
         "kernels": kernels,
         "e2e": {"value": aggregate_tokens_per_s(wl.T, ws, e2e_ms), "unit": "tokens/s", "ms_per_step": round(e2e_ms, 4),
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "api": "moe_layer_fwd" +
-                ("+moe_layer_bwd" if wl.bwd else "")},
+                (("+moe_layer_bwd_mxfp8" if L.mx else "+moe_layer_bwd") if wl.bwd else ""),
+                "copies": "H2D and D2H on their own streams, overlapping the neighbouring steps (double-buffered)"},
         "graph": graph,
         "gpu_launches": L.launches_per_step() * args.steps,
         "clocks": clocks,

@@ -73,18 +73,20 @@ struct QtArgs {
   uint8_t* sf;               // [C, ldd / 32] (WEIGHT: [B, C, ldd / 32]) ue8m0
 };
 
-// One block: 32 consecutive output positions (padded rows) x 128 columns. The 32 x 128 tile is staged
-// in fp32 through shared memory; then each warp takes 16 columns: lane i holds position i, a warp max
-// gives the 32-row block's amax, and each column's 32 codes leave as one 32-byte store. The padded
-// offsets are read into shared memory first, so finding the tile's expert is a shared-memory search.
+// One block: 64 consecutive output positions (padded rows; never two experts: segments start on 128-row
+// boundaries) x 128 columns. The 64 x 128 tile is staged in fp32 through shared memory; then each thread
+// quantises one column of one 32-row half (a 1x32 block along the output's K) and stores its 32 codes.
+// The padded offsets are read into shared memory first, so finding the tile's expert is a shared-memory
+// search.
 constexpr int QT_COLS = 128;
+constexpr int QT_ROWS = 64;
 template <int MODE>
 __global__ void __launch_bounds__(256) quant_t_kernel(const QtArgs a) {
-  __shared__ float tile[32][QT_COLS + 1];
+  __shared__ float tile[QT_ROWS][QT_COLS + 1];
   __shared__ int s_poff[513];
-  __shared__ int s_meta[2];  // first source row of the tile (-1: none), valid rows in the tile
+  __shared__ int s_meta[3];  // first source row (-1: none), valid rows, rows to write
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const int p0 = blockIdx.x * 32;  // first output position (padded row)
+  const int p0 = blockIdx.x * QT_ROWS;  // first output position (padded row)
   const int c0 = blockIdx.y * QT_COLS;
   const int b = MODE == MODE_WEIGHT ? blockIdx.z : 0;
   if constexpr (MODE != MODE_WEIGHT) {
@@ -92,10 +94,10 @@ __global__ void __launch_bounds__(256) quant_t_kernel(const QtArgs a) {
     __syncthreads();
   }
   if (tid == 0) {
-    int r0 = -1, nv = 0;
+    int r0 = -1, nv = 0, nw = 0;
     if constexpr (MODE == MODE_WEIGHT) {
       r0 = p0;
-      nv = min(32, a.R - p0);
+      nv = nw = min(QT_ROWS, a.R - p0);  // R % 32 == 0: 32 or 64
     } else if (p0 < s_poff[a.E]) {
       int lo = 0, hi = a.E - 1;  // expert whose padded segment holds p0
       while (lo < hi) {
@@ -106,18 +108,20 @@ __global__ void __launch_bounds__(256) quant_t_kernel(const QtArgs a) {
       const int i = p0 - s_poff[lo];
       const int cnt = a.off[lo + 1] - a.off[lo];
       r0 = a.off[lo] + i;
-      nv = max(0, min(32, cnt - i));
+      nv = max(0, min(QT_ROWS, cnt - i));
+      nw = QT_ROWS;  // pad rows are written (zero)
     }
     s_meta[0] = r0;
     s_meta[1] = nv;
+    s_meta[2] = nw;
   }
   __syncthreads();
-  const int r0 = s_meta[0], nv = s_meta[1];
+  const int r0 = s_meta[0], nv = s_meta[1], nw = s_meta[2];
   if (r0 < 0) return;  // past the padded total (block-uniform)
-  // load: thread t -> rows t/16 and t/16 + 16, columns 8*(t%16) .. +7 of the tile
+  // load: thread t -> rows t/16 + 16 i, columns 8*(t%16) .. +7 of the tile
 #pragma unroll
-  for (int half = 0; half < 2; ++half) {
-    const int rr = (tid >> 4) + 16 * half, cc = (tid & 15) * 8;
+  for (int it = 0; it < QT_ROWS / 16; ++it) {
+    const int rr = (tid >> 4) + 16 * it, cc = (tid & 15) * 8;
     float f[8];
 #pragma unroll
     for (int q = 0; q < 8; ++q) f[q] = 0.f;
@@ -149,24 +153,38 @@ __global__ void __launch_bounds__(256) quant_t_kernel(const QtArgs a) {
     dst += (long long)b * a.C * a.ldd;
     sf += (long long)b * a.C * (a.ldd / 32);
   }
-#pragma unroll 4
-  for (int j = 0; j < QT_COLS / 8; ++j) {
-    const int c = warp * (QT_COLS / 8) + j;
-    if (c0 + c >= a.C) break;  // warp-uniform
-    const float v = tile[lane][c];
-    float am = fabsf(v);
+  // quantise: thread t takes column t % 128 of the 32-row half t / 128 -- one 1x32 block in registers, its
+  // amax by a plain loop, its 32 codes as two 16-byte stores
+  {
+    const int c = tid % QT_COLS, hb = tid / QT_COLS;
+    if (c0 + c < a.C && 32 * hb < nw) {
+      float v[32];
+      float am = 0.f;
 #pragma unroll
-    for (int o = 16; o > 0; o >>= 1) am = fmaxf(am, __shfl_xor_sync(0xffffffffu, am, o));
-    const uint8_t sb = mx_scale_byte(am);
-    const float inv = mx_inv_scale(sb);
-    const __nv_fp8_storage_t code = __nv_cvt_float_to_fp8(v * inv, __NV_SATFINITE, __NV_E4M3);
-    dst[(long long)(c0 + c) * a.ldd + p0 + lane] = code;
-    if (lane == 0) {
+      for (int i = 0; i < 32; ++i) {
+        v[i] = tile[32 * hb + i][c];
+        am = fmaxf(am, fabsf(v[i]));
+      }
+      const uint8_t sb = mx_scale_byte(am);
+      const float inv = mx_inv_scale(sb);
+      uint32_t w[8];
+#pragma unroll
+      for (int q = 0; q < 8; ++q) {
+        const __nv_fp8x2_storage_t lo =
+            __nv_cvt_float2_to_fp8x2(make_float2(v[4 * q] * inv, v[4 * q + 1] * inv), __NV_SATFINITE, __NV_E4M3);
+        const __nv_fp8x2_storage_t hi =
+            __nv_cvt_float2_to_fp8x2(make_float2(v[4 * q + 2] * inv, v[4 * q + 3] * inv), __NV_SATFINITE, __NV_E4M3);
+        w[q] = (uint32_t)lo | ((uint32_t)hi << 16);
+      }
+      const int p = p0 + 32 * hb;
+      uint4* d4 = reinterpret_cast<uint4*>(dst + (long long)(c0 + c) * a.ldd + p);
+      d4[0] = make_uint4(w[0], w[1], w[2], w[3]);
+      d4[1] = make_uint4(w[4], w[5], w[6], w[7]);
       if constexpr (MODE == MODE_WEIGHT) {
-        sf[(long long)(c0 + c) * (a.ldd / 32) + p0 / 32] = sb;  // natural [C, ldd/32]
+        sf[(long long)(c0 + c) * (a.ldd / 32) + p / 32] = sb;  // natural [C, ldd/32]
       } else {
         // tiled for the weight-gradient GEMM: chunk (row block, k-block of 128), then the UTCCP order
-        const int r = c0 + c, kb32 = p0 / 32;
+        const int r = c0 + c, kb32 = p / 32;
         sf[((long long)(r / 128) * (a.ldd / 128) + kb32 / 4) * 512 + (r % 32) * 16 + ((r % 128) / 32) * 4 + kb32 % 4] =
             sb;
       }
@@ -204,7 +222,8 @@ int quant_t_rows(int mode, const void* src, const int32_t* src_of, const float* 
   a.ldd = ldd;
   a.sf = sf;
   const long long pmax = rows + (long long)mxb::PAD * E;
-  const dim3 grid((unsigned)((pmax + 31) / 32), (unsigned)((C + mxb::QT_COLS - 1) / mxb::QT_COLS));
+  const dim3 grid((unsigned)((pmax + mxb::QT_ROWS - 1) / mxb::QT_ROWS),
+                  (unsigned)((C + mxb::QT_COLS - 1) / mxb::QT_COLS));
   if (mode == 0) mxb::quant_t_kernel<mxb::MODE_ROWS><<<grid, 256, 0, st>>>(a);
   else if (mode == 1) mxb::quant_t_kernel<mxb::MODE_GATHER><<<grid, 256, 0, st>>>(a);
   else mxb::quant_t_kernel<mxb::MODE_AP><<<grid, 256, 0, st>>>(a);
@@ -306,7 +325,8 @@ extern "C" int moe_quantize_mxfp8_t(const void* src, int32_t batch, int32_t R, i
   a.dst = static_cast<uint8_t*>(dst);
   a.ldd = ldd;
   a.sf = sf;
-  const dim3 grid((unsigned)(R / 32), (unsigned)((C + mxb::QT_COLS - 1) / mxb::QT_COLS), (unsigned)batch);
+  const dim3 grid((unsigned)((R + mxb::QT_ROWS - 1) / mxb::QT_ROWS), (unsigned)((C + mxb::QT_COLS - 1) / mxb::QT_COLS),
+                  (unsigned)batch);
   mxb::quant_t_kernel<mxb::MODE_WEIGHT><<<grid, 256, 0, static_cast<cudaStream_t>(stream)>>>(a);
   MOE_CHECK_LAUNCH();
   return MOE_OK;
