@@ -14,7 +14,7 @@ tensors into it and chains its steps in the order the pages give:
 Parity status: every oracle function is pinned by a test in
 tests/test_oracle.py against something other than itself (brute force,
 closed forms, library routines, finite differences, hand-computed OCP MX
-values); none is "parity unpinned".
+and NVFP4 values); none is "parity unpinned".
 """
 from __future__ import annotations
 
@@ -31,9 +31,9 @@ _LIB = os.path.join(_HERE, "libmoe_oracle.so")
 _lock = threading.Lock()
 _lib = None
 
-OC_BF16, OC_MXFP8, OC_F64 = 0, 1, 2
+OC_BF16, OC_MXFP8, OC_F64, OC_NVFP4 = 0, 1, 2, 3
 # rounding points of the precision recipes (see moe_oracle.c)
-RECIPES = {"exact": 0, "mxfp8": 1, "bf16": 2}
+RECIPES = {"exact": 0, "mxfp8": 1, "bf16": 2, "nvfp4": 3}
 
 
 def build(force: bool = False) -> str:
@@ -48,7 +48,8 @@ def build(force: bool = False) -> str:
 
 class _Mat(ctypes.Structure):
     _fields_ = [("kind", ctypes.c_int32), ("cols", ctypes.c_int32), ("rows", ctypes.c_int64),
-                ("data", ctypes.c_void_p), ("sf", ctypes.c_void_p)]
+                ("data", ctypes.c_void_p), ("sf", ctypes.c_void_p), ("gs", ctypes.c_void_p),
+                ("gs_rows", ctypes.c_int64)]
 
 
 def lib():
@@ -66,6 +67,18 @@ def lib():
             _lib.oc_bf16_round.restype = ctypes.c_double
             _lib.oc_bf16_round.argtypes = [ctypes.c_double]
             _lib.oc_num_threads.restype = ctypes.c_int
+            _lib.oc_e2m1_decode.restype = ctypes.c_double
+            _lib.oc_e2m1_decode.argtypes = [ctypes.c_uint8]
+            _lib.oc_e2m1_encode.restype = ctypes.c_uint8
+            _lib.oc_e2m1_encode.argtypes = [ctypes.c_double]
+            _lib.oc_nvfp4_global_scale.restype = ctypes.c_float
+            _lib.oc_nvfp4_global_scale.argtypes = [ctypes.c_float]
+            _lib.oc_nvfp4_scale_byte.restype = ctypes.c_uint8
+            _lib.oc_nvfp4_scale_byte.argtypes = [ctypes.c_float, ctypes.c_float]
+            _lib.oc_nvfp4_quantize_bf16.argtypes = [ctypes.c_long, ctypes.c_int, ctypes.c_void_p, ctypes.c_float,
+                                                    ctypes.c_void_p, ctypes.c_void_p]
+            _lib.oc_bf16_amax.restype = ctypes.c_float
+            _lib.oc_bf16_amax.argtypes = [ctypes.c_long, ctypes.c_void_p]
         return _lib
 
 
@@ -83,18 +96,20 @@ def _chk(t, dtype):
 
 
 class Mat:
-    """A row-major matrix the oracle can read: bf16, MXFP8 (codes+scales) or fp64.
+    """A row-major matrix the oracle can read: bf16, MXFP8 (codes+scales), NVFP4
+    (packed codes + scales + per-matrix encode scales) or fp64.
 
     Keeps the backing tensors alive while the C side holds raw pointers.
     """
 
-    def __init__(self, kind, data, sf=None, rows=None, cols=None):
-        self.kind, self.data, self.sf = kind, data, sf
+    def __init__(self, kind, data, sf=None, rows=None, cols=None, gs=None, gs_rows=0):
+        self.kind, self.data, self.sf, self.gs = kind, data, sf, gs
         if cols is None:
             cols = data.shape[-1]
         if rows is None:
             rows = data.numel() // cols
-        self.s = _Mat(kind, cols, rows, data.data_ptr(), 0 if sf is None else sf.data_ptr())
+        self.s = _Mat(kind, cols, rows, data.data_ptr(), 0 if sf is None else sf.data_ptr(),
+                      0 if gs is None else gs.data_ptr(), gs_rows)
 
     @property
     def ref(self):
@@ -113,6 +128,17 @@ def mat(t: torch.Tensor) -> Mat:
 
 def mat_mx(codes: torch.Tensor, sf: torch.Tensor) -> Mat:
     return Mat(OC_MXFP8, _chk(codes.contiguous(), torch.uint8), _chk(sf.contiguous(), torch.uint8))
+
+
+def mat_nv(packed: torch.Tensor, sf: torch.Tensor, gs: torch.Tensor | None) -> Mat:
+    """NVFP4 matrix: packed [..., R, C/2], sf [..., R, C/16], gs [...] fp32 (one G per [R, C] matrix) or None."""
+    packed = _chk(packed.contiguous(), torch.uint8)
+    cols = 2 * packed.shape[-1]
+    R = packed.shape[-2] if packed.dim() >= 2 else 1
+    if gs is not None:
+        gs = _chk(gs.reshape(-1).contiguous(), torch.float32)
+    return Mat(OC_NVFP4, packed, _chk(sf.contiguous(), torch.uint8), rows=packed.numel() * 2 // cols, cols=cols,
+               gs=gs, gs_rows=R)
 
 
 def nthreads() -> int:
@@ -165,6 +191,63 @@ def mxfp8_decode(codes: torch.Tensor, scales: torch.Tensor) -> torch.Tensor:
     v = table[codes.long()]
     s = torch.pow(2.0, scales.to(torch.float64) - 127.0)
     return v * s.repeat_interleave(32, dim=-1)
+
+
+# ----------------------------------------------------------------- NVFP4
+
+def e2m1_encode(v: float) -> int:
+    return int(lib().oc_e2m1_encode(float(v)))
+
+
+def e2m1_decode(c: int) -> float:
+    return float(lib().oc_e2m1_decode(int(c)))
+
+
+def nvfp4_global_scale(amax: float) -> float:
+    return float(lib().oc_nvfp4_global_scale(float(amax)))
+
+
+def nvfp4_scale_byte(amax: float, G: float = 1.0) -> int:
+    return int(lib().oc_nvfp4_scale_byte(float(amax), float(G)))
+
+
+def nvfp4_quantize(src: torch.Tensor, per_matrix: bool = False):
+    """src [..., K] bf16 (K % 16 == 0) -> (packed uint8 [..., K/2], scales uint8 [..., K/16], G fp32).
+
+    per_matrix: each [R, K] matrix of src [..., R, K] gets G = 6*448/amax(matrix)
+    (G is then [...]); otherwise G = 1 (a 0-d tensor)."""
+    assert src.dtype == torch.bfloat16
+    K = src.shape[-1]
+    assert K % 16 == 0
+    src = src.contiguous()
+    packed = torch.empty(tuple(src.shape[:-1]) + (K // 2,), dtype=torch.uint8)
+    scales = torch.empty(tuple(src.shape[:-1]) + (K // 16,), dtype=torch.uint8)
+    if not per_matrix:
+        lib().oc_nvfp4_quantize_bf16(src.numel() // K, K, _p(src), 1.0, _p(packed), _p(scales))
+        return packed, scales, torch.tensor(1.0, dtype=torch.float32)
+    R = src.shape[-2]
+    mats = src.view(-1, R, K)
+    pk, sc = packed.view(-1, R, K // 2), scales.view(-1, R, K // 16)
+    G = torch.empty(mats.shape[0], dtype=torch.float32)
+    for b in range(mats.shape[0]):
+        m = mats[b]
+        G[b] = float(lib().oc_nvfp4_global_scale(lib().oc_bf16_amax(m.numel(), _p(m))))
+        lib().oc_nvfp4_quantize_bf16(R, K, _p(m), float(G[b]), _p(pk[b]), _p(sc[b]))
+    return packed, scales, G.view(src.shape[:-2])
+
+
+def nvfp4_decode(packed: torch.Tensor, scales: torch.Tensor, G=None) -> torch.Tensor:
+    """Exact-up-to-the-final-division fp64 values: E2M1 code * E4M3 scale / G (G per [R, K] matrix)."""
+    e2 = torch.tensor([e2m1_decode(c) for c in range(16)], dtype=torch.float64)
+    e4 = torch.tensor([e4m3_decode(c) for c in range(256)], dtype=torch.float64)
+    lo, hi = (packed & 15).long(), (packed >> 4).long()
+    codes = torch.stack([lo, hi], dim=-1).flatten(-2)
+    v = e2[codes] * e4[scales.long()].repeat_interleave(16, dim=-1)
+    if G is not None and G.dim() > 0:
+        v = v / G.to(torch.float64).reshape(tuple(G.shape) + (1, 1))
+    elif G is not None:
+        v = v / float(G)
+    return v
 
 
 # ----------------------------------------------------------------- routing
@@ -288,7 +371,10 @@ def route(logits: torch.Tensor, k: int, score: str = "softmax", norm: bool = Tru
 # ----------------------------------------------------------------- experts
 
 def _wmat(W, sf=None):
-    """Expert weight [E, R, C] (or [R, C]) bf16 / fp64, or MXFP8 codes with sf."""
+    """Expert weight [E, R, C] (or [R, C]) bf16 / fp64, MXFP8 codes with sf, or NVFP4
+    packed codes with sf = (scales, G)."""
+    if isinstance(sf, tuple):
+        return mat_nv(W, sf[0], sf[1])
     if sf is not None:
         return mat_mx(W.reshape(-1, W.shape[-1]), sf.reshape(-1, sf.shape[-1]))
     return mat(W.reshape(-1, W.shape[-1]))
@@ -298,12 +384,13 @@ def moe_fwd_tokens(x, W_g, W_u, W_d, idx, g, toks=None, *, recipe="exact", fold=
                    sf_g=None, sf_u=None, sf_d=None, shared=None, return_shared=False):
     """Layer output rows y[toks] (fp64, unrounded) for given routing (idx [T,k], gates g [T,k] fp64).
 
-    recipe: "exact" (no rounding), "bf16" (the BF16 recipe's rounding points) or
-    "mxfp8" (the weight tensors are MXFP8 codes and sf_* their scales).
+    recipe: "exact" (no rounding), "bf16" (the BF16 recipe's rounding points),
+    "mxfp8" (the weight tensors are MXFP8 codes and sf_* their scales) or "nvfp4"
+    (the weights are packed NVFP4 codes, sf_* = (scales, G) pairs).
     shared = (W_gs, W_us, W_ds[, sf_gs, sf_us, sf_ds]) adds the always-on shared expert.
     """
     rc = _recipe(recipe)
-    mx = rc == RECIPES["mxfp8"]
+    mx = rc in (RECIPES["mxfp8"], RECIPES["nvfp4"])
     T, H = x.shape
     E, F = W_g.shape[0], W_g.shape[1]
     k = idx.shape[1]
@@ -459,7 +546,8 @@ def layer_fwd(wl, inp: dict, toks=None, logits=None, mx_weights=None, recipe=Non
     Routing is computed for every token; outputs y are computed for `toks`
     (default all). logits may be given (fp64/fp32 [T,E]); else the oracle's own.
     mx_weights: for the MXFP8 recipe, the oracle-quantised weights
-    dict(W_g=(codes, sf), W_u=..., W_d=..., [W_gs, W_us, W_ds]).
+    dict(W_g=(codes, sf), W_u=..., W_d=..., [W_gs, W_us, W_ds]); for the NVFP4
+    recipe dict(W_g=(packed, sf, G), ...).
     """
     if logits is None:
         logits = router_logits(inp["x"], inp["W_r"], inp.get("logit_bias"))
@@ -467,12 +555,13 @@ def layer_fwd(wl, inp: dict, toks=None, logits=None, mx_weights=None, recipe=Non
               with_aux=wl.aux and wl.score == "softmax", capacity_factor=getattr(wl, "capacity_factor", 0.0),
               expert_bias=inp.get("expert_bias"), n_group=getattr(wl, "n_group", 0),
               topk_group=getattr(wl, "topk_group", 0))
-    mx = wl.dtype == "mxfp8"
+    mx = wl.dtype in ("mxfp8", "nvfp4")
     if recipe is None:
-        recipe = "mxfp8" if mx else "exact"
+        recipe = wl.dtype if mx else "exact"
     kw = {}
     if mx:
-        W = mx_weights
+        # MXFP8: (codes, scales) pairs; NVFP4: (packed, scales, G) triples
+        W = {n: (w[0], w[1] if len(w) == 2 else (w[1], w[2])) for n, w in mx_weights.items()}
         kw = dict(sf_g=W["W_g"][1], sf_u=W["W_u"][1], sf_d=W["W_d"][1])
         wg, wu, wd = W["W_g"][0], W["W_u"][0], W["W_d"][0]
         shared = None

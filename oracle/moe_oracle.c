@@ -25,6 +25,15 @@
  *    UE8M0 byte, and each element is v/scale rounded to E4M3 (nearest-even,
  *    clamped to +-448).
  *
+ *  - NVFP4 (section 2.4 of the summary runs the expert GEMMs in FP8/FP4, and
+ *    section 3 lists an NVFP4 recipe): NVIDIA's 4-bit format. Elements are
+ *    OCP MX v1.0 FP4 E2M1 (section 5.3.3: magnitudes 0, 0.5, 1, 1.5, 2, 3, 4,
+ *    6); every 16 consecutive elements along K share one positive E4M3 scale
+ *    (amax / 6 times a per-tensor encode scale G, rounded to E4M3), and the
+ *    tensor's fp32 G = 6 * 448 / amax(tensor) makes the largest block scale
+ *    448. The pages fix none of this; the readings used: G per expert
+ *    weight matrix, G = 1 for activations, nearest-even everywhere.
+ *
  * Everything is plain loops in double precision. Expert operands are reached
  * through oc_mat, which decodes one row at a time from bf16, MXFP8 or fp64
  * storage; decoding is exact in every case.
@@ -70,10 +79,12 @@ double oc_bf16_round(double v) {
  *             gate-folded activation, each expert's output; in the backward
  *             the saved pre-activations, dgate/dup, the per-row dXp and the
  *             router-gradient operand). */
-enum { OC_EXACT = 0, OC_MX = 1, OC_BF16R = 2 };
+enum { OC_EXACT = 0, OC_MX = 1, OC_BF16R = 2, OC_NV = 3 };
+/*   OC_NV     NVFP4 recipe: as OC_MX with NVFP4 operands (16-blocks along K,
+ *             activations with G = 1), bf16 expert GEMM outputs. */
 
 static void round_vec(double* v, int n, int recipe) {
-    if (recipe == OC_BF16R || recipe == OC_MX)
+    if (recipe == OC_BF16R || recipe == OC_MX || recipe == OC_NV)
         for (int i = 0; i < n; ++i) v[i] = oc_bf16_round(v[i]);
 }
 
@@ -179,17 +190,109 @@ void oc_mxfp8_quantize_bf16(long rows, int K, const uint16_t* src, uint8_t* code
     }
 }
 
+/* ------------------------------------------------------------ NVFP4 */
+
+/* E2M1 (OCP MX v1.0 section 5.3.3): code bits s.ee.m, exponent bias 1,
+ * exponent field 0 is subnormal (m * 0.5); no Inf or NaN; largest 6. */
+double oc_e2m1_decode(uint8_t c) {
+    int s = (c >> 3) & 1, ef = (c >> 1) & 3, m = c & 1;
+    double v = ef == 0 ? 0.5 * m : ldexp(1.0 + 0.5 * m, ef - 1);
+    return s ? -v : v;
+}
+
+/* Nearest E2M1 code of v: magnitudes above 6 saturate to 6, a tie goes to the
+ * code whose mantissa bit is 0 (round half to even); the sign is kept, zero
+ * included. v is finite. */
+uint8_t oc_e2m1_encode(double v) {
+    uint8_t sign = signbit(v) ? 8 : 0;
+    double a = fabs(v);
+    if (a > 6.0) a = 6.0;
+    int best = 0;
+    double bd = INFINITY;
+    for (int c = 0; c < 8; ++c) {
+        double d = fabs(oc_e2m1_decode((uint8_t)c) - a);
+        if (d < bd || (d == bd && (c & 1) == 0)) {
+            best = c;
+            bd = d;
+        }
+    }
+    return sign | (uint8_t)best;
+}
+
+/* Encode scale G of a tensor with largest magnitude amax: 6 * 448 / amax in
+ * fp32, so that the block holding amax gets the largest E4M3 scale; 1 for an
+ * all-zero tensor. */
+float oc_nvfp4_global_scale(float amax) { return amax > 0.0f ? 2688.0f / amax : 1.0f; }
+
+/* E4M3 scale byte of a 16-block with largest magnitude amax, tensor scale G:
+ * (amax / 6) * G in fp32, rounded to E4M3 (nearest-even, at most 448). */
+uint8_t oc_nvfp4_scale_byte(float amax, float G) {
+    float s = amax / 6.0f;
+    s = s * G;
+    return oc_e4m3_encode((double)s);
+}
+
+/* One 16-block t[16] -> codes[16] (one E2M1 code per byte) and its scale byte.
+ * Element i is t[i] * (G / scale) in fp32, rounded to E2M1; a zero scale
+ * multiplies by 0. Decoding: code * scale / G. */
+static uint8_t nv_block(const float* t, float G, uint8_t* codes) {
+    float amax = 0.0f;
+    for (int i = 0; i < 16; ++i)
+        if (fabsf(t[i]) > amax) amax = fabsf(t[i]);
+    uint8_t sb = oc_nvfp4_scale_byte(amax, G);
+    float sd = (float)oc_e4m3_decode(sb);
+    float r = sd > 0.0f ? G / sd : 0.0f;
+    for (int i = 0; i < 16; ++i) {
+        float u = t[i] * r;
+        codes[i] = oc_e2m1_encode((double)u);
+    }
+    return sb;
+}
+
+/* Quantise rows x K (K % 16 == 0) of bf16 values with tensor scale G:
+ * packed [rows, K/2] (element 2i in the low nibble of byte i, 2i+1 in the
+ * high nibble), scales [rows, K/16]. */
+void oc_nvfp4_quantize_bf16(long rows, int K, const uint16_t* src, float G, uint8_t* packed, uint8_t* scales) {
+    long r;
+#pragma omp parallel for schedule(static)
+    for (r = 0; r < rows; ++r) {
+        float t[16];
+        uint8_t c[16];
+        for (int b = 0; b < K / 16; ++b) {
+            for (int i = 0; i < 16; ++i) t[i] = (float)bf16_to_double(src[r * (long)K + b * 16 + i]);
+            scales[r * (long)(K / 16) + b] = nv_block(t, G, c);
+            for (int i = 0; i < 8; ++i)
+                packed[r * (long)(K / 2) + b * 8 + i] = (uint8_t)(c[2 * i] | (c[2 * i + 1] << 4));
+        }
+    }
+}
+
+/* Largest magnitude of n bf16 values (the input of oc_nvfp4_global_scale). */
+float oc_bf16_amax(long n, const uint16_t* src) {
+    double m = 0.0;
+    for (long i = 0; i < n; ++i) {
+        double a = fabs(bf16_to_double(src[i]));
+        if (a > m) m = a;
+    }
+    return (float)m;
+}
+
 /* ------------------------------------------------------------ matrices */
 
-enum { OC_BF16 = 0, OC_MXFP8 = 1, OC_F64 = 2 };
+enum { OC_BF16 = 0, OC_MXFP8 = 1, OC_F64 = 2, OC_NVFP4 = 3 };
 
-/* Row-major matrix [rows, cols]; for OC_MXFP8, sf holds rows x cols/32 bytes. */
+/* Row-major matrix [rows, cols]; for OC_MXFP8, sf holds rows x cols/32 bytes.
+ * OC_NVFP4: data holds rows x cols/2 packed E2M1 bytes, sf rows x cols/16 E4M3
+ * scales, and gs one encode scale G per gs_rows consecutive rows (one per
+ * expert matrix; NULL: G = 1). */
 typedef struct {
     int32_t kind;
     int32_t cols;
     int64_t rows;
     const void* data;
     const uint8_t* sf;
+    const float* gs;
+    int64_t gs_rows;
 } oc_mat;
 
 static void oc_row(const oc_mat* m, int64_t r, double* out) {
@@ -201,6 +304,14 @@ static void oc_row(const oc_mat* m, int64_t r, double* out) {
         const uint8_t* p = (const uint8_t*)m->data + r * C;
         const uint8_t* s = m->sf + r * (C / 32);
         for (int c = 0; c < C; ++c) out[c] = oc_e4m3_decode(p[c]) * ldexp(1.0, (int)s[c / 32] - 127);
+    } else if (m->kind == OC_NVFP4) {
+        const uint8_t* p = (const uint8_t*)m->data + r * (C / 2);
+        const uint8_t* s = m->sf + r * (C / 16);
+        double G = m->gs ? (double)m->gs[r / m->gs_rows] : 1.0;
+        for (int c = 0; c < C; ++c) {
+            uint8_t code = (p[c / 2] >> (4 * (c & 1))) & 15;
+            out[c] = oc_e2m1_decode(code) * oc_e4m3_decode(s[c / 16]) / G;
+        }
     } else {
         const double* p = (const double*)m->data + r * C;
         for (int c = 0; c < C; ++c) out[c] = p[c];
@@ -215,6 +326,11 @@ static oc_mat oc_slice(const oc_mat* m, int64_t r0, int64_t nrows) {
     else if (m->kind == OC_MXFP8) {
         s.data = (const uint8_t*)m->data + r0 * m->cols;
         s.sf = m->sf + r0 * (m->cols / 32);
+    } else if (m->kind == OC_NVFP4) {
+        /* slices start on a G boundary (one expert matrix) */
+        s.data = (const uint8_t*)m->data + r0 * (m->cols / 2);
+        s.sf = m->sf + r0 * (m->cols / 16);
+        if (m->gs) s.gs = m->gs + r0 / m->gs_rows;
     } else s.data = (const double*)m->data + r0 * m->cols;
     return s;
 }
@@ -276,6 +392,19 @@ static void mx_roundtrip_strided(double* v, long n, long stride) {
         uint8_t sb = oc_mx_scale_byte(amax);
         double X = ldexp(1.0, (int)sb - 127);
         for (long i = 0; i < nb; ++i) v[(b0 + i) * stride] = oc_e4m3_decode(oc_e4m3_encode((double)t[i] / X)) * X;
+    }
+}
+
+/* Round a double vector to the NVFP4 grid of its 16-blocks with G = 1 (the
+ * activation reading), in place: fp32 first, then quantised and decoded. */
+static void nv_roundtrip(double* v, int n) {
+    for (int b = 0; b < n / 16; ++b) {
+        float t[16];
+        uint8_t c[16];
+        for (int i = 0; i < 16; ++i) t[i] = (float)v[b * 16 + i];
+        uint8_t sb = nv_block(t, 1.0f, c);
+        double sd = oc_e4m3_decode(sb);
+        for (int i = 0; i < 16; ++i) v[b * 16 + i] = oc_e2m1_decode(c[i]) * sd;
     }
 }
 
@@ -503,6 +632,7 @@ static void expert_act(const oc_mat* Wg, const oc_mat* Wu, const double* xv, dou
  * along F (MXFP8 recipe) or bf16 (BF16 recipe). */
 static void round_act(double* a, int F, int recipe) {
     if (recipe == OC_MX) mx_roundtrip(a, F);
+    else if (recipe == OC_NV) nv_roundtrip(a, F);
     else if (recipe == OC_BF16R) round_vec(a, F, recipe);
 }
 
@@ -515,13 +645,15 @@ static void round_act(double* a, int F, int recipe) {
  * A slot with idx < 0 (a pair dropped at an expert's capacity) is skipped.
  * fold = 1 evaluates W_d (g a) (the memory-efficient permutation order),
  * fold = 0 evaluates g (W_d a); the two agree up to rounding.
- * recipe (OC_EXACT / OC_MX / OC_BF16R) selects the rounding points:
+ * recipe (OC_EXACT / OC_MX / OC_BF16R / OC_NV) selects the rounding points:
  *   OC_MX: x is rounded to MXFP8 (1x32 blocks along H) before the expert
  *     GEMMs, the gate-folded activation g*a (and the shared expert's a) to
  *     MXFP8 along F before the down projection; the weights are given as
  *     OC_MXFP8 matrices (already quantised);
+ *   OC_NV: as OC_MX with NVFP4 (16-blocks, G = 1) in place of MXFP8 and
+ *     OC_NVFP4 weight matrices;
  *   OC_BF16R: g*a (and the shared a) is rounded to bf16;
- *   both: each expert's down-projection output is rounded to bf16 before
+ *   all three: each expert's down-projection output is rounded to bf16 before
  *     the sum. y itself is returned unrounded.
  * Weight layouts: Wg, Wu [E*F, H]; Wd [E*H, F]; shared Wgs, Wus [F, H], Wds [H, F].
  */
@@ -545,6 +677,7 @@ int oc_moe_fwd_tokens(int T, int H, int E, int k, int F, int S, int recipe, int 
         double* y = y_out + (long)i * H;
         oc_row(x, t, xv);
         if (recipe == OC_MX) mx_roundtrip(xv, H);
+        else if (recipe == OC_NV) nv_roundtrip(xv, H);
         for (int h = 0; h < H; ++h) y[h] = 0.0;
         for (int j = 0; j < k; ++j) {
             int e = idx[(long)t * k + j];
@@ -635,6 +768,7 @@ int oc_expert_rows(int H, int F, int recipe, const oc_mat* xp, const int32_t* e_
         double* rowbuf = (double*)malloc(sizeof(double) * maxd);
         oc_row(xp, r, xv);
         if (recipe == OC_MX) mx_roundtrip(xv, H);
+        else if (recipe == OC_NV) nv_roundtrip(xv, H);
         oc_mat we_g = oc_slice(Wg, (int64_t)e * F, F);
         oc_mat we_u = oc_slice(Wu, (int64_t)e * F, F);
         oc_mat we_d = oc_slice(Wd, (int64_t)e * H, H);

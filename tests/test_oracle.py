@@ -1,9 +1,10 @@
 """Pins of the CPU oracle against things other than itself (no GPU).
 
 Each test ties one oracle function to an independent fact: a dense brute
-force, a library routine (torch fp64 matmul / sort / float8 cast), a closed
-form, an invariant, central finite differences, or hand-computed OCP MX
-values (tests/golden/mxfp8_ocp_cases.txt). A plausible mistake anywhere in the
+force, a library routine (torch fp64 matmul / sort / float8 cast, numpy's
+half-even rounding), a closed form, an invariant, central finite differences,
+or hand-computed OCP MX and NVFP4 values (tests/golden/mxfp8_ocp_cases.txt,
+tests/golden/nvfp4_cases.txt). A plausible mistake anywhere in the
 oracle (a dropped term, a wrong sign or index, a transposed operand) fails at
 least one of them.
 """
@@ -662,3 +663,189 @@ def test_mxfp8_backward_stays_near_exact(oracle):
     assert rms(dx_m - dx_e) <= 0.08 * rms(dx_e)
     for a, b in zip(gw_m, gw_e):
         assert rms(a - b) <= 0.12 * rms(b)
+
+
+# --------------------------------------------------------------- NVFP4
+
+GOLDEN_NV = os.path.join(os.path.dirname(__file__), "golden", "nvfp4_cases.txt")
+
+
+def _golden_nv():
+    elems, scales, blocks = [], [], []
+    with open(GOLDEN_NV) as f:
+        for line in f:
+            line = line.split("#")[0].strip()
+            if not line:
+                continue
+            kind, rest = line.split(None, 1)
+            if kind == "elem":
+                v, c = rest.split()
+                elems.append((float(v), int(c, 16)))
+            elif kind == "scale":
+                a, G, b = rest.split()
+                scales.append((float(a), float(G), int(b, 16)))
+            else:
+                head, tail = rest.split(" : ")
+                name, G, byte = head.split()
+                vals, codes = tail.split(" => ")
+                blocks.append((name, float(G), int(byte, 16), [float(v) for v in vals.split()],
+                               [int(c, 16) for c in codes.split()]))
+    return elems, scales, blocks
+
+
+def test_nvfp4_golden_elements_and_scales(oracle):
+    elems, scales, _ = _golden_nv()
+    assert len(elems) > 20 and len(scales) > 5
+    for v, c in elems:
+        assert oracle.e2m1_encode(v) == c, (v, hex(oracle.e2m1_encode(v)), hex(c))
+    for a, G, b in scales:
+        assert oracle.nvfp4_scale_byte(a, G) == b, (a, G, hex(oracle.nvfp4_scale_byte(a, G)), hex(b))
+
+
+def _nv_quantize_block(vals, G):
+    """One 16-block through the oracle's matrix quantiser with a given G (via a 1-matrix tensor)."""
+    import oracle
+    v = torch.zeros(1, 16, dtype=torch.float32)
+    v[0, :len(vals)] = torch.tensor(vals, dtype=torch.float32)
+    packed = torch.empty(1, 8, dtype=torch.uint8)
+    sc = torch.empty(1, 1, dtype=torch.uint8)
+    src = v.bfloat16()
+    assert torch.equal(src.float(), v), "golden block values must be exact in bf16"
+    oracle.lib().oc_nvfp4_quantize_bf16(1, 16, oracle._p(src), float(G), oracle._p(packed), oracle._p(sc))
+    codes = torch.stack([packed[0] & 15, packed[0] >> 4], dim=-1).flatten().tolist()
+    return int(sc[0, 0]), codes
+
+
+def test_nvfp4_golden_blocks(oracle):
+    _, _, blocks = _golden_nv()
+    for name, G, byte, vals, codes in blocks:
+        sb, got = _nv_quantize_block(vals, G)
+        assert sb == byte, (name, hex(sb), hex(byte))
+        assert got == codes + [0] * (16 - len(codes)), (name, got)
+
+
+def test_e2m1_decode_is_the_ocp_value_table(oracle):
+    mags = [0.0, 0.5, 1.0, 1.5, 2.0, 3.0, 4.0, 6.0]
+    assert [oracle.e2m1_decode(c) for c in range(8)] == mags
+    assert [oracle.e2m1_decode(8 + c) for c in range(8)] == [-m for m in mags]
+
+
+def _e2m1_generic(u: torch.Tensor) -> torch.Tensor:
+    """Round fp64 magnitudes to a 2-bit-significand float with exponents 0..2 and
+    subnormal quantum 0.5, half to even, saturated at 6 (numpy's half-even round)."""
+    import numpy as np
+    a = np.abs(u.numpy())
+    q = np.where(a < 2, 0.5, np.where(a < 4, 1.0, 2.0))
+    r = np.minimum(np.round(a / q) * q, 6.0)
+    return torch.from_numpy(np.copysign(r, u.numpy()))
+
+
+def test_e2m1_encode_matches_generic_half_even_rounding(oracle):
+    g = torch.Generator().manual_seed(5)
+    u = torch.cat([(torch.rand(3000, generator=g, dtype=torch.float64) * 2 - 1) * 7.5,
+                   torch.tensor([0.25, 0.75, 1.25, 1.75, 2.5, 3.5, 5.0, -5.0, 7.0, 0.0])])
+    mine = torch.tensor([oracle.e2m1_decode(oracle.e2m1_encode(float(x))) for x in u], dtype=torch.float64)
+    assert torch.equal(mine, _e2m1_generic(u))
+
+
+def test_nvfp4_quantizer_matches_library_casts_and_error_bound(oracle):
+    """Scales against torch's float8_e4m3fn cast of (amax/6)*G, elements against the generic
+    half-even rounding of v*(G/scale) in fp32; each element within half a grid step of v."""
+    g = torch.Generator().manual_seed(6)
+    w = (torch.randn(3, 24, 64, generator=g) * torch.tensor([0.02, 1.0, 30.0]).view(3, 1, 1)).bfloat16()
+    packed, sc, G = oracle.nvfp4_quantize(w, per_matrix=True)
+    assert G.shape == (3,)
+    for b in range(3):
+        v = w[b].float()
+        amax_t = v.abs().max()
+        assert float(G[b]) == float(torch.tensor(2688.0, dtype=torch.float32) / amax_t)
+        blk = v.view(24, 4, 16)
+        s_f = (blk.abs().amax(-1) / 6.0) * G[b]
+        ref_sb = s_f.to(torch.float8_e4m3fn)
+        assert torch.equal(sc[b].view(24, 4), ref_sb.view(torch.uint8))
+        sd = ref_sb.float()
+        r = torch.where(sd > 0, G[b] / sd, torch.zeros_like(sd))
+        u = (blk * r.unsqueeze(-1)).double()
+        dec = oracle.nvfp4_decode(packed[b], sc[b])  # code * scale (G not divided out)
+        assert torch.equal(dec.view(24, 4, 16) / sd.double().unsqueeze(-1).clamp_min(1e-300)
+                           * (sd.double().unsqueeze(-1) > 0), _e2m1_generic(u) * (sd.double().unsqueeze(-1) > 0))
+        # the block holding the tensor's amax gets the largest scale
+        assert int(sc[b].max()) == 0x7E
+        # round trip within half a grid step (or the saturation gap above 6)
+        full = oracle.nvfp4_decode(packed[b], sc[b], G[b]).view(24, 4, 16)
+        step = torch.where(u.abs() < 2, 0.5, torch.where(u.abs() < 4, 1.0, 2.0))
+        # (+ 1e-6 |u|: u = v * (G / scale) carries fp32 rounding)
+        bound = (torch.where(u.abs() <= 6, step / 2, u.abs() - 6) + 1e-6 * u.abs()) \
+            * (sd.double() / G[b].double()).unsqueeze(-1)
+        assert ((full - blk.double()).abs() <= bound).all()
+
+
+def test_nvfp4_matrix_decode_in_expert_rows_matches_fp64_weights(oracle):
+    """The oracle's NVFP4 matrix reader (nibble order, scale index, G per expert) equals
+    the table decode of the same codes fed as fp64 matrices."""
+    wl = small(T=10, H=64, E=3, k=2, F=32)
+    inp = make_inputs(wl, seed=41)
+    nv = {n: oracle.nvfp4_quantize(inp[n], per_matrix=True) for n in ("W_g", "W_u", "W_d")}
+    dec = {n: oracle.nvfp4_decode(*nv[n]) for n in nv}
+    xp = inp["x"][torch.arange(10) % 10]
+    e_of = torch.tensor([0, 1, 2, 1, 0, 2, 2, 1, 0, 0], dtype=torch.int32)
+    g_of = torch.rand(10, dtype=torch.float64)
+    a = oracle.expert_rows(xp, e_of, g_of, nv["W_g"][0], nv["W_u"][0], nv["W_d"][0],
+                           sf_g=(nv["W_g"][1], nv["W_g"][2]), sf_u=(nv["W_u"][1], nv["W_u"][2]),
+                           sf_d=(nv["W_d"][1], nv["W_d"][2]), want=("zg", "zu", "o"))
+    b = oracle.expert_rows(xp, e_of, g_of, dec["W_g"], dec["W_u"], dec["W_d"], want=("zg", "zu", "o"))
+    for key in ("zg", "zu", "o"):
+        assert torch.allclose(a[key], b[key], rtol=1e-12, atol=1e-15), key
+
+
+def _nv_roundtrip_ref(t: torch.Tensor) -> torch.Tensor:
+    """NVFP4 round trip with G = 1 along the last dim, written with torch casts."""
+    v = t.float().view(*t.shape[:-1], -1, 16)
+    sd = (v.abs().amax(-1) / 6.0).to(torch.float8_e4m3fn).float()
+    r = torch.where(sd > 0, 1.0 / sd, torch.zeros_like(sd))
+    u = (v * r.unsqueeze(-1)).double()
+    return (_e2m1_generic(u) * sd.double().unsqueeze(-1)).view(t.shape)
+
+
+def test_nvfp4_forward_composes_from_quantised_operands(oracle):
+    """recipe nvfp4 = fp64 products of NVFP4 x (G=1), NVFP4 weights (G per expert),
+    the gate-folded activation rounded to NVFP4 (G=1) and bf16 expert outputs."""
+    wl = small(T=16, H=64, E=4, k=2, F=48, S=1)
+    inp = make_inputs(wl, seed=43)
+    logits = oracle.router_logits(inp["x"], inp["W_r"])
+    r = oracle.route(logits, wl.k, "softmax", True, 1.0)
+    names = ("W_g", "W_u", "W_d", "W_gs", "W_us", "W_ds")
+    nv = {n: oracle.nvfp4_quantize(inp[n], per_matrix=True) for n in names}
+    y = oracle.moe_fwd_tokens(inp["x"], nv["W_g"][0], nv["W_u"][0], nv["W_d"][0], r["idx"], r["gates"],
+                              recipe="nvfp4", sf_g=nv["W_g"][1:], sf_u=nv["W_u"][1:], sf_d=nv["W_d"][1:],
+                              shared=(nv["W_gs"][0], nv["W_us"][0], nv["W_ds"][0], nv["W_gs"][1:],
+                                      nv["W_us"][1:], nv["W_ds"][1:]))
+    dec = {n: oracle.nvfp4_decode(*nv[n]) for n in names}
+    xq = _nv_roundtrip_ref(inp["x"])
+    ref = torch.zeros(wl.T, wl.H, dtype=torch.float64)
+    bf = lambda t: t.float().bfloat16().double()  # noqa: E731
+    for t in range(wl.T):
+        for j in range(wl.k):
+            e = int(r["idx"][t, j])
+            zg, zu = dec["W_g"][e] @ xq[t], dec["W_u"][e] @ xq[t]
+            ap = _nv_roundtrip_ref(float(r["gates"][t, j]) * torch.nn.functional.silu(zg) * zu)
+            ref[t] += bf(dec["W_d"][e] @ ap)
+        zg, zu = dec["W_gs"] @ xq[t], dec["W_us"] @ xq[t]
+        ref[t] += bf(dec["W_ds"] @ _nv_roundtrip_ref(torch.nn.functional.silu(zg) * zu))
+    assert torch.allclose(y, ref, rtol=1e-9, atol=1e-12)
+
+
+def test_nvfp4_forward_stays_near_exact(oracle):
+    """NVFP4 is coarse, but the recipe's output tracks the exact forward (a missing 1/G
+    or a misplaced scale would be off by orders of magnitude)."""
+    wl = small(T=32, H=128, E=4, k=2, F=64)
+    inp = make_inputs(wl, seed=44)
+    logits = oracle.router_logits(inp["x"], inp["W_r"])
+    r = oracle.route(logits, wl.k, "softmax", True, 1.0)
+    nv = {n: oracle.nvfp4_quantize(inp[n], per_matrix=True) for n in ("W_g", "W_u", "W_d")}
+    y = oracle.moe_fwd_tokens(inp["x"], nv["W_g"][0], nv["W_u"][0], nv["W_d"][0], r["idx"], r["gates"],
+                              recipe="nvfp4", sf_g=nv["W_g"][1:], sf_u=nv["W_u"][1:], sf_d=nv["W_d"][1:])
+    y0 = oracle.moe_fwd_tokens(inp["x"], inp["W_g"], inp["W_u"], inp["W_d"], r["idx"], r["gates"])
+    rms = y0.pow(2).mean().sqrt()
+    rel = (y - y0).pow(2).mean().sqrt() / rms
+    assert 0.01 < rel < 0.3, float(rel)
