@@ -202,7 +202,11 @@ class Layer:
         d = make_inputs(wl, device="cuda", seed=seed)
         T, H, E, k, F = wl.T, wl.H, wl.E, wl.k, wl.F
         rows = T * k
-        self.mx = wl.dtype == "mxfp8"
+        # block-scaled operands (MXFP8, or NVFP4: two E2M1 codes per byte and a scale per 16)
+        self.mx = wl.dtype in ("mxfp8", "nvfp4")
+        self.nv = wl.dtype == "nvfp4"
+        cw = (lambda K: K // 2) if self.nv else (lambda K: K)       # code bytes per row of K elements
+        sw = (lambda K: K // 16) if self.nv else (lambda K: K // 32)  # scale bytes per row
         if self.mx:
             q = {}
             if wl.bwd:
@@ -216,9 +220,16 @@ class Layer:
                 moe.moe_quantize_mxfp8_t(d["W_u"], self.wgu, self.wgu_sf, ldd=2 * F, col0=F)
             for name in ["W_g", "W_u", "W_d"] + (["W_gs", "W_us", "W_ds"] if wl.S else []):
                 w = d[name]
-                codes = torch.empty(w.shape, dtype=torch.uint8, device="cuda")
-                sf = torch.empty(w.shape[:-1] + (w.shape[-1] // 32,), dtype=torch.uint8, device="cuda")
-                moe.moe_quantize_mxfp8(w, codes, sf)
+                codes = torch.empty(w.shape[:-1] + (cw(w.shape[-1]),), dtype=torch.uint8, device="cuda")
+                if self.nv:
+                    # one buffer: the block scales, then one fp32 encode scale per expert matrix
+                    R, C = w.shape[-2], w.shape[-1]
+                    sf = torch.empty(moe.moe_nvfp4_sf_bytes(w.numel() // (R * C), R, C), dtype=torch.uint8,
+                                     device="cuda")
+                    moe.moe_quantize_nvfp4(w, codes, sf)
+                else:
+                    sf = torch.empty(w.shape[:-1] + (w.shape[-1] // 32,), dtype=torch.uint8, device="cuda")
+                    moe.moe_quantize_mxfp8(w, codes, sf)
                 q[name] = (codes, sf)
                 d[name] = None
             torch.cuda.synchronize()
@@ -235,10 +246,12 @@ class Layer:
         self.row_of = torch.empty(T, k, dtype=torch.int32, device=dev)
         self.src_of = torch.empty(rows, dtype=torch.int32, device=dev)
         self.row_gate = torch.empty(rows, dtype=torch.float32, device=dev)
-        self.xp = torch.empty(rows, H, dtype=torch.uint8 if self.mx else torch.bfloat16, device=dev)
-        self.xp_sf = torch.empty(rows, H // 32, dtype=torch.uint8, device=dev) if self.mx else None
-        self.ap = torch.empty(rows, F, dtype=torch.uint8 if self.mx else torch.bfloat16, device=dev)
-        self.ap_sf = torch.empty(rows, F // 32, dtype=torch.uint8, device=dev) if self.mx else None
+        self.xp = torch.empty(rows, cw(H), dtype=torch.uint8, device=dev) if self.mx else \
+            torch.empty(rows, H, dtype=torch.bfloat16, device=dev)
+        self.xp_sf = torch.empty(rows, sw(H), dtype=torch.uint8, device=dev) if self.mx else None
+        self.ap = torch.empty(rows, cw(F), dtype=torch.uint8, device=dev) if self.mx else \
+            torch.empty(rows, F, dtype=torch.bfloat16, device=dev)
+        self.ap_sf = torch.empty(rows, sw(F), dtype=torch.uint8, device=dev) if self.mx else None
         self.o = torch.empty(rows, H, dtype=torch.bfloat16, device=dev)
         self.y = torch.empty(T, H, dtype=torch.bfloat16, device=dev)
         self.ws_r = moe.workspace(moe.moe_router_workspace_size(self.cfg))
@@ -259,14 +272,15 @@ class Layer:
                                         else moe.moe_layer_bwd_workspace_size(self.cfg))
         if wl.S:
             self.off2 = torch.tensor([0, T], dtype=torch.int32, device=dev)
-            self.as_ = torch.empty(T, F, dtype=torch.uint8 if self.mx else torch.bfloat16, device=dev)
-            self.as_sf = torch.empty(T, F // 32, dtype=torch.uint8, device=dev) if self.mx else None
+            self.as_ = torch.empty(T, cw(F), dtype=torch.uint8, device=dev) if self.mx else \
+                torch.empty(T, F, dtype=torch.bfloat16, device=dev)
+            self.as_sf = torch.empty(T, sw(F), dtype=torch.uint8, device=dev) if self.mx else None
             self.so = torch.empty(T, H, dtype=torch.bfloat16, device=dev)
             self.cfg_sh = moe.make_config(wl, T=T, E=1, k=1, n_shared=0, compute_aux=0, save_for_bwd=0, n_group=0,
                                           topk_group=0, capacity_factor=0.0)
             if self.mx:
-                self.xq = torch.empty(T, H, dtype=torch.uint8, device=dev)
-                self.xq_sf = torch.empty(T, H // 32, dtype=torch.uint8, device=dev)
+                self.xq = torch.empty(T, cw(H), dtype=torch.uint8, device=dev)
+                self.xq_sf = torch.empty(T, sw(H), dtype=torch.uint8, device=dev)
 
     def w(self, name):
         return self.q[name] if self.mx else (self.d[name], None)
@@ -303,7 +317,10 @@ class Layer:
             Wus, sus = self.w("W_us")
             Wds, sds = self.w("W_ds")
             xin, xsf = d["x"], None
-            if self.mx:
+            if self.nv:
+                m.moe_quantize_nvfp4_act(d["x"], self.xq, self.xq_sf)
+                xin, xsf = self.xq, self.xq_sf
+            elif self.mx:
                 m.moe_quantize_mxfp8(d["x"], self.xq, self.xq_sf)
                 xin, xsf = self.xq, self.xq_sf
             m.moe_grouped_gemm_fwd(cs, 0, xin, xsf, Wgs, sgs, Wus, sus, self.off2, None, self.as_, self.as_sf, None,
@@ -318,7 +335,7 @@ class Layer:
     def launches_per_step(self):
         """Kernels of ours launched per step (as the ncu launch list shows them): router GEMM,
         top-k, finalize (+ aux when computed), rank, scan, scatter, gate/up GEMM, down GEMM,
-        unpermute; + the shared expert's two GEMMs (and, for MXFP8, its input quantiser); and
+        unpermute; + the shared expert's two GEMMs (and, block-scaled, its input quantiser); and
         for fwd+bwd the nine kernels of moe_layer_bwd (dY gather, down dgrad with the SwiGLU
         backward, two weight-gradient GEMMs, gate/up dgrad, router backward, two router
         GEMMs, dXp unpermute)."""
@@ -454,6 +471,9 @@ def run_ours(args, rank, ws):
     if wl.dtype == "mxfp8":
         peak_t = P.get("bf16_tflops_sustained", P["bf16_tflops"]) * 2.0
         peak_note = "mxfp8 peak = 2 x measured sustained bf16 (nominal fp8:bf16 ratio)"
+    elif wl.dtype == "nvfp4":
+        peak_t = P.get("bf16_tflops_sustained", P["bf16_tflops"]) * 4.0
+        peak_note = "nvfp4 peak = 4 x measured sustained bf16 (nominal fp4:bf16 ratio, 9 : 2.25 PFLOP/s dense)"
     else:
         peak_t = P.get("bf16_tflops_sustained", P["bf16_tflops"])
         peak_note = "measured sustained bf16 (cuBLAS, seconds-long loop)"
@@ -468,7 +488,8 @@ def run_ours(args, rank, ws):
                 "traffic": measured_traffic(wl.name) if wl.dtype == "bf16" else None,
                 "peak_source": f"{P['source']}: {peak_note}"}
         hbm = P["hbm_gbs"]
-        perm_bytes = T * H * 2 + rows * H * (1 + 1 / 32 if wl.dtype == "mxfp8" else 2) + 16 * rows
+        per_elem = {"mxfp8": 1 + 1 / 32, "nvfp4": 0.5 + 1 / 16}.get(wl.dtype, 2)
+        perm_bytes = T * H * 2 + rows * H * per_elem + 16 * rows
         unperm_bytes = rows * H * 2 + T * H * 2 + (T * H * 2 if wl.S else 0)
         kernels = {
             "router_ms": round(stage_ms["router"], 4),
@@ -565,7 +586,7 @@ def run_ours(args, rank, ws):
         "higher_is_better": True,
         "scaling": "weak",
         "vs_baseline": None,
-        "dtype": "mxfp8" if wl.dtype == "mxfp8" else "bf16",
+        "dtype": wl.dtype,
         "data": DATA,
         "config": cfg_line,
         "roofline": roof,
@@ -594,9 +615,11 @@ class OracleTimer:
         self.h = {k: (v.cpu() if torch.is_tensor(v) else v) for k, v in d.items()}
         del d
         self.mxw = None
+        names = ["W_g", "W_u", "W_d"] + (["W_gs", "W_us", "W_ds"] if wl.S else [])
         if wl.dtype == "mxfp8":
-            names = ["W_g", "W_u", "W_d"] + (["W_gs", "W_us", "W_ds"] if wl.S else [])
             self.mxw = {n: oracle.mxfp8_quantize(self.h[n]) for n in names}
+        elif wl.dtype == "nvfp4":
+            self.mxw = {n: oracle.nvfp4_quantize(self.h[n], per_matrix=True) for n in names}
 
     def run(self, n):
         """Seconds the oracle's layer forward takes on the first n tokens."""

@@ -14,7 +14,10 @@
  *     sync-free kernels: expert sizes stay on the device, no entry point ever
  *     synchronises the host, so every call can be captured in a CUDA graph;
  *   - 3 (contributions) the MXFP8 training recipe on Blackwell: E4M3 elements
- *     with one UE8M0 scale per 1x32 block (OCP MX v1.0).
+ *     with one UE8M0 scale per 1x32 block (OCP MX v1.0); and the NVFP4 tier
+ *     that 2.4 and 3 name for the expert GEMMs (forward only here): E2M1
+ *     elements, one E4M3 scale per 1x16 block and an fp32 encode scale per
+ *     weight matrix (see moe_quantize_nvfp4).
  *
  * Conventions for every entry point:
  *   - All tensor pointers are DEVICE pointers to row-major, contiguous memory
@@ -22,7 +25,8 @@
  *     synchronises; scratch memory is the caller's `ws` buffer, sized by the
  *     matching *_workspace_size() query. Pointers must be 16-byte aligned.
  *   - bf16 = IEEE bfloat16 stored as uint16; e4m3 = OCP FP8 E4M3 ("fn") byte;
- *     ue8m0 = power-of-two scale byte 2^(b-127).
+ *     ue8m0 = power-of-two scale byte 2^(b-127); e2m1 = OCP FP4 E2M1 nibble,
+ *     two per byte, element 2i in the low nibble of byte i ("packed").
  *   - `stream` is a cudaStream_t (NULL = legacy default stream). Work is only
  *     enqueued; results are ready when the stream reaches them.
  *   - Return value: MOE_OK, or an error code returned BEFORE anything is
@@ -59,11 +63,11 @@ typedef enum {
 } moe_status;
 
 typedef enum { MOE_SCORE_SOFTMAX = 0, MOE_SCORE_SIGMOID = 1 } moe_score_fn;
-typedef enum { MOE_DT_BF16 = 0, MOE_DT_MXFP8 = 1 } moe_dtype;
+typedef enum { MOE_DT_BF16 = 0, MOE_DT_MXFP8 = 1, MOE_DT_NVFP4 = 2 } moe_dtype;
 typedef enum { MOE_GEMM_GATEUP_SWIGLU = 0, MOE_GEMM_DOWN = 1 } moe_gemm_kind;
 
 /* Layer shape and routing recipe. Limits: 1 <= k <= min(E, 16); E <= 512;
- * H % 128 == 0; F % 128 == 0 (MXFP8: H, F % 128 too); T >= 1. */
+ * H % 128 == 0; F % 128 == 0 (NVFP4: H, F % 256); T >= 1. */
 typedef struct moe_config {
     int32_t T, H, E, k, F;
     int32_t n_shared;     /* 0, or 1 always-on shared expert of width F */
@@ -141,7 +145,9 @@ int moe_router_topk(const moe_config* cfg, const void* x, const void* W_r, const
  *   xp[row_of[t,j], :] = x[t, :].
  * For expert_dtype == MXFP8 each row is quantised on the way (1x32 blocks
  * along H; block-local, so it commutes with the permutation): xp is e4m3
- * [T*k, H] and xp_sf ue8m0 [T*k, H/32].
+ * [T*k, H] and xp_sf ue8m0 [T*k, H/32]. For NVFP4: xp packed e2m1
+ * [T*k, H/2] and xp_sf e4m3 [T*k, H/16] (encode scale 1, see
+ * moe_quantize_nvfp4_act).
  * Arguments: x [T,H] bf16; idx [T,k] int32 (k distinct experts per token,
  * each in [0,E) -- checked on the device, violations set the status word);
  * gates [T,k] fp32 or NULL (then row_gate must be NULL); outputs as above,
@@ -193,6 +199,11 @@ int moe_permute_noalloc(const moe_config* cfg, const void* x, const int32_t* idx
  * dtype MXFP8: A, B e4m3 with ue8m0 scales per 1x32 block along K (A_sf
  *   [rows, K/32], B_sf [E, N, K/32]); GATEUP writes C as e4m3 + C_sf
  *   [rows, F/32] (quantised from the fp32 epilogue values); DOWN writes bf16.
+ * dtype NVFP4 (H % 256 == 0, F % 256 == 0): A packed e2m1 [rows, K/2] with
+ *   A_sf e4m3 [rows, K/16] (encode scale 1); B, B_sf as moe_quantize_nvfp4
+ *   writes them for [E, N, K] (B_sf ends with the E encode scales G, which the
+ *   epilogue divides out); GATEUP writes C packed [rows, F/2] + C_sf
+ *   [rows, F/16] (encode scale 1); DOWN writes bf16; save_gateup must be NULL.
  * rows = T*k (the routed rows). offsets [E+1] device int32.
  * ------------------------------------------------------------------------ */
 size_t moe_grouped_gemm_workspace_size(const moe_config* cfg, int which);
@@ -245,6 +256,29 @@ int moe_unpermute(const moe_config* cfg, const void* o, const int32_t* row_of, c
  * K % 32 == 0. Used once per weight tensor (W_g, W_u: K = H; W_d: K = F).
  * ------------------------------------------------------------------------ */
 int moe_quantize_mxfp8(const void* src, int64_t rows, int32_t K, uint8_t* dst, uint8_t* sf, void* stream);
+
+/* ------------------------------------------------------------------------
+ * NVFP4 quantisation (the 4-bit tier of 2.4 / 3 of the summary; the format is
+ * NVIDIA's, the elements OCP MX v1.0 5.3.3 E2M1). Per 1x16 block along K with
+ * the tensor's fp32 encode scale G, each step one IEEE fp32 operation:
+ *   scale byte s = e4m3_rn_sat((amax / 6) * G)   (0 for an all-zero block),
+ *   element     = e2m1_rn_sat(v * (G / s))       (0 when s == 0),
+ *   value       = element * s / G.
+ * moe_quantize_nvfp4: weights. src [batch, R, C] bf16 (C % 16 == 0), each
+ *   [R, C] matrix with its own G = 6*448 / amax(matrix) (1 if all zero), so its
+ *   largest block scale is 448. dst packed [batch, R, C/2]; sf is ONE buffer of
+ *   moe_nvfp4_sf_bytes(batch, R, C) bytes: the scales [batch, R, C/16], then
+ *   the batch's G values as fp32 [batch] (batch*R*C/16 must be a multiple of
+ *   4; sf 4-byte aligned). Once per weight tensor: W_g, W_u [E,F,H] (batch E,
+ *   R = F, C = H), W_d [E,H,F]; the shared expert's [F,H] / [H,F] with batch 1.
+ *   Enqueues a 4-byte-per-matrix clear and three kernels.
+ * moe_quantize_nvfp4_act: activations, G = 1: src [rows, K] bf16 -> dst packed
+ *   [rows, K/2], sf [rows, K/16] (no G values).
+ * ------------------------------------------------------------------------ */
+size_t moe_nvfp4_sf_bytes(int32_t batch, int64_t R, int32_t C);
+int moe_quantize_nvfp4(const void* src, int32_t batch, int64_t R, int32_t C, uint8_t* dst, uint8_t* sf,
+                       void* stream);
+int moe_quantize_nvfp4_act(const void* src, int64_t rows, int32_t K, uint8_t* dst, uint8_t* sf, void* stream);
 
 /* ------------------------------------------------------------------------
  * Transposed MXFP8 operands of the MXFP8 backward (the same 1x32 quantiser,
@@ -330,12 +364,16 @@ int moe_layer_bwd_mxfp8(const moe_config* cfg, const void* dY, float d_aux, cons
  *   BF16: W_g, W_u [E,F,H], W_d [E,H,F] bf16, *_sf NULL;
  *   MXFP8: the same tensors as e4m3 with ue8m0 scales (W_g_sf, W_u_sf
  *     [E,F,H/32], W_d_sf [E,H,F/32]), as moe_quantize_mxfp8 produces them;
+ *   NVFP4 (H % 256 == 0, F % 256 == 0, save_for_bwd = 0): packed e2m1 weights
+ *     with their moe_quantize_nvfp4 scale buffers (batch E; the shared
+ *     expert's with batch 1); x is quantised with encode scale 1 on the way;
  *   shared expert (n_shared = 1): Ws_g, Ws_u [F,H], Ws_d [H,F] (+ scales);
  *   y [T,H] bf16 out; aux [1] fp32 out or NULL; idx [T,k], gates [T,k],
  *   counts [E], offsets [E+1] optional outputs (NULL to skip): counts are the
  *   router's (every selected pair, as aux counts them), offsets those of the
  *   kept rows (they differ only under a capacity factor);
- *   saved: moe_layer_saved_size() bytes, filled when save_for_bwd (else NULL).
+ *   saved: moe_layer_saved_size() bytes, filled when save_for_bwd (else NULL;
+ *   0 bytes for NVFP4, which has no backward).
  * ------------------------------------------------------------------------ */
 size_t moe_layer_workspace_size(const moe_config* cfg);
 size_t moe_layer_saved_size(const moe_config* cfg);

@@ -20,7 +20,8 @@ _lock = threading.Lock()
 _lib = None
 
 MOE_SCORE_SOFTMAX, MOE_SCORE_SIGMOID = 0, 1
-MOE_DT_BF16, MOE_DT_MXFP8 = 0, 1
+MOE_DT_BF16, MOE_DT_MXFP8, MOE_DT_NVFP4 = 0, 1, 2
+_DTYPES = {"bf16": MOE_DT_BF16, "mxfp8": MOE_DT_MXFP8, "nvfp4": MOE_DT_NVFP4}
 MOE_GEMM_GATEUP_SWIGLU, MOE_GEMM_DOWN = 0, 1
 
 
@@ -58,6 +59,9 @@ _SIGS = {
     "moe_grouped_gemm_bwd": (_I, [_CFG, _I, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _SZ, _VP]),
     "moe_unpermute": (_I, [_CFG, _VP, _VP, _VP, _VP, _VP]),
     "moe_quantize_mxfp8": (_I, [_VP, ctypes.c_int64, ctypes.c_int32, _VP, _VP, _VP]),
+    "moe_nvfp4_sf_bytes": (_SZ, [ctypes.c_int32, ctypes.c_int64, ctypes.c_int32]),
+    "moe_quantize_nvfp4": (_I, [_VP, ctypes.c_int32, ctypes.c_int64, ctypes.c_int32, _VP, _VP, _VP]),
+    "moe_quantize_nvfp4_act": (_I, [_VP, ctypes.c_int64, ctypes.c_int32, _VP, _VP, _VP]),
     "moe_layer_workspace_size": (_SZ, [_CFG]),
     "moe_layer_saved_size": (_SZ, [_CFG]),
     "moe_layer_fwd": (_I, [_CFG, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP,
@@ -136,7 +140,7 @@ def make_config(wl=None, **kw) -> moe_config:
         d.update(T=wl.T, H=wl.H, E=wl.E, k=wl.k, F=wl.F, n_shared=wl.S,
                  score=MOE_SCORE_SOFTMAX if wl.score == "softmax" else MOE_SCORE_SIGMOID,
                  norm_topk=int(wl.norm_topk), route_scale=wl.route_scale,
-                 expert_dtype=MOE_DT_BF16 if wl.dtype == "bf16" else MOE_DT_MXFP8,
+                 expert_dtype=_DTYPES[wl.dtype],
                  compute_aux=int(wl.aux and wl.score == "softmax"), save_for_bwd=int(wl.bwd),
                  capacity_factor=wl.capacity_factor, n_group=wl.n_group, topk_group=wl.topk_group)
     d.update(kw)
@@ -225,6 +229,25 @@ def moe_quantize_mxfp8(src, dst, sf, stream=None):
     K = src.shape[-1]
     rows = src.numel() // K
     return _check("moe_quantize_mxfp8", load().moe_quantize_mxfp8(_p(src), rows, K, _p(dst), _p(sf), _st(stream)))
+
+
+def moe_nvfp4_sf_bytes(batch: int, R: int, C: int) -> int:
+    return int(load().moe_nvfp4_sf_bytes(batch, R, C))
+
+
+def moe_quantize_nvfp4(src, dst, sf, stream=None):
+    """src [batch, R, C] (or [R, C]) bf16 -> dst packed uint8 [..., C/2], sf uint8 of moe_nvfp4_sf_bytes bytes."""
+    C = src.shape[-1]
+    R = src.shape[-2]
+    batch = src.numel() // (R * C)
+    return _check("moe_quantize_nvfp4", load().moe_quantize_nvfp4(_p(src), batch, R, C, _p(dst), _p(sf), _st(stream)))
+
+
+def moe_quantize_nvfp4_act(src, dst, sf, stream=None):
+    K = src.shape[-1]
+    rows = src.numel() // K
+    return _check("moe_quantize_nvfp4_act",
+                  load().moe_quantize_nvfp4_act(_p(src), rows, K, _p(dst), _p(sf), _st(stream)))
 
 
 def moe_layer_workspace_size(cfg) -> int:

@@ -27,11 +27,22 @@
 // run while they finish the element-wise work.
 // Roles: warp 0 TMA producer, warp 1 MMA issuer (+ TMEM owner), warp 2 scale
 // loader, warps 3..10 epilogue. All waits are bounded like gemm.cuh.
+//
+// NVFP4 (template flag NV; formats in nvfp4.cuh): the same kernel with packed
+// E2M1 operands -- a 128-byte stage row is 256 elements -- and one E4M3 scale
+// per 16 elements: tcgen05.mma kind::mxf4nvf4 with scale_vec::4X, M128 N256
+// K64, four per k-block. A row's 16 scale bytes of one k-block hold the four
+// MMAs' scale words, so one k-block is one scale batch of the same 6 KB (the
+// loader is unchanged: its four "sub-blocks" are the four MMAs instead of four
+// k-blocks), and each MMA reads its own A/B chunks (12 TMEM columns) from a
+// 48-column slot. The weights' per-expert encode scales G are divided out in
+// the epilogue; activations have G = 1.
 #pragma once
 
 #include <cuda_fp8.h>
 
 #include "common.cuh"
+#include "nvfp4.cuh"
 
 namespace ggmx {
 
@@ -54,12 +65,13 @@ constexpr int SF_BATCH_BYTES = SB * SF_KB_BYTES;
 constexpr int TMEM_COLS = 512;
 constexpr int SF_COL = 256;             // TMEM scale slots after the accumulator
 constexpr int SF_SLOT_COLS = 12;        // one k-block: SFA 4 columns, SFB 8 columns
+constexpr int SF_SLOT_COLS_NV = 48;     // NVFP4: four MMAs of 12 columns each
 constexpr int BAR_BYTES = 1024;
 constexpr int STG_WARP_BYTES = 32 * 32;  // bf16 epilogue staging: 32 rows x 16 columns per epilogue warp
 constexpr int SMEM_BYTES =
     1024 + kStages * STAGE_BYTES + kSfBufs * SF_BATCH_BYTES + BAR_BYTES + 2 * (MAX_G + 1) * 4 + 16 +
     8 * STG_WARP_BYTES;
-static_assert(SF_COL + 2 * SF_SLOT_COLS <= TMEM_COLS, "tmem");
+static_assert(SF_COL + 2 * SF_SLOT_COLS_NV <= TMEM_COLS, "tmem");
 static_assert(SMEM_BYTES <= 232448, "smem");
 
 enum Epi : int {
@@ -101,6 +113,9 @@ struct __align__(64) Params {
   __nv_bfloat16* save_gateup;
   const __nv_bfloat16* gateup;
   float* dg_part;
+  // NVFP4: per-group encode scales G of B0 and B1 (NULL: 1); the accumulators are divided by them
+  const float* gscale0;
+  const float* gscale1;
 };
 
 struct Tile {
@@ -142,6 +157,16 @@ __device__ __forceinline__ Tile get_tile(const Params& p, int t, const int* s_of
   return ti;
 }
 
+MOE_DEV void mma_nvf4(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc, uint32_t sfa_tmem,
+                      uint32_t sfb_tmem, uint32_t accumulate) {
+  asm volatile(
+      "{ .reg .pred p; setp.ne.b32 p, %4, 0; "
+      "tcgen05.mma.cta_group::1.kind::mxf4nvf4.block_scale.scale_vec::4X [%0], %1, %2, %3, [%5], [%6], p; }" ::"r"(
+          d_tmem),
+      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate), "r"(sfa_tmem), "r"(sfb_tmem)
+      : "memory");
+}
+
 MOE_DEV void mma_mxf8(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc, uint32_t sfa_tmem,
                       uint32_t sfb_tmem, uint32_t accumulate) {
   asm volatile(
@@ -172,6 +197,12 @@ __host__ __device__ constexpr uint32_t idesc_mx(int M, int N, int sf_id) {
          ((uint32_t)(M >> 4) << 24) | ((uint32_t)sf_id << 29);
 }
 
+// Block-scaled instruction descriptor: E2M1 x E2M1 (format 1 of kind::mxf4nvf4), UE4M3 scales (bit 23 clear),
+// K-major, dense K64.
+__host__ __device__ constexpr uint32_t idesc_nv(int M, int N) {
+  return (1u << 7) | (1u << 10) | ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
+}
+
 // UE8M0 byte of a 1x32 block: clamp(floor(log2 amax) - 8 + 127, 0, 254), 0 for amax == 0.
 MOE_DEV uint8_t mx_scale_byte(float amax) {
   const uint32_t b = __float_as_uint(amax);
@@ -195,8 +226,10 @@ MOE_DEV void quant32(const float* v, float inv, uint32_t (&w)[8]) {
   }
 }
 
-template <int EPI, bool SPLIT_N, bool GK>
+template <int EPI, bool SPLIT_N, bool GK, bool NV>
 __global__ void __launch_bounds__(NUM_THREADS, 1) gemm_mx_kernel(const __grid_constant__ Params p) {
+  static_assert(!(NV && GK), "NVFP4: forward GEMMs only");
+  static_assert(!(NV && EPI == EPI_MX_SWIGLU_BWD), "NVFP4: forward GEMMs only");
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* sf_area = smem + kStages * STAGE_BYTES;
@@ -349,7 +382,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) gemm_mx_kernel(const __grid_co
     // ======================= scale loader: natural [rows, K/32] bytes -> UTCCP chunk order, SB k-blocks at a time
     // (grouped along K the producer bulk-copies tiled scales instead, and this warp has nothing to do)
     if constexpr (!GK) {
-    const int kw = p.K / 32;  // scale bytes per row (a multiple of 4)
+    const int kw = NV ? p.K / 8 : p.K / 32;  // scale bytes per row (a multiple of 4; p.K is A's row bytes)
     const uint8_t* sfb1 = SPLIT_N ? p.sfb1 : p.sfb0;
     // one 16-byte load per row and batch where every row start is 16-byte aligned
     const bool v16 = (kw % 16) == 0 &&
@@ -360,9 +393,11 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) gemm_mx_kernel(const __grid_co
     for (int t = blockIdx.x; t < total && !aborted; t += gridDim.x) {
       const Tile ti = get_tile<GK>(p, t, s_off, s_tstart, N_STEP);
       const long long brow = (GK ? 0LL : (long long)ti.g * p.b_group_rows) + ti.n0;
-      for (int kb0 = 0; kb0 < ti.nkb; kb0 += SB) {
-        const int nb = min(SB, ti.nkb - kb0);
-        const int kbg = ti.kb0 + kb0;  // the batch's first k-block in the operands' K
+      // a batch is SB scale words per row: SB k-blocks (MXFP8) or the SB MMAs of one k-block (NVFP4)
+      const int nbatch = NV ? ti.nkb : (ti.nkb + SB - 1) / SB;
+      for (int bi = 0; bi < nbatch; ++bi) {
+        const int nb = NV ? SB : min(SB, ti.nkb - bi * SB);
+        const int kbg = NV ? SB * (ti.kb0 + bi) : ti.kb0 + bi * SB;  // the batch's first scale word in a row
         if (!__all_sync(0xffffffffu,
                         mbar_wait(&sempty[sb], sphase ^ 1, abort_flag, p.status, DEV_WAIT_TIMEOUT_PRODUCER))) {
           aborted = true;
@@ -449,8 +484,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) gemm_mx_kernel(const __grid_co
       }
       tc_fence_after();
       for (int kb = 0; kb < ti.nkb; ++kb) {
-        const int j = kb % SB;
-        const bool batch_end = (j == SB - 1) || (kb == ti.nkb - 1);
+        const int j = NV ? 0 : kb % SB;
+        const bool batch_end = NV || (j == SB - 1) || (kb == ti.nkb - 1);
         if (j == 0) {
           // a new scale batch in shared memory
           if (!__all_sync(0xffffffffu,
@@ -464,7 +499,25 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) gemm_mx_kernel(const __grid_co
           break;
         }
         tc_fence_after();
-        if (lane == 0) {
+        if (NV && lane == 0) {
+          // four K64 MMAs, each right after the copies of its own A/B scale chunks into its part of the
+          // k-block's slot (slots alternate by k-block, as below)
+          uint8_t* sA = smem + stage * STAGE_BYTES;
+          uint8_t* sB = sA + A_BYTES;
+          const uint32_t a0 = smem_u32(sA), b0 = smem_u32(sB);
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            const uint32_t sa = smem_u32(sf_area + sb * SF_BATCH_BYTES + q * SF_KB_BYTES);
+            const uint32_t col = tmem_base + SF_COL + SF_SLOT_COLS_NV * (kb & 1) + SF_SLOT_COLS * q;
+            tmem_cp_32x128b_x4(col, sf_desc(sa));
+            tmem_cp_32x128b_x4(col + 4, sf_desc(sa + SFA_BYTES));
+            tmem_cp_32x128b_x4(col + 8, sf_desc(sa + SFA_BYTES + 512));
+            mma_nvf4(tmem_base, smem_desc_sw128(a0 + q * 32, 16, 1024), smem_desc_sw128(b0 + q * 32, 16, 1024),
+                     idesc_nv(BM, BN), col, col + 4, (kb | q) != 0 ? 1u : 0u);
+          }
+          mma_commit(&sempty[sb]);
+          mma_commit(&empty[stage]);
+        } else if (!NV && lane == 0) {
           // this k-block's scale chunks into its TMEM slot (alternating by k-block; in issue order
           // after the MMAs that read the slot two k-blocks ago), copied right before its MMAs:
           // on B200 three copies per k-block cost the tensor pipe far less than a batch of twelve
@@ -546,6 +599,13 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) gemm_mx_kernel(const __grid_co
       __syncwarp();
       if (lane == 0) mbar_arrive(tempty);  // accumulator free: the next tile's MMAs may start
       acc_phase ^= 1;
+      if constexpr (NV) {
+        // divide out the weights' encode scales: gate (or down) by G0, up by G1
+        const float i0 = p.gscale0 ? 1.0f / p.gscale0[ti.g] : 1.0f;
+        const float i1 = (EPI == EPI_MX_SWIGLU && p.gscale1) ? 1.0f / p.gscale1[ti.g] : i0;
+#pragma unroll
+        for (int i = 0; i < 128; ++i) v[i] *= i < 64 ? i0 : i1;
+      }
       const bool valid = row < ti.m_valid;
       const long long orow = (long long)ti.row0 + row;
       if (valid) {
@@ -570,22 +630,35 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) gemm_mx_kernel(const __grid_co
           // a = g silu(gate) up, in place over the gate values
 #pragma unroll
           for (int i = 0; i < 64; ++i) v[i] = g * silu_f(v[i]) * v[64 + i];
-          uint8_t* out = reinterpret_cast<uint8_t*>(p.C) + orow * p.ldc + col0;
-          uint8_t sb[2];
-#pragma unroll
-          for (int b = 0; b < 2; ++b) {
-            float am = 0.f;
-#pragma unroll
-            for (int i = 0; i < 32; ++i) am = fmaxf(am, fabsf(v[32 * b + i]));
-            sb[b] = mx_scale_byte(am);
+          if constexpr (NV) {
+            // four 16-blocks: 32 bytes of packed E2M1 (ldc = N/2 bytes per row) and four E4M3 scale bytes
             uint32_t w[8];
-            quant32(v + 32 * b, mx_inv_scale(sb[b]), w);
-            uint4* o4 = reinterpret_cast<uint4*>(out + 32 * b);
+            uint32_t sbw = 0;
+#pragma unroll
+            for (int b = 0; b < 4; ++b)
+              sbw |= (uint32_t)nvq::quant16(v + 16 * b, 1.0f, w[2 * b], w[2 * b + 1]) << (8 * b);
+            uint4* o4 = reinterpret_cast<uint4*>(reinterpret_cast<uint8_t*>(p.C) + orow * p.ldc + col0 / 2);
             o4[0] = make_uint4(w[0], w[1], w[2], w[3]);
             o4[1] = make_uint4(w[4], w[5], w[6], w[7]);
+            *reinterpret_cast<uint32_t*>(p.C_sf + orow * (p.N / 16) + col0 / 16) = sbw;
+          } else {
+            uint8_t* out = reinterpret_cast<uint8_t*>(p.C) + orow * p.ldc + col0;
+            uint8_t sb[2];
+#pragma unroll
+            for (int b = 0; b < 2; ++b) {
+              float am = 0.f;
+#pragma unroll
+              for (int i = 0; i < 32; ++i) am = fmaxf(am, fabsf(v[32 * b + i]));
+              sb[b] = mx_scale_byte(am);
+              uint32_t w[8];
+              quant32(v + 32 * b, mx_inv_scale(sb[b]), w);
+              uint4* o4 = reinterpret_cast<uint4*>(out + 32 * b);
+              o4[0] = make_uint4(w[0], w[1], w[2], w[3]);
+              o4[1] = make_uint4(w[4], w[5], w[6], w[7]);
+            }
+            *reinterpret_cast<uint16_t*>(p.C_sf + orow * (p.ldc / 32) + col0 / 32) =
+                (uint16_t)sb[0] | ((uint16_t)sb[1] << 8);
           }
-          *reinterpret_cast<uint16_t*>(p.C_sf + orow * (p.ldc / 32) + col0 / 32) =
-              (uint16_t)sb[0] | ((uint16_t)sb[1] << 8);
         } else if (EPI == EPI_MX_SWIGLU_BWD) {
           // columns [col0, col0 + 128) of F: dgate, dup from the saved bf16 pre-activations z
           const float g = p.row_gate[orow];
@@ -668,10 +741,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) gemm_mx_kernel(const __grid_co
   }
 }
 
-template <int EPI, bool SPLIT_N, bool GK = false>
+template <int EPI, bool SPLIT_N, bool GK = false, bool NV = false>
 int launch(const Params& p, int max_tiles, cudaStream_t stream) {
   if (max_tiles <= 0) return MOE_OK;
-  auto kern = gemm_mx_kernel<EPI, SPLIT_N, GK>;
+  auto kern = gemm_mx_kernel<EPI, SPLIT_N, GK, NV>;
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES) != cudaSuccess) {
     (void)cudaGetLastError();
     return MOE_ERR_CUDA;

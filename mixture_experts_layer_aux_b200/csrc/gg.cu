@@ -221,6 +221,8 @@ extern "C" int moe_grouped_gemm_fwd(const moe_config* cfg, int which, const void
     return grouped_gemm_fwd(cfg, which, A, A_sf, B0, B0_sf, B1, B1_sf, offsets, row_gate, C, C_sf, save_gateup, ws,
                             ws_bytes, st);
   }
+  if (cfg->expert_dtype == MOE_DT_NVFP4)
+    return grouped_gemm_fwd_nv(cfg, which, A, A_sf, B0, B0_sf, B1, B1_sf, offsets, row_gate, C, C_sf, save_gateup, st);
   if (A_sf || B0_sf || B1_sf || C_sf) return MOE_ERR_INVALID_ARG;
   if (which == MOE_GEMM_GATEUP_SWIGLU)
     return gemm_gateup_bf16(rows, cfg->E, cfg->H, cfg->F, A, B0, B1, offsets, row_gate, C, save_gateup, st);

@@ -429,7 +429,7 @@ extern "C" int moe_layer_bwd_mxfp8(const moe_config* cfg, const void* dY, float 
 
 extern "C" size_t moe_layer_workspace_size(const moe_config* cfg) {
   if (check_cfg(cfg)) return 0;
-  if (cfg->expert_dtype == MOE_DT_MXFP8) return layer_ws_mxfp8(cfg);
+  if (cfg->expert_dtype != MOE_DT_BF16) return layer_ws_mxfp8(cfg);
   FwdWs w;
   return carve_fwd(nullptr, cfg, &w);
 }
@@ -437,6 +437,7 @@ extern "C" size_t moe_layer_workspace_size(const moe_config* cfg) {
 extern "C" size_t moe_layer_saved_size(const moe_config* cfg) {
   if (check_cfg(cfg)) return 0;
   Carve cv(nullptr);
+  if (cfg->expert_dtype == MOE_DT_NVFP4) return 0;  // no NVFP4 backward: nothing is saved
   if (cfg->expert_dtype == MOE_DT_MXFP8) carve_saved_mx(cv, cfg);
   else carve_saved(cv, cfg);
   return cv.used;
@@ -459,7 +460,7 @@ extern "C" int moe_layer_fwd(const moe_config* cfg, const void* x, const void* W
   for (const void* p : ptrs)
     if (p && !al16(p)) return MOE_ERR_ALIGNMENT;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  if (cfg->expert_dtype == MOE_DT_MXFP8) {
+  if (cfg->expert_dtype != MOE_DT_BF16) {
     return layer_fwd_mxfp8(cfg, x, W_r, logit_bias, expert_bias, W_g, W_u, W_d, W_g_sf, W_u_sf, W_d_sf, Ws_g, Ws_u, Ws_d, Ws_g_sf,
                            Ws_u_sf, Ws_d_sf, y, aux, idx, gates, counts, offsets, saved, ws, ws_bytes, st);
   }

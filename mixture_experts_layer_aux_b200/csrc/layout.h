@@ -74,6 +74,17 @@ int gemm_dgrad_gateup_mx(int rows, int E, int H, int F, const void* dguq, const 
                          const uint8_t* WguT_sf, const int32_t* offsets, void* dxp, cudaStream_t st);
 int gemm_wgrad_mx(int E, int M, int N, long long ldp, const void* AT, const uint8_t* AT_sf, const void* BT,
                   const uint8_t* BT_sf, const int32_t* poff, void* C, void* C2, int split, cudaStream_t st);
+size_t nvfp4_sf_bytes(long long batch, long long R, long long C);
+int quantize_nvfp4(const void* src, int batch, long long R, int C, uint8_t* dst, uint8_t* sf, cudaStream_t st);
+int quantize_nvfp4_act(const void* src, long long rows, int K, uint8_t* dst, uint8_t* sf, cudaStream_t st);
+int gemm_gateup_nv(int rows, int groups, int H, int F, const void* A, const uint8_t* A_sf, const void* Wg,
+                   const uint8_t* Wg_sf, const float* Wg_gs, const void* Wu, const uint8_t* Wu_sf, const float* Wu_gs,
+                   const int32_t* offsets, const float* row_gate, void* C, uint8_t* C_sf, cudaStream_t st);
+int gemm_down_nv(int rows, int groups, int H, int F, const void* A, const uint8_t* A_sf, const void* Wd,
+                 const uint8_t* Wd_sf, const float* Wd_gs, const int32_t* offsets, void* C, cudaStream_t st);
+int grouped_gemm_fwd_nv(const moe_config* c, int which, const void* A, const uint8_t* A_sf, const void* B0,
+                        const uint8_t* B0_sf, const void* B1, const uint8_t* B1_sf, const int32_t* offsets,
+                        const float* row_gate, void* C, uint8_t* C_sf, void* save, cudaStream_t st);
 int quant_t_rows(int mode, const void* src, const int32_t* src_of, const float* row_gate, const int32_t* off,
                  const int32_t* poff, int E, long long rows, int C, uint8_t* dst, uint8_t* sf, long long ldd,
                  cudaStream_t st);

@@ -1,9 +1,10 @@
 // mxfp8.cu -- MXFP8 expert GEMMs (E4M3 operands, UE8M0 1x32 block scales,
-// fp32 accumulate) and the MXFP8 layer forward:
-//   router -> permute (rows quantised to MXFP8 on the way) -> gate/up GEMM
-//   whose epilogue folds the gate, applies the SwiGLU and re-quantises the
-//   activation to MXFP8 along F -> down GEMM (bf16 out) -> shared expert
-//   (x quantised once, the same two GEMMs as one group) -> unpermute-sum.
+// fp32 accumulate) and the block-scaled layer forward (MXFP8, or NVFP4 with the
+// GEMM hosts of nvfp4.cu):
+//   router -> permute (rows quantised on the way) -> gate/up GEMM whose
+//   epilogue folds the gate, applies the SwiGLU and re-quantises the activation
+//   along F -> down GEMM (bf16 out) -> shared expert (x quantised once, the same
+//   two GEMMs as one group) -> unpermute-sum.
 #include "common.cuh"
 #include "gemm_mx.cuh"
 #include "layout.h"
@@ -105,6 +106,15 @@ struct MxWs {
   __nv_bfloat16* so;
 };
 
+// Byte sizes of a block-scaled [n, K] operand: codes (1 byte per MXFP8 element, 2 NVFP4 elements per byte)
+// and scales (one per 32 or 16 elements).
+static size_t q_bytes(const moe_config* c, size_t n, size_t K) {
+  return c->expert_dtype == MOE_DT_NVFP4 ? n * K / 2 : n * K;
+}
+static size_t sf_bytes(const moe_config* c, size_t n, size_t K) {
+  return c->expert_dtype == MOE_DT_NVFP4 ? n * K / 16 : n * K / 32;
+}
+
 static size_t carve_mx(void* ws, const moe_config* c, MxWs* w) {
   Carve cv(ws);
   const size_t T = c->T, E = c->E, k = c->k, H = c->H, F = c->F, rows = T * k;
@@ -119,17 +129,17 @@ static size_t carve_mx(void* ws, const moe_config* c, MxWs* w) {
   w->row_of = cv.take<int32_t>(T * k);
   w->src_of = cv.take<int32_t>(rows);
   w->row_gate = cv.take<float>(rows);
-  w->xp = cv.take<uint8_t>(rows * H);
-  w->xp_sf = cv.take<uint8_t>(rows * H / 32);
-  w->ap = cv.take<uint8_t>(rows * F);
-  w->ap_sf = cv.take<uint8_t>(rows * F / 32);
+  w->xp = cv.take<uint8_t>(q_bytes(c, rows, H));
+  w->xp_sf = cv.take<uint8_t>(sf_bytes(c, rows, H));
+  w->ap = cv.take<uint8_t>(q_bytes(c, rows, F));
+  w->ap_sf = cv.take<uint8_t>(sf_bytes(c, rows, F));
   w->o = cv.take<__nv_bfloat16>(rows * H);
   w->off2 = cv.take<int32_t>(2);
   if (c->n_shared) {
-    w->xq = cv.take<uint8_t>(T * H);
-    w->xq_sf = cv.take<uint8_t>(T * H / 32);
-    w->as_ = cv.take<uint8_t>(T * F);
-    w->as_sf = cv.take<uint8_t>(T * F / 32);
+    w->xq = cv.take<uint8_t>(q_bytes(c, T, H));
+    w->xq_sf = cv.take<uint8_t>(sf_bytes(c, T, H));
+    w->as_ = cv.take<uint8_t>(q_bytes(c, T, F));
+    w->as_sf = cv.take<uint8_t>(sf_bytes(c, T, F));
     w->so = cv.take<__nv_bfloat16>(T * H);
   } else {
     w->xq = w->xq_sf = w->as_ = w->as_sf = nullptr;
@@ -165,7 +175,9 @@ int layer_fwd_mxfp8(const moe_config* c, const void* x, const void* W_r, const f
                     const uint8_t* Ws_g_sf, const uint8_t* Ws_u_sf, const uint8_t* Ws_d_sf, void* y, float* aux,
                     int32_t* idx, float* gates, int32_t* counts, int32_t* offsets, void* saved, void* ws,
                     size_t ws_bytes, cudaStream_t st) {
-  if (c->H % 256 != 0 || c->F % 128 != 0) return MOE_ERR_UNSUPPORTED;
+  const bool nv = c->expert_dtype == MOE_DT_NVFP4;
+  if (c->H % 256 != 0 || c->F % (nv ? 256 : 128) != 0) return MOE_ERR_UNSUPPORTED;
+  if (nv && c->save_for_bwd) return MOE_ERR_UNSUPPORTED;  // there is no NVFP4 backward
   if (!W_g_sf || !W_u_sf || !W_d_sf) return MOE_ERR_INVALID_ARG;
   if (c->n_shared && (!Ws_g_sf || !Ws_u_sf || !Ws_d_sf)) return MOE_ERR_INVALID_ARG;
   const uint8_t* sfs[] = {W_g_sf, W_u_sf, W_d_sf, Ws_g_sf, Ws_u_sf, Ws_d_sf};
@@ -194,15 +206,32 @@ int layer_fwd_mxfp8(const moe_config* c, const void* x, const void* W_r, const f
                   w.router_ws, router_ws(c), st));
   RCM(permute(c, x, w.idx, w.gates, nullptr, w.offsets, w.row_of, w.src_of, w.row_gate, w.xp, w.xp_sf,
               w.permute_ws, permute_ws(c), st));
-  RCM(gemm_gateup_mx(rows, E, H, F, w.xp, w.xp_sf, W_g, W_g_sf, W_u, W_u_sf, w.offsets, w.row_gate, w.ap, w.ap_sf,
-                     save_gu, st));
-  RCM(gemm_down_mx(rows, E, H, F, w.ap, w.ap_sf, W_d, W_d_sf, w.offsets, w.o, st));
-  if (c->n_shared) {
-    RCM(fill_offsets2(w.off2, T, st));
-    RCM(quantize_mxfp8(x, T, H, w.xq, w.xq_sf, st));
-    RCM(gemm_gateup_mx(T, 1, H, F, w.xq, w.xq_sf, Ws_g, Ws_g_sf, Ws_u, Ws_u_sf, w.off2, nullptr, w.as_, w.as_sf,
-                       nullptr, st));
-    RCM(gemm_down_mx(T, 1, H, F, w.as_, w.as_sf, Ws_d, Ws_d_sf, w.off2, w.so, st));
+  if (nv) {
+    // NVFP4 weights: each scale buffer ends with the per-expert encode scales G (fp32)
+    const size_t ef = (size_t)E * F * (H / 16);
+    const auto gsf = [](const uint8_t* sf, size_t off) { return reinterpret_cast<const float*>(sf + off); };
+    RCM(gemm_gateup_nv(rows, E, H, F, w.xp, w.xp_sf, W_g, W_g_sf, gsf(W_g_sf, ef), W_u, W_u_sf, gsf(W_u_sf, ef),
+                       w.offsets, w.row_gate, w.ap, w.ap_sf, st));
+    RCM(gemm_down_nv(rows, E, H, F, w.ap, w.ap_sf, W_d, W_d_sf, gsf(W_d_sf, ef), w.offsets, w.o, st));
+    if (c->n_shared) {
+      const size_t sfh = (size_t)F * (H / 16);
+      RCM(fill_offsets2(w.off2, T, st));
+      RCM(quantize_nvfp4_act(x, T, H, w.xq, w.xq_sf, st));
+      RCM(gemm_gateup_nv(T, 1, H, F, w.xq, w.xq_sf, Ws_g, Ws_g_sf, gsf(Ws_g_sf, sfh), Ws_u, Ws_u_sf,
+                         gsf(Ws_u_sf, sfh), w.off2, nullptr, w.as_, w.as_sf, st));
+      RCM(gemm_down_nv(T, 1, H, F, w.as_, w.as_sf, Ws_d, Ws_d_sf, gsf(Ws_d_sf, sfh), w.off2, w.so, st));
+    }
+  } else {
+    RCM(gemm_gateup_mx(rows, E, H, F, w.xp, w.xp_sf, W_g, W_g_sf, W_u, W_u_sf, w.offsets, w.row_gate, w.ap,
+                       w.ap_sf, save_gu, st));
+    RCM(gemm_down_mx(rows, E, H, F, w.ap, w.ap_sf, W_d, W_d_sf, w.offsets, w.o, st));
+    if (c->n_shared) {
+      RCM(fill_offsets2(w.off2, T, st));
+      RCM(quantize_mxfp8(x, T, H, w.xq, w.xq_sf, st));
+      RCM(gemm_gateup_mx(T, 1, H, F, w.xq, w.xq_sf, Ws_g, Ws_g_sf, Ws_u, Ws_u_sf, w.off2, nullptr, w.as_, w.as_sf,
+                         nullptr, st));
+      RCM(gemm_down_mx(T, 1, H, F, w.as_, w.as_sf, Ws_d, Ws_d_sf, w.off2, w.so, st));
+    }
   }
   RCM(unpermute(c, w.o, w.row_of, w.so, y, st));
   RCM(copy_out(idx, w.idx, (size_t)T * k * 4, st));

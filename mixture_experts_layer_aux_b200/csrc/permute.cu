@@ -16,7 +16,8 @@
 //   scatter  one warp per token: row = base[block, e] + rank; writes row_of,
 //            src_of, row_gate; copies the token's row once from HBM and writes
 //            it to its k destination rows with 16-byte vector stores
-//            (quantising each 1x32 block to MXFP8 on the way when asked).
+//            (quantising each 1x32 block to MXFP8, or each 1x16 block to NVFP4,
+//            on the way when asked).
 //   unpermute one warp per token: fp32 sum of its k rows in slot order, 16-byte
 //            loads, one bf16 rounding.
 #include <cuda_fp8.h>
@@ -26,6 +27,7 @@
 
 #include "common.cuh"
 #include "layout.h"
+#include "nvfp4.cuh"
 
 namespace perm {
 
@@ -165,7 +167,10 @@ __device__ __forceinline__ uint2 quant8(const float (&f)[8], float inv) {
 
 // MODE 0: rows computed here from (idx, lrank, base) -- the permute itself.
 // MODE 1: rows read from row_of -- a plain scatter of another [T,H] tensor.
-template <int MODE, bool MX>
+// QF: what is written -- bf16 rows (QF_BF16), MXFP8 rows (QF_MX: e4m3 [rows, H] + ue8m0 per 32) or NVFP4 rows
+// (QF_NV: packed e2m1 [rows, H/2] + e4m3 per 16, tensor scale 1).
+enum { QF_BF16 = 0, QF_MX = 1, QF_NV = 2 };
+template <int MODE, int QF>
 __global__ void __launch_bounds__(SC_WARPS * 32) scatter_kernel(
     const __nv_bfloat16* __restrict__ x, int T, int H, int E, int k, const int32_t* __restrict__ idx,
     const int32_t* __restrict__ lrank, const int* __restrict__ base, const int32_t* __restrict__ offsets,
@@ -205,12 +210,30 @@ __global__ void __launch_bounds__(SC_WARPS * 32) scatter_kernel(
     const int i = i0 + lane;
     const bool v = i < nchunk;
     const uint4 d = v ? src[i] : make_uint4(0, 0, 0, 0);
-    if constexpr (!MX) {
+    if constexpr (QF == QF_BF16) {
       if (v) {
 #pragma unroll
         for (int j = 0; j < 16; ++j)
           if (j < k && rows[j] >= 0)
             reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(xp) + (long long)rows[j] * H)[i] = d;
+      }
+    } else if constexpr (QF == QF_NV) {
+      // a 16-block is the 8-element chunks of lanes 2m and 2m+1 (H % 16 == 0, so pairs share validity)
+      float f[8];
+      unpack_bf16x8(d, f);
+      float am = 0.f;
+#pragma unroll
+      for (int q = 0; q < 8; ++q) am = fmaxf(am, fabsf(f[q]));
+      am = fmaxf(am, __shfl_xor_sync(0xffffffffu, am, 1));
+      const uint8_t sb = nvq::scale_byte(am, 1.0f);
+      const uint32_t w = nvq::pack8(f, nvq::elem_mult(sb, 1.0f));
+      if (v) {
+#pragma unroll
+        for (int j = 0; j < 16; ++j)
+          if (j < k && rows[j] >= 0) {
+            reinterpret_cast<uint32_t*>(static_cast<uint8_t*>(xp) + (long long)rows[j] * (H / 2))[i] = w;
+            if ((i & 1) == 0) xp_sf[(long long)rows[j] * (H / 16) + (i >> 1)] = sb;
+          }
       }
     } else {
       float f[8];
@@ -347,8 +370,8 @@ int permute(const moe_config* c, const void* x, const int32_t* idx, const float*
   if (!idx || !offsets || !row_of || !src_of) return MOE_ERR_INVALID_ARG;
   if (row_gate && !gates) return MOE_ERR_INVALID_ARG;
   if (xp && !x) return MOE_ERR_INVALID_ARG;
-  const bool mx = c->expert_dtype == MOE_DT_MXFP8;
-  if (xp && mx && !xp_sf) return MOE_ERR_INVALID_ARG;
+  const bool mx = c->expert_dtype == MOE_DT_MXFP8, nv = c->expert_dtype == MOE_DT_NVFP4;
+  if (xp && (mx || nv) && !xp_sf) return MOE_ERR_INVALID_ARG;
   if ((x && !al16(x)) || (xp && !al16(xp))) return MOE_ERR_ALIGNMENT;
   if (!ws || ws_bytes < permute_ws(c)) return MOE_ERR_WORKSPACE;
   const int nblk = (c->T + perm::RANK_TOK - 1) / perm::RANK_TOK;
@@ -370,11 +393,15 @@ int permute(const moe_config* c, const void* x, const int32_t* idx, const float*
   MOE_CHECK_LAUNCH();
   const int sgrid = (c->T + perm::SC_WARPS - 1) / perm::SC_WARPS;
   if (mx)
-    perm::scatter_kernel<0, true><<<sgrid, perm::SC_WARPS * 32, 0, st>>>(
+    perm::scatter_kernel<0, perm::QF_MX><<<sgrid, perm::SC_WARPS * 32, 0, st>>>(
+        static_cast<const __nv_bfloat16*>(x), c->T, c->H, c->E, c->k, idx, lrank, base, offsets, gates, row_of,
+        src_of, row_gate, xp, xp_sf);
+  else if (nv)
+    perm::scatter_kernel<0, perm::QF_NV><<<sgrid, perm::SC_WARPS * 32, 0, st>>>(
         static_cast<const __nv_bfloat16*>(x), c->T, c->H, c->E, c->k, idx, lrank, base, offsets, gates, row_of,
         src_of, row_gate, xp, xp_sf);
   else
-    perm::scatter_kernel<0, false><<<sgrid, perm::SC_WARPS * 32, 0, st>>>(
+    perm::scatter_kernel<0, perm::QF_BF16><<<sgrid, perm::SC_WARPS * 32, 0, st>>>(
         static_cast<const __nv_bfloat16*>(x), c->T, c->H, c->E, c->k, idx, lrank, base, offsets, gates, row_of,
         src_of, row_gate, xp, nullptr);
   MOE_CHECK_LAUNCH();
@@ -383,7 +410,7 @@ int permute(const moe_config* c, const void* x, const int32_t* idx, const float*
 
 int scatter_rows(const moe_config* c, const void* x, const int32_t* row_of, void* xp, cudaStream_t st) {
   const int sgrid = (c->T + perm::SC_WARPS - 1) / perm::SC_WARPS;
-  perm::scatter_kernel<1, false><<<sgrid, perm::SC_WARPS * 32, 0, st>>>(
+  perm::scatter_kernel<1, perm::QF_BF16><<<sgrid, perm::SC_WARPS * 32, 0, st>>>(
       static_cast<const __nv_bfloat16*>(x), c->T, c->H, c->E, c->k, nullptr, nullptr, nullptr, nullptr, nullptr,
       const_cast<int32_t*>(row_of), nullptr, nullptr, xp, nullptr);
   MOE_CHECK_LAUNCH();
@@ -394,7 +421,7 @@ int scatter_rows(const moe_config* c, const void* x, const int32_t* row_of, void
 int scatter_rows_mx(const moe_config* c, const void* x, const int32_t* row_of, uint8_t* xq, uint8_t* xq_sf,
                     cudaStream_t st) {
   const int sgrid = (c->T + perm::SC_WARPS - 1) / perm::SC_WARPS;
-  perm::scatter_kernel<1, true><<<sgrid, perm::SC_WARPS * 32, 0, st>>>(
+  perm::scatter_kernel<1, perm::QF_MX><<<sgrid, perm::SC_WARPS * 32, 0, st>>>(
       static_cast<const __nv_bfloat16*>(x), c->T, c->H, c->E, c->k, nullptr, nullptr, nullptr, nullptr, nullptr,
       const_cast<int32_t*>(row_of), nullptr, nullptr, xq, xq_sf);
   MOE_CHECK_LAUNCH();

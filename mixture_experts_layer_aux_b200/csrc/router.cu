@@ -296,7 +296,8 @@ int check_cfg(const moe_config* c) {
   if (c->k > c->E || c->k > 16 || c->E > 512) return MOE_ERR_UNSUPPORTED;
   if (c->H % 128 != 0 || c->F % 128 != 0) return MOE_ERR_UNSUPPORTED;
   if (c->score != MOE_SCORE_SOFTMAX && c->score != MOE_SCORE_SIGMOID) return MOE_ERR_INVALID_ARG;
-  if (c->expert_dtype != MOE_DT_BF16 && c->expert_dtype != MOE_DT_MXFP8) return MOE_ERR_INVALID_ARG;
+  if (c->expert_dtype != MOE_DT_BF16 && c->expert_dtype != MOE_DT_MXFP8 && c->expert_dtype != MOE_DT_NVFP4)
+    return MOE_ERR_INVALID_ARG;
   if (c->n_shared != 0 && c->n_shared != 1) return MOE_ERR_UNSUPPORTED;
   if (c->compute_aux && c->score != MOE_SCORE_SOFTMAX) return MOE_ERR_UNSUPPORTED;
   if ((long long)c->T * c->k >= (1LL << 31) / 2) return MOE_ERR_UNSUPPORTED;

@@ -12,7 +12,8 @@ for):
   mixtral  T=4096 H=4096 E=8   k=2 F=14336 softmax top-2 renormalised
   qwen3    T=8192 H=4096 E=128 k=8 F=1536  softmax top-8 renormalised + aux loss
   dsv3     T=8192 H=7168 E=256 k=8 F=2048  + 1 shared expert, sigmoid scores,
-           selected-normalised x2.5, MXFP8 expert operands
+           selected-normalised x2.5, MXFP8 expert operands (dsv3-nvfp4: the
+           same with NVFP4 expert operands)
   skewed   qwen3 shape with a per-expert logit bias (log-Zipf s=1.2, and the
            last four experts pushed out), forward + backward with dY~N(0,1)
 
@@ -42,7 +43,7 @@ class Workload:
     score: str = "softmax"     # "softmax" | "sigmoid"
     norm_topk: bool = True
     route_scale: float = 1.0
-    dtype: str = "bf16"        # expert operand dtype: "bf16" | "mxfp8"
+    dtype: str = "bf16"        # expert operand dtype: "bf16" | "mxfp8" | "nvfp4"
     aux: bool = True           # compute the load-balancing aux statistic
     skew: bool = False         # add the skew logit bias
     bwd: bool = False          # the workload includes the backward pass
@@ -63,8 +64,8 @@ class Workload:
         return 6.0 * self.H * self.F * (self.T * self.k + self.T * self.S)
 
     def expert_weight_bytes(self) -> float:
-        """Bytes of the routed and shared expert weights (bf16, or fp8 + 1/32 scale bytes)."""
-        per = 1.0 + 1.0 / 32 if self.dtype == "mxfp8" else 2.0
+        """Bytes of the routed and shared expert weights (bf16; fp8 + 1/32 scale bytes; fp4 + 1/16)."""
+        per = {"mxfp8": 1.0 + 1.0 / 32, "nvfp4": 0.5 + 1.0 / 16}.get(self.dtype, 2.0)
         return 3.0 * self.H * self.F * (self.E + self.S) * per
 
     def router_flops(self) -> float:
@@ -83,6 +84,9 @@ WORKLOADS = {
     # and the capacity factor (1.25) on the skewed fwd+bwd step
     "dsv3-grouped": Workload("dsv3-grouped", T=8192, H=7168, E=256, k=8, F=2048, S=1, score="sigmoid",
                              route_scale=2.5, dtype="mxfp8", aux=False, n_group=8, topk_group=4, sel_bias=True),
+    # the DeepSeek-V3 forward with NVFP4 expert operands (E2M1 + E4M3 per 16, per-expert encode scales)
+    "dsv3-nvfp4": Workload("dsv3-nvfp4", T=8192, H=7168, E=256, k=8, F=2048, S=1, score="sigmoid",
+                           route_scale=2.5, dtype="nvfp4", aux=False),
     # the MXFP8 backward on the DeepSeek-V3 routed experts (the backward has no shared expert)
     "dsv3-train": Workload("dsv3-train", T=8192, H=7168, E=256, k=8, F=2048, score="sigmoid", route_scale=2.5,
                            dtype="mxfp8", aux=False, bwd=True),

@@ -77,6 +77,8 @@ def lib():
             _lib.oc_nvfp4_scale_byte.argtypes = [ctypes.c_float, ctypes.c_float]
             _lib.oc_nvfp4_quantize_bf16.argtypes = [ctypes.c_long, ctypes.c_int, ctypes.c_void_p, ctypes.c_float,
                                                     ctypes.c_void_p, ctypes.c_void_p]
+            _lib.oc_nvfp4_quantize_f32.argtypes = [ctypes.c_long, ctypes.c_int, ctypes.c_void_p, ctypes.c_float,
+                                                   ctypes.c_void_p, ctypes.c_void_p]
             _lib.oc_bf16_amax.restype = ctypes.c_float
             _lib.oc_bf16_amax.argtypes = [ctypes.c_long, ctypes.c_void_p]
         return _lib
@@ -212,16 +214,20 @@ def nvfp4_scale_byte(amax: float, G: float = 1.0) -> int:
 
 
 def nvfp4_quantize(src: torch.Tensor, per_matrix: bool = False):
-    """src [..., K] bf16 (K % 16 == 0) -> (packed uint8 [..., K/2], scales uint8 [..., K/16], G fp32).
+    """src [..., K] bf16 or fp32 (K % 16 == 0) -> (packed uint8 [..., K/2], scales uint8 [..., K/16], G fp32).
 
-    per_matrix: each [R, K] matrix of src [..., R, K] gets G = 6*448/amax(matrix)
+    per_matrix (bf16 only): each [R, K] matrix of src [..., R, K] gets G = 6*448/amax(matrix)
     (G is then [...]); otherwise G = 1 (a 0-d tensor)."""
-    assert src.dtype == torch.bfloat16
     K = src.shape[-1]
     assert K % 16 == 0
     src = src.contiguous()
     packed = torch.empty(tuple(src.shape[:-1]) + (K // 2,), dtype=torch.uint8)
     scales = torch.empty(tuple(src.shape[:-1]) + (K // 16,), dtype=torch.uint8)
+    if src.dtype == torch.float32:
+        assert not per_matrix
+        lib().oc_nvfp4_quantize_f32(src.numel() // K, K, _p(src), 1.0, _p(packed), _p(scales))
+        return packed, scales, torch.tensor(1.0, dtype=torch.float32)
+    assert src.dtype == torch.bfloat16
     if not per_matrix:
         lib().oc_nvfp4_quantize_bf16(src.numel() // K, K, _p(src), 1.0, _p(packed), _p(scales))
         return packed, scales, torch.tensor(1.0, dtype=torch.float32)

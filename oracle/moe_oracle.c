@@ -267,6 +267,20 @@ void oc_nvfp4_quantize_bf16(long rows, int K, const uint16_t* src, float G, uint
     }
 }
 
+/* Same, from fp32 values. */
+void oc_nvfp4_quantize_f32(long rows, int K, const float* src, float G, uint8_t* packed, uint8_t* scales) {
+    long r;
+#pragma omp parallel for schedule(static)
+    for (r = 0; r < rows; ++r) {
+        uint8_t c[16];
+        for (int b = 0; b < K / 16; ++b) {
+            scales[r * (long)(K / 16) + b] = nv_block(src + r * (long)K + b * 16, G, c);
+            for (int i = 0; i < 8; ++i)
+                packed[r * (long)(K / 2) + b * 8 + i] = (uint8_t)(c[2 * i] | (c[2 * i + 1] << 4));
+        }
+    }
+}
+
 /* Largest magnitude of n bf16 values (the input of oc_nvfp4_global_scale). */
 float oc_bf16_amax(long n, const uint16_t* src) {
     double m = 0.0;

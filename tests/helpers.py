@@ -4,6 +4,9 @@ import torch
 # Floating-point bars: max |err| <= TOL * rms(ref) over the compared tensor.
 TOL_BF16 = 2e-2
 TOL_MXFP8 = 6e-2
+# NVFP4 against an oracle that quantises at the same points: the block-scaled bar of MXFP8 (the two sides
+# differ only by fp32-vs-fp64 accumulation and the rare E2M1 / E4M3 rounding decisions it moves)
+TOL_NVFP4 = 6e-2
 
 
 def rms(t: torch.Tensor) -> float:
@@ -89,4 +92,31 @@ def check_mx(got_dq: torch.Tensor, ref_dq: torch.Tensor, scale: torch.Tensor, to
         step = e4m3_ulp(torch.maximum(g.abs(), r.abs()) / s) * s
         assert bool((d[bad] <= step[bad] * (1 + 1e-9)).all()), f"MXFP8 values more than one step apart"
         assert flips <= max(1, max_flip_frac * g.numel()), f"{flips} MXFP8 step differences beyond {tol}*rms"
+    return float(d.max()) / den, flips
+
+
+def e2m1_step(u: torch.Tensor) -> torch.Tensor:
+    """Spacing of the E2M1 grid around |u| (u already divided by its block scale)."""
+    a = u.abs()
+    return torch.where(a < 2, 0.5, torch.where(a < 4, 1.0, 2.0)).double()
+
+
+def check_nv(got: torch.Tensor, ref: torch.Tensor, s_got: torch.Tensor, s_ref: torch.Tensor, tol: float = TOL_NVFP4,
+             max_flip_frac: float = 1e-2):
+    """Compare dequantised NVFP4 kernel values with the oracle's NVFP4 values of the same tensor
+    (identical quantisation; s_* = each element's decoded block scale). Elements beyond tol*rms(ref)
+    come from a rounding decision taken differently from slightly different fp32 inputs: they must be
+    within one E2M1 step at the larger scale plus 6x the difference of the two block scales (a block
+    scale that itself rounded the other way), and be at most max_flip_frac of all."""
+    g, r = got.double().cpu(), ref.double().cpu()
+    sg, sr = s_got.double().cpu(), s_ref.double().cpu()
+    den = max(float(r.pow(2).mean().sqrt()), 1e-30)
+    d = (g - r).abs()
+    bad = d > tol * den
+    flips = int(bad.sum())
+    if flips:
+        sm = torch.maximum(sg, sr)
+        step = e2m1_step(torch.maximum(g.abs(), r.abs()) / sm.clamp_min(1e-30)) * sm + 6 * (sg - sr).abs()
+        assert bool((d[bad] <= step[bad] * (1 + 1e-9)).all()), "NVFP4 values more than one step apart"
+        assert flips <= max(1, max_flip_frac * g.numel()), f"{flips} NVFP4 step differences beyond {tol}*rms"
     return float(d.max()) / den, flips

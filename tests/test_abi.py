@@ -153,3 +153,36 @@ def test_gemm_and_layer_argument_errors(lib, B):
     cbm = cfg(B, expert_dtype=1)
     assert bw(ctypes.byref(cbm), FAKE, ctypes.c_float(0.0), FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE,
               FAKE, None, FAKE, bws, None) == UNSUPPORTED
+
+
+def test_nvfp4_argument_errors(lib, B):
+    # scale-buffer size: batch*R*C/16 scale bytes + batch fp32 encode scales
+    assert lib.moe_nvfp4_sf_bytes(2, 3, 32) == 2 * 3 * 2 + 8
+    assert lib.moe_nvfp4_sf_bytes(1, 4, 24) == 0
+    q = lib.moe_quantize_nvfp4
+    assert q(FAKE, 1, 4, 24, FAKE, FAKE, None) == UNSUPPORTED       # C % 16 != 0
+    assert q(FAKE, 1, 4, 8, FAKE, FAKE, None) == INVALID            # C < 16
+    assert q(None, 1, 4, 32, FAKE, FAKE, None) == INVALID
+    assert q(FAKE, 1, 4, 32, FAKE, FAKE + 2, None) == ALIGN         # sf not 4-byte aligned
+    assert q(FAKE, 1, 1, 16, FAKE, FAKE, None) == ALIGN             # G slots would not be 4-byte aligned
+    qa = lib.moe_quantize_nvfp4_act
+    assert qa(FAKE, 4, 24, FAKE, FAKE, None) == UNSUPPORTED
+    assert qa(FAKE + 8, 4, 32, FAKE, FAKE, None) == ALIGN
+    c = cfg(B, H=512, F=384, expert_dtype=B.MOE_DT_NVFP4)           # NVFP4 needs F % 256 == 0
+    lw = lib.moe_layer_workspace_size(ctypes.byref(c))
+    L = lib.moe_layer_fwd
+    args = [FAKE, FAKE, None, None, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, None, None, None, None, None, None, FAKE, None,
+            None, None, None, None, None]
+    assert L(ctypes.byref(c), *args, FAKE, lw, None) == UNSUPPORTED
+    cs = cfg(B, H=512, F=512, expert_dtype=B.MOE_DT_NVFP4, save_for_bwd=1)  # no NVFP4 backward
+    assert lib.moe_layer_saved_size(ctypes.byref(cs)) == 0
+    args_s = list(args)
+    args_s[22] = FAKE  # saved
+    assert L(ctypes.byref(cs), *args_s, FAKE, lib.moe_layer_workspace_size(ctypes.byref(cs)), None) == UNSUPPORTED
+    g = lib.moe_grouped_gemm_fwd
+    ws = lib.moe_grouped_gemm_workspace_size(ctypes.byref(c), 0)
+    assert g(ctypes.byref(c), 0, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, None, FAKE, ws,
+             None) == UNSUPPORTED
+    c2 = cfg(B, H=512, F=512, expert_dtype=B.MOE_DT_NVFP4)
+    assert g(ctypes.byref(c2), 0, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, ws,
+             None) == INVALID  # save_gateup is not supported

@@ -849,3 +849,11 @@ def test_nvfp4_forward_stays_near_exact(oracle):
     rms = y0.pow(2).mean().sqrt()
     rel = (y - y0).pow(2).mean().sqrt() / rms
     assert 0.01 < rel < 0.3, float(rel)
+
+
+def test_nvfp4_bf16_and_fp32_entry_points_agree(oracle):
+    g = torch.Generator().manual_seed(7)
+    v = (torch.randn(16, 128, generator=g) * 0.5).bfloat16()
+    a = oracle.nvfp4_quantize(v)
+    b = oracle.nvfp4_quantize(v.float())
+    assert torch.equal(a[0], b[0]) and torch.equal(a[1], b[1])
