@@ -264,16 +264,20 @@ int moe_quantize_mxfp8(const void* src, int64_t rows, int32_t K, uint8_t* dst, u
  *   scale byte s = e4m3_rn_sat((amax / 6) * G)   (0 for an all-zero block),
  *   element     = e2m1_rn_sat(v * (G / s))       (0 when s == 0),
  *   value       = element * s / G.
- * moe_quantize_nvfp4: weights. src [batch, R, C] bf16 (C % 16 == 0), each
- *   [R, C] matrix with its own G = 6*448 / amax(matrix) (1 if all zero), so its
- *   largest block scale is 448. dst packed [batch, R, C/2]; sf is ONE buffer of
- *   moe_nvfp4_sf_bytes(batch, R, C) bytes: the scales [batch, R, C/16], then
- *   the batch's G values as fp32 [batch] (batch*R*C/16 must be a multiple of
- *   4; sf 4-byte aligned). Once per weight tensor: W_g, W_u [E,F,H] (batch E,
- *   R = F, C = H), W_d [E,H,F]; the shared expert's [F,H] / [H,F] with batch 1.
- *   Enqueues a 4-byte-per-matrix clear and three kernels.
+ * moe_quantize_nvfp4: weights. src [batch, R, C] bf16 (R % 128 == 0,
+ *   C % 64 == 0), each [R, C] matrix with its own G = 6*448 / amax(matrix) (1
+ *   if all zero), so its largest block scale is 448. dst packed
+ *   [batch, R, C/2]; sf is ONE 16-byte aligned buffer of
+ *   moe_nvfp4_sf_bytes(batch, R, C) bytes: the batch*R*C/16 scale bytes TILED
+ *   in the order of the GEMM's tensor-memory scale copies -- with r the row
+ *   in [0, batch*R) and c the 16-block of the row, byte
+ *     ((r/128) * (C/64) + c/4) * 512 + 16 (r % 32) + 4 ((r % 128) / 32) + c % 4
+ *   -- then the batch's G values as fp32 [batch]. Once per weight tensor: W_g,
+ *   W_u [E,F,H] (batch E, R = F, C = H), W_d [E,H,F]; the shared expert's
+ *   [F,H] / [H,F] with batch 1. Enqueues a 4-byte-per-matrix clear and three
+ *   kernels.
  * moe_quantize_nvfp4_act: activations, G = 1: src [rows, K] bf16 -> dst packed
- *   [rows, K/2], sf [rows, K/16] (no G values).
+ *   [rows, K/2], sf row-major [rows, K/16] (no G values).
  * ------------------------------------------------------------------------ */
 size_t moe_nvfp4_sf_bytes(int32_t batch, int64_t R, int32_t C);
 int moe_quantize_nvfp4(const void* src, int32_t batch, int64_t R, int32_t C, uint8_t* dst, uint8_t* sf,

@@ -31,12 +31,16 @@
 // NVFP4 (template flag NV; formats in nvfp4.cuh): the same kernel with packed
 // E2M1 operands -- a 128-byte stage row is 256 elements -- and one E4M3 scale
 // per 16 elements: tcgen05.mma kind::mxf4nvf4 with scale_vec::4X, M128 N256
-// K64, four per k-block. A row's 16 scale bytes of one k-block hold the four
-// MMAs' scale words, so one k-block is one scale batch of the same 6 KB (the
-// loader is unchanged: its four "sub-blocks" are the four MMAs instead of four
-// k-blocks), and each MMA reads its own A/B chunks (12 TMEM columns) from a
-// 48-column slot. The weights' per-expert encode scales G are divided out in
-// the epilogue; activations have G = 1.
+// K64, four per k-block. One k-block is one 6 KB scale batch holding the four
+// MMAs' chunks of A (2 KB), B0 and B1 (2 KB each). The weights' scales are
+// stored tiled in chunk order (moe_quantize_nvfp4), so the producer bulk-copies
+// each k-block's two 2 KB runs; the loader warp rearranges only the 128
+// activation rows (one 16-byte load per row). Each MMA reads its own A/B
+// chunks (12 TMEM columns) from a 48-column slot. On B200 the twelve
+// 32x128b.warpx4 copies per k-block take about as long as the four MMAs
+// (a tensor-pipe probe: ~700 vs ~650 clocks), which bounds this design near
+// 55% of the FP4 peak. The weights' per-expert encode scales G are divided out
+// in the epilogue; activations have G = 1.
 #pragma once
 
 #include <cuda_fp8.h>
@@ -257,7 +261,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) gemm_mx_kernel(const __grid_co
       mbar_init(&empty[i], 1);
     }
     for (int i = 0; i < kSfBufs; ++i) {
-      mbar_init(&sfull[i], 1);
+      mbar_init(&sfull[i], NV ? 2 : 1);  // NVFP4: the loader's A chunks and the producer's B chunks
       mbar_init(&sempty[i], 1);
     }
     mbar_init(tfull, 1);
@@ -309,6 +313,28 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) gemm_mx_kernel(const __grid_co
         const Tile ti = get_tile<GK>(p, t, s_off, s_tstart, N_STEP);
         const int brow = (GK ? 0 : ti.g * p.b_group_rows) + ti.n0;
         for (int kb = 0; kb < ti.nkb; ++kb) {
+          if constexpr (NV) {
+            // the weights' tiled scale chunks of this k-block: four MMAs' chunks of one 128-row n-block are
+            // 2 KB in a row; B0 (gate, or the first 128 rows) and B1 (up, or the next 128 rows)
+            if (!mbar_wait(&sempty[sb], sphase ^ 1, abort_flag, p.status, DEV_WAIT_TIMEOUT_PRODUCER)) {
+              aborted = true;
+              break;
+            }
+            mbar_arrive_expect_tx(&sfull[sb], 4096u);
+            s_issued_mask |= 1u << sb;
+            s_issued_par = (s_issued_par & ~(1u << sb)) | (sphase << sb);
+            uint8_t* sf = sf_area + sb * SF_BATCH_BYTES;
+            const long long kq = p.K / 32;  // K64 groups per row (p.K bytes = 2 p.K elements)
+            const long long nb = brow / 128;
+            const long long c0 = (nb * kq + 4LL * kb) * 512;
+            bulk_load(sf + 2048, p.sfb0 + c0, 2048, &sfull[sb]);
+            if (SPLIT_N) bulk_load(sf + 4096, p.sfb1 + c0, 2048, &sfull[sb]);
+            else bulk_load(sf + 4096, p.sfb0 + c0 + kq * 512, 2048, &sfull[sb]);
+            if (++sb == kSfBufs) {
+              sb = 0;
+              sphase ^= 1;
+            }
+          }
           if (GK && kb % SB == 0) {
             // the batch's tiled scale chunks: SFA of the m-block, SFB of the (one or two) n-blocks
             if (!mbar_wait(&sempty[sb], sphase ^ 1, abort_flag, p.status, DEV_WAIT_TIMEOUT_PRODUCER)) {
@@ -381,8 +407,61 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) gemm_mx_kernel(const __grid_co
   } else if (warp == 2) {
     // ======================= scale loader: natural [rows, K/32] bytes -> UTCCP chunk order, SB k-blocks at a time
     // (grouped along K the producer bulk-copies tiled scales instead, and this warp has nothing to do)
-    if constexpr (!GK) {
-    const int kw = NV ? p.K / 8 : p.K / 32;  // scale bytes per row (a multiple of 4; p.K is A's row bytes)
+    if constexpr (NV) {
+      // NVFP4: the 128 activation rows only (the producer bulk-copies the weights' tiled chunks). Per k-block
+      // a row's 16 scale bytes are the four MMAs' words: word q goes to chunk q of the batch's A region.
+      const int kw = p.K / 8;  // A's scale bytes per row
+      const bool v16 = (kw % 16) == 0 && (reinterpret_cast<uintptr_t>(p.sfa) & 15u) == 0;
+      int sb = 0;
+      uint32_t sphase = 0;
+      for (int t = blockIdx.x; t < total && !aborted; t += gridDim.x) {
+        const Tile ti = get_tile<GK>(p, t, s_off, s_tstart, N_STEP);
+        for (int kb = 0; kb < ti.nkb; ++kb) {
+          if (!__all_sync(0xffffffffu,
+                          mbar_wait(&sempty[sb], sphase ^ 1, abort_flag, p.status, DEV_WAIT_TIMEOUT_PRODUCER))) {
+            aborted = true;
+            break;
+          }
+          uint8_t* sf = sf_area + sb * SF_BATCH_BYTES;
+          const uint8_t* src[4];
+          bool ok[4];
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            long long r = ti.row0 + lane + 32 * i;
+            ok[i] = r < p.M;  // rows past A's end read row 0 and are zeroed
+            if (!ok[i]) r = 0;
+            src[i] = p.sfa + r * kw + 16 * kb;
+          }
+          uint32_t w[4][4];
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            if (v16) {
+              const uint4 u = __ldg(reinterpret_cast<const uint4*>(src[i]));
+              w[i][0] = u.x;
+              w[i][1] = u.y;
+              w[i][2] = u.z;
+              w[i][3] = u.w;
+            } else {
+#pragma unroll
+              for (int q = 0; q < 4; ++q) w[i][q] = __ldg(reinterpret_cast<const uint32_t*>(src[i]) + q);
+            }
+          }
+#pragma unroll
+          for (int i = 0; i < 4; ++i)
+#pragma unroll
+            for (int q = 0; q < 4; ++q)
+              *reinterpret_cast<uint32_t*>(sf + q * 512 + 16 * lane + 4 * i) = ok[i] ? w[i][q] : 0u;
+          fence_proxy_async_smem();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&sfull[sb]);
+          if (++sb == kSfBufs) {
+            sb = 0;
+            sphase ^= 1;
+          }
+        }
+      }
+    } else if constexpr (!GK) {
+    const int kw = p.K / 32;  // scale bytes per row (a multiple of 4)
     const uint8_t* sfb1 = SPLIT_N ? p.sfb1 : p.sfb0;
     // one 16-byte load per row and batch where every row start is 16-byte aligned
     const bool v16 = (kw % 16) == 0 &&
@@ -393,11 +472,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) gemm_mx_kernel(const __grid_co
     for (int t = blockIdx.x; t < total && !aborted; t += gridDim.x) {
       const Tile ti = get_tile<GK>(p, t, s_off, s_tstart, N_STEP);
       const long long brow = (GK ? 0LL : (long long)ti.g * p.b_group_rows) + ti.n0;
-      // a batch is SB scale words per row: SB k-blocks (MXFP8) or the SB MMAs of one k-block (NVFP4)
-      const int nbatch = NV ? ti.nkb : (ti.nkb + SB - 1) / SB;
-      for (int bi = 0; bi < nbatch; ++bi) {
-        const int nb = NV ? SB : min(SB, ti.nkb - bi * SB);
-        const int kbg = NV ? SB * (ti.kb0 + bi) : ti.kb0 + bi * SB;  // the batch's first scale word in a row
+      for (int kb0 = 0; kb0 < ti.nkb; kb0 += SB) {
+        const int nb = min(SB, ti.nkb - kb0);
+        const int kbg = ti.kb0 + kb0;  // the batch's first k-block in the operands' K
         if (!__all_sync(0xffffffffu,
                         mbar_wait(&sempty[sb], sphase ^ 1, abort_flag, p.status, DEV_WAIT_TIMEOUT_PRODUCER))) {
           aborted = true;
@@ -500,18 +577,24 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) gemm_mx_kernel(const __grid_co
         }
         tc_fence_after();
         if (NV && lane == 0) {
-          // four K64 MMAs, each right after the copies of its own A/B scale chunks into its part of the
-          // k-block's slot (slots alternate by k-block, as below)
+          // the k-block's twelve scale chunks into its slot (slots alternate by k-block, as below), then its
+          // four K64 MMAs: on B200 the copies cost the tensor pipe less issued together than interleaved
           uint8_t* sA = smem + stage * STAGE_BYTES;
           uint8_t* sB = sA + A_BYTES;
           const uint32_t a0 = smem_u32(sA), b0 = smem_u32(sB);
+          const uint32_t col0 = tmem_base + SF_COL + SF_SLOT_COLS_NV * (kb & 1);
 #pragma unroll
           for (int q = 0; q < 4; ++q) {
-            const uint32_t sa = smem_u32(sf_area + sb * SF_BATCH_BYTES + q * SF_KB_BYTES);
-            const uint32_t col = tmem_base + SF_COL + SF_SLOT_COLS_NV * (kb & 1) + SF_SLOT_COLS * q;
+            // batch layout: A chunks at q * 512, B0 at 2048 + q * 512, B1 at 4096 + q * 512
+            const uint32_t sa = smem_u32(sf_area + sb * SF_BATCH_BYTES + q * 512);
+            const uint32_t col = col0 + SF_SLOT_COLS * q;
             tmem_cp_32x128b_x4(col, sf_desc(sa));
-            tmem_cp_32x128b_x4(col + 4, sf_desc(sa + SFA_BYTES));
-            tmem_cp_32x128b_x4(col + 8, sf_desc(sa + SFA_BYTES + 512));
+            tmem_cp_32x128b_x4(col + 4, sf_desc(sa + 2048));
+            tmem_cp_32x128b_x4(col + 8, sf_desc(sa + 4096));
+          }
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            const uint32_t col = col0 + SF_SLOT_COLS * q;
             mma_nvf4(tmem_base, smem_desc_sw128(a0 + q * 32, 16, 1024), smem_desc_sw128(b0 + q * 32, 16, 1024),
                      idesc_nv(BM, BN), col, col + 4, (kb | q) != 0 ? 1u : 0u);
           }

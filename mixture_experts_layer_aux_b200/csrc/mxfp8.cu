@@ -182,7 +182,7 @@ int layer_fwd_mxfp8(const moe_config* c, const void* x, const void* W_r, const f
   if (c->n_shared && (!Ws_g_sf || !Ws_u_sf || !Ws_d_sf)) return MOE_ERR_INVALID_ARG;
   const uint8_t* sfs[] = {W_g_sf, W_u_sf, W_d_sf, Ws_g_sf, Ws_u_sf, Ws_d_sf};
   for (const uint8_t* s : sfs)
-    if (s && !a4(s)) return MOE_ERR_ALIGNMENT;
+    if (s && !(nv ? a16(s) : a4(s))) return MOE_ERR_ALIGNMENT;  // NVFP4 weight scales are bulk-copied
   MxWs w;
   if (!ws || ws_bytes < carve_mx(nullptr, c, &w)) return MOE_ERR_WORKSPACE;
   carve_mx(ws, c, &w);
@@ -238,7 +238,6 @@ int layer_fwd_mxfp8(const moe_config* c, const void* x, const void* W_r, const f
   RCM(copy_out(gates, w.gates, (size_t)T * k * 4, st));
   RCM(copy_out(counts, w.counts, (size_t)E * 4, st));
   RCM(copy_out(offsets, w.offsets, (size_t)(E + 1) * 4, st));
-  (void)a16;
   return MOE_OK;
 }
 

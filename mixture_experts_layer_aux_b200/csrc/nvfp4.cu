@@ -3,8 +3,11 @@
 // Weights: moe_quantize_nvfp4 gives each [R, C] matrix of a [batch, R, C] bf16
 // tensor its own encode scale G = 6 * 448 / amax(matrix) and writes
 //   dst  packed E2M1 [batch, R, C/2],
-//   sf   E4M3 block scales [batch, R, C/16], followed (at byte batch*R*C/16) by
-//        the batch's G values as fp32 [batch] -- one buffer per quantised tensor.
+//   sf   the E4M3 block scales (batch*R*C/16 bytes) TILED in the order the GEMM's
+//        scale copies read them: the 512-byte chunk of 128-row block rb and
+//        64-column group kq sits at (rb * C/64 + kq) * 512, row r of it at byte
+//        16 (r % 32) + 4 ((r % 128) / 32), its four 16-blocks' scales in a row --
+//        followed by the batch's G values as fp32 [batch]: one buffer per tensor.
 // Three kernels: the per-matrix amax (block max, then an integer atomicMax on
 // the fp32 bits, valid for non-negative floats) into the G slots, the
 // quantisation (each block turns its matrix's amax into G itself), and the
@@ -44,11 +47,12 @@ __global__ void __launch_bounds__(256) amax_kernel(const __nv_bfloat16* __restri
   }
 }
 
-// One thread per 16-block of matrix blockIdx.y ([R, C], C % 16 == 0). gslot[blockIdx.y] holds the matrix's
-// amax (fp32 bits), from which G is derived; without gslot, G = 1.
+// One thread per 16-block of matrix blockIdx.y ([R, C], C % 16 == 0; cb = C/16 blocks per row).
+// gslot[blockIdx.y] holds the matrix's amax (fp32 bits), from which G is derived; without gslot, G = 1.
+// tiled: scales in the chunk order above (R % 128 == 0, C % 64 == 0), else row-major [rows, C/16].
 __global__ void __launch_bounds__(256) quant_kernel(const __nv_bfloat16* __restrict__ src, long long nblocks,
                                                    uint8_t* __restrict__ dst, uint8_t* __restrict__ sf,
-                                                   const unsigned int* __restrict__ gslot) {
+                                                   const unsigned int* __restrict__ gslot, int cb, int tiled) {
   const long long mb = blockIdx.y;
   const float G = gslot ? global_scale(__uint_as_float(gslot[mb])) : 1.0f;
   for (long long b = blockIdx.x * (long long)blockDim.x + threadIdx.x; b < nblocks;
@@ -59,7 +63,13 @@ __global__ void __launch_bounds__(256) quant_kernel(const __nv_bfloat16* __restr
     unpack_bf16x8(s4[0], *reinterpret_cast<float(*)[8]>(f));
     unpack_bf16x8(s4[1], *reinterpret_cast<float(*)[8]>(f + 8));
     uint32_t w0, w1;
-    sf[gb] = nvq::quant16(f, G, w0, w1);
+    long long si = gb;
+    if (tiled) {
+      const long long grow = gb / cb;
+      const int c = (int)(gb - grow * cb);
+      si = ((grow / 128) * (cb / 4) + c / 4) * 512 + 16 * (grow % 32) + 4 * ((grow % 128) / 32) + (c % 4);
+    }
+    sf[si] = nvq::quant16(f, G, w0, w1);
     reinterpret_cast<uint2*>(dst)[gb] = make_uint2(w0, w1);
   }
 }
@@ -80,10 +90,9 @@ size_t nvfp4_sf_bytes(long long batch, long long R, long long C) { return (size_
 
 int quantize_nvfp4(const void* src, int batch, long long R, int C, uint8_t* dst, uint8_t* sf, cudaStream_t st) {
   if (!src || !dst || !sf || batch < 1 || R < 1 || C < 16) return MOE_ERR_INVALID_ARG;
-  if (C % 16 != 0) return MOE_ERR_UNSUPPORTED;
-  if (!a16(src) || !a16(dst) || !a4(sf)) return MOE_ERR_ALIGNMENT;
+  if (C % 64 != 0 || R % 128 != 0) return MOE_ERR_UNSUPPORTED;  // whole scale chunks
+  if (!a16(src) || !a16(dst) || !a16(sf)) return MOE_ERR_ALIGNMENT;
   const long long nblk = R * (C / 16);  // blocks per matrix; the G slots follow batch * nblk scale bytes
-  if ((batch * nblk) % 4 != 0) return MOE_ERR_ALIGNMENT;
   unsigned int* gslot = reinterpret_cast<unsigned int*>(sf + batch * nblk);
   if (cudaMemsetAsync(gslot, 0, 4 * (size_t)batch, st) != cudaSuccess) {
     (void)cudaGetLastError();
@@ -95,7 +104,8 @@ int quantize_nvfp4(const void* src, int batch, long long R, int C, uint8_t* dst,
   nvk::amax_kernel<<<dim3(gx, batch), 256, 0, st>>>(static_cast<const __nv_bfloat16*>(src), n, gslot);
   MOE_CHECK_LAUNCH();
   gx = (int)std::max(1LL, std::min<long long>((nblk + 255) / 256, 148LL * 16 / batch));
-  nvk::quant_kernel<<<dim3(gx, batch), 256, 0, st>>>(static_cast<const __nv_bfloat16*>(src), nblk, dst, sf, gslot);
+  nvk::quant_kernel<<<dim3(gx, batch), 256, 0, st>>>(static_cast<const __nv_bfloat16*>(src), nblk, dst, sf, gslot,
+                                                      C / 16, 1);
   MOE_CHECK_LAUNCH();
   nvk::finalize_kernel<<<(batch + 255) / 256, 256, 0, st>>>(gslot, batch);
   MOE_CHECK_LAUNCH();
@@ -108,7 +118,8 @@ int quantize_nvfp4_act(const void* src, long long rows, int K, uint8_t* dst, uin
   if (!a16(src) || !a16(dst)) return MOE_ERR_ALIGNMENT;
   const long long nblk = rows * (K / 16);
   const int gx = (int)std::min<long long>((nblk + 255) / 256, 148LL * 16);
-  nvk::quant_kernel<<<dim3(gx, 1), 256, 0, st>>>(static_cast<const __nv_bfloat16*>(src), nblk, dst, sf, nullptr);
+  nvk::quant_kernel<<<dim3(gx, 1), 256, 0, st>>>(static_cast<const __nv_bfloat16*>(src), nblk, dst, sf, nullptr,
+                                                  K / 16, 0);
   MOE_CHECK_LAUNCH();
   return MOE_OK;
 }
@@ -175,7 +186,8 @@ int grouped_gemm_fwd_nv(const moe_config* c, int which, const void* A, const uin
                         const float* row_gate, void* C, uint8_t* C_sf, void* save, cudaStream_t st) {
   if (c->H % 256 != 0 || c->F % 256 != 0) return MOE_ERR_UNSUPPORTED;
   if (!A_sf || !B0_sf || save) return MOE_ERR_INVALID_ARG;
-  if (!a4(A_sf) || !a4(B0_sf) || (B1_sf && !a4(B1_sf)) || (C_sf && !a4(C_sf))) return MOE_ERR_ALIGNMENT;
+  // the weights' tiled scale chunks are bulk-copied: 16-byte aligned
+  if (!a4(A_sf) || !a16(B0_sf) || (B1_sf && !a16(B1_sf)) || (C_sf && !a4(C_sf))) return MOE_ERR_ALIGNMENT;
   const int rows = c->T * c->k;
   const long long E = c->E, H = c->H, F = c->F;
   if (which == MOE_GEMM_GATEUP_SWIGLU) {

@@ -160,11 +160,11 @@ def test_nvfp4_argument_errors(lib, B):
     assert lib.moe_nvfp4_sf_bytes(2, 3, 32) == 2 * 3 * 2 + 8
     assert lib.moe_nvfp4_sf_bytes(1, 4, 24) == 0
     q = lib.moe_quantize_nvfp4
-    assert q(FAKE, 1, 4, 24, FAKE, FAKE, None) == UNSUPPORTED       # C % 16 != 0
-    assert q(FAKE, 1, 4, 8, FAKE, FAKE, None) == INVALID            # C < 16
-    assert q(None, 1, 4, 32, FAKE, FAKE, None) == INVALID
-    assert q(FAKE, 1, 4, 32, FAKE, FAKE + 2, None) == ALIGN         # sf not 4-byte aligned
-    assert q(FAKE, 1, 1, 16, FAKE, FAKE, None) == ALIGN             # G slots would not be 4-byte aligned
+    assert q(FAKE, 1, 128, 48, FAKE, FAKE, None) == UNSUPPORTED     # C % 64 != 0 (whole scale chunks)
+    assert q(FAKE, 1, 100, 64, FAKE, FAKE, None) == UNSUPPORTED     # R % 128 != 0
+    assert q(FAKE, 1, 128, 8, FAKE, FAKE, None) == INVALID          # C < 16
+    assert q(None, 1, 128, 64, FAKE, FAKE, None) == INVALID
+    assert q(FAKE, 1, 128, 64, FAKE, FAKE + 4, None) == ALIGN       # sf is bulk-copied: 16-byte aligned
     qa = lib.moe_quantize_nvfp4_act
     assert qa(FAKE, 4, 24, FAKE, FAKE, None) == UNSUPPORTED
     assert qa(FAKE + 8, 4, 32, FAKE, FAKE, None) == ALIGN

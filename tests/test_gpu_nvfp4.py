@@ -31,10 +31,16 @@ def _gpu_quant_w(moe, w):
 
 
 def _split_sf(sf, batch, R, C):
-    """moe_quantize_nvfp4's scale buffer -> (scales [batch, R, C/16] uint8, G [batch] fp32)."""
+    """moe_quantize_nvfp4's scale buffer -> (row-major scales [batch, R, C/16] uint8, G [batch] fp32).
+
+    The buffer holds the scales tiled: byte ((r/128) * C/64 + c/4) * 512 + 16 (r%32) + 4 ((r%128)/32) + c%4
+    for global row r and 16-block c."""
     n = batch * R * (C // 16)
     s = sf.cpu()
-    return s[:n].view(batch, R, C // 16), s[n:].view(torch.float32)
+    r = torch.arange(batch * R).view(-1, 1)
+    c = torch.arange(C // 16).view(1, -1)
+    idx = ((r // 128) * (C // 64) + c // 4) * 512 + 16 * (r % 32) + 4 * ((r % 128) // 32) + c % 4
+    return s[:n][idx].view(batch, R, C // 16), s[n:].view(torch.float32)
 
 
 def _decoded_scales(oracle, sf_bytes):
@@ -45,7 +51,7 @@ def _decoded_scales(oracle, sf_bytes):
 # ------------------------------------------------------------------ quantisers
 
 
-@pytest.mark.parametrize("batch,R,C", [(3, 64, 256), (2, 300, 7168), (1, 7, 2048)])
+@pytest.mark.parametrize("batch,R,C", [(3, 128, 256), (2, 384, 7168), (1, 128, 2048)])
 def test_quantize_nvfp4_weights_bit_exact(moe, oracle, batch, R, C):
     w = randn_bf16((batch, R, C), 0.02, seed=R + C, scale_rows=True)
     w[0, 0, :16] = 0  # an all-zero block
