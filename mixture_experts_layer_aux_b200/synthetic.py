@@ -87,6 +87,10 @@ WORKLOADS = {
     # the DeepSeek-V3 forward with NVFP4 expert operands (E2M1 + E4M3 per 16, per-expert encode scales)
     "dsv3-nvfp4": Workload("dsv3-nvfp4", T=8192, H=7168, E=256, k=8, F=2048, S=1, score="sigmoid",
                            route_scale=2.5, dtype="nvfp4", aux=False),
+    # the same with 64 experts and T=2048: the same ~256 rows per expert (so the same tile structure) on a
+    # quarter of the weights, about 1.5 GB on the device
+    "dsv3-nvfp4-e64": Workload("dsv3-nvfp4-e64", T=2048, H=7168, E=64, k=8, F=2048, S=1, score="sigmoid",
+                               route_scale=2.5, dtype="nvfp4", aux=False),
     # the MXFP8 backward on the DeepSeek-V3 routed experts (the backward has no shared expert)
     "dsv3-train": Workload("dsv3-train", T=8192, H=7168, E=256, k=8, F=2048, score="sigmoid", route_scale=2.5,
                            dtype="mxfp8", aux=False, bwd=True),
