@@ -4,8 +4,8 @@ Every call of the C ABI launches on the caller's stream, reads its problem
 sizes from device memory (expert offsets) and never synchronises or
 allocates, so a captured layer step replays without the host. These tests
 capture moe_layer_fwd + moe_layer_bwd (BF16, with a ragged expert mix and
-a zero-token expert) and moe_layer_fwd (MXFP8, with a shared expert) in a
-CUDA graph, replay it, and require every output to equal the eager run bit
+a zero-token expert) and moe_layer_fwd (MXFP8 and NVFP4, with a shared
+expert) in a CUDA graph, replay it, and require every output to equal the eager run bit
 for bit (the kernels are deterministic: fixed-order reductions, no atomics
 on floating point).
 """
@@ -95,6 +95,34 @@ def test_layer_fwd_mxfp8_graph_replay_equals_eager(moe):
         sf = torch.empty(w.shape[:-1] + (w.shape[-1] // 32,), dtype=torch.uint8, device="cuda")
         moe.moe_quantize_mxfp8(w, codes, sf)
         q[name] = (codes, sf)
+    torch.cuda.synchronize()
+
+    def make():
+        cfg = moe.make_config(wl)
+        o = dict(y=empty((wl.T, wl.H), torch.bfloat16), idx=empty((wl.T, wl.k), torch.int32),
+                 gates=empty((wl.T, wl.k), torch.float32))
+        ws = moe.workspace(moe.moe_layer_workspace_size(cfg))
+
+        def step():
+            moe.moe_layer_fwd(cfg, d["x"], d["W_r"], None, q["W_g"][0], q["W_u"][0], q["W_d"][0], q["W_g"][1],
+                              q["W_u"][1], q["W_d"][1], q["W_gs"][0], q["W_us"][0], q["W_ds"][0], q["W_gs"][1],
+                              q["W_us"][1], q["W_ds"][1], o["y"], None, o["idx"], o["gates"], None, None, None, ws)
+        return o, step
+    _capture_and_compare(moe, make)
+
+
+def test_layer_fwd_nvfp4_graph_replay_equals_eager(moe):
+    wl = Workload("graph_nv", T=640, H=512, E=8, k=2, F=256, S=1, score="sigmoid", route_scale=2.5, aux=False,
+                  dtype="nvfp4")
+    d = make_inputs(wl, device="cuda", seed=13)
+    q = {}
+    for name in ["W_g", "W_u", "W_d", "W_gs", "W_us", "W_ds"]:
+        w = d[name]
+        R, C = w.shape[-2], w.shape[-1]
+        packed = torch.empty(w.shape[:-1] + (C // 2,), dtype=torch.uint8, device="cuda")
+        sf = torch.empty(moe.moe_nvfp4_sf_bytes(w.numel() // (R * C), R, C), dtype=torch.uint8, device="cuda")
+        moe.moe_quantize_nvfp4(w, packed, sf)
+        q[name] = (packed, sf)
     torch.cuda.synchronize()
 
     def make():

@@ -195,7 +195,7 @@ def check_fwd_nv(moe, oracle, wl, n_sample=None, seed=0):
         toks = toks.to(torch.int32)
     toks = toks[same[toks.long()]]
     # the oracle quantises the bf16 weights itself, only the experts the sampled tokens use (G per expert)
-    need = sorted(set(r["idx"][toks.long()].flatten().tolist()))
+    need = sorted(set(r["idx"][toks.long()].flatten().tolist()) - {-1})
     nv = {}
     for name in ("W_g", "W_u", "W_d"):
         W = d[name]
@@ -211,8 +211,8 @@ def check_fwd_nv(moe, oracle, wl, n_sample=None, seed=0):
             nv[name] = oracle.nvfp4_quantize(d[name].cpu(), per_matrix=True)
     shared = (nv["W_gs"][0], nv["W_us"][0], nv["W_ds"][0], nv["W_gs"][1:], nv["W_us"][1:], nv["W_ds"][1:]) \
         if wl.S else None
-    y_ref = oracle.moe_fwd_tokens(d["x"].cpu(), nv["W_g"][0], nv["W_u"][0], nv["W_d"][0], r["idx"], r["gates"], toks,
-                                  recipe="nvfp4", sf_g=nv["W_g"][1:], sf_u=nv["W_u"][1:], sf_d=nv["W_d"][1:],
+    y_ref = oracle.moe_fwd_tokens(d["x"].cpu(), nv["W_g"][0], nv["W_u"][0], nv["W_d"][0], r["idx_kept"], r["gates"],
+                                  toks, recipe="nvfp4", sf_g=nv["W_g"][1:], sf_u=nv["W_u"][1:], sf_d=nv["W_d"][1:],
                                   shared=shared)
     e = check_bf16(y.cpu()[toks.long()], y_ref, tol=TOL_NVFP4)
     assert moe.moe_get_device_status() == 0
@@ -227,6 +227,13 @@ def test_layer_fwd_nvfp4_small_full_oracle(moe, oracle):
 
 def test_layer_fwd_nvfp4_softmax_ragged_full_oracle(moe, oracle):
     wl = Workload("nv-ragged", T=333, H=768, E=12, k=3, F=512, dtype="nvfp4", aux=True)
+    check_fwd_nv(moe, oracle, wl)
+
+
+def test_layer_fwd_nvfp4_deepseek_router_and_capacity_full_oracle(moe, oracle):
+    # the DeepSeek-V3 router variant (selection bias, 4 groups, 2 kept) with a capacity factor that drops pairs
+    wl = Workload("nv-dsv3-cap", T=320, H=512, E=32, k=4, F=256, S=1, score="sigmoid", route_scale=2.5, aux=False,
+                  dtype="nvfp4", n_group=4, topk_group=2, sel_bias=True, capacity_factor=1.0)
     check_fwd_nv(moe, oracle, wl)
 
 
