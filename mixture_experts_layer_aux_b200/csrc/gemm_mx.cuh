@@ -548,14 +548,15 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) gemm_mx_kernel(const __grid_co
     }
     }
   } else if (warp == 1) {
-    // ======================= MMA issuer
+    // ======================= MMA issuer: one thread (no warp votes or syncs per k-block)
+    if (lane == 0) {
     int stage = 0;
     uint32_t phase = 0, acc_phase = 0;
     int sb = 0;  // scale batch in shared memory
     uint32_t sphase = 0;
     for (int t = blockIdx.x; t < total && !aborted; t += gridDim.x) {
       const Tile ti = get_tile<GK>(p, t, s_off, s_tstart, N_STEP);
-      if (!__all_sync(0xffffffffu, mbar_wait(tempty, acc_phase ^ 1, abort_flag, p.status, DEV_WAIT_TIMEOUT_MMA))) {
+      if (!mbar_wait(tempty, acc_phase ^ 1, abort_flag, p.status, DEV_WAIT_TIMEOUT_MMA)) {
         aborted = true;
         break;
       }
@@ -565,18 +566,17 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) gemm_mx_kernel(const __grid_co
         const bool batch_end = NV || (j == SB - 1) || (kb == ti.nkb - 1);
         if (j == 0) {
           // a new scale batch in shared memory
-          if (!__all_sync(0xffffffffu,
-                          mbar_wait(&sfull[sb], sphase, abort_flag, p.status, DEV_WAIT_TIMEOUT_MMA))) {
+          if (!mbar_wait(&sfull[sb], sphase, abort_flag, p.status, DEV_WAIT_TIMEOUT_MMA)) {
             aborted = true;
             break;
           }
         }
-        if (!__all_sync(0xffffffffu, mbar_wait(&full[stage], phase, abort_flag, p.status, DEV_WAIT_TIMEOUT_MMA))) {
+        if (!mbar_wait(&full[stage], phase, abort_flag, p.status, DEV_WAIT_TIMEOUT_MMA)) {
           aborted = true;
           break;
         }
         tc_fence_after();
-        if (NV && lane == 0) {
+        if (NV) {
           // the k-block's twelve scale chunks into its slot (slots alternate by k-block, as below), then its
           // four K64 MMAs: on B200 the copies cost the tensor pipe less issued together than interleaved
           uint8_t* sA = smem + stage * STAGE_BYTES;
@@ -600,7 +600,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) gemm_mx_kernel(const __grid_co
           }
           mma_commit(&sempty[sb]);
           mma_commit(&empty[stage]);
-        } else if (!NV && lane == 0) {
+        } else {
           // this k-block's scale chunks into its TMEM slot (alternating by k-block; in issue order
           // after the MMAs that read the slot two k-blocks ago), copied right before its MMAs:
           // on B200 three copies per k-block cost the tensor pipe far less than a batch of twelve
@@ -626,7 +626,6 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) gemm_mx_kernel(const __grid_co
           }
           mma_commit(&empty[stage]);
         }
-        __syncwarp();
         if (batch_end && ++sb == kSfBufs) {
           sb = 0;
           sphase ^= 1;
@@ -637,15 +636,15 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) gemm_mx_kernel(const __grid_co
         }
       }
       if (aborted) break;
-      if (lane == 0) mma_commit(tfull);
-      __syncwarp();
+      mma_commit(tfull);
       acc_phase ^= 1;
     }
-    if (*abort_flag && lane == 0) {
+    if (*abort_flag) {
       mma_commit(drain);
       const uint64_t t0 = globaltimer_ns();
       while (!mbar_try_wait(drain, 0) && globaltimer_ns() - t0 < MOE_WAIT_NS) {
       }
+    }
     }
     __syncwarp();
   } else {

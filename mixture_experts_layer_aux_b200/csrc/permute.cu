@@ -206,10 +206,9 @@ __global__ void __launch_bounds__(SC_WARPS * 32) scatter_kernel(
   for (int j = 0; j < 16; ++j) rows[j] = __shfl_sync(0xffffffffu, r, j < k ? j : 0);
   const uint4* src = reinterpret_cast<const uint4*>(x + (long long)t * H);
   const int nchunk = H / 8;
-  for (int i0 = 0; i0 < nchunk; i0 += 32) {
-    const int i = i0 + lane;
+  // one 8-element chunk (16 bytes) of the row, to its k destinations
+  auto emit = [&](const int i, const uint4 d) {
     const bool v = i < nchunk;
-    const uint4 d = v ? src[i] : make_uint4(0, 0, 0, 0);
     if constexpr (QF == QF_BF16) {
       if (v) {
 #pragma unroll
@@ -254,6 +253,18 @@ __global__ void __launch_bounds__(SC_WARPS * 32) scatter_kernel(
           }
       }
     }
+  };
+  // four chunks per lane in flight before any is written (the row is read once; the writes dominate)
+  constexpr int U = 4;
+  for (int i0 = 0; i0 < nchunk; i0 += 32 * U) {
+    uint4 d[U];
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      const int i = i0 + 32 * u + lane;
+      d[u] = i < nchunk ? src[i] : make_uint4(0, 0, 0, 0);
+    }
+#pragma unroll
+    for (int u = 0; u < U; ++u) emit(i0 + 32 * u + lane, d[u]);
   }
 }
 
