@@ -73,8 +73,20 @@ constexpr int SF_SLOT_COLS_NV = 48;     // NVFP4: four MMAs of 12 columns each
 constexpr int BAR_BYTES = 1024;
 constexpr int STG_WARP_BYTES = 32 * 32;  // bf16 epilogue staging: 32 rows x 16 columns per epilogue warp
 constexpr int SMEM_BYTES =
-    1024 + kStages * STAGE_BYTES + kSfBufs * SF_BATCH_BYTES + BAR_BYTES + 2 * (MAX_G + 1) * 4 + 16 +
+    1024 + kStages * STAGE_BYTES + kSfBufs * SF_BATCH_BYTES + BAR_BYTES + 2 * (MAX_G + 1) * 4 + 128 +
     8 * STG_WARP_BYTES;
+// Grouped along K (weight gradients, short K per tile, a bf16 output that dominates the traffic): three TMA
+// stages, and four staging buffers per epilogue warp so that its TMA stores stay in flight
+constexpr int kStagesGK = 3;
+constexpr int STG_BUFS_GK = 4;
+template <bool GK>
+constexpr int stages() { return GK ? kStagesGK : kStages; }
+template <bool GK>
+constexpr int smem_bytes() {
+  return 1024 + stages<GK>() * STAGE_BYTES + kSfBufs * SF_BATCH_BYTES + BAR_BYTES + 2 * (MAX_G + 1) * 4 + 128 +
+         8 * STG_WARP_BYTES * (GK ? STG_BUFS_GK : 1);
+}
+static_assert(smem_bytes<true>() <= 232448, "smem");
 static_assert(SF_COL + 2 * SF_SLOT_COLS_NV <= TMEM_COLS, "tmem");
 static_assert(SMEM_BYTES <= 232448, "smem");
 
@@ -89,6 +101,10 @@ struct __align__(64) Params {
   CUtensorMap tmA;
   CUtensorMap tmB0;
   CUtensorMap tmB1;
+  // GROUP_K bf16 output through TMA stores (tma_store != 0): C and C2 as [G * c_rows_per_group, N] bf16,
+  // no swizzle, 16 x 32 boxes
+  CUtensorMap tmC;
+  CUtensorMap tmC2;
   int M;              // rows of A (all groups)
   int N;              // output columns per group
   int K;              // reduction length (multiple of 128)
@@ -120,6 +136,8 @@ struct __align__(64) Params {
   // NVFP4: per-group encode scales G of B0 and B1 (NULL: 1); the accumulators are divided by them
   const float* gscale0;
   const float* gscale1;
+  long long c_rows_per_group;  // GROUP_K TMA stores: rows of one group in tmC / tmC2
+  int tma_store;
 };
 
 struct Tile {
@@ -230,13 +248,28 @@ MOE_DEV void quant32(const float* v, float inv, uint32_t (&w)[8]) {
   }
 }
 
+// TMA store of a shared-memory box to global (bulk-group completion), and the waits on those groups.
+MOE_DEV void tma_store_2d(const CUtensorMap* m, const void* smem_src, int x, int y) {
+  asm volatile("cp.async.bulk.tensor.2d.global.shared::cta.bulk_group [%0, {%1, %2}], [%3];" ::"l"(
+                   reinterpret_cast<uint64_t>(m)),
+               "r"(x), "r"(y), "r"(smem_u32(smem_src))
+               : "memory");
+}
+MOE_DEV void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
+template <int N>
+MOE_DEV void bulk_wait_read() {
+  asm volatile("cp.async.bulk.wait_group.read %0;" ::"n"(N) : "memory");
+}
+MOE_DEV void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
+
 template <int EPI, bool SPLIT_N, bool GK, bool NV>
 __global__ void __launch_bounds__(NUM_THREADS, 1) gemm_mx_kernel(const __grid_constant__ Params p) {
   static_assert(!(NV && GK), "NVFP4: forward GEMMs only");
   static_assert(!(NV && EPI == EPI_MX_SWIGLU_BWD), "NVFP4: forward GEMMs only");
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint8_t* sf_area = smem + kStages * STAGE_BYTES;
+  constexpr int NST = stages<GK>();
+  uint8_t* sf_area = smem + NST * STAGE_BYTES;
   uint8_t* bar_area = sf_area + kSfBufs * SF_BATCH_BYTES;
   uint64_t* full = reinterpret_cast<uint64_t*>(bar_area);
   uint64_t* empty = full + kStages;
@@ -249,8 +282,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) gemm_mx_kernel(const __grid_co
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   int* s_off = reinterpret_cast<int*>(bar_area + BAR_BYTES);
   int* s_tstart = s_off + (MAX_G + 1);
+  // 128-byte aligned: the TMA stores read their boxes from here
   uint8_t* stg_area =
-      reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(s_tstart + (MAX_G + 1)) + 15) & ~uintptr_t(15));
+      reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(s_tstart + (MAX_G + 1)) + 127) & ~uintptr_t(127));
   constexpr int N_STEP = SPLIT_N ? BN / 2 : BN;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -380,7 +414,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) gemm_mx_kernel(const __grid_co
             tma_load_2d(sB, &p.tmB0, kc, brow, &full[stage]);
             tma_load_2d(sB + 128 * BK, &p.tmB0, kc, brow + 128, &full[stage]);
           }
-          if (++stage == kStages) {
+          if (++stage == NST) {
             stage = 0;
             phase ^= 1;
           }
@@ -630,7 +664,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) gemm_mx_kernel(const __grid_co
           sb = 0;
           sphase ^= 1;
         }
-        if (++stage == kStages) {
+        if (++stage == NST) {
           stage = 0;
           phase ^= 1;
         }
@@ -653,6 +687,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) gemm_mx_kernel(const __grid_co
     const int h = (warp - 3) >> 2;
     const int row = q * 32 + lane;
     uint32_t acc_phase = 0;
+    uint32_t stg_seq = 0;  // GROUP_K TMA stores: slices issued by this warp (picks the staging buffer)
     for (int t = blockIdx.x; t < total && !aborted; t += gridDim.x) {
       const Tile ti = get_tile<GK>(p, t, s_off, s_tstart, N_STEP);
       if (!__all_sync(0xffffffffu, mbar_wait(tfull, acc_phase, abort_flag, p.status, DEV_WAIT_TIMEOUT_EPILOGUE))) {
@@ -775,45 +810,85 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) gemm_mx_kernel(const __grid_co
         }
       }
       if constexpr (EPI == EPI_MX_BF16) {
-        // 16 columns at a time through shared memory, so that each warp store writes whole 32-byte
-        // sectors: lanes 2i, 2i+1 write the two halves of one row's 32 bytes (16 rows per store)
-        uint8_t* stg = stg_area + (warp - 3) * STG_WARP_BYTES;
-        const int ncol = min(128, p.N - ti.n0 - 128 * h);  // columns of this half inside the output
-#pragma unroll
-        for (int pass = 0; pass < 8; ++pass) {
-          if (16 * pass >= ncol) break;  // warp-uniform
-          *reinterpret_cast<uint4*>(stg + lane * 32) =
-              make_uint4(pack_bf16x2(v[16 * pass], v[16 * pass + 1]), pack_bf16x2(v[16 * pass + 2], v[16 * pass + 3]),
-                         pack_bf16x2(v[16 * pass + 4], v[16 * pass + 5]),
-                         pack_bf16x2(v[16 * pass + 6], v[16 * pass + 7]));
-          *reinterpret_cast<uint4*>(stg + lane * 32 + 16) =
-              make_uint4(pack_bf16x2(v[16 * pass + 8], v[16 * pass + 9]),
-                         pack_bf16x2(v[16 * pass + 10], v[16 * pass + 11]),
-                         pack_bf16x2(v[16 * pass + 12], v[16 * pass + 13]),
-                         pack_bf16x2(v[16 * pass + 14], v[16 * pass + 15]));
-          __syncwarp();
-#pragma unroll
-          for (int i = 0; i < 2; ++i) {
-            const int rr = 16 * i + (lane >> 1);
-            const int trow = q * 32 + rr;  // row within the tile
-            if (trow < ti.m_valid) {
-              long long r = (long long)ti.row0 + trow;
-              __nv_bfloat16* base = reinterpret_cast<__nv_bfloat16*>(p.C);
-              if constexpr (GK) {
-                if (p.c2_row_split > 0 && r >= p.c2_row_split) {
-                  r -= p.c2_row_split;
-                  base = reinterpret_cast<__nv_bfloat16*>(p.C2);
-                }
-                base += ti.g * p.c_group_stride;
-              }
-              *reinterpret_cast<uint4*>(base + r * p.ldc + ti.n0 + 128 * h + 16 * pass + 8 * (lane & 1)) =
-                  *reinterpret_cast<const uint4*>(stg + rr * 32 + 16 * (lane & 1));
-            }
+        if (GK && p.tma_store) {
+          if (32 * q >= ti.m_valid) continue;  // warp-uniform: a 32-row block past the output (M % 32 == 0)
+          // grouped along K: each 32-row x 16-column slice leaves through a TMA store from one of four
+          // staging buffers of this warp (a buffer is rewritten once the store issued four slices earlier has
+          // read it), so the epilogue issues no global stores of its own
+          uint8_t* stg_w = stg_area + (warp - 3) * STG_WARP_BYTES * STG_BUFS_GK;
+          const int ncol = min(128, p.N - ti.n0 - 128 * h);
+          long long r0 = (long long)ti.row0 + 32 * q;
+          const CUtensorMap* tm = &p.tmC;
+          if (p.c2_row_split > 0 && r0 >= p.c2_row_split) {
+            r0 -= p.c2_row_split;
+            tm = &p.tmC2;
           }
-          __syncwarp();
+          const int y = (int)(ti.g * p.c_rows_per_group + r0);
+#pragma unroll
+          for (int pass = 0; pass < 8; ++pass) {
+            if (16 * pass >= ncol) break;  // warp-uniform
+            uint8_t* stg = stg_w + (stg_seq & (STG_BUFS_GK - 1)) * STG_WARP_BYTES;
+            if (lane == 0) bulk_wait_read<STG_BUFS_GK - 1>();
+            __syncwarp();
+            *reinterpret_cast<uint4*>(stg + lane * 32) =
+                make_uint4(pack_bf16x2(v[16 * pass], v[16 * pass + 1]), pack_bf16x2(v[16 * pass + 2], v[16 * pass + 3]),
+                           pack_bf16x2(v[16 * pass + 4], v[16 * pass + 5]),
+                           pack_bf16x2(v[16 * pass + 6], v[16 * pass + 7]));
+            *reinterpret_cast<uint4*>(stg + lane * 32 + 16) =
+                make_uint4(pack_bf16x2(v[16 * pass + 8], v[16 * pass + 9]),
+                           pack_bf16x2(v[16 * pass + 10], v[16 * pass + 11]),
+                           pack_bf16x2(v[16 * pass + 12], v[16 * pass + 13]),
+                           pack_bf16x2(v[16 * pass + 14], v[16 * pass + 15]));
+            fence_proxy_async_smem();  // the generic-proxy writes, for the TMA engine's reads
+            __syncwarp();
+            if (lane == 0) {
+              tma_store_2d(tm, stg, ti.n0 + 128 * h + 16 * pass, y);
+              bulk_commit();
+            }
+            ++stg_seq;
+          }
+        } else {
+          // 16 columns at a time through shared memory, so that each warp store writes whole 32-byte
+          // sectors: lanes 2i, 2i+1 write the two halves of one row's 32 bytes (16 rows per store)
+          uint8_t* stg = stg_area + (warp - 3) * STG_WARP_BYTES * (GK ? STG_BUFS_GK : 1);
+          const int ncol = min(128, p.N - ti.n0 - 128 * h);  // columns of this half inside the output
+#pragma unroll
+          for (int pass = 0; pass < 8; ++pass) {
+            if (16 * pass >= ncol) break;  // warp-uniform
+            *reinterpret_cast<uint4*>(stg + lane * 32) =
+                make_uint4(pack_bf16x2(v[16 * pass], v[16 * pass + 1]), pack_bf16x2(v[16 * pass + 2], v[16 * pass + 3]),
+                           pack_bf16x2(v[16 * pass + 4], v[16 * pass + 5]),
+                           pack_bf16x2(v[16 * pass + 6], v[16 * pass + 7]));
+            *reinterpret_cast<uint4*>(stg + lane * 32 + 16) =
+                make_uint4(pack_bf16x2(v[16 * pass + 8], v[16 * pass + 9]),
+                           pack_bf16x2(v[16 * pass + 10], v[16 * pass + 11]),
+                           pack_bf16x2(v[16 * pass + 12], v[16 * pass + 13]),
+                           pack_bf16x2(v[16 * pass + 14], v[16 * pass + 15]));
+            __syncwarp();
+#pragma unroll
+            for (int i = 0; i < 2; ++i) {
+              const int rr = 16 * i + (lane >> 1);
+              const int trow = q * 32 + rr;  // row within the tile
+              if (trow < ti.m_valid) {
+                long long r = (long long)ti.row0 + trow;
+                __nv_bfloat16* base = reinterpret_cast<__nv_bfloat16*>(p.C);
+                if constexpr (GK) {
+                  if (p.c2_row_split > 0 && r >= p.c2_row_split) {
+                    r -= p.c2_row_split;
+                    base = reinterpret_cast<__nv_bfloat16*>(p.C2);
+                  }
+                  base += ti.g * p.c_group_stride;
+                }
+                *reinterpret_cast<uint4*>(base + r * p.ldc + ti.n0 + 128 * h + 16 * pass + 8 * (lane & 1)) =
+                    *reinterpret_cast<const uint4*>(stg + rr * 32 + 16 * (lane & 1));
+              }
+            }
+            __syncwarp();
+          }
         }
       }
     }
+    if (GK && lane == 0) bulk_wait_all();  // every TMA store has read its staging buffer and landed
   }
 
   __syncthreads();
@@ -827,13 +902,14 @@ template <int EPI, bool SPLIT_N, bool GK = false, bool NV = false>
 int launch(const Params& p, int max_tiles, cudaStream_t stream) {
   if (max_tiles <= 0) return MOE_OK;
   auto kern = gemm_mx_kernel<EPI, SPLIT_N, GK, NV>;
-  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES) != cudaSuccess) {
+  constexpr int SMEM = smem_bytes<GK>();
+  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM) != cudaSuccess) {
     (void)cudaGetLastError();
     return MOE_ERR_CUDA;
   }
   int grid = moe_host::num_sms();
   if (grid > max_tiles) grid = max_tiles;
-  kern<<<grid, NUM_THREADS, SMEM_BYTES, stream>>>(p);
+  kern<<<grid, NUM_THREADS, SMEM, stream>>>(p);
   MOE_CHECK_LAUNCH();
   return MOE_OK;
 }

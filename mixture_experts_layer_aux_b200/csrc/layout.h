@@ -22,6 +22,12 @@ struct Carve {
   }
 };
 
+namespace moe_host {
+// 2D tensor map without swizzle (for TMA stores of row-major staging boxes); see encode_tmap_2d.
+bool encode_tmap_2d_plain(CUtensorMap* m, CUtensorMapDataType dt, const void* base, uint64_t inner, uint64_t outer,
+                          uint64_t row_stride_bytes, uint32_t box_inner, uint32_t box_outer);
+}  // namespace moe_host
+
 namespace moe_impl {
 // What the MXFP8 backward reads from an MXFP8 forward that saved for it.
 struct SavedMx {
