@@ -16,6 +16,8 @@
 //     and its 32-row scale blocks never straddle two experts.
 #include <cuda_fp8.h>
 
+#include <type_traits>
+
 #include "common.cuh"
 #include "gemm_mx.cuh"
 #include "layout.h"
@@ -73,43 +75,45 @@ struct QtArgs {
   uint8_t* sf;               // [C, ldd / 32] (WEIGHT: [B, C, ldd / 32]) ue8m0
 };
 
-// One block: 64 consecutive output positions (padded rows; never two experts: segments start on 128-row
-// boundaries) x 128 columns. The 64 x 128 tile is staged in fp32 through shared memory; then each thread
-// quantises one column of one 32-row half (a 1x32 block along the output's K) and stores its 32 codes.
-// The padded offsets are read into shared memory first, so finding the tile's expert is a shared-memory
-// search.
+// One block: TR consecutive output positions (padded rows; never two experts: segments start on 128-row
+// boundaries) x 128 columns, TR = 128 when the source is bf16 (staged as bf16: exact) and 64 for the
+// gate-folded activation, which is computed and staged in fp32. Each thread then quantises TR/64 consecutive
+// 1x32 blocks of one column (the output's K) and stores their codes as one run of 32 or 64 bytes. One
+// thread finds the tile's expert by a binary search of the padded offsets.
 constexpr int QT_COLS = 128;
-constexpr int QT_ROWS = 64;
+constexpr int QT_ROWS = 64;    // fp32-staged tiles (MODE_AP)
+constexpr int QT_ROWS_BF = 128;  // bf16-staged tiles
+__host__ __device__ constexpr int qt_rows(int mode) { return mode == 2 ? QT_ROWS : QT_ROWS_BF; }
 template <int MODE>
 __global__ void __launch_bounds__(256) quant_t_kernel(const QtArgs a) {
-  __shared__ float tile[QT_ROWS][QT_COLS + 1];
-  __shared__ int s_poff[513];
+  constexpr bool F32 = MODE == MODE_AP;
+  constexpr int TR = qt_rows(MODE);
+  constexpr int PADC = F32 ? 1 : 8;  // row padding (elements): conflict-free column reads, 16-byte row starts
+  using TT = typename std::conditional<F32, float, __nv_bfloat16>::type;
+  __shared__ __align__(16) TT tile[TR][QT_COLS + PADC];
   __shared__ int s_meta[3];  // first source row (-1: none), valid rows, rows to write
-  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const int p0 = blockIdx.x * QT_ROWS;  // first output position (padded row)
+  const int tid = threadIdx.x;
+  const int p0 = blockIdx.x * TR;  // first output position (padded row)
   const int c0 = blockIdx.y * QT_COLS;
   const int b = MODE == MODE_WEIGHT ? blockIdx.z : 0;
-  if constexpr (MODE != MODE_WEIGHT) {
-    for (int i = tid; i <= a.E; i += blockDim.x) s_poff[i] = a.poff[i];
-    __syncthreads();
-  }
   if (tid == 0) {
     int r0 = -1, nv = 0, nw = 0;
     if constexpr (MODE == MODE_WEIGHT) {
       r0 = p0;
-      nv = nw = min(QT_ROWS, a.R - p0);  // R % 32 == 0: 32 or 64
-    } else if (p0 < s_poff[a.E]) {
+      nv = nw = min(TR, a.R - p0);  // R % 32 == 0: a multiple of 32
+    } else if (p0 < __ldg(a.poff + a.E)) {
       int lo = 0, hi = a.E - 1;  // expert whose padded segment holds p0
       while (lo < hi) {
         const int mid = (lo + hi + 1) >> 1;
-        if (s_poff[mid] <= p0) lo = mid;
+        if (__ldg(a.poff + mid) <= p0) lo = mid;
         else hi = mid - 1;
       }
-      const int i = p0 - s_poff[lo];
-      const int cnt = a.off[lo + 1] - a.off[lo];
-      r0 = a.off[lo] + i;
-      nv = max(0, min(QT_ROWS, cnt - i));
-      nw = QT_ROWS;  // pad rows are written (zero)
+      const int i = p0 - __ldg(a.poff + lo);
+      const int o = __ldg(a.off + lo);
+      const int cnt = __ldg(a.off + lo + 1) - o;
+      r0 = o + i;
+      nv = max(0, min(TR, cnt - i));
+      nw = TR;  // pad rows are written (zero)
     }
     s_meta[0] = r0;
     s_meta[1] = nv;
@@ -120,14 +124,15 @@ __global__ void __launch_bounds__(256) quant_t_kernel(const QtArgs a) {
   if (r0 < 0) return;  // past the padded total (block-uniform)
   // load: thread t -> rows t/16 + 16 i, columns 8*(t%16) .. +7 of the tile
 #pragma unroll
-  for (int it = 0; it < QT_ROWS / 16; ++it) {
+  for (int it = 0; it < TR / 16; ++it) {
     const int rr = (tid >> 4) + 16 * it, cc = (tid & 15) * 8;
-    float f[8];
+    const bool ok = rr < nv && c0 + cc < a.C;
+    if constexpr (F32) {
+      float f[8];
 #pragma unroll
-    for (int q = 0; q < 8; ++q) f[q] = 0.f;
-    if (rr < nv && c0 + cc < a.C) {
-      const long long r = r0 + rr;
-      if constexpr (MODE == MODE_AP) {
+      for (int q = 0; q < 8; ++q) f[q] = 0.f;
+      if (ok) {
+        const long long r = r0 + rr;
         const __nv_bfloat16* gp = a.src + r * 2LL * a.C + c0 + cc;
         float zg[8], zu[8];
         unpack_bf16x8(*reinterpret_cast<const uint4*>(gp), zg);
@@ -135,16 +140,20 @@ __global__ void __launch_bounds__(256) quant_t_kernel(const QtArgs a) {
         const float g = a.row_gate[r];
 #pragma unroll
         for (int q = 0; q < 8; ++q) f[q] = g * silu_f(zg[q]) * zu[q];
-      } else {
-        long long sr = r;
-        if constexpr (MODE == MODE_GATHER) sr = a.src_of[r];
+      }
+#pragma unroll
+      for (int q = 0; q < 8; ++q) tile[rr][cc + q] = f[q];
+    } else {
+      uint4 u = make_uint4(0, 0, 0, 0);
+      if (ok) {
+        long long sr = r0 + rr;
+        if constexpr (MODE == MODE_GATHER) sr = a.src_of[sr];
         const __nv_bfloat16* base = a.src;
         if constexpr (MODE == MODE_WEIGHT) base += (long long)b * a.R * a.C;
-        unpack_bf16x8(*reinterpret_cast<const uint4*>(base + sr * a.C + c0 + cc), f);
+        u = *reinterpret_cast<const uint4*>(base + sr * a.C + c0 + cc);
       }
+      *reinterpret_cast<uint4*>(&tile[rr][cc]) = u;
     }
-#pragma unroll
-    for (int q = 0; q < 8; ++q) tile[rr][cc + q] = f[q];
   }
   __syncthreads();
   uint8_t* dst = a.dst;
@@ -153,41 +162,51 @@ __global__ void __launch_bounds__(256) quant_t_kernel(const QtArgs a) {
     dst += (long long)b * a.C * a.ldd;
     sf += (long long)b * a.C * (a.ldd / 32);
   }
-  // quantise: thread t takes column t % 128 of the 32-row half t / 128 -- one 1x32 block in registers, its
-  // amax by a plain loop, its 32 codes as two 16-byte stores
-  {
-    const int c = tid % QT_COLS, hb = tid / QT_COLS;
-    if (c0 + c < a.C && 32 * hb < nw) {
-      float v[32];
-      float am = 0.f;
+  // quantise: thread t takes column t % 128 and the TR/2 rows of half t / 128: TR/64 blocks of 32, each with
+  // its amax by a plain loop; the codes of the half leave as one contiguous run
+  const int c = tid % QT_COLS, hb = tid / QT_COLS;
+  constexpr int NB = TR / 64;  // 32-row blocks per thread
+  if (c0 + c >= a.C) return;
+  uint32_t w[NB][8];
+  uint8_t sbv[NB];
 #pragma unroll
-      for (int i = 0; i < 32; ++i) {
-        v[i] = tile[32 * hb + i][c];
-        am = fmaxf(am, fabsf(v[i]));
-      }
-      const uint8_t sb = mx_scale_byte(am);
-      const float inv = mx_inv_scale(sb);
-      uint32_t w[8];
+  for (int bb = 0; bb < NB; ++bb) {
+    const int rb = (TR / 2) * hb + 32 * bb;  // first tile row of the block
+    float v[32];
+    float am = 0.f;
 #pragma unroll
-      for (int q = 0; q < 8; ++q) {
-        const __nv_fp8x2_storage_t lo =
-            __nv_cvt_float2_to_fp8x2(make_float2(v[4 * q] * inv, v[4 * q + 1] * inv), __NV_SATFINITE, __NV_E4M3);
-        const __nv_fp8x2_storage_t hi =
-            __nv_cvt_float2_to_fp8x2(make_float2(v[4 * q + 2] * inv, v[4 * q + 3] * inv), __NV_SATFINITE, __NV_E4M3);
-        w[q] = (uint32_t)lo | ((uint32_t)hi << 16);
-      }
-      const int p = p0 + 32 * hb;
-      uint4* d4 = reinterpret_cast<uint4*>(dst + (long long)(c0 + c) * a.ldd + p);
-      d4[0] = make_uint4(w[0], w[1], w[2], w[3]);
-      d4[1] = make_uint4(w[4], w[5], w[6], w[7]);
-      if constexpr (MODE == MODE_WEIGHT) {
-        sf[(long long)(c0 + c) * (a.ldd / 32) + p / 32] = sb;  // natural [C, ldd/32]
-      } else {
-        // tiled for the weight-gradient GEMM: chunk (row block, k-block of 128), then the UTCCP order
-        const int r = c0 + c, kb32 = p / 32;
-        sf[((long long)(r / 128) * (a.ldd / 128) + kb32 / 4) * 512 + (r % 32) * 16 + ((r % 128) / 32) * 4 + kb32 % 4] =
-            sb;
-      }
+    for (int i = 0; i < 32; ++i) {
+      if constexpr (F32) v[i] = tile[rb + i][c];
+      else v[i] = __bfloat162float(tile[rb + i][c]);
+      am = fmaxf(am, fabsf(v[i]));
+    }
+    const uint8_t sb = mx_scale_byte(am);
+    sbv[bb] = sb;
+    const float inv = mx_inv_scale(sb);
+#pragma unroll
+    for (int q = 0; q < 8; ++q) {
+      const __nv_fp8x2_storage_t lo =
+          __nv_cvt_float2_to_fp8x2(make_float2(v[4 * q] * inv, v[4 * q + 1] * inv), __NV_SATFINITE, __NV_E4M3);
+      const __nv_fp8x2_storage_t hi =
+          __nv_cvt_float2_to_fp8x2(make_float2(v[4 * q + 2] * inv, v[4 * q + 3] * inv), __NV_SATFINITE, __NV_E4M3);
+      w[bb][q] = (uint32_t)lo | ((uint32_t)hi << 16);
+    }
+  }
+  const int pbase = p0 + (TR / 2) * hb;
+  uint4* d4 = reinterpret_cast<uint4*>(dst + (long long)(c0 + c) * a.ldd + pbase);
+#pragma unroll
+  for (int bb = 0; bb < NB; ++bb) {
+    if ((TR / 2) * hb + 32 * bb >= nw) break;  // rows past a weight matrix's end (R % 32 == 0)
+    d4[2 * bb] = make_uint4(w[bb][0], w[bb][1], w[bb][2], w[bb][3]);
+    d4[2 * bb + 1] = make_uint4(w[bb][4], w[bb][5], w[bb][6], w[bb][7]);
+    const int p = pbase + 32 * bb;
+    if constexpr (MODE == MODE_WEIGHT) {
+      sf[(long long)(c0 + c) * (a.ldd / 32) + p / 32] = sbv[bb];  // natural [C, ldd/32]
+    } else {
+      // tiled for the weight-gradient GEMM: chunk (row block, k-block of 128), then the UTCCP order
+      const int r = c0 + c, kb32 = p / 32;
+      sf[((long long)(r / 128) * (a.ldd / 128) + kb32 / 4) * 512 + (r % 32) * 16 + ((r % 128) / 32) * 4 + kb32 % 4] =
+          sbv[bb];
     }
   }
 }
@@ -222,8 +241,8 @@ int quant_t_rows(int mode, const void* src, const int32_t* src_of, const float* 
   a.ldd = ldd;
   a.sf = sf;
   const long long pmax = rows + (long long)mxb::PAD * E;
-  const dim3 grid((unsigned)((pmax + mxb::QT_ROWS - 1) / mxb::QT_ROWS),
-                  (unsigned)((C + mxb::QT_COLS - 1) / mxb::QT_COLS));
+  const int tr = mxb::qt_rows(mode);
+  const dim3 grid((unsigned)((pmax + tr - 1) / tr), (unsigned)((C + mxb::QT_COLS - 1) / mxb::QT_COLS));
   if (mode == 0) mxb::quant_t_kernel<mxb::MODE_ROWS><<<grid, 256, 0, st>>>(a);
   else if (mode == 1) mxb::quant_t_kernel<mxb::MODE_GATHER><<<grid, 256, 0, st>>>(a);
   else mxb::quant_t_kernel<mxb::MODE_AP><<<grid, 256, 0, st>>>(a);
@@ -337,8 +356,8 @@ extern "C" int moe_quantize_mxfp8_t(const void* src, int32_t batch, int32_t R, i
   a.dst = static_cast<uint8_t*>(dst);
   a.ldd = ldd;
   a.sf = sf;
-  const dim3 grid((unsigned)((R + mxb::QT_ROWS - 1) / mxb::QT_ROWS), (unsigned)((C + mxb::QT_COLS - 1) / mxb::QT_COLS),
-                  (unsigned)batch);
+  const dim3 grid((unsigned)((R + mxb::QT_ROWS_BF - 1) / mxb::QT_ROWS_BF),
+                  (unsigned)((C + mxb::QT_COLS - 1) / mxb::QT_COLS), (unsigned)batch);
   mxb::quant_t_kernel<mxb::MODE_WEIGHT><<<grid, 256, 0, static_cast<cudaStream_t>(stream)>>>(a);
   MOE_CHECK_LAUNCH();
   return MOE_OK;
