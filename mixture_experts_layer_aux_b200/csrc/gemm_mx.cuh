@@ -506,20 +506,13 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) gemm_mx_kernel(const __grid_co
     for (int t = blockIdx.x; t < total && !aborted; t += gridDim.x) {
       const Tile ti = get_tile<GK>(p, t, s_off, s_tstart, N_STEP);
       const long long brow = (GK ? 0LL : (long long)ti.g * p.b_group_rows) + ti.n0;
-      for (int kb0 = 0; kb0 < ti.nkb; kb0 += SB) {
+      // lane l: rows l, l+32, l+64, l+96 of A (i < 4), and of each 128-row half of B (i >= 4). All twelve
+      // rows' loads of a batch are issued together, and those of the next batch go out before this one waits
+      // for its buffer, so two batches' latencies overlap; rows past A's end read row 0 and are zeroed.
+      auto load_batch = [&](const int kb0, uint32_t (&w)[12][SB], bool (&ok)[12]) {
         const int nb = min(SB, ti.nkb - kb0);
         const int kbg = ti.kb0 + kb0;  // the batch's first k-block in the operands' K
-        if (!__all_sync(0xffffffffu,
-                        mbar_wait(&sempty[sb], sphase ^ 1, abort_flag, p.status, DEV_WAIT_TIMEOUT_PRODUCER))) {
-          aborted = true;
-          break;
-        }
-        uint8_t* sf = sf_area + sb * SF_BATCH_BYTES;
-        // lane l: rows l, l+32, l+64, l+96 of A (i < 4), and of each 128-row half of B (i >= 4).
-        // All twelve rows' loads are issued before any is used, so their latencies overlap;
-        // rows past A's end read row 0 and are zeroed.
         const uint8_t* src[12];
-        bool ok[12];
 #pragma unroll
         for (int i = 0; i < 12; ++i) {
           const uint8_t* base;
@@ -539,14 +532,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) gemm_mx_kernel(const __grid_co
               base = p.sfb0;
               r = brow + lane + 32 * ib;
             }
-            if (GK) {  // B [N, K] is shared by the groups: rows past N read row 0 and are zeroed
-              ok[i] = r < p.N;
-              if (!ok[i]) r = 0;
-            }
           }
           src[i] = base + r * kw + 4 * kbg;
         }
-        uint32_t w[12][SB];
         if (v16 && nb == SB && (kbg & 3) == 0) {
 #pragma unroll
           for (int i = 0; i < 12; ++i) {
@@ -562,6 +550,20 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) gemm_mx_kernel(const __grid_co
 #pragma unroll
             for (int j = 0; j < SB; ++j) w[i][j] = __ldg(reinterpret_cast<const uint32_t*>(src[i]) + min(j, nb - 1));
         }
+      };
+      uint32_t w[12][SB], wn[12][SB];
+      bool ok[12], okn[12];
+      if (ti.nkb > 0) load_batch(0, w, ok);
+      for (int kb0 = 0; kb0 < ti.nkb; kb0 += SB) {
+        const int nb = min(SB, ti.nkb - kb0);
+        const bool more = kb0 + SB < ti.nkb;
+        if (more) load_batch(kb0 + SB, wn, okn);
+        if (!__all_sync(0xffffffffu,
+                        mbar_wait(&sempty[sb], sphase ^ 1, abort_flag, p.status, DEV_WAIT_TIMEOUT_PRODUCER))) {
+          aborted = true;
+          break;
+        }
+        uint8_t* sf = sf_area + sb * SF_BATCH_BYTES;
 #pragma unroll
         for (int i = 0; i < 12; ++i) {
           const int ib = i - 4;
@@ -574,6 +576,14 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) gemm_mx_kernel(const __grid_co
         fence_proxy_async_smem();
         __syncwarp();
         if (lane == 0) mbar_arrive(&sfull[sb]);
+        if (more) {
+#pragma unroll
+          for (int i = 0; i < 12; ++i) {
+            ok[i] = okn[i];
+#pragma unroll
+            for (int j = 0; j < SB; ++j) w[i][j] = wn[i][j];
+          }
+        }
         if (++sb == kSfBufs) {
           sb = 0;
           sphase ^= 1;
