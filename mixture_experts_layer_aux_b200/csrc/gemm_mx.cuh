@@ -594,101 +594,101 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) gemm_mx_kernel(const __grid_co
   } else if (warp == 1) {
     // ======================= MMA issuer: one thread (no warp votes or syncs per k-block)
     if (lane == 0) {
-    int stage = 0;
-    uint32_t phase = 0, acc_phase = 0;
-    int sb = 0;  // scale batch in shared memory
-    uint32_t sphase = 0;
-    for (int t = blockIdx.x; t < total && !aborted; t += gridDim.x) {
-      const Tile ti = get_tile<GK>(p, t, s_off, s_tstart, N_STEP);
-      if (!mbar_wait(tempty, acc_phase ^ 1, abort_flag, p.status, DEV_WAIT_TIMEOUT_MMA)) {
-        aborted = true;
-        break;
-      }
-      tc_fence_after();
-      for (int kb = 0; kb < ti.nkb; ++kb) {
-        const int j = NV ? 0 : kb % SB;
-        const bool batch_end = NV || (j == SB - 1) || (kb == ti.nkb - 1);
-        if (j == 0) {
-          // a new scale batch in shared memory
-          if (!mbar_wait(&sfull[sb], sphase, abort_flag, p.status, DEV_WAIT_TIMEOUT_MMA)) {
-            aborted = true;
-            break;
-          }
-        }
-        if (!mbar_wait(&full[stage], phase, abort_flag, p.status, DEV_WAIT_TIMEOUT_MMA)) {
+      int stage = 0;
+      uint32_t phase = 0, acc_phase = 0;
+      int sb = 0;  // scale batch in shared memory
+      uint32_t sphase = 0;
+      for (int t = blockIdx.x; t < total && !aborted; t += gridDim.x) {
+        const Tile ti = get_tile<GK>(p, t, s_off, s_tstart, N_STEP);
+        if (!mbar_wait(tempty, acc_phase ^ 1, abort_flag, p.status, DEV_WAIT_TIMEOUT_MMA)) {
           aborted = true;
           break;
         }
         tc_fence_after();
-        if (NV) {
-          // the k-block's twelve scale chunks into its slot (slots alternate by k-block, as below), then its
-          // four K64 MMAs: on B200 the copies cost the tensor pipe less issued together than interleaved
-          uint8_t* sA = smem + stage * STAGE_BYTES;
-          uint8_t* sB = sA + A_BYTES;
-          const uint32_t a0 = smem_u32(sA), b0 = smem_u32(sB);
-          const uint32_t col0 = tmem_base + SF_COL + SF_SLOT_COLS_NV * (kb & 1);
+        for (int kb = 0; kb < ti.nkb; ++kb) {
+          const int j = NV ? 0 : kb % SB;
+          const bool batch_end = NV || (j == SB - 1) || (kb == ti.nkb - 1);
+          if (j == 0) {
+            // a new scale batch in shared memory
+            if (!mbar_wait(&sfull[sb], sphase, abort_flag, p.status, DEV_WAIT_TIMEOUT_MMA)) {
+              aborted = true;
+              break;
+            }
+          }
+          if (!mbar_wait(&full[stage], phase, abort_flag, p.status, DEV_WAIT_TIMEOUT_MMA)) {
+            aborted = true;
+            break;
+          }
+          tc_fence_after();
+          if (NV) {
+            // the k-block's twelve scale chunks into its slot (slots alternate by k-block, as below), then its
+            // four K64 MMAs: on B200 the copies cost the tensor pipe less issued together than interleaved
+            uint8_t* sA = smem + stage * STAGE_BYTES;
+            uint8_t* sB = sA + A_BYTES;
+            const uint32_t a0 = smem_u32(sA), b0 = smem_u32(sB);
+            const uint32_t col0 = tmem_base + SF_COL + SF_SLOT_COLS_NV * (kb & 1);
 #pragma unroll
-          for (int q = 0; q < 4; ++q) {
-            // batch layout: A chunks at q * 512, B0 at 2048 + q * 512, B1 at 4096 + q * 512
-            const uint32_t sa = smem_u32(sf_area + sb * SF_BATCH_BYTES + q * 512);
-            const uint32_t col = col0 + SF_SLOT_COLS * q;
+            for (int q = 0; q < 4; ++q) {
+              // batch layout: A chunks at q * 512, B0 at 2048 + q * 512, B1 at 4096 + q * 512
+              const uint32_t sa = smem_u32(sf_area + sb * SF_BATCH_BYTES + q * 512);
+              const uint32_t col = col0 + SF_SLOT_COLS * q;
+              tmem_cp_32x128b_x4(col, sf_desc(sa));
+              tmem_cp_32x128b_x4(col + 4, sf_desc(sa + 2048));
+              tmem_cp_32x128b_x4(col + 8, sf_desc(sa + 4096));
+            }
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+              const uint32_t col = col0 + SF_SLOT_COLS * q;
+              mma_nvf4(tmem_base, smem_desc_sw128(a0 + q * 32, 16, 1024), smem_desc_sw128(b0 + q * 32, 16, 1024),
+                       idesc_nv(BM, BN), col, col + 4, (kb | q) != 0 ? 1u : 0u);
+            }
+            mma_commit(&sempty[sb]);
+            mma_commit(&empty[stage]);
+          } else {
+            // this k-block's scale chunks into its TMEM slot (alternating by k-block; in issue order
+            // after the MMAs that read the slot two k-blocks ago), copied right before its MMAs:
+            // on B200 three copies per k-block cost the tensor pipe far less than a batch of twelve
+            const uint8_t* sf = sf_area + sb * SF_BATCH_BYTES + j * SF_KB_BYTES;
+            const uint32_t col = tmem_base + SF_COL + SF_SLOT_COLS * (kb & 1);
+            const uint32_t sa = smem_u32(sf);
             tmem_cp_32x128b_x4(col, sf_desc(sa));
-            tmem_cp_32x128b_x4(col + 4, sf_desc(sa + 2048));
-            tmem_cp_32x128b_x4(col + 8, sf_desc(sa + 4096));
-          }
+            tmem_cp_32x128b_x4(col + 4, sf_desc(sa + SFA_BYTES));
+            tmem_cp_32x128b_x4(col + 8, sf_desc(sa + SFA_BYTES + 512));
+            if (batch_end) mma_commit(&sempty[sb]);  // the batch's shared memory is free once its copies are done
+            uint8_t* sA = smem + stage * STAGE_BYTES;
+            uint8_t* sB = sA + A_BYTES;
+            const uint32_t sfa_t = col;
+            const uint32_t sfb_t = col + 4;
+            const uint32_t a0 = smem_u32(sA), b0 = smem_u32(sB);
 #pragma unroll
-          for (int q = 0; q < 4; ++q) {
-            const uint32_t col = col0 + SF_SLOT_COLS * q;
-            mma_nvf4(tmem_base, smem_desc_sw128(a0 + q * 32, 16, 1024), smem_desc_sw128(b0 + q * 32, 16, 1024),
-                     idesc_nv(BM, BN), col, col + 4, (kb | q) != 0 ? 1u : 0u);
+            for (int q = 0; q < BK / 32; ++q) {
+              // scale byte q of each 32-bit TMEM word: in the descriptor's sf ids and in
+              // the top two bits of the scale addresses
+              mma_mxf8(tmem_base, smem_desc_sw128(a0 + q * 32, 16, 1024), smem_desc_sw128(b0 + q * 32, 16, 1024),
+                       idesc_mx(BM, BN, q), sfa_t | ((uint32_t)q << 30), sfb_t | ((uint32_t)q << 30),
+                       (kb | q) != 0 ? 1u : 0u);
+            }
+            mma_commit(&empty[stage]);
           }
-          mma_commit(&sempty[sb]);
-          mma_commit(&empty[stage]);
-        } else {
-          // this k-block's scale chunks into its TMEM slot (alternating by k-block; in issue order
-          // after the MMAs that read the slot two k-blocks ago), copied right before its MMAs:
-          // on B200 three copies per k-block cost the tensor pipe far less than a batch of twelve
-          const uint8_t* sf = sf_area + sb * SF_BATCH_BYTES + j * SF_KB_BYTES;
-          const uint32_t col = tmem_base + SF_COL + SF_SLOT_COLS * (kb & 1);
-          const uint32_t sa = smem_u32(sf);
-          tmem_cp_32x128b_x4(col, sf_desc(sa));
-          tmem_cp_32x128b_x4(col + 4, sf_desc(sa + SFA_BYTES));
-          tmem_cp_32x128b_x4(col + 8, sf_desc(sa + SFA_BYTES + 512));
-          if (batch_end) mma_commit(&sempty[sb]);  // the batch's shared memory is free once its copies are done
-          uint8_t* sA = smem + stage * STAGE_BYTES;
-          uint8_t* sB = sA + A_BYTES;
-          const uint32_t sfa_t = col;
-          const uint32_t sfb_t = col + 4;
-          const uint32_t a0 = smem_u32(sA), b0 = smem_u32(sB);
-#pragma unroll
-          for (int q = 0; q < BK / 32; ++q) {
-            // scale byte q of each 32-bit TMEM word: in the descriptor's sf ids and in
-            // the top two bits of the scale addresses
-            mma_mxf8(tmem_base, smem_desc_sw128(a0 + q * 32, 16, 1024), smem_desc_sw128(b0 + q * 32, 16, 1024),
-                     idesc_mx(BM, BN, q), sfa_t | ((uint32_t)q << 30), sfb_t | ((uint32_t)q << 30),
-                     (kb | q) != 0 ? 1u : 0u);
+          if (batch_end && ++sb == kSfBufs) {
+            sb = 0;
+            sphase ^= 1;
           }
-          mma_commit(&empty[stage]);
+          if (++stage == NST) {
+            stage = 0;
+            phase ^= 1;
+          }
         }
-        if (batch_end && ++sb == kSfBufs) {
-          sb = 0;
-          sphase ^= 1;
-        }
-        if (++stage == NST) {
-          stage = 0;
-          phase ^= 1;
+        if (aborted) break;
+        mma_commit(tfull);
+        acc_phase ^= 1;
+      }
+      if (*abort_flag) {
+        mma_commit(drain);
+        const uint64_t t0 = globaltimer_ns();
+        while (!mbar_try_wait(drain, 0) && globaltimer_ns() - t0 < MOE_WAIT_NS) {
         }
       }
-      if (aborted) break;
-      mma_commit(tfull);
-      acc_phase ^= 1;
-    }
-    if (*abort_flag) {
-      mma_commit(drain);
-      const uint64_t t0 = globaltimer_ns();
-      while (!mbar_try_wait(drain, 0) && globaltimer_ns() - t0 < MOE_WAIT_NS) {
-      }
-    }
     }
     __syncwarp();
   } else {
