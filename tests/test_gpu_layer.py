@@ -308,8 +308,8 @@ def check_fwd_mx(moe, oracle, wl, n_sample=None, seed=0):
             mx[name] = oracle.mxfp8_quantize(d[name].cpu())
     shared = (mx["W_gs"][0], mx["W_us"][0], mx["W_ds"][0], mx["W_gs"][1], mx["W_us"][1], mx["W_ds"][1]) if wl.S \
         else None
-    y_ref = oracle.moe_fwd_tokens(d["x"].cpu(), mx["W_g"][0], mx["W_u"][0], mx["W_d"][0], r["idx"], r["gates"], toks,
-                                  recipe="mxfp8", sf_g=mx["W_g"][1], sf_u=mx["W_u"][1], sf_d=mx["W_d"][1],
+    y_ref = oracle.moe_fwd_tokens(d["x"].cpu(), mx["W_g"][0], mx["W_u"][0], mx["W_d"][0], r["idx_kept"], r["gates"],
+                                  toks, recipe="mxfp8", sf_g=mx["W_g"][1], sf_u=mx["W_u"][1], sf_d=mx["W_d"][1],
                                   shared=shared)
     e = check_bf16(y.cpu()[toks.long()], y_ref, tol=6e-2)
     assert moe.moe_get_device_status() == 0
@@ -325,6 +325,13 @@ def test_layer_fwd_mxfp8_small_full_oracle(moe, oracle):
 def test_layer_fwd_mxfp8_deepseek_router_variant(moe, oracle):
     wl = Workload("mx-dsv3-router", T=256, H=512, E=32, k=4, F=256, S=1, score="sigmoid", route_scale=2.5,
                   aux=False, dtype="mxfp8", n_group=4, topk_group=2, sel_bias=True)
+    check_fwd_mx(moe, oracle, wl)
+
+
+def test_layer_fwd_mxfp8_deepseek_router_with_capacity(moe, oracle):
+    # the DeepSeek-V3 router variant with a capacity factor that drops pairs (dropped pairs: no row, no output)
+    wl = Workload("mx-dsv3-cap", T=320, H=512, E=32, k=4, F=256, S=1, score="sigmoid", route_scale=2.5,
+                  aux=False, dtype="mxfp8", n_group=4, topk_group=2, sel_bias=True, capacity_factor=1.0)
     check_fwd_mx(moe, oracle, wl)
 
 
