@@ -79,14 +79,23 @@ constexpr int SMEM_BYTES =
 // stages, and four staging buffers per epilogue warp so that its TMA stores stay in flight
 constexpr int kStagesGK = 3;
 constexpr int STG_BUFS_GK = 4;
-template <bool GK>
-constexpr int stages() { return GK ? kStagesGK : kStages; }
-template <bool GK>
-constexpr int smem_bytes() {
-  return 1024 + stages<GK>() * STAGE_BYTES + kSfBufs * SF_BATCH_BYTES + BAR_BYTES + 2 * (MAX_G + 1) * 4 + 128 +
-         8 * STG_WARP_BYTES * (GK ? STG_BUFS_GK : 1);
+// The SwiGLU-backward epilogue stages the saved gate/up of its 32 rows, 32 columns at a time (64 bytes per
+// row, padded to 80), and its dgate/dup on the way out: 5 KB per warp, the room of the fourth TMA stage.
+constexpr int STG_ROW_BWD = 80;
+constexpr int STG_BWD_WARP_BYTES = 2 * 32 * STG_ROW_BWD;
+template <int EPI, bool GK>
+constexpr int stages() { return (GK || EPI == 2) ? kStagesGK : kStages; }
+template <int EPI, bool GK>
+constexpr int stg_warp_bytes() {
+  return GK ? STG_WARP_BYTES * STG_BUFS_GK : (EPI == 2 ? STG_BWD_WARP_BYTES : STG_WARP_BYTES);
 }
-static_assert(smem_bytes<true>() <= 232448, "smem");
+template <int EPI, bool GK>
+constexpr int smem_bytes() {
+  return 1024 + stages<EPI, GK>() * STAGE_BYTES + kSfBufs * SF_BATCH_BYTES + BAR_BYTES + 2 * (MAX_G + 1) * 4 +
+         128 + 8 * stg_warp_bytes<EPI, GK>();
+}
+static_assert(smem_bytes<1, true>() <= 232448, "smem");
+static_assert(smem_bytes<2, false>() <= 232448, "smem");
 static_assert(SF_COL + 2 * SF_SLOT_COLS_NV <= TMEM_COLS, "tmem");
 static_assert(SMEM_BYTES <= 232448, "smem");
 
@@ -268,7 +277,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) gemm_mx_kernel(const __grid_co
   static_assert(!(NV && EPI == EPI_MX_SWIGLU_BWD), "NVFP4: forward GEMMs only");
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  constexpr int NST = stages<GK>();
+  constexpr int NST = stages<EPI, GK>();
   uint8_t* sf_area = smem + NST * STAGE_BYTES;
   uint8_t* bar_area = sf_area + kSfBufs * SF_BATCH_BYTES;
   uint64_t* full = reinterpret_cast<uint64_t*>(bar_area);
@@ -786,22 +795,44 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) gemm_mx_kernel(const __grid_co
             *reinterpret_cast<uint16_t*>(p.C_sf + orow * (p.ldc / 32) + col0 / 32) =
                 (uint16_t)sb[0] | ((uint16_t)sb[1] << 8);
           }
-        } else if (EPI == EPI_MX_SWIGLU_BWD) {
-          // columns [col0, col0 + 128) of F: dgate, dup from the saved bf16 pre-activations z
-          const float g = p.row_gate[orow];
-          const int col0 = ti.n0 + 128 * h;
-          const __nv_bfloat16* zp = p.gateup + orow * 2LL * p.N + col0;
-          __nv_bfloat16* dp = reinterpret_cast<__nv_bfloat16*>(p.C) + orow * 2LL * p.N + col0;
-          float part = 0.f;
+        }
+      }
+      if constexpr (EPI == EPI_MX_SWIGLU_BWD) {
+        // columns [col0, col0 + 128) of F, 32 at a time: the saved bf16 gate/up of the warp's 32 rows come into
+        // shared memory row-contiguously (4 lanes x 16 bytes per row), each lane forms its row's dgate/dup
+        // there from its accumulator values, and they leave the same way
+        uint8_t* sG = stg_area + (warp - 3) * STG_BWD_WARP_BYTES;
+        uint8_t* sU = sG + 32 * STG_ROW_BWD;
+        const int col0 = ti.n0 + 128 * h;
+        const float g = valid ? p.row_gate[orow] : 0.f;
+        const int st_piece = lane & 3, st_r0 = lane >> 2;
+        const long long ld2 = 2LL * p.N;
+        __nv_bfloat16* dgu = reinterpret_cast<__nv_bfloat16*>(p.C);
+        float part = 0.f;
 #pragma unroll
-          for (int c = 0; c < 16; ++c) {
+        for (int c = 0; c < 4; ++c) {
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            const int r = 8 * i + st_r0;
+            uint4 zg4 = make_uint4(0, 0, 0, 0), zu4 = make_uint4(0, 0, 0, 0);
+            if (q * 32 + r < ti.m_valid) {
+              const __nv_bfloat16* src = p.gateup + ((long long)ti.row0 + q * 32 + r) * ld2 + col0 + 32 * c + 8 * st_piece;
+              zg4 = *reinterpret_cast<const uint4*>(src);
+              zu4 = *reinterpret_cast<const uint4*>(src + p.N);
+            }
+            *reinterpret_cast<uint4*>(sG + r * STG_ROW_BWD + 16 * st_piece) = zg4;
+            *reinterpret_cast<uint4*>(sU + r * STG_ROW_BWD + 16 * st_piece) = zu4;
+          }
+          __syncwarp();
+#pragma unroll
+          for (int j = 0; j < 4; ++j) {
             float zg[8], zu[8];
-            unpack_bf16x8(reinterpret_cast<const uint4*>(zp)[c], zg);
-            unpack_bf16x8(reinterpret_cast<const uint4*>(zp + p.N)[c], zu);
+            unpack_bf16x8(*reinterpret_cast<const uint4*>(sG + lane * STG_ROW_BWD + 16 * j), zg);
+            unpack_bf16x8(*reinterpret_cast<const uint4*>(sU + lane * STG_ROW_BWD + 16 * j), zu);
             float dgv[8], duv[8];
 #pragma unroll
             for (int i = 0; i < 8; ++i) {
-              const float vv = v[8 * c + i];
+              const float vv = v[32 * c + 8 * j + i];
               const float sg = 1.0f / (1.0f + __expf(-zg[i]));
               const float sl = zg[i] * sg;
               part += vv * sl * zu[i];
@@ -809,15 +840,27 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) gemm_mx_kernel(const __grid_co
               dgv[i] = da * zu[i] * sg * (1.f + zg[i] * (1.f - sg));
               duv[i] = da * sl;
             }
-            reinterpret_cast<uint4*>(dp)[c] =
+            *reinterpret_cast<uint4*>(sG + lane * STG_ROW_BWD + 16 * j) =
                 make_uint4(pack_bf16x2(dgv[0], dgv[1]), pack_bf16x2(dgv[2], dgv[3]), pack_bf16x2(dgv[4], dgv[5]),
                            pack_bf16x2(dgv[6], dgv[7]));
-            reinterpret_cast<uint4*>(dp + p.N)[c] =
+            *reinterpret_cast<uint4*>(sU + lane * STG_ROW_BWD + 16 * j) =
                 make_uint4(pack_bf16x2(duv[0], duv[1]), pack_bf16x2(duv[2], duv[3]), pack_bf16x2(duv[4], duv[5]),
                            pack_bf16x2(duv[6], duv[7]));
           }
-          p.dg_part[orow * (long long)(p.N / 128) + col0 / 128] = part;
+          __syncwarp();
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            const int r = 8 * i + st_r0;
+            if (q * 32 + r < ti.m_valid) {
+              __nv_bfloat16* dst = dgu + ((long long)ti.row0 + q * 32 + r) * ld2 + col0 + 32 * c + 8 * st_piece;
+              *reinterpret_cast<uint4*>(dst) = *reinterpret_cast<const uint4*>(sG + r * STG_ROW_BWD + 16 * st_piece);
+              *reinterpret_cast<uint4*>(dst + p.N) =
+                  *reinterpret_cast<const uint4*>(sU + r * STG_ROW_BWD + 16 * st_piece);
+            }
+          }
+          __syncwarp();
         }
+        if (valid) p.dg_part[orow * (long long)(p.N / 128) + col0 / 128] = part;
       }
       if constexpr (EPI == EPI_MX_BF16) {
         if (GK && p.tma_store) {
@@ -912,7 +955,7 @@ template <int EPI, bool SPLIT_N, bool GK = false, bool NV = false>
 int launch(const Params& p, int max_tiles, cudaStream_t stream) {
   if (max_tiles <= 0) return MOE_OK;
   auto kern = gemm_mx_kernel<EPI, SPLIT_N, GK, NV>;
-  constexpr int SMEM = smem_bytes<GK>();
+  constexpr int SMEM = smem_bytes<EPI, GK>();
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM) != cudaSuccess) {
     (void)cudaGetLastError();
     return MOE_ERR_CUDA;
