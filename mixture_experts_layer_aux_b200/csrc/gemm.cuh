@@ -85,8 +85,7 @@ struct Cfg {
   static constexpr int EPI = EPI_;
   static constexpr int GROUP = GROUP_;
   static constexpr int BMODE = BMODE_;
-  // the SwiGLU backward's staging buffers take the room of a fourth stage
-  static constexpr int kStages = (BN == 256) ? (EPI == EPI_SWIGLU_BWD ? 3 : 4) : 6;
+  static constexpr int kStages = (BN == 256) ? 4 : 6;
   static constexpr int A_BYTES = BM * BK * 2;
   static constexpr int B_BYTES = BN * BK * 2;
   static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
@@ -97,8 +96,9 @@ struct Cfg {
   static constexpr int EPI_WARPS = 8;
   static constexpr int NH = EPI_WARPS / 4;  // column slices per lane quadrant
   static constexpr int NUM_THREADS = 64 + 32 * EPI_WARPS;
-  // staging: per epilogue warp 32 rows x (64 + 16) bytes (x2 for the SwiGLU backward's gate and up)
-  static constexpr int STG_ROW = 80;
+  // staging: per epilogue warp 32 rows x (64 + 16) bytes; the SwiGLU backward stages 16 columns of gate and of
+  // up at a time, 32 rows x (32 + 16) bytes each, so that four TMA stages still fit
+  static constexpr int STG_ROW = (EPI == EPI_SWIGLU_BWD) ? 48 : 80;
   static constexpr int STG_BYTES = EPI_WARPS * 32 * STG_ROW * (EPI == EPI_SWIGLU_BWD ? 2 : 1);
   static constexpr int SMEM_BYTES = 1024 + kStages * STAGE_BYTES + BAR_BYTES + 2 * (MAX_G + 1) * 4 + 128 + STG_BYTES;
   static_assert(BN == 128 || BN == 256, "BN");
@@ -567,71 +567,76 @@ __global__ void __launch_bounds__(C::NUM_THREADS, 1) gemm_kernel(const __grid_co
         }
       } else if constexpr (C::EPI == EPI_SWIGLU_BWD) {
         // acc = v = W_d^T dO for columns [n0, n0 + BN) of F; this warp takes the slice
-        // [n0 + h W, n0 + (h + 1) W). Per 32 columns: the saved gate/up of the warp's 32 rows
-        // are loaded row-contiguously into shared memory, each lane computes its row, and
-        // dgate/dup leave the same way. dg partial sums: one per row and W-wide slice.
+        // [n0 + h W, n0 + (h + 1) W). Per 16 columns: the saved gate/up of the warp's 32 rows
+        // are loaded row-contiguously into shared memory (2 lanes x 16 bytes per row), each lane
+        // computes its row, and dgate/dup leave the same way. dg partial sums: one per row and
+        // W-wide slice.
         constexpr int W = C::BN / C::NH;
         const float g = valid ? p.row_gate[orow] : 0.f;
         const long long ld2 = 2LL * p.F;
         uint8_t* sG = stg;
         uint8_t* sU = stg + 32 * C::STG_ROW;
         __nv_bfloat16* dgu = reinterpret_cast<__nv_bfloat16*>(p.C);
+        const int sp = lane & 1, sr0 = lane >> 1;
         float part = 0.f;
 #pragma unroll 1
         for (int c = h * W; c < (h + 1) * W; c += 32) {
-#pragma unroll
-          for (int i = 0; i < 4; ++i) {
-            const int r = 8 * i + st_r0;
-            uint4 zg4 = make_uint4(0, 0, 0, 0), zu4 = make_uint4(0, 0, 0, 0);
-            if (q * 32 + r < ti.m_valid) {
-              const __nv_bfloat16* src = p.gateup + ((long long)ti.row0 + q * 32 + r) * ld2 + ti.n0 + c + 8 * st_piece;
-              zg4 = *reinterpret_cast<const uint4*>(src);
-              zu4 = *reinterpret_cast<const uint4*>(src + p.F);
-            }
-            *reinterpret_cast<uint4*>(sG + r * C::STG_ROW + 16 * st_piece) = zg4;
-            *reinterpret_cast<uint4*>(sU + r * C::STG_ROW + 16 * st_piece) = zu4;
-          }
           float v[32];
           tmem_ld32(tb + c, v);
           tmem_ld_wait();
-          __syncwarp();
 #pragma unroll
-          for (int j = 0; j < 4; ++j) {
-            float zg[8], zu[8];
-            unpack_bf16x8(*reinterpret_cast<const uint4*>(sG + lane * C::STG_ROW + 16 * j), zg);
-            unpack_bf16x8(*reinterpret_cast<const uint4*>(sU + lane * C::STG_ROW + 16 * j), zu);
-            uint32_t pg[4], pu[4];
+          for (int hf = 0; hf < 2; ++hf) {
+            const int cc = c + 16 * hf;
 #pragma unroll
-            for (int i = 0; i < 8; i += 2) {
-              float dgv[2], duv[2];
-#pragma unroll
-              for (int hh = 0; hh < 2; ++hh) {
-                const float z = zg[i + hh], u = zu[i + hh], vv = v[8 * j + i + hh];
-                const float sg = sigmoid_f(z);
-                const float sl = z * sg;
-                part += vv * sl * u;
-                const float da = g * vv;
-                dgv[hh] = da * u * sg * (1.f + z * (1.f - sg));
-                duv[hh] = da * sl;
+            for (int i = 0; i < 2; ++i) {
+              const int r = 16 * i + sr0;
+              uint4 zg4 = make_uint4(0, 0, 0, 0), zu4 = make_uint4(0, 0, 0, 0);
+              if (q * 32 + r < ti.m_valid) {
+                const __nv_bfloat16* src = p.gateup + ((long long)ti.row0 + q * 32 + r) * ld2 + ti.n0 + cc + 8 * sp;
+                zg4 = *reinterpret_cast<const uint4*>(src);
+                zu4 = *reinterpret_cast<const uint4*>(src + p.F);
               }
-              pg[i / 2] = pack_bf16x2(dgv[0], dgv[1]);
-              pu[i / 2] = pack_bf16x2(duv[0], duv[1]);
+              *reinterpret_cast<uint4*>(sG + r * C::STG_ROW + 16 * sp) = zg4;
+              *reinterpret_cast<uint4*>(sU + r * C::STG_ROW + 16 * sp) = zu4;
             }
-            *reinterpret_cast<uint4*>(sG + lane * C::STG_ROW + 16 * j) = make_uint4(pg[0], pg[1], pg[2], pg[3]);
-            *reinterpret_cast<uint4*>(sU + lane * C::STG_ROW + 16 * j) = make_uint4(pu[0], pu[1], pu[2], pu[3]);
-          }
-          __syncwarp();
+            __syncwarp();
 #pragma unroll
-          for (int i = 0; i < 4; ++i) {
-            const int r = 8 * i + st_r0;
-            if (q * 32 + r < ti.m_valid) {
-              __nv_bfloat16* dst = dgu + ((long long)ti.row0 + q * 32 + r) * ld2 + ti.n0 + c + 8 * st_piece;
-              *reinterpret_cast<uint4*>(dst) = *reinterpret_cast<const uint4*>(sG + r * C::STG_ROW + 16 * st_piece);
-              *reinterpret_cast<uint4*>(dst + p.F) =
-                  *reinterpret_cast<const uint4*>(sU + r * C::STG_ROW + 16 * st_piece);
+            for (int jj = 0; jj < 2; ++jj) {
+              float zg[8], zu[8];
+              unpack_bf16x8(*reinterpret_cast<const uint4*>(sG + lane * C::STG_ROW + 16 * jj), zg);
+              unpack_bf16x8(*reinterpret_cast<const uint4*>(sU + lane * C::STG_ROW + 16 * jj), zu);
+              uint32_t pg[4], pu[4];
+#pragma unroll
+              for (int i = 0; i < 8; i += 2) {
+                float dgv[2], duv[2];
+#pragma unroll
+                for (int hh = 0; hh < 2; ++hh) {
+                  const float z = zg[i + hh], u = zu[i + hh], vv = v[16 * hf + 8 * jj + i + hh];
+                  const float sg = sigmoid_f(z);
+                  const float sl = z * sg;
+                  part += vv * sl * u;
+                  const float da = g * vv;
+                  dgv[hh] = da * u * sg * (1.f + z * (1.f - sg));
+                  duv[hh] = da * sl;
+                }
+                pg[i / 2] = pack_bf16x2(dgv[0], dgv[1]);
+                pu[i / 2] = pack_bf16x2(duv[0], duv[1]);
+              }
+              *reinterpret_cast<uint4*>(sG + lane * C::STG_ROW + 16 * jj) = make_uint4(pg[0], pg[1], pg[2], pg[3]);
+              *reinterpret_cast<uint4*>(sU + lane * C::STG_ROW + 16 * jj) = make_uint4(pu[0], pu[1], pu[2], pu[3]);
             }
+            __syncwarp();
+#pragma unroll
+            for (int i = 0; i < 2; ++i) {
+              const int r = 16 * i + sr0;
+              if (q * 32 + r < ti.m_valid) {
+                __nv_bfloat16* dst = dgu + ((long long)ti.row0 + q * 32 + r) * ld2 + ti.n0 + cc + 8 * sp;
+                *reinterpret_cast<uint4*>(dst) = *reinterpret_cast<const uint4*>(sG + r * C::STG_ROW + 16 * sp);
+                *reinterpret_cast<uint4*>(dst + p.F) = *reinterpret_cast<const uint4*>(sU + r * C::STG_ROW + 16 * sp);
+              }
+            }
+            __syncwarp();
           }
-          __syncwarp();
         }
         if (valid) p.dg_part[orow * (long long)(p.N / W) + (ti.n0 + h * W) / W] = part;
       }
