@@ -13,18 +13,24 @@
 //   from the natural [rows, K/32] layout; word = the 4 UE8M0 bytes of one
 //   k-block, byte j = 32-wide block j) and stores them into the order that
 //   tcgen05.cp 32x128b.warpx4 expects, one 512-byte chunk per 128 rows and
-//   k-block: the 16 bytes of lane l hold rows l, l+32, l+64, l+96. The loader
-//   fences the generic-proxy stores for the async proxy before it arrives on
-//   the batch's barrier, so the MMA thread does no fence of its own.
-// MMA: per k-block, tcgen05.cp copies its chunks from the batch into one of
-// two TMEM scale slots (SFA 4 columns, SFB 8 columns; alternating by k-block)
-// right before four M128 N256 K32 MMAs that select scale byte j through the
-// instruction descriptor; after a batch's last k-block a commit frees its
-// shared memory.
+//   k-block: the 16 bytes of lane l hold rows l, l+32, l+64, l+96. The next
+//   batch's loads are issued before the loader waits for the current batch's
+//   buffer. The loader fences the generic-proxy stores for the async proxy
+//   before it arrives on the batch's barrier, so the MMA thread does no fence
+//   of its own.
+// MMA (one thread): per k-block, tcgen05.cp copies its chunks from the batch
+// into one of two TMEM scale slots (SFA 4 columns, SFB 8 columns; alternating
+// by k-block) right before four M128 N256 K32 MMAs that select scale byte j
+// through the instruction descriptor; after a batch's last k-block a commit
+// frees its shared memory.
 // TMEM: one 256-column fp32 accumulator and the two scale slots; eight
 // epilogue warps (two per lane quadrant, 128 columns each) first copy their
 // accumulator columns into registers and release TMEM, so the next tile's MMAs
-// run while they finish the element-wise work.
+// run while they finish the element-wise work. The bf16 output of the
+// grouped-along-K weight gradients leaves through TMA stores (four 1 KB
+// staging buffers per warp); the SwiGLU backward stages its saved gate/up and
+// dgate/dup through shared memory, 64 contiguous bytes per row. Those two
+// instantiations have three TMA stages, the others four.
 // Roles: warp 0 TMA producer, warp 1 MMA issuer (+ TMEM owner), warp 2 scale
 // loader, warps 3..10 epilogue. All waits are bounded like gemm.cuh.
 //
