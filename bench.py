@@ -56,9 +56,44 @@ def measured_traffic(workload: str):
         return None
     h = hashlib.sha256()
     for f in meta["sources"]:
-        with open(os.path.join(ROOT, f), "rb") as fh:
-            h.update(fh.read())
+        with open(os.path.join(ROOT, f)) as fh:
+            h.update(code_tokens(fh.read()).encode())
     return meta["dram_bytes_per_launch"] if h.hexdigest() == meta["sources_sha256"] else None
+
+
+def code_tokens(src: str) -> str:
+    """C/CUDA source with its comments removed and every run of whitespace outside string and character
+    literals folded to one space: edits to comments or layout leave it unchanged, any change to the code
+    changes it."""
+    out, i, n = [], 0, len(src)
+
+    def sp():
+        if out and out[-1] != " ":
+            out.append(" ")
+
+    while i < n:
+        c = src[i]
+        if src.startswith("//", i):
+            j = src.find("\n", i)
+            i = n if j < 0 else j
+        elif src.startswith("/*", i):
+            j = src.find("*/", i + 2)
+            i = n if j < 0 else j + 2
+            sp()
+        elif c in "\"'":
+            j = i + 1
+            while j < n and src[j] != c:
+                j += 2 if src[j] == "\\" else 1
+            out.append(src[i:j + 1])
+            i = j + 1
+        elif c.isspace():
+            while i < n and src[i].isspace():
+                i += 1
+            sp()
+        else:
+            out.append(c)
+            i += 1
+    return "".join(out).strip()
 
 
 def peaks():

@@ -23,13 +23,11 @@ namespace moe_impl {
 
 using gg::Cfg;
 
-// The SM-pair kernel (256-row tiles) pays off when experts are large: it
-// halves each SM's operand traffic per FLOP but pads each expert to a
-// multiple of 256 rows. Used when the average rows per group reach this
-// threshold (MOE_B200_PAIR_MIN_ROWS overrides it; a huge value disables it).
-// The SM-pair kernel is opt-in: MOE_B200_PAIR_MIN_ROWS=n selects it for GEMMs whose experts
-// average at least n rows. On B200 it matches the one-SM kernel on aligned experts and loses on
-// ragged ones (its 256-row tiles waste more rows at each expert's end).
+// The SM-pair kernel (256-row tiles over two SMs) halves each SM's operand
+// traffic per FLOP but pads each expert to a multiple of 256 rows. It is
+// opt-in: MOE_B200_PAIR_MIN_ROWS=n selects it for GEMMs whose experts average
+// at least n rows. On B200 it matches the one-SM kernel on aligned experts and
+// loses on ragged ones (its 256-row tiles waste more rows at each expert's end).
 static bool use_pair_kernel(int rows, int groups) {
   long long thr = 1LL << 40;
   if (const char* e = std::getenv("MOE_B200_PAIR_MIN_ROWS")) thr = std::atoll(e);

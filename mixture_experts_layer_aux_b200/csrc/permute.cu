@@ -1,5 +1,5 @@
 // permute.cu -- sync-free token permutation into expert-contiguous order,
-// unpermute-sum, and MXFP8 quantisation.
+// unpermute-sum, and MXFP8 / NVFP4 quantisation of the permuted rows.
 //
 // Memory-efficient permutation (section 2.2 of the Megatron Core MoE technical
 // summary): the routing weight is not applied to the gathered rows; it travels
