@@ -237,6 +237,13 @@ def test_layer_bwd_capacity_factor_full_oracle(moe, oracle):
     check_bwd(moe, oracle, wl, seed=2, d_aux=0.3)
 
 
+def test_layer_bwd_deepseek_router_variant_full_oracle(moe, oracle):
+    """Backward through selection on sigmoid score + per-expert bias within the best expert groups."""
+    wl = Workload("bwd-dsv3-router", T=512, H=256, E=32, k=4, F=256, score="sigmoid", route_scale=2.5, aux=False,
+                  bwd=True, n_group=4, topk_group=2, sel_bias=True)
+    check_bwd(moe, oracle, wl, seed=5, d_aux=0.0)
+
+
 def test_layer_bwd_skewed_workload_sampled(moe, oracle):
     wl = WORKLOADS["skewed"]
     d = make_inputs(wl, device="cuda", seed=0, with_dy=True)

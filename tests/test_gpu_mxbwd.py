@@ -259,7 +259,8 @@ def _mx_layer(moe, oracle, wl, seed, d_aux=0.2):
     saved = moe.workspace(moe.moe_layer_saved_size(cfg))
     moe.moe_layer_fwd(cfg, d["x"], d["W_r"], d.get("logit_bias"), q["W_g"][0], q["W_u"][0], q["W_d"][0],
                       q["W_g"][1], q["W_u"][1], q["W_d"][1], None, None, None, None, None, None, y, aux, idx, None,
-                      None, None, saved, moe.workspace(moe.moe_layer_workspace_size(cfg)))
+                      None, None, saved, moe.workspace(moe.moe_layer_workspace_size(cfg)),
+                      expert_bias=d.get("expert_bias"))
     o = dict(dX=empty((T, H), torch.bfloat16), dW_r=empty((E, H), torch.bfloat16),
              dW_g=empty((E, F, H), torch.bfloat16), dW_u=empty((E, F, H), torch.bfloat16),
              dW_d=empty((E, H, F), torch.bfloat16), dlogits=empty((T, E), torch.float32))
@@ -271,7 +272,8 @@ def _mx_layer(moe, oracle, wl, seed, d_aux=0.2):
     # oracle: the MXFP8 backward recipe on the same routing
     h = {n: (v.cpu() if torch.is_tensor(v) else v) for n, v in d.items()}
     logits = oracle.router_logits(h["x"], h["W_r"], h.get("logit_bias"))
-    r = oracle.route(logits, k, wl.score, wl.norm_topk, wl.route_scale, with_aux=wl.aux and wl.score == "softmax")
+    r = oracle.route(logits, k, wl.score, wl.norm_topk, wl.route_scale, with_aux=wl.aux and wl.score == "softmax",
+                     expert_bias=h.get("expert_bias"), n_group=wl.n_group, topk_group=wl.topk_group)
     assert torch.equal(idx.cpu(), r["idx"]), "full-oracle parity needs identical routing"
     mx = {n: (q[n][0].cpu(), q[n][1].cpu()) for n in q}
     mx.update(W_dT=(wdt.cpu(), wdt_sf.cpu()), W_gT=(wgu.cpu()[:, :, :F].contiguous(), wgu_sf.cpu()[:, :, :F // 32].contiguous()),
@@ -304,3 +306,12 @@ def test_layer_bwd_mxfp8_sigmoid_router(moe, oracle):
     wl = Workload("mx-bwd-sig", T=256, H=512, E=16, k=4, F=256, dtype="mxfp8", score="sigmoid", route_scale=2.5,
                   aux=False, bwd=True)
     _mx_layer(moe, oracle, wl, seed=4, d_aux=0.0)
+
+
+def test_layer_bwd_mxfp8_deepseek_router_variant(moe, oracle):
+    """Backward through the DeepSeek-V3 router shape: selection on sigmoid score + per-expert bias
+    within the best expert groups, gates from the unbiased scores."""
+    from mixture_experts_layer_aux_b200.synthetic import Workload
+    wl = Workload("mx-bwd-dsv3-router", T=256, H=512, E=32, k=4, F=256, dtype="mxfp8", score="sigmoid",
+                  route_scale=2.5, aux=False, bwd=True, n_group=4, topk_group=2, sel_bias=True)
+    _mx_layer(moe, oracle, wl, seed=6, d_aux=0.0)

@@ -415,7 +415,8 @@ def _loss(o, t, cfg, logits=None):
     if logits is None:
         logits = o.router_logits(t["x"], t["W_r"], None, round_f32=False)
     r = o.route(logits, cfg["k"], cfg["score"], cfg["norm"], cfg["scale"], with_aux=cfg["aux_on"],
-                capacity_factor=cfg.get("cf", 0.0))
+                capacity_factor=cfg.get("cf", 0.0), expert_bias=cfg.get("expert_bias"),
+                n_group=cfg.get("n_group", 0), topk_group=cfg.get("topk_group", 0))
     y = o.moe_fwd_tokens(t["x"], t["W_g"], t["W_u"], t["W_d"], r["idx_kept"], r["gates"])
     L = (t["dY"] * y).sum().item()
     if cfg["aux_on"]:
@@ -428,12 +429,32 @@ def _loss(o, t, cfg, logits=None):
                                                         ("softmax", False, 1.0, True, 0.0),
                                                         ("softmax", True, 1.0, True, 0.75)])
 def test_backward_matches_central_finite_differences(oracle, score, norm, scale, aux_on, cf):
-    o = oracle
     t, cfg = _fd_setup(score, norm, scale, aux_on)
     cfg["cf"] = cf
-    L0, r = _loss(o, t, cfg)
+    r = _fd_check(oracle, t, cfg)
     if cf > 0:
         assert int((r["keep"] == 0).sum()) > 0                                  # the case drops pairs
+
+
+@pytest.mark.parametrize("norm,n_group,topk_group", [(True, 4, 2), (False, 4, 2), (True, 0, 0)])
+def test_backward_deepseek_router_matches_central_finite_differences(oracle, norm, n_group, topk_group):
+    """Sigmoid scores, selection on score + per-expert bias within the best groups, gates from the
+    unbiased scores: the bias and the group limit move the selection only, so the derivative at a
+    fixed selection is the sigmoid router's."""
+    t, cfg = _fd_setup("sigmoid", norm, 2.5, False, seed=5, E=8, k=3)
+    cfg.update(expert_bias=torch.tensor([0.3, -0.2, 0.0, 0.5, -0.4, 0.1, 0.25, -0.1]), n_group=n_group,
+               topk_group=topk_group)
+    r = _fd_check(oracle, t, cfg)
+    plain = oracle.route(r["logits"], 3, "sigmoid", norm, 2.5, with_aux=False)
+    assert not torch.equal(r["idx"], plain["idx"])                             # the variant changes selection
+
+
+def _fd_check(o, t, cfg):
+    """Analytic gradients of the oracle's backward against central differences of its forward loss, on
+    inputs and weights, and on the logits themselves; entries whose perturbation changes the selection
+    are skipped. Returns the routing at the unperturbed point."""
+    score, norm, scale, aux_on = cfg["score"], cfg["norm"], cfg["scale"], cfg["aux_on"]
+    L0, r = _loss(o, t, cfg)
     E = t["W_r"].shape[0]
     dx, dl, dg = o.moe_bwd_tokens(t["x"], t["W_r"], t["W_g"], t["W_u"], t["W_d"], t["dY"], r, score=score,
                                   norm=norm, route_scale=scale, aux_on=aux_on, d_aux=cfg["d_aux"])
@@ -473,6 +494,7 @@ def test_backward_matches_central_finite_differences(oracle, score, norm, scale,
                 continue
             fd = (Lp - Lm) / (2 * h)
             assert abs(fd - dl[tt, e].item()) <= 1e-6 * max(1.0, abs(fd)), (tt, e, fd, dl[tt, e].item())
+    return r
 
 
 def test_zero_token_expert_gets_exact_zero_weight_grads(oracle):
