@@ -75,140 +75,200 @@ struct QtArgs {
   uint8_t* sf;               // [C, ldd / 32] (WEIGHT: [B, C, ldd / 32]) ue8m0
 };
 
+// 16 bytes global -> shared through L2 (cp.async.cg); with full == false nothing is read and the 16 bytes are
+// zero-filled
+__device__ __forceinline__ void cp_async16(void* sdst, const void* gsrc, bool full) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;\n" ::"r"(smem_u32(sdst)), "l"(gsrc),
+               "r"(full ? 16 : 0)
+               : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;\n" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait() {
+  asm volatile("cp.async.wait_group %0;\n" ::"n"(N) : "memory");
+}
+
 // One block: TR consecutive output positions (padded rows; never two experts: segments start on 128-row
-// boundaries) x 128 columns, TR = 128 when the source is bf16 (staged as bf16: exact) and 64 for the
-// gate-folded activation, which is computed and staged in fp32. Each thread then quantises TR/64 consecutive
-// 1x32 blocks of one column (the output's K) and stores their codes as one run of 32 or 64 bytes. One
-// thread finds the tile's expert by a binary search of the padded offsets.
+// boundaries) x up to QT_NCT tiles of 128 columns; TR = 128, or 64 for the gate-folded activation, whose gate
+// and up tiles are both staged. The block finds its expert once (every thread tests the padded segments of its
+// experts: one round of independent loads) and its source rows once. The column tiles are staged as bf16
+// through two shared-memory buffers by asynchronous copies, the next tile's copies in flight while the current
+// one is quantised: each thread quantises TR/64 consecutive 1x32 blocks of one column (the output's K) and
+// stores their codes as one run of 32 or 64 bytes.
 constexpr int QT_COLS = 128;
-constexpr int QT_ROWS = 64;    // fp32-staged tiles (MODE_AP)
-constexpr int QT_ROWS_BF = 128;  // bf16-staged tiles
+constexpr int QT_NCT = 4;              // column tiles per block
+constexpr int QT_ROWS = 64;            // MODE_AP tiles (gate and up staged)
+constexpr int QT_ROWS_BF = 128;        // other tiles
+constexpr int QT_LDS = QT_COLS + 8;    // staged row stride (bf16 elements): 16-byte aligned row starts
 __host__ __device__ constexpr int qt_rows(int mode) { return mode == 2 ? QT_ROWS : QT_ROWS_BF; }
+__host__ __device__ constexpr int qt_nsrc(int mode) { return mode == 2 ? 2 : 1; }
+// dynamic shared memory: two buffers of qt_nsrc staged bf16 tiles [TR][QT_LDS], then TR fp32 row gates
+__host__ __device__ constexpr int qt_smem(int mode) {
+  return 2 * qt_nsrc(mode) * qt_rows(mode) * QT_LDS * 2 + qt_rows(mode) * 4;
+}
 template <int MODE>
 __global__ void __launch_bounds__(256) quant_t_kernel(const QtArgs a) {
-  constexpr bool F32 = MODE == MODE_AP;
+  constexpr bool AP = MODE == MODE_AP;
   constexpr int TR = qt_rows(MODE);
-  constexpr int PADC = F32 ? 1 : 8;  // row padding (elements): conflict-free column reads, 16-byte row starts
-  using TT = typename std::conditional<F32, float, __nv_bfloat16>::type;
-  __shared__ __align__(16) TT tile[TR][QT_COLS + PADC];
+  constexpr int NIT = TR / 16;  // 16-byte copies per thread per staged tile
+  constexpr int NSRC = qt_nsrc(MODE);
+  constexpr int TILE = TR * QT_LDS;  // elements of one staged tile
+  extern __shared__ __align__(16) uint8_t qt_dyn[];
+  __nv_bfloat16* stg = reinterpret_cast<__nv_bfloat16*>(qt_dyn);        // [2][NSRC][TR][QT_LDS]
+  float* s_rg = reinterpret_cast<float*>(qt_dyn + 2 * NSRC * TILE * 2);  // [TR] (MODE_AP)
   __shared__ int s_meta[3];  // first source row (-1: none), valid rows, rows to write
   const int tid = threadIdx.x;
   const int p0 = blockIdx.x * TR;  // first output position (padded row)
-  const int c0 = blockIdx.y * QT_COLS;
   const int b = MODE == MODE_WEIGHT ? blockIdx.z : 0;
-  if (tid == 0) {
-    int r0 = -1, nv = 0, nw = 0;
-    if constexpr (MODE == MODE_WEIGHT) {
-      r0 = p0;
-      nv = nw = min(TR, a.R - p0);  // R % 32 == 0: a multiple of 32
-    } else if (p0 < __ldg(a.poff + a.E)) {
-      int lo = 0, hi = a.E - 1;  // expert whose padded segment holds p0
-      while (lo < hi) {
-        const int mid = (lo + hi + 1) >> 1;
-        if (__ldg(a.poff + mid) <= p0) lo = mid;
-        else hi = mid - 1;
-      }
-      const int i = p0 - __ldg(a.poff + lo);
-      const int o = __ldg(a.off + lo);
-      const int cnt = __ldg(a.off + lo + 1) - o;
-      r0 = o + i;
-      nv = max(0, min(TR, cnt - i));
-      nw = TR;  // pad rows are written (zero)
+  if constexpr (MODE == MODE_WEIGHT) {
+    if (tid == 0) {
+      s_meta[0] = p0;
+      s_meta[1] = s_meta[2] = min(TR, a.R - p0);  // R % 32 == 0: a multiple of 32
     }
-    s_meta[0] = r0;
-    s_meta[1] = nv;
-    s_meta[2] = nw;
+  } else {
+    // the expert whose padded segment [poff[e], poff[e+1]) holds p0 (E <= 512: two experts per thread);
+    // segments of empty experts are empty, so at most one thread matches, none past the padded total
+    int lo[2], hi[2], o0[2], o1[2];
+#pragma unroll
+    for (int q = 0; q < 2; ++q) {
+      const int e = tid + 256 * q;
+      lo[q] = hi[q] = o0[q] = o1[q] = 0;
+      if (e < a.E) {
+        lo[q] = __ldg(a.poff + e);
+        hi[q] = __ldg(a.poff + e + 1);
+        o0[q] = __ldg(a.off + e);
+        o1[q] = __ldg(a.off + e + 1);
+      }
+    }
+    if (tid == 0) s_meta[0] = -1;
+    __syncthreads();
+#pragma unroll
+    for (int q = 0; q < 2; ++q)
+      if (lo[q] <= p0 && p0 < hi[q]) {
+        const int i = p0 - lo[q];
+        s_meta[0] = o0[q] + i;
+        s_meta[1] = max(0, min(TR, o1[q] - o0[q] - i));
+        s_meta[2] = TR;  // pad rows are written (zero)
+      }
   }
   __syncthreads();
   const int r0 = s_meta[0], nv = s_meta[1], nw = s_meta[2];
   if (r0 < 0) return;  // past the padded total (block-uniform)
-  // load: thread t -> rows t/16 + 16 i, columns 8*(t%16) .. +7 of the tile
+  // this thread's staged rows (t/16 + 16 i) and 16-byte column chunk (8 * (t % 16)); their source rows are the
+  // same for every column tile
+  const int cc = (tid & 15) * 8;
+  const __nv_bfloat16* base = a.src;
+  if constexpr (MODE == MODE_WEIGHT) base += (long long)b * a.R * a.C;
+  int srow[NIT];  // source row of each staged row (-1: none)
 #pragma unroll
-  for (int it = 0; it < TR / 16; ++it) {
-    const int rr = (tid >> 4) + 16 * it, cc = (tid & 15) * 8;
-    const bool ok = rr < nv && c0 + cc < a.C;
-    if constexpr (F32) {
-      float f[8];
-#pragma unroll
-      for (int q = 0; q < 8; ++q) f[q] = 0.f;
-      if (ok) {
-        const long long r = r0 + rr;
-        const __nv_bfloat16* gp = a.src + r * 2LL * a.C + c0 + cc;
-        float zg[8], zu[8];
-        unpack_bf16x8(*reinterpret_cast<const uint4*>(gp), zg);
-        unpack_bf16x8(*reinterpret_cast<const uint4*>(gp + a.C), zu);
-        const float g = a.row_gate[r];
-#pragma unroll
-        for (int q = 0; q < 8; ++q) f[q] = g * silu_f(zg[q]) * zu[q];
-      }
-#pragma unroll
-      for (int q = 0; q < 8; ++q) tile[rr][cc + q] = f[q];
-    } else {
-      uint4 u = make_uint4(0, 0, 0, 0);
-      if (ok) {
-        long long sr = r0 + rr;
-        if constexpr (MODE == MODE_GATHER) sr = a.src_of[sr];
-        const __nv_bfloat16* base = a.src;
-        if constexpr (MODE == MODE_WEIGHT) base += (long long)b * a.R * a.C;
-        u = *reinterpret_cast<const uint4*>(base + sr * a.C + c0 + cc);
-      }
-      *reinterpret_cast<uint4*>(&tile[rr][cc]) = u;
+  for (int it = 0; it < NIT; ++it) {
+    const int rr = (tid >> 4) + 16 * it;
+    srow[it] = -1;
+    if (rr < nv) {
+      int sr = r0 + rr;
+      if constexpr (MODE == MODE_GATHER) sr = __ldg(a.src_of + sr);
+      srow[it] = sr;
     }
   }
-  __syncthreads();
+  if constexpr (AP)
+    for (int i = tid; i < TR; i += 256) s_rg[i] = i < nv ? __ldg(a.row_gate + r0 + i) : 0.f;
   uint8_t* dst = a.dst;
   uint8_t* sf = a.sf;
   if constexpr (MODE == MODE_WEIGHT) {
     dst += (long long)b * a.C * a.ldd;
     sf += (long long)b * a.C * (a.ldd / 32);
   }
-  // quantise: thread t takes column t % 128 and the TR/2 rows of half t / 128: TR/64 blocks of 32, each with
-  // its amax by a plain loop; the codes of the half leave as one contiguous run
+  const int ntiles = (a.C + QT_COLS - 1) / QT_COLS - blockIdx.y * QT_NCT;
+  const int nct = ntiles < QT_NCT ? ntiles : QT_NCT;  // >= 1 by the grid
+  const auto stage = [&](int ct) {
+    const int c0 = (blockIdx.y * QT_NCT + ct) * QT_COLS;
+    const bool cok = c0 + cc < a.C;
+    __nv_bfloat16* buf = stg + (ct & 1) * NSRC * TILE;
+#pragma unroll
+    for (int it = 0; it < NIT; ++it) {
+      const int rr = (tid >> 4) + 16 * it;
+      const bool ok = srow[it] >= 0 && cok;
+      const __nv_bfloat16* g = ok ? base + (long long)srow[it] * NSRC * a.C + c0 + cc : a.src;
+      cp_async16(buf + rr * QT_LDS + cc, g, ok);
+      if constexpr (AP) cp_async16(buf + TILE + rr * QT_LDS + cc, ok ? g + a.C : a.src, ok);
+    }
+    cp_async_commit();
+  };
   const int c = tid % QT_COLS, hb = tid / QT_COLS;
-  constexpr int NB = TR / 64;  // 32-row blocks per thread
-  if (c0 + c >= a.C) return;
-  uint32_t w[NB][8];
-  uint8_t sbv[NB];
-#pragma unroll
-  for (int bb = 0; bb < NB; ++bb) {
-    const int rb = (TR / 2) * hb + 32 * bb;  // first tile row of the block
-    float v[32];
-    float am = 0.f;
-#pragma unroll
-    for (int i = 0; i < 32; ++i) {
-      if constexpr (F32) v[i] = tile[rb + i][c];
-      else v[i] = __bfloat162float(tile[rb + i][c]);
-      am = fmaxf(am, fabsf(v[i]));
-    }
-    const uint8_t sb = mx_scale_byte(am);
-    sbv[bb] = sb;
-    const float inv = mx_inv_scale(sb);
-#pragma unroll
-    for (int q = 0; q < 8; ++q) {
-      const __nv_fp8x2_storage_t lo =
-          __nv_cvt_float2_to_fp8x2(make_float2(v[4 * q] * inv, v[4 * q + 1] * inv), __NV_SATFINITE, __NV_E4M3);
-      const __nv_fp8x2_storage_t hi =
-          __nv_cvt_float2_to_fp8x2(make_float2(v[4 * q + 2] * inv, v[4 * q + 3] * inv), __NV_SATFINITE, __NV_E4M3);
-      w[bb][q] = (uint32_t)lo | ((uint32_t)hi << 16);
-    }
-  }
-  const int pbase = p0 + (TR / 2) * hb;
-  uint4* d4 = reinterpret_cast<uint4*>(dst + (long long)(c0 + c) * a.ldd + pbase);
-#pragma unroll
-  for (int bb = 0; bb < NB; ++bb) {
-    if ((TR / 2) * hb + 32 * bb >= nw) break;  // rows past a weight matrix's end (R % 32 == 0)
-    d4[2 * bb] = make_uint4(w[bb][0], w[bb][1], w[bb][2], w[bb][3]);
-    d4[2 * bb + 1] = make_uint4(w[bb][4], w[bb][5], w[bb][6], w[bb][7]);
-    const int p = pbase + 32 * bb;
-    if constexpr (MODE == MODE_WEIGHT) {
-      sf[(long long)(c0 + c) * (a.ldd / 32) + p / 32] = sbv[bb];  // natural [C, ldd/32]
+  stage(0);
+  for (int ct = 0; ct < nct; ++ct) {
+    if (ct + 1 < nct) {
+      stage(ct + 1);  // into the buffer read two tiles ago (released by the barrier that ended that tile)
+      cp_async_wait<1>();
     } else {
-      // tiled for the weight-gradient GEMM: chunk (row block, k-block of 128), then the UTCCP order
-      const int r = c0 + c, kb32 = p / 32;
-      sf[((long long)(r / 128) * (a.ldd / 128) + kb32 / 4) * 512 + (r % 32) * 16 + ((r % 128) / 32) * 4 + kb32 % 4] =
-          sbv[bb];
+      cp_async_wait<0>();
     }
+    __syncthreads();  // tile ct is staged by every thread (and the row gates are in place)
+    const int c0 = (blockIdx.y * QT_NCT + ct) * QT_COLS;
+    const __nv_bfloat16* buf = stg + (ct & 1) * NSRC * TILE;
+    // quantise: thread t takes column t % 128 and the TR/2 rows of half t / 128: TR/64 blocks of 32, each
+    // with its amax by a plain loop; the codes of the half leave as one contiguous run
+    constexpr int NB = TR / 64;  // 32-row blocks per thread
+    if (c0 + c < a.C) {
+      uint32_t w[NB][8];
+      uint8_t sbv[NB];
+#pragma unroll
+      for (int bb = 0; bb < NB; ++bb) {
+        const int rb = (TR / 2) * hb + 32 * bb;  // first tile row of the block
+        float v[32];
+        float am = 0.f;
+#pragma unroll
+        for (int i = 0; i < 32; ++i) {
+          const float x0 = __bfloat162float(buf[(rb + i) * QT_LDS + c]);
+          if constexpr (AP) v[i] = s_rg[rb + i] * silu_f(x0) * __bfloat162float(buf[TILE + (rb + i) * QT_LDS + c]);
+          else v[i] = x0;
+          am = fmaxf(am, fabsf(v[i]));
+        }
+        const uint8_t sb = mx_scale_byte(am);
+        sbv[bb] = sb;
+        const float inv = mx_inv_scale(sb);
+#pragma unroll
+        for (int q = 0; q < 8; ++q) {
+          const __nv_fp8x2_storage_t lo = __nv_cvt_float2_to_fp8x2(make_float2(v[4 * q] * inv, v[4 * q + 1] * inv),
+                                                                   __NV_SATFINITE, __NV_E4M3);
+          const __nv_fp8x2_storage_t hi = __nv_cvt_float2_to_fp8x2(
+              make_float2(v[4 * q + 2] * inv, v[4 * q + 3] * inv), __NV_SATFINITE, __NV_E4M3);
+          w[bb][q] = (uint32_t)lo | ((uint32_t)hi << 16);
+        }
+      }
+      const int pbase = p0 + (TR / 2) * hb;
+      uint4* d4 = reinterpret_cast<uint4*>(dst + (long long)(c0 + c) * a.ldd + pbase);
+#pragma unroll
+      for (int bb = 0; bb < NB; ++bb) {
+        if ((TR / 2) * hb + 32 * bb >= nw) break;  // rows past a weight matrix's end (R % 32 == 0)
+        d4[2 * bb] = make_uint4(w[bb][0], w[bb][1], w[bb][2], w[bb][3]);
+        d4[2 * bb + 1] = make_uint4(w[bb][4], w[bb][5], w[bb][6], w[bb][7]);
+        const int p = pbase + 32 * bb;
+        if constexpr (MODE == MODE_WEIGHT) {
+          sf[(long long)(c0 + c) * (a.ldd / 32) + p / 32] = sbv[bb];  // natural [C, ldd/32]
+        } else {
+          // tiled for the weight-gradient GEMM: chunk (row block, k-block of 128), then the UTCCP order
+          const int r = c0 + c, kb32 = p / 32;
+          sf[((long long)(r / 128) * (a.ldd / 128) + kb32 / 4) * 512 + (r % 32) * 16 + ((r % 128) / 32) * 4 +
+             kb32 % 4] = sbv[bb];
+        }
+      }
+    }
+    __syncthreads();  // buffer ct & 1 has been read before tile ct + 2 is staged into it
   }
+}
+
+// Launch of a transposing quantiser: its staging buffers exceed the static shared-memory limit.
+template <int MODE>
+int launch_quant_t(dim3 grid, const QtArgs& a, cudaStream_t st) {
+  constexpr int SMEM = qt_smem(MODE);
+  if (cudaFuncSetAttribute(quant_t_kernel<MODE>, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM) != cudaSuccess) {
+    (void)cudaGetLastError();
+    return MOE_ERR_CUDA;
+  }
+  quant_t_kernel<MODE><<<grid, 256, SMEM, st>>>(a);
+  MOE_CHECK_LAUNCH();
+  return MOE_OK;
 }
 
 }  // namespace mxb
@@ -242,12 +302,11 @@ int quant_t_rows(int mode, const void* src, const int32_t* src_of, const float* 
   a.sf = sf;
   const long long pmax = rows + (long long)mxb::PAD * E;
   const int tr = mxb::qt_rows(mode);
-  const dim3 grid((unsigned)((pmax + tr - 1) / tr), (unsigned)((C + mxb::QT_COLS - 1) / mxb::QT_COLS));
-  if (mode == 0) mxb::quant_t_kernel<mxb::MODE_ROWS><<<grid, 256, 0, st>>>(a);
-  else if (mode == 1) mxb::quant_t_kernel<mxb::MODE_GATHER><<<grid, 256, 0, st>>>(a);
-  else mxb::quant_t_kernel<mxb::MODE_AP><<<grid, 256, 0, st>>>(a);
-  MOE_CHECK_LAUNCH();
-  return MOE_OK;
+  const dim3 grid((unsigned)((pmax + tr - 1) / tr),
+                  (unsigned)((C + mxb::QT_COLS * mxb::QT_NCT - 1) / (mxb::QT_COLS * mxb::QT_NCT)));
+  if (mode == 0) return mxb::launch_quant_t<mxb::MODE_ROWS>(grid, a, st);
+  if (mode == 1) return mxb::launch_quant_t<mxb::MODE_GATHER>(grid, a, st);
+  return mxb::launch_quant_t<mxb::MODE_AP>(grid, a, st);
 }
 
 static bool tmap_u8b(CUtensorMap* m, const void* base, uint64_t inner, uint64_t outer) {
@@ -357,10 +416,8 @@ extern "C" int moe_quantize_mxfp8_t(const void* src, int32_t batch, int32_t R, i
   a.ldd = ldd;
   a.sf = sf;
   const dim3 grid((unsigned)((R + mxb::QT_ROWS_BF - 1) / mxb::QT_ROWS_BF),
-                  (unsigned)((C + mxb::QT_COLS - 1) / mxb::QT_COLS), (unsigned)batch);
-  mxb::quant_t_kernel<mxb::MODE_WEIGHT><<<grid, 256, 0, static_cast<cudaStream_t>(stream)>>>(a);
-  MOE_CHECK_LAUNCH();
-  return MOE_OK;
+                  (unsigned)((C + mxb::QT_COLS * mxb::QT_NCT - 1) / (mxb::QT_COLS * mxb::QT_NCT)), (unsigned)batch);
+  return mxb::launch_quant_t<mxb::MODE_WEIGHT>(grid, a, static_cast<cudaStream_t>(stream));
 }
 
 extern "C" int64_t moe_mxfp8_t_padded_rows(const moe_config* cfg) {
