@@ -135,6 +135,21 @@ def test_permute_then_unpermute_is_k_times_identity(oracle):
     assert torch.equal(oracle.unpermute(o, row_of), x)
 
 
+def test_unpermute_sums_every_slot_and_the_shared_row(oracle):
+    """unpermute-sum = each token's k rows gathered by torch indexing and summed, plus the shared
+    expert's row of that token when one is given."""
+    from mixture_experts_layer_aux_b200.synthetic import random_routing
+    T, E, k, H = 30, 5, 3, 16
+    idx = random_routing(T, E, k, seed=7)
+    _, _, row_of, _ = oracle.maps(idx, E)
+    g = torch.Generator().manual_seed(8)
+    o = torch.randn(T * k, H, generator=g, dtype=torch.float64)
+    sh = torch.randn(T, H, generator=g, dtype=torch.float64)
+    gathered = o[row_of.long()].sum(1)
+    assert torch.allclose(oracle.unpermute(o, row_of), gathered, rtol=1e-14, atol=1e-14)
+    assert torch.allclose(oracle.unpermute(o, row_of, sh), gathered + sh, rtol=1e-14, atol=1e-14)
+
+
 # --------------------------------------------------------------- experts
 
 
@@ -627,6 +642,35 @@ def _mx_bwd_case(seed=31):
     mx["W_gT"] = o.mxfp8_quantize(inp["W_g"].transpose(1, 2).contiguous())
     mx["W_uT"] = o.mxfp8_quantize(inp["W_u"].transpose(1, 2).contiguous())
     return wl, inp, mx
+
+
+def test_mxfp8_forward_composes_from_quantised_operands(oracle):
+    """recipe mxfp8 = fp64 products of x rounded to MXFP8 along H, the MXFP8 weights, the gate-folded
+    activation (and the shared expert's activation) rounded to MXFP8 along F, and bf16 expert outputs
+    (torch fp64 + the pinned quantiser; a missing rounding point fails it)."""
+    wl = small(T=16, H=64, E=4, k=2, F=64, S=1)
+    inp = make_inputs(wl, seed=45)
+    r = oracle.route(oracle.router_logits(inp["x"], inp["W_r"]), wl.k, "softmax", True, 1.0)
+    names = ("W_g", "W_u", "W_d", "W_gs", "W_us", "W_ds")
+    mx = {n: oracle.mxfp8_quantize(inp[n]) for n in names}
+    y = oracle.moe_fwd_tokens(inp["x"], mx["W_g"][0], mx["W_u"][0], mx["W_d"][0], r["idx"], r["gates"],
+                              recipe="mxfp8", sf_g=mx["W_g"][1], sf_u=mx["W_u"][1], sf_d=mx["W_d"][1],
+                              shared=(mx["W_gs"][0], mx["W_us"][0], mx["W_ds"][0], mx["W_gs"][1], mx["W_us"][1],
+                                      mx["W_ds"][1]))
+    dec = {n: oracle.mxfp8_decode(*mx[n]) for n in names}
+    xq = _mxq(inp["x"].double())
+    silu = torch.nn.functional.silu
+    bf = lambda t: t.float().bfloat16().double()  # noqa: E731
+    ref = torch.zeros(wl.T, wl.H, dtype=torch.float64)
+    for t in range(wl.T):
+        for j in range(wl.k):
+            e = int(r["idx"][t, j])
+            zg, zu = dec["W_g"][e] @ xq[t], dec["W_u"][e] @ xq[t]
+            ap = _mxq(((silu(zg) * zu) * float(r["gates"][t, j])).unsqueeze(0))[0]
+            ref[t] += bf(dec["W_d"][e] @ ap)
+        zg, zu = dec["W_gs"] @ xq[t], dec["W_us"] @ xq[t]
+        ref[t] += bf(dec["W_ds"] @ _mxq((silu(zg) * zu).unsqueeze(0))[0])
+    assert torch.allclose(y, ref, rtol=1e-9, atol=1e-12)
 
 
 def test_mxfp8_backward_composes_from_quantised_operands(oracle):

@@ -5,6 +5,9 @@ index, another rounding rule, a swapped operand. For each, a temporary copy of t
 change is compiled and tests/test_oracle.py is run against it in a separate process; the run must end with
 at least one failed pin. An unchanged copy run the same way must pass, so a broken harness cannot pass
 these tests. Nothing here touches the CUDA path or the oracle in the tree.
+
+Equivalent mutants (no entry point can observe them) are left out: e.g. reading every row of an NVFP4
+weight with its first matrix's G, since the oracle reads expert weights only through per-expert slices.
 """
 import concurrent.futures as cf
 import os
@@ -62,6 +65,39 @@ MUTANTS = [
     ("aux_backward_drops_mean", "dl[e] += d_aux * ss[e] * (ce - sc);", "dl[e] += d_aux * ss[e] * ce;"),
     ("wd_grad_drops_gate", "for (int f = 0; f < F; ++f) a[f] *= gl[i];", "for (int f = 0; f < F; ++f) a[f] *= 1.0;"),
     ("dz_grad_drops_gate", "                double da = gl[i] * v[f];", "                double da = v[f];"),
+    ("dwg_uses_dzu", "gG[(long)f * H + h] += cg * xv[h];", "gG[(long)f * H + h] += cu * xv[h];"),
+    ("dx_drops_up_path", "                matvec_t_acc(&we_u, dzu, dxp, rowbuf);\n", ""),
+    ("dx_drops_router_path", "            for (int h = 0; h < H; ++h) dxp[h] += c * rowbuf[h];",
+     "            for (int h = 0; h < H; ++h) dxp[h] += 0.0 * c * rowbuf[h];"),
+    ("router_dwr_transposed", "double c = dl[(long)t * E + e];", "double c = dl[(long)e * T + t];"),
+    ("router_dwr_unrounded_dl", "if (round_dl) c = oc_bf16_round(c);", "if (0) c = oc_bf16_round(c);"),
+    # precision recipes and block-scaled matrices
+    ("mx_recipe_skips_x", "        if (recipe == OC_MX) mx_roundtrip(xv, H);\n        else if (recipe == OC_NV) nv_roundtrip(xv, H);"
+     "\n        for (int h = 0; h < H; ++h) y[h] = 0.0;",
+     "        if (0) mx_roundtrip(xv, H);\n        else if (recipe == OC_NV) nv_roundtrip(xv, H);"
+     "\n        for (int h = 0; h < H; ++h) y[h] = 0.0;"),
+    ("bf16_recipe_skips_act", "else if (recipe == OC_BF16R) round_vec(a, F, recipe);", "else if (0) round_vec(a, F, recipe);"),
+    ("mx_roundtrip_scale_off", "        uint8_t sb = oc_mx_scale_byte(amax);\n        double X = ldexp(1.0, (int)sb - 127);"
+     "\n        for (int i = 0; i < 32; ++i)",
+     "        uint8_t sb = oc_mx_scale_byte(amax);\n        double X = ldexp(1.0, (int)sb - 126);"
+     "\n        for (int i = 0; i < 32; ++i)"),
+    ("mx_strided_ignores_stride", "t[i] = (float)v[(b0 + i) * stride];", "t[i] = (float)v[b0 + i];"),
+    ("nv_roundtrip_drops_scale", "for (int i = 0; i < 16; ++i) v[b * 16 + i] = oc_e2m1_decode(c[i]) * sd;",
+     "for (int i = 0; i < 16; ++i) v[b * 16 + i] = oc_e2m1_decode(c[i]);"),
+    ("nvfp4_matrix_multiplies_G", "out[c] = oc_e2m1_decode(code) * oc_e4m3_decode(s[c / 16]) / G;",
+     "out[c] = oc_e2m1_decode(code) * oc_e4m3_decode(s[c / 16]) * G;"),
+    ("nvfp4_slice_keeps_first_G", "if (m->gs) s.gs = m->gs + r0 / m->gs_rows;", "if (m->gs) s.gs = m->gs;"),
+    ("nvfp4_pack_nibbles_swapped", "(uint8_t)(c[2 * i] | (c[2 * i + 1] << 4))", "(uint8_t)(c[2 * i + 1] | (c[2 * i] << 4))",
+     True),
+    ("nvfp4_read_nibbles_swapped", "uint8_t code = (p[c / 2] >> (4 * (c & 1))) & 15;",
+     "uint8_t code = (p[c / 2] >> (4 * (1 - (c & 1)))) & 15;"),
+    # forward output
+    ("shared_expert_dropped", "            for (int h = 0; h < H; ++h) y[h] += o[h];\n            if (shared_out)",
+     "            for (int h = 0; h < H; ++h) y[h] += 0.0 * o[h];\n            if (shared_out)"),
+    ("unfolded_path_drops_gate", "for (int h = 0; h < H; ++h) y[h] += g * o[h];", "for (int h = 0; h < H; ++h) y[h] += o[h];"),
+    ("unpermute_drops_shared", "if (shared) s += shared[(long)t * H + h];", "if (shared) s += 0.0;"),
+    ("unpermute_first_slot_only", "for (int j = 0; j < k; ++j) s += o[(long)row_of[(long)t * k + j] * H + h];",
+     "for (int j = 0; j < 1; ++j) s += o[(long)row_of[(long)t * k + j] * H + h];"),
 ]
 
 
