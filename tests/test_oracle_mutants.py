@@ -98,6 +98,28 @@ MUTANTS = [
     ("unpermute_drops_shared", "if (shared) s += shared[(long)t * H + h];", "if (shared) s += 0.0;"),
     ("unpermute_first_slot_only", "for (int j = 0; j < k; ++j) s += o[(long)row_of[(long)t * k + j] * H + h];",
      "for (int j = 0; j < 1; ++j) s += o[(long)row_of[(long)t * k + j] * H + h];"),
+    # more number-format edges
+    ("e4m3_no_subnormal_quantum", "    if (e < -6) e = -6;                     /* subnormal range shares the 2^-9 quantum */\n",
+     ""),
+    ("e4m3_saturates_too_high", "if (val > 448.0) val = 448.0;", "if (val > 480.0) val = 480.0;"),
+    ("nvfp4_global_scale_constant", "return amax > 0.0f ? 2688.0f / amax : 1.0f;", "return amax > 0.0f ? 448.0f / amax : 1.0f;"),
+    # grouped router
+    ("group_filter_ignored", "if (!gkeep[e / G]) continue;", "if (0) continue;"),
+    ("group_second_best_not_updated", "else if (v[e] > a2) { a2 = v[e]; }", "else if (0) { a2 = v[e]; }"),
+    ("group_ties_to_higher", "if (best < 0 || gscore[g] > gscore[best]) best = g;", "if (best < 0 || gscore[g] >= gscore[best]) best = g;"),
+    # aux and backward details
+    ("aux_without_E", "    return (double)E * acc;", "    return acc;"),
+    ("bwd_gates_unnormalised", "            if (norm) gj /= Z;\n            g[j] = gj * route_scale;",
+     "            g[j] = gj * route_scale;"),
+    ("bwd_dropped_pair_contributes", "dg[j] = 0.0; /* dropped at capacity: the output does not depend on its gate */\n"
+     "                continue;", "dg[j] = 0.0; /* dropped at capacity: the output does not depend on its gate */"),
+    ("sigmoid_unnormalised_drops_slope", "dl[e] += route_scale * dg[j] * sj * (1.0 - sj);",
+     "dl[e] += route_scale * dg[j] * sj;"),
+    ("expert_dw_silu_instead_of_grad", "DZG[(long)i * F + f] = da * zu[f] * silu_grad(zg[f]);",
+     "DZG[(long)i * F + f] = da * zu[f] * silu(zg[f]);"),
+    ("mx_dgrad_reads_forward_weight", "oc_mat wt_d = oc_slice(WdT, (int64_t)e * F, F);   /* W_d^T [F, H], MXFP8 along H */\n"
+     "                matvec(&wt_d, dye, v, rowbuf);",
+     "for (int f = 0; f < F; ++f) v[f] = 0.0;\n                matvec_t_acc(&we_d, dye, v, rowbuf);"),
 ]
 
 
@@ -112,7 +134,7 @@ def _run_pins(workdir: str, source: str):
         shutil.copy(os.path.join(ROOT, "tests", name), os.path.join(workdir, "tests"))
     shutil.copytree(os.path.join(ROOT, "tests", "golden"), os.path.join(workdir, "tests", "golden"))
     # the scratch tree's oracle first; the synthetic-input module from the repository
-    env = dict(os.environ, PYTHONPATH=workdir + os.pathsep + ROOT, OMP_NUM_THREADS="2")
+    env = dict(os.environ, PYTHONPATH=workdir + os.pathsep + ROOT, OMP_NUM_THREADS="1")
     r = subprocess.run([sys.executable, "-m", "pytest", "-x", "-q", "-p", "no:cacheprovider", "tests/test_oracle.py"],
                        cwd=workdir, env=env, capture_output=True, text=True, timeout=900)
     return r.returncode, r.stdout[-3000:] + r.stderr[-2000:]
@@ -131,7 +153,7 @@ def outcomes():
         jobs[name] = src.replace(old, new)
     tmp = tempfile.mkdtemp(prefix="oracle_mutants_")
     try:
-        with cf.ThreadPoolExecutor(max_workers=max(1, min(8, (os.cpu_count() or 2) // 2))) as ex:
+        with cf.ThreadPoolExecutor(max_workers=max(1, min(16, os.cpu_count() or 1))) as ex:
             futs = {name: ex.submit(_run_pins, os.path.join(tmp, f"m{i}"), s) for i, (name, s) in enumerate(jobs.items())}
             yield {name: fu.result() for name, fu in futs.items()}
     finally:
