@@ -186,3 +186,80 @@ def test_nvfp4_argument_errors(lib, B):
     c2 = cfg(B, H=512, F=512, expert_dtype=B.MOE_DT_NVFP4)
     assert g(ctypes.byref(c2), 0, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, ws,
              None) == INVALID  # save_gateup is not supported
+
+
+def test_backward_argument_errors(lib, B):
+    # BF16 grouped backward GEMMs
+    c = cfg(B)
+    gb = lib.moe_grouped_gemm_bwd
+    wsb = lib.moe_grouped_gemm_bwd_workspace_size(ctypes.byref(c), 1)
+    assert gb(ctypes.byref(cfg(B, expert_dtype=1)), 1, FAKE, FAKE, FAKE, FAKE, FAKE, None, FAKE, FAKE, FAKE, None,
+              None, FAKE, wsb, None) == UNSUPPORTED
+    assert gb(ctypes.byref(c), 1, None, FAKE, FAKE, FAKE, FAKE, None, FAKE, FAKE, FAKE, None, None, FAKE, wsb,
+              None) == INVALID                                                      # dO missing
+    assert gb(ctypes.byref(c), 1, FAKE, FAKE, FAKE, FAKE, None, None, FAKE, FAKE, FAKE, None, None, FAKE, wsb,
+              None) == INVALID                                                      # dgrad without W_d
+    assert gb(ctypes.byref(c), 1, FAKE, FAKE, FAKE, FAKE, FAKE, None, FAKE, FAKE, FAKE, None, None, FAKE, wsb - 1,
+              None) == WS
+    assert gb(ctypes.byref(c), 7, FAKE, FAKE, FAKE, FAKE, FAKE, None, FAKE, FAKE, FAKE, None, None, FAKE, wsb,
+              None) == INVALID                                                      # no such GEMM
+    # MXFP8 transposed quantisers
+    qt = lib.moe_quantize_mxfp8_t
+    assert qt(None, 1, 64, 64, FAKE, 64, FAKE, None) == INVALID
+    assert qt(FAKE, 0, 64, 64, FAKE, 64, FAKE, None) == INVALID
+    assert qt(FAKE, 1, 48, 64, FAKE, 64, FAKE, None) == UNSUPPORTED                # R % 32 != 0
+    assert qt(FAKE, 1, 64, 12, FAKE, 64, FAKE, None) == UNSUPPORTED                # C % 8 != 0
+    assert qt(FAKE, 1, 64, 64, FAKE, 32, FAKE, None) == UNSUPPORTED                # ldd < R
+    assert qt(FAKE, 1, 64, 64, FAKE, 80, FAKE, None) == UNSUPPORTED                # ldd % 32 != 0
+    assert qt(FAKE + 8, 1, 64, 64, FAKE, 64, FAKE, None) == ALIGN
+    cm = cfg(B, expert_dtype=1)
+    ldp = lib.moe_mxfp8_t_padded_rows(ctypes.byref(cm))
+    T, k, E = 512, 2, 8
+    assert ldp == -(-(T * k + 128 * E) // 512) * 512                                # each expert padded to 128 rows
+    assert lib.moe_mxfp8_t_padded_rows(ctypes.byref(cfg(B, k=0))) == 0
+    qg = lib.moe_quantize_mxfp8_t_grouped
+    assert qg(ctypes.byref(cm), 3, FAKE, FAKE, FAKE, FAKE, FAKE, 256, FAKE, ldp, FAKE, None) == INVALID   # mode
+    assert qg(ctypes.byref(cm), 1, FAKE, None, None, FAKE, FAKE, 256, FAKE, ldp, FAKE, None) == INVALID   # no src_of
+    assert qg(ctypes.byref(cm), 2, FAKE, None, None, FAKE, FAKE, 256, FAKE, ldp, FAKE, None) == INVALID   # no gate
+    assert qg(ctypes.byref(cm), 0, FAKE, None, None, FAKE, FAKE, 96, FAKE, ldp, FAKE, None) == UNSUPPORTED
+    assert qg(ctypes.byref(cm), 0, FAKE, None, None, FAKE, FAKE, 256, FAKE, ldp - 512, FAKE, None) == INVALID
+    assert qg(ctypes.byref(cm), 0, FAKE, None, None, FAKE, FAKE, 256, FAKE, ldp + 32, FAKE, None) == INVALID
+    assert qg(ctypes.byref(cm), 0, FAKE + 4, None, None, FAKE, FAKE, 256, FAKE, ldp, FAKE, None) == ALIGN
+    # MXFP8 grouped data- and weight-gradient GEMMs
+    dg = lib.moe_grouped_gemm_dgrad_mxfp8
+    need = T * k * (512 // 128) * 4
+    assert dg(ctypes.byref(cfg(B, expert_dtype=1, F=384)), 1, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE,
+              FAKE, need, None) == UNSUPPORTED                                      # F % 256 != 0
+    assert dg(ctypes.byref(cm), 1, None, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, need, None) == INVALID
+    assert dg(ctypes.byref(cm), 1, FAKE + 8, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, need,
+              None) == ALIGN
+    assert dg(ctypes.byref(cm), 1, FAKE, FAKE, FAKE, FAKE, FAKE, None, FAKE, FAKE, FAKE, FAKE, need,
+              None) == INVALID                                                      # SwiGLU backward needs gate/up
+    assert dg(ctypes.byref(cm), 1, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, need - 4,
+              None) == WS
+    assert dg(ctypes.byref(cm), 7, FAKE, FAKE, FAKE, FAKE, FAKE, None, None, FAKE, None, None, 0, None) == INVALID
+    wg = lib.moe_grouped_gemm_wgrad_mxfp8
+    assert wg(ctypes.byref(cm), 1, None, FAKE, FAKE, FAKE, FAKE, ldp, FAKE, None, None) == INVALID
+    assert wg(ctypes.byref(cm), 1, FAKE, FAKE, FAKE, FAKE, FAKE, ldp - 512, FAKE, None, None) == INVALID
+    assert wg(ctypes.byref(cm), 1, FAKE, FAKE, FAKE, FAKE, FAKE, ldp + 32, FAKE, None, None) == INVALID
+    assert wg(ctypes.byref(cm), 0, FAKE, FAKE, FAKE, FAKE, FAKE, ldp, FAKE, None, None) == INVALID   # gate/up: dW_u
+    assert wg(ctypes.byref(cm), 7, FAKE, FAKE, FAKE, FAKE, FAKE, ldp, FAKE, FAKE, None) == INVALID
+    # MXFP8 layer backward
+    lb = lib.moe_layer_bwd_mxfp8
+    cmb = cfg(B, expert_dtype=1, save_for_bwd=1)
+    lws = lib.moe_layer_bwd_mxfp8_workspace_size(ctypes.byref(cmb))
+    assert lws > 0
+    args = [FAKE, ctypes.c_float(0.0), FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, None]
+    assert lb(ctypes.byref(cfg(B, save_for_bwd=1)), *args, FAKE, lws, None) == INVALID     # not an MXFP8 layer
+    assert lb(ctypes.byref(cfg(B, expert_dtype=1, save_for_bwd=1, n_shared=1)), *args, FAKE, lws,
+              None) == UNSUPPORTED                                                  # no shared-expert backward
+    bad = list(args)
+    bad[0] = None
+    assert lb(ctypes.byref(cmb), *bad, FAKE, lws, None) == INVALID                  # dY missing
+    bad = list(args)
+    bad[2] = FAKE + 8
+    assert lb(ctypes.byref(cmb), *bad, FAKE, lws, None) == ALIGN                    # x
+    bad = list(args)
+    bad[5] = FAKE + 2
+    assert lb(ctypes.byref(cmb), *bad, FAKE, lws, None) == ALIGN                    # W_d^T scales: 4-byte aligned
+    assert lb(ctypes.byref(cmb), *args, FAKE, lws - 1, None) == WS
