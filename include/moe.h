@@ -292,7 +292,8 @@ int moe_quantize_nvfp4_act(const void* src, int64_t rows, int32_t K, uint8_t* ds
  *   e4m3 with dst[b, c, r] the code of src[b, r, c], quantised in blocks of
  *   32 consecutive r; sf [batch, C, ldd/32]. R % 32 == 0, C % 8 == 0,
  *   ldd >= R and ldd % 32 == 0 (ldd > R leaves room to place W_g^T and W_u^T
- *   side by side in one [E, H, 2F] buffer: pass dst + F, sf + F/32).
+ *   side by side in one [E, H, 2F] buffer: pass dst + F, sf + F/32); src and
+ *   dst 16-byte aligned (MOE_ERR_ALIGNMENT).
  *   Once per weight update: W_d [E,H,F] -> W_d^T [E,F,H] (blocks along H),
  *   W_g, W_u [E,F,H] -> W_g^T | W_u^T [E,H,2F] (blocks along F).
  *
@@ -310,7 +311,8 @@ int moe_quantize_nvfp4_act(const void* src, int64_t rows, int32_t K, uint8_t* ds
  *   (src [T, C], e.g. x or dY through the permutation); 2 the gate-folded
  *   activation row_gate[r] * silu(gate) * up recomputed from the saved
  *   pre-activations src [T*k, 2C] (gate columns, then up). C % 128 == 0;
- *   ldd >= moe_mxfp8_t_padded_rows(cfg) and ldd % 512 == 0.
+ *   ldd >= moe_mxfp8_t_padded_rows(cfg) and ldd % 512 == 0; src and dst
+ *   16-byte aligned (MOE_ERR_ALIGNMENT).
  * ------------------------------------------------------------------------ */
 int moe_quantize_mxfp8_t(const void* src, int32_t batch, int32_t R, int32_t C, void* dst, int64_t ldd, uint8_t* sf,
                          void* stream);

@@ -407,7 +407,8 @@ extern "C" int moe_quantize_mxfp8_t(const void* src, int32_t batch, int32_t R, i
                                     uint8_t* sf, void* stream) {
   if (!src || !dst || !sf || batch < 1 || R < 1 || C < 1) return MOE_ERR_INVALID_ARG;
   if (R % 32 != 0 || C % 8 != 0 || ldd < R || ldd % 32 != 0) return MOE_ERR_UNSUPPORTED;
-  if ((reinterpret_cast<uintptr_t>(src) & 15u) != 0) return MOE_ERR_ALIGNMENT;
+  // 16-byte loads of src rows; 16-byte stores of code runs into dst rows
+  if (((reinterpret_cast<uintptr_t>(src) | reinterpret_cast<uintptr_t>(dst)) & 15u) != 0) return MOE_ERR_ALIGNMENT;
   mxb::QtArgs a{};
   a.src = static_cast<const __nv_bfloat16*>(src);
   a.R = R;
@@ -436,7 +437,7 @@ extern "C" int moe_quantize_mxfp8_t_grouped(const moe_config* cfg, int32_t mode,
   if (C < 1 || C % 128 != 0) return MOE_ERR_UNSUPPORTED;
   const long long rows = (long long)cfg->T * cfg->k;
   if (ldd < moe_impl::padded_rows_max(rows, cfg->E) || ldd % 512 != 0) return MOE_ERR_INVALID_ARG;
-  if ((reinterpret_cast<uintptr_t>(src) & 15u) != 0) return MOE_ERR_ALIGNMENT;
+  if (((reinterpret_cast<uintptr_t>(src) | reinterpret_cast<uintptr_t>(dst)) & 15u) != 0) return MOE_ERR_ALIGNMENT;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   rc = moe_impl::pad_offsets(offsets, cfg->E, poff, st);
   if (rc) return rc;

@@ -212,6 +212,7 @@ def test_backward_argument_errors(lib, B):
     assert qt(FAKE, 1, 64, 64, FAKE, 32, FAKE, None) == UNSUPPORTED                # ldd < R
     assert qt(FAKE, 1, 64, 64, FAKE, 80, FAKE, None) == UNSUPPORTED                # ldd % 32 != 0
     assert qt(FAKE + 8, 1, 64, 64, FAKE, 64, FAKE, None) == ALIGN
+    assert qt(FAKE, 1, 64, 64, FAKE + 8, 64, FAKE, None) == ALIGN                 # dst: 16-byte code runs
     cm = cfg(B, expert_dtype=1)
     ldp = lib.moe_mxfp8_t_padded_rows(ctypes.byref(cm))
     T, k, E = 512, 2, 8
@@ -225,6 +226,7 @@ def test_backward_argument_errors(lib, B):
     assert qg(ctypes.byref(cm), 0, FAKE, None, None, FAKE, FAKE, 256, FAKE, ldp - 512, FAKE, None) == INVALID
     assert qg(ctypes.byref(cm), 0, FAKE, None, None, FAKE, FAKE, 256, FAKE, ldp + 32, FAKE, None) == INVALID
     assert qg(ctypes.byref(cm), 0, FAKE + 4, None, None, FAKE, FAKE, 256, FAKE, ldp, FAKE, None) == ALIGN
+    assert qg(ctypes.byref(cm), 0, FAKE, None, None, FAKE, FAKE, 256, FAKE + 4, ldp, FAKE, None) == ALIGN
     # MXFP8 grouped data- and weight-gradient GEMMs
     dg = lib.moe_grouped_gemm_dgrad_mxfp8
     need = T * k * (512 // 128) * 4
