@@ -28,6 +28,7 @@ import os
 import statistics
 import subprocess
 import sys
+import tempfile
 import time
 
 import torch
@@ -180,7 +181,9 @@ class ClockSampler:
     def __init__(self, index: int):
         self.index = index
         self.proc = None
-        self.path = os.path.join(ROOT, "gpurun_out", f"clocks_rank{index}.csv")
+        # the raw samples stay on disk for inspection: MOE_BENCH_CLOCKS_DIR, else the system temp directory
+        d = os.environ.get("MOE_BENCH_CLOCKS_DIR") or os.path.join(tempfile.gettempdir(), "moe_bench_clocks")
+        self.path = os.path.join(d, f"clocks_rank{index}.csv")
 
     def __enter__(self):
         try:
