@@ -98,6 +98,13 @@ const char* moe_status_string(int status);
  * `clear` != 0 resets the word to 0 afterwards. */
 int moe_get_device_status(int32_t* word_out, int clear);
 
+/* Self-test of the failure path: enqueues one CTA whose thread waits, with the
+ * bounded wait the GEMM kernels use, on an mbarrier that nothing completes.
+ * After 2 s of %globaltimer the wait gives up, records 0x1F0 in the device
+ * status word (if it is still 0) and the kernel returns; the context stays
+ * usable. Read and clear the word with moe_get_device_status afterwards. */
+int moe_selftest_wait_timeout(void* stream);
+
 /* ------------------------------------------------------------------------
  * Router: logits, scores, top-k, gates, counts, aux.
  *   logits[t,e] = sum_h x[t,h] W_r[e,h] (+ logit_bias[e]), fp32 accumulate

@@ -47,6 +47,7 @@ _CFG = ctypes.POINTER(moe_config)
 _SIGS = {
     "moe_status_string": (ctypes.c_char_p, [_I]),
     "moe_get_device_status": (_I, [ctypes.POINTER(ctypes.c_int32), _I]),
+    "moe_selftest_wait_timeout": (_I, [_VP]),
     "moe_router_workspace_size": (_SZ, [_CFG]),
     "moe_router_topk": (_I, [_CFG, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _SZ, _VP]),
     "moe_permute_workspace_size": (_SZ, [_CFG]),
@@ -163,6 +164,10 @@ def moe_get_device_status(clear: bool = True) -> int:
     if rc not in (0, 6):
         _check("moe_get_device_status", rc)
     return int(w.value)
+
+
+def moe_selftest_wait_timeout(stream=None):
+    return _check("moe_selftest_wait_timeout", load().moe_selftest_wait_timeout(_st(stream)))
 
 
 def moe_router_workspace_size(cfg) -> int:

@@ -128,3 +128,26 @@ extern "C" int moe_get_device_status(int32_t* word_out, int clear) {
   }
   return v == 0 ? MOE_OK : MOE_ERR_DEVICE;
 }
+
+namespace {
+// One thread waits, through the bounded wait every GEMM role uses, on an mbarrier that nothing completes
+// (the phase of parity 0 of a fresh barrier); the wait gives up after MOE_WAIT_NS and records its code.
+__global__ void wait_selftest_kernel(int* status) {
+  __shared__ __align__(8) uint64_t bar;
+  __shared__ int abort_flag;
+  if (threadIdx.x == 0) {
+    abort_flag = 0;
+    mbar_init(&bar, 1);
+    fence_mbar_init();
+    (void)mbar_wait(&bar, 0, &abort_flag, status, DEV_WAIT_TIMEOUT_SELFTEST);
+  }
+}
+}  // namespace
+
+extern "C" int moe_selftest_wait_timeout(void* stream) {
+  int* p = moe_host::device_status_ptr();
+  if (!p) return MOE_ERR_CUDA;
+  wait_selftest_kernel<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>(p);
+  MOE_CHECK_LAUNCH();
+  return MOE_OK;
+}
