@@ -130,6 +130,8 @@ extern "C" int moe_get_device_status(int32_t* word_out, int clear) {
 }
 
 namespace {
+constexpr int DEV_WAIT_TIMEOUT_SELFTEST = 0x1F0;  // device status code of moe_selftest_wait_timeout
+
 // One thread waits, through the bounded wait every GEMM role uses, on an mbarrier that nothing completes
 // (the phase of parity 0 of a fresh barrier); the wait gives up after MOE_WAIT_NS and records its code.
 __global__ void wait_selftest_kernel(int* status) {

@@ -19,7 +19,6 @@ enum MoeDevStatus : int {
   DEV_WAIT_TIMEOUT_MMA = 0x102,
   DEV_WAIT_TIMEOUT_EPILOGUE = 0x103,
   DEV_WAIT_TIMEOUT_DRAIN = 0x104,
-  DEV_WAIT_TIMEOUT_SELFTEST = 0x1F0,  // moe_selftest_wait_timeout
   DEV_BAD_OFFSETS = 0x201,
   DEV_BAD_INDEX = 0x202,
 };
