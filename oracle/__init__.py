@@ -14,7 +14,9 @@ tensors into it and chains its steps in the order the pages give:
 Parity status: every oracle function is pinned by a test in
 tests/test_oracle.py against something other than itself (brute force,
 closed forms, library routines, finite differences, hand-computed OCP MX
-and NVFP4 values); none is "parity unpinned".
+and NVFP4 values); none is "parity unpinned". tests/test_oracle_mutants.py
+plants one mistake at a time in a scratch copy of moe_oracle.c and checks
+that each fails at least one of those pins.
 """
 from __future__ import annotations
 
