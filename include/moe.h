@@ -177,7 +177,10 @@ int moe_permute(const moe_config* cfg, const void* x, const int32_t* idx, const 
  *   it until the process exits. A configuration whose moe_permute workspace
  *   would exceed it is rejected with MOE_ERR_UNSUPPORTED before any launch.
  *   The first call on each device looks up the array's device address (no
- *   allocation); make that first call before any stream capture.
+ *   allocation); make that first call before any stream capture. The address
+ *   is cached for the life of the process: after cudaDeviceReset (or any reset
+ *   of the device's primary context) the cached address is stale, so do not
+ *   call this entry point again in that process after such a reset.
  *   All calls share the one array: two calls whose kernels overlap on the GPU
  *   (different streams, or different host threads, on the same device) race.
  *   Every scratch word is written before it is read within a call, so nothing

@@ -512,7 +512,10 @@ namespace {
 
 // Device address of the scratch array for the current device. The runtime only
 // knows it per device, so it is looked up once per device (with that device
-// current) and cached; the lookup allocates nothing.
+// current) and cached for the life of the process; the lookup allocates
+// nothing. A device reset (cudaDeviceReset, or a reset of the primary context)
+// makes the cached address stale; the header tells callers not to use this
+// entry point again after one.
 void* noalloc_scratch_ptr() {
   static void* ptrs[64] = {};
   static std::mutex mu;
