@@ -34,8 +34,10 @@ _lock = threading.Lock()
 _lib = None
 
 OC_BF16, OC_MXFP8, OC_F64, OC_NVFP4 = 0, 1, 2, 3
-# rounding points of the precision recipes (see moe_oracle.c)
-RECIPES = {"exact": 0, "mxfp8": 1, "bf16": 2, "nvfp4": 3}
+# rounding points of the precision recipes (see moe_oracle.c); "mxfp8-q" / "nvfp4-q" keep only the
+# block-scaled formats' quantisation points (no bf16 rounding anywhere else)
+RECIPES = {"exact": 0, "mxfp8": 1, "bf16": 2, "nvfp4": 3, "mxfp8-q": 4, "nvfp4-q": 5}
+MX_RECIPES = ("mxfp8", "mxfp8-q")
 
 
 def build(force: bool = False) -> str:
@@ -394,11 +396,12 @@ def moe_fwd_tokens(x, W_g, W_u, W_d, idx, g, toks=None, *, recipe="exact", fold=
 
     recipe: "exact" (no rounding), "bf16" (the BF16 recipe's rounding points),
     "mxfp8" (the weight tensors are MXFP8 codes and sf_* their scales) or "nvfp4"
-    (the weights are packed NVFP4 codes, sf_* = (scales, G) pairs).
+    (the weights are packed NVFP4 codes, sf_* = (scales, G) pairs); "mxfp8-q" /
+    "nvfp4-q" take the same operands but round nothing to bf16.
     shared = (W_gs, W_us, W_ds[, sf_gs, sf_us, sf_ds]) adds the always-on shared expert.
     """
     rc = _recipe(recipe)
-    mx = rc in (RECIPES["mxfp8"], RECIPES["nvfp4"])
+    mx = rc in (RECIPES["mxfp8"], RECIPES["nvfp4"], RECIPES["mxfp8-q"], RECIPES["nvfp4-q"])
     T, H = x.shape
     E, F = W_g.shape[0], W_g.shape[1]
     k = idx.shape[1]
@@ -483,9 +486,10 @@ def moe_bwd_tokens(x, W_r, W_g, W_u, W_d, dY, r: dict, toks=None, *, score="soft
 
     recipe "mxfp8" (the MXFP8 backward) takes mx = dict of (codes, scales) pairs: W_g, W_u, W_d
     (the forward's, MXFP8 along their K) and W_dT [E,F,H], W_gT, W_uT [E,H,F] (transposed, MXFP8
-    along H resp. F); W_g, W_u, W_d are then ignored."""
+    along H resp. F); W_g, W_u, W_d are then ignored. "mxfp8-q" takes the same operands and
+    rounds nothing to bf16."""
     T, H = x.shape
-    E, F = (mx["W_g"][0] if recipe == "mxfp8" else W_g).shape[:2]
+    E, F = (mx["W_g"][0] if recipe in MX_RECIPES else W_g).shape[:2]
     k = r["idx"].shape[1]
     if toks is None:
         toks = torch.arange(T, dtype=torch.int32)
@@ -495,7 +499,7 @@ def moe_bwd_tokens(x, W_r, W_g, W_u, W_d, dY, r: dict, toks=None, *, score="soft
     dl = torch.empty((n, E), dtype=torch.float64)
     dg = torch.empty((n, k), dtype=torch.float64)
     s_soft = r["probs"] if score == "softmax" else scores(r["logits"], "softmax")
-    if recipe == "mxfp8":
+    if recipe in MX_RECIPES:
         wg, wu, wd, wdt, wgt, wut = _mx_mats(mx, ["W_g", "W_u", "W_d", "W_dT", "W_gT", "W_uT"])
     else:
         wg, wu, wd = _wmat(W_g), _wmat(W_u), _wmat(W_d)
@@ -515,16 +519,16 @@ def moe_bwd_tokens(x, W_r, W_g, W_u, W_d, dY, r: dict, toks=None, *, score="soft
 def moe_bwd_expert_dw(x, W_g, W_u, W_d, dY, idx, g, experts, recipe="exact", mx=None):
     """dW_g, dW_u [n,F,H] and dW_d [n,H,F] (fp64) for the listed experts.
 
-    recipe "mxfp8" takes mx as moe_bwd_tokens does (W_g, W_u, W_d, W_dT are used)."""
+    recipe "mxfp8" / "mxfp8-q" take mx as moe_bwd_tokens does (W_g, W_u, W_d, W_dT are used)."""
     T, H = x.shape
-    E, F = (mx["W_g"][0] if recipe == "mxfp8" else W_g).shape[:2]
+    E, F = (mx["W_g"][0] if recipe in MX_RECIPES else W_g).shape[:2]
     k = idx.shape[1]
     experts = _chk(torch.as_tensor(experts, dtype=torch.int32).contiguous(), torch.int32)
     n = experts.numel()
     dWg = torch.empty((n, F, H), dtype=torch.float64)
     dWu = torch.empty((n, F, H), dtype=torch.float64)
     dWd = torch.empty((n, H, F), dtype=torch.float64)
-    if recipe == "mxfp8":
+    if recipe in MX_RECIPES:
         wg, wu, wd, wdt = _mx_mats(mx, ["W_g", "W_u", "W_d", "W_dT"])
     else:
         wg, wu, wd, wdt = _wmat(W_g), _wmat(W_u), _wmat(W_d), None

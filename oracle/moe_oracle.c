@@ -79,9 +79,18 @@ double oc_bf16_round(double v) {
  *             gate-folded activation, each expert's output; in the backward
  *             the saved pre-activations, dgate/dup, the per-row dXp and the
  *             router-gradient operand). */
-enum { OC_EXACT = 0, OC_MX = 1, OC_BF16R = 2, OC_NV = 3 };
+enum { OC_EXACT = 0, OC_MX = 1, OC_BF16R = 2, OC_NV = 3, OC_MXQ = 4, OC_NVQ = 5 };
 /*   OC_NV     NVFP4 recipe: as OC_MX with NVFP4 operands (16-blocks along K,
- *             activations with G = 1), bf16 expert GEMM outputs. */
+ *             activations with G = 1), bf16 expert GEMM outputs.
+ *   OC_MXQ, OC_NVQ  the block-scaled formats' quantisation points only: the
+ *             operands are quantised exactly as under OC_MX / OC_NV (and, in
+ *             the backward, every MXFP8 operand of OC_MX), but no value is
+ *             rounded to bf16 anywhere (not the expert outputs, the saved
+ *             pre-activations, dgate/dup, dXp nor the router-gradient
+ *             operand): fp64 everywhere else. This is the exact layer up to
+ *             the quantisation the format itself defines. */
+static int is_mx(int recipe) { return recipe == OC_MX || recipe == OC_MXQ; }
+static int is_nv(int recipe) { return recipe == OC_NV || recipe == OC_NVQ; }
 
 static void round_vec(double* v, int n, int recipe) {
     if (recipe == OC_BF16R || recipe == OC_MX || recipe == OC_NV)
@@ -645,8 +654,8 @@ static void expert_act(const oc_mat* Wg, const oc_mat* Wu, const double* xv, dou
 /* The gate-folded activation as the down projection's operand: MXFP8 blocks
  * along F (MXFP8 recipe) or bf16 (BF16 recipe). */
 static void round_act(double* a, int F, int recipe) {
-    if (recipe == OC_MX) mx_roundtrip(a, F);
-    else if (recipe == OC_NV) nv_roundtrip(a, F);
+    if (is_mx(recipe)) mx_roundtrip(a, F);
+    else if (is_nv(recipe)) nv_roundtrip(a, F);
     else if (recipe == OC_BF16R) round_vec(a, F, recipe);
 }
 
@@ -669,6 +678,8 @@ static void round_act(double* a, int F, int recipe) {
  *   OC_BF16R: g*a (and the shared a) is rounded to bf16;
  *   all three: each expert's down-projection output is rounded to bf16 before
  *     the sum. y itself is returned unrounded.
+ *   OC_MXQ / OC_NVQ: the quantisation points of OC_MX / OC_NV only (x, the
+ *     weights and the gate-folded activation); expert outputs stay unrounded.
  * Weight layouts: Wg, Wu [E*F, H]; Wd [E*H, F]; shared Wgs, Wus [F, H], Wds [H, F].
  */
 int oc_moe_fwd_tokens(int T, int H, int E, int k, int F, int S, int recipe, int fold, const oc_mat* x,
@@ -690,8 +701,8 @@ int oc_moe_fwd_tokens(int T, int H, int E, int k, int F, int S, int recipe, int 
         double* rowbuf = (double*)malloc(sizeof(double) * maxd);
         double* y = y_out + (long)i * H;
         oc_row(x, t, xv);
-        if (recipe == OC_MX) mx_roundtrip(xv, H);
-        else if (recipe == OC_NV) nv_roundtrip(xv, H);
+        if (is_mx(recipe)) mx_roundtrip(xv, H);
+        else if (is_nv(recipe)) nv_roundtrip(xv, H);
         for (int h = 0; h < H; ++h) y[h] = 0.0;
         for (int j = 0; j < k; ++j) {
             int e = idx[(long)t * k + j];
@@ -781,8 +792,8 @@ int oc_expert_rows(int H, int F, int recipe, const oc_mat* xp, const int32_t* e_
         double* a = (double*)malloc(sizeof(double) * F);
         double* rowbuf = (double*)malloc(sizeof(double) * maxd);
         oc_row(xp, r, xv);
-        if (recipe == OC_MX) mx_roundtrip(xv, H);
-        else if (recipe == OC_NV) nv_roundtrip(xv, H);
+        if (is_mx(recipe)) mx_roundtrip(xv, H);
+        else if (is_nv(recipe)) nv_roundtrip(xv, H);
         oc_mat we_g = oc_slice(Wg, (int64_t)e * F, F);
         oc_mat we_u = oc_slice(Wu, (int64_t)e * F, F);
         oc_mat we_d = oc_slice(Wd, (int64_t)e * H, H);
@@ -831,7 +842,9 @@ int oc_expert_rows(int H, int F, int recipe, const oc_mat* xp, const int32_t* e_
  * H; dz_g, dz_u are rounded to bf16 and then to MXFP8 along F, and the gate/up
  * dgrad takes WgT, WuT (W_g^T, W_u^T [E*H, F], MXFP8 along F); its result and
  * the router path are rounded as under OC_BF16R. (WdT, WgT, WuT are unused
- * otherwise and may be NULL.)
+ * otherwise and may be NULL.) OC_MXQ takes the same MXFP8 operands as OC_MX
+ * but rounds nothing to bf16 (z, dz_g, dz_u, the dXp contributions and the
+ * router path stay fp64).
  * logits, s (scores), gates, idx and counts are the forward's (counts: every
  * selected pair, as the router counted them for aux). keep: NULL, or the
  * capacity mask of oc_capacity_keep: a dropped pair contributes nothing to y,
@@ -870,7 +883,7 @@ int oc_moe_bwd_tokens(int T, int H, int E, int k, int F, int score, int norm, do
         double* dye = dy;          /* dY as the down dgrad's operand */
         double* xq = NULL;
         double* dyq = NULL;
-        if (recipe == OC_MX) {
+        if (is_mx(recipe)) {
             xq = (double*)malloc(sizeof(double) * H);
             dyq = (double*)malloc(sizeof(double) * H);
             memcpy(xq, xv, sizeof(double) * H);
@@ -905,7 +918,7 @@ int oc_moe_bwd_tokens(int T, int H, int E, int k, int F, int score, int norm, do
                 for (int f = 0; f < F; ++f) { zg[f] = oc_bf16_round(zg[f]); zu[f] = oc_bf16_round(zu[f]); }
                 for (int f = 0; f < F; ++f) a[f] = silu(zg[f]) * zu[f];
             }
-            if (recipe == OC_MX) {
+            if (is_mx(recipe)) {
                 oc_mat wt_d = oc_slice(WdT, (int64_t)e * F, F);   /* W_d^T [F, H], MXFP8 along H */
                 matvec(&wt_d, dye, v, rowbuf);                      /* v = W_d^T dY_t */
             } else {
@@ -922,7 +935,7 @@ int oc_moe_bwd_tokens(int T, int H, int E, int k, int F, int score, int norm, do
                 for (int f = 0; f < F; ++f) { dzg[f] = oc_bf16_round(dzg[f]); dzu[f] = oc_bf16_round(dzu[f]); }
             }
             for (int h = 0; h < H; ++h) dxp[h] = 0.0;
-            if (recipe == OC_MX) {
+            if (is_mx(recipe)) {
                 /* dgate/dup as the gate/up dgrad's operand: MXFP8 along F; W_g^T, W_u^T [H, F] MXFP8 along F */
                 mx_roundtrip(dzg, F);
                 mx_roundtrip(dzu, F);
@@ -1016,7 +1029,8 @@ int oc_moe_bwd_tokens(int T, int H, int E, int k, int F, int score, int norm, do
  * v = W_d^T dY uses WdT (W_d^T [E*F, H], MXFP8 along H) and dY in MXFP8 along
  * H; dz_g, dz_u are rounded to bf16; then every weight-gradient operand (g a,
  * dz_g, dz_u, x, dY) is quantised to MXFP8 along the expert's tokens, in blocks
- * of 32 consecutive tokens of its stable order.
+ * of 32 consecutive tokens of its stable order. OC_MXQ: the same quantisation
+ * with z, dz_g and dz_u unrounded.
  */
 int oc_moe_bwd_expert_dw(int T, int H, int E, int k, int F, int recipe, const oc_mat* x, const oc_mat* Wg,
                          const oc_mat* Wu, const oc_mat* Wd, const oc_mat* WdT, const oc_mat* dY, const int32_t* idx,
@@ -1062,9 +1076,9 @@ int oc_moe_bwd_expert_dw(int T, int H, int E, int k, int F, int recipe, const oc
             double* a = A + (long)i * F;
             oc_row(x, tl[i], xv);
             oc_row(dY, tl[i], dy);
-            if (recipe == OC_MX) {
+            if (is_mx(recipe)) {
                 /* the forward's gate/up GEMM saw x in MXFP8 along H; its bf16 pre-activations were
-                 * saved, and the backward recomputes g a from them */
+                 * saved (OC_MX; unrounded under OC_MXQ), and the backward recomputes g a from them */
                 double* xq = (double*)malloc(sizeof(double) * H);
                 double* dyq = (double*)malloc(sizeof(double) * H);
                 memcpy(xq, xv, sizeof(double) * H);
@@ -1072,7 +1086,8 @@ int oc_moe_bwd_expert_dw(int T, int H, int E, int k, int F, int recipe, const oc
                 mx_roundtrip(xq, H);
                 mx_roundtrip(dyq, H);
                 expert_act(&we_g, &we_u, xq, zg, zu, a, rowbuf);
-                for (int f = 0; f < F; ++f) { zg[f] = oc_bf16_round(zg[f]); zu[f] = oc_bf16_round(zu[f]); }
+                if (recipe == OC_MX)
+                    for (int f = 0; f < F; ++f) { zg[f] = oc_bf16_round(zg[f]); zu[f] = oc_bf16_round(zu[f]); }
                 for (int f = 0; f < F; ++f) a[f] = gl[i] * silu(zg[f]) * zu[f];
                 oc_mat wt_d = oc_slice(WdT, (int64_t)e * F, F);
                 matvec(&wt_d, dyq, v, rowbuf);                      /* v = W_d^T dY_t, MXFP8 along H */
@@ -1101,7 +1116,7 @@ int oc_moe_bwd_expert_dw(int T, int H, int E, int k, int F, int recipe, const oc
             }
             free(zg); free(zu); free(v); free(rowbuf);
         }
-        if (recipe == OC_MX) {
+        if (is_mx(recipe)) {
             /* weight-gradient GEMM operands: MXFP8 along the expert's tokens (K = its rows), in blocks of
              * 32 consecutive tokens of its stable order; x and dY from their bf16 values */
             int c;

@@ -644,23 +644,25 @@ def _mx_bwd_case(seed=31):
     return wl, inp, mx
 
 
-def test_mxfp8_forward_composes_from_quantised_operands(oracle):
+@pytest.mark.parametrize("recipe", ["mxfp8", "mxfp8-q"])
+def test_mxfp8_forward_composes_from_quantised_operands(oracle, recipe):
     """recipe mxfp8 = fp64 products of x rounded to MXFP8 along H, the MXFP8 weights, the gate-folded
     activation (and the shared expert's activation) rounded to MXFP8 along F, and bf16 expert outputs
-    (torch fp64 + the pinned quantiser; a missing rounding point fails it)."""
+    (torch fp64 + the pinned quantiser; a missing rounding point fails it). mxfp8-q: the same MXFP8
+    quantisation points with unrounded expert outputs."""
     wl = small(T=16, H=64, E=4, k=2, F=64, S=1)
     inp = make_inputs(wl, seed=45)
     r = oracle.route(oracle.router_logits(inp["x"], inp["W_r"]), wl.k, "softmax", True, 1.0)
     names = ("W_g", "W_u", "W_d", "W_gs", "W_us", "W_ds")
     mx = {n: oracle.mxfp8_quantize(inp[n]) for n in names}
     y = oracle.moe_fwd_tokens(inp["x"], mx["W_g"][0], mx["W_u"][0], mx["W_d"][0], r["idx"], r["gates"],
-                              recipe="mxfp8", sf_g=mx["W_g"][1], sf_u=mx["W_u"][1], sf_d=mx["W_d"][1],
+                              recipe=recipe, sf_g=mx["W_g"][1], sf_u=mx["W_u"][1], sf_d=mx["W_d"][1],
                               shared=(mx["W_gs"][0], mx["W_us"][0], mx["W_ds"][0], mx["W_gs"][1], mx["W_us"][1],
                                       mx["W_ds"][1]))
     dec = {n: oracle.mxfp8_decode(*mx[n]) for n in names}
     xq = _mxq(inp["x"].double())
     silu = torch.nn.functional.silu
-    bf = lambda t: t.float().bfloat16().double()  # noqa: E731
+    bf = (lambda t: t) if recipe.endswith("-q") else (lambda t: t.float().bfloat16().double())  # noqa: E731
     ref = torch.zeros(wl.T, wl.H, dtype=torch.float64)
     for t in range(wl.T):
         for j in range(wl.k):
@@ -673,21 +675,23 @@ def test_mxfp8_forward_composes_from_quantised_operands(oracle):
     assert torch.allclose(y, ref, rtol=1e-9, atol=1e-12)
 
 
-def test_mxfp8_backward_composes_from_quantised_operands(oracle):
+@pytest.mark.parametrize("recipe", ["mxfp8", "mxfp8-q"])
+def test_mxfp8_backward_composes_from_quantised_operands(oracle, recipe):
     """The MXFP8 backward equals fp64 products of the operands rounded at the recipe's points:
     dY and x along H, W_d^T along H, dgate/dup to bf16 then along F, W_g^T / W_u^T along F, and
     for the weight gradients every operand along the expert's tokens (torch fp64 + the pinned
-    quantiser; a transposed operand or a missing rounding point fails it)."""
+    quantiser; a transposed operand or a missing rounding point fails it). mxfp8-q: the same MXFP8
+    quantisation points, with none of the bf16 roundings (saved z, dgate/dup, dXp, router path)."""
     wl, inp, mx = _mx_bwd_case()
     r = oracle.route(oracle.router_logits(inp["x"], inp["W_r"]).double(), wl.k, with_aux=False)
     dx, dl, dg = oracle.moe_bwd_tokens(inp["x"], inp["W_r"], None, None, None, inp["dY"], r, aux_on=False,
-                                       recipe="mxfp8", mx=mx)
+                                       recipe=recipe, mx=mx)
     dWg, dWu, dWd = oracle.moe_bwd_expert_dw(inp["x"], None, None, None, inp["dY"], r["idx"], r["gates"],
-                                             list(range(wl.E)), recipe="mxfp8", mx=mx)
+                                             list(range(wl.E)), recipe=recipe, mx=mx)
     dec = {n: oracle.mxfp8_decode(*mx[n]) for n in mx}
     x, dY = inp["x"].double(), inp["dY"].double()
     xq, dYq = _mxq(x), _mxq(dY)
-    bf = lambda t: t.float().bfloat16().double()
+    bf = (lambda t: t) if recipe.endswith("-q") else (lambda t: t.float().bfloat16().double())
     silu = torch.nn.functional.silu
     ref_dx = torch.zeros_like(x)
     rows = {e: [] for e in range(wl.E)}
@@ -873,9 +877,11 @@ def _nv_roundtrip_ref(t: torch.Tensor) -> torch.Tensor:
     return (_e2m1_generic(u) * sd.double().unsqueeze(-1)).view(t.shape)
 
 
-def test_nvfp4_forward_composes_from_quantised_operands(oracle):
+@pytest.mark.parametrize("recipe", ["nvfp4", "nvfp4-q"])
+def test_nvfp4_forward_composes_from_quantised_operands(oracle, recipe):
     """recipe nvfp4 = fp64 products of NVFP4 x (G=1), NVFP4 weights (G per expert),
-    the gate-folded activation rounded to NVFP4 (G=1) and bf16 expert outputs."""
+    the gate-folded activation rounded to NVFP4 (G=1) and bf16 expert outputs;
+    nvfp4-q: the same quantisation points with unrounded expert outputs."""
     wl = small(T=16, H=64, E=4, k=2, F=48, S=1)
     inp = make_inputs(wl, seed=43)
     logits = oracle.router_logits(inp["x"], inp["W_r"])
@@ -883,13 +889,13 @@ def test_nvfp4_forward_composes_from_quantised_operands(oracle):
     names = ("W_g", "W_u", "W_d", "W_gs", "W_us", "W_ds")
     nv = {n: oracle.nvfp4_quantize(inp[n], per_matrix=True) for n in names}
     y = oracle.moe_fwd_tokens(inp["x"], nv["W_g"][0], nv["W_u"][0], nv["W_d"][0], r["idx"], r["gates"],
-                              recipe="nvfp4", sf_g=nv["W_g"][1:], sf_u=nv["W_u"][1:], sf_d=nv["W_d"][1:],
+                              recipe=recipe, sf_g=nv["W_g"][1:], sf_u=nv["W_u"][1:], sf_d=nv["W_d"][1:],
                               shared=(nv["W_gs"][0], nv["W_us"][0], nv["W_ds"][0], nv["W_gs"][1:],
                                       nv["W_us"][1:], nv["W_ds"][1:]))
     dec = {n: oracle.nvfp4_decode(*nv[n]) for n in names}
     xq = _nv_roundtrip_ref(inp["x"])
     ref = torch.zeros(wl.T, wl.H, dtype=torch.float64)
-    bf = lambda t: t.float().bfloat16().double()  # noqa: E731
+    bf = (lambda t: t) if recipe.endswith("-q") else (lambda t: t.float().bfloat16().double())  # noqa: E731
     for t in range(wl.T):
         for j in range(wl.k):
             e = int(r["idx"][t, j])

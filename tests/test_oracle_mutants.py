@@ -72,9 +72,9 @@ MUTANTS = [
     ("router_dwr_transposed", "double c = dl[(long)t * E + e];", "double c = dl[(long)e * T + t];"),
     ("router_dwr_unrounded_dl", "if (round_dl) c = oc_bf16_round(c);", "if (0) c = oc_bf16_round(c);"),
     # precision recipes and block-scaled matrices
-    ("mx_recipe_skips_x", "        if (recipe == OC_MX) mx_roundtrip(xv, H);\n        else if (recipe == OC_NV) nv_roundtrip(xv, H);"
+    ("mx_recipe_skips_x", "        if (is_mx(recipe)) mx_roundtrip(xv, H);\n        else if (is_nv(recipe)) nv_roundtrip(xv, H);"
      "\n        for (int h = 0; h < H; ++h) y[h] = 0.0;",
-     "        if (0) mx_roundtrip(xv, H);\n        else if (recipe == OC_NV) nv_roundtrip(xv, H);"
+     "        if (0) mx_roundtrip(xv, H);\n        else if (is_nv(recipe)) nv_roundtrip(xv, H);"
      "\n        for (int h = 0; h < H; ++h) y[h] = 0.0;"),
     ("bf16_recipe_skips_act", "else if (recipe == OC_BF16R) round_vec(a, F, recipe);", "else if (0) round_vec(a, F, recipe);"),
     ("mx_roundtrip_scale_off", "        uint8_t sb = oc_mx_scale_byte(amax);\n        double X = ldexp(1.0, (int)sb - 127);"
@@ -120,6 +120,15 @@ MUTANTS = [
     ("mx_dgrad_reads_forward_weight", "oc_mat wt_d = oc_slice(WdT, (int64_t)e * F, F);   /* W_d^T [F, H], MXFP8 along H */\n"
      "                matvec(&wt_d, dye, v, rowbuf);",
      "for (int f = 0; f < F; ++f) v[f] = 0.0;\n                matvec_t_acc(&we_d, dye, v, rowbuf);"),
+    # the quantisation-points-only recipes
+    ("mxq_skips_mx_quantisation", "static int is_mx(int recipe) { return recipe == OC_MX || recipe == OC_MXQ; }",
+     "static int is_mx(int recipe) { return recipe == OC_MX; }"),
+    ("nvq_skips_nv_quantisation", "static int is_nv(int recipe) { return recipe == OC_NV || recipe == OC_NVQ; }",
+     "static int is_nv(int recipe) { return recipe == OC_NV; }"),
+    ("q_recipes_round_expert_outputs", "if (recipe == OC_BF16R || recipe == OC_MX || recipe == OC_NV)\n",
+     "if (recipe != OC_EXACT)\n"),
+    ("mxq_rounds_saved_z_in_weight_grads", "                if (recipe == OC_MX)\n                    for (int f = 0; f < F; ++f) { zg[f]",
+     "                if (is_mx(recipe))\n                    for (int f = 0; f < F; ++f) { zg[f]"),
 ]
 
 
