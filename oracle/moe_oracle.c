@@ -108,15 +108,20 @@ double oc_e4m3_decode(uint8_t c) {
     return s ? -v : v;
 }
 
+/* The binade of a positive finite double: the e with 2^e <= a < 2^(e+1).
+ * frexp returns a = m 2^x with m in [0.5, 1) exactly, so e = x - 1. */
+static int binade(double a) {
+    int x;
+    frexp(a, &x);
+    return x - 1;
+}
+
 /* Round |v| to the E4M3 grid, nearest-even, clamp to 448. v is finite. */
 uint8_t oc_e4m3_encode(double v) {
     uint8_t sign = (signbit(v) ? 0x80 : 0x00);
     double a = fabs(v);
     if (a == 0.0) return sign;
-    int e = (int)floor(log2(a));
-    /* guard against log2 rounding at exact powers of two */
-    if (ldexp(1.0, e) > a) e -= 1;
-    if (ldexp(1.0, e + 1) <= a) e += 1;
+    int e = binade(a);
     if (e < -6) e = -6;                     /* subnormal range shares the 2^-9 quantum */
     double q = ldexp(1.0, e - 3);           /* spacing of the grid in this binade */
     double r = a / q;                       /* exact: power-of-two division */
@@ -130,9 +135,7 @@ uint8_t oc_e4m3_encode(double v) {
     if (val > 448.0) val = 448.0;
     if (val == 0.0) return sign;
     /* encode val */
-    int ve = (int)floor(log2(val));
-    if (ldexp(1.0, ve) > val) ve -= 1;
-    if (ldexp(1.0, ve + 1) <= val) ve += 1;
+    int ve = binade(val);
     uint8_t code;
     if (ve < -6) {
         code = (uint8_t)(val / ldexp(1.0, -9));          /* subnormal: m = val / 2^-9 */
@@ -146,9 +149,7 @@ uint8_t oc_e4m3_encode(double v) {
 /* UE8M0 scale byte of one block, OCP MX v1.0 section 6.3 with E4M3 emax = 8. */
 uint8_t oc_mx_scale_byte(double amax) {
     if (!(amax > 0.0)) return 0;
-    int e = (int)floor(log2(amax));
-    if (ldexp(1.0, e) > amax) e -= 1;
-    if (ldexp(1.0, e + 1) <= amax) e += 1;
+    int e = binade(amax);
     int b = e - 8 + 127;
     if (b < 0) b = 0;
     if (b > 254) b = 254;
@@ -318,6 +319,14 @@ typedef struct {
     int64_t gs_rows;
 } oc_mat;
 
+/* Every E4M3 and E2M1 value, read from the decoders above once at load time
+ * (the matrix reader looks codes up here instead of decoding each element). */
+static double g_e4m3[256], g_e2m1[16];
+__attribute__((constructor)) static void oc_decode_tables(void) {
+    for (int c = 0; c < 256; ++c) g_e4m3[c] = oc_e4m3_decode((uint8_t)c);
+    for (int c = 0; c < 16; ++c) g_e2m1[c] = oc_e2m1_decode((uint8_t)c);
+}
+
 static void oc_row(const oc_mat* m, int64_t r, double* out) {
     int C = m->cols;
     if (m->kind == OC_BF16) {
@@ -326,14 +335,17 @@ static void oc_row(const oc_mat* m, int64_t r, double* out) {
     } else if (m->kind == OC_MXFP8) {
         const uint8_t* p = (const uint8_t*)m->data + r * C;
         const uint8_t* s = m->sf + r * (C / 32);
-        for (int c = 0; c < C; ++c) out[c] = oc_e4m3_decode(p[c]) * ldexp(1.0, (int)s[c / 32] - 127);
+        for (int b = 0; b < C / 32; ++b) {
+            const double X = ldexp(1.0, (int)s[b] - 127);
+            for (int c = 32 * b; c < 32 * b + 32; ++c) out[c] = g_e4m3[p[c]] * X;
+        }
     } else if (m->kind == OC_NVFP4) {
         const uint8_t* p = (const uint8_t*)m->data + r * (C / 2);
         const uint8_t* s = m->sf + r * (C / 16);
         double G = m->gs ? (double)m->gs[r / m->gs_rows] : 1.0;
         for (int c = 0; c < C; ++c) {
             uint8_t code = (p[c / 2] >> (4 * (c & 1))) & 15;
-            out[c] = oc_e2m1_decode(code) * oc_e4m3_decode(s[c / 16]) / G;
+            out[c] = g_e2m1[code] * g_e4m3[s[c / 16]] / G;
         }
     } else {
         const double* p = (const double*)m->data + r * C;

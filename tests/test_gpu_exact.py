@@ -1,0 +1,420 @@
+"""Floating outputs of the whole layer against the exact oracle, at the literal bar.
+
+Every floating output -- y; in the backward dX, dlogits, dW_g, dW_u, dW_d and dW_r -- is compared with
+the oracle's value computed with no rounding other than what the expert operand format itself defines:
+
+  BF16 layer         fp64 throughout on the bf16 inputs (recipe "exact");
+  MXFP8 / NVFP4      x, the weights and the gate-folded activation (and in the MXFP8 backward every
+                     MXFP8 GEMM operand) quantised as the format defines, nothing rounded to bf16
+                     (recipes "mxfp8-q" / "nvfp4-q").
+
+The bar is max |got - ref| <= 2e-2 rms(ref) for the BF16 layer and 6e-2 rms(ref) for the block-scaled
+ones, with no exception for any element. Beside it runs the tighter check against the oracle that rounds
+at the kernels' own points (recipes "bf16" / "mxfp8" / "nvfp4"), which prints how many elements took a
+rounding decision the other way.
+
+Sizes: the tiny workload in full; each full-size workload on 512 seeded tokens (all of their outputs)
+and, for the backward, the weight gradients of expert 0, the heaviest expert, two median experts and the
+zero-token experts. A weight gradient is compared expert by expert: each expert's matrix is a parameter
+tensor of its own, and its bar is the rms of that matrix. dW_r, a sum over every token, is compared in
+full where the oracle runs the whole backward (the tiny workload) and otherwise checked as the product
+bf16(dlogits)^T x of the GPU's own dlogits, whose sampled rows are compared with the exact oracle.
+
+Routing indices, counts and offsets are compared bit for bit (a token whose top-k differs must be a
+near-tie of the logits, and floating outputs are compared on the tokens whose routing agrees).
+"""
+import json
+import os
+import time
+
+import pytest
+import torch
+
+from helpers import TOL_BF16, TOL_MXFP8, TOL_NVFP4, check_bf16, empty, err_rms
+from mixture_experts_layer_aux_b200.synthetic import WORKLOADS, Workload, make_inputs
+from test_gpu_layer import host, routing_agreement, run_bwd, run_fwd
+
+pytestmark = pytest.mark.gpu
+
+N_TOK = 512
+
+
+def _record(name, res):
+    """Print the errors; also append them to $MOE_PARITY_LOG (a JSON-lines file) when it is set."""
+    print(name, {k: (round(v, 5) if isinstance(v, float) else v) for k, v in res.items()})
+    p = os.environ.get("MOE_PARITY_LOG")
+    if p:
+        with open(p, "a") as f:
+            f.write(json.dumps({"case": name, **res}) + "\n")
+
+
+def _sample_tokens(T, n, seed):
+    if n >= T:
+        return torch.arange(T, dtype=torch.int32)
+    g = torch.Generator().manual_seed(seed)
+    return torch.randperm(T, generator=g)[:n].sort().values.to(torch.int32)
+
+
+def _sample_experts(counts):
+    """Expert 0, the heaviest, two median experts (among those with tokens) and the zero-token experts."""
+    counts = counts.cpu()
+    nz = (counts > 0).nonzero().flatten()
+    order = nz[counts[nz].argsort(stable=True)]
+    ex = {0, int(order[-1])}
+    if len(order) >= 2:
+        ex |= {int(order[len(order) // 2]), int(order[(len(order) - 1) // 2])}
+    ex |= set((counts == 0).nonzero().flatten().tolist()[:2])
+    return sorted(ex)
+
+
+def _exact(got, ref, tol):
+    """max |got - ref| / rms(ref), ref the exact oracle value; the bar has no exception."""
+    return err_rms(got, ref), tol
+
+
+class Checks:
+    """Collects (value, bar) pairs and asserts them all at the end, so one run reports every error."""
+
+    def __init__(self, name):
+        self.name, self.res, self.bad = name, {}, []
+
+    def exact(self, key, got, ref, tol):
+        e = err_rms(got, ref)
+        self.res[key] = e
+        if not e <= tol:
+            self.bad.append(f"{key}: {e:.4g} > {tol}")
+
+    def recipe(self, key, got, ref, tol):
+        try:
+            strict, _, flips = check_bf16(got, ref, tol=tol)
+            self.res[key + "@recipe"] = strict
+            self.res[key + "@flips"] = flips
+        except AssertionError as ex:
+            self.res[key + "@recipe"] = str(ex)
+            self.bad.append(f"{key} (identical quantisation): {ex}")
+
+    def bound(self, key, value, tol):
+        self.res[key] = value
+        if not value <= tol:
+            self.bad.append(f"{key}: {value:.4g} > {tol}")
+
+    def done(self, moe):
+        _record(self.name, self.res)
+        assert moe.moe_get_device_status() == 0
+        assert not self.bad, "; ".join(self.bad)
+
+
+# ------------------------------------------------------------------ forward, BF16
+
+
+def _fwd_bf16(moe, oracle, wl, n_tok, seed=0):
+    d = make_inputs(wl, device="cuda", seed=seed)
+    out = run_fwd(moe, wl, d)
+    h = host(d)
+    r, same = routing_agreement(oracle, wl, h, out["idx"])
+    if bool(same.all()):
+        assert torch.equal(out["counts"].cpu(), r["counts"]) and torch.equal(out["offsets"].cpu(), r["offsets"])
+    toks = _sample_tokens(wl.T, n_tok, seed + 99)
+    toks = toks[same[toks.long()]]
+    shared = (h["W_gs"], h["W_us"], h["W_ds"]) if wl.S else None
+    c = Checks(f"fwd {wl.name} ({toks.numel()} tokens)")
+    y = out["y"].cpu()[toks.long()]
+    ref = oracle.moe_fwd_tokens(h["x"], h["W_g"], h["W_u"], h["W_d"], r["idx_kept"], r["gates"], toks,
+                                shared=shared, recipe="exact")
+    c.exact("y", y, ref, TOL_BF16)
+    c.recipe("y", y, oracle.moe_fwd_tokens(h["x"], h["W_g"], h["W_u"], h["W_d"], r["idx_kept"], r["gates"], toks,
+                                           shared=shared, recipe="bf16"), TOL_BF16)
+    c.bound("gates", (out["gates"].cpu().double()[toks.long()] - r["gates"][toks.long()]).abs().max().item(), 1e-5)
+    if out["aux"] is not None:
+        c.bound("aux_rel", abs(out["aux"].item() - r["aux"]) / abs(r["aux"]), 1e-4)
+    c.done(moe)
+
+
+def test_exact_fwd_tiny_full(moe, oracle):
+    _fwd_bf16(moe, oracle, WORKLOADS["tiny"], WORKLOADS["tiny"].T)
+
+
+@pytest.mark.parametrize("name", ["mixtral", "qwen3"])
+def test_exact_fwd_full_size_512_tokens(moe, oracle, name):
+    _fwd_bf16(moe, oracle, WORKLOADS[name], N_TOK)
+
+
+# ------------------------------------------------------------------ forward, block-scaled
+
+
+def _oracle_weights(oracle, d, names, experts, fmt):
+    """The oracle's own quantisation of the bf16 weights (only `experts` of the [E, R, C] tensors)."""
+    out = {}
+    for name in names:
+        W = d[name]
+        if W.dim() == 2:
+            out[name] = oracle.mxfp8_quantize(W.cpu()) if fmt == "mxfp8" else \
+                oracle.nvfp4_quantize(W.cpu(), per_matrix=True)
+            continue
+        E, R, C = W.shape
+        if fmt == "mxfp8":
+            codes = torch.zeros((E, R, C), dtype=torch.uint8)
+            sf = torch.zeros((E, R, C // 32), dtype=torch.uint8)
+            for e in experts:
+                codes[e], sf[e] = oracle.mxfp8_quantize(W[e].cpu())
+            out[name] = (codes, sf)
+        else:
+            packed = torch.zeros((E, R, C // 2), dtype=torch.uint8)
+            sf = torch.zeros((E, R, C // 16), dtype=torch.uint8)
+            G = torch.ones(E, dtype=torch.float32)
+            for e in experts:
+                packed[e], sf[e], G[e] = oracle.nvfp4_quantize(W[e].cpu(), per_matrix=True)
+            out[name] = (packed, sf, G)
+    return out
+
+
+def _gpu_weights(moe, d, names, fmt):
+    q = {}
+    for name in names:
+        w = d[name]
+        if fmt == "mxfp8":
+            codes = torch.empty(w.shape, dtype=torch.uint8, device="cuda")
+            sf = torch.empty(w.shape[:-1] + (w.shape[-1] // 32,), dtype=torch.uint8, device="cuda")
+            moe.moe_quantize_mxfp8(w, codes, sf)
+        else:
+            R, C = w.shape[-2], w.shape[-1]
+            codes = torch.empty(w.shape[:-1] + (C // 2,), dtype=torch.uint8, device="cuda")
+            sf = torch.empty(moe.moe_nvfp4_sf_bytes(w.numel() // (R * C), R, C), dtype=torch.uint8, device="cuda")
+            moe.moe_quantize_nvfp4(w.contiguous(), codes, sf)
+        q[name] = (codes, sf)
+    return q
+
+
+def _fwd_block_scaled(moe, oracle, wl, n_tok, seed=0):
+    fmt = wl.dtype
+    d = make_inputs(wl, device="cuda", seed=seed)
+    names = ["W_g", "W_u", "W_d"] + (["W_gs", "W_us", "W_ds"] if wl.S else [])
+    q = _gpu_weights(moe, d, names, fmt)
+    cfg = moe.make_config(wl)
+    T, k, H = wl.T, wl.k, wl.H
+    y, idx, gates = empty((T, H), torch.bfloat16), empty((T, k), torch.int32), empty((T, k), torch.float32)
+    sh = [None] * 6
+    if wl.S:
+        sh = [q["W_gs"][0], q["W_us"][0], q["W_ds"][0], q["W_gs"][1], q["W_us"][1], q["W_ds"][1]]
+    moe.moe_layer_fwd(cfg, d["x"], d["W_r"], d.get("logit_bias"), q["W_g"][0], q["W_u"][0], q["W_d"][0],
+                      q["W_g"][1], q["W_u"][1], q["W_d"][1], *sh, y, None, idx, gates, None, None, None,
+                      moe.workspace(moe.moe_layer_workspace_size(cfg)), expert_bias=d.get("expert_bias"))
+    torch.cuda.synchronize()
+    del q
+    h = {"x": d["x"].cpu(), "W_r": d["W_r"].cpu(),
+         "expert_bias": None if d.get("expert_bias") is None else d["expert_bias"].cpu()}
+    r, same = routing_agreement(oracle, wl, h, idx)
+    toks = _sample_tokens(T, n_tok, seed + 7)
+    toks = toks[same[toks.long()]]
+    need = sorted(set(r["idx"][toks.long()].flatten().tolist()) - {-1})
+    W = _oracle_weights(oracle, {n: d[n] for n in names}, names, need, fmt)
+    sfs = {n: (W[n][1] if fmt == "mxfp8" else W[n][1:]) for n in names}
+    shared = (W["W_gs"][0], W["W_us"][0], W["W_ds"][0], sfs["W_gs"], sfs["W_us"], sfs["W_ds"]) if wl.S else None
+    c = Checks(f"fwd {wl.name} ({toks.numel()} tokens)")
+    got = y.cpu()[toks.long()]
+    tol = TOL_MXFP8 if fmt == "mxfp8" else TOL_NVFP4
+    for recipe in (fmt + "-q", fmt):
+        ref = oracle.moe_fwd_tokens(h["x"], W["W_g"][0], W["W_u"][0], W["W_d"][0], r["idx_kept"], r["gates"], toks,
+                                    recipe=recipe, sf_g=sfs["W_g"], sf_u=sfs["W_u"], sf_d=sfs["W_d"], shared=shared)
+        if recipe.endswith("-q"):
+            c.exact("y", got, ref, tol)
+        else:
+            c.recipe("y", got, ref, tol)
+    c.bound("gates", (gates.cpu().double()[toks.long()] - r["gates"][toks.long()]).abs().max().item(), 1e-5)
+    c.done(moe)
+
+
+def test_exact_fwd_mxfp8_small_full(moe, oracle):
+    wl = Workload("mx-small", T=256, H=512, E=16, k=4, F=256, S=1, score="sigmoid", route_scale=2.5, dtype="mxfp8",
+                  aux=False)
+    _fwd_block_scaled(moe, oracle, wl, wl.T)
+
+
+def test_exact_fwd_dsv3_mxfp8_512_tokens(moe, oracle):
+    _fwd_block_scaled(moe, oracle, WORKLOADS["dsv3"], N_TOK)
+
+
+def test_exact_fwd_dsv3_nvfp4_512_tokens(moe, oracle):
+    _fwd_block_scaled(moe, oracle, WORKLOADS["dsv3-nvfp4"], N_TOK)
+
+
+# ------------------------------------------------------------------ backward, BF16
+
+
+def _dw_checks(c, got, ref_exact, ref_recipe, experts, kept_counts, tol):
+    """Per-expert comparison of one weight gradient (rows of `experts`); zero-token experts exact zeros."""
+    worst_exact, worst_whole = 0.0, 0.0
+    for q, e in enumerate(experts):
+        if int(kept_counts[e]) == 0:
+            assert bool((got[e] == 0).all()), e
+            continue
+        c.exact(f"[e{e}]", got[e], ref_exact[q], tol)
+        worst_exact = max(worst_exact, c.res[f"[e{e}]"])
+        if ref_recipe is not None:
+            c.recipe(f"[e{e}]", got[e], ref_recipe[q], tol)
+    ex = torch.tensor(experts).long()
+    worst_whole = err_rms(got[ex], ref_exact)
+    return worst_exact, worst_whole
+
+
+def _bwd_bf16(moe, oracle, wl, n_tok, d_aux, seed=0):
+    d = make_inputs(wl, device="cuda", seed=seed, with_dy=True)
+    fwd = run_fwd(moe, wl, d, save=True)
+    g = run_bwd(moe, wl, d, fwd, d_aux)
+    h = host(d)
+    del d
+    r, same = routing_agreement(oracle, wl, h, fwd["idx"])
+    full = n_tok >= wl.T
+    toks = _sample_tokens(wl.T, n_tok, seed)
+    toks = toks[same[toks.long()]]
+    experts = _sample_experts(fwd["counts"]) if not full else list(range(wl.E))
+    if not bool(same.all()):
+        flipped = set(fwd["idx"].cpu()[~same].flatten().tolist()) | set(r["idx"][~same].flatten().tolist())
+        experts = [e for e in experts if e not in flipped]
+    aux_on = wl.aux and wl.score == "softmax"
+    c = Checks(f"bwd {wl.name} ({toks.numel()} tokens, experts {experts})")
+    t0 = time.time()
+    refs = {}
+    for recipe in ("exact", "bf16"):
+        refs[recipe] = oracle.moe_bwd_tokens(h["x"], h["W_r"], h["W_g"], h["W_u"], h["W_d"], h["dY"], r, toks,
+                                             score=wl.score, norm=wl.norm_topk, route_scale=wl.route_scale,
+                                             aux_on=aux_on, d_aux=d_aux, recipe=recipe)
+    dX = g["dX"].cpu()[toks.long()]
+    c.exact("dX", dX, refs["exact"][0], TOL_BF16)
+    c.recipe("dX", dX, refs["bf16"][0], TOL_BF16)
+    c.exact("dlogits", g["dlogits"].cpu()[toks.long()], refs["exact"][1], TOL_BF16)
+    dws = {rc: oracle.moe_bwd_expert_dw(h["x"], h["W_g"], h["W_u"], h["W_d"], h["dY"], r["idx_kept"], r["gates"],
+                                        experts, recipe=rc) for rc in ("exact", "bf16")}
+    for i, name in enumerate(("dW_g", "dW_u", "dW_d")):
+        sub = Checks(name)
+        worst, whole = _dw_checks(sub, g[name].cpu(), dws["exact"][i], dws["bf16"][i], experts, r["kept_counts"],
+                                  TOL_BF16)
+        c.res[name + " worst expert"] = worst
+        c.res[name + " (whole-set rms)"] = whole
+        c.res.update({name + k: v for k, v in sub.res.items() if "@" in k})
+        c.bad += [name + b for b in sub.bad]
+    if full:
+        c.exact("dW_r", g["dW_r"].cpu(), oracle.router_dwr(refs["exact"][1], h["x"]), TOL_BF16)
+    else:
+        dl16 = g["dlogits"].double().cpu().float().bfloat16().double()
+        c.exact("dW_r (GPU dlogits)", g["dW_r"].cpu(), dl16.T @ h["x"].double(), TOL_BF16)
+    c.res["oracle_s"] = round(time.time() - t0, 1)
+    c.done(moe)
+
+
+def test_exact_bwd_tiny_full(moe, oracle):
+    wl = WORKLOADS["tiny"].with_(name="tiny-bwd", bwd=True)
+    _bwd_bf16(moe, oracle, wl, wl.T, d_aux=0.01)
+
+
+def test_exact_bwd_skewed_512_tokens(moe, oracle):
+    _bwd_bf16(moe, oracle, WORKLOADS["skewed"], N_TOK, d_aux=0.01)
+
+
+# ------------------------------------------------------------------ backward, MXFP8 (the training step)
+
+
+def _transposed_mx_oracle(oracle, W, experts, ldd=None, col0=0, out=None):
+    """Oracle MXFP8 codes of W[e]^T (blocks along W's rows) for the listed experts."""
+    E, R, C = W.shape
+    ldd = ldd or R
+    if out is None:
+        out = (torch.zeros((E, C, ldd), dtype=torch.uint8), torch.zeros((E, C, ldd // 32), dtype=torch.uint8))
+    for e in experts:
+        codes, sf = oracle.mxfp8_quantize(W[e].cpu().T.contiguous())
+        out[0][e, :, col0:col0 + R] = codes
+        out[1][e, :, col0 // 32:(col0 + R) // 32] = sf
+    return out
+
+
+def _train_mxfp8(moe, oracle, wl, n_tok, d_aux=0.0, seed=0):
+    d = make_inputs(wl, device="cuda", seed=seed, with_dy=True)
+    T, H, E, k, F = wl.T, wl.H, wl.E, wl.k, wl.F
+    cfg = moe.make_config(wl, save_for_bwd=1)
+    q = _gpu_weights(moe, d, ["W_g", "W_u", "W_d"], "mxfp8")
+    wdt = torch.empty((E, F, H), dtype=torch.uint8, device="cuda")
+    wdt_sf = torch.empty((E, F, H // 32), dtype=torch.uint8, device="cuda")
+    moe.moe_quantize_mxfp8_t(d["W_d"], wdt, wdt_sf)
+    wgu = torch.empty((E, H, 2 * F), dtype=torch.uint8, device="cuda")
+    wgu_sf = torch.empty((E, H, 2 * F // 32), dtype=torch.uint8, device="cuda")
+    moe.moe_quantize_mxfp8_t(d["W_g"], wgu, wgu_sf, ldd=2 * F)
+    moe.moe_quantize_mxfp8_t(d["W_u"], wgu, wgu_sf, ldd=2 * F, col0=F)
+    y, idx = empty((T, H), torch.bfloat16), empty((T, k), torch.int32)
+    counts = empty((E,), torch.int32)
+    aux = empty((1,), torch.float32) if cfg.compute_aux else None
+    saved = moe.workspace(moe.moe_layer_saved_size(cfg))
+    moe.moe_layer_fwd(cfg, d["x"], d["W_r"], d.get("logit_bias"), q["W_g"][0], q["W_u"][0], q["W_d"][0],
+                      q["W_g"][1], q["W_u"][1], q["W_d"][1], None, None, None, None, None, None, y, aux, idx, None,
+                      counts, None, saved, moe.workspace(moe.moe_layer_workspace_size(cfg)),
+                      expert_bias=d.get("expert_bias"))
+    o = dict(dX=empty((T, H), torch.bfloat16), dW_r=empty((E, H), torch.bfloat16),
+             dW_g=empty((E, F, H), torch.bfloat16), dW_u=empty((E, F, H), torch.bfloat16),
+             dW_d=empty((E, H, F), torch.bfloat16), dlogits=empty((T, E), torch.float32))
+    moe.moe_layer_bwd_mxfp8(cfg, d["dY"], d_aux, d["x"], d["W_r"], wdt, wdt_sf, wgu, wgu_sf, saved, o["dX"],
+                            o["dW_r"], o["dW_g"], o["dW_u"], o["dW_d"], o["dlogits"],
+                            moe.workspace(moe.moe_layer_bwd_mxfp8_workspace_size(cfg)))
+    torch.cuda.synchronize()
+    assert moe.moe_get_device_status() == 0
+    del q, wdt, wdt_sf, wgu, wgu_sf, saved
+    g = {n: v.cpu() for n, v in o.items()}
+    del o
+    h = host(d)
+    del d
+    torch.cuda.empty_cache()
+    r, same = routing_agreement(oracle, wl, h, idx)
+    full = n_tok >= T
+    toks = _sample_tokens(T, n_tok, seed)
+    toks = toks[same[toks.long()]]
+    experts = list(range(E)) if full else _sample_experts(counts)
+    if not bool(same.all()):
+        flipped = set(idx.cpu()[~same].flatten().tolist()) | set(r["idx"][~same].flatten().tolist())
+        experts = [e for e in experts if e not in flipped]
+    need = sorted(set(r["idx"][toks.long()].flatten().tolist()) | set(experts))
+    # the oracle quantises the bf16 weights itself: forward operands along K, the backward's transposed
+    # operands (W_d^T along H, W_g^T and W_u^T along F)
+    t0 = time.time()
+    mx = _oracle_weights(oracle, h, ["W_g", "W_u", "W_d"], need, "mxfp8")
+    mx["W_dT"] = _transposed_mx_oracle(oracle, h["W_d"], need)
+    mx["W_gT"] = _transposed_mx_oracle(oracle, h["W_g"], need)
+    mx["W_uT"] = _transposed_mx_oracle(oracle, h["W_u"], need)
+    aux_on = wl.aux and wl.score == "softmax"
+    c = Checks(f"train {wl.name} ({toks.numel()} tokens, experts {experts})")
+    got_y = y.cpu()[toks.long()]
+    sfs = {n: mx[n][1] for n in ("W_g", "W_u", "W_d")}
+    for recipe in ("mxfp8-q", "mxfp8"):
+        ref = oracle.moe_fwd_tokens(h["x"], mx["W_g"][0], mx["W_u"][0], mx["W_d"][0], r["idx"], r["gates"], toks,
+                                    recipe=recipe, sf_g=sfs["W_g"], sf_u=sfs["W_u"], sf_d=sfs["W_d"])
+        (c.exact if recipe.endswith("-q") else c.recipe)("y", got_y, ref, TOL_MXFP8)
+    refs = {rc: oracle.moe_bwd_tokens(h["x"], h["W_r"], None, None, None, h["dY"], r, toks, score=wl.score,
+                                      norm=wl.norm_topk, route_scale=wl.route_scale, aux_on=aux_on, d_aux=d_aux,
+                                      recipe=rc, mx=mx) for rc in ("mxfp8-q", "mxfp8")}
+    dX = g["dX"][toks.long()]
+    c.exact("dX", dX, refs["mxfp8-q"][0], TOL_MXFP8)
+    c.recipe("dX", dX, refs["mxfp8"][0], TOL_MXFP8)
+    c.exact("dlogits", g["dlogits"][toks.long()], refs["mxfp8-q"][1], TOL_MXFP8)
+    dws = {rc: oracle.moe_bwd_expert_dw(h["x"], None, None, None, h["dY"], r["idx"], r["gates"], experts,
+                                        recipe=rc, mx=mx) for rc in ("mxfp8-q", "mxfp8")}
+    for i, name in enumerate(("dW_g", "dW_u", "dW_d")):
+        sub = Checks(name)
+        worst, whole = _dw_checks(sub, g[name], dws["mxfp8-q"][i], dws["mxfp8"][i], experts, r["counts"], TOL_MXFP8)
+        c.res[name + " worst expert"] = worst
+        c.res[name + " (whole-set rms)"] = whole
+        c.res.update({name + k: v for k, v in sub.res.items() if "@" in k})
+        c.bad += [name + b for b in sub.bad]
+    if full:
+        c.exact("dW_r", g["dW_r"], oracle.router_dwr(refs["mxfp8-q"][1], h["x"]), TOL_MXFP8)
+    else:
+        dl16 = g["dlogits"].double().float().bfloat16().double()
+        c.exact("dW_r (GPU dlogits)", g["dW_r"], dl16.T @ h["x"].double(), TOL_BF16)
+    c.res["oracle_s"] = round(time.time() - t0, 1)
+    c.done(moe)
+
+
+def test_exact_train_mxfp8_small_full(moe, oracle):
+    wl = Workload("mx-train-small", T=384, H=256, E=8, k=2, F=256, dtype="mxfp8", skew=True, bwd=True)
+    _train_mxfp8(moe, oracle, wl, wl.T, d_aux=0.2, seed=3)
+
+
+def test_exact_train_dsv3_mxfp8_512_tokens(moe, oracle):
+    """The MXFP8 training step at the DeepSeek-V3 shape (T=8192, H=7168, E=256, k=8, F=2048)."""
+    _train_mxfp8(moe, oracle, WORKLOADS["dsv3-train"], N_TOK)

@@ -29,8 +29,8 @@ MUTANTS = [
     ("e4m3_decode_bias", "else v = ldexp(1.0 + m / 8.0, ef - 7);", "else v = ldexp(1.0 + m / 8.0, ef - 8);"),
     ("e4m3_ties_away", "else n = (fmod(fl, 2.0) == 0.0) ? fl : fl + 1.0;", "else n = fl + 1.0;"),
     ("mx_scale_emax", "int b = e - 8 + 127;", "int b = e - 7 + 127;"),
-    ("mx_matrix_scale_bias", "out[c] = oc_e4m3_decode(p[c]) * ldexp(1.0, (int)s[c / 32] - 127);",
-     "out[c] = oc_e4m3_decode(p[c]) * ldexp(1.0, (int)s[c / 32] - 128);"),
+    ("mx_matrix_scale_bias", "const double X = ldexp(1.0, (int)s[b] - 127);",
+     "const double X = ldexp(1.0, (int)s[b] - 128);"),
     ("e2m1_ties_odd", "if (d < bd || (d == bd && (c & 1) == 0)) {", "if (d < bd || (d == bd && (c & 1) == 1)) {"),
     ("nvfp4_scale_divisor", "float s = amax / 6.0f;", "float s = amax / 4.0f;"),
     ("nvfp4_inverted_scale", "float r = sd > 0.0f ? G / sd : 0.0f;", "float r = sd > 0.0f ? sd / G : 0.0f;"),
@@ -84,8 +84,8 @@ MUTANTS = [
     ("mx_strided_ignores_stride", "t[i] = (float)v[(b0 + i) * stride];", "t[i] = (float)v[b0 + i];"),
     ("nv_roundtrip_drops_scale", "for (int i = 0; i < 16; ++i) v[b * 16 + i] = oc_e2m1_decode(c[i]) * sd;",
      "for (int i = 0; i < 16; ++i) v[b * 16 + i] = oc_e2m1_decode(c[i]);"),
-    ("nvfp4_matrix_multiplies_G", "out[c] = oc_e2m1_decode(code) * oc_e4m3_decode(s[c / 16]) / G;",
-     "out[c] = oc_e2m1_decode(code) * oc_e4m3_decode(s[c / 16]) * G;"),
+    ("nvfp4_matrix_multiplies_G", "out[c] = g_e2m1[code] * g_e4m3[s[c / 16]] / G;",
+     "out[c] = g_e2m1[code] * g_e4m3[s[c / 16]] * G;"),
     ("nvfp4_slice_keeps_first_G", "if (m->gs) s.gs = m->gs + r0 / m->gs_rows;", "if (m->gs) s.gs = m->gs;"),
     ("nvfp4_pack_nibbles_swapped", "(uint8_t)(c[2 * i] | (c[2 * i + 1] << 4))", "(uint8_t)(c[2 * i + 1] | (c[2 * i] << 4))",
      True),
