@@ -46,7 +46,8 @@ struct TopkArgs {
   int n_group, topk_group, sel_mode;
 };
 
-__device__ __forceinline__ bool better(float v1, int i1, float v2, int i2) {
+template <typename V>
+__device__ __forceinline__ bool better(V v1, int i1, V v2, int i2) {
   return (v1 > v2) || (v1 == v2 && i1 < i2);
 }
 
@@ -125,8 +126,9 @@ __global__ void __launch_bounds__(WARPS * 32) topk_kernel(TopkArgs a) {
       }
       if (a.n_group > 1) {
         const int G = a.E / a.n_group;
-        // lane g ends up with group g's score: the sum of its two largest selection values
-        float my_gs = -INFINITY;
+        // lane g ends up with group g's score: the sum of its two largest selection values, added in
+        // double, where the sum of two fp32 values is exact (so near-equal group scores order exactly)
+        double my_gs = -INFINITY;
         for (int g = 0; g < a.n_group; ++g) {
           float b1 = -INFINITY, b2 = -INFINITY;
 #pragma unroll
@@ -149,16 +151,16 @@ __global__ void __launch_bounds__(WARPS * 32) topk_kernel(TopkArgs a) {
             b1 = fmaxf(b1, o1);
             b2 = n2;
           }
-          if (lane == g) my_gs = (G >= 2) ? b1 + b2 : b1;
+          if (lane == g) my_gs = (G >= 2) ? (double)b1 + (double)b2 : (double)b1;
         }
         // the topk_group best groups (score desc, group index asc)
         uint32_t kept = 0;
         for (int r = 0; r < a.topk_group; ++r) {
-          float bv = ((kept >> lane) & 1u) ? -INFINITY : my_gs;
+          double bv = ((kept >> lane) & 1u) ? -INFINITY : my_gs;
           int bi = (lane < a.n_group && !((kept >> lane) & 1u)) ? lane : 0x7fffffff;
 #pragma unroll
           for (int o = 16; o > 0; o >>= 1) {
-            const float ov = __shfl_xor_sync(0xffffffffu, bv, o);
+            const double ov = __shfl_xor_sync(0xffffffffu, bv, o);
             const int oi = __shfl_xor_sync(0xffffffffu, bi, o);
             if (better(ov, oi, bv, bi)) {
               bv = ov;

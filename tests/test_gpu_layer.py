@@ -101,11 +101,6 @@ def test_layer_fwd_small_cases_full_oracle(moe, oracle, wl):
     check_fwd(moe, oracle, wl)
 
 
-@pytest.mark.parametrize("name,n", [("mixtral", 48), ("qwen3", 96)])
-def test_layer_fwd_workload_sampled(moe, oracle, name, n):
-    check_fwd(moe, oracle, WORKLOADS[name], n_sample=n)
-
-
 @pytest.mark.parametrize("cf", [0.6, 1.0])
 def test_layer_fwd_capacity_factor_full_oracle(moe, oracle, cf):
     """Each expert keeps its first ceil(cf T k / E) pairs in token order; dropped pairs add nothing."""
@@ -244,21 +239,6 @@ def test_layer_bwd_deepseek_router_variant_full_oracle(moe, oracle):
     check_bwd(moe, oracle, wl, seed=5, d_aux=0.0)
 
 
-def test_layer_bwd_skewed_workload_sampled(moe, oracle):
-    wl = WORKLOADS["skewed"]
-    d = make_inputs(wl, device="cuda", seed=0, with_dy=True)
-    fwd = run_fwd(moe, wl, d, save=True)
-    counts = fwd["counts"].cpu()
-    assert int((counts == 0).sum()) >= 1, "the skewed workload must leave some experts without tokens"
-    nz = (counts > 0).nonzero().flatten()
-    order = nz[counts[nz].argsort()]
-    experts = sorted(set([0, int(order[0]), int(order[len(order) // 2])] +
-                         (counts == 0).nonzero().flatten().tolist()[:2]))
-    del d, fwd
-    torch.cuda.empty_cache()
-    check_bwd(moe, oracle, wl, seed=0, d_aux=0.01, n_tok=48, experts=experts)
-
-
 # ------------------------------------------------------------------ MXFP8 layer
 
 
@@ -341,6 +321,3 @@ def test_layer_fwd_mxfp8_deepseek_router_with_capacity(moe, oracle):
                   aux=False, dtype="mxfp8", n_group=4, topk_group=2, sel_bias=True, capacity_factor=1.0)
     check_fwd_mx(moe, oracle, wl)
 
-
-def test_layer_fwd_dsv3_mxfp8_sampled(moe, oracle):
-    check_fwd_mx(moe, oracle, WORKLOADS["dsv3"], n_sample=8)

@@ -275,9 +275,17 @@ def _mx_layer(moe, oracle, wl, seed, d_aux=0.2):
     r = oracle.route(logits, k, wl.score, wl.norm_topk, wl.route_scale, with_aux=wl.aux and wl.score == "softmax",
                      expert_bias=h.get("expert_bias"), n_group=wl.n_group, topk_group=wl.topk_group)
     assert torch.equal(idx.cpu(), r["idx"]), "full-oracle parity needs identical routing"
-    mx = {n: (q[n][0].cpu(), q[n][1].cpu()) for n in q}
-    mx.update(W_dT=(wdt.cpu(), wdt_sf.cpu()), W_gT=(wgu.cpu()[:, :, :F].contiguous(), wgu_sf.cpu()[:, :, :F // 32].contiguous()),
-              W_uT=(wgu.cpu()[:, :, F:].contiguous(), wgu_sf.cpu()[:, :, F // 32:].contiguous()))
+    # the oracle quantises the bf16 weights itself (forward operands along K; W_d^T along H, W_g^T and
+    # W_u^T along F), and the GPU's codes must be the same bytes
+    mx = {n: oracle.mxfp8_quantize(h[n]) for n in ("W_g", "W_u", "W_d")}
+    mx.update(W_dT=oracle.mxfp8_quantize(h["W_d"].transpose(1, 2).contiguous()),
+              W_gT=oracle.mxfp8_quantize(h["W_g"].transpose(1, 2).contiguous()),
+              W_uT=oracle.mxfp8_quantize(h["W_u"].transpose(1, 2).contiguous()))
+    for n in ("W_g", "W_u", "W_d"):
+        assert torch.equal(q[n][0].cpu(), mx[n][0]) and torch.equal(q[n][1].cpu(), mx[n][1]), n
+    assert torch.equal(wdt.cpu(), mx["W_dT"][0]) and torch.equal(wdt_sf.cpu(), mx["W_dT"][1])
+    assert torch.equal(wgu.cpu(), torch.cat([mx["W_gT"][0], mx["W_uT"][0]], dim=2))
+    assert torch.equal(wgu_sf.cpu(), torch.cat([mx["W_gT"][1], mx["W_uT"][1]], dim=2))
     aux_on = wl.aux and wl.score == "softmax"
     dx, dl, _ = oracle.moe_bwd_tokens(h["x"], h["W_r"], None, None, None, h["dY"], r, score=wl.score,
                                       norm=wl.norm_topk, route_scale=wl.route_scale, aux_on=aux_on, d_aux=d_aux,

@@ -236,6 +236,3 @@ def test_layer_fwd_nvfp4_deepseek_router_and_capacity_full_oracle(moe, oracle):
                   dtype="nvfp4", n_group=4, topk_group=2, sel_bias=True, capacity_factor=1.0)
     check_fwd_nv(moe, oracle, wl)
 
-
-def test_layer_fwd_dsv3_nvfp4_sampled(moe, oracle):
-    check_fwd_nv(moe, oracle, WORKLOADS["dsv3-nvfp4"], n_sample=8)
