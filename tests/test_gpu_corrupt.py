@@ -103,7 +103,8 @@ def test_permute_flags_and_drops_bad_expert_indices(moe, oracle, dtype):
 def _offsets_cases(rows, E):
     good = torch.linspace(0, rows, E + 1).round().to(torch.int32)
     non_monotone = good.clone()
-    non_monotone[3], non_monotone[4] = non_monotone[4], non_monotone[3]
+    non_monotone[3] = int(good[4])          # offsets[3] > offsets[4]
+    non_monotone[4] = int(good[3])
     past_end = good.clone()
     past_end[-1] = rows + 128
     negative = good.clone()

@@ -929,3 +929,28 @@ def test_nvfp4_bf16_and_fp32_entry_points_agree(oracle):
     a = oracle.nvfp4_quantize(v)
     b = oracle.nvfp4_quantize(v.float())
     assert torch.equal(a[0], b[0]) and torch.equal(a[1], b[1])
+
+
+# --------------------------------------------------------------- what a bf16 output can reach
+
+
+def test_literal_bar_is_out_of_reach_of_a_correctly_rounded_bf16_weight_gradient(oracle):
+    """The literal bar max |got - ref| <= 2e-2 rms(ref) cannot be met by any bf16 output of a tensor whose
+    largest elements lie far out in its tail: the exact value rounded to bf16 (the best a bf16 output can
+    be) already misses it. Shown on the oracle's exact weight gradient of a small expert (a few tokens make
+    dW_d a sum of a few outer products, heavy-tailed), with the rounding error inside the bound 2^-8 max|v|
+    that the format allows."""
+    wl = small(T=64, H=128, E=8, k=2, F=128)
+    inp = make_inputs(wl, seed=21, with_dy=True)
+    t = torch.arange(64)
+    idx = torch.stack([torch.zeros(64, dtype=torch.long), 2 + t % 6], dim=1).to(torch.int32)
+    idx[:2, 1] = 1                                           # expert 1 gets two tokens
+    g = torch.full((64, 2), 0.5, dtype=torch.float64)
+    small_e = 1
+    _, _, dWd = oracle.moe_bwd_expert_dw(inp["x"], inp["W_g"], inp["W_u"], inp["W_d"], inp["dY"], idx, g,
+                                         [small_e])
+    v = dWd[0]
+    rms = float(v.pow(2).mean().sqrt())
+    rounding = float((v.float().bfloat16().double() - v).abs().max())
+    assert rounding <= 2.0 ** -8 * float(v.abs().max())
+    assert rounding > 2e-2 * rms, (rounding / rms, float(v.abs().max()) / rms)
