@@ -109,6 +109,21 @@ MOE_DEV void tma_load_2d(void* smem_dst, const CUtensorMap* m, int x, int y, uin
 // Generic-proxy writes to shared memory -> visible to the async proxy (TMA, tensor core).
 MOE_DEV void fence_proxy_async_smem() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
 
+// TMA store of a shared-memory box to global (bulk-group completion), and the waits on those groups.
+MOE_DEV void tma_store_2d(const CUtensorMap* m, const void* smem_src, int x, int y) {
+  asm volatile("cp.async.bulk.tensor.2d.global.shared::cta.bulk_group [%0, {%1, %2}], [%3];" ::"l"(
+                   reinterpret_cast<uint64_t>(m)),
+               "r"(x), "r"(y), "r"(smem_u32(smem_src))
+               : "memory");
+}
+MOE_DEV void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
+template <int N>
+MOE_DEV void bulk_wait_read() {
+  asm volatile("cp.async.bulk.wait_group.read %0;" ::"n"(N) : "memory");
+}
+MOE_DEV void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
+
+
 // ------------------------------------------------------------------ tcgen05
 
 MOE_DEV void tmem_alloc(uint32_t* smem_dst, uint32_t ncols) {

@@ -53,6 +53,12 @@ struct __align__(64) Params {
   CUtensorMap tmA;
   CUtensorMap tmB0;
   CUtensorMap tmB1;
+  // GROUP_K bf16 output through TMA stores (tma_store != 0): C and C2 as [G * c_rows_per_group, N] bf16,
+  // no swizzle, 16-column x 32-row boxes
+  CUtensorMap tmC;
+  CUtensorMap tmC2;
+  long long c_rows_per_group;
+  int tma_store;
   int M;             // GROUP_M: total rows of A; otherwise the output row count
   int N;             // output columns (per group)
   int K;             // reduction length (GROUP_K: unused, per group from offsets)
@@ -77,15 +83,19 @@ struct __align__(64) Params {
   int* status;
 };
 
-template <int BN_, bool A_MN_, bool B_MN_, int EPI_, int GROUP_, int BMODE_>
+template <int BN_, bool A_MN_, bool B_MN_, int EPI_, int GROUP_, int BMODE_, bool TMA_ST_ = false>
 struct Cfg {
   static constexpr int BN = BN_;
+  // grouped along K with a bf16 output leaving through TMA stores: three TMA stages, and four 1 KB staging
+  // slices (32 rows x 16 columns) per epilogue warp, so that its stores stay in flight
+  static constexpr bool TMA_ST = TMA_ST_;
+  static constexpr int TMA_ST_BUFS = 4;
   static constexpr bool A_MN = A_MN_;
   static constexpr bool B_MN = B_MN_;
   static constexpr int EPI = EPI_;
   static constexpr int GROUP = GROUP_;
   static constexpr int BMODE = BMODE_;
-  static constexpr int kStages = (BN == 256) ? 4 : 6;
+  static constexpr int kStages = TMA_ST ? 3 : ((BN == 256) ? 4 : 6);
   static constexpr int A_BYTES = BM * BK * 2;
   static constexpr int B_BYTES = BN * BK * 2;
   static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
@@ -99,10 +109,12 @@ struct Cfg {
   // staging: per epilogue warp 32 rows x (64 + 16) bytes; the SwiGLU backward stages 16 columns of gate and of
   // up at a time, 32 rows x (32 + 16) bytes each, so that four TMA stages still fit
   static constexpr int STG_ROW = (EPI == EPI_SWIGLU_BWD) ? 48 : 80;
-  static constexpr int STG_BYTES = EPI_WARPS * 32 * STG_ROW * (EPI == EPI_SWIGLU_BWD ? 2 : 1);
+  static constexpr int STG_BYTES =
+      TMA_ST ? EPI_WARPS * TMA_ST_BUFS * 1024 : EPI_WARPS * 32 * STG_ROW * (EPI == EPI_SWIGLU_BWD ? 2 : 1);
   static constexpr int SMEM_BYTES = 1024 + kStages * STAGE_BYTES + BAR_BYTES + 2 * (MAX_G + 1) * 4 + 128 + STG_BYTES;
   static_assert(BN == 128 || BN == 256, "BN");
   static_assert(!(BMODE == B_SPLIT_N && B_MN), "split-N is for K-major weights");
+  static_assert(!TMA_ST || (GROUP == GROUP_K && EPI == EPI_BF16), "TMA-store epilogue: weight gradients");
 };
 
 struct Tile {
@@ -416,7 +428,9 @@ __global__ void __launch_bounds__(C::NUM_THREADS, 1) gemm_kernel(const __grid_co
     const int q = warp & 3;
     const int h = ew >> 2;
     const int row = q * 32 + lane;
-    uint8_t* stg = stg_area + ew * 32 * C::STG_ROW * (C::EPI == EPI_SWIGLU_BWD ? 2 : 1);
+    uint8_t* stg = stg_area + (C::TMA_ST ? ew * C::TMA_ST_BUFS * 1024
+                                         : ew * 32 * C::STG_ROW * (C::EPI == EPI_SWIGLU_BWD ? 2 : 1));
+    uint32_t stg_seq = 0;  // TMA stores issued by this warp (picks the staging slice)
     int acc = 0;
     uint32_t acc_phase = 0;
     for (int t = blockIdx.x; t < total && !aborted; t += gridDim.x) {
@@ -472,12 +486,14 @@ __global__ void __launch_bounds__(C::NUM_THREADS, 1) gemm_kernel(const __grid_co
         // 32 columns at a time: convert, stage in shared memory, store row-contiguously
         __nv_bfloat16* out_base;
         long long ld, rbase;
+        bool to_c2 = false;
         if constexpr (C::GROUP == GROUP_K) {
           rbase = ti.row0;
           __nv_bfloat16* base = reinterpret_cast<__nv_bfloat16*>(p.C);
           ld = p.ldc;
           if (p.c2_row_split > 0 && rbase >= p.c2_row_split) {  // whole tile on one side (split % 128 == 0)
             rbase -= p.c2_row_split;
+            to_c2 = true;
             base = reinterpret_cast<__nv_bfloat16*>(p.C2);
             ld = p.ldc2;
           }
@@ -499,6 +515,38 @@ __global__ void __launch_bounds__(C::NUM_THREADS, 1) gemm_kernel(const __grid_co
           } else {
 #pragma unroll
             for (int i = 0; i < 32; ++i) v[i] = 0.f;
+          }
+          if constexpr (C::TMA_ST) {
+            if (p.tma_store) {
+              // each 32-row x 16-column slice goes out through a TMA store from one of this warp's staging
+              // slices (a slice is rewritten once the store issued TMA_ST_BUFS slices earlier has read it)
+              if (32 * q >= ti.m_valid) break;  // warp-uniform: a 32-row block past the output (M % 32 == 0)
+              const CUtensorMap* tm = to_c2 ? &p.tmC2 : &p.tmC;
+              const int y = (int)(ti.g * p.c_rows_per_group + rbase + 32 * q);
+#pragma unroll
+              for (int pass = 0; pass < 2; ++pass) {
+                uint8_t* sl = stg + (stg_seq & (C::TMA_ST_BUFS - 1)) * 1024;
+                if (lane == 0) bulk_wait_read<C::TMA_ST_BUFS - 1>();
+                __syncwarp();
+                *reinterpret_cast<uint4*>(sl + lane * 32) =
+                    make_uint4(pack_bf16x2(v[16 * pass], v[16 * pass + 1]), pack_bf16x2(v[16 * pass + 2], v[16 * pass + 3]),
+                               pack_bf16x2(v[16 * pass + 4], v[16 * pass + 5]),
+                               pack_bf16x2(v[16 * pass + 6], v[16 * pass + 7]));
+                *reinterpret_cast<uint4*>(sl + lane * 32 + 16) =
+                    make_uint4(pack_bf16x2(v[16 * pass + 8], v[16 * pass + 9]),
+                               pack_bf16x2(v[16 * pass + 10], v[16 * pass + 11]),
+                               pack_bf16x2(v[16 * pass + 12], v[16 * pass + 13]),
+                               pack_bf16x2(v[16 * pass + 14], v[16 * pass + 15]));
+                fence_proxy_async_smem();  // the generic-proxy writes, for the TMA engine's reads
+                __syncwarp();
+                if (lane == 0) {
+                  tma_store_2d(tm, sl, ti.n0 + c + 16 * pass, y);
+                  bulk_commit();
+                }
+                ++stg_seq;
+              }
+              continue;
+            }
           }
 #pragma unroll
           for (int j = 0; j < 4; ++j)
@@ -650,6 +698,7 @@ __global__ void __launch_bounds__(C::NUM_THREADS, 1) gemm_kernel(const __grid_co
     }
   }
 
+  if (C::TMA_ST && warp >= 2 && lane == 0) bulk_wait_all();  // every TMA store has read its slice and landed
   __syncthreads();
   if (warp == 1) {
     tc_fence_after();

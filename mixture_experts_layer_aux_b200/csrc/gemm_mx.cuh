@@ -263,20 +263,6 @@ MOE_DEV void quant32(const float* v, float inv, uint32_t (&w)[8]) {
   }
 }
 
-// TMA store of a shared-memory box to global (bulk-group completion), and the waits on those groups.
-MOE_DEV void tma_store_2d(const CUtensorMap* m, const void* smem_src, int x, int y) {
-  asm volatile("cp.async.bulk.tensor.2d.global.shared::cta.bulk_group [%0, {%1, %2}], [%3];" ::"l"(
-                   reinterpret_cast<uint64_t>(m)),
-               "r"(x), "r"(y), "r"(smem_u32(smem_src))
-               : "memory");
-}
-MOE_DEV void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
-template <int N>
-MOE_DEV void bulk_wait_read() {
-  asm volatile("cp.async.bulk.wait_group.read %0;" ::"n"(N) : "memory");
-}
-MOE_DEV void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
-
 template <int EPI, bool SPLIT_N, bool GK, bool NV>
 __global__ void __launch_bounds__(NUM_THREADS, 1) gemm_mx_kernel(const __grid_constant__ Params p) {
   static_assert(!(NV && GK), "NVFP4: forward GEMMs only");

@@ -28,6 +28,14 @@ using gg::Cfg;
 // opt-in: MOE_B200_PAIR_MIN_ROWS=n selects it for GEMMs whose experts average
 // at least n rows. On B200 it matches the one-SM kernel on aligned experts and
 // loses on ragged ones (its 256-row tiles waste more rows at each expert's end).
+static bool wgrad_tma_store() {
+  static const bool v = [] {
+    const char* e = std::getenv("MOE_B200_WGRAD_TMA_STORE");
+    return !(e && std::atoi(e) == 0);
+  }();
+  return v;
+}
+
 static bool use_pair_kernel(int rows, int groups) {
   long long thr = 1LL << 40;
   if (const char* e = std::getenv("MOE_B200_PAIR_MIN_ROWS")) thr = std::atoll(e);
@@ -160,6 +168,21 @@ int gemm_wgrad(int rows, int groups, int M, int N, const void* dO, int ld_dO, co
   p.c_group_stride = (long long)(split > 0 ? split : M) * N;
   p.status = moe_host::device_status_ptr();
   const int tiles = groups * ((M + 127) / 128) * (N / 256);
+  // the bf16 weight gradients through TMA stores: [groups * rows per group, N], 16 x 32 boxes (whole 32-row
+  // blocks); MOE_B200_WGRAD_TMA_STORE=0 keeps the epilogue's own stores
+  const long long rpg = split > 0 ? split : M;
+  const bool al = ((reinterpret_cast<uintptr_t>(C) | reinterpret_cast<uintptr_t>(C2 ? C2 : C)) & 15u) == 0;
+  if (wgrad_tma_store() && M % 32 == 0 && split % 32 == 0 && N % 8 == 0 && al &&
+      (long long)groups * rpg < (1LL << 31)) {
+    if (!moe_host::encode_tmap_2d_plain(&p.tmC, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, C, N, (uint64_t)groups * rpg,
+                                        (uint64_t)N * 2, 16, 32) ||
+        !moe_host::encode_tmap_2d_plain(&p.tmC2, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, C2 ? C2 : C, N,
+                                        (uint64_t)groups * rpg, (uint64_t)N * 2, 16, 32))
+      return MOE_ERR_CUDA;
+    p.c_rows_per_group = rpg;
+    p.tma_store = 1;
+    return gg::launch<Cfg<256, true, true, gg::EPI_BF16, gg::GROUP_K, gg::B_SINGLE, true>>(p, tiles, st);
+  }
   return gg::launch<Cfg<256, true, true, gg::EPI_BF16, gg::GROUP_K, gg::B_SINGLE>>(p, tiles, st);
 }
 
