@@ -94,6 +94,9 @@ WORKLOADS = {
     # the MXFP8 layer on the same small case (~1.9 GB on the device): the full ncu capture of the MXFP8 GEMM
     "dsv3-e64": Workload("dsv3-e64", T=2048, H=7168, E=64, k=8, F=2048, S=1, score="sigmoid", route_scale=2.5,
                          dtype="mxfp8", aux=False),
+    # the token-side traffic of the Qwen3 shape (T=8192, H=4096, k=8) on 16 small experts, about 1.5 GB on the
+    # device: the small case of the permutation and unpermute kernels' DRAM captures
+    "qwen3-mem": Workload("qwen3-mem", T=8192, H=4096, E=16, k=8, F=512),
     # the MXFP8 backward on the DeepSeek-V3 routed experts (the backward has no shared expert)
     "dsv3-train": Workload("dsv3-train", T=8192, H=7168, E=256, k=8, F=2048, score="sigmoid", route_scale=2.5,
                            dtype="mxfp8", aux=False, bwd=True),
