@@ -113,29 +113,59 @@ __global__ void __launch_bounds__(512) scan_kernel(const int* __restrict__ hist,
                                                    int32_t* __restrict__ offsets) {
   __shared__ int s[512];
   const int e = threadIdx.x;
+  // the expert's per-block counts are read eight at a time, so their latencies overlap
+  constexpr int U = 8;
   int run = 0;
   if (e < E) {
-    for (int b = 0; b < nblk; ++b) {
-      base[(long long)b * E + e] = run;
-      run += hist[(long long)b * E + e];
+    for (int b0 = 0; b0 < nblk; b0 += U) {
+      int h[U];
+#pragma unroll
+      for (int i = 0; i < U; ++i) h[i] = (b0 + i < nblk) ? hist[(long long)(b0 + i) * E + e] : 0;
+#pragma unroll
+      for (int i = 0; i < U; ++i) run += h[i];
     }
     run = min(run, cap);
     if (counts) counts[e] = run;
   }
-  s[e] = (e < E) ? run : 0;
-  __syncthreads();
-  for (int o = 1; o < 512; o <<= 1) {  // inclusive Hillis-Steele scan
-    const int v = (e >= o) ? s[e - o] : 0;
-    __syncthreads();
-    s[e] += v;
-    __syncthreads();
+  // inclusive scan over the 512 experts: within each warp by shuffles, then over the 16 warp totals
+  const int lane = e & 31, w = e >> 5;
+  int incl = (e < E) ? run : 0;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int v = __shfl_up_sync(0xffffffffu, incl, o);
+    if (lane >= o) incl += v;
   }
-  const int excl = s[e] - ((e < E) ? run : 0);
+  if (lane == 31) s[w] = incl;
+  __syncthreads();
+  if (w == 0) {
+    int t = lane < 16 ? s[lane] : 0;
+#pragma unroll
+    for (int o = 1; o < 16; o <<= 1) {
+      const int v = __shfl_up_sync(0xffffffffu, t, o);
+      if (lane >= o) t += v;
+    }
+    if (lane < 16) s[16 + lane] = t;  // inclusive totals of warps 0..lane
+  }
+  __syncthreads();
+  incl += (w > 0) ? s[16 + w - 1] : 0;
+  const int excl = incl - ((e < E) ? run : 0);
   if (e < E) {
     offsets[e] = excl;
-    for (int b = 0; b < nblk; ++b) base[(long long)b * E + e] += excl;
+    // base[b, e] = offsets[e] + the counts of the blocks before b (unclamped: past the capacity is dropped)
+    int acc = excl;
+    for (int b0 = 0; b0 < nblk; b0 += U) {
+      int h[U];
+#pragma unroll
+      for (int i = 0; i < U; ++i) h[i] = (b0 + i < nblk) ? hist[(long long)(b0 + i) * E + e] : 0;
+#pragma unroll
+      for (int i = 0; i < U; ++i)
+        if (b0 + i < nblk) {
+          base[(long long)(b0 + i) * E + e] = acc;
+          acc += h[i];
+        }
+    }
   }
-  if (e == E - 1) offsets[E] = s[e];
+  if (e == E - 1) offsets[E] = incl;
 }
 
 __device__ __forceinline__ uint8_t mx_scale_byte(float amax) {
