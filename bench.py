@@ -426,7 +426,7 @@ class Layer:
 
     def launches_per_step(self):
         """Kernels of ours launched per step (as the ncu launch list shows them): router GEMM,
-        top-k, finalize (+ aux when computed), rank, scan, scatter, gate/up GEMM, down GEMM,
+        top-k, finalize (+ aux when computed), rank, scan, permute, gate/up GEMM, down GEMM,
         unpermute; + the shared expert's two GEMMs (and, block-scaled, its input quantiser); and
         for fwd+bwd the nine kernels of moe_layer_bwd (dY gather, down dgrad with the SwiGLU
         backward, two weight-gradient GEMMs, gate/up dgrad, router backward, two router

@@ -19,6 +19,7 @@ enum MoeDevStatus : int {
   DEV_WAIT_TIMEOUT_MMA = 0x102,
   DEV_WAIT_TIMEOUT_EPILOGUE = 0x103,
   DEV_WAIT_TIMEOUT_DRAIN = 0x104,
+  DEV_WAIT_TIMEOUT_COPY = 0x105,  // a bulk global->shared copy did not land
   DEV_BAD_OFFSETS = 0x201,
   DEV_BAD_INDEX = 0x202,
 };
@@ -105,6 +106,13 @@ MOE_DEV void tma_load_2d(void* smem_dst, const CUtensorMap* m, int x, int y, uin
       "l"(reinterpret_cast<uint64_t>(m)), "r"(x), "r"(y), "r"(smem_u32(bar))
       : "memory");
 }
+
+// Programmatic dependent launch: a kernel launched with programmatic stream serialisation may start
+// while its predecessor in the stream still runs (once every predecessor CTA has called
+// griddep_launch_dependents or exited); griddep_wait blocks until the predecessor has completed and
+// its memory writes are visible. Both are no-ops for a kernel launched the ordinary way.
+MOE_DEV void griddep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+MOE_DEV void griddep_launch_dependents() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
 
 // Generic-proxy writes to shared memory -> visible to the async proxy (TMA, tensor core).
 MOE_DEV void fence_proxy_async_smem() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }

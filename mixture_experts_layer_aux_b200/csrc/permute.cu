@@ -12,12 +12,18 @@
 //            expert (a lane bitmask per expert in shared memory, popc of the
 //            lanes below), a per-expert scan over the warps turns that into the
 //            stable in-block rank of every (t, j), and the block's histogram.
-//   scan     one block: counts, exclusive-scan offsets, per-block bases.
-//   scatter  one warp per token: row = base[block, e] + rank; writes row_of,
-//            src_of, row_gate; copies the token's row once from HBM and writes
-//            it to its k destination rows with 16-byte vector stores
-//            (quantising each 1x32 block to MXFP8, or each 1x16 block to NVFP4,
-//            on the way when asked).
+//   scan     one block: counts, exclusive-scan offsets, and per rank block and
+//            expert the pair (first row, one past the expert's last kept row).
+//   permute  one warp per token, four per CTA: row = first row + rank; writes
+//            row_of, src_of, row_gate; copies the token's row once from HBM
+//            and writes it to its k destination rows with 16-byte vector
+//            stores (quantising each 1x32 block to MXFP8, or each 1x16 block to
+//            NVFP4, on the way when asked).
+//   scan and permute are programmatic dependent launches (outside stream
+//   capture): their CTAs start while the kernel before them runs, and the
+//   permute warps fetch their token's experts and row before they wait.
+//   scatter  the same copy for an existing map (row_of) of another [T, H]
+//            tensor.
 //   unpermute one warp per token: fp32 sum of its k rows in slot order, 16-byte
 //            loads, one bf16 rounding.
 #include <cuda_fp8.h>
@@ -38,6 +44,7 @@ constexpr int SC_WARPS = 8;    // warps per scatter / unpermute block
 __global__ void __launch_bounds__(RANK_WARPS * 32) rank_kernel(const int32_t* __restrict__ idx, int T, int E,
                                                                 int k, int32_t* __restrict__ lrank,
                                                                 int* __restrict__ hist, int* status) {
+  griddep_launch_dependents();  // the scan may start now: it waits for this kernel before reading its output
   extern __shared__ uint32_t s_rank[];
   uint32_t* mask = s_rank;                                         // [RANK_WARPS][E]: lanes holding expert e
   int* cnt = reinterpret_cast<int*>(s_rank + RANK_WARPS * E);      // [RANK_WARPS][E]: count, then warp base
@@ -105,24 +112,48 @@ __global__ void __launch_bounds__(RANK_WARPS * 32) rank_kernel(const int32_t* __
   }
 }
 
-// counts, offsets [E+1], base[b,e] = offsets[e] + sum_{b'<b} hist[b',e]. With an expert
-// capacity `cap`, counts and offsets count min(count, cap) kept rows per expert; a pair
-// whose row base + rank reaches offsets[e+1] is then a dropped one.
+// counts, offsets [E+1] and the per-rank-block table bt[b, e] = (first row of rank block b's pairs of
+// expert e = offsets[e] + sum_{b'<b} hist[b', e], one past the expert's last kept row = offsets[e+1]).
+// With an expert capacity `cap`, counts and offsets count min(count, cap) kept rows per expert; a pair whose
+// row reaches bt[b, e].y is a dropped one. One CTA, thread e = expert e. Launched as a programmatic
+// dependent of the rank kernel; the histograms are staged in shared memory by one pass of independent loads
+// when they fit (nblk * E <= SCAN_SMEM_INTS), else read twice from L2.
+constexpr int SCAN_SMEM_INTS = 12288;  // 48 KB
 __global__ void __launch_bounds__(512) scan_kernel(const int* __restrict__ hist, int nblk, int E, int cap,
-                                                   int* __restrict__ base, int32_t* __restrict__ counts,
+                                                   int2* __restrict__ bt, int32_t* __restrict__ counts,
                                                    int32_t* __restrict__ offsets) {
-  __shared__ int s[512];
+  griddep_launch_dependents();
+  extern __shared__ int sh[];  // staged histograms
+  __shared__ int s[32];
   const int e = threadIdx.x;
-  // the expert's per-block counts are read eight at a time, so their latencies overlap
+  griddep_wait();
+  const int nh = nblk * E;
+  const bool staged = nh <= SCAN_SMEM_INTS;
   constexpr int U = 8;
+  if (staged) {
+    for (int i0 = threadIdx.x; i0 < nh; i0 += 512 * U) {
+      int v[U];
+#pragma unroll
+      for (int u = 0; u < U; ++u) v[u] = (i0 + 512 * u < nh) ? __ldcg(hist + i0 + 512 * u) : 0;
+#pragma unroll
+      for (int u = 0; u < U; ++u)
+        if (i0 + 512 * u < nh) sh[i0 + 512 * u] = v[u];
+    }
+    __syncthreads();
+  }
   int run = 0;
   if (e < E) {
-    for (int b0 = 0; b0 < nblk; b0 += U) {
-      int h[U];
+    if (staged) {
+      for (int b = 0; b < nblk; ++b) run += sh[b * E + e];
+    } else {
+      // the expert's per-block counts, eight loads in flight at a time
+      for (int b0 = 0; b0 < nblk; b0 += U) {
+        int h[U];
 #pragma unroll
-      for (int i = 0; i < U; ++i) h[i] = (b0 + i < nblk) ? hist[(long long)(b0 + i) * E + e] : 0;
+        for (int i = 0; i < U; ++i) h[i] = (b0 + i < nblk) ? __ldcg(hist + (long long)(b0 + i) * E + e) : 0;
 #pragma unroll
-      for (int i = 0; i < U; ++i) run += h[i];
+        for (int i = 0; i < U; ++i) run += h[i];
+      }
     }
     run = min(run, cap);
     if (counts) counts[e] = run;
@@ -151,18 +182,25 @@ __global__ void __launch_bounds__(512) scan_kernel(const int* __restrict__ hist,
   const int excl = incl - ((e < E) ? run : 0);
   if (e < E) {
     offsets[e] = excl;
-    // base[b, e] = offsets[e] + the counts of the blocks before b (unclamped: past the capacity is dropped)
+    // first rows: offsets[e] + the counts of the blocks before b (unclamped: past the capacity is dropped)
     int acc = excl;
-    for (int b0 = 0; b0 < nblk; b0 += U) {
-      int h[U];
+    if (staged) {
+      for (int b = 0; b < nblk; ++b) {
+        bt[(long long)b * E + e] = make_int2(acc, incl);
+        acc += sh[b * E + e];
+      }
+    } else {
+      for (int b0 = 0; b0 < nblk; b0 += U) {
+        int h[U];
 #pragma unroll
-      for (int i = 0; i < U; ++i) h[i] = (b0 + i < nblk) ? hist[(long long)(b0 + i) * E + e] : 0;
+        for (int i = 0; i < U; ++i) h[i] = (b0 + i < nblk) ? __ldcg(hist + (long long)(b0 + i) * E + e) : 0;
 #pragma unroll
-      for (int i = 0; i < U; ++i)
-        if (b0 + i < nblk) {
-          base[(long long)(b0 + i) * E + e] = acc;
-          acc += h[i];
-        }
+        for (int i = 0; i < U; ++i)
+          if (b0 + i < nblk) {
+            bt[(long long)(b0 + i) * E + e] = make_int2(acc, incl);
+            acc += h[i];
+          }
+      }
     }
   }
   if (e == E - 1) offsets[E] = incl;
@@ -195,111 +233,222 @@ __device__ __forceinline__ uint2 quant8(const float (&f)[8], float inv) {
   return make_uint2(w[0], w[1]);
 }
 
-// MODE 0: rows computed here from (idx, lrank, base) -- the permute itself.
-// MODE 1: rows read from row_of -- a plain scatter of another [T,H] tensor.
-// QF: what is written -- bf16 rows (QF_BF16), MXFP8 rows (QF_MX: e4m3 [rows, H] + ue8m0 per 32) or NVFP4 rows
-// (QF_NV: packed e2m1 [rows, H/2] + e4m3 per 16, tensor scale 1).
+// What a scatter writes: bf16 rows (QF_BF16), MXFP8 rows (QF_MX: e4m3 [rows, H] + ue8m0 per 32) or NVFP4
+// rows (QF_NV: packed e2m1 [rows, H/2] + e4m3 per 16, tensor scale 1).
 enum { QF_BF16 = 0, QF_MX = 1, QF_NV = 2 };
-template <int MODE, int QF>
-__global__ void __launch_bounds__(SC_WARPS * 32) scatter_kernel(
-    const __nv_bfloat16* __restrict__ x, int T, int H, int E, int k, const int32_t* __restrict__ idx,
-    const int32_t* __restrict__ lrank, const int* __restrict__ base, const int32_t* __restrict__ offsets,
-    const float* __restrict__ gates,
-    int32_t* __restrict__ row_of, int32_t* __restrict__ src_of, float* __restrict__ row_gate, void* __restrict__ xp,
-    uint8_t* __restrict__ xp_sf) {
+constexpr int SC_U = 4;  // 16-byte chunks per lane held in registers before any is written
+
+// One 8-element chunk (16 bytes) of a token's row, chunk i of nchunk, to the token's k destination rows
+// (rows[j] < 0: no destination). Called by all 32 lanes of the warp together (the quantising forms
+// reduce the block amax across lanes); chunks past nchunk are computed but not stored.
+template <int QF>
+__device__ __forceinline__ void emit_chunk(const int (&rows)[16], int k, int H, int nchunk, int i, const uint4 d,
+                                           void* __restrict__ xp, uint8_t* __restrict__ xp_sf) {
+  const bool v = i < nchunk;
+  if constexpr (QF == QF_BF16) {
+    if (v) {
+#pragma unroll
+      for (int j = 0; j < 16; ++j)
+        if (j < k && rows[j] >= 0)
+          reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(xp) + (long long)rows[j] * H)[i] = d;
+    }
+  } else if constexpr (QF == QF_NV) {
+    // a 16-block is the 8-element chunks of lanes 2m and 2m+1 (H % 16 == 0, so pairs share validity)
+    float f[8];
+    unpack_bf16x8(d, f);
+    float am = 0.f;
+#pragma unroll
+    for (int q = 0; q < 8; ++q) am = fmaxf(am, fabsf(f[q]));
+    am = fmaxf(am, __shfl_xor_sync(0xffffffffu, am, 1));
+    const uint8_t sb = nvq::scale_byte(am, 1.0f);
+    const uint32_t w = nvq::pack8(f, nvq::elem_mult(sb, 1.0f));
+    if (v) {
+#pragma unroll
+      for (int j = 0; j < 16; ++j)
+        if (j < k && rows[j] >= 0) {
+          reinterpret_cast<uint32_t*>(static_cast<uint8_t*>(xp) + (long long)rows[j] * (H / 2))[i] = w;
+          if ((i & 1) == 0) xp_sf[(long long)rows[j] * (H / 16) + (i >> 1)] = sb;
+        }
+    }
+  } else {
+    float f[8];
+    unpack_bf16x8(d, f);
+    float am = 0.f;
+#pragma unroll
+    for (int q = 0; q < 8; ++q) am = fmaxf(am, fabsf(f[q]));
+    am = fmaxf(am, __shfl_xor_sync(0xffffffffu, am, 1));
+    am = fmaxf(am, __shfl_xor_sync(0xffffffffu, am, 2));
+    const uint8_t sb = mx_scale_byte(am);
+    const uint2 codes = quant8(f, mx_inv_scale(sb));
+    if (v) {
+#pragma unroll
+      for (int j = 0; j < 16; ++j)
+        if (j < k && rows[j] >= 0) {
+          reinterpret_cast<uint2*>(static_cast<uint8_t*>(xp) + (long long)rows[j] * H)[i] = codes;
+          if ((i & 3) == 0) xp_sf[(long long)rows[j] * (H / 32) + (i >> 2)] = sb;
+        }
+    }
+  }
+}
+
+// Plain scatter of a [T, H] tensor by an existing map: row_of[t, j] (< 0: none). One warp per token; the
+// row is read once, SC_U chunks per lane in flight before any is written.
+template <int QF>
+__global__ void __launch_bounds__(SC_WARPS * 32, 4) scatter_kernel(const __nv_bfloat16* __restrict__ x, int T,
+                                                                   int H, int k, const int32_t* __restrict__ row_of,
+                                                                   void* __restrict__ xp,
+                                                                   uint8_t* __restrict__ xp_sf) {
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int t = blockIdx.x * SC_WARPS + warp;
   if (t >= T) return;
   const int rows_total = T * k;
   int r = -1;
   if (lane < k) {
-    if (MODE == 0) {
-      const int e = idx[(long long)t * k + lane];
-      const int lr = lrank[(long long)t * k + lane];
-      if (e >= 0 && e < E && lr >= 0) {
-        r = base[(long long)(t / RANK_TOK) * E + e] + lr;
-        if (r >= offsets[e + 1]) r = -1;  // past the expert's capacity: dropped
-      }
-      row_of[(long long)t * k + lane] = r;
-      if (r >= 0) {
-        src_of[r] = t;
-        if (row_gate) row_gate[r] = gates[(long long)t * k + lane];
-      }
-    } else {
-      r = row_of[(long long)t * k + lane];
-      if (r < 0 || r >= rows_total) r = -1;
-    }
+    r = row_of[(long long)t * k + lane];
+    if (r < 0 || r >= rows_total) r = -1;
   }
-  if (xp == nullptr) return;
   int rows[16];
 #pragma unroll
   for (int j = 0; j < 16; ++j) rows[j] = __shfl_sync(0xffffffffu, r, j < k ? j : 0);
   const uint4* src = reinterpret_cast<const uint4*>(x + (long long)t * H);
   const int nchunk = H / 8;
-  // one 8-element chunk (16 bytes) of the row, to its k destinations
-  auto emit = [&](const int i, const uint4 d) {
-    const bool v = i < nchunk;
-    if constexpr (QF == QF_BF16) {
-      if (v) {
+  for (int i0 = 0; i0 < nchunk; i0 += 32 * SC_U) {
+    uint4 d[SC_U];
 #pragma unroll
-        for (int j = 0; j < 16; ++j)
-          if (j < k && rows[j] >= 0)
-            reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(xp) + (long long)rows[j] * H)[i] = d;
-      }
-    } else if constexpr (QF == QF_NV) {
-      // a 16-block is the 8-element chunks of lanes 2m and 2m+1 (H % 16 == 0, so pairs share validity)
-      float f[8];
-      unpack_bf16x8(d, f);
-      float am = 0.f;
-#pragma unroll
-      for (int q = 0; q < 8; ++q) am = fmaxf(am, fabsf(f[q]));
-      am = fmaxf(am, __shfl_xor_sync(0xffffffffu, am, 1));
-      const uint8_t sb = nvq::scale_byte(am, 1.0f);
-      const uint32_t w = nvq::pack8(f, nvq::elem_mult(sb, 1.0f));
-      if (v) {
-#pragma unroll
-        for (int j = 0; j < 16; ++j)
-          if (j < k && rows[j] >= 0) {
-            reinterpret_cast<uint32_t*>(static_cast<uint8_t*>(xp) + (long long)rows[j] * (H / 2))[i] = w;
-            if ((i & 1) == 0) xp_sf[(long long)rows[j] * (H / 16) + (i >> 1)] = sb;
-          }
-      }
-    } else {
-      float f[8];
-      unpack_bf16x8(d, f);
-      float am = 0.f;
-#pragma unroll
-      for (int q = 0; q < 8; ++q) am = fmaxf(am, fabsf(f[q]));
-      am = fmaxf(am, __shfl_xor_sync(0xffffffffu, am, 1));
-      am = fmaxf(am, __shfl_xor_sync(0xffffffffu, am, 2));
-      const uint8_t sb = mx_scale_byte(am);
-      const uint2 codes = quant8(f, mx_inv_scale(sb));
-      if (v) {
-#pragma unroll
-        for (int j = 0; j < 16; ++j)
-          if (j < k && rows[j] >= 0) {
-            reinterpret_cast<uint2*>(static_cast<uint8_t*>(xp) + (long long)rows[j] * H)[i] = codes;
-            if ((i & 3) == 0) xp_sf[(long long)rows[j] * (H / 32) + (i >> 2)] = sb;
-          }
-      }
-    }
-  };
-  // four chunks per lane in flight before any is written (the row is read once; the writes dominate)
-  constexpr int U = 4;
-  for (int i0 = 0; i0 < nchunk; i0 += 32 * U) {
-    uint4 d[U];
-#pragma unroll
-    for (int u = 0; u < U; ++u) {
+    for (int u = 0; u < SC_U; ++u) {
       const int i = i0 + 32 * u + lane;
       d[u] = i < nchunk ? src[i] : make_uint4(0, 0, 0, 0);
     }
 #pragma unroll
-    for (int u = 0; u < U; ++u) emit(i0 + 32 * u + lane, d[u]);
+    for (int u = 0; u < SC_U; ++u) emit_chunk<QF>(rows, k, H, nchunk, i0 + 32 * u + lane, d[u], xp, xp_sf);
   }
 }
 
-template <int KM>  // compile-time bound on k: the per-slot arrays hold KM entries
-__global__ void __launch_bounds__(SC_WARPS * 32) unpermute_kernel(const __nv_bfloat16* __restrict__ o,
+// The permutation's gather / scatter: one warp per token, PW_WARPS tokens per CTA.
+//
+// Launched as a programmatic dependent of the scan kernel, so its CTAs start while the rank and scan kernels
+// run. Before waiting, each warp fetches what does not depend on the ranks: the token's k experts, the first
+// 32 * SC_U chunks of its row into registers, and (lane 0, one bulk copy) the rest of the row into its
+// shared-memory slot. The row reads thus overlap the ranking. After the wait the CTA reads the one row of
+// the scan's table that its rank block owns (E (first row, end) pairs: a few contiguous lines per CTA, so
+// the CTAs do not all read the same lines), each warp computes its k rows = first row + in-block rank (a
+// pair whose row reaches its expert's end is dropped: capacity) and writes them.
+constexpr int PW_WARPS = 4;
+constexpr int PW_THREADS = PW_WARPS * 32;
+constexpr int STAGE_MAX_CHUNKS = 384;  // 6 KB per warp (8 CTAs per SM); chunks past it (H > 4096) are read after the wait
+
+// dynamic shared memory of permute_kernel: barriers, the rank block's (first row, end) pairs, then one row
+// slot per warp
+struct PermSmem {
+  int stage_bytes;  // per warp: the row past the register chunks (at most STAGE_MAX_CHUNKS), 128-byte multiple
+  int bt_off, rows_off, total;
+};
+__host__ __device__ inline PermSmem perm_smem(int H, int E) {
+  PermSmem m;
+  const int rest = min(H / 8 - 32 * SC_U, STAGE_MAX_CHUNKS);
+  m.stage_bytes = rest > 0 ? ((rest * 16 + 127) / 128) * 128 : 0;
+  m.bt_off = 128;  // PW_WARPS mbarriers first
+  m.rows_off = ((m.bt_off + 8 * E + 127) / 128) * 128;
+  m.total = m.rows_off + PW_WARPS * m.stage_bytes;
+  return m;
+}
+
+template <int QF>
+__global__ void __launch_bounds__(PW_THREADS, QF == QF_BF16 ? 8 : 7) permute_kernel(
+    const __nv_bfloat16* __restrict__ x, int T, int H, int E, int k, const int32_t* __restrict__ idx,
+    const int32_t* __restrict__ lrank, const int2* __restrict__ bt, const float* __restrict__ gates,
+    int32_t* __restrict__ row_of, int32_t* __restrict__ src_of, float* __restrict__ row_gate, void* __restrict__ xp,
+    uint8_t* __restrict__ xp_sf, int* status) {
+  extern __shared__ __align__(128) uint8_t sm[];
+  const PermSmem L = perm_smem(H, E);
+  uint64_t* bar = reinterpret_cast<uint64_t*>(sm);
+  int2* s_bt = reinterpret_cast<int2*>(sm + L.bt_off);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int t = blockIdx.x * PW_WARPS + warp;
+  const bool tv = t < T;
+  const int nchunk = H / 8;
+  const bool copy = xp != nullptr && tv;
+  const uint4* src = reinterpret_cast<const uint4*>(x + (long long)(tv ? t : 0) * H);
+  uint8_t* slot = sm + L.rows_off + warp * L.stage_bytes;
+  const int n_staged = max(0, min(nchunk - 32 * SC_U, STAGE_MAX_CHUNKS));  // chunks in the shared-memory slot
+  const uint32_t rest_bytes = (uint32_t)n_staged * 16u;
+  const bool staged = copy && rest_bytes > 0;
+
+  // ---- independent of the ranks: experts, the row's first chunks, the bulk copy of the rest
+  if (lane == 0) {
+    mbar_init(&bar[warp], 1);
+    fence_mbar_init();
+  }
+  __syncwarp();
+  if (staged && lane == 0) {
+    mbar_arrive_expect_tx(&bar[warp], rest_bytes);
+    bulk_load(slot, src + 32 * SC_U, rest_bytes, &bar[warp]);
+  }
+  int e = -1;
+  if (tv && lane < k) e = idx[(long long)t * k + lane];
+  uint4 d[SC_U];
+#pragma unroll
+  for (int u = 0; u < SC_U; ++u) {
+    const int i = 32 * u + lane;
+    d[u] = (copy && i < nchunk) ? src[i] : make_uint4(0, 0, 0, 0);
+  }
+
+  griddep_wait();
+
+  // ---- the rank block's (first row, end) pairs, and this token's rows and maps
+  int lr = -1;
+  if (tv && lane < k) lr = __ldcg(lrank + (long long)t * k + lane);
+  const int rb = (blockIdx.x * PW_WARPS) / RANK_TOK;
+  for (int ee = threadIdx.x; ee < E; ee += PW_THREADS) s_bt[ee] = __ldcg(bt + (long long)rb * E + ee);
+  __syncthreads();
+  int r = -1;
+  if (tv && lane < k) {
+    if (e >= 0 && e < E && lr >= 0) {
+      const int2 be = s_bt[e];
+      r = be.x + lr;
+      if (r >= be.y) r = -1;  // past the expert's capacity: dropped
+    }
+    row_of[(long long)t * k + lane] = r;
+    if (r >= 0) {
+      src_of[r] = t;
+      if (row_gate) row_gate[r] = gates[(long long)t * k + lane];
+    }
+  }
+  if (!copy) return;
+  int rows[16];
+#pragma unroll
+  for (int j = 0; j < 16; ++j) rows[j] = __shfl_sync(0xffffffffu, r, j < k ? j : 0);
+#pragma unroll
+  for (int u = 0; u < SC_U; ++u) emit_chunk<QF>(rows, k, H, nchunk, 32 * u + lane, d[u], xp, xp_sf);
+  if (!staged) return;
+  // ---- the rest of the row, from its shared-memory slot (bounded wait for the bulk copy)
+  bool ok = mbar_try_wait(&bar[warp], 0);
+  if (!ok) {
+    const uint64_t t0 = globaltimer_ns();
+    while (!(ok = mbar_try_wait(&bar[warp], 0)) && globaltimer_ns() - t0 < MOE_WAIT_NS) {
+    }
+  }
+  if (!__all_sync(0xffffffffu, ok)) {
+    // nothing is written from the slot; the copy must still land before the CTA may exit
+    if (lane == 0) record_status(status, DEV_WAIT_TIMEOUT_COPY);
+    const uint64_t t0 = globaltimer_ns();
+    while (!mbar_try_wait(&bar[warp], 0) && globaltimer_ns() - t0 < MOE_WAIT_NS) {
+    }
+    return;
+  }
+  const uint4* s4 = reinterpret_cast<const uint4*>(slot);
+  const int staged_end = 32 * SC_U + n_staged;
+  for (int i0 = 32 * SC_U; i0 < nchunk; i0 += 32) {
+    const int i = i0 + lane;
+    const uint4 v = i < staged_end ? s4[i - 32 * SC_U] : (i < nchunk ? src[i] : make_uint4(0, 0, 0, 0));
+    emit_chunk<QF>(rows, k, H, nchunk, i, v, xp, xp_sf);
+  }
+}
+
+// KM: compile-time bound on k (the per-slot arrays hold KM entries); EX: an extra [T, H] term is added
+// (four CTAs per SM where the registers allow: one wave for 4096 tokens)
+template <int KM, bool EX>
+__global__ void __launch_bounds__(SC_WARPS * 32, KM > 8 ? 1 : ((KM == 2 && EX) ? 3 : 4)) unpermute_kernel(const __nv_bfloat16* __restrict__ o,
                                                                   const int32_t* __restrict__ row_of,
                                                                   const __nv_bfloat16* __restrict__ extra, int T,
                                                                   int H, int k, __nv_bfloat16* __restrict__ y) {
@@ -330,8 +479,8 @@ __global__ void __launch_bounds__(SC_WARPS * 32) unpermute_kernel(const __nv_bfl
         if (j < k)
           d[u][j] = (i < nchunk && rows[j] >= 0) ? reinterpret_cast<const uint4*>(o + (long long)rows[j] * H)[i]
                                                  : make_uint4(0, 0, 0, 0);
-      ex[u] = (extra && i < nchunk) ? reinterpret_cast<const uint4*>(extra + (long long)t * H)[i]
-                                    : make_uint4(0, 0, 0, 0);
+      if constexpr (EX)
+        ex[u] = (i < nchunk) ? reinterpret_cast<const uint4*>(extra + (long long)t * H)[i] : make_uint4(0, 0, 0, 0);
     }
 #pragma unroll
     for (int u = 0; u < UNP_ILP; ++u) {
@@ -348,7 +497,7 @@ __global__ void __launch_bounds__(SC_WARPS * 32) unpermute_kernel(const __nv_bfl
 #pragma unroll
           for (int q = 0; q < 8; ++q) acc[q] += f[q];
         }
-      if (extra) {
+      if constexpr (EX) {
         float f[8];
         unpack_bf16x8(ex[u], f);
 #pragma unroll
@@ -396,11 +545,43 @@ __global__ void fill_offsets2_kernel(int32_t* off, int n) {
 
 static bool al16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
+namespace {
+
+// A launch that may overlap the kernel before it in the stream (programmatic dependent launch). Not while
+// the stream is being captured: measured on B200, replaying a graph of the Mixtral-shaped step whose
+// permutation kernels carry the programmatic edges took 2.42-2.45 ms against 2.36-2.37 ms without them.
+template <typename... KArgs, typename... Args>
+cudaError_t launch_dep(void (*kern)(KArgs...), int grid, int block, int smem, cudaStream_t st, Args... args) {
+  cudaStreamCaptureStatus cap = cudaStreamCaptureStatusNone;
+  if (cudaStreamIsCapturing(st, &cap) != cudaSuccess) {
+    (void)cudaGetLastError();
+    cap = cudaStreamCaptureStatusActive;  // unknown: launch the ordinary way
+  }
+  if (smem > 48 * 1024) {
+    const cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (e != cudaSuccess) return e;
+  }
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(grid);
+  cfg.blockDim = dim3(block);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = cap == cudaStreamCaptureStatusNone ? 1 : 0;
+  return cudaLaunchKernelEx(&cfg, kern, static_cast<KArgs>(args)...);
+}
+
+}  // namespace
+
 namespace moe_impl {
 
 size_t permute_ws(const moe_config* c) {
   const size_t nblk = (c->T + perm::RANK_TOK - 1) / perm::RANK_TOK;
-  return ws_round((size_t)c->T * c->k * sizeof(int32_t)) + 2 * ws_round(nblk * c->E * sizeof(int));
+  return ws_round((size_t)c->T * c->k * sizeof(int32_t)) + ws_round(nblk * c->E * sizeof(int)) +
+         ws_round(nblk * c->E * sizeof(int2));
 }
 
 int permute(const moe_config* c, const void* x, const int32_t* idx, const float* gates, int32_t* counts,
@@ -419,7 +600,7 @@ int permute(const moe_config* c, const void* x, const int32_t* idx, const float*
   Carve cv(ws);
   int32_t* lrank = cv.take<int32_t>((size_t)c->T * c->k);
   int* hist = cv.take<int>((size_t)nblk * c->E);
-  int* base = cv.take<int>((size_t)nblk * c->E);
+  int2* bt = cv.take<int2>((size_t)nblk * c->E);
   int* status = moe_host::device_status_ptr();
   perm::rank_kernel<<<nblk, perm::RANK_WARPS * 32, 2 * perm::RANK_WARPS * c->E * sizeof(uint32_t), st>>>(
       idx, c->T, c->E, c->k, lrank, hist, status);
@@ -430,30 +611,41 @@ int permute(const moe_config* c, const void* x, const int32_t* idx, const float*
     const double cd = std::ceil((double)c->capacity_factor * c->T * c->k / c->E);
     if (cd < (double)cap) cap = (int)cd;
   }
-  perm::scan_kernel<<<1, 512, 0, st>>>(hist, nblk, c->E, cap, base, counts, offsets);
-  MOE_CHECK_LAUNCH();
-  const int sgrid = (c->T + perm::SC_WARPS - 1) / perm::SC_WARPS;
+  // scan and permute each start while the kernel before them runs (programmatic dependent launches)
+  const int nh = nblk * c->E;
+  const int scan_smem = nh <= perm::SCAN_SMEM_INTS ? nh * (int)sizeof(int) : 0;
+  cudaError_t err = launch_dep(perm::scan_kernel, 1, 512, scan_smem, st, (const int*)hist, nblk, c->E, cap, bt,
+                               counts, offsets);
+  if (err != cudaSuccess) {
+    (void)cudaGetLastError();
+    return MOE_ERR_CUDA;
+  }
+  const int pgrid = (c->T + perm::PW_WARPS - 1) / perm::PW_WARPS;
+  const auto* x16 = static_cast<const __nv_bfloat16*>(x);
+  const int smem = perm::perm_smem(c->H, c->E).total;
   if (mx)
-    perm::scatter_kernel<0, perm::QF_MX><<<sgrid, perm::SC_WARPS * 32, 0, st>>>(
-        static_cast<const __nv_bfloat16*>(x), c->T, c->H, c->E, c->k, idx, lrank, base, offsets, gates, row_of,
-        src_of, row_gate, xp, xp_sf);
+    err = launch_dep(perm::permute_kernel<perm::QF_MX>, pgrid, perm::PW_THREADS, smem, st, x16, c->T, c->H, c->E,
+                     c->k, idx, (const int32_t*)lrank, (const int2*)bt, gates, row_of, src_of, row_gate, xp, xp_sf,
+                     status);
   else if (nv)
-    perm::scatter_kernel<0, perm::QF_NV><<<sgrid, perm::SC_WARPS * 32, 0, st>>>(
-        static_cast<const __nv_bfloat16*>(x), c->T, c->H, c->E, c->k, idx, lrank, base, offsets, gates, row_of,
-        src_of, row_gate, xp, xp_sf);
+    err = launch_dep(perm::permute_kernel<perm::QF_NV>, pgrid, perm::PW_THREADS, smem, st, x16, c->T, c->H, c->E,
+                     c->k, idx, (const int32_t*)lrank, (const int2*)bt, gates, row_of, src_of, row_gate, xp, xp_sf,
+                     status);
   else
-    perm::scatter_kernel<0, perm::QF_BF16><<<sgrid, perm::SC_WARPS * 32, 0, st>>>(
-        static_cast<const __nv_bfloat16*>(x), c->T, c->H, c->E, c->k, idx, lrank, base, offsets, gates, row_of,
-        src_of, row_gate, xp, nullptr);
-  MOE_CHECK_LAUNCH();
+    err = launch_dep(perm::permute_kernel<perm::QF_BF16>, pgrid, perm::PW_THREADS, smem, st, x16, c->T, c->H,
+                     c->E, c->k, idx, (const int32_t*)lrank, (const int2*)bt, gates, row_of, src_of, row_gate, xp,
+                     (uint8_t*)nullptr, status);
+  if (err != cudaSuccess) {
+    (void)cudaGetLastError();
+    return MOE_ERR_CUDA;
+  }
   return MOE_OK;
 }
 
 int scatter_rows(const moe_config* c, const void* x, const int32_t* row_of, void* xp, cudaStream_t st) {
   const int sgrid = (c->T + perm::SC_WARPS - 1) / perm::SC_WARPS;
-  perm::scatter_kernel<1, perm::QF_BF16><<<sgrid, perm::SC_WARPS * 32, 0, st>>>(
-      static_cast<const __nv_bfloat16*>(x), c->T, c->H, c->E, c->k, nullptr, nullptr, nullptr, nullptr, nullptr,
-      const_cast<int32_t*>(row_of), nullptr, nullptr, xp, nullptr);
+  perm::scatter_kernel<perm::QF_BF16><<<sgrid, perm::SC_WARPS * 32, 0, st>>>(
+      static_cast<const __nv_bfloat16*>(x), c->T, c->H, c->k, row_of, xp, nullptr);
   MOE_CHECK_LAUNCH();
   return MOE_OK;
 }
@@ -462,9 +654,8 @@ int scatter_rows(const moe_config* c, const void* x, const int32_t* row_of, void
 int scatter_rows_mx(const moe_config* c, const void* x, const int32_t* row_of, uint8_t* xq, uint8_t* xq_sf,
                     cudaStream_t st) {
   const int sgrid = (c->T + perm::SC_WARPS - 1) / perm::SC_WARPS;
-  perm::scatter_kernel<1, perm::QF_MX><<<sgrid, perm::SC_WARPS * 32, 0, st>>>(
-      static_cast<const __nv_bfloat16*>(x), c->T, c->H, c->E, c->k, nullptr, nullptr, nullptr, nullptr, nullptr,
-      const_cast<int32_t*>(row_of), nullptr, nullptr, xq, xq_sf);
+  perm::scatter_kernel<perm::QF_MX><<<sgrid, perm::SC_WARPS * 32, 0, st>>>(
+      static_cast<const __nv_bfloat16*>(x), c->T, c->H, c->k, row_of, xq, xq_sf);
   MOE_CHECK_LAUNCH();
   return MOE_OK;
 }
@@ -478,10 +669,18 @@ int unpermute(const moe_config* c, const void* o, const int32_t* row_of, const v
   const auto* o16 = static_cast<const __nv_bfloat16*>(o);
   const auto* e16 = static_cast<const __nv_bfloat16*>(extra);
   auto* y16 = static_cast<__nv_bfloat16*>(y);
-  if (c->k <= 2) perm::unpermute_kernel<2><<<grid, perm::SC_WARPS * 32, 0, st>>>(o16, row_of, e16, c->T, c->H, c->k, y16);
-  else if (c->k <= 4) perm::unpermute_kernel<4><<<grid, perm::SC_WARPS * 32, 0, st>>>(o16, row_of, e16, c->T, c->H, c->k, y16);
-  else if (c->k <= 8) perm::unpermute_kernel<8><<<grid, perm::SC_WARPS * 32, 0, st>>>(o16, row_of, e16, c->T, c->H, c->k, y16);
-  else perm::unpermute_kernel<16><<<grid, perm::SC_WARPS * 32, 0, st>>>(o16, row_of, e16, c->T, c->H, c->k, y16);
+  auto go = [&](auto kern) { kern<<<grid, perm::SC_WARPS * 32, 0, st>>>(o16, row_of, e16, c->T, c->H, c->k, y16); };
+  if (e16) {
+    if (c->k <= 2) go(perm::unpermute_kernel<2, true>);
+    else if (c->k <= 4) go(perm::unpermute_kernel<4, true>);
+    else if (c->k <= 8) go(perm::unpermute_kernel<8, true>);
+    else go(perm::unpermute_kernel<16, true>);
+  } else {
+    if (c->k <= 2) go(perm::unpermute_kernel<2, false>);
+    else if (c->k <= 4) go(perm::unpermute_kernel<4, false>);
+    else if (c->k <= 8) go(perm::unpermute_kernel<8, false>);
+    else go(perm::unpermute_kernel<16, false>);
+  }
   MOE_CHECK_LAUNCH();
   return MOE_OK;
 }
