@@ -54,7 +54,7 @@ struct __align__(64) Params {
   CUtensorMap tmB0;
   CUtensorMap tmB1;
   // GROUP_K bf16 output through TMA stores (tma_store != 0): C and C2 as [G * c_rows_per_group, N] bf16,
-  // no swizzle, 16-column x 32-row boxes
+  // 64-column x 32-row boxes, 128-byte swizzle
   CUtensorMap tmC;
   CUtensorMap tmC2;
   long long c_rows_per_group;
@@ -86,10 +86,10 @@ struct __align__(64) Params {
 template <int BN_, bool A_MN_, bool B_MN_, int EPI_, int GROUP_, int BMODE_, bool TMA_ST_ = false>
 struct Cfg {
   static constexpr int BN = BN_;
-  // grouped along K with a bf16 output leaving through TMA stores: three TMA stages, and four 1 KB staging
-  // slices (32 rows x 16 columns) per epilogue warp, so that its stores stay in flight
+  // grouped along K with a bf16 output leaving through TMA stores: three TMA stages, and a 4 KB staging
+  // buffer per epilogue warp (one 32-row x 64-column box, 128-byte swizzled)
   static constexpr bool TMA_ST = TMA_ST_;
-  static constexpr int TMA_ST_BUFS = 4;
+  static constexpr int TMA_ST_BUFS = 4;  // KB of staging per epilogue warp
   static constexpr bool A_MN = A_MN_;
   static constexpr bool B_MN = B_MN_;
   static constexpr int EPI = EPI_;
@@ -111,7 +111,8 @@ struct Cfg {
   static constexpr int STG_ROW = (EPI == EPI_SWIGLU_BWD) ? 48 : 80;
   static constexpr int STG_BYTES =
       TMA_ST ? EPI_WARPS * TMA_ST_BUFS * 1024 : EPI_WARPS * 32 * STG_ROW * (EPI == EPI_SWIGLU_BWD ? 2 : 1);
-  static constexpr int SMEM_BYTES = 1024 + kStages * STAGE_BYTES + BAR_BYTES + 2 * (MAX_G + 1) * 4 + 128 + STG_BYTES;
+  static constexpr int SMEM_BYTES =
+      1024 + kStages * STAGE_BYTES + BAR_BYTES + 2 * (MAX_G + 1) * 4 + (TMA_ST ? 1024 : 128) + STG_BYTES;
   static_assert(BN == 128 || BN == 256, "BN");
   static_assert(!(BMODE == B_SPLIT_N && B_MN), "split-N is for K-major weights");
   static_assert(!TMA_ST || (GROUP == GROUP_K && EPI == EPI_BF16), "TMA-store epilogue: weight gradients");
@@ -203,8 +204,10 @@ __global__ void __launch_bounds__(C::NUM_THREADS, 1) gemm_kernel(const __grid_co
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   int* s_off = reinterpret_cast<int*>(bar_area + C::BAR_BYTES);
   int* s_tstart = s_off + (MAX_G + 1);
+  // 128-byte aligned (1024 for the TMA-store epilogue, whose boxes are 128-byte swizzled)
+  constexpr uintptr_t STG_ALIGN = C::TMA_ST ? 1024 : 128;
   uint8_t* stg_area = reinterpret_cast<uint8_t*>(
-      (reinterpret_cast<uintptr_t>(s_tstart + (MAX_G + 1)) + 127) & ~uintptr_t(127));
+      (reinterpret_cast<uintptr_t>(s_tstart + (MAX_G + 1)) + STG_ALIGN - 1) & ~(STG_ALIGN - 1));
   (void)stg_area;
 
   const int warp = threadIdx.x >> 5;
@@ -430,7 +433,6 @@ __global__ void __launch_bounds__(C::NUM_THREADS, 1) gemm_kernel(const __grid_co
     const int row = q * 32 + lane;
     uint8_t* stg = stg_area + (C::TMA_ST ? ew * C::TMA_ST_BUFS * 1024
                                          : ew * 32 * C::STG_ROW * (C::EPI == EPI_SWIGLU_BWD ? 2 : 1));
-    uint32_t stg_seq = 0;  // TMA stores issued by this warp (picks the staging slice)
     int acc = 0;
     uint32_t acc_phase = 0;
     for (int t = blockIdx.x; t < total && !aborted; t += gridDim.x) {
@@ -505,8 +507,48 @@ __global__ void __launch_bounds__(C::NUM_THREADS, 1) gemm_kernel(const __grid_co
         }
         constexpr int W = C::BN / C::NH;
         const int nvalid = min(C::BN, p.N - ti.n0);
+        bool stored = false;  // left through TMA stores
+        if constexpr (C::TMA_ST) {
+          if (p.tma_store) {
+            // the warp's 32 rows x W columns leave as 32 x 64 boxes through TMA stores from its 4 KB staging
+            // buffer, 128-byte swizzled (16-byte chunk j of row r at chunk j ^ (r % 8), so the lanes' chunk
+            // writes fall on distinct banks); the buffer is rewritten once the previous box's store has read it
+            stored = true;
+            const CUtensorMap* tm = to_c2 ? &p.tmC2 : &p.tmC;
+            const int y = (int)(ti.g * p.c_rows_per_group + rbase + 32 * q);
 #pragma unroll 1
-        for (int c = h * W; c < (h + 1) * W; c += 32) {
+            for (int c = h * W; c < (h + 1) * W; c += 64) {
+              // warp-uniform: columns past the output, or a 32-row block past it (M % 32 == 0)
+              if (c >= nvalid || 32 * q >= ti.m_valid) break;
+              float v[64];
+              if (!empty_k) {
+                tmem_ld32(tb + c, *reinterpret_cast<float(*)[32]>(&v[0]));
+                tmem_ld32(tb + c + 32, *reinterpret_cast<float(*)[32]>(&v[32]));
+                tmem_ld_wait();
+              } else {
+#pragma unroll
+                for (int i = 0; i < 64; ++i) v[i] = 0.f;
+              }
+              if (lane == 0) bulk_wait_read<0>();
+              __syncwarp();
+#pragma unroll
+              for (int j = 0; j < 8; ++j) {
+                const float* w = v + 8 * j;
+                *reinterpret_cast<uint4*>(stg + lane * 128 + ((j ^ (lane & 7)) << 4)) =
+                    make_uint4(pack_bf16x2(w[0], w[1]), pack_bf16x2(w[2], w[3]), pack_bf16x2(w[4], w[5]),
+                               pack_bf16x2(w[6], w[7]));
+              }
+              fence_proxy_async_smem();  // the generic-proxy writes, for the TMA engine's reads
+              __syncwarp();
+              if (lane == 0) {
+                tma_store_2d(tm, stg, ti.n0 + c, y);
+                bulk_commit();
+              }
+            }
+          }
+        }
+#pragma unroll 1
+        for (int c = h * W; c < (h + 1) * W && !stored; c += 32) {
           if (c >= nvalid) break;  // warp-uniform
           float v[32];
           if (!empty_k) {
@@ -515,38 +557,6 @@ __global__ void __launch_bounds__(C::NUM_THREADS, 1) gemm_kernel(const __grid_co
           } else {
 #pragma unroll
             for (int i = 0; i < 32; ++i) v[i] = 0.f;
-          }
-          if constexpr (C::TMA_ST) {
-            if (p.tma_store) {
-              // each 32-row x 16-column slice goes out through a TMA store from one of this warp's staging
-              // slices (a slice is rewritten once the store issued TMA_ST_BUFS slices earlier has read it)
-              if (32 * q >= ti.m_valid) break;  // warp-uniform: a 32-row block past the output (M % 32 == 0)
-              const CUtensorMap* tm = to_c2 ? &p.tmC2 : &p.tmC;
-              const int y = (int)(ti.g * p.c_rows_per_group + rbase + 32 * q);
-#pragma unroll
-              for (int pass = 0; pass < 2; ++pass) {
-                uint8_t* sl = stg + (stg_seq & (C::TMA_ST_BUFS - 1)) * 1024;
-                if (lane == 0) bulk_wait_read<C::TMA_ST_BUFS - 1>();
-                __syncwarp();
-                *reinterpret_cast<uint4*>(sl + lane * 32) =
-                    make_uint4(pack_bf16x2(v[16 * pass], v[16 * pass + 1]), pack_bf16x2(v[16 * pass + 2], v[16 * pass + 3]),
-                               pack_bf16x2(v[16 * pass + 4], v[16 * pass + 5]),
-                               pack_bf16x2(v[16 * pass + 6], v[16 * pass + 7]));
-                *reinterpret_cast<uint4*>(sl + lane * 32 + 16) =
-                    make_uint4(pack_bf16x2(v[16 * pass + 8], v[16 * pass + 9]),
-                               pack_bf16x2(v[16 * pass + 10], v[16 * pass + 11]),
-                               pack_bf16x2(v[16 * pass + 12], v[16 * pass + 13]),
-                               pack_bf16x2(v[16 * pass + 14], v[16 * pass + 15]));
-                fence_proxy_async_smem();  // the generic-proxy writes, for the TMA engine's reads
-                __syncwarp();
-                if (lane == 0) {
-                  tma_store_2d(tm, sl, ti.n0 + c + 16 * pass, y);
-                  bulk_commit();
-                }
-                ++stg_seq;
-              }
-              continue;
-            }
           }
 #pragma unroll
           for (int j = 0; j < 4; ++j)
@@ -698,7 +708,7 @@ __global__ void __launch_bounds__(C::NUM_THREADS, 1) gemm_kernel(const __grid_co
     }
   }
 
-  if (C::TMA_ST && warp >= 2 && lane == 0) bulk_wait_all();  // every TMA store has read its slice and landed
+  if (C::TMA_ST && warp >= 2 && lane == 0) bulk_wait_all();  // every TMA store has read its box and landed
   __syncthreads();
   if (warp == 1) {
     tc_fence_after();

@@ -27,9 +27,10 @@
 // epilogue warps (two per lane quadrant, 128 columns each) first copy their
 // accumulator columns into registers and release TMEM, so the next tile's MMAs
 // run while they finish the element-wise work. The bf16 output of the
-// grouped-along-K weight gradients leaves through TMA stores (four 1 KB
-// staging buffers per warp); the SwiGLU backward stages its saved gate/up and
-// dgate/dup through shared memory, 64 contiguous bytes per row. Those two
+// grouped-along-K weight gradients leaves through TMA stores (two 32 x 64
+// boxes per warp and tile, 128-byte swizzled in a 4 KB staging buffer); the
+// SwiGLU backward stages its saved gate/up and dgate/dup through shared
+// memory, 64 contiguous bytes per row. Those two
 // instantiations have three TMA stages, the others four.
 // Roles: warp 0 TMA producer, warp 1 MMA issuer (+ TMEM owner), warp 2 scale
 // loader, warps 3..10 epilogue. All waits are bounded like gemm.cuh.
@@ -82,7 +83,7 @@ constexpr int SMEM_BYTES =
     1024 + kStages * STAGE_BYTES + kSfBufs * SF_BATCH_BYTES + BAR_BYTES + 2 * (MAX_G + 1) * 4 + 128 +
     8 * STG_WARP_BYTES;
 // Grouped along K (weight gradients, short K per tile, a bf16 output that dominates the traffic): three TMA
-// stages, and four staging buffers per epilogue warp so that its TMA stores stay in flight
+// stages, and 4 KB of staging per epilogue warp: one 32-row x 64-column box of its TMA stores
 constexpr int kStagesGK = 3;
 constexpr int STG_BUFS_GK = 4;
 // The SwiGLU-backward epilogue stages the saved gate/up of its 32 rows, 32 columns at a time (64 bytes per
@@ -98,7 +99,7 @@ constexpr int stg_warp_bytes() {
 template <int EPI, bool GK>
 constexpr int smem_bytes() {
   return 1024 + stages<EPI, GK>() * STAGE_BYTES + kSfBufs * SF_BATCH_BYTES + BAR_BYTES + 2 * (MAX_G + 1) * 4 +
-         128 + 8 * stg_warp_bytes<EPI, GK>();
+         (GK ? 1024 : 128) + 8 * stg_warp_bytes<EPI, GK>();
 }
 static_assert(smem_bytes<1, true>() <= 232448, "smem");
 static_assert(smem_bytes<2, false>() <= 232448, "smem");
@@ -117,7 +118,7 @@ struct __align__(64) Params {
   CUtensorMap tmB0;
   CUtensorMap tmB1;
   // GROUP_K bf16 output through TMA stores (tma_store != 0): C and C2 as [G * c_rows_per_group, N] bf16,
-  // no swizzle, 16 x 32 boxes
+  // 64-column x 32-row boxes, 128-byte swizzle
   CUtensorMap tmC;
   CUtensorMap tmC2;
   int M;              // rows of A (all groups)
@@ -284,8 +285,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) gemm_mx_kernel(const __grid_co
   int* s_off = reinterpret_cast<int*>(bar_area + BAR_BYTES);
   int* s_tstart = s_off + (MAX_G + 1);
   // 128-byte aligned: the TMA stores read their boxes from here
-  uint8_t* stg_area =
-      reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(s_tstart + (MAX_G + 1)) + 127) & ~uintptr_t(127));
+  // 128-byte aligned (1024 for the grouped-along-K TMA stores, whose boxes are 128-byte swizzled)
+  constexpr uintptr_t STG_ALIGN = GK ? 1024 : 128;
+  uint8_t* stg_area = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(s_tstart + (MAX_G + 1)) + STG_ALIGN - 1) &
+                                                 ~(STG_ALIGN - 1));
   constexpr int N_STEP = SPLIT_N ? BN / 2 : BN;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -698,7 +701,6 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) gemm_mx_kernel(const __grid_co
     const int h = (warp - 3) >> 2;
     const int row = q * 32 + lane;
     uint32_t acc_phase = 0;
-    uint32_t stg_seq = 0;  // GROUP_K TMA stores: slices issued by this warp (picks the staging buffer)
     for (int t = blockIdx.x; t < total && !aborted; t += gridDim.x) {
       const Tile ti = get_tile<GK>(p, t, s_off, s_tstart, N_STEP);
       if (!__all_sync(0xffffffffu, mbar_wait(tfull, acc_phase, abort_flag, p.status, DEV_WAIT_TIMEOUT_EPILOGUE))) {
@@ -857,10 +859,11 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) gemm_mx_kernel(const __grid_co
       if constexpr (EPI == EPI_MX_BF16) {
         if (GK && p.tma_store) {
           if (32 * q >= ti.m_valid) continue;  // warp-uniform: a 32-row block past the output (M % 32 == 0)
-          // grouped along K: each 32-row x 16-column slice leaves through a TMA store from one of four
-          // staging buffers of this warp (a buffer is rewritten once the store issued four slices earlier has
-          // read it), so the epilogue issues no global stores of its own
-          uint8_t* stg_w = stg_area + (warp - 3) * STG_WARP_BYTES * STG_BUFS_GK;
+          // grouped along K: the warp's 32 rows x 128 columns leave as two 32 x 64 boxes through TMA stores
+          // from its 4 KB staging buffer, 128-byte swizzled (16-byte chunk j of row r at chunk j ^ (r % 8), so
+          // the 32 lanes' chunk writes fall on distinct banks); the buffer is rewritten once the previous
+          // box's store has read it
+          uint8_t* stg = stg_area + (warp - 3) * STG_WARP_BYTES * STG_BUFS_GK;
           const int ncol = min(128, p.N - ti.n0 - 128 * h);
           long long r0 = (long long)ti.row0 + 32 * q;
           const CUtensorMap* tm = &p.tmC;
@@ -870,27 +873,23 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) gemm_mx_kernel(const __grid_co
           }
           const int y = (int)(ti.g * p.c_rows_per_group + r0);
 #pragma unroll
-          for (int pass = 0; pass < 8; ++pass) {
-            if (16 * pass >= ncol) break;  // warp-uniform
-            uint8_t* stg = stg_w + (stg_seq & (STG_BUFS_GK - 1)) * STG_WARP_BYTES;
-            if (lane == 0) bulk_wait_read<STG_BUFS_GK - 1>();
+          for (int half = 0; half < 2; ++half) {
+            if (64 * half >= ncol) break;  // warp-uniform
+            if (lane == 0) bulk_wait_read<0>();
             __syncwarp();
-            *reinterpret_cast<uint4*>(stg + lane * 32) =
-                make_uint4(pack_bf16x2(v[16 * pass], v[16 * pass + 1]), pack_bf16x2(v[16 * pass + 2], v[16 * pass + 3]),
-                           pack_bf16x2(v[16 * pass + 4], v[16 * pass + 5]),
-                           pack_bf16x2(v[16 * pass + 6], v[16 * pass + 7]));
-            *reinterpret_cast<uint4*>(stg + lane * 32 + 16) =
-                make_uint4(pack_bf16x2(v[16 * pass + 8], v[16 * pass + 9]),
-                           pack_bf16x2(v[16 * pass + 10], v[16 * pass + 11]),
-                           pack_bf16x2(v[16 * pass + 12], v[16 * pass + 13]),
-                           pack_bf16x2(v[16 * pass + 14], v[16 * pass + 15]));
+#pragma unroll
+            for (int j = 0; j < 8; ++j) {
+              const float* w = v + 64 * half + 8 * j;
+              *reinterpret_cast<uint4*>(stg + lane * 128 + ((j ^ (lane & 7)) << 4)) =
+                  make_uint4(pack_bf16x2(w[0], w[1]), pack_bf16x2(w[2], w[3]), pack_bf16x2(w[4], w[5]),
+                             pack_bf16x2(w[6], w[7]));
+            }
             fence_proxy_async_smem();  // the generic-proxy writes, for the TMA engine's reads
             __syncwarp();
             if (lane == 0) {
-              tma_store_2d(tm, stg, ti.n0 + 128 * h + 16 * pass, y);
+              tma_store_2d(tm, stg, ti.n0 + 128 * h + 64 * half, y);
               bulk_commit();
             }
-            ++stg_seq;
           }
         } else {
           // 16 columns at a time through shared memory, so that each warp store writes whole 32-byte

@@ -174,10 +174,11 @@ int gemm_wgrad(int rows, int groups, int M, int N, const void* dO, int ld_dO, co
   const bool al = ((reinterpret_cast<uintptr_t>(C) | reinterpret_cast<uintptr_t>(C2 ? C2 : C)) & 15u) == 0;
   if (wgrad_tma_store() && M % 32 == 0 && split % 32 == 0 && N % 8 == 0 && al &&
       (long long)groups * rpg < (1LL << 31)) {
-    if (!moe_host::encode_tmap_2d_plain(&p.tmC, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, C, N, (uint64_t)groups * rpg,
-                                        (uint64_t)N * 2, 16, 32) ||
-        !moe_host::encode_tmap_2d_plain(&p.tmC2, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, C2 ? C2 : C, N,
-                                        (uint64_t)groups * rpg, (uint64_t)N * 2, 16, 32))
+    // 64 x 32 boxes, 128-byte swizzle (columns past N are clipped by the store)
+    if (!moe_host::encode_tmap_2d(&p.tmC, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, C, N, (uint64_t)groups * rpg,
+                                  (uint64_t)N * 2, 64, 32) ||
+        !moe_host::encode_tmap_2d(&p.tmC2, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, C2 ? C2 : C, N, (uint64_t)groups * rpg,
+                                  (uint64_t)N * 2, 64, 32))
       return MOE_ERR_CUDA;
     p.c_rows_per_group = rpg;
     p.tma_store = 1;

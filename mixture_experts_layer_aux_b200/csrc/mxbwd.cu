@@ -384,14 +384,15 @@ int gemm_wgrad_mx(int E, int M, int N, long long ldp, const void* AT, const uint
   p.c2_row_split = split;
   p.ldc = N;
   p.c_group_stride = (long long)(split > 0 ? split : M) * N;
-  // the bf16 output through TMA stores: [E * rows per group, N], 16 x 32 boxes (whole 32-row blocks)
+  // the bf16 output through TMA stores: [E * rows per group, N], 64 x 32 boxes, 128-byte swizzle (whole
+  // 32-row blocks; columns past N are clipped by the store)
   const long long rpg = split > 0 ? split : M;
   const bool al = ((reinterpret_cast<uintptr_t>(C) | reinterpret_cast<uintptr_t>(C2 ? C2 : C)) & 15u) == 0;
   if (M % 32 == 0 && split % 32 == 0 && N % 8 == 0 && al && (long long)E * rpg < (1LL << 31)) {
-    if (!moe_host::encode_tmap_2d_plain(&p.tmC, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, C, N, (uint64_t)E * rpg,
-                                        (uint64_t)N * 2, 16, 32) ||
-        !moe_host::encode_tmap_2d_plain(&p.tmC2, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, C2 ? C2 : C, N,
-                                        (uint64_t)E * rpg, (uint64_t)N * 2, 16, 32))
+    if (!moe_host::encode_tmap_2d(&p.tmC, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, C, N, (uint64_t)E * rpg,
+                                  (uint64_t)N * 2, 64, 32) ||
+        !moe_host::encode_tmap_2d(&p.tmC2, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, C2 ? C2 : C, N, (uint64_t)E * rpg,
+                                  (uint64_t)N * 2, 64, 32))
       return MOE_ERR_CUDA;
     p.c_rows_per_group = rpg;
     p.tma_store = 1;
