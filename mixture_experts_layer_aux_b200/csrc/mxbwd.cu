@@ -102,10 +102,16 @@ constexpr int QT_ROWS_BF = 128;        // other tiles
 constexpr int QT_LDS = QT_COLS + 8;    // staged row stride (bf16 elements): 16-byte aligned row starts
 __host__ __device__ constexpr int qt_rows(int mode) { return mode == 2 ? QT_ROWS : QT_ROWS_BF; }
 __host__ __device__ constexpr int qt_nsrc(int mode) { return mode == 2 ? 2 : 1; }
+// the quantised codes of one column tile, [QT_COLS][TR + 16] bytes, written over the tile's staged bf16 once
+// it has been read: a padded row stride, so that both the column-wise writes and the row-wise reads of
+// 16-byte chunks fall on distinct banks
+__host__ __device__ constexpr int qt_code_ld(int mode) { return qt_rows(mode) + 16; }
 // dynamic shared memory: two buffers of qt_nsrc staged bf16 tiles [TR][QT_LDS], then TR fp32 row gates
 __host__ __device__ constexpr int qt_smem(int mode) {
   return 2 * qt_nsrc(mode) * qt_rows(mode) * QT_LDS * 2 + qt_rows(mode) * 4;
 }
+static_assert(QT_COLS * qt_code_ld(0) <= qt_nsrc(0) * qt_rows(0) * QT_LDS * 2, "code tile");
+static_assert(QT_COLS * qt_code_ld(2) <= qt_nsrc(2) * qt_rows(2) * QT_LDS * 2, "code tile");
 template <int MODE>
 __global__ void __launch_bounds__(256) quant_t_kernel(const QtArgs a) {
   constexpr bool AP = MODE == MODE_AP;
@@ -114,6 +120,7 @@ __global__ void __launch_bounds__(256) quant_t_kernel(const QtArgs a) {
   constexpr int NSRC = qt_nsrc(MODE);
   constexpr int TILE = TR * QT_LDS;  // elements of one staged tile
   extern __shared__ __align__(16) uint8_t qt_dyn[];
+  constexpr int CLD = qt_code_ld(MODE);
   __nv_bfloat16* stg = reinterpret_cast<__nv_bfloat16*>(qt_dyn);        // [2][NSRC][TR][QT_LDS]
   float* s_rg = reinterpret_cast<float*>(qt_dyn + 2 * NSRC * TILE * 2);  // [TR] (MODE_AP)
   __shared__ int s_meta[3];  // first source row (-1: none), valid rows, rows to write
@@ -209,8 +216,8 @@ __global__ void __launch_bounds__(256) quant_t_kernel(const QtArgs a) {
     // quantise: thread t takes column t % 128 and the TR/2 rows of half t / 128: TR/64 blocks of 32, each
     // with its amax by a plain loop; the codes of the half leave as one contiguous run
     constexpr int NB = TR / 64;  // 32-row blocks per thread
+    uint32_t w[NB][8];
     if (c0 + c < a.C) {
-      uint32_t w[NB][8];
       uint8_t sbv[NB];
 #pragma unroll
       for (int bb = 0; bb < NB; ++bb) {
@@ -237,12 +244,9 @@ __global__ void __launch_bounds__(256) quant_t_kernel(const QtArgs a) {
         }
       }
       const int pbase = p0 + (TR / 2) * hb;
-      uint4* d4 = reinterpret_cast<uint4*>(dst + (long long)(c0 + c) * a.ldd + pbase);
 #pragma unroll
       for (int bb = 0; bb < NB; ++bb) {
         if ((TR / 2) * hb + 32 * bb >= nw) break;  // rows past a weight matrix's end (R % 32 == 0)
-        d4[2 * bb] = make_uint4(w[bb][0], w[bb][1], w[bb][2], w[bb][3]);
-        d4[2 * bb + 1] = make_uint4(w[bb][4], w[bb][5], w[bb][6], w[bb][7]);
         const int p = pbase + 32 * bb;
         if constexpr (MODE == MODE_WEIGHT) {
           sf[(long long)(c0 + c) * (a.ldd / 32) + p / 32] = sbv[bb];  // natural [C, ldd/32]
@@ -254,7 +258,32 @@ __global__ void __launch_bounds__(256) quant_t_kernel(const QtArgs a) {
         }
       }
     }
-    __syncthreads();  // buffer ct & 1 has been read before tile ct + 2 is staged into it
+    __syncthreads();  // every thread has read staged tile ct: its buffer takes the codes
+    // the codes go to the code tile (column c, this half's positions); they leave row-wise below
+    uint8_t* s_code = reinterpret_cast<uint8_t*>(stg + (ct & 1) * NSRC * TILE);
+    if (c0 + c < a.C) {
+      uint4* c4 = reinterpret_cast<uint4*>(s_code + c * CLD + (TR / 2) * hb);
+#pragma unroll
+      for (int bb = 0; bb < NB; ++bb) {
+        c4[2 * bb] = make_uint4(w[bb][0], w[bb][1], w[bb][2], w[bb][3]);
+        c4[2 * bb + 1] = make_uint4(w[bb][4], w[bb][5], w[bb][6], w[bb][7]);
+      }
+    }
+    __syncthreads();  // the code tile is complete
+    // output row c0 + r gets the tile's nw code bytes as 16-byte chunks: consecutive threads take consecutive
+    // chunks of a row, so a warp writes whole rows (TR / 16 chunks each)
+    {
+      constexpr int CPR = TR / 16;  // chunks per output row
+#pragma unroll
+      for (int k = 0; k < QT_COLS * CPR / 256; ++k) {
+        const int i = tid + 256 * k;
+        const int r = i / CPR, ch = i % CPR;
+        if (c0 + r < a.C && 16 * ch < nw)
+          *reinterpret_cast<uint4*>(dst + (long long)(c0 + r) * a.ldd + p0 + 16 * ch) =
+              *reinterpret_cast<const uint4*>(s_code + r * CLD + 16 * ch);
+      }
+    }
+    __syncthreads();  // buffer ct & 1 and the code tile have been read before they are rewritten
   }
 }
 
