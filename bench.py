@@ -178,7 +178,8 @@ class ClockSampler:
 
     A background thread reads them through NVML (read-only queries) every ~2 ms, so even a timed region of
     a few tens of milliseconds gets tens of samples; where NVML is unavailable, nvidia-smi polls at its own
-    rate instead. Nothing here changes any GPU setting."""
+    rate instead. While it runs, the interpreter's thread switch interval is cut to 0.5 ms, so the launching
+    thread cannot hold the sampler off for the default 5 ms. Nothing here changes any GPU setting."""
 
     REASONS = (("hw_slowdown", "nvmlClocksEventReasonHwSlowdown"),
                ("hw_thermal_slowdown", "nvmlClocksEventReasonHwThermalSlowdown"),
@@ -205,7 +206,10 @@ class ClockSampler:
             return pynvml, pynvml.nvmlDeviceGetHandleByIndex(self.index)
 
     def __enter__(self):
+        import sys
         import threading
+        self._switch = sys.getswitchinterval()
+        sys.setswitchinterval(min(self._switch, 0.0005))
         try:
             nv, h = self._nvml_handle()
             self.max_mhz = float(nv.nvmlDeviceGetMaxClockInfo(h, nv.NVML_CLOCK_SM))
@@ -242,6 +246,8 @@ class ClockSampler:
             self.proc = None
 
     def __exit__(self, *a):
+        import sys
+        sys.setswitchinterval(self._switch)
         if self.thread is not None:
             self._stop.set()
             self.thread.join(timeout=5)
