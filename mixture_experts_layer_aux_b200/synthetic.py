@@ -100,6 +100,10 @@ WORKLOADS = {
     # the MXFP8 backward on the DeepSeek-V3 routed experts (the backward has no shared expert)
     "dsv3-train": Workload("dsv3-train", T=8192, H=7168, E=256, k=8, F=2048, score="sigmoid", route_scale=2.5,
                            dtype="mxfp8", aux=False, bwd=True),
+    # the same MXFP8 training step on 16 experts with the same ~256 rows each (~4 GB on the device): the small
+    # case of the backward kernels' section captures
+    "dsv3-train-e16": Workload("dsv3-train-e16", T=512, H=7168, E=16, k=8, F=2048, score="sigmoid", route_scale=2.5,
+                               dtype="mxfp8", aux=False, bwd=True),
     "skewed-capacity": Workload("skewed-capacity", T=8192, H=4096, E=128, k=8, F=1536, skew=True, bwd=True,
                                 capacity_factor=1.25),
 }
