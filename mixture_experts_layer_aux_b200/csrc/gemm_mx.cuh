@@ -163,19 +163,14 @@ struct Tile {
 
 template <bool GK>
 __device__ __forceinline__ Tile get_tile(const Params& p, int t, const int* s_off, const int* s_tstart, int n_step) {
-  int lo = 0, hi = p.G - 1;
-  while (lo < hi) {
-    const int mid = (lo + hi + 1) >> 1;
-    if (s_tstart[mid] <= t) lo = mid;
-    else hi = mid - 1;
-  }
-  const int g = lo;
-  const int local = t - s_tstart[g];
   Tile ti;
-  ti.g = g;
   if constexpr (GK) {
-    // every group: the whole [M, N] output; its K range is the group's segment
+    // every group: the whole [M, N] output, the same tile count per group; its K range is the group's segment
     const int MB = (p.M + BM - 1) / BM;
+    const int per_g = MB * ((p.N + n_step - 1) / n_step);
+    const int g = t / per_g;
+    const int local = t - g * per_g;
+    ti.g = g;
     ti.m0 = (local % MB) * BM;
     ti.n0 = (local / MB) * n_step;
     ti.row0 = ti.m0;
@@ -183,6 +178,16 @@ __device__ __forceinline__ Tile get_tile(const Params& p, int t, const int* s_of
     ti.kb0 = s_off[g] / BK;
     ti.nkb = (s_off[g + 1] - s_off[g]) / BK;
   } else {
+    // grouped along M: the last group whose first tile is at or before t
+    int lo = 0, hi = p.G - 1;
+    while (lo < hi) {
+      const int mid = (lo + hi + 1) >> 1;
+      if (s_tstart[mid] <= t) lo = mid;
+      else hi = mid - 1;
+    }
+    const int g = lo;
+    const int local = t - s_tstart[g];
+    ti.g = g;
     const int mg = s_off[g + 1] - s_off[g];
     const int MB = (mg + BM - 1) / BM;
     ti.m0 = (local % MB) * BM;
