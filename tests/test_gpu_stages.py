@@ -131,6 +131,10 @@ PERMUTE_CASES = [
     (1, 256, 4, 4, 0, 0.0),
     (130, 7168, 256, 8, 0, 0.0),
     (257, 256, 16, 1, 15, 0.0),  # every token on expert 0
+    # more rank blocks x experts than the scan stages in shared memory (its two-pass path): without and with
+    # rows long enough for the permute kernel's shared-memory staging
+    (8192, 128, 512, 2, 37, 0.0),
+    (7000, 2048, 512, 2, 5, 0.0),
 ]
 
 
