@@ -83,7 +83,7 @@ def test_quantize_nvfp4_activations_bit_exact(moe, oracle, R, K):
     assert torch.equal(dst.cpu(), q)
 
 
-@pytest.mark.parametrize("T,H,E,k", [(300, 256, 8, 2), (1024, 7168, 256, 8)])
+@pytest.mark.parametrize("T,H,E,k", [(300, 256, 8, 2), (1024, 7168, 256, 8), (300, 4864, 16, 4)])
 def test_permute_nvfp4_bit_exact(moe, oracle, T, H, E, k):
     idx = random_routing(T, E, k, seed=T + 2)
     x = randn_bf16((T, H), 1.0, seed=T + 6, scale_rows=True)

@@ -135,6 +135,8 @@ PERMUTE_CASES = [
     # rows long enough for the permute kernel's shared-memory staging
     (8192, 128, 512, 2, 37, 0.0),
     (7000, 2048, 512, 2, 5, 0.0),
+    # rows past the permute kernel's register chunks and shared-memory slot (H > 4096): a ragged last group
+    (300, 4480, 16, 2, 0, 0.0),
 ]
 
 
@@ -164,7 +166,7 @@ def test_permute_bit_exact(moe, oracle, T, H, E, k, zero, hot):
     _status_clean(moe)
 
 
-@pytest.mark.parametrize("T,H,E,k", [(300, 256, 8, 2), (1024, 7168, 256, 8)])
+@pytest.mark.parametrize("T,H,E,k", [(300, 256, 8, 2), (1024, 7168, 256, 8), (300, 4480, 16, 4)])
 def test_permute_mxfp8_bit_exact(moe, oracle, T, H, E, k):
     idx = random_routing(T, E, k, seed=T + 1)
     x = randn_bf16((T, H), 1.0, seed=T + 5, scale_rows=True)
