@@ -17,7 +17,9 @@
 //   batch's loads are issued before the loader waits for the current batch's
 //   buffer. The loader fences the generic-proxy stores for the async proxy
 //   before it arrives on the batch's barrier, so the MMA thread does no fence
-//   of its own.
+//   of its own. Grouped along K (the weight gradients) the transposed
+//   quantisers already write the scales in this chunk order, so the producer
+//   bulk-copies each k-block's chunks into the batch and the loader is idle.
 // MMA (one thread): per k-block, tcgen05.cp copies its chunks from the batch
 // into one of two TMEM scale slots (SFA 4 columns, SFB 8 columns; alternating
 // by k-block) right before four M128 N256 K32 MMAs that select scale byte j
