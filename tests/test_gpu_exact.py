@@ -16,11 +16,11 @@ its value, which alone exceeds 2e-2 rms on tensors whose largest elements pass ~
 gradients of small experts, dW_r of skewed routing; tests/test_oracle.py pins this on the oracle's exact
 values), and MXFP8 quantisation of computed backward operands turns any upstream difference into whole
 E4M3 steps. The bar that decides pass or fail is the comparison with the oracle that applies the identical
-quantisation (recipes "bf16" / "mxfp8" / "nvfp4", the kernels' own rounding points: north_star's "where the
-oracle applies the identical quantisation"): every output must meet it, element by element, except
-elements whose two sides took a bf16 rounding decision the other way (at most two bf16 ulps of the element:
-its own rounding and one flipped term no larger than itself, on at most 0.1% of the elements), which are
-counted and printed.
+quantisation (recipes "bf16" / "mxfp8" / "nvfp4", the kernels' own rounding points): every output must meet
+it, element by element, except elements whose two sides took a bf16 rounding decision the other way. Such
+an element sums `terms` rounded contributions; it may differ by one bf16 ulp of its row's largest element per
+contribution plus one for its own rounding, on at most 0.1% of the elements (helpers.check_bf16), and these
+are counted and printed.
 
 Sizes: the tiny workload in full; each full-size workload on 512 seeded tokens (all of their outputs)
 and, for the backward, the weight gradients of expert 0, the heaviest expert, two median experts and the
