@@ -513,26 +513,45 @@ __global__ void __launch_bounds__(SC_WARPS * 32, KM > 8 ? 1 : ((KM == 2 && EX) ?
   }
 }
 
-// One thread per 1x32 block.
-__global__ void quantize_kernel(const __nv_bfloat16* __restrict__ src, long long nblocks, uint8_t* __restrict__ dst,
-                                uint8_t* __restrict__ sf) {
-  for (long long b = blockIdx.x * (long long)blockDim.x + threadIdx.x; b < nblocks;
-       b += (long long)gridDim.x * blockDim.x) {
-    const uint4* s4 = reinterpret_cast<const uint4*>(src + b * 32);
-    float f[4][8];
-    float am = 0.f;
+// Row-wise MXFP8 quantisation of a [rows, K] bf16 tensor, seen as one run of 16-byte chunks (8 elements;
+// a 1x32 block is four consecutive chunks, and K % 32 == 0, so blocks never straddle rows). A warp takes
+// 32 * QZ_U consecutive chunks per step, all QZ_U loads in flight before any is used: lane l holds chunks
+// l, l + 32, ..., the four lanes of a block reduce its amax by two shuffles, and each warp store writes 256
+// contiguous code bytes (the scale byte by the block's first lane).
+constexpr int QZ_U = 4;
+constexpr int QZ_THREADS = 256;
+__global__ void __launch_bounds__(QZ_THREADS, 4) quantize_kernel(const __nv_bfloat16* __restrict__ src,
+                                                              long long nchunks, uint8_t* __restrict__ dst,
+                                                              uint8_t* __restrict__ sf) {
+  const int lane = threadIdx.x & 31;
+  const long long warp = (blockIdx.x * (long long)QZ_THREADS + threadIdx.x) >> 5;
+  const long long nwarps = ((long long)gridDim.x * QZ_THREADS) >> 5;
+  const uint4* s4 = reinterpret_cast<const uint4*>(src);
+  uint2* d2 = reinterpret_cast<uint2*>(dst);
+  for (long long c0 = warp * (32 * QZ_U); c0 < nchunks; c0 += nwarps * (32 * QZ_U)) {
+    uint4 d[QZ_U];
 #pragma unroll
-    for (int q = 0; q < 4; ++q) {
-      unpack_bf16x8(s4[q], f[q]);
-#pragma unroll
-      for (int i = 0; i < 8; ++i) am = fmaxf(am, fabsf(f[q][i]));
+    for (int u = 0; u < QZ_U; ++u) {
+      const long long i = c0 + 32 * u + lane;
+      d[u] = i < nchunks ? __ldg(s4 + i) : make_uint4(0, 0, 0, 0);
     }
-    const uint8_t sb = mx_scale_byte(am);
-    const float inv = mx_inv_scale(sb);
-    uint2* d2 = reinterpret_cast<uint2*>(dst + b * 32);
 #pragma unroll
-    for (int q = 0; q < 4; ++q) d2[q] = quant8(f[q], inv);
-    sf[b] = sb;
+    for (int u = 0; u < QZ_U; ++u) {
+      const long long i = c0 + 32 * u + lane;  // nchunks % 4 == 0: a block's four lanes are all in or all out
+      float f[8];
+      unpack_bf16x8(d[u], f);
+      float am = 0.f;
+#pragma unroll
+      for (int q = 0; q < 8; ++q) am = fmaxf(am, fabsf(f[q]));
+      am = fmaxf(am, __shfl_xor_sync(0xffffffffu, am, 1));
+      am = fmaxf(am, __shfl_xor_sync(0xffffffffu, am, 2));
+      const uint8_t sb = mx_scale_byte(am);
+      const uint2 codes = quant8(f, mx_inv_scale(sb));
+      if (i < nchunks) {
+        d2[i] = codes;
+        if ((lane & 3) == 0) sf[i >> 2] = sb;
+      }
+    }
   }
 }
 
@@ -689,10 +708,12 @@ int quantize_mxfp8(const void* src, int64_t rows, int32_t K, uint8_t* dst, uint8
   if (!src || !dst || !sf || rows < 1 || K < 32) return MOE_ERR_INVALID_ARG;
   if (K % 32 != 0) return MOE_ERR_UNSUPPORTED;
   if (!al16(src) || !al16(dst)) return MOE_ERR_ALIGNMENT;
-  const long long nb = (long long)rows * (K / 32);
-  long long grid = (nb + 255) / 256;
-  if (grid > 148LL * 16) grid = 148LL * 16;
-  perm::quantize_kernel<<<(int)grid, 256, 0, st>>>(static_cast<const __nv_bfloat16*>(src), nb, dst, sf);
+  const long long nchunks = (long long)rows * (K / 8);
+  constexpr long long per_cta = (perm::QZ_THREADS / 32) * 32 * perm::QZ_U;  // chunks per CTA per step
+  long long grid = (nchunks + per_cta - 1) / per_cta;
+  if (grid > 148LL * 4) grid = 148LL * 4;  // the four CTAs per SM its registers allow; grid-stride beyond
+  perm::quantize_kernel<<<(int)grid, perm::QZ_THREADS, 0, st>>>(static_cast<const __nv_bfloat16*>(src), nchunks,
+                                                                dst, sf);
   MOE_CHECK_LAUNCH();
   return MOE_OK;
 }
