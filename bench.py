@@ -42,24 +42,23 @@ PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 
 
 def measured_traffic(workload: str):
-    """DRAM bytes per launch of the gate/up GEMM from the committed ncu capture, or None when the
-    capture is of another workload or the kernel's sources have changed since it was taken."""
+    """DRAM bytes per launch of the workload's gate/up GEMM from a committed ncu capture (a ```json traffic
+    block in a profiles/*.md summary), or None when no capture is of this workload or the captured kernel's
+    sources have changed since it was taken."""
+    import glob
     import hashlib
     import re
-    p = os.path.join(ROOT, "profiles", "gemm_gateup_mixtral.md")
-    if not os.path.exists(p):
-        return None
-    m = re.search(r"```json traffic\n(.*?)\n```", open(p).read(), re.S)
-    if not m:
-        return None
-    meta = json.loads(m.group(1))
-    if meta.get("workload") != workload:
-        return None
-    h = hashlib.sha256()
-    for f in meta["sources"]:
-        with open(os.path.join(ROOT, f)) as fh:
-            h.update(code_tokens(fh.read()).encode())
-    return meta["dram_bytes_per_launch"] if h.hexdigest() == meta["sources_sha256"] else None
+    for p in sorted(glob.glob(os.path.join(ROOT, "profiles", "*.md"))):
+        for block in re.findall(r"```json traffic\n(.*?)\n```", open(p).read(), re.S):
+            meta = json.loads(block)
+            if meta.get("workload") != workload:
+                continue
+            h = hashlib.sha256()
+            for f in meta["sources"]:
+                with open(os.path.join(ROOT, f)) as fh:
+                    h.update(code_tokens(fh.read()).encode())
+            return meta["dram_bytes_per_launch"] if h.hexdigest() == meta["sources_sha256"] else None
+    return None
 
 
 def code_tokens(src: str) -> str:
@@ -596,7 +595,7 @@ def measure(moe, wl, args, ws, rank, P, headline):
         ach = flops_gateup / (g_ms * 1e-3) / 1e12
         roof = {"kernel": "grouped GEMM gate/up + SwiGLU epilogue", "bound": "tensor", "achieved": round(ach, 1),
                 "peak": round(peak_t, 1), "unit": "TFLOP/s", "frac": round(ach / peak_t, 4),
-                "traffic": measured_traffic(wl.name) if wl.dtype == "bf16" else None,
+                "traffic": measured_traffic(wl.name),
                 "peak_source": peak_note + " (of measured)" if P["source"] == "measured" else peak_note,
                 "clock_normalised": clock_normalised(flops_gateup, g_ms, clocks, wl.dtype)}
         per_elem = {"mxfp8": 1 + 1 / 32, "nvfp4": 0.5 + 1 / 16}.get(wl.dtype, 2)

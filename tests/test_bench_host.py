@@ -1,5 +1,6 @@
-"""Host logic of bench.py that needs no GPU: the source fingerprint that decides whether the committed
-DRAM-traffic capture of the gate/up GEMM still describes the kernel being timed."""
+"""Host logic of bench.py that needs no GPU: the source fingerprint that decides whether a committed
+DRAM-traffic capture of a workload's gate/up GEMM (a json traffic block in a profiles/*.md summary) still
+describes the kernel being timed."""
 import os
 import sys
 
@@ -30,3 +31,26 @@ def test_code_tokens_keeps_literals():
 def test_traffic_only_for_the_captured_workload():
     # a capture of one workload never stands in for another
     assert bench.measured_traffic("no-such-workload") is None
+
+
+def _fake_tree(tmp_path, src_text, captured_text, workload="wl-a"):
+    import hashlib
+    import json
+    (tmp_path / "profiles").mkdir()
+    (tmp_path / "k.cu").write_text(src_text)
+    h = hashlib.sha256(bench.code_tokens(captured_text).encode()).hexdigest()
+    meta = {"workload": workload, "dram_bytes_per_launch": 12345, "sources": ["k.cu"], "sources_sha256": h}
+    (tmp_path / "profiles" / "cap.md").write_text("# capture\n\n```json traffic\n" + json.dumps(meta) + "\n```\n")
+
+
+def test_traffic_found_in_any_profile_while_its_sources_match(tmp_path, monkeypatch):
+    _fake_tree(tmp_path, "int f() { return 1; }  // now with a comment", "int f() { return 1; }")
+    monkeypatch.setattr(bench, "ROOT", str(tmp_path))
+    assert bench.measured_traffic("wl-a") == 12345     # comments and layout do not matter
+    assert bench.measured_traffic("wl-b") is None      # another workload's capture never stands in
+
+
+def test_traffic_dropped_once_the_captured_code_changes(tmp_path, monkeypatch):
+    _fake_tree(tmp_path, "int f() { return 2; }", "int f() { return 1; }")
+    monkeypatch.setattr(bench, "ROOT", str(tmp_path))
+    assert bench.measured_traffic("wl-a") is None
