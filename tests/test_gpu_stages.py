@@ -23,7 +23,11 @@ def _status_clean(moe):
 
 
 @pytest.mark.parametrize("T,H,E,bias", [(512, 256, 8, False), (300, 512, 128, True), (1000, 4096, 128, False),
-                                        (129, 7168, 256, True), (1, 256, 8, False)])
+                                        (129, 7168, 256, True), (1, 256, 8, False),
+                                        # E <= 16: logits computed inside the top-k kernel; a ragged last round
+                                        # of 16-byte chunks (H = 384: 48 chunks over 32 lanes), an odd T, fewer
+                                        # chunks than lanes (H = 128), and the Mixtral shape
+                                        (333, 384, 16, True), (77, 128, 4, True), (4096, 4096, 8, False)])
 def test_router_logits_match_oracle(moe, oracle, T, H, E, bias):
     x = randn_bf16((T, H), 1.0, seed=T, device="cuda")
     W_r = randn_bf16((E, H), 0.02, seed=T + 1, device="cuda")
