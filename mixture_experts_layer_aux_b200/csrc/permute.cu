@@ -26,6 +26,9 @@
 //            tensor.
 //   unpermute one warp per token: fp32 sum of its k rows in slot order, 16-byte
 //            loads, one bf16 rounding.
+//   quantize row-wise MXFP8 of a [rows, K] bf16 tensor (the expert weights,
+//            dgate|dup, the shared expert's x): four lanes per 1x32 block,
+//            coalesced 16-byte loads, 256 contiguous code bytes per warp store.
 #include <cuda_fp8.h>
 
 #include <cmath>
