@@ -97,6 +97,10 @@ WORKLOADS = {
     # the token-side traffic of the Qwen3 shape (T=8192, H=4096, k=8) on 16 small experts, about 1.5 GB on the
     # device: the small case of the permutation and unpermute kernels' DRAM captures
     "qwen3-mem": Workload("qwen3-mem", T=8192, H=4096, E=16, k=8, F=512),
+    # the token-side traffic of the DeepSeek-V3 MXFP8 shape (T=8192, H=7168, k=8, MXFP8 permutation) on 16 small
+    # experts without the shared one, a few GB on the device: the small case of the MXFP8 permutation's captures
+    "dsv3-mem": Workload("dsv3-mem", T=8192, H=7168, E=16, k=8, F=256, score="sigmoid", route_scale=2.5,
+                         dtype="mxfp8", aux=False),
     # the MXFP8 backward on the DeepSeek-V3 routed experts (the backward has no shared expert)
     "dsv3-train": Workload("dsv3-train", T=8192, H=7168, E=256, k=8, F=2048, score="sigmoid", route_scale=2.5,
                            dtype="mxfp8", aux=False, bwd=True),
